@@ -1,0 +1,189 @@
+"""CPU oracle for the local MoE expert forward on the non-expand layout.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU
+baseline leg of ``bench.py`` may use it; the product path never does.  It is a
+plain C file (``moe_oracle.c``) compiled here with gcc into ``_oracle.so`` and
+called through ctypes; it shares no code with the CUDA library.
+
+The functions follow the definitions written at the top of ``moe_oracle.c``
+(sonic-moe issue #68 metadata list and question 3; qwen3_5.py commit notes,
+CCCL segmented-sort recipe; sonic-moe write-up, weight-layout section).
+Arithmetic is double precision on bf16 inputs, with no intermediate rounding.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_oracle.so")
+_lock = threading.Lock()
+_libs = {}
+
+LAYOUT_INTERLEAVED = 0
+LAYOUT_CONCATENATED = 1
+
+
+def compile_source(src: str, out: str) -> str:
+    """Compile a C file of the oracle's interface with gcc (OpenMP)."""
+    tmp = out + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", tmp, src, "-lm"]
+    subprocess.check_call(cmd)
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle if the shared object is missing or stale."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    return compile_source(_SRC, _LIB_PATH)
+
+
+def _load(path: str | None = None):
+    """The oracle library (or, for the mutation pins, a variant compiled
+    from an edited copy of its source at ``path``)."""
+    with _lock:
+        key = path or _LIB_PATH
+        if key in _libs:
+            return _libs[key]
+        lib = ctypes.CDLL(build() if path is None else path)
+        P = ctypes.c_void_p
+        i64, i32 = ctypes.c_int64, ctypes.c_int32
+        lib.oracle_metadata.restype = i64
+        lib.oracle_metadata.argtypes = [i64, i32, i32, P, P, P, P, P, P, P, P, P, P]
+        lib.oracle_expert_row.restype = None
+        lib.oracle_expert_row.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P]
+        lib.oracle_forward_rows.restype = None
+        lib.oracle_forward_rows.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, P,
+                                            i64, P, P, i32]
+        lib.oracle_combine.restype = None
+        lib.oracle_combine.argtypes = [i64, i32, P, P, P, P, P]
+        lib.oracle_pair_rows.restype = None
+        lib.oracle_pair_rows.argtypes = [i32, i32, i32, P, P, P, P, P, i64, P, P, P, P, i32]
+        _libs[key] = lib
+        return lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bf16_bits(t):
+    """Raw bf16 bit patterns (uint16) of a torch bf16 tensor, or None."""
+    if t is None:
+        return None
+    import torch
+    assert t.dtype == torch.bfloat16
+    return np.ascontiguousarray(t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def metadata(topk_idx: np.ndarray, topk_w: np.ndarray, E: int, lib_path: str | None = None) -> dict:
+    """Routing metadata of a [N,K] non-expand layout.  Returns a dict with
+    freq [E], off [E+1], x_gather_idx / s_scatter_idx / s_reverse_scatter_idx
+    [P], token_offset [N+1], scores [P], P and bad_ids."""
+    lib = _load(lib_path)
+    idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    N, K = idx.shape
+    cap = max(1, N * K)
+    freq = np.zeros(E, np.int32)
+    off = np.zeros(E + 1, np.int32)
+    xg = np.zeros(cap, np.int32)
+    ss = np.zeros(cap, np.int32)
+    sr = np.zeros(cap, np.int32)
+    to = np.zeros(N + 1, np.int32)
+    sc = np.zeros(cap, np.float32)
+    bad = np.zeros(1, np.int64)
+    P = lib.oracle_metadata(N, K, E, _ptr(idx), _ptr(w), _ptr(freq), _ptr(off), _ptr(xg),
+                            _ptr(ss), _ptr(sr), _ptr(to), _ptr(sc), _ptr(bad))
+    return dict(freq=freq, off=off, x_gather_idx=xg[:P].copy(), s_scatter_idx=ss[:P].copy(),
+                s_reverse_scatter_idx=sr[:P].copy(), token_offset=to, scores=sc[:P].copy(),
+                P=int(P), bad_ids=int(bad[0]))
+
+
+def expert_row(x_row, w1e, b1e, w2e, b2e, layout: int = LAYOUT_INTERLEAVED, lib_path: str | None = None):
+    """One expert on one token row (bf16 torch tensors in, float64 numpy out):
+    returns (z [2I], h [I], y [H])."""
+    lib = _load(lib_path)
+    xr, a, b, c, d = (_bf16_bits(v) for v in (x_row, w1e, b1e, w2e, b2e))
+    H = xr.shape[0]
+    I = c.shape[0]
+    z = np.zeros(2 * I, np.float64)
+    h = np.zeros(I, np.float64)
+    y = np.zeros(H, np.float64)
+    lib.oracle_expert_row(H, I, layout, _ptr(xr), _ptr(a), _ptr(b), _ptr(c), _ptr(d),
+                          _ptr(z), _ptr(h), _ptr(y))
+    return z, h, y
+
+
+class Weights:
+    """Host bf16 bit copies of the forward's dense inputs, made once."""
+
+    def __init__(self, x, w1, b1, w2, b2):
+        self.x = _bf16_bits(x)
+        self.w1 = _bf16_bits(w1)
+        self.b1 = _bf16_bits(b1)
+        self.w2 = _bf16_bits(w2)
+        self.b2 = _bf16_bits(b2)
+        self.N, self.H = self.x.shape
+        self.E, _, two_i = self.w1.shape
+        self.I = two_i // 2
+
+
+def forward_rows(wts: Weights, topk_idx: np.ndarray, topk_w: np.ndarray, tokens=None,
+                 layout: int = LAYOUT_INTERLEAVED, n_threads: int = 0, lib_path: str | None = None) -> np.ndarray:
+    """Output rows [len(tokens), H] (float64) of the forward for the chosen
+    tokens (all tokens when None)."""
+    lib = _load(lib_path)
+    idx = np.ascontiguousarray(topk_idx, dtype=np.int32)
+    w = np.ascontiguousarray(topk_w, dtype=np.float32)
+    N, K = idx.shape
+    if tokens is None:
+        tokens = np.arange(N, dtype=np.int64)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    out = np.zeros((tokens.shape[0], wts.H), np.float64)
+    if n_threads <= 0:
+        n_threads = len(os.sched_getaffinity(0))
+    lib.oracle_forward_rows(N, wts.H, wts.I, wts.E, K, layout, _ptr(wts.x), _ptr(idx), _ptr(w),
+                            _ptr(wts.w1), _ptr(wts.b1), _ptr(wts.w2), _ptr(wts.b2),
+                            tokens.shape[0], _ptr(tokens), _ptr(out), n_threads)
+    return out
+
+
+def pair_rows(wts: Weights, tokens, experts, layout: int = LAYOUT_INTERLEAVED, n_threads: int = 0, lib_path: str | None = None):
+    """(h [n,I], y [n,H]) float64 for the given (token, expert) pairs."""
+    lib = _load(lib_path)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    experts = np.ascontiguousarray(experts, dtype=np.int32)
+    n = tokens.shape[0]
+    h = np.zeros((n, wts.I), np.float64)
+    y = np.zeros((n, wts.H), np.float64)
+    if n_threads <= 0:
+        n_threads = len(os.sched_getaffinity(0))
+    lib.oracle_pair_rows(wts.H, wts.I, layout, _ptr(wts.x), _ptr(wts.w1), _ptr(wts.b1),
+                         _ptr(wts.w2), _ptr(wts.b2), n, _ptr(tokens), _ptr(experts),
+                         _ptr(h), _ptr(y), n_threads)
+    return h, y
+
+
+def combine(token_offset: np.ndarray, s_rev: np.ndarray, scores: np.ndarray,
+            ysorted: np.ndarray, lib_path: str | None = None) -> np.ndarray:
+    """out [N,H] float64 = per token, sum over its pairs q (in q order) of
+    scores[q] * ysorted[s_rev[q]]."""
+    lib = _load(lib_path)
+    to = np.ascontiguousarray(token_offset, dtype=np.int32)
+    sr = np.ascontiguousarray(s_rev, dtype=np.int32)
+    sc = np.ascontiguousarray(scores, dtype=np.float32)
+    ys = np.ascontiguousarray(ysorted, dtype=np.float64)
+    N = to.shape[0] - 1
+    H = ys.shape[1]
+    out = np.zeros((N, H), np.float64)
+    lib.oracle_combine(N, H, _ptr(to), _ptr(sr), _ptr(sc), _ptr(ys), _ptr(out))
+    return out

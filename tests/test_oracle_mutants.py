@@ -1,0 +1,101 @@
+"""The oracle's pins must catch plausible mistakes.
+
+Each case plants one mistake in a copy of the oracle's C source (on the CPU;
+the real oracle is untouched), compiles it, and checks that at least one pin
+of tests/test_oracle_pins.py -- the hand-worked fixtures, the torch-CPU sort
+recipe, the invariants -- rejects the mutant.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from mixture_experts_routed_non_b200 import synthetic
+from test_oracle_pins import (GOLDEN, _bf, _load, _num, _recipe_torch_cpu,
+                              check_metadata_invariants)
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")
+
+MUTANTS = {
+    "gate_up_swapped": ("h[j] = g / (1.0 + exp(-g)) * u;", "h[j] = u / (1.0 + exp(-u)) * g;"),
+    "silu_sign": ("h[j] = g / (1.0 + exp(-g)) * u;", "h[j] = g / (1.0 + exp(g)) * u;"),
+    "b1_dropped": ("z[j] = b1e ? bf16_value(b1e[j]) : 0.0;", "z[j] = 0.0;"),
+    "b2_dropped": ("y[n] = b2e ? bf16_value(b2e[n]) : 0.0;", "y[n] = 0.0;"),
+    "concat_wrong_up": ("else             { g = z[j];     u = z[I + j]; }",
+                        "else             { g = z[j];     u = z[j + 1]; }"),
+    "interleave_wrong": ("if (layout == 0) { g = z[2 * j]; u = z[2 * j + 1]; }",
+                         "if (layout == 0) { g = z[j]; u = z[I + j]; }"),
+    "score_ignored": ("for (int32_t n = 0; n < H; ++n) o[n] += w * y[n];",
+                      "for (int32_t n = 0; n < H; ++n) o[n] += y[n];"),
+    "w2_transposed_index": ("const uint16_t *wr = w2e + (size_t)j * H;\n        for (int32_t n = 0; n < H; ++n) y[n] += hv * bf16_value(wr[n]);",
+                            "for (int32_t n = 0; n < H; ++n) y[n] += hv * bf16_value(w2e[(size_t)n * I + (j % I)]);"),
+    "sort_unstable": ("for (int64_t i = 0; i < q; ++i) {\n        int32_t p = cursor[pair_expert[i]]++;",
+                      "for (int64_t i = q - 1; i >= 0; --i) {\n        int32_t p = cursor[pair_expert[i]]++;"),
+    "token_offset_late": ("        token_offset[t] = (int32_t)q;\n        for (int32_t k = 0; k < K; ++k) {",
+                          "        for (int32_t k = 0; k < K; ++k) {"),
+    "offsets_inclusive": ("off[e + 1] = off[e] + freq[e];", "off[e + 1] = off[e] + freq[e] + (e == 0);"),
+    "invalid_counted": ("if (e >= 0 && e < E) {", "if (e < E) { if (e < 0) e = 0;"),
+}
+
+
+def _mutant(tmp_path, name):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert old in src, f"mutation anchor missing for {name}"
+    path = tmp_path / f"mut_{name}.c"
+    path.write_text(src.replace(old, new, 1))
+    so = str(tmp_path / f"mut_{name}.so")
+    oracle.compile_source(str(path), so)
+    return so
+
+
+def _pins_pass(lib):
+    """Run the library-level pins against one build; True when all agree."""
+    try:
+        # hand-worked metadata example
+        g = _load("metadata_worked_example.json")
+        idx = np.array(g["topk_idx"], np.int32)
+        w = np.array([[_num(v) for v in r] for r in g["topk_w"]], np.float32)
+        md = oracle.metadata(idx, w, g["E"], lib_path=lib)
+        ex = g["expected"]
+        if (md["off"].tolist() != ex["expert_frequency_offset"]
+                or md["s_scatter_idx"].tolist() != ex["s_scatter_idx"]
+                or md["token_offset"].tolist() != ex["num_activated_expert_per_token_offset"]
+                or md["x_gather_idx"].tolist() != ex["x_gather_idx"]):
+            return False
+        check_metadata_invariants(idx, w, g["E"], md)
+        # closed-form SwiGLU fixture, both layouts
+        g = _load("swiglu_closed_form.json")
+        x, w1, b1, w2, b2 = (_bf(g[k]) for k in ("x", "w1", "b1", "w2", "b2"))
+        idx = np.array(g["topk_idx"], np.int32)
+        w = np.array([[_num(v) for v in r] for r in g["topk_w"]], np.float32)
+        wts = oracle.Weights(x, w1, b1, w2, b2)
+        env = {"exp": math.exp}
+        for layout, key in ((0, "interleaved"), (1, "concatenated")):
+            out = oracle.forward_rows(wts, idx, w, layout=layout, lib_path=lib)
+            out_ex = [eval(s, env) for s in g["expected_closed_form"][key]["out"]]
+            if not np.allclose(out[0], out_ex, rtol=1e-12, atol=1e-12):
+                return False
+        # torch-CPU sort recipe on the tiny workload
+        inp = synthetic.make_inputs("tiny", device="cpu")
+        wts = oracle.Weights(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+        for layout in (0, 1):
+            out = oracle.forward_rows(wts, inp.topk_idx.numpy(), inp.topk_w.numpy(),
+                                      layout=layout, lib_path=lib)
+            if not np.allclose(out, _recipe_torch_cpu(inp, layout), rtol=1e-9, atol=1e-10):
+                return False
+        return True
+    except AssertionError:
+        return False
+
+
+def test_unmutated_oracle_passes_pins():
+    assert _pins_pass(None)
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_rejected(tmp_path, name):
+    assert not _pins_pass(_mutant(tmp_path, name)), f"pins did not catch mutant {name}"
