@@ -1,0 +1,440 @@
+"""Benchmark of the local MoE expert forward on the non-expand routed layout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill] [--layout 0|1]
+
+One step = one moe_nonexpand_forward (metadata, grouped GEMM up + SwiGLU,
+grouped GEMM down, combine) over one batch of seeded synthetic inputs of the
+named workload, inputs resident in HBM.  Prints one JSON line on rank 0.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica on
+its own token batch (the path has no exchange step), so scaling is weak and
+the value is all ranks' tokens divided by the slowest rank's time.
+
+--impl reference times the CPU oracle (the only reference this method has)
+on the host cores, on a bounded token sample per step, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE fwd tokens/sec and grouped-GEMM TFLOP/s (% bf16 peak) on 1 B200"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        for ts, line in self.lines:
+            if not (t0 <= ts <= t1):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[0]), max=float(parts[1]), active=parts[3],
+                                 hw=parts[4], hwt=parts[5], swt=parts[6], pcap=parts[7]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["max"] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# roofline bookkeeping
+# ---------------------------------------------------------------------------
+def gemm_flops(P: int, H: int, I: int):
+    return 4.0 * P * H * I, 2.0 * P * H * I
+
+
+def algorithmic_bytes(inp, P: int, freq):
+    """x read once + the weights of experts with at least one pair + routing
+    tensors + out written."""
+    wl = inp.wl
+    active = int((freq > 0).sum())
+    per_expert = (wl.H * 2 * wl.I + wl.I * wl.H) * 2
+    return wl.N * wl.H * 2 + active * per_expert + wl.N * wl.K * 8 + wl.N * wl.H * 2
+
+
+def traffic_record(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary, valid
+    only while the kernel's sources are unchanged (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    srcs = ["mixture_experts_routed_non_b200/csrc/grouped_gemm_sm100.cu",
+            "mixture_experts_routed_non_b200/csrc/common.cuh"]
+    h = hashlib.sha256()
+    for s in srcs:
+        with open(os.path.join(ROOT, s), "rb") as f:
+            h.update(f.read())
+    digest = h.hexdigest()[:16]
+    with open(path) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            kv = dict(p.split("=", 1) for p in line.split() if "=" in p)
+            if (kv.get("kernel") == kernel and kv.get("workload") == workload
+                    and kv.get("sources") == digest):
+                return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+# ---------------------------------------------------------------------------
+def oracle_tokens_per_s(inp, target_s: float, rng_seed: int = 123, max_tokens=None):
+    """Time the oracle on a seeded token sample sized for about target_s of
+    wall time.  Returns (tokens/s, tokens, seconds, threads)."""
+    import numpy as np
+
+    import oracle
+    wts = oracle.Weights(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    idx = inp.topk_idx.cpu().numpy()
+    w = inp.topk_w.cpu().numpy()
+    threads = len(os.sched_getaffinity(0))
+    rng = np.random.default_rng(rng_seed)
+    N = inp.wl.N
+    n = min(N, 8)
+    oracle.forward_rows(wts, idx, w, tokens=np.arange(min(N, 2)), n_threads=threads)  # load + warm
+    while True:
+        toks = np.sort(rng.choice(N, size=n, replace=False))
+        t0 = time.perf_counter()
+        oracle.forward_rows(wts, idx, w, tokens=toks, n_threads=threads)
+        dt = time.perf_counter() - t0
+        if dt >= target_s * 0.5 or n >= N or (max_tokens and n >= max_tokens):
+            return n / dt, n, dt, threads
+        grow = max(2.0, min(16.0, target_s / max(dt, 1e-3)))
+        n = min(N, int(n * grow) + 1)
+        if max_tokens:
+            n = min(n, max_tokens)
+
+
+# ---------------------------------------------------------------------------
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill")
+    ap.add_argument("--layout", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, rank 0 only."""
+    if rank != 0:
+        return
+    import torch  # noqa: F401
+    from mixture_experts_routed_non_b200 import synthetic
+    wl = synthetic.WORKLOADS[args.workload]
+    inp = synthetic.make_inputs(wl, device="cpu")
+    import numpy as np
+
+    import oracle
+    wts = oracle.Weights(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    idx = inp.topk_idx.numpy()
+    w = inp.topk_w.numpy()
+    threads = len(os.sched_getaffinity(0))
+    # sample size per step: about 6 s of oracle work
+    probe = np.arange(min(wl.N, 4))
+    t0 = time.perf_counter()
+    oracle.forward_rows(wts, idx, w, tokens=probe, layout=args.layout, n_threads=threads)
+    per_tok = (time.perf_counter() - t0) / len(probe)
+    n = int(max(1, min(wl.N, 6.0 / max(per_tok, 1e-6))))
+    rng = np.random.default_rng(7)
+    times = []
+    for step in range(args.warmup + args.steps):
+        toks = np.sort(rng.choice(wl.N, size=n, replace=False))
+        t0 = time.perf_counter()
+        oracle.forward_rows(wts, idx, w, tokens=toks, layout=args.layout, n_threads=threads)
+        dt = time.perf_counter() - t0
+        if step >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = n * len(times) / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * total / len(times), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "N": wl.N, "H": wl.H, "I": wl.I, "E": wl.E, "K": wl.K,
+                   "layout": args.layout, "sample_tokens_per_step": n},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{n} seeded tokens of the {wl.name} workload per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from mixture_experts_routed_non_b200 import binding, synthetic
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: no CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    wl = synthetic.WORKLOADS[args.workload]
+    inp = synthetic.make_inputs(wl, device=dev, seed=wl.seed + 1000 * rank)
+    N, H, I, E, K = wl.N, wl.H, wl.I, wl.E, wl.K
+    w1, b1 = inp.w1, inp.b1
+    if args.layout == 1:
+        w1 = torch.cat([w1[:, :, 0::2], w1[:, :, 1::2]], dim=2).contiguous()
+        b1 = None if b1 is None else torch.cat([b1[:, 0::2], b1[:, 1::2]], dim=1).contiguous()
+    ws = binding.alloc_workspace(N, H, I, E, K, -1, dev)
+    out = torch.empty(N, H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None):
+        binding.forward(inp.x, inp.topk_idx, inp.topk_w, w1, inp.w2, b1, inp.b2, layout=args.layout,
+                        out=out, ws=ws, events=events)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    err = binding.read_error(ws)
+    if err:
+        raise SystemExit(f"bench.py: device error word {err:#x}")
+    meta = binding.meta_from_workspace(ws, N, H, I, E, K)
+    freq = meta["expert_frequency"].cpu().numpy()
+    P = int(freq.sum())
+
+    # ---- timed region: K steps, stage events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(ev[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.15)
+    sampler.stop()
+    elapsed_ms = start.elapsed_time(end)
+    stage_ms = np.zeros(4)
+    for e in ev:
+        for j in range(4):
+            stage_ms[j] += e[j].elapsed_time(e[j + 1])
+    stage_ms /= args.steps
+    max_ms = elapsed_ms
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        max_ms = float(t.item())
+    ms_per_step = max_ms / args.steps
+    value = N * world * args.steps / (max_ms / 1000.0)
+
+    # ---- end to end: pinned host inputs in, result out, every step
+    x_h = inp.x.cpu().pin_memory()
+    idx_h = inp.topk_idx.cpu().pin_memory()
+    w_h = inp.topk_w.cpu().pin_memory()
+    out_h = torch.empty(N, H, dtype=torch.bfloat16).pin_memory()
+    x_d = torch.empty_like(inp.x)
+    idx_d = torch.empty_like(inp.topk_idx)
+    w_d = torch.empty_like(inp.topk_w)
+    e2e_steps = max(3, min(args.steps, 100))
+
+    def e2e_step():
+        x_d.copy_(x_h, non_blocking=True)
+        idx_d.copy_(idx_h, non_blocking=True)
+        w_d.copy_(w_h, non_blocking=True)
+        binding.forward(x_d, idx_d, w_d, w1, inp.w2, b1, inp.b2, layout=args.layout, out=out, ws=ws)
+        out_h.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    s2 = torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = s2.elapsed_time(e2)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = N * world * e2e_steps / (e2e_ms / 1000.0)
+    h2d = x_h.numel() * 2 + idx_h.numel() * 4 + w_h.numel() * 4
+    d2h = out_h.numel() * 2
+
+    peaks, peaks_src = load_peaks()
+    up_flops, down_flops = gemm_flops(P, H, I)
+    up_tflops = up_flops / (stage_ms[1] * 1e-3) / 1e12
+    down_tflops = down_flops / (stage_ms[2] * 1e-3) / 1e12
+    gemm_tflops = (up_flops + down_flops) / ((stage_ms[1] + stage_ms[2]) * 1e-3) / 1e12
+    peak_tf = peaks["bf16_tflops"]
+    comb_bytes = P * H * 2 + N * H * 2 + (N + 1) * 4 + P * 8
+    meta_bytes = N * K * 8 + 4 * P * 4 + 4 * (N + 1) + 8 * E
+    alg_bytes = algorithmic_bytes(inp, P, freq)
+    total_flops = up_flops + down_flops
+    t_roof = max(total_flops / (peak_tf * 1e12), alg_bytes / (peaks["hbm_gbs"] * 1e9))
+    clocks = sampler.summary(t_wall0, t_wall1)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        tps, n_tok, secs, threads = oracle_tokens_per_s(inp, args.cpu_seconds)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{n_tok} seeded tokens of the {wl.name} workload ({secs:.1f} s of oracle time)"}
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "N": N, "H": H, "I": I, "E": E, "K": K, "P": P,
+                   "layout": "interleaved" if args.layout == 0 else "concatenated",
+                   "routing": wl.description, "parallelism": f"replicas x{world} (token shards)",
+                   "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (
+                       (inp.w1.numel() + inp.w2.numel()) * 2 / 1e9)},
+        "roofline": {"bound": "tensor", "kernel": "grouped GEMM up (gather + SwiGLU)",
+                     "achieved": up_tflops, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": up_tflops / peak_tf, "peak_source": f"{peaks_src} bf16 burst",
+                     "traffic": traffic_record("gemm_up", wl.name)},
+        "gemm_tflops": gemm_tflops,
+        "gemm_frac_of_peak": gemm_tflops / peak_tf,
+        "step_frac_of_roofline": (t_roof * 1e3) / ms_per_step,
+        "stages_ms": {"metadata": stage_ms[0], "gemm_up": stage_ms[1], "gemm_down": stage_ms[2],
+                      "combine": stage_ms[3]},
+        "stages": {
+            "gemm_up_tflops": up_tflops, "gemm_down_tflops": down_tflops,
+            "combine_gbs": comb_bytes / (stage_ms[3] * 1e-3) / 1e9,
+            "combine_frac_hbm": comb_bytes / (stage_ms[3] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "metadata_gbs": meta_bytes / (stage_ms[0] * 1e-3) / 1e9,
+        },
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clocks,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,213 @@
+/*
+ * moe_nonexpand.h -- C ABI of the local MoE expert forward on the "non-expand"
+ * routed layout, for NVIDIA B200 (sm_100a).
+ *
+ * The problem statement follows sonic-moe issue #68 ("End-to-end DeepEP v2
+ * non-expand + SonicMoE integration"):
+ *   - input layout (the non-expand receive block): x [N,H], topk_idx [N,K]
+ *     holding a local expert id or -1 for an invalid slot, topk_w [N,K];
+ *   - the proposed entry point moe_deepep_nonexpand_inputs(recv_x,
+ *     recv_topk_idx, recv_topk_weights, total_pairs, w1, b1, w2, b2, E,
+ *     stream_id, activation_type, ...), which these calls follow;
+ *   - the list of metadata the entry point builds directly from [N,K]
+ *     (expert_frequency, expert_frequency_offset, x_gather_idx,
+ *     s_scatter_idx, s_reverse_scatter_idx,
+ *     num_activated_expert_per_token_offset, compact router_scores [P]);
+ *   - the target dataflow: the local expert compute yields local_out [N,H].
+ * The expert MLP is the gated up projection with "silu times up" and the down
+ * projection (qwen3_5.py commit notes, CCCL segmented-sort recipe, steps 3-5;
+ * sonic-moe write-up, "The MoE class takes a routing count and a kernel
+ * backend": SWIGLU and optional biases).  The gate/up columns of w1 are
+ * interleaved (g0,u0,g1,u1,...) or concatenated (all gates, then all ups)
+ * (sonic-moe write-up, "Interleaved by default, concatenated if your model
+ * is HuggingFace").
+ *
+ * Definitions used throughout:
+ *   pair q     -- the q-th valid slot in row-major (token, slot) order; a slot
+ *                 is valid when 0 <= topk_idx[t,k] < E.  P = number of pairs.
+ *   position p -- index in the stable expert-sorted order of the pairs
+ *                 (expert ascending, then q ascending).
+ *   out[t,:]   = sum over token t's pairs q, in q order, of
+ *                topk_w[t,k(q)] * ( silu(g) * u ) . w2[e] + b2[e] ),
+ *                with [g|u] taken from x[t,:] . w1[e] + b1[e].
+ *                A token without a valid slot gets a zero row.
+ *
+ * Conventions:
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise, and
+ *     every buffer is owned by the caller.  The library allocates nothing and
+ *     keeps no state besides per-device launch settings.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream).  Only moe_nonexpand_read_error synchronises the host.
+ *   - Layouts are dense row-major; x, w1, w2, out must be 16-byte aligned.
+ *   - Dtypes: x, w1, b1, w2, b2, out are bf16; topk_idx int32; topk_w fp32.
+ *   - Return value: MOE_OK or one of the MOE_ERR_* codes below; on error
+ *     nothing has been enqueued.  Errors found on the device (bad expert ids,
+ *     a pair count that disagrees with total_pairs, an internal wait that
+ *     timed out) are recorded in the workspace's device error word and read
+ *     with moe_nonexpand_read_error.
+ *   - Supported sizes: N >= 0, 1 <= K <= 32, 1 <= E <= 1024, N*K < 2^31,
+ *     H and I multiples of 64 (tensor-memory-access and MMA alignment), and
+ *     P_cap * max(H, I) < 2^31 where P_cap is total_pairs when it is given
+ *     and N*K otherwise.
+ */
+#ifndef MOE_NONEXPAND_H
+#define MOE_NONEXPAND_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host return codes. */
+#define MOE_OK 0
+#define MOE_ERR_ARG 1         /* null required pointer, bad N/K/E, bad enum, misaligned pointer */
+#define MOE_ERR_SHAPE 2       /* H or I not a multiple of 64, or sizes overflow 32-bit indexing */
+#define MOE_ERR_WS 3          /* workspace too small (or null) */
+#define MOE_ERR_CUDA 4        /* a CUDA runtime call or launch failed */
+#define MOE_ERR_DEVICE 5      /* current device is not sm_100 (B200-class) */
+
+/* Bits of the device error word (moe_nonexpand_read_error). */
+#define MOE_DEVERR_BAD_EXPERT_ID 0x1u /* an id outside {-1} U [0,E) was seen; that slot was skipped */
+#define MOE_DEVERR_PAIR_COUNT 0x2u    /* counted P != total_pairs (total_pairs >= 0) or P > P_cap */
+#define MOE_DEVERR_TIMEOUT 0x4u       /* an internal pipeline wait gave up; outputs are invalid */
+#define MOE_DEVERR_ABORTED 0x8u       /* P > P_cap: GEMMs and combine were skipped, out unwritten */
+
+/* activation argument */
+#define MOE_ACT_SWIGLU 0
+/* gate_up_layout argument */
+#define MOE_LAYOUT_INTERLEAVED 0
+#define MOE_LAYOUT_CONCATENATED 1
+
+/* The routing metadata of issue #68's list, in caller-owned device memory.
+ * P_cap = total_pairs if total_pairs >= 0, else N*K. */
+typedef struct moe_meta_t {
+    int32_t *expert_frequency;         /* [E]     pairs per expert                          */
+    int32_t *expert_frequency_offset;  /* [E+1]   exclusive prefix sum; [E] = P             */
+    int32_t *x_gather_idx;             /* [P_cap] token (row of x) at sorted position p     */
+    int32_t *s_scatter_idx;            /* [P_cap] pair index q at sorted position p         */
+    int32_t *s_reverse_scatter_idx;    /* [P_cap] sorted position p of pair q               */
+    int32_t *token_offset;             /* [N+1]   num_activated_expert_per_token_offset:
+                                          pairs of token t are q in [off[t], off[t+1])      */
+    float *scores;                     /* [P_cap] compact router scores, scores[q]          */
+} moe_meta_t;
+
+/* Opaque CUDA handles, ABI-compatible with cudaStream_t / cudaEvent_t. */
+typedef struct CUstream_st *moe_stream_t;
+typedef struct CUevent_st *moe_event_t;
+
+/*
+ * Bytes of workspace needed by moe_nonexpand_forward for these sizes (pass
+ * H = I = 0 for what moe_nonexpand_metadata alone needs).  The workspace
+ * holds the per-tile histograms, the GEMM tile table, the metadata when the
+ * caller does not provide it, and the bf16 intermediates h [P_cap,I] and
+ * y [P_cap,H].  It must be zero-filled ONCE after allocation; the library
+ * leaves it in a reusable state after every call.  One workspace must not be
+ * used by two calls that can run at the same time.
+ * Returns 0 for arguments outside the supported sizes.
+ */
+MOE_API size_t moe_nonexpand_workspace_bytes(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
+                                     int64_t total_pairs);
+
+/*
+ * Routing metadata only (issue #68 metadata list), built from [N,K]:
+ * histogram, exclusive offsets, stable counting sort of the pairs by expert,
+ * per-token pair offsets and compact scores.  Results are bit-exact and
+ * deterministic.  `meta` (host struct of device pointers) must be non-null
+ * with every field set.  Invalid slots' weights are never read.
+ */
+MOE_API int moe_nonexpand_metadata(const int32_t *topk_idx, const float *topk_w,
+                           int64_t N, int32_t K, int32_t E, int64_t total_pairs,
+                           const moe_meta_t *meta, void *ws, size_t ws_bytes,
+                           moe_stream_t stream);
+
+/*
+ * The whole local expert forward: metadata, gathered grouped GEMM up with
+ * bias and SwiGLU fused in its epilogue (rows of x are gathered straight
+ * through x_gather_idx; no permuted copy of x is made), grouped GEMM down
+ * with bias, and the deterministic score-weighted combine (each token sums
+ * its pairs in slot order through s_reverse_scatter_idx; no atomics).
+ *   x    [N,H]   bf16       w1 [E,H,2I] bf16     b1 [E,2I] bf16 or NULL
+ *   w2   [E,I,H] bf16       b2 [E,H]    bf16 or NULL
+ *   out  [N,H]   bf16 (written; rounded to nearest even from an fp32 sum)
+ *   meta_out: NULL keeps the metadata inside the workspace; otherwise the
+ *             metadata is also left in the caller's buffers.
+ * Intermediates h = silu(g)*u and y = h.w2 + b2 are stored as bf16.
+ */
+MOE_API int moe_nonexpand_forward(const void *x, const int32_t *topk_idx, const float *topk_w,
+                          int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
+                          int64_t total_pairs,
+                          const void *w1, const void *b1, const void *w2, const void *b2,
+                          int32_t activation, int32_t gate_up_layout,
+                          void *out, const moe_meta_t *meta_out,
+                          void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Same as moe_nonexpand_forward, and records five caller-created CUDA events
+ * on `stream` (a host array of 5 moe_event_t, none null): before the
+ * metadata, after the metadata, after the GEMM up, after the GEMM down and
+ * after the combine.  Used to time each stage on the launching stream.
+ */
+MOE_API int moe_nonexpand_forward_timed(const void *x, const int32_t *topk_idx, const float *topk_w,
+                                int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
+                                int64_t total_pairs,
+                                const void *w1, const void *b1, const void *w2, const void *b2,
+                                int32_t activation, int32_t gate_up_layout,
+                                void *out, const moe_meta_t *meta_out,
+                                void *ws, size_t ws_bytes, moe_stream_t stream,
+                                const moe_event_t *stage_events);
+
+/*
+ * The combine step alone (issue #68 dataflow, local_out [N,H]):
+ *   out[t,:] = bf16( sum over q in [token_offset[t], token_offset[t+1]), in q
+ *              order, of scores[q] * y[s_reverse_scatter_idx[q], :] )
+ * with an fp32 accumulator.  y is [P_cap,H] bf16 in expert-sorted order.
+ * Reads only the token_offset, s_reverse_scatter_idx and scores fields of
+ * `meta`.  No workspace is used.
+ */
+MOE_API int moe_nonexpand_combine(const void *y, const moe_meta_t *meta, int64_t N, int32_t H,
+                          void *out, moe_stream_t stream);
+
+/* Byte offsets of the workspace's internal arrays (for inspection and tests).
+ * Offsets of arrays that the given sizes do not need are 0. */
+typedef struct moe_ws_layout_t {
+    size_t total;              /* == moe_nonexpand_workspace_bytes(...)       */
+    size_t header;             /* 256-byte header; error word at byte 4       */
+    size_t tile_hist;          /* int32 [T,E] per-tile histograms, then bases */
+    size_t tile_valid;         /* int32 [T]                                   */
+    size_t tile_pair_base;     /* int32 [T]                                   */
+    size_t gemm_tile_offset;   /* int32 [E+1] prefix of ceil(freq/128)        */
+    size_t meta_freq, meta_off, meta_x_gather, meta_s_scatter, meta_s_rev,
+           meta_token_offset, meta_scores;  /* metadata kept in the workspace */
+    size_t h;                  /* bf16 [P_cap,I] */
+    size_t y;                  /* bf16 [P_cap,H] */
+    int64_t p_cap;
+    int32_t meta_tiles;        /* T */
+    int32_t meta_tile_slots;   /* slots per metadata tile */
+} moe_ws_layout_t;
+
+MOE_API int moe_nonexpand_workspace_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
+                                   int64_t total_pairs, moe_ws_layout_t *layout_out);
+
+/*
+ * Copies the device error word of the last call that used `ws` to *err_word
+ * (MOE_DEVERR_* bits; 0 = no error) after synchronising `stream`.  This is
+ * the only call that blocks the host.
+ */
+MOE_API int moe_nonexpand_read_error(const void *ws, moe_stream_t stream, uint32_t *err_word);
+
+/* Static string for a MOE_OK / MOE_ERR_* code. */
+MOE_API const char *moe_nonexpand_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_NONEXPAND_H */

@@ -1,0 +1,304 @@
+"""Thin ctypes binding of ``libmoe_nonexpand.so`` (C ABI in include/moe_nonexpand.h).
+
+Argument marshalling only: torch tensors are checked for dtype, shape,
+device and contiguity, and their device pointers plus the current CUDA stream
+are handed to the library; every step of the computation runs in the
+library's CUDA kernels.  The library is required: importing works anywhere,
+but any call without a built library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_nonexpand.so")
+
+MOE_OK = 0
+MOE_ERR_ARG = 1
+MOE_ERR_SHAPE = 2
+MOE_ERR_WS = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_DEVICE = 5
+
+DEVERR_BAD_EXPERT_ID = 0x1
+DEVERR_PAIR_COUNT = 0x2
+DEVERR_TIMEOUT = 0x4
+DEVERR_ABORTED = 0x8
+
+ACT_SWIGLU = 0
+LAYOUT_INTERLEAVED = 0
+LAYOUT_CONCATENATED = 1
+
+EXPORTED = (
+    "moe_nonexpand_workspace_bytes",
+    "moe_nonexpand_metadata",
+    "moe_nonexpand_forward",
+    "moe_nonexpand_forward_timed",
+    "moe_nonexpand_combine",
+    "moe_nonexpand_workspace_layout",
+    "moe_nonexpand_read_error",
+    "moe_nonexpand_strerror",
+)
+
+
+class MoeMeta(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "expert_frequency", "expert_frequency_offset", "x_gather_idx", "s_scatter_idx",
+        "s_reverse_scatter_idx", "token_offset", "scores")]
+
+
+class WsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in (
+        "total", "header", "tile_hist", "tile_valid", "tile_pair_base", "gemm_tile_offset",
+        "meta_freq", "meta_off", "meta_x_gather", "meta_s_scatter", "meta_s_rev",
+        "meta_token_offset", "meta_scores", "h", "y")] + [
+        ("p_cap", ctypes.c_int64), ("meta_tiles", ctypes.c_int32), ("meta_tile_slots", ctypes.c_int32)]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {strerror(status)} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the CUDA library (fails loudly when it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library missing: {LIB_PATH}; build it with "
+                           f"`python -m mixture_experts_routed_non_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    lib.moe_nonexpand_workspace_bytes.restype = sz
+    lib.moe_nonexpand_workspace_bytes.argtypes = [i64, i32, i32, i32, i32, i64]
+    lib.moe_nonexpand_metadata.restype = ctypes.c_int
+    lib.moe_nonexpand_metadata.argtypes = [P, P, i64, i32, i32, i64, ctypes.POINTER(MoeMeta), P, sz, P]
+    fwd = [P, P, P, i64, i32, i32, i32, i32, i64, P, P, P, P, i32, i32, P, ctypes.POINTER(MoeMeta), P, sz, P]
+    lib.moe_nonexpand_forward.restype = ctypes.c_int
+    lib.moe_nonexpand_forward.argtypes = fwd
+    lib.moe_nonexpand_forward_timed.restype = ctypes.c_int
+    lib.moe_nonexpand_forward_timed.argtypes = fwd + [P]
+    lib.moe_nonexpand_combine.restype = ctypes.c_int
+    lib.moe_nonexpand_combine.argtypes = [P, ctypes.POINTER(MoeMeta), i64, i32, P, P]
+    lib.moe_nonexpand_workspace_layout.restype = ctypes.c_int
+    lib.moe_nonexpand_workspace_layout.argtypes = [i64, i32, i32, i32, i32, i64, ctypes.POINTER(WsLayout)]
+    lib.moe_nonexpand_read_error.restype = ctypes.c_int
+    lib.moe_nonexpand_read_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.moe_nonexpand_strerror.restype = ctypes.c_char_p
+    lib.moe_nonexpand_strerror.argtypes = [ctypes.c_int]
+    _lib = lib
+    return lib
+
+
+def strerror(status: int) -> str:
+    return load().moe_nonexpand_strerror(status).decode()
+
+
+def _check(status: int, what: str):
+    if status != MOE_OK:
+        raise MoeError(status, what)
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape, device):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name}: expected device {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+# ---------------------------------------------------------------------------
+# Sizes and workspace
+# ---------------------------------------------------------------------------
+
+def p_cap(N: int, K: int, total_pairs: int = -1) -> int:
+    return total_pairs if total_pairs >= 0 else N * K
+
+
+def workspace_bytes(N: int, H: int, I: int, E: int, K: int, total_pairs: int = -1) -> int:
+    n = load().moe_nonexpand_workspace_bytes(N, H, I, E, K, total_pairs)
+    if n == 0:
+        raise MoeError(MOE_ERR_ARG, "moe_nonexpand_workspace_bytes")
+    return n
+
+
+def workspace_layout(N: int, H: int, I: int, E: int, K: int, total_pairs: int = -1) -> WsLayout:
+    out = WsLayout()
+    _check(load().moe_nonexpand_workspace_layout(N, H, I, E, K, total_pairs, ctypes.byref(out)),
+           "moe_nonexpand_workspace_layout")
+    return out
+
+
+def alloc_workspace(N: int, H: int, I: int, E: int, K: int, total_pairs: int = -1,
+                    device=None) -> torch.Tensor:
+    """A zero-filled workspace of the required size (zero-filled once, as
+    the library requires)."""
+    n = workspace_bytes(N, H, I, E, K, total_pairs)
+    return torch.zeros(n, dtype=torch.uint8, device=device or torch.device("cuda"))
+
+
+def alloc_meta(N: int, K: int, E: int, total_pairs: int = -1, device=None) -> dict:
+    dev = device or torch.device("cuda")
+    pc = max(1, p_cap(N, K, total_pairs))
+    i32 = torch.int32
+    return dict(
+        expert_frequency=torch.empty(E, dtype=i32, device=dev),
+        expert_frequency_offset=torch.empty(E + 1, dtype=i32, device=dev),
+        x_gather_idx=torch.empty(pc, dtype=i32, device=dev),
+        s_scatter_idx=torch.empty(pc, dtype=i32, device=dev),
+        s_reverse_scatter_idx=torch.empty(pc, dtype=i32, device=dev),
+        token_offset=torch.empty(N + 1, dtype=i32, device=dev),
+        scores=torch.empty(pc, dtype=torch.float32, device=dev),
+    )
+
+
+def _meta_struct(meta: dict) -> MoeMeta:
+    return MoeMeta(*[meta[f].data_ptr() for f, _ in MoeMeta._fields_])
+
+
+def meta_from_workspace(ws: torch.Tensor, N: int, H: int, I: int, E: int, K: int,
+                        total_pairs: int = -1) -> dict:
+    """Views of the metadata that moe_nonexpand_forward keeps in the workspace."""
+    lay = workspace_layout(N, H, I, E, K, total_pairs)
+    pc = lay.p_cap
+
+    def view(off, n, dtype):
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        return ws[off:off + nbytes].view(dtype)
+
+    return dict(
+        expert_frequency=view(lay.meta_freq, E, torch.int32),
+        expert_frequency_offset=view(lay.meta_off, E + 1, torch.int32),
+        x_gather_idx=view(lay.meta_x_gather, pc, torch.int32),
+        s_scatter_idx=view(lay.meta_s_scatter, pc, torch.int32),
+        s_reverse_scatter_idx=view(lay.meta_s_rev, pc, torch.int32),
+        token_offset=view(lay.meta_token_offset, N + 1, torch.int32),
+        scores=view(lay.meta_scores, pc, torch.float32),
+    )
+
+
+def intermediates_from_workspace(ws: torch.Tensor, N: int, H: int, I: int, E: int, K: int,
+                                 total_pairs: int = -1):
+    """Views (h [P_cap,I], y [P_cap,H], both bf16, expert-sorted rows) of the
+    intermediates that moe_nonexpand_forward keeps in the workspace."""
+    lay = workspace_layout(N, H, I, E, K, total_pairs)
+    pc = lay.p_cap
+    h = ws[lay.h:lay.h + pc * I * 2].view(torch.bfloat16).view(pc, I)
+    y = ws[lay.y:lay.y + pc * H * 2].view(torch.bfloat16).view(pc, H)
+    return h, y
+
+
+# ---------------------------------------------------------------------------
+# Entry points
+# ---------------------------------------------------------------------------
+
+def metadata(topk_idx: torch.Tensor, topk_w: torch.Tensor, E: int, total_pairs: int = -1,
+             meta: Optional[dict] = None, ws: Optional[torch.Tensor] = None,
+             stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """Routing metadata of [N,K] (moe_nonexpand_metadata).  Returns the dict of
+    device tensors (P_cap-sized pair arrays; the first P entries are valid)."""
+    N, K = topk_idx.shape
+    dev = topk_idx.device
+    _need(topk_idx, "topk_idx", torch.int32, (N, K), dev)
+    _need(topk_w, "topk_w", torch.float32, (N, K), dev)
+    if meta is None:
+        meta = alloc_meta(N, K, E, total_pairs, dev)
+    if ws is None:
+        ws = alloc_workspace(N, 0, 0, E, K, total_pairs, dev)
+    m = _meta_struct(meta)
+    _check(load().moe_nonexpand_metadata(topk_idx.data_ptr(), topk_w.data_ptr(), N, K, E, total_pairs,
+                                         ctypes.byref(m), ws.data_ptr(), ws.numel(), _stream_handle(stream)),
+           "moe_nonexpand_metadata")
+    return meta
+
+
+def forward(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
+            w1: torch.Tensor, w2: torch.Tensor, b1: Optional[torch.Tensor] = None,
+            b2: Optional[torch.Tensor] = None, *, layout: int = LAYOUT_INTERLEAVED,
+            total_pairs: int = -1, out: Optional[torch.Tensor] = None,
+            ws: Optional[torch.Tensor] = None, meta: Optional[dict] = None,
+            stream: Optional[torch.cuda.Stream] = None,
+            events: Optional[Sequence[torch.cuda.Event]] = None) -> torch.Tensor:
+    """Local expert forward on the non-expand layout (moe_nonexpand_forward).
+
+    x [N,H] bf16, topk_idx [N,K] int32 (-1 = invalid slot), topk_w [N,K] fp32,
+    w1 [E,H,2I], w2 [E,I,H], b1 [E,2I] / b2 [E,H] bf16 or None.  Returns
+    out [N,H] bf16.  ``events`` (five timing-enabled CUDA events) are recorded
+    before/after each stage on the launching stream."""
+    N, H = x.shape
+    K = topk_idx.shape[1]
+    E, H1, I2 = w1.shape
+    I = I2 // 2
+    dev = x.device
+    _need(x, "x", torch.bfloat16, (N, H), dev)
+    _need(topk_idx, "topk_idx", torch.int32, (N, K), dev)
+    _need(topk_w, "topk_w", torch.float32, (N, K), dev)
+    _need(w1, "w1", torch.bfloat16, (E, H, 2 * I), dev)
+    _need(w2, "w2", torch.bfloat16, (E, I, H), dev)
+    if b1 is not None:
+        _need(b1, "b1", torch.bfloat16, (E, 2 * I), dev)
+    if b2 is not None:
+        _need(b2, "b2", torch.bfloat16, (E, H), dev)
+    if out is None:
+        out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (N, H), dev)
+    if ws is None:
+        ws = alloc_workspace(N, H, I, E, K, total_pairs, dev)
+    m = _meta_struct(meta) if meta is not None else None
+    mp = ctypes.byref(m) if m is not None else None
+    args = (x.data_ptr(), topk_idx.data_ptr(), topk_w.data_ptr(), N, H, I, E, K, total_pairs,
+            w1.data_ptr(), _ptr(b1), w2.data_ptr(), _ptr(b2), ACT_SWIGLU, layout,
+            out.data_ptr(), mp, ws.data_ptr(), ws.numel(), _stream_handle(stream))
+    lib = load()
+    if events is None:
+        _check(lib.moe_nonexpand_forward(*args), "moe_nonexpand_forward")
+    else:
+        if len(events) != 5:
+            raise ValueError("events: expected 5 CUDA events")
+        arr = (ctypes.c_void_p * 5)(*[ev.cuda_event for ev in events])
+        _check(lib.moe_nonexpand_forward_timed(*args, arr), "moe_nonexpand_forward_timed")
+    return out
+
+
+def combine(y: torch.Tensor, meta: dict, N: int, out: Optional[torch.Tensor] = None,
+            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """The combine step alone (moe_nonexpand_combine): y [P_cap,H] bf16 in
+    expert-sorted order -> out [N,H] bf16."""
+    H = y.shape[1]
+    if y.dtype != torch.bfloat16 or not y.is_contiguous():
+        raise TypeError("y: expected contiguous bf16")
+    if out is None:
+        out = torch.empty((N, H), dtype=torch.bfloat16, device=y.device)
+    m = _meta_struct(meta)
+    _check(load().moe_nonexpand_combine(y.data_ptr(), ctypes.byref(m), N, H, out.data_ptr(),
+                                        _stream_handle(stream)), "moe_nonexpand_combine")
+    return out
+
+
+def read_error(ws: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """The device error word of the last call that used ``ws`` (syncs the stream)."""
+    v = ctypes.c_uint32(0)
+    _check(load().moe_nonexpand_read_error(ws.data_ptr(), _stream_handle(stream), ctypes.byref(v)),
+           "moe_nonexpand_read_error")
+    return int(v.value)

@@ -1,0 +1,429 @@
+// Host side of the C ABI declared in include/moe_nonexpand.h: argument
+// checks, workspace layout, tensor-map encoding and the launch sequence
+//   metadata (count + last-block scan, scatter) -> grouped GEMM up (+b1,
+//   SwiGLU) -> grouped GEMM down (+b2) -> combine
+// all on the caller's stream, with no host synchronisation (the proposed
+// entry point of sonic-moe issue #68 takes a stream and is meant to be
+// sync-free when the pair count comes from the caller).
+#include <mutex>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+
+
+namespace moe {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Layout {
+    moe_ws_layout_t l;
+};
+
+// Slots per metadata tile: a multiple of the block size, sized so that the
+// grid holds about two CTAs per SM of a B200, capped to keep the per-tile
+// histogram table small.
+void meta_tiling(int64_t NK, int32_t *tile_slots, int32_t *tiles) {
+    const int64_t target_ctas = 2 * 148;
+    int64_t c = (NK + (int64_t)kMetaThreads * target_ctas - 1) / ((int64_t)kMetaThreads * target_ctas);
+    if (c < 1) c = 1;
+    if (c > 256) c = 256;
+    const int64_t S = kMetaThreads * c;
+    int64_t T = (NK + S - 1) / S;
+    if (T < 1) T = 1;
+    *tile_slots = (int32_t)S;
+    *tiles = (int32_t)T;
+}
+
+int check_sizes(int64_t N, int32_t E, int32_t K, int64_t total_pairs) {
+    if (N < 0 || K < 1 || K > 32 || E < 1 || E > kMaxExperts) return MOE_ERR_ARG;
+    if (N * (int64_t)K >= (int64_t)(1u << 31) - (1 << 20)) return MOE_ERR_ARG;
+    if (total_pairs < -1 || total_pairs > N * K) return MOE_ERR_ARG;
+    return MOE_OK;
+}
+
+int check_dense(int64_t p_cap, int32_t H, int32_t I, int32_t E) {
+    if (H <= 0 || I <= 0 || (H % 64) != 0 || (I % 64) != 0) return MOE_ERR_SHAPE;
+    const int64_t big = (int64_t)1 << 31;
+    if ((int64_t)E * H >= big || (int64_t)E * I >= big) return MOE_ERR_SHAPE;
+    if (p_cap * (int64_t)H >= big * 8 || p_cap * (int64_t)I >= big * 8) return MOE_ERR_SHAPE;
+    return MOE_OK;
+}
+
+moe_ws_layout_t compute_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K, int64_t total_pairs) {
+    moe_ws_layout_t l;
+    memset(&l, 0, sizeof l);
+    const int64_t NK = N * K;
+    const int64_t pc = total_pairs >= 0 ? total_pairs : NK;
+    l.p_cap = pc;
+    meta_tiling(NK, &l.meta_tile_slots, &l.meta_tiles);
+    const size_t T = (size_t)l.meta_tiles;
+    size_t o = 0;
+    l.header = o;
+    o = align_up(o + sizeof(WsHeader), kAlign);
+    l.tile_hist = o;
+    o = align_up(o + T * E * 4, kAlign);
+    l.tile_valid = o;
+    o = align_up(o + T * 4, kAlign);
+    l.tile_pair_base = o;
+    o = align_up(o + T * 4, kAlign);
+    const size_t tile_err = o;  // follows tile_pair_base
+    o = align_up(tile_err + T * 4, kAlign);
+    l.gemm_tile_offset = o;
+    o = align_up(o + (size_t)(E + 1) * 4, kAlign);
+    l.meta_freq = o;
+    o = align_up(o + (size_t)E * 4, kAlign);
+    l.meta_off = o;
+    o = align_up(o + (size_t)(E + 1) * 4, kAlign);
+    l.meta_x_gather = o;
+    o = align_up(o + (size_t)pc * 4, kAlign);
+    l.meta_s_scatter = o;
+    o = align_up(o + (size_t)pc * 4, kAlign);
+    l.meta_s_rev = o;
+    o = align_up(o + (size_t)pc * 4, kAlign);
+    l.meta_token_offset = o;
+    o = align_up(o + (size_t)(N + 1) * 4, kAlign);
+    l.meta_scores = o;
+    o = align_up(o + (size_t)pc * 4, kAlign);
+    if (H > 0 && I > 0) {
+        o = align_up(o, 1024);
+        l.h = o;
+        o = align_up(o + (size_t)pc * I * 2, 1024);
+        l.y = o;
+        o = align_up(o + (size_t)pc * H * 2, 1024);
+    }
+    l.total = o;
+    return l;
+}
+
+size_t tile_err_offset(const moe_ws_layout_t &l) { return align_up(l.tile_pair_base + (size_t)l.meta_tiles * 4, kAlign); }
+
+// ---------------------------------------------------------------------------
+// Per-device facts.
+// ---------------------------------------------------------------------------
+struct DeviceInfo {
+    bool ok = false;
+    int sms = 0;
+    int status = MOE_ERR_DEVICE;
+};
+
+int device_info(DeviceInfo *out) {
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    static bool have[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 0 || dev >= 64) return MOE_ERR_DEVICE;
+    if (!have[dev]) {
+        DeviceInfo d;
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        d.sms = sms;
+        d.ok = (major == 10 && minor == 0);
+        d.status = d.ok ? MOE_OK : MOE_ERR_DEVICE;
+        cache[dev] = d;
+        have[dev] = true;
+    }
+    *out = cache[dev];
+    return out->status;
+}
+
+// ---------------------------------------------------------------------------
+// Tensor maps through the driver entry point (no link against libcuda).
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                 uint32_t box_outer) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// w1 in the concatenated layout viewed as [rows][2][I]: (i, half, row).
+bool make_map_w1_concat(CUtensorMap *m, const void *ptr, uint64_t I, uint64_t rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {I, 2, rows};
+    cuuint64_t strides[2] = {I * 2, I * 4};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kBK};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+MetaArgs meta_args(const int32_t *topk_idx, const float *topk_w, int64_t N, int32_t K, int32_t E,
+                   int64_t total_pairs, const moe_ws_layout_t &l, uint8_t *ws, const moe_meta_t &meta) {
+    MetaArgs a;
+    a.topk_idx = topk_idx;
+    a.topk_w = topk_w;
+    a.NK = N * K;
+    a.K = K;
+    a.E = E;
+    a.total_pairs = total_pairs;
+    a.p_cap = l.p_cap;
+    a.tiles = l.meta_tiles;
+    a.tile_slots = l.meta_tile_slots;
+    a.hdr = reinterpret_cast<WsHeader *>(ws + l.header);
+    a.tile_hist = reinterpret_cast<int32_t *>(ws + l.tile_hist);
+    a.tile_valid = reinterpret_cast<int32_t *>(ws + l.tile_valid);
+    a.tile_pbase = reinterpret_cast<int32_t *>(ws + l.tile_pair_base);
+    a.tile_err = reinterpret_cast<int32_t *>(ws + tile_err_offset(l));
+    a.gemm_tile_off = reinterpret_cast<int32_t *>(ws + l.gemm_tile_offset);
+    a.meta = meta;
+    a.N = N;
+    return a;
+}
+
+moe_meta_t ws_meta(const moe_ws_layout_t &l, uint8_t *ws) {
+    moe_meta_t m;
+    m.expert_frequency = reinterpret_cast<int32_t *>(ws + l.meta_freq);
+    m.expert_frequency_offset = reinterpret_cast<int32_t *>(ws + l.meta_off);
+    m.x_gather_idx = reinterpret_cast<int32_t *>(ws + l.meta_x_gather);
+    m.s_scatter_idx = reinterpret_cast<int32_t *>(ws + l.meta_s_scatter);
+    m.s_reverse_scatter_idx = reinterpret_cast<int32_t *>(ws + l.meta_s_rev);
+    m.token_offset = reinterpret_cast<int32_t *>(ws + l.meta_token_offset);
+    m.scores = reinterpret_cast<float *>(ws + l.meta_scores);
+    return m;
+}
+
+bool meta_complete(const moe_meta_t *m) {
+    return m && m->expert_frequency && m->expert_frequency_offset && m->x_gather_idx && m->s_scatter_idx &&
+           m->s_reverse_scatter_idx && m->token_offset && m->scores;
+}
+
+int record(const moe_event_t *ev, int i, cudaStream_t s) {
+    if (!ev) return MOE_OK;
+    return cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, int64_t N, int32_t H, int32_t I,
+                 int32_t E, int32_t K, int64_t total_pairs, const void *w1, const void *b1, const void *w2,
+                 const void *b2, int32_t activation, int32_t layout_kind, void *out, const moe_meta_t *meta_out,
+                 void *ws, size_t ws_bytes, cudaStream_t s, const moe_event_t *ev) {
+    int st = check_sizes(N, E, K, total_pairs);
+    if (st) return st;
+    if (!x || !topk_idx || !topk_w || !w1 || !w2 || !out) return MOE_ERR_ARG;
+    if (activation != MOE_ACT_SWIGLU) return MOE_ERR_ARG;
+    if (layout_kind != MOE_LAYOUT_INTERLEAVED && layout_kind != MOE_LAYOUT_CONCATENATED) return MOE_ERR_ARG;
+    if (meta_out && !meta_complete(meta_out)) return MOE_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(out, 16) ||
+        (b1 && !aligned(b1, 16)) || (b2 && !aligned(b2, 16)) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+        return MOE_ERR_ARG;
+    const moe_ws_layout_t l = compute_layout(N, H, I, E, K, total_pairs);
+    st = check_dense(l.p_cap, H, I, E);
+    if (st) return st;
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MOE_ERR_WS;
+    DeviceInfo dev;
+    st = device_info(&dev);
+    if (st) return st;
+
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    const moe_meta_t meta = meta_out ? *meta_out : ws_meta(l, w);
+    const MetaArgs ma = meta_args(topk_idx, topk_w, N, K, E, total_pairs, l, w, meta);
+    WsHeader *hdr = ma.hdr;
+
+    if ((st = record(ev, 0, s))) return st;
+    if (launch_meta(ma, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((st = record(ev, 1, s))) return st;
+
+    __nv_bfloat16 *hbuf = reinterpret_cast<__nv_bfloat16 *>(w + l.h);
+    __nv_bfloat16 *ybuf = reinterpret_cast<__nv_bfloat16 *>(w + l.y);
+    if (l.p_cap > 0) {
+        const int64_t cap_mtiles = (l.p_cap + kBM - 1) / kBM + E;
+        // ---- up: x gathered rows . w1 -> h
+        GemmArgs up;
+        memset(&up, 0, sizeof up);
+        if (!make_map_2d(&up.tmap_a, x, (uint64_t)H, (uint64_t)N, 64, 1)) return MOE_ERR_CUDA;
+        if (layout_kind == MOE_LAYOUT_CONCATENATED) {
+            if (!make_map_w1_concat(&up.tmap_b, w1, (uint64_t)I, (uint64_t)E * H)) return MOE_ERR_CUDA;
+        } else {
+            if (!make_map_2d(&up.tmap_b, w1, (uint64_t)2 * I, (uint64_t)E * H, 64, kBK)) return MOE_ERR_CUDA;
+        }
+        up.x_gather_idx = meta.x_gather_idx;
+        up.expert_off = meta.expert_frequency_offset;
+        up.tile_off = ma.gemm_tile_off;
+        up.bias = static_cast<const __nv_bfloat16 *>(b1);
+        up.out = hbuf;
+        up.hdr = hdr;
+        up.E = E;
+        up.k_dim = H;
+        up.n_dim = 2 * I;
+        up.n_tiles = (2 * I + kBN - 1) / kBN;
+        up.out_cols = I;
+        up.I = I;
+        up.layout = layout_kind;
+        int64_t grid = cap_mtiles * up.n_tiles;
+        if (grid > dev.sms) grid = dev.sms;
+        if (launch_gemm_up(up, (int)grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if ((st = record(ev, 2, s))) return st;
+
+        // ---- down: h . w2 -> y
+        GemmArgs dn;
+        memset(&dn, 0, sizeof dn);
+        if (!make_map_2d(&dn.tmap_a, hbuf, (uint64_t)I, (uint64_t)l.p_cap, 64, kBM)) return MOE_ERR_CUDA;
+        if (!make_map_2d(&dn.tmap_b, w2, (uint64_t)H, (uint64_t)E * I, 64, kBK)) return MOE_ERR_CUDA;
+        dn.expert_off = meta.expert_frequency_offset;
+        dn.tile_off = ma.gemm_tile_off;
+        dn.bias = static_cast<const __nv_bfloat16 *>(b2);
+        dn.out = ybuf;
+        dn.hdr = hdr;
+        dn.E = E;
+        dn.k_dim = I;
+        dn.n_dim = H;
+        dn.n_tiles = (H + kBN - 1) / kBN;
+        dn.out_cols = H;
+        dn.I = I;
+        dn.layout = MOE_LAYOUT_INTERLEAVED;
+        grid = cap_mtiles * dn.n_tiles;
+        if (grid > dev.sms) grid = dev.sms;
+        if (launch_gemm_down(dn, (int)grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if ((st = record(ev, 3, s))) return st;
+    } else {
+        if ((st = record(ev, 2, s))) return st;
+        if ((st = record(ev, 3, s))) return st;
+    }
+    if (launch_combine(ybuf, meta.token_offset, meta.s_reverse_scatter_idx, meta.scores, N, H,
+                       static_cast<__nv_bfloat16 *>(out), hdr, dev.sms, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if ((st = record(ev, 4, s))) return st;
+    return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" MOE_API size_t moe_nonexpand_workspace_bytes(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
+                                             int64_t total_pairs) {
+    if (check_sizes(N, E, K, total_pairs)) return 0;
+    if (H < 0 || I < 0) return 0;
+    const moe_ws_layout_t l = compute_layout(N, H, I, E, K, total_pairs);
+    if (H > 0 || I > 0) {
+        if (check_dense(l.p_cap, H, I, E)) return 0;
+    }
+    return l.total;
+}
+
+extern "C" MOE_API int moe_nonexpand_workspace_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
+                                           int64_t total_pairs, moe_ws_layout_t *layout_out) {
+    if (!layout_out) return MOE_ERR_ARG;
+    int st = check_sizes(N, E, K, total_pairs);
+    if (st) return st;
+    if (H < 0 || I < 0) return MOE_ERR_SHAPE;
+    *layout_out = compute_layout(N, H, I, E, K, total_pairs);
+    return MOE_OK;
+}
+
+extern "C" MOE_API int moe_nonexpand_metadata(const int32_t *topk_idx, const float *topk_w, int64_t N, int32_t K,
+                                   int32_t E, int64_t total_pairs, const moe_meta_t *meta, void *ws,
+                                   size_t ws_bytes, moe_stream_t stream) {
+    int st = check_sizes(N, E, K, total_pairs);
+    if (st) return st;
+    if (!topk_idx || !topk_w || !meta_complete(meta)) return MOE_ERR_ARG;
+    if (!aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_ARG;
+    const moe_ws_layout_t l = compute_layout(N, 0, 0, E, K, total_pairs);
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MOE_ERR_WS;
+    DeviceInfo dev;
+    st = device_info(&dev);
+    if (st) return st;
+    const MetaArgs ma = meta_args(topk_idx, topk_w, N, K, E, total_pairs, l, static_cast<uint8_t *>(ws), *meta);
+    return launch_meta(ma, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" MOE_API int moe_nonexpand_forward(const void *x, const int32_t *topk_idx, const float *topk_w, int64_t N,
+                                  int32_t H, int32_t I, int32_t E, int32_t K, int64_t total_pairs,
+                                  const void *w1, const void *b1, const void *w2, const void *b2,
+                                  int32_t activation, int32_t gate_up_layout, void *out,
+                                  const moe_meta_t *meta_out, void *ws, size_t ws_bytes, moe_stream_t stream) {
+    return forward_impl(x, topk_idx, topk_w, N, H, I, E, K, total_pairs, w1, b1, w2, b2, activation,
+                        gate_up_layout, out, meta_out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                        nullptr);
+}
+
+extern "C" MOE_API int moe_nonexpand_forward_timed(const void *x, const int32_t *topk_idx, const float *topk_w, int64_t N,
+                                        int32_t H, int32_t I, int32_t E, int32_t K, int64_t total_pairs,
+                                        const void *w1, const void *b1, const void *w2, const void *b2,
+                                        int32_t activation, int32_t gate_up_layout, void *out,
+                                        const moe_meta_t *meta_out, void *ws, size_t ws_bytes,
+                                        moe_stream_t stream, const moe_event_t *stage_events) {
+    if (!stage_events) return MOE_ERR_ARG;
+    for (int i = 0; i < 5; ++i)
+        if (!stage_events[i]) return MOE_ERR_ARG;
+    return forward_impl(x, topk_idx, topk_w, N, H, I, E, K, total_pairs, w1, b1, w2, b2, activation,
+                        gate_up_layout, out, meta_out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                        stage_events);
+}
+
+extern "C" MOE_API int moe_nonexpand_combine(const void *y, const moe_meta_t *meta, int64_t N, int32_t H, void *out,
+                                  moe_stream_t stream) {
+    if (!y || !meta || !meta->token_offset || !meta->s_reverse_scatter_idx || !meta->scores || !out)
+        return MOE_ERR_ARG;
+    if (N < 0) return MOE_ERR_ARG;
+    if (H <= 0 || (H % 64) != 0) return MOE_ERR_SHAPE;
+    if (!aligned(y, 16) || !aligned(out, 16)) return MOE_ERR_ARG;
+    DeviceInfo dev;
+    int st = device_info(&dev);
+    if (st) return st;
+    return launch_combine(static_cast<const __nv_bfloat16 *>(y), meta->token_offset, meta->s_reverse_scatter_idx,
+                          meta->scores, N, H, static_cast<__nv_bfloat16 *>(out), nullptr, dev.sms,
+                          reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+extern "C" MOE_API int moe_nonexpand_read_error(const void *ws, moe_stream_t stream, uint32_t *err_word) {
+    if (!ws || !err_word) return MOE_ERR_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const WsHeader *hdr = static_cast<const WsHeader *>(ws);
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, &hdr->err, sizeof v, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    *err_word = v;
+    return MOE_OK;
+}
+
+extern "C" MOE_API const char *moe_nonexpand_strerror(int status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_ARG: return "invalid argument";
+        case MOE_ERR_SHAPE: return "unsupported shape (H and I must be multiples of 64)";
+        case MOE_ERR_WS: return "workspace missing, misaligned or too small";
+        case MOE_ERR_CUDA: return "CUDA runtime or launch failure";
+        case MOE_ERR_DEVICE: return "current device is not an sm_100 (B200-class) GPU";
+        default: return "unknown status";
+    }
+}

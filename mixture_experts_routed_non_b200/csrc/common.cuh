@@ -1,0 +1,299 @@
+// Shared definitions of the CUDA library: workspace header, launch-side
+// structs and the sm_100a inline-PTX primitives the kernels use (mbarrier,
+// TMA bulk-tensor loads, tcgen05 MMA / TMEM).  Only this library includes it.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe_nonexpand.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// Workspace header (first 256 bytes of the workspace).
+// ---------------------------------------------------------------------------
+struct WsHeader {
+    uint32_t ticket;   // blocks of the count kernel that finished; reset to 0 by the last one
+    uint32_t err;      // MOE_DEVERR_* bits of the current call
+    int32_t P;         // pairs counted on the device
+    uint32_t abort;    // nonzero: later kernels of this call skip their work
+    uint32_t pad[60];
+};
+static_assert(sizeof(WsHeader) == 256, "header size");
+
+// Tile sizes of the grouped GEMMs.
+constexpr int kBM = 128;        // rows (pairs) per tile = UMMA M
+constexpr int kBN = 256;        // accumulator columns per tile = UMMA N
+constexpr int kBK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
+constexpr int kStages = 4;      // shared-memory pipeline depth
+
+// Metadata kernels.
+constexpr int kMetaThreads = 512;
+constexpr int kMetaWarps = kMetaThreads / 32;
+constexpr int kMaxExperts = 1024;
+
+// Timeout of every pipeline wait (ns of %globaltimer).
+constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;
+
+// ---------------------------------------------------------------------------
+// Host-side launch descriptions (filled by capi.cu).
+// ---------------------------------------------------------------------------
+struct MetaArgs {
+    const int32_t *topk_idx;
+    const float *topk_w;
+    int64_t NK;
+    int32_t K;
+    int32_t E;
+    int64_t total_pairs;  // -1: unknown
+    int64_t p_cap;
+    int32_t tiles;        // T
+    int32_t tile_slots;   // slots per tile
+    WsHeader *hdr;
+    int32_t *tile_hist;   // [T,E]
+    int32_t *tile_valid;  // [T]
+    int32_t *tile_pbase;  // [T]
+    int32_t *tile_err;    // [T] (alias of nothing else)
+    int32_t *gemm_tile_off;  // [E+1]
+    moe_meta_t meta;
+    int64_t N;
+};
+
+struct GemmArgs {
+    CUtensorMap tmap_a;       // up: x [N,H] (gather4 rows); down: h [P_cap,I]
+    CUtensorMap tmap_b;       // up: w1; down: w2
+    const int32_t *x_gather_idx;
+    const int32_t *expert_off;    // [E+1]
+    const int32_t *tile_off;      // [E+1]
+    const __nv_bfloat16 *bias;    // b1 [E,2I] / b2 [E,H] or null
+    __nv_bfloat16 *out;           // h [P_cap,I] / y [P_cap,H]
+    WsHeader *hdr;
+    int32_t E;
+    int32_t k_dim;        // H (up) / I (down)
+    int32_t n_dim;        // 2I (up) / H (down): accumulator columns of one expert
+    int32_t n_tiles;      // ceil(n_dim / kBN)
+    int32_t out_cols;     // I (up) / H (down)
+    int32_t I;            // intermediate size (up, concatenated layout)
+    int32_t layout;       // MOE_LAYOUT_*
+};
+
+// Launchers (each defined next to its kernel).
+cudaError_t launch_meta(const MetaArgs &a, cudaStream_t s);
+cudaError_t launch_gemm_up(const GemmArgs &a, int grid, cudaStream_t s);
+cudaError_t launch_gemm_down(const GemmArgs &a, int grid, cudaStream_t s);
+cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *token_offset, const int32_t *s_rev,
+                           const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
+                           const WsHeader *hdr, int num_sms, cudaStream_t s);
+size_t gemm_smem_bytes();
+
+// ---------------------------------------------------------------------------
+// Device primitives.
+// ---------------------------------------------------------------------------
+#if defined(__CUDACC__)
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// --- mbarrier ---------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `parity` to complete.  Gives up (returns false) when
+// another role of the CTA raised *abort or after kWaitTimeoutNs, in which case
+// it raises *abort itself.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  volatile uint32_t *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 31u) == 0) {
+            if (*abort) return false;
+            if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+                *abort = 1u;
+                return false;
+            }
+        }
+    }
+}
+
+// Same, ignoring the abort flag: used only to drain copies already in flight.
+__device__ __forceinline__ bool mbar_wait_timed(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (globaltimer_ns() - t0 > kWaitTimeoutNs) return false;
+    }
+}
+
+// --- TMA (tensor bulk copies, CTA-local destination, no multicast) ----------
+__device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint32_t bar, int32_t c0,
+                                            int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, uint32_t bar, int32_t c0,
+                                            int32_t c1, int32_t c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// Four rows (r0..r3) of a 2-D tensor, columns [c0, c0 + box), into four
+// consecutive 128-byte rows of shared memory.  The tensor map's box is one row
+// high.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, uint32_t bar, int32_t c0,
+                                            int32_t r0, int32_t r1, int32_t r2, int32_t r3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
+// --- tcgen05 / TMEM ---------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16 in, fp32 accumulate).
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive once on `bar` when all previously issued tcgen05 async ops of this
+// thread have completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i gets lane (base_lane + i).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05), 128-byte swizzle.
+//   bits  0-13 start address >> 4; 16-29 leading byte offset >> 4;
+//   32-45 stride byte offset >> 4; 46-47 version (1 on sm_100);
+//   49-51 base offset (0: atoms 1024-byte aligned); 61-63 layout (2 = 128B swizzle).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= 1ull << 46;
+    d |= 2ull << 61;
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B,
+// A K-major, B MN-major (N contiguous), shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+    return (1u << 4)                              // D format: f32
+           | (1u << 7)                            // A format: bf16
+           | (1u << 10)                           // B format: bf16
+           | ((b_mn_major ? 1u : 0u) << 16)       // B major
+           | ((static_cast<uint32_t>(N) >> 3) << 17)
+           | ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+#endif  // __CUDACC__
+
+}  // namespace moe

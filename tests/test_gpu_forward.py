@@ -1,0 +1,179 @@
+"""GPU forward (moe_nonexpand_forward) against the oracle.
+
+Small cases are compared element by element on every output; the full-size
+workloads, in the launch configuration the benchmark times, are compared on a
+seeded sample of tokens the oracle computes one by one.  Metadata is compared
+bit-exactly in every case, and the bf16 intermediates h and y are checked
+against the oracle's per-pair rows so a failure points at the stage.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_close, check_meta_equal, to_np, within_tolerance
+from mixture_experts_routed_non_b200 import binding, synthetic
+
+pytestmark = pytest.mark.gpu
+
+
+def _concat_from_interleaved(w1, b1):
+    w1c = torch.cat([w1[:, :, 0::2], w1[:, :, 1::2]], dim=2).contiguous()
+    b1c = None if b1 is None else torch.cat([b1[:, 0::2], b1[:, 1::2]], dim=1).contiguous()
+    return w1c, b1c
+
+
+def run_case(inp, layout=0, total_pairs=-1, sample=None, check_stages=True, seed=0):
+    wl = inp.wl
+    N, H, I, E, K = wl.N, wl.H, wl.I, wl.E, wl.K
+    w1, b1 = inp.w1, inp.b1
+    if layout == 1:
+        w1, b1 = _concat_from_interleaved(w1, b1)
+    ws = binding.alloc_workspace(N, H, I, E, K, total_pairs, inp.x.device)
+    out = binding.forward(inp.x, inp.topk_idx, inp.topk_w, w1, inp.w2, b1, inp.b2, layout=layout,
+                          total_pairs=total_pairs, ws=ws)
+    err = binding.read_error(ws)
+    assert err == 0, f"device error word {err:#x}"
+
+    idx = inp.topk_idx.cpu().numpy()
+    w = inp.topk_w.cpu().numpy()
+    ref_meta = oracle.metadata(idx, w, E)
+    check_meta_equal(binding.meta_from_workspace(ws, N, H, I, E, K, total_pairs), ref_meta)
+
+    wts = oracle.Weights(inp.x, w1, b1, inp.w2, inp.b2)
+    if sample is None:
+        tokens = np.arange(N)
+    else:
+        tokens = np.sort(np.random.default_rng(seed).choice(N, size=min(sample, N), replace=False))
+    if check_stages and ref_meta["P"] > 0:
+        # intermediates of the pairs of the sampled tokens
+        P = ref_meta["P"]
+        h_gpu, y_gpu = binding.intermediates_from_workspace(ws, N, H, I, E, K, total_pairs)
+        to = ref_meta["token_offset"]
+        qs = np.concatenate([np.arange(to[t], to[t + 1]) for t in tokens[:64]] + [np.zeros(0, np.int64)])
+        if qs.size:
+            ps = ref_meta["s_reverse_scatter_idx"][qs]
+            tok = ref_meta["x_gather_idx"][ps]
+            ex = np.searchsorted(ref_meta["off"], ps, side="right") - 1
+            h_ref, y_ref = oracle.pair_rows(wts, tok, ex, layout=layout)
+            ps_t = torch.from_numpy(ps.astype(np.int64)).to(h_gpu.device)
+            assert_close(to_np(h_gpu[ps_t]), h_ref, "h (up GEMM + SwiGLU)")
+            assert_close(to_np(y_gpu[ps_t]), y_ref, "y (down GEMM)")
+            assert P <= h_gpu.shape[0]
+    ref = oracle.forward_rows(wts, idx, w, tokens=tokens, layout=layout)
+    got = to_np(out)[tokens]
+    assert_close(got, ref, f"out ({wl.name}, layout {layout})")
+    return out, ws
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_tiny_workload_full(layout):
+    inp = synthetic.make_inputs("tiny", device="cuda", invalid_value=float("nan"))
+    run_case(inp, layout=layout)
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_tiny_workload_with_total_pairs(layout):
+    inp = synthetic.make_inputs("tiny", device="cuda")
+    run_case(inp, layout=layout, total_pairs=inp.total_pairs)
+
+
+@pytest.mark.parametrize("N,H,I,E,K,p_invalid,bias,seed", [
+    (1, 64, 64, 1, 1, 0.0, True, 1),          # one token, one expert, smallest tile
+    (300, 256, 192, 5, 3, 0.2, True, 2),      # I % 128 == 64: partial last column tile
+    (129, 192, 128, 3, 2, 0.0, False, 3),     # H % 256 == 192: partial down tile
+    (700, 128, 64, 9, 4, 0.3, True, 4),       # I = 64
+    (1000, 512, 256, 64, 8, 0.1, False, 5),   # many small segments
+    (64, 320, 320, 2, 1, 0.5, True, 6),
+])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_ragged_shapes_full(N, H, I, E, K, p_invalid, bias, seed, layout):
+    wl = synthetic.custom(N, H, I, E, K, p_invalid=p_invalid, bias=bias, seed=seed,
+                          routing_kind="uniform" if K <= E else "ranklocal")
+    if K > E:
+        pytest.skip("distinct routing needs K <= E")
+    inp = synthetic.make_inputs(wl, device="cuda", invalid_value=float("nan"))
+    run_case(inp, layout=layout)
+
+
+def test_single_expert_single_slot_dense():
+    wl = synthetic.custom(1000, 256, 256, 1, 1, bias=True, seed=7, scores_kind="uniform")
+    inp = synthetic.make_inputs(wl, device="cuda")
+    inp.topk_w.fill_(1.0)
+    run_case(inp)
+
+
+def test_duplicate_experts_and_tail_segments():
+    """Long segments that are not a multiple of 128 rows, with the same expert
+    twice in a row."""
+    wl = synthetic.custom(2000, 128, 128, 4, 2, bias=True, seed=8)
+    inp = synthetic.make_inputs(wl, device="cuda")
+    idx = torch.tensor(np.random.default_rng(8).integers(0, 4, size=(2000, 2)), dtype=torch.int32)
+    inp.topk_idx.copy_(idx)
+    run_case(inp)
+
+
+def test_all_slots_invalid_gives_zero():
+    wl = synthetic.custom(50, 128, 64, 3, 2, seed=9)
+    inp = synthetic.make_inputs(wl, device="cuda")
+    inp.topk_idx.fill_(-1)
+    inp.topk_w.fill_(float("nan"))
+    ws = binding.alloc_workspace(50, 128, 64, 3, 2, -1)
+    out = binding.forward(inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, ws=ws)
+    assert binding.read_error(ws) == 0
+    assert torch.count_nonzero(out) == 0
+    out = binding.forward(inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, total_pairs=0)
+    assert torch.count_nonzero(out) == 0
+
+
+def test_forward_deterministic():
+    inp = synthetic.make_inputs("tiny", device="cuda")
+    ws = binding.alloc_workspace(256, 128, 256, 8, 2, -1)
+    a = binding.forward(inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, inp.b1, inp.b2, ws=ws).clone()
+    for _ in range(3):
+        b = binding.forward(inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, inp.b1, inp.b2, ws=ws)
+        assert torch.equal(a, b)
+
+
+def test_bad_ids_flagged_forward_still_right():
+    inp = synthetic.make_inputs("tiny", device="cuda")
+    idx = inp.topk_idx.clone()
+    idx[3, 0] = 99
+    inp.topk_idx.copy_(idx)
+    ws = binding.alloc_workspace(256, 128, 256, 8, 2, -1)
+    out = binding.forward(inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, inp.b1, inp.b2, ws=ws)
+    assert binding.read_error(ws) == binding.DEVERR_BAD_EXPERT_ID
+    wts = oracle.Weights(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    ref = oracle.forward_rows(wts, inp.topk_idx.cpu().numpy(), inp.topk_w.cpu().numpy())
+    assert_close(to_np(out), ref, "out with a bad id")
+
+
+# ---- full-size workloads (the benchmark's launch configuration) ------------
+
+@pytest.mark.parametrize("name,sample", [("prefill", 192), ("ranklocal", 48), ("decode256", None),
+                                         ("prefill256", 192)])
+def test_full_size_workloads_sampled(name, sample):
+    inp = synthetic.make_inputs(name, device="cuda")
+    run_case(inp, sample=sample, seed=17)
+    torch.cuda.empty_cache()
+
+
+def test_prefill_with_total_pairs_and_concat_layout():
+    inp = synthetic.make_inputs("prefill", device="cuda")
+    run_case(inp, layout=1, total_pairs=inp.total_pairs, sample=96, seed=18)
+
+
+def test_full_size_properties_hold_everywhere():
+    """Properties that hold at any size, over all rows: finite output, zero
+    rows exactly for tokens with no valid slot, and a bitwise repeat."""
+    inp = synthetic.make_inputs("ranklocal", device="cuda")
+    inp.topk_idx[::97] = -1
+    ws = binding.alloc_workspace(8192, 7168, 2048, 32, 8, -1)
+    out = binding.forward(inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, ws=ws).clone()
+    assert binding.read_error(ws) == 0
+    assert torch.isfinite(out.float()).all()
+    empty = (inp.topk_idx < 0).all(dim=1)
+    assert torch.count_nonzero(out[empty]) == 0
+    assert torch.count_nonzero(out[~empty].float().abs().sum(1) == 0) == 0
+    out2 = binding.forward(inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, ws=ws)
+    assert torch.equal(out, out2)
