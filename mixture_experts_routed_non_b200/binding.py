@@ -276,6 +276,10 @@ def forward(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
     else:
         if len(events) != 5:
             raise ValueError("events: expected 5 CUDA events")
+        s = stream if stream is not None else torch.cuda.current_stream()
+        for ev in events:
+            if not ev.cuda_event:  # torch creates the CUDA event on its first record
+                ev.record(s)
         arr = (ctypes.c_void_p * 5)(*[ev.cuda_event for ev in events])
         _check(lib.moe_nonexpand_forward_timed(*args, arr), "moe_nonexpand_forward_timed")
     return out

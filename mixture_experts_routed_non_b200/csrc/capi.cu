@@ -235,7 +235,8 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
                  void *ws, size_t ws_bytes, cudaStream_t s, const moe_event_t *ev) {
     int st = check_sizes(N, E, K, total_pairs);
     if (st) return st;
-    if (!x || !topk_idx || !topk_w || !w1 || !w2 || !out) return MOE_ERR_ARG;
+    // with N == 0 the token-sized buffers may be empty (null)
+    if ((N > 0 && (!x || !topk_idx || !topk_w || !out)) || !w1 || !w2) return MOE_ERR_ARG;
     if (activation != MOE_ACT_SWIGLU) return MOE_ERR_ARG;
     if (layout_kind != MOE_LAYOUT_INTERLEAVED && layout_kind != MOE_LAYOUT_CONCATENATED) return MOE_ERR_ARG;
     if (meta_out && !meta_complete(meta_out)) return MOE_ERR_ARG;
@@ -353,7 +354,10 @@ extern "C" MOE_API int moe_nonexpand_metadata(const int32_t *topk_idx, const flo
                                    size_t ws_bytes, moe_stream_t stream) {
     int st = check_sizes(N, E, K, total_pairs);
     if (st) return st;
-    if (!topk_idx || !topk_w || !meta_complete(meta)) return MOE_ERR_ARG;
+    if ((N > 0 && (!topk_idx || !topk_w)) || !meta || !meta->token_offset || !meta->expert_frequency ||
+        !meta->expert_frequency_offset)
+        return MOE_ERR_ARG;
+    if (N > 0 && !meta_complete(meta)) return MOE_ERR_ARG;
     if (!aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_ARG;
     const moe_ws_layout_t l = compute_layout(N, 0, 0, E, K, total_pairs);
     if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MOE_ERR_WS;
