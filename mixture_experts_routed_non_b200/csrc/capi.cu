@@ -169,15 +169,33 @@ bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// w1 in the concatenated layout viewed as [rows][2][I]: (i, half, row).
+// A row-major weight [rows][ncols] (ncols % 64 == 0) viewed as
+// (64 columns, rows, ncols/64 column chunks): one box of 64 x kBK x 4 lands in
+// shared memory as four 64-column chunks of kBK rows each, 8 KB apart -- the
+// N-major operand layout of a 256-column stage.
+bool make_map_b_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {64, rows, ncols / 64};
+    cuuint64_t strides[2] = {ncols * 2, 128};
+    cuuint32_t box[3] = {64, (cuuint32_t)kBK, (cuuint32_t)(kBN / 64)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// w1 in the concatenated layout [rows][2][I] viewed as (64 columns, rows,
+// I/64 chunks, gate/up half): one box of 64 x kBK x 2 x 2 lands as gate chunks
+// 0,1 then up chunks 0,1 (8 KB apart).
 bool make_map_w1_concat(CUtensorMap *m, const void *ptr, uint64_t I, uint64_t rows) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
-    cuuint64_t dims[3] = {I, 2, rows};
-    cuuint64_t strides[2] = {I * 2, I * 4};
-    cuuint32_t box[3] = {64, 1, (cuuint32_t)kBK};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+    cuuint64_t dims[4] = {64, rows, I / 64, 2};
+    cuuint64_t strides[3] = {I * 4, 128, I * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)kBK, 2, 2};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -267,12 +285,12 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
         // ---- up: x gathered rows . w1 -> h
         GemmArgs up;
         memset(&up, 0, sizeof up);
-        if (!make_map_2d(&up.tmap_a, x, (uint64_t)H, (uint64_t)N, 64, 1)) return MOE_ERR_CUDA;
         if (layout_kind == MOE_LAYOUT_CONCATENATED) {
             if (!make_map_w1_concat(&up.tmap_b, w1, (uint64_t)I, (uint64_t)E * H)) return MOE_ERR_CUDA;
         } else {
-            if (!make_map_2d(&up.tmap_b, w1, (uint64_t)2 * I, (uint64_t)E * H, 64, kBK)) return MOE_ERR_CUDA;
+            if (!make_map_b_chunks(&up.tmap_b, w1, (uint64_t)2 * I, (uint64_t)E * H)) return MOE_ERR_CUDA;
         }
+        up.x = static_cast<const __nv_bfloat16 *>(x);
         up.x_gather_idx = meta.x_gather_idx;
         up.expert_off = meta.expert_frequency_offset;
         up.tile_off = ma.gemm_tile_off;
@@ -295,7 +313,7 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
         GemmArgs dn;
         memset(&dn, 0, sizeof dn);
         if (!make_map_2d(&dn.tmap_a, hbuf, (uint64_t)I, (uint64_t)l.p_cap, 64, kBM)) return MOE_ERR_CUDA;
-        if (!make_map_2d(&dn.tmap_b, w2, (uint64_t)H, (uint64_t)E * I, 64, kBK)) return MOE_ERR_CUDA;
+        if (!make_map_b_chunks(&dn.tmap_b, w2, (uint64_t)H, (uint64_t)E * I)) return MOE_ERR_CUDA;
         dn.expert_off = meta.expert_frequency_offset;
         dn.tile_off = ma.gemm_tile_off;
         dn.bias = static_cast<const __nv_bfloat16 *>(b2);

@@ -29,7 +29,7 @@ constexpr int kBM = 128;        // rows (pairs) per tile = UMMA M
 constexpr int kBN = 256;        // accumulator columns per tile = UMMA N
 constexpr int kBK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
-constexpr int kStages = 4;      // shared-memory pipeline depth
+constexpr int kStages = 4;      // shared-memory pipeline depth (4 x 48 KB)
 
 // Metadata kernels.
 constexpr int kMetaThreads = 512;
@@ -63,8 +63,10 @@ struct MetaArgs {
 };
 
 struct GemmArgs {
-    CUtensorMap tmap_a;       // up: x [N,H] (gather4 rows); down: h [P_cap,I]
-    CUtensorMap tmap_b;       // up: w1; down: w2
+    CUtensorMap tmap_a;       // down: h [P_cap,I], box 64 x 128 (up: unused)
+    CUtensorMap tmap_b;       // w1 / w2 viewed as (64 columns, K rows, column chunk[, half]):
+                              // one box = a whole 64 x 256 stage of B
+    const __nv_bfloat16 *x;   // up: x [N,H], rows gathered with cp.async
     const int32_t *x_gather_idx;
     const int32_t *expert_off;    // [E+1]
     const int32_t *tile_off;      // [E+1]
@@ -202,6 +204,29 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, uint
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+        : "memory");
+}
+
+// --- cp.async (16-byte, L2 only) feeding shared memory ----------------------
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the arrival is one of the barrier's expected arrivals).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void *tmap, uint32_t bar, int32_t c0,
+                                            int32_t c1, int32_t c2, int32_t c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
 

@@ -7,8 +7,10 @@
 //
 //   up   (kUp = true):  acc = x[x_gather_idx[p], :] . w1[e] (+ b1[e]),
 //                       h[p, j] = silu(gate_j) * up_j   (bf16 [P_cap, I])
-//        The A rows are gathered from x by TMA tile::gather4 (4 rows per
-//        copy), so no permuted copy of x is ever written.  The SwiGLU ("silu
+//        The A rows are gathered from x by four producer warps with 16-byte
+//        cp.async copies written straight into the 128-byte-swizzled stage
+//        (one TMA instruction per four rows proved too slow: a stage needed 32
+//        of them), so no permuted copy of x is ever written.  The SwiGLU ("silu
 //        times up", qwen3_5.py commit notes, recipe step 4) runs in the
 //        epilogue on the fp32 accumulator.  Interleaved w1 columns
 //        (g0,u0,g1,u1,...) give gate/up in adjacent accumulator columns;
@@ -18,8 +20,10 @@
 //        columns, so gate and up land in columns c and c+128.
 //   down (kUp = false): y[p, :] = h[p, :] . w2[e] (+ b2[e])  (bf16 [P_cap, H])
 //
-// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM allocator and
-// single-thread MMA issuer, warps 2-5 = epilogue (TMEM lane quarter warp%4).
+// Warp roles: warp 0 = TMA producer (B; and A for the down GEMM), warp 1 =
+// TMEM allocator and single-thread MMA issuer, warps 2-5 = epilogue (TMEM lane
+// quarter warp%4), warps 6-9 (up only) = A-row gather.  Each B stage (64 K-rows
+// x 256 columns) is one TMA box of a 3-D / 4-D view of the weights.
 // Pipeline: kStages shared-memory stages (A 128x64 + B 64x256 bf16, 128-byte
 // swizzle), two TMEM accumulators of 128x256 fp32 so the epilogue of one tile
 // overlaps the MMAs of the next.  Rows past the end of an expert's segment are
@@ -34,7 +38,9 @@ namespace moe {
 
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kGatherWarps = 4;
+constexpr int kGatherThreads = 32 * kGatherWarps;
+__host__ __device__ constexpr int threads_of(bool up) { return up ? 192 + kGatherThreads : 192; }
 constexpr uint32_t kStageA = kBM * kBK * 2;   // 16 KB
 constexpr uint32_t kStageB = kBK * kBN * 2;   // 32 KB: 4 chunks of 64 K-rows x 64 N-columns
 constexpr uint32_t kChunkB = kBK * 64 * 2;    // 8 KB
@@ -88,7 +94,8 @@ __device__ __forceinline__ void load_bias32(const __nv_bfloat16 *b, float (&v)[3
 }
 
 template <bool kUp>
-__global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
+__global__ void __launch_bounds__(threads_of(kUp), 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
+    constexpr int kThreads = threads_of(kUp);
     extern __shared__ uint8_t smem_raw[];
     if (*(volatile uint32_t *)&a.hdr->abort) return;
 
@@ -112,7 +119,9 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(full_bar(s), 1);
+            // TMA producer's arrive (+ transaction bytes), plus one cp.async
+            // arrival per gather thread in the up GEMM
+            mbar_init(full_bar(s), 1 + (kUp ? kGatherThreads : 0));
             mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -124,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         fence_barrier_init();
     }
     if (threadIdx.x == 32) {
-        tma_prefetch_desc(&a.tmap_a);
+        if (!kUp) tma_prefetch_desc(&a.tmap_a);
         tma_prefetch_desc(&a.tmap_b);
     }
     for (int i = threadIdx.x; i <= E; i += kThreads) {
@@ -147,68 +156,38 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
+        constexpr uint32_t kTxBytes = kUp ? kStageB : kStageBytes;
         int stage = 0;
         uint32_t phase = 0;
         uint32_t issued = 0, issued_parity = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x) {
-            const Tile t = decode_tile(tile, n_tiles, E, tile_off_s, off_s);
-            int rows[4] = {0, 0, 0, 0};
-            if (kUp) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int p = min(t.m0 + 4 * lane + j, t.m_end - 1);
-                    rows[j] = __ldg(a.x_gather_idx + p);
-                }
-            }
-            const int brow0 = t.e * a.k_dim;
-            for (int kb = 0; kb < nk; ++kb) {
-                bool w = true;
-                if (lane == 0) w = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort);
-                w = __shfl_sync(0xffffffffu, w, 0);
-                if (!w) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) mbar_arrive_expect_tx(full_bar(stage), kStageBytes);
-                __syncwarp();
-                const int k0 = kb * kBK;
-                const uint32_t a_dst = sA + stage * kStageA;
-                const uint32_t b_dst = sB + stage * kStageB;
-                if (kUp) {
-                    tma_gather4(a_dst + lane * 4 * 128, &a.tmap_a, full_bar(stage), k0, rows[0], rows[1],
-                                rows[2], rows[3]);
-                } else if (lane == 0) {
-                    tma_load_2d(a_dst, &a.tmap_a, full_bar(stage), k0, t.m0);
-                }
-                if (lane == 0) {
-                    if (kUp && a.layout == MOE_LAYOUT_CONCATENATED) {
-                        const int c0 = t.nt * (kBN / 2);
-#pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-                            tma_load_3d(b_dst + c * kChunkB, &a.tmap_b, full_bar(stage), c0 + 64 * c, 0,
-                                        brow0 + k0);
-                            tma_load_3d(b_dst + (2 + c) * kChunkB, &a.tmap_b, full_bar(stage), c0 + 64 * c,
-                                        1, brow0 + k0);
-                        }
-                    } else {
-                        const int c0 = t.nt * kBN;
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            tma_load_2d(b_dst + c * kChunkB, &a.tmap_b, full_bar(stage), c0 + 64 * c,
-                                        brow0 + k0);
+        if (lane == 0) {
+            for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+                const Tile t = decode_tile(tile, n_tiles, E, tile_off_s, off_s);
+                const int brow0 = t.e * a.k_dim;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(full_bar(stage), kTxBytes);
+                    const int k0 = kb * kBK;
+                    const uint32_t b_dst = sB + stage * kStageB;
+                    if (!kUp) tma_load_2d(sA + stage * kStageA, &a.tmap_a, full_bar(stage), k0, t.m0);
+                    if (kUp && a.layout == MOE_LAYOUT_CONCATENATED)
+                        tma_load_4d(b_dst, &a.tmap_b, full_bar(stage), 0, brow0 + k0, t.nt * 2, 0);
+                    else
+                        tma_load_3d(b_dst, &a.tmap_b, full_bar(stage), 0, brow0 + k0, t.nt * 4);
+                    issued |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kStages) {
+                        stage = 0;
+                        phase ^= 1u;
                     }
                 }
-                issued |= 1u << stage;
-                issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-                if (++stage == kStages) {
-                    stage = 0;
-                    phase ^= 1u;
-                }
+                if (!ok) break;
             }
-        }
-        // every copy this CTA issued must land before the CTA may exit
-        if (lane == 0) {
+            // every copy this CTA issued must land before the CTA may exit
             for (int s = 0; s < kStages; ++s)
                 if (issued & (1u << s)) mbar_wait_timed(full_bar(s), (issued_parity >> s) & 1u);
         }
@@ -231,6 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
                         ok = false;
                         break;
                     }
+                    if (kUp) fence_proxy_async_smem();
                     tc_fence_after();
                     const uint32_t a_addr = sA + stage * kStageA;
                     const uint32_t b_addr = sB + stage * kStageB;
@@ -257,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
             mbar_wait_timed(drain_bar, 0);
         }
         __syncwarp();
-    } else {
+    } else if (warp < 6) {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
@@ -378,6 +358,72 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const __grid_
         }
     }
 
+    if (kUp && warp >= 6) {
+        // ------------------------------------------------------- A-row gather
+        // thread g: 16-byte chunk (g & 7) of rows (g >> 3) + 16 i, i = 0..7,
+        // stored at row * 128 + ((chunk ^ (row & 7)) << 4): the 128-byte
+        // swizzle the MMA descriptors expect.
+        const int g = threadIdx.x - 192;
+        const int chunk = g & 7;
+        const int r0 = g >> 3;
+        const int gl = g & 31;
+        int stage = 0;
+        uint32_t phase = 0;
+        const char *xb = reinterpret_cast<const char *>(a.x);
+        const size_t ld = (size_t)a.k_dim * 2;
+        int tile = blockIdx.x;
+        Tile t{};
+        const char *src[8];
+        auto load_rows = [&](const Tile &tt, const char *(&p)[8]) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int pr = min(tt.m0 + r0 + 16 * i, tt.m_end - 1);
+                p[i] = xb + (size_t)__ldg(a.x_gather_idx + pr) * ld + chunk * 16;
+            }
+        };
+        if (tile < total_tiles) {
+            t = decode_tile(tile, n_tiles, E, tile_off_s, off_s);
+            load_rows(t, src);
+        }
+        bool ok = true;
+        for (; ok && tile < total_tiles; tile += gridDim.x) {
+            const int next = tile + gridDim.x;
+            Tile tn = t;
+            const char *nsrc[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) nsrc[i] = src[i];
+            if (next < total_tiles) {
+                tn = decode_tile(next, n_tiles, E, tile_off_s, off_s);
+                if (tn.m0 != t.m0) load_rows(tn, nsrc);
+            }
+            for (int kb = 0; kb < nk; ++kb) {
+                bool w = true;
+                if (gl == 0) w = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort);
+                w = __shfl_sync(0xffffffffu, w, 0);
+                if (!w) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t a_dst = sA + stage * kStageA;
+                const size_t koff = (size_t)kb * kBK * 2;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int row = r0 + 16 * i;
+                    cp_async_16(a_dst + row * 128 + ((chunk ^ (row & 7)) << 4), src[i] + koff);
+                }
+                cp_async_arrive_noinc(full_bar(stage));
+                if (++stage == kStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            t = tn;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) src[i] = nsrc[i];
+        }
+        cp_async_wait_all();
+    }
+
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -399,7 +445,7 @@ cudaError_t launch(const GemmArgs &a, int grid, cudaStream_t s) {
         if (err != cudaSuccess) return err;
         configured[dev] = true;
     }
-    grouped_gemm_kernel<kUp><<<grid, kThreads, kSmemBytes, s>>>(a);
+    grouped_gemm_kernel<kUp><<<grid, threads_of(kUp), kSmemBytes, s>>>(a);
     return cudaGetLastError();
 }
 
