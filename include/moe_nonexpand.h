@@ -108,9 +108,9 @@ typedef struct CUevent_st *moe_event_t;
  * H = I = 0 for what moe_nonexpand_metadata alone needs).  The workspace
  * holds the per-tile histograms, the GEMM tile table, the metadata when the
  * caller does not provide it, and the bf16 intermediates h [P_cap,I] and
- * y [P_cap,H].  It must be zero-filled ONCE after allocation; the library
- * leaves it in a reusable state after every call.  One workspace must not be
- * used by two calls that can run at the same time.
+ * y [P_cap,H].  Its contents need no initialisation: every call writes what
+ * it reads.  One workspace must not be used by two calls that can run at the
+ * same time.
  * Returns 0 for arguments outside the supported sizes.
  */
 MOE_API size_t moe_nonexpand_workspace_bytes(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
@@ -180,9 +180,9 @@ MOE_API int moe_nonexpand_combine(const void *y, const moe_meta_t *meta, int64_t
 typedef struct moe_ws_layout_t {
     size_t total;              /* == moe_nonexpand_workspace_bytes(...)       */
     size_t header;             /* 256-byte header; error word at byte 4       */
-    size_t tile_hist;          /* int32 [T,E] per-tile histograms, then bases */
-    size_t tile_valid;         /* int32 [T]                                   */
-    size_t tile_pair_base;     /* int32 [T]                                   */
+    size_t tile_hist;          /* int32 [T,E] per-tile expert histograms      */
+    size_t tile_valid;         /* int32 [T]   valid slots per tile            */
+    size_t tile_err;           /* int32 [T]   error bits per tile             */
     size_t gemm_tile_offset;   /* int32 [E+1] prefix of ceil(freq/128)        */
     size_t meta_freq, meta_off, meta_x_gather, meta_s_scatter, meta_s_rev,
            meta_token_offset, meta_scores;  /* metadata kept in the workspace */

@@ -53,7 +53,7 @@ class MoeMeta(ctypes.Structure):
 
 class WsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
-        "total", "header", "tile_hist", "tile_valid", "tile_pair_base", "gemm_tile_offset",
+        "total", "header", "tile_hist", "tile_valid", "tile_err", "gemm_tile_offset",
         "meta_freq", "meta_off", "meta_x_gather", "meta_s_scatter", "meta_s_rev",
         "meta_token_offset", "meta_scores", "h", "y")] + [
         ("p_cap", ctypes.c_int64), ("meta_tiles", ctypes.c_int32), ("meta_tile_slots", ctypes.c_int32)]
@@ -152,10 +152,9 @@ def workspace_layout(N: int, H: int, I: int, E: int, K: int, total_pairs: int = 
 
 def alloc_workspace(N: int, H: int, I: int, E: int, K: int, total_pairs: int = -1,
                     device=None) -> torch.Tensor:
-    """A zero-filled workspace of the required size (zero-filled once, as
-    the library requires)."""
+    """A workspace of the required size (its contents need no initialisation)."""
     n = workspace_bytes(N, H, I, E, K, total_pairs)
-    return torch.zeros(n, dtype=torch.uint8, device=device or torch.device("cuda"))
+    return torch.empty(n, dtype=torch.uint8, device=device or torch.device("cuda"))
 
 
 def alloc_meta(N: int, K: int, E: int, total_pairs: int = -1, device=None) -> dict:

@@ -1,6 +1,6 @@
 // Host side of the C ABI declared in include/moe_nonexpand.h: argument
 // checks, workspace layout, tensor-map encoding and the launch sequence
-//   metadata (count + last-block scan, scatter) -> grouped GEMM up (+b1,
+//   metadata (count, scan + scatter) -> grouped GEMM up (+b1,
 //   SwiGLU) -> grouped GEMM down (+b2) -> combine
 // all on the caller's stream, with no host synchronisation (the proposed
 // entry point of sonic-moe issue #68 takes a stream and is meant to be
@@ -23,15 +23,14 @@ struct Layout {
     moe_ws_layout_t l;
 };
 
-// Slots per metadata tile: a multiple of the block size, sized so that the
-// grid holds about two CTAs per SM of a B200, capped to keep the per-tile
-// histogram table small.
+// Slots per metadata tile: a multiple of kMetaTileUnit, sized so that there
+// are at most kMetaMaxTiles tiles (one CTA per SM of a B200); the scatter
+// kernel reads the whole [T,E] histogram table, which stays small.
 void meta_tiling(int64_t NK, int32_t *tile_slots, int32_t *tiles) {
-    const int64_t target_ctas = 2 * 148;
-    int64_t c = (NK + (int64_t)kMetaThreads * target_ctas - 1) / ((int64_t)kMetaThreads * target_ctas);
+    const int64_t per = (int64_t)kMetaTileUnit * kMetaMaxTiles;
+    int64_t c = (NK + per - 1) / per;
     if (c < 1) c = 1;
-    if (c > 256) c = 256;
-    const int64_t S = kMetaThreads * c;
+    const int64_t S = (int64_t)kMetaTileUnit * c;
     int64_t T = (NK + S - 1) / S;
     if (T < 1) T = 1;
     *tile_slots = (int32_t)S;
@@ -68,10 +67,8 @@ moe_ws_layout_t compute_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32
     o = align_up(o + T * E * 4, kAlign);
     l.tile_valid = o;
     o = align_up(o + T * 4, kAlign);
-    l.tile_pair_base = o;
+    l.tile_err = o;
     o = align_up(o + T * 4, kAlign);
-    const size_t tile_err = o;  // follows tile_pair_base
-    o = align_up(tile_err + T * 4, kAlign);
     l.gemm_tile_offset = o;
     o = align_up(o + (size_t)(E + 1) * 4, kAlign);
     l.meta_freq = o;
@@ -98,8 +95,6 @@ moe_ws_layout_t compute_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32
     l.total = o;
     return l;
 }
-
-size_t tile_err_offset(const moe_ws_layout_t &l) { return align_up(l.tile_pair_base + (size_t)l.meta_tiles * 4, kAlign); }
 
 // ---------------------------------------------------------------------------
 // Per-device facts.
@@ -217,8 +212,7 @@ MetaArgs meta_args(const int32_t *topk_idx, const float *topk_w, int64_t N, int3
     a.hdr = reinterpret_cast<WsHeader *>(ws + l.header);
     a.tile_hist = reinterpret_cast<int32_t *>(ws + l.tile_hist);
     a.tile_valid = reinterpret_cast<int32_t *>(ws + l.tile_valid);
-    a.tile_pbase = reinterpret_cast<int32_t *>(ws + l.tile_pair_base);
-    a.tile_err = reinterpret_cast<int32_t *>(ws + tile_err_offset(l));
+    a.tile_err = reinterpret_cast<int32_t *>(ws + l.tile_err);
     a.gemm_tile_off = reinterpret_cast<int32_t *>(ws + l.gemm_tile_offset);
     a.meta = meta;
     a.N = N;

@@ -5,20 +5,24 @@
 // s_reverse_scatter_idx, num_activated_expert_per_token_offset, compact
 // router_scores -- and question 3: pairs are numbered in ascending token
 // order).  The sort by expert is a stable counting sort (the segmented-sort
-// recipe of the qwen3_5.py commit notes, steps 1-2), done in two kernels:
+// recipe of the qwen3_5.py commit notes, steps 1-2), in two kernels over T
+// tiles of consecutive slots (T <= number of SMs):
 //
-//   meta_count_kernel   one CTA per tile of slots: expert histogram in shared
-//                       memory (match_any aggregation), per-tile valid count.
-//                       The last CTA to finish (atomic ticket, no waiting)
-//                       scans: totals, offsets, per-(tile,expert) bases,
-//                       per-tile pair bases and the GEMM tile table.
-//   meta_scatter_kernel one CTA per tile again: each warp owns a contiguous
-//                       slice of the tile; per-warp counts give each warp its
-//                       base per expert, and inside a 32-slot step the rank of
-//                       a slot among equal experts is popc(peers & lanes
-//                       below).  Every result is a pure function of the input
-//                       (no atomics decide an order), so the output is
-//                       bit-exact and deterministic.
+//   meta_count_kernel    per tile: expert histogram in shared memory (match_any
+//                        aggregation) and valid-slot count -> hist[T][E].
+//   meta_scatter_kernel  per tile: reads the whole (small) hist table and
+//                        derives, with no inter-block waiting, the global
+//                        offsets, this tile's base per expert and its pair base;
+//                        then each warp ranks its own contiguous slice (per-warp
+//                        counts, then popc(peers & lanes below) inside each
+//                        32-slot step) and writes the outputs.  Block 0 also
+//                        writes the histogram, offsets, the GEMM tile table and
+//                        the call's error word.
+//
+// Every result is a pure function of the input (no atomic decides an order),
+// so the output is bit-exact and deterministic.  Each lane keeps kV slots in
+// flight (all loads issued before use) so that a warp pays one memory latency
+// per 32*kV slots.
 #include "common.cuh"
 
 namespace moe {
@@ -26,23 +30,19 @@ namespace moe {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
+constexpr int kV = 8;                     // slots per lane per step
+constexpr int kWarpChunk = 32 * kV;       // slots per warp step
 
-// Exclusive scan of n ints from `in` into `out` (either may be shared or
-// global; in == out allowed) by the whole block; returns the total.
-__device__ int block_exclusive_scan(const int *in, int *out, int n, bool in_global) {
+// Exclusive scan of n ints in shared memory (in place allowed) by the whole
+// block; returns the total.
+__device__ int block_exclusive_scan(const int *in, int *out, int n) {
     __shared__ int warp_tot[kMetaWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int carry = 0;
     for (int base = 0; base < n; base += 2 * kMetaThreads) {
         const int i0 = base + 2 * threadIdx.x, i1 = i0 + 1;
-        int v0 = 0, v1 = 0;
-        if (in_global) {
-            if (i0 < n) v0 = __ldcg(in + i0);
-            if (i1 < n) v1 = __ldcg(in + i1);
-        } else {
-            if (i0 < n) v0 = in[i0];
-            if (i1 < n) v1 = in[i1];
-        }
+        const int v0 = i0 < n ? in[i0] : 0;
+        const int v1 = i1 < n ? in[i1] : 0;
         const int s = v0 + v1;
         int x = s;
 #pragma unroll
@@ -71,110 +71,35 @@ __device__ int block_exclusive_scan(const int *in, int *out, int n, bool in_glob
     return carry;
 }
 
-// Shared memory of the count kernel / last-block scan (ints).
-constexpr int kScanPart = kMaxExperts;          // part[G*E] (G*E <= max(E, kMetaThreads))
-constexpr int kCountSmemInts = kScanPart + 3 * (kMaxExperts + 1) + 8;
+// Sum over the block of one int per thread.
+__device__ int block_sum(int v) {
+    __shared__ int part[kMetaWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    if (lane == 0) part[warp] = v;
+    __syncthreads();
+    int t = 0;
+#pragma unroll
+    for (int w = 0; w < kMetaWarps; ++w) t += part[w];
+    __syncthreads();
+    return t;
+}
 
-__device__ void last_block_scan(const MetaArgs &a, int *sm) {
-    const int E = a.E, T = a.tiles;
-    int *part = sm;                             // [G][E]
-    int *freq = sm + kScanPart;                 // [E]
-    int *off = freq + (kMaxExperts + 1);        // [E+1]
-    int *gtile = off + (kMaxExperts + 1);       // [E+1]
-    __shared__ unsigned s_err;
-
-    int G = E <= kMetaThreads ? kMetaThreads / E : 1;
-    if (G > T) G = T;
-    const int chunk = (T + G - 1) / G;
-
-    // 1. per-group partial column sums of the tile histograms
-    for (int i = threadIdx.x; i < G * E; i += kMetaThreads) {
-        const int g = i / E, e = i - g * E;
-        const int t0 = g * chunk, t1 = min(T, t0 + chunk);
-        int sum = 0;
-        int t = t0;
-        for (; t + 4 <= t1; t += 4) {
-            const int v0 = __ldcg(a.tile_hist + (size_t)(t + 0) * E + e);
-            const int v1 = __ldcg(a.tile_hist + (size_t)(t + 1) * E + e);
-            const int v2 = __ldcg(a.tile_hist + (size_t)(t + 2) * E + e);
-            const int v3 = __ldcg(a.tile_hist + (size_t)(t + 3) * E + e);
-            sum += v0 + v1 + v2 + v3;
-        }
-        for (; t < t1; ++t) sum += __ldcg(a.tile_hist + (size_t)t * E + e);
-        part[i] = sum;
-    }
-    if (threadIdx.x == 0) s_err = 0;
-    __syncthreads();
-    // 2. per expert: exclusive prefix over groups, total = frequency
-    for (int e = threadIdx.x; e < E; e += kMetaThreads) {
-        int run = 0;
-        for (int g = 0; g < G; ++g) {
-            const int v = part[g * E + e];
-            part[g * E + e] = run;
-            run += v;
-        }
-        freq[e] = run;
-        gtile[e] = (run + kBM - 1) / kBM;
-    }
-    __syncthreads();
-    // 3. offsets and GEMM tile table
-    const int P = block_exclusive_scan(freq, off, E, false);
-    const int GT = block_exclusive_scan(gtile, gtile, E, false);
-    for (int e = threadIdx.x; e < E; e += kMetaThreads) {
-        a.meta.expert_frequency[e] = freq[e];
-        a.meta.expert_frequency_offset[e] = off[e];
-        a.gemm_tile_off[e] = gtile[e];
-    }
-    if (threadIdx.x == 0) {
-        off[E] = P;
-        a.meta.expert_frequency_offset[E] = P;
-        a.gemm_tile_off[E] = GT;
-    }
-    __syncthreads();
-    // 4. per-(tile, expert) global bases, written over the histograms
-    for (int i = threadIdx.x; i < G * E; i += kMetaThreads) {
-        const int g = i / E, e = i - g * E;
-        const int t0 = g * chunk, t1 = min(T, t0 + chunk);
-        int base = off[e] + part[i];
-        for (int t = t0; t < t1; ++t) {
-            int *cell = a.tile_hist + (size_t)t * E + e;
-            const int v = __ldcg(cell);
-            *cell = base;
-            base += v;
-        }
-    }
-    // 5. per-tile pair bases
-    block_exclusive_scan(a.tile_valid, a.tile_pbase, T, true);
-    // 6. errors of this call, pair-count check, abort decision
-    unsigned err = 0;
-    for (int t = threadIdx.x; t < T; t += kMetaThreads) err |= (unsigned)__ldcg(a.tile_err + t);
-    if (err) atomicOr(&s_err, err);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        unsigned e = s_err;
-        unsigned abort = 0;
-        if (a.total_pairs >= 0 && (int64_t)P != a.total_pairs) e |= MOE_DEVERR_PAIR_COUNT;
-        if ((int64_t)P > a.p_cap) {
-            e |= MOE_DEVERR_PAIR_COUNT | MOE_DEVERR_ABORTED;
-            abort = 1;
-        }
-        a.meta.token_offset[a.N] = P;
-        a.hdr->P = P;
-        a.hdr->err = e;
-        a.hdr->abort = abort;
-        __threadfence();
-        a.hdr->ticket = 0;  // ready for the next call
+__device__ __forceinline__ void load_chunk(const int32_t *idx, int base, int end, int lane, int (&e)[kV]) {
+#pragma unroll
+    for (int v = 0; v < kV; ++v) {
+        const int s = base + 32 * v + lane;
+        e[v] = s < end ? __ldg(idx + s) : -1;
     }
 }
 
 __global__ void __launch_bounds__(kMetaThreads) meta_count_kernel(const MetaArgs a) {
-    extern __shared__ int sm[];
+    extern __shared__ int hist[];  // [E]
     __shared__ int s_valid;
     __shared__ unsigned s_err;
-    __shared__ int s_last;
-    int *hist = sm;
     const int E = a.E;
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int e = threadIdx.x; e < E; e += kMetaThreads) hist[e] = 0;
     if (threadIdx.x == 0) {
         s_valid = 0;
@@ -187,15 +112,18 @@ __global__ void __launch_bounds__(kMetaThreads) meta_count_kernel(const MetaArgs
     const int s1 = (int)min((int64_t)s0 + a.tile_slots, a.NK);
     int my_valid = 0;
     unsigned my_err = 0;
-    for (int base = s0; base < s1; base += kMetaThreads) {  // same trip count in every thread
-        const int s = base + threadIdx.x;
-        const int e = s < s1 ? __ldg(a.topk_idx + s) : -1;
-        const bool valid = (e >= 0) && (e < E);
-        if (!valid && e != -1) my_err = MOE_DEVERR_BAD_EXPERT_ID;
-        const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
-        if (valid && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
-        const unsigned vb = __ballot_sync(kFull, valid);
-        my_valid += __popc(vb);
+    for (int base = s0 + warp * kWarpChunk; base < s1; base += kMetaWarps * kWarpChunk) {
+        int ev[kV];
+        load_chunk(a.topk_idx, base, s1, lane, ev);
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+            const int e = ev[v];
+            const bool valid = (e >= 0) && (e < E);
+            if (!valid && e != -1) my_err = MOE_DEVERR_BAD_EXPERT_ID;
+            const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
+            if (valid && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
+            my_valid += __popc(__ballot_sync(kFull, valid));
+        }
     }
     if (lane == 0 && my_valid) atomicAdd(&s_valid, my_valid);
     if (my_err) atomicOr(&s_err, my_err);
@@ -206,54 +134,122 @@ __global__ void __launch_bounds__(kMetaThreads) meta_count_kernel(const MetaArgs
         a.tile_valid[tile] = s_valid;
         a.tile_err[tile] = (int)s_err;
     }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const unsigned t = atomicAdd(&a.hdr->ticket, 1u);
-        s_last = (t == (unsigned)(a.tiles - 1));
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    last_block_scan(a, sm);
 }
 
+// Shared memory of the scatter kernel (ints), after cnt[kMetaWarps][E].
+constexpr int kPartInts = kMaxExperts;   // G*E <= max(kMetaThreads, E) <= kMaxExperts
+
 __global__ void __launch_bounds__(kMetaThreads) meta_scatter_kernel(const MetaArgs a) {
-    extern __shared__ int cnt[];  // [kMetaWarps][E]: per-warp running base of each expert
+    extern __shared__ int sm[];
+    const int E = a.E, K = a.K, T = a.tiles;
+    int *cnt = sm;                              // [kMetaWarps][E]
+    int *part_all = cnt + kMetaWarps * E;       // [G][E]
+    int *part_before = part_all + kPartInts;    // [G][E]
+    int *off = part_before + kPartInts;         // [E+1]
+    int *gt = off + (kMaxExperts + 1);          // [E+1]
     __shared__ int wq[kMetaWarps];
-    if (*(volatile uint32_t *)&a.hdr->abort) return;
-    const int E = a.E, K = a.K;
+    __shared__ unsigned s_err;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t lt = lanemask_lt();
     const int tile = blockIdx.x;
-    for (int i = threadIdx.x; i < kMetaWarps * E; i += kMetaThreads) cnt[i] = 0;
-    __syncthreads();
 
+    // ---- 1. global column sums and this tile's column prefix, from hist[T][E]
+    int G = E <= kMetaThreads ? kMetaThreads / E : 1;
+    if (G > T) G = T;
+    for (int i = threadIdx.x; i < G * E; i += kMetaThreads) {
+        const int g = i / E, e = i - g * E;
+        int all = 0, before = 0;
+        for (int t0 = g; t0 < T; t0 += 8 * G) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int t = t0 + u * G;
+                v[u] = t < T ? __ldcg(a.tile_hist + (size_t)t * E + e) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                all += v[u];
+                if (t0 + u * G < tile) before += v[u];
+            }
+        }
+        part_all[i] = all;
+        part_before[i] = before;
+    }
+    for (int i = threadIdx.x; i < kMetaWarps * E; i += kMetaThreads) cnt[i] = 0;
+    int tv = 0, tv_before = 0;
+    unsigned terr = 0;
+    for (int t = threadIdx.x; t < T; t += kMetaThreads) {
+        const int v = __ldcg(a.tile_valid + t);
+        tv += v;
+        if (t < tile) tv_before += v;
+        terr |= (unsigned)__ldcg(a.tile_err + t);
+    }
+    if (threadIdx.x == 0) s_err = 0;
+    __syncthreads();
+    if (terr) atomicOr(&s_err, terr);
+    for (int e = threadIdx.x; e < E; e += kMetaThreads) {
+        int all = 0, before = 0;
+        for (int g = 0; g < G; ++g) {
+            all += part_all[g * E + e];
+            before += part_before[g * E + e];
+        }
+        off[e] = all;             // scanned below
+        part_before[e] = before;  // this tile's prefix per expert (rows g > 0 no longer needed)
+        gt[e] = (all + kBM - 1) / kBM;
+    }
+    __syncthreads();
+    const int P = block_exclusive_scan(off, off, E);
+    const int pbase = block_sum(tv_before);
+    const bool abort = (int64_t)P > a.p_cap;
+
+    if (tile == 0) {
+        const int GT = block_exclusive_scan(gt, gt, E);
+        for (int e = threadIdx.x; e < E; e += kMetaThreads) {
+            a.meta.expert_frequency[e] = (e + 1 < E ? off[e + 1] : P) - off[e];
+            a.meta.expert_frequency_offset[e] = off[e];
+            a.gemm_tile_off[e] = gt[e];
+        }
+        if (threadIdx.x == 0) {
+            unsigned err = s_err;
+            if (a.total_pairs >= 0 && (int64_t)P != a.total_pairs) err |= MOE_DEVERR_PAIR_COUNT;
+            if (abort) err |= MOE_DEVERR_PAIR_COUNT | MOE_DEVERR_ABORTED;
+            a.meta.expert_frequency_offset[E] = P;
+            a.gemm_tile_off[E] = GT;
+            a.meta.token_offset[a.N] = P;
+            a.hdr->P = P;
+            a.hdr->err = err;
+            a.hdr->abort = abort ? 1u : 0u;
+        }
+    }
+    if (abort) return;  // the pair arrays are too small for the pairs seen
+
+    // ---- 2. per-warp counts of this tile's slots
     const int s0 = tile * a.tile_slots;
     const int s1 = (int)min((int64_t)s0 + a.tile_slots, a.NK);
     const int sub = a.tile_slots / kMetaWarps;
     const int w0 = s0 + warp * sub;
     const int w1 = min(w0 + sub, s1);
     int *mycnt = cnt + warp * E;
-
-    // pass 1: per-warp counts of each expert and of valid slots
     int nvalid = 0;
-    for (int base = w0; base < w1; base += 32) {
-        const int s = base + lane;
-        const int e = s < w1 ? __ldg(a.topk_idx + s) : -1;
-        const bool valid = (e >= 0) && (e < E);
-        const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
-        if (valid && lane == __ffs(peers) - 1) mycnt[e] += __popc(peers);
-        nvalid += __popc(__ballot_sync(kFull, valid));
-        __syncwarp();
+    for (int base = w0; base < w1; base += kWarpChunk) {
+        int ev[kV];
+        load_chunk(a.topk_idx, base, w1, lane, ev);
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+            const int e = ev[v];
+            const bool valid = (e >= 0) && (e < E);
+            const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
+            if (valid && lane == __ffs(peers) - 1) mycnt[e] += __popc(peers);
+            nvalid += __popc(__ballot_sync(kFull, valid));
+            __syncwarp();
+        }
     }
     if (lane == 0) wq[warp] = nvalid;
     __syncthreads();
 
-    // bases: the tile's global base per expert (from the scan) plus the
-    // counts of the warps before this one
+    // ---- 3. bases: global offset + earlier tiles + earlier warps of this tile
     for (int e = threadIdx.x; e < E; e += kMetaThreads) {
-        int run = __ldcg(a.tile_hist + (size_t)tile * E + e);
+        int run = off[e] + part_before[e];
         for (int w = 0; w < kMetaWarps; ++w) {
             const int c = cnt[w * E + e];
             cnt[w * E + e] = run;
@@ -261,7 +257,7 @@ __global__ void __launch_bounds__(kMetaThreads) meta_scatter_kernel(const MetaAr
         }
     }
     if (threadIdx.x == 0) {
-        int run = __ldcg(a.tile_pbase + tile);
+        int run = pbase;
         for (int w = 0; w < kMetaWarps; ++w) {
             const int c = wq[w];
             wq[w] = run;
@@ -270,47 +266,64 @@ __global__ void __launch_bounds__(kMetaThreads) meta_scatter_kernel(const MetaAr
     }
     __syncthreads();
 
-    // pass 2: positions, in slot order
+    // ---- 4. positions, in slot order
     int q_run = wq[warp];
-    for (int base = w0; base < w1; base += 32) {
-        const int s = base + lane;
-        const bool in = s < w1;
-        const int e = in ? __ldg(a.topk_idx + s) : -1;
-        const bool valid = (e >= 0) && (e < E);
-        const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
-        const int pbase = valid ? mycnt[e] : 0;
-        __syncwarp();
-        if (valid && lane == __ffs(peers) - 1) mycnt[e] = pbase + __popc(peers);
-        const unsigned vb = __ballot_sync(kFull, valid);
-        const int q = q_run + __popc(vb & lt);
-        if (valid) {
-            const int p = pbase + __popc(peers & lt);
-            const int t = s / K;
-            a.meta.x_gather_idx[p] = t;
-            a.meta.s_scatter_idx[p] = q;
-            a.meta.s_reverse_scatter_idx[q] = p;
-            a.meta.scores[q] = __ldg(a.topk_w + s);
+    for (int base = w0; base < w1; base += kWarpChunk) {
+        int ev[kV];
+        float wv[kV];
+        load_chunk(a.topk_idx, base, w1, lane, ev);
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+            const int s = base + 32 * v + lane;
+            const bool valid = (ev[v] >= 0) && (ev[v] < E);
+            wv[v] = valid ? __ldg(a.topk_w + s) : 0.f;  // invalid slots' weights are never read
         }
-        if (in && (s % K) == 0) a.meta.token_offset[s / K] = q;
-        q_run += __popc(vb);
-        __syncwarp();
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+            const int s = base + 32 * v + lane;
+            const int e = ev[v];
+            const bool valid = (e >= 0) && (e < E);
+            const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
+            const int pb = valid ? mycnt[e] : 0;
+            __syncwarp();
+            if (valid && lane == __ffs(peers) - 1) mycnt[e] = pb + __popc(peers);
+            const unsigned vb = __ballot_sync(kFull, valid);
+            const int q = q_run + __popc(vb & lt);
+            if (valid) {
+                const int p = pb + __popc(peers & lt);
+                a.meta.x_gather_idx[p] = s / K;
+                a.meta.s_scatter_idx[p] = q;
+                a.meta.s_reverse_scatter_idx[q] = p;
+                a.meta.scores[q] = wv[v];
+            }
+            if (s < w1 && (s % K) == 0) a.meta.token_offset[s / K] = q;
+            q_run += __popc(vb);
+            __syncwarp();
+        }
     }
 }
 
 }  // namespace
 
+size_t meta_scatter_smem_bytes(int E) {
+    return ((size_t)kMetaWarps * E + 2 * kPartInts + 2 * (kMaxExperts + 1)) * sizeof(int);
+}
+
 cudaError_t launch_meta(const MetaArgs &a, cudaStream_t s) {
-    static_assert(kCountSmemInts * 4 <= 48 * 1024, "count kernel shared memory");
-    meta_count_kernel<<<a.tiles, kMetaThreads, kCountSmemInts * sizeof(int), s>>>(a);
-    cudaError_t err = cudaGetLastError();
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    const size_t scatter_smem = (size_t)kMetaWarps * a.E * sizeof(int);
-    if (scatter_smem > 48 * 1024) {
+    if (dev < 64 && !configured[dev]) {
         err = cudaFuncSetAttribute(meta_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)(kMetaWarps * kMaxExperts * sizeof(int)));
+                                   (int)meta_scatter_smem_bytes(kMaxExperts));
         if (err != cudaSuccess) return err;
+        configured[dev] = true;
     }
-    meta_scatter_kernel<<<a.tiles, kMetaThreads, scatter_smem, s>>>(a);
+    meta_count_kernel<<<a.tiles, kMetaThreads, a.E * sizeof(int), s>>>(a);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    meta_scatter_kernel<<<a.tiles, kMetaThreads, meta_scatter_smem_bytes(a.E), s>>>(a);
     return cudaGetLastError();
 }
 

@@ -65,14 +65,14 @@ def test_workspace_layout_is_consistent(lib):
                  (65536, 0, 0, 128, 8, -1)]:
         lay = binding.workspace_layout(*args)
         assert lay.total == lib.moe_nonexpand_workspace_bytes(*args)
-        offs = [lay.header, lay.tile_hist, lay.tile_valid, lay.tile_pair_base, lay.gemm_tile_offset,
+        offs = [lay.header, lay.tile_hist, lay.tile_valid, lay.tile_err, lay.gemm_tile_offset,
                 lay.meta_freq, lay.meta_off, lay.meta_x_gather, lay.meta_s_scatter, lay.meta_s_rev,
                 lay.meta_token_offset, lay.meta_scores]
         assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
         if args[1]:
             assert lay.h % 1024 == 0 and lay.y % 1024 == 0
             assert lay.y > lay.h if lay.p_cap > 0 else lay.y == lay.h
-        assert lay.meta_tile_slots % 512 == 0
+        assert lay.meta_tile_slots % 4096 == 0 and lay.meta_tiles <= 148
         assert lay.meta_tiles * lay.meta_tile_slots >= args[0] * args[4]
 
 
