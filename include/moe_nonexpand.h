@@ -183,7 +183,7 @@ typedef struct moe_ws_layout_t {
     size_t tile_hist;          /* int32 [T,E] per-tile expert histograms      */
     size_t tile_valid;         /* int32 [T]   valid slots per tile            */
     size_t tile_err;           /* int32 [T]   error bits per tile             */
-    size_t gemm_tile_offset;   /* int32 [E+1] prefix of ceil(freq/128)        */
+    size_t gemm_tile_offset;   /* int32 [E+1] prefix of ceil(freq/256)        */
     size_t meta_freq, meta_off, meta_x_gather, meta_s_scatter, meta_s_rev,
            meta_token_offset, meta_scores;  /* metadata kept in the workspace */
     size_t h;                  /* bf16 [P_cap,I] */

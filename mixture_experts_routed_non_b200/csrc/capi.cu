@@ -165,15 +165,15 @@ bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer
 }
 
 // A row-major weight [rows][ncols] (ncols % 64 == 0) viewed as
-// (64 columns, rows, ncols/64 column chunks): one box of 64 x kBK x 4 lands in
-// shared memory as four 64-column chunks of kBK rows each, 8 KB apart -- the
-// N-major operand layout of a 256-column stage.
+// (64 columns, rows, ncols/64 column chunks): one box of 64 x kBK x 2 lands in
+// shared memory as two 64-column chunks of kBK rows each, 8 KB apart -- the
+// N-major operand layout of one CTA's 128-column half of a 256-column stage.
 bool make_map_b_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t rows) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
     cuuint64_t dims[3] = {64, rows, ncols / 64};
     cuuint64_t strides[2] = {ncols * 2, 128};
-    cuuint32_t box[3] = {64, (cuuint32_t)kBK, (cuuint32_t)(kBN / 64)};
+    cuuint32_t box[3] = {64, (cuuint32_t)kBK, (cuuint32_t)(kBN / 128)};
     cuuint32_t estr[3] = {1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -181,14 +181,14 @@ bool make_map_b_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t
 }
 
 // w1 in the concatenated layout [rows][2][I] viewed as (64 columns, rows,
-// I/64 chunks, gate/up half): one box of 64 x kBK x 2 x 2 lands as gate chunks
-// 0,1 then up chunks 0,1 (8 KB apart).
+// I/64 chunks, gate/up half): one box of 64 x kBK x 2 x 1 is two 64-column
+// chunks of the gate half (even CTA) or of the up half (odd CTA), 8 KB apart.
 bool make_map_w1_concat(CUtensorMap *m, const void *ptr, uint64_t I, uint64_t rows) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
     cuuint64_t dims[4] = {64, rows, I / 64, 2};
     cuuint64_t strides[3] = {I * 4, 128, I * 2};
-    cuuint32_t box[4] = {64, (cuuint32_t)kBK, 2, 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)kBK, 2, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -275,7 +275,7 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
     __nv_bfloat16 *hbuf = reinterpret_cast<__nv_bfloat16 *>(w + l.h);
     __nv_bfloat16 *ybuf = reinterpret_cast<__nv_bfloat16 *>(w + l.y);
     if (l.p_cap > 0) {
-        const int64_t cap_mtiles = (l.p_cap + kBM - 1) / kBM + E;
+        const int64_t cap_mtiles = (l.p_cap + kTileRows - 1) / kTileRows + E;
         // ---- up: x gathered rows . w1 -> h
         GemmArgs up;
         memset(&up, 0, sizeof up);
@@ -285,6 +285,7 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
             if (!make_map_b_chunks(&up.tmap_b, w1, (uint64_t)2 * I, (uint64_t)E * H)) return MOE_ERR_CUDA;
         }
         up.x = static_cast<const __nv_bfloat16 *>(x);
+        if (!make_map_2d(&up.tmap_out, hbuf, (uint64_t)I, (uint64_t)l.p_cap, 64, 32)) return MOE_ERR_CUDA;
         up.x_gather_idx = meta.x_gather_idx;
         up.expert_off = meta.expert_frequency_offset;
         up.tile_off = ma.gemm_tile_off;
@@ -298,9 +299,9 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
         up.out_cols = I;
         up.I = I;
         up.layout = layout_kind;
-        int64_t grid = cap_mtiles * up.n_tiles;
-        if (grid > dev.sms) grid = dev.sms;
-        if (launch_gemm_up(up, (int)grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+        int64_t clusters = cap_mtiles * up.n_tiles;
+        if (clusters > dev.sms / 2) clusters = dev.sms / 2;
+        if (launch_gemm_up(up, (int)clusters, s) != cudaSuccess) return MOE_ERR_CUDA;
         if ((st = record(ev, 2, s))) return st;
 
         // ---- down: h . w2 -> y
@@ -308,6 +309,7 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
         memset(&dn, 0, sizeof dn);
         if (!make_map_2d(&dn.tmap_a, hbuf, (uint64_t)I, (uint64_t)l.p_cap, 64, kBM)) return MOE_ERR_CUDA;
         if (!make_map_b_chunks(&dn.tmap_b, w2, (uint64_t)H, (uint64_t)E * I)) return MOE_ERR_CUDA;
+        if (!make_map_2d(&dn.tmap_out, ybuf, (uint64_t)H, (uint64_t)l.p_cap, 64, 32)) return MOE_ERR_CUDA;
         dn.expert_off = meta.expert_frequency_offset;
         dn.tile_off = ma.gemm_tile_off;
         dn.bias = static_cast<const __nv_bfloat16 *>(b2);
@@ -320,9 +322,9 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
         dn.out_cols = H;
         dn.I = I;
         dn.layout = MOE_LAYOUT_INTERLEAVED;
-        grid = cap_mtiles * dn.n_tiles;
-        if (grid > dev.sms) grid = dev.sms;
-        if (launch_gemm_down(dn, (int)grid, s) != cudaSuccess) return MOE_ERR_CUDA;
+        clusters = cap_mtiles * dn.n_tiles;
+        if (clusters > dev.sms / 2) clusters = dev.sms / 2;
+        if (launch_gemm_down(dn, (int)clusters, s) != cudaSuccess) return MOE_ERR_CUDA;
         if ((st = record(ev, 3, s))) return st;
     } else {
         if ((st = record(ev, 2, s))) return st;

@@ -25,7 +25,8 @@ struct WsHeader {
 static_assert(sizeof(WsHeader) == 256, "header size");
 
 // Tile sizes of the grouped GEMMs.
-constexpr int kBM = 128;        // rows (pairs) per tile = UMMA M
+constexpr int kBM = 128;        // rows (pairs) per CTA of a tile
+constexpr int kTileRows = 256;  // rows per GEMM tile (a CTA pair); the metadata's tile table counts these
 constexpr int kBN = 256;        // accumulator columns per tile = UMMA N
 constexpr int kBK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
 constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
@@ -58,7 +59,7 @@ struct MetaArgs {
     int32_t *tile_hist;   // [T,E]
     int32_t *tile_valid;  // [T]
     int32_t *tile_err;    // [T]
-    int32_t *gemm_tile_off;  // [E+1]
+    int32_t *gemm_tile_off;  // [E+1] prefix of ceil(freq / kTileRows)
     moe_meta_t meta;
     int64_t N;
 };
@@ -66,7 +67,8 @@ struct MetaArgs {
 struct GemmArgs {
     CUtensorMap tmap_a;       // down: h [P_cap,I], box 64 x 128 (up: unused)
     CUtensorMap tmap_b;       // w1 / w2 viewed as (64 columns, K rows, column chunk[, half]):
-                              // one box = a whole 64 x 256 stage of B
+                              // one box = this CTA's 64 x 128 half of a B stage
+    CUtensorMap tmap_out;     // h [P_cap,I] / y [P_cap,H], box 64 columns x 32 rows (stores)
     const __nv_bfloat16 *x;   // up: x [N,H], rows gathered with cp.async
     const int32_t *x_gather_idx;
     const int32_t *expert_off;    // [E+1]
@@ -85,8 +87,8 @@ struct GemmArgs {
 
 // Launchers (each defined next to its kernel).
 cudaError_t launch_meta(const MetaArgs &a, cudaStream_t s);
-cudaError_t launch_gemm_up(const GemmArgs &a, int grid, cudaStream_t s);
-cudaError_t launch_gemm_down(const GemmArgs &a, int grid, cudaStream_t s);
+cudaError_t launch_gemm_up(const GemmArgs &a, int max_clusters, cudaStream_t s);
+cudaError_t launch_gemm_down(const GemmArgs &a, int max_clusters, cudaStream_t s);
 cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *token_offset, const int32_t *s_rev,
                            const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
                            const WsHeader *hdr, int num_sms, cudaStream_t s);
@@ -218,6 +220,25 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// TMA store of a shared-memory box to global memory (bulk-group completion).
+__device__ __forceinline__ void tma_store_2d(const void *tmap, uint32_t src, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// The shared-memory sources of this thread's committed stores have been read.
+__device__ __forceinline__ void bulk_wait_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// This thread's committed stores are complete.
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -243,9 +264,11 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
 }
-// Arrive on an mbarrier given by its cluster address (possibly in the peer CTA).
+// Arrive on an mbarrier given by its cluster address (possibly in the peer
+// CTA), with the default (CTA-scope release) semantics: a cluster-scope
+// release made every arrive cost about three stages' worth of MMA time.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // Whole-cluster barrier, called by every thread of both CTAs.
 __device__ __forceinline__ void cluster_sync_all() {

@@ -1,7 +1,6 @@
-// Grouped GEMMs over the expert-sorted pair segments, tcgen05 + TMEM + TMA,
-// for sm_100a.  One persistent CTA per SM walks a static round-robin list of
-// output tiles; a tile is (expert e, 128 rows of e's segment, 256 accumulator
-// columns).  The grouped GEMM is the compute core of the layer (sonic-moe
+// Grouped GEMMs over the expert-sorted pair segments on sm_100a: tcgen05 MMAs
+// with TMEM accumulators, issued for a CTA pair (cta_group::2), fed by TMA and
+// cp.async.  The grouped GEMM is the compute core of the layer (sonic-moe
 // write-up, "CuTeDSL, Triton and QuACK grouped GEMM kernels"; issue #68: the
 // grouped GEMM consumes the metadata unchanged).
 //
@@ -9,50 +8,65 @@
 //                       h[p, j] = silu(gate_j) * up_j   (bf16 [P_cap, I])
 //        The A rows are gathered from x by four producer warps with 16-byte
 //        cp.async copies written straight into the 128-byte-swizzled stage
-//        (one TMA instruction per four rows proved too slow: a stage needed 32
-//        of them), so no permuted copy of x is ever written.  The SwiGLU ("silu
-//        times up", qwen3_5.py commit notes, recipe step 4) runs in the
-//        epilogue on the fp32 accumulator.  Interleaved w1 columns
-//        (g0,u0,g1,u1,...) give gate/up in adjacent accumulator columns;
-//        concatenated w1 (all gates, then all ups; sonic-moe write-up,
-//        "Interleaved by default, concatenated if your model is
-//        HuggingFace") is loaded as 128 gate columns + the matching 128 up
-//        columns, so gate and up land in columns c and c+128.
+//        (one TMA tile::gather4 per four rows proved too slow: a stage needed
+//        32 of them and the TMA unit became the bottleneck), so no permuted
+//        copy of x is ever written.  The SwiGLU ("silu times up", qwen3_5.py
+//        commit notes, recipe step 4) runs in the epilogue on the fp32
+//        accumulator.  Interleaved w1 columns (g0,u0,g1,u1,...) give gate/up in
+//        adjacent accumulator columns; with concatenated w1 (all gates, then
+//        all ups; sonic-moe write-up, "Interleaved by default, concatenated if
+//        your model is HuggingFace") the even CTA loads 128 gate columns and
+//        the odd CTA the matching 128 up columns, so gate and up land in
+//        accumulator columns c and c+128.
 //   down (kUp = false): y[p, :] = h[p, :] . w2[e] (+ b2[e])  (bf16 [P_cap, H])
 //
-// Warp roles: warp 0 = TMA producer (B; and A for the down GEMM), warp 1 =
-// TMEM allocator and single-thread MMA issuer, warps 2-5 = epilogue (TMEM lane
-// quarter warp%4), warps 6-9 (up only) = A-row gather.  Each B stage (64 K-rows
-// x 256 columns) is one TMA box of a 3-D / 4-D view of the weights.
-// Pipeline: kStages shared-memory stages (A 128x64 + B 64x256 bf16, 128-byte
-// swizzle), two TMEM accumulators of 128x256 fp32 so the epilogue of one tile
-// overlaps the MMAs of the next.  Rows past the end of an expert's segment are
-// computed (clamped gather / neighbouring rows) but never stored.
+// Tiles: a cluster of two CTAs owns a tile of 256 rows of one expert's
+// segment x 256 accumulator columns.  CTA r holds A rows [128r, 128r+128) and
+// B columns [128r, 128r+128) of each stage (16 KB + 16 KB), and its TMEM holds
+// the fp32 accumulator of its 128 rows.  The even CTA issues the pair MMA
+// (M=256, N=256, K=16) for both; commits are multicast to both CTAs' barriers.
+// Clusters walk a static round-robin list of tiles, row-tile major so that
+// consecutive clusters share the gathered A rows in L2.
 //
-// Every wait is bounded (common.cuh); on a timeout the CTA raises a shared
-// abort flag, records MOE_DEVERR_TIMEOUT, drains its in-flight copies and
-// MMAs, frees its TMEM and returns.
+// Warp roles per CTA: warp 0 = TMA producer (B; A for the down GEMM), warp 1 =
+// TMEM allocator, and the MMA issuer (even CTA) or, in the up GEMM, the relay
+// that tells the even CTA when the odd CTA's gathered rows have landed (odd
+// CTA); warps 2-5 = epilogue (TMEM lane quarter warp%4); warps 6-9 (up only)
+// = A-row gather.  Six shared-memory stages; two TMEM accumulators so the
+// epilogue of one tile overlaps the MMAs of the next.  Rows past the end of an
+// expert's segment are computed (clamped gather / neighbouring rows) but never
+// stored.
+//
+// Every wait is bounded (common.cuh); on a timeout a CTA raises its abort
+// flag, records MOE_DEVERR_TIMEOUT, drains what it has in flight and returns
+// through the final cluster barrier with its TMEM freed.
 #include "common.cuh"
 
 namespace moe {
 
 namespace {
 
+constexpr int kPairM = 256;                     // rows per tile (two CTAs x kBM)
+constexpr int kPairStages = 6;
 constexpr int kGatherWarps = 4;
 constexpr int kGatherThreads = 32 * kGatherWarps;
-__host__ __device__ constexpr int threads_of(bool up) { return up ? 192 + kGatherThreads : 192; }
-constexpr uint32_t kStageA = kBM * kBK * 2;   // 16 KB
-constexpr uint32_t kStageB = kBK * kBN * 2;   // 32 KB: 4 chunks of 64 K-rows x 64 N-columns
-constexpr uint32_t kChunkB = kBK * 64 * 2;    // 8 KB
+constexpr uint32_t kStageA = kBM * kBK * 2;     // 16 KB: this CTA's 128 rows x 64 K
+constexpr uint32_t kStageB = kBK * (kBN / 2) * 2;  // 16 KB: this CTA's 128 columns x 64 K
+constexpr uint32_t kChunkB = kBK * 64 * 2;      // 8 KB: 64 columns x 64 K
 constexpr uint32_t kStageBytes = kStageA + kStageB;
-constexpr uint32_t kTmemCols = 2 * kBN;       // two accumulators
-constexpr uint32_t kNumBars = 2 * kStages + 5;
-constexpr uint32_t kIdesc = idesc_bf16_f32(kBM, kBN, /*b_mn_major=*/true);
+constexpr uint32_t kTmemCols = 2 * kBN;         // two accumulators
+constexpr uint32_t kNumBars = 3 * kPairStages + 5;
+constexpr uint32_t kIdesc = idesc_bf16_f32(kPairM, kBN, /*b_mn_major=*/true);
+constexpr unsigned long long kAbortSettleNs = 2000000ull;
 
-constexpr size_t kSmemBarOff = (size_t)kStages * kStageBytes;
+constexpr uint32_t kStoreBuf = 32 * 128;        // 4 KB per epilogue warp: 32 rows x 64 bf16
+constexpr size_t kSmemStoreOff = (size_t)kPairStages * kStageBytes;
+constexpr size_t kSmemBarOff = kSmemStoreOff + 4 * kStoreBuf;
 constexpr size_t kSmemMiscOff = kSmemBarOff + 8 * kNumBars;
 constexpr size_t kSmemTableOff = kSmemMiscOff + 16;
 constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kSmemTableOff + 2 * (kMaxExperts + 1) * 4;
+
+__host__ __device__ constexpr int threads_of(bool up) { return up ? 192 + kGatherThreads : 192; }
 
 struct Tile {
     int e, m0, m_end, nt;
@@ -70,63 +84,75 @@ __device__ __forceinline__ Tile decode_tile(int tile, int n_tiles, int E, const 
         else hi = mid - 1;
     }
     t.e = lo;
-    t.m0 = off[lo] + (mt - tile_off[lo]) * kBM;
+    t.m0 = off[lo] + (mt - tile_off[lo]) * kPairM;
     t.m_end = off[lo + 1];
     return t;
 }
 
-__device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+// silu(g) * u; for very negative g the quotient underflows to 0 as silu does.
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
-__device__ __forceinline__ void load_bias32(const __nv_bfloat16 *b, float (&v)[32]) {
+// r[i] (fp32 bits) += bias[i] for 32 consecutive columns; nothing when bias is null.
+__device__ __forceinline__ void add_bias32(uint32_t (&r)[32], const __nv_bfloat16 *b) {
+    if (!b) return;
     const uint4 *p = reinterpret_cast<const uint4 *>(b);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint4 w = __ldg(p + i);
-        v[8 * i + 0] = bf16lo(w.x);
-        v[8 * i + 1] = bf16hi(w.x);
-        v[8 * i + 2] = bf16lo(w.y);
-        v[8 * i + 3] = bf16hi(w.y);
-        v[8 * i + 4] = bf16lo(w.z);
-        v[8 * i + 5] = bf16hi(w.z);
-        v[8 * i + 6] = bf16lo(w.w);
-        v[8 * i + 7] = bf16hi(w.w);
+        const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            r[8 * i + 2 * j] = __float_as_uint(__uint_as_float(r[8 * i + 2 * j]) + bf16lo(q[j]));
+            r[8 * i + 2 * j + 1] = __float_as_uint(__uint_as_float(r[8 * i + 2 * j + 1]) + bf16hi(q[j]));
+        }
+    }
+}
+
+__device__ __forceinline__ void settle_after_abort() {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < kAbortSettleNs) {
     }
 }
 
 template <bool kUp>
-__global__ void __launch_bounds__(threads_of(kUp), 1) grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
+    grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
     constexpr int kThreads = threads_of(kUp);
     extern __shared__ uint8_t smem_raw[];
+    // uniform for both CTAs of the pair: they return together
     if (*(volatile uint32_t *)&a.hdr->abort) return;
 
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *base_ptr = smem_raw + (base - raw);
     const uint32_t sA = base;
-    const uint32_t sB = base + kStages * kStageA;
+    const uint32_t sB = base + kPairStages * kStageA;
     const uint32_t bars = base + (uint32_t)kSmemBarOff;
     auto full_bar = [&](int s) { return bars + 8u * s; };
-    auto empty_bar = [&](int s) { return bars + 8u * (kStages + s); };
-    auto tfull_bar = [&](int b) { return bars + 8u * (2 * kStages + b); };
-    auto tempty_bar = [&](int b) { return bars + 8u * (2 * kStages + 2 + b); };
-    const uint32_t drain_bar = bars + 8u * (2 * kStages + 4);
+    auto empty_bar = [&](int s) { return bars + 8u * (kPairStages + s); };
+    auto gfull_bar = [&](int s) { return bars + 8u * (2 * kPairStages + s); };
+    auto tfull_bar = [&](int b) { return bars + 8u * (3 * kPairStages + b); };
+    auto tempty_bar = [&](int b) { return bars + 8u * (3 * kPairStages + 2 + b); };
+    const uint32_t drain_bar = bars + 8u * (3 * kPairStages + 4);
     uint32_t *misc = reinterpret_cast<uint32_t *>(base_ptr + kSmemMiscOff);
     int *tile_off_s = reinterpret_cast<int *>(base_ptr + kSmemTableOff);
     int *off_s = tile_off_s + (kMaxExperts + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
     const int E = a.E;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            // TMA producer's arrive (+ transaction bytes), plus one cp.async
-            // arrival per gather thread in the up GEMM
-            mbar_init(full_bar(s), 1 + (kUp ? kGatherThreads : 0));
+        for (int s = 0; s < kPairStages; ++s) {
+            // even CTA: producer's arrive (+ both CTAs' TMA bytes), plus the odd
+            // CTA's relay in the up GEMM
+            mbar_init(full_bar(s), 1 + (kUp ? 1 : 0));
             mbar_init(empty_bar(s), 1);
+            mbar_init(gfull_bar(s), kGatherThreads);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), 4);
+            mbar_init(tempty_bar(b), 8);  // 4 epilogue warps x 2 CTAs
         }
         mbar_init(drain_bar, 1);
         misc[1] = 0;
@@ -141,11 +167,11 @@ __global__ void __launch_bounds__(threads_of(kUp), 1) grouped_gemm_kernel(const 
         off_s[i] = __ldg(a.expert_off + i);
     }
     if (warp == 1) {
-        tmem_alloc(smem_u32(&misc[0]), kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_u32(&misc[0]), kTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // barriers of both CTAs initialised before any remote arrive
     tc_fence_after();
 
     const uint32_t tmem_base = misc[0];
@@ -153,15 +179,18 @@ __global__ void __launch_bounds__(threads_of(kUp), 1) grouped_gemm_kernel(const 
     const int n_tiles = a.n_tiles;
     const int total_tiles = tile_off_s[E] * n_tiles;
     const int nk = a.k_dim / kBK;
+    const int cluster = blockIdx.x >> 1;
+    const int n_clusters = gridDim.x >> 1;
+    const int row0 = (int)rank * kBM;  // this CTA's first row inside a tile
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        constexpr uint32_t kTxBytes = kUp ? kStageB : kStageBytes;
+        constexpr uint32_t kTxBytes = 2 * (kUp ? kStageB : kStageBytes);  // both CTAs' TMA bytes
         int stage = 0;
         uint32_t phase = 0;
         uint32_t issued = 0, issued_parity = 0;
         if (lane == 0) {
-            for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+            for (int tile = cluster; tile < total_tiles; tile += n_clusters) {
                 const Tile t = decode_tile(tile, n_tiles, E, tile_off_s, off_s);
                 const int brow0 = t.e * a.k_dim;
                 bool ok = true;
@@ -170,79 +199,106 @@ __global__ void __launch_bounds__(threads_of(kUp), 1) grouped_gemm_kernel(const 
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(full_bar(stage), kTxBytes);
+                    if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), kTxBytes);
+                    const uint32_t fb = mapa_shared(full_bar(stage), 0);
                     const int k0 = kb * kBK;
                     const uint32_t b_dst = sB + stage * kStageB;
-                    if (!kUp) tma_load_2d(sA + stage * kStageA, &a.tmap_a, full_bar(stage), k0, t.m0);
+                    if (!kUp) tma_load_2d_pair(sA + stage * kStageA, &a.tmap_a, fb, k0, t.m0 + row0);
                     if (kUp && a.layout == MOE_LAYOUT_CONCATENATED)
-                        tma_load_4d(b_dst, &a.tmap_b, full_bar(stage), 0, brow0 + k0, t.nt * 2, 0);
+                        tma_load_4d_pair(b_dst, &a.tmap_b, fb, 0, brow0 + k0, t.nt * 2, (int)rank);
                     else
-                        tma_load_3d(b_dst, &a.tmap_b, full_bar(stage), 0, brow0 + k0, t.nt * 4);
+                        tma_load_3d_pair(b_dst, &a.tmap_b, fb, 0, brow0 + k0, t.nt * 4 + 2 * (int)rank);
                     issued |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-                    if (++stage == kStages) {
+                    if (++stage == kPairStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
             }
-            // every copy this CTA issued must land before the CTA may exit
-            for (int s = 0; s < kStages; ++s)
-                if (issued & (1u << s)) mbar_wait_timed(full_bar(s), (issued_parity >> s) & 1u);
+            // the even CTA's full barriers count both CTAs' bytes: wait for every
+            // phase this CTA issued before the CTA may exit
+            if (rank == 0)
+                for (int s = 0; s < kPairStages; ++s)
+                    if (issued & (1u << s)) mbar_wait_timed(full_bar(s), (issued_parity >> s) & 1u);
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        if (rank == 0) {
+            // ---------------------------------------------------- MMA issuer
+            if (lane == 0) {
+                int stage = 0;
+                uint32_t phase = 0;
+                int tcount = 0;
+                bool ok = true;
+                for (int tile = cluster; ok && tile < total_tiles; tile += n_clusters, ++tcount) {
+                    const int acc = tcount & 1;
+                    const uint32_t acc_phase = (tcount >> 1) & 1;
+                    if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort)) break;
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + acc * kBN;
+                    for (int kb = 0; kb < nk; ++kb) {
+                        if (!mbar_wait_bounded(full_bar(stage), phase, abort) ||
+                            (kUp && !mbar_wait_bounded(gfull_bar(stage), phase, abort))) {
+                            ok = false;
+                            break;
+                        }
+                        if (kUp) fence_proxy_async_smem();
+                        tc_fence_after();
+                        const uint32_t a_addr = sA + stage * kStageA;
+                        const uint32_t b_addr = sB + stage * kStageB;
+#pragma unroll
+                        for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                            // A: K-major, 128-byte rows, 8-row atoms 1024 B apart; K step 32 B.
+                            const uint64_t adesc = smem_desc_sw128(a_addr + kk * (kUmmaK * 2), 16, 1024);
+                            // B: N-major, 64-column chunks 8 KB apart (LBO), 8-row K atoms
+                            // 1024 B apart (SBO); K step = 16 rows = 2 KB.
+                            const uint64_t bdesc =
+                                smem_desc_sw128(b_addr + kk * (kUmmaK * 128), kChunkB, 1024);
+                            umma_f16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                        umma_commit_pair_mc(empty_bar(stage), 0x3);
+                        if (++stage == kPairStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit_pair_mc(tfull_bar(acc), 0x3);
+                }
+                // all pair MMAs issued here complete before TMEM is freed
+                umma_commit_pair(drain_bar);
+                mbar_wait_timed(drain_bar, 0);
+            }
+        } else if (kUp && lane == 0) {
+            // ------------------------------------------- relay (odd CTA, up)
             int stage = 0;
             uint32_t phase = 0;
-            int tcount = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total_tiles; tile += gridDim.x, ++tcount) {
-                const int acc = tcount & 1;
-                const uint32_t acc_phase = (tcount >> 1) & 1;
-                if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * kBN;
+            for (int tile = cluster; ok && tile < total_tiles; tile += n_clusters) {
                 for (int kb = 0; kb < nk; ++kb) {
-                    if (!mbar_wait_bounded(full_bar(stage), phase, abort)) {
+                    if (!mbar_wait_bounded(gfull_bar(stage), phase, abort)) {
                         ok = false;
                         break;
                     }
-                    if (kUp) fence_proxy_async_smem();
-                    tc_fence_after();
-                    const uint32_t a_addr = sA + stage * kStageA;
-                    const uint32_t b_addr = sB + stage * kStageB;
-#pragma unroll
-                    for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-                        // A: K-major, 128-byte rows, 8-row atoms 1024 B apart; K step = 32 B.
-                        const uint64_t adesc = smem_desc_sw128(a_addr + kk * (kUmmaK * 2), 16, 1024);
-                        // B: N-major, 64-column chunks 8 KB apart (LBO), 8-row K atoms
-                        // 1024 B apart (SBO); K step = 16 rows = 2 KB.
-                        const uint64_t bdesc = smem_desc_sw128(b_addr + kk * (kUmmaK * 128), kChunkB, 1024);
-                        umma_f16(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
-                    }
-                    umma_commit(empty_bar(stage));
-                    if (++stage == kStages) {
+                    fence_proxy_async_smem();
+                    mbar_arrive_cluster(mapa_shared(full_bar(stage), 0));
+                    if (++stage == kPairStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
-                if (!ok) break;
-                umma_commit(tfull_bar(acc));
             }
-            // all MMAs issued by this thread complete before TMEM is freed
-            umma_commit(drain_bar);
-            mbar_wait_timed(drain_bar, 0);
         }
         __syncwarp();
     } else if (warp < 6) {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;
-        const int row = quarter * 32 + lane;
+        const int row = row0 + quarter * 32 + lane;
+        const uint32_t store_buf = base + (uint32_t)kSmemStoreOff + (uint32_t)(warp - 2) * kStoreBuf;
         int tcount = 0;
-        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++tcount) {
+        for (int tile = cluster; tile < total_tiles; tile += n_clusters, ++tcount) {
             const Tile t = decode_tile(tile, n_tiles, E, tile_off_s, off_s);
             const int acc = tcount & 1;
             const uint32_t acc_phase = (tcount >> 1) & 1;
@@ -253,116 +309,133 @@ __global__ void __launch_bounds__(threads_of(kUp), 1) grouped_gemm_kernel(const 
             tc_fence_after();
             const int p = t.m0 + row;
             const bool valid = p < t.m_end;
+            // whole warp inside the segment: stage in shared memory, one TMA store
+            // per 32 x 64 block; otherwise masked per-row stores
+            const bool warp_full = t.m0 + row0 + quarter * 32 + 31 < t.m_end;
+            const int wrow0 = t.m0 + row0 + quarter * 32;
             const uint32_t tbase = tmem_base + acc * kBN + ((uint32_t)(quarter * 32) << 16);
             __nv_bfloat16 *orow = a.out + (size_t)(valid ? p : 0) * a.out_cols;
             const __nv_bfloat16 *brow = a.bias ? a.bias + (size_t)t.e * a.n_dim : nullptr;
 
+            // 64 output columns (32 packed bf16 pairs) of this thread's row
+            auto store64 = [&](int col0, const uint32_t (&v)[32]) {
+                if (warp_full) {
+                    if (lane == 0) bulk_wait_read0();  // the buffer's previous store has been read
+                    __syncwarp();
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const int rr = lane;  // row inside the warp's 32-row block
+                        st_shared_v4(store_buf + rr * 128 + ((c ^ (rr & 7)) << 4), v[4 * c], v[4 * c + 1],
+                                     v[4 * c + 2], v[4 * c + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&a.tmap_out, store_buf, col0, wrow0);
+                        bulk_commit();
+                    }
+                } else if (valid) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + col0);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        dst[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                }
+            };
+
             if (kUp && a.layout == MOE_LAYOUT_CONCATENATED) {
                 // gate = accumulator columns [0,128), up = [128,256)
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    const int col = t.nt * (kBN / 2) + c * 32;  // output column = gate column
-                    if (col >= a.I) break;
-                    uint32_t g[32], u[32];
-                    tmem_ld_32x32b_x32(tbase + c * 32, g);
-                    tmem_ld_32x32b_x32(tbase + 128 + c * 32, u);
-                    tmem_ld_wait();
-                    float bg[32], bu[32];
-                    if (brow) {
-                        load_bias32(brow + col, bg);
-                        load_bias32(brow + a.I + col, bu);
-                    } else {
+                for (int gi = 0; gi < 2; ++gi) {
+                    const int col0 = t.nt * (kBN / 2) + gi * 64;  // output column = gate column
+                    if (col0 >= a.I) break;
+                    uint32_t packed[32];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) bg[i] = bu[i] = 0.f;
-                    }
-                    uint32_t packed[16];
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int c = 2 * gi + hf;
+                        uint32_t g[32], u[32];
+                        tmem_ld_32x32b_x32(tbase + c * 32, g);
+                        tmem_ld_32x32b_x32(tbase + 128 + c * 32, u);
+                        tmem_ld_wait();
+                        if (brow) {
+                            add_bias32(g, brow + col0 + hf * 32);
+                            add_bias32(u, brow + a.I + col0 + hf * 32);
+                        }
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float h0 = silu_mul(__uint_as_float(g[2 * i]) + bg[2 * i],
-                                                  __uint_as_float(u[2 * i]) + bu[2 * i]);
-                        const float h1 = silu_mul(__uint_as_float(g[2 * i + 1]) + bg[2 * i + 1],
-                                                  __uint_as_float(u[2 * i + 1]) + bu[2 * i + 1]);
-                        packed[i] = pack_bf16x2(h0, h1);
+                        for (int i = 0; i < 16; ++i) {
+                            const float h0 = silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]));
+                            const float h1 =
+                                silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]));
+                            packed[16 * hf + i] = pack_bf16x2(h0, h1);
+                        }
                     }
-                    if (valid) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
-                                                packed[4 * i + 3]);
-                    }
+                    store64(col0, packed);
                 }
             } else if (kUp) {
                 // interleaved: accumulator columns (2j, 2j+1) = (gate_j, up_j)
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    const int acol = t.nt * kBN + c * 32;  // column of w1
-                    if (acol >= a.n_dim) break;
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tbase + c * 32, r);
-                    tmem_ld_wait();
-                    float b[32];
-                    if (brow) {
-                        load_bias32(brow + acol, b);
-                    } else {
+                for (int gi = 0; gi < 2; ++gi) {
+                    const int col0 = t.nt * (kBN / 2) + gi * 64;  // output column
+                    if (col0 >= a.out_cols) break;
+                    uint32_t packed[32];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) b[i] = 0.f;
-                    }
-                    uint32_t packed[8];
+                    for (int hf = 0; hf < 2; ++hf) {
+                        const int c = 4 * gi + 2 * hf;  // first of two 32-column accumulator chunks
+                        uint32_t r0[32], r1[32];
+                        tmem_ld_32x32b_x32(tbase + c * 32, r0);
+                        tmem_ld_32x32b_x32(tbase + (c + 1) * 32, r1);
+                        tmem_ld_wait();
+                        const int acol = t.nt * kBN + c * 32;
+                        if (brow) {
+                            add_bias32(r0, brow + acol);
+                            add_bias32(r1, brow + acol + 32);
+                        }
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float h0 = silu_mul(__uint_as_float(r[4 * i + 0]) + b[4 * i + 0],
-                                                  __uint_as_float(r[4 * i + 1]) + b[4 * i + 1]);
-                        const float h1 = silu_mul(__uint_as_float(r[4 * i + 2]) + b[4 * i + 2],
-                                                  __uint_as_float(r[4 * i + 3]) + b[4 * i + 3]);
-                        packed[i] = pack_bf16x2(h0, h1);
+                        for (int i = 0; i < 8; ++i) {
+                            packed[16 * hf + i] =
+                                pack_bf16x2(silu_mul(__uint_as_float(r0[4 * i]), __uint_as_float(r0[4 * i + 1])),
+                                            silu_mul(__uint_as_float(r0[4 * i + 2]), __uint_as_float(r0[4 * i + 3])));
+                            packed[16 * hf + 8 + i] =
+                                pack_bf16x2(silu_mul(__uint_as_float(r1[4 * i]), __uint_as_float(r1[4 * i + 1])),
+                                            silu_mul(__uint_as_float(r1[4 * i + 2]), __uint_as_float(r1[4 * i + 3])));
+                        }
                     }
-                    if (valid) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + acol / 2);
-                        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-                    }
+                    store64(col0, packed);
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    const int col = t.nt * kBN + c * 32;
-                    if (col >= a.n_dim) break;
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(tbase + c * 32, r);
+                for (int gi = 0; gi < 4; ++gi) {
+                    const int col0 = t.nt * kBN + gi * 64;
+                    if (col0 >= a.n_dim) break;
+                    uint32_t r0[32], r1[32];
+                    tmem_ld_32x32b_x32(tbase + gi * 64, r0);
+                    tmem_ld_32x32b_x32(tbase + gi * 64 + 32, r1);
                     tmem_ld_wait();
-                    float b[32];
+                    uint32_t packed[32];
                     if (brow) {
-                        load_bias32(brow + col, b);
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) b[i] = 0.f;
+                        add_bias32(r0, brow + col0);
+                        add_bias32(r1, brow + col0 + 32);
                     }
-                    uint32_t packed[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        packed[i] = pack_bf16x2(__uint_as_float(r[2 * i]) + b[2 * i],
-                                                __uint_as_float(r[2 * i + 1]) + b[2 * i + 1]);
-                    if (valid) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + col);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2],
-                                                packed[4 * i + 3]);
+                    for (int i = 0; i < 16; ++i) {
+                        packed[i] = pack_bf16x2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+                        packed[16 + i] = pack_bf16x2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
                     }
+                    store64(col0, packed);
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(acc));
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(tempty_bar(acc));
+                else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+            }
         }
-    }
-
-    if (kUp && warp >= 6) {
+        if (lane == 0) bulk_wait0();  // this warp's stores have landed
+    } else if (kUp) {
         // ------------------------------------------------------- A-row gather
-        // thread g: 16-byte chunk (g & 7) of rows (g >> 3) + 16 i, i = 0..7,
-        // stored at row * 128 + ((chunk ^ (row & 7)) << 4): the 128-byte
-        // swizzle the MMA descriptors expect.
+        // thread g: 16-byte chunk (g & 7) of rows (g >> 3) + 16 i, i = 0..7 of
+        // this CTA's 128 rows, stored at row * 128 + ((chunk ^ (row & 7)) << 4):
+        // the 128-byte swizzle the MMA descriptors expect.
         const int g = threadIdx.x - 192;
         const int chunk = g & 7;
         const int r0 = g >> 3;
@@ -371,14 +444,14 @@ __global__ void __launch_bounds__(threads_of(kUp), 1) grouped_gemm_kernel(const 
         uint32_t phase = 0;
         const char *xb = reinterpret_cast<const char *>(a.x);
         const size_t ld = (size_t)a.k_dim * 2;
-        int tile = blockIdx.x;
+        int tile = cluster;
         Tile t{};
         const char *src[8];
-        auto load_rows = [&](const Tile &tt, const char *(&p)[8]) {
+        auto load_rows = [&](const Tile &tt, const char *(&pp)[8]) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int pr = min(tt.m0 + r0 + 16 * i, tt.m_end - 1);
-                p[i] = xb + (size_t)__ldg(a.x_gather_idx + pr) * ld + chunk * 16;
+                const int pr = min(tt.m0 + row0 + r0 + 16 * i, tt.m_end - 1);
+                pp[i] = xb + (size_t)__ldg(a.x_gather_idx + pr) * ld + chunk * 16;
             }
         };
         if (tile < total_tiles) {
@@ -386,8 +459,8 @@ __global__ void __launch_bounds__(threads_of(kUp), 1) grouped_gemm_kernel(const 
             load_rows(t, src);
         }
         bool ok = true;
-        for (; ok && tile < total_tiles; tile += gridDim.x) {
-            const int next = tile + gridDim.x;
+        for (; ok && tile < total_tiles; tile += n_clusters) {
+            const int next = tile + n_clusters;
             Tile tn = t;
             const char *nsrc[8];
 #pragma unroll
@@ -408,11 +481,11 @@ __global__ void __launch_bounds__(threads_of(kUp), 1) grouped_gemm_kernel(const 
                 const size_t koff = (size_t)kb * kBK * 2;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const int row = r0 + 16 * i;
-                    cp_async_16(a_dst + row * 128 + ((chunk ^ (row & 7)) << 4), src[i] + koff);
+                    const int rr = r0 + 16 * i;
+                    cp_async_16(a_dst + rr * 128 + ((chunk ^ (rr & 7)) << 4), src[i] + koff);
                 }
-                cp_async_arrive_noinc(full_bar(stage));
-                if (++stage == kStages) {
+                cp_async_arrive_noinc(gfull_bar(stage));
+                if (++stage == kPairStages) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -424,28 +497,50 @@ __global__ void __launch_bounds__(threads_of(kUp), 1) grouped_gemm_kernel(const 
         cp_async_wait_all();
     }
 
+    // ---------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
+    if (*abort) {
+        if (threadIdx.x == 0) atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);
+        settle_after_abort();  // let copies issued by the peer CTA land
+    }
+    cluster_sync_all();  // no CTA leaves while its peer may still touch it
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
-    if (threadIdx.x == 0 && *abort) atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);
 }
 
 template <bool kUp>
-cudaError_t launch(const GemmArgs &a, int grid, cudaStream_t s) {
-    static bool configured[64] = {};
+cudaError_t launch(const GemmArgs &a, int max_clusters, cudaStream_t s) {
+    static int clusters_cache[64][2] = {};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
-    if (dev < 64 && !configured[dev]) {
+    if (dev >= 64) return cudaErrorInvalidDevice;
+    int &fit = clusters_cache[dev][kUp ? 1 : 0];
+    if (fit == 0) {
         err = cudaFuncSetAttribute(grouped_gemm_kernel<kUp>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)kSmemBytes);
         if (err != cudaSuccess) return err;
-        configured[dev] = true;
+        int sms = 0;
+        err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (err != cudaSuccess) return err;
+        // the kernel's cluster shape (2,1,1) is compiled in (__cluster_dims__)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(sms & ~1));
+        cfg.blockDim = dim3(threads_of(kUp));
+        cfg.dynamicSmemBytes = kSmemBytes;
+        cfg.attrs = nullptr;
+        cfg.numAttrs = 0;
+        int n = 0;
+        err = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<kUp>, &cfg);
+        if (err != cudaSuccess) return err;
+        fit = n > 0 ? n : 1;
     }
-    grouped_gemm_kernel<kUp><<<grid, threads_of(kUp), kSmemBytes, s>>>(a);
+    int clusters = fit < max_clusters ? fit : max_clusters;
+    if (clusters < 1) clusters = 1;
+    grouped_gemm_kernel<kUp><<<2 * clusters, threads_of(kUp), kSmemBytes, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -453,7 +548,11 @@ cudaError_t launch(const GemmArgs &a, int grid, cudaStream_t s) {
 
 size_t gemm_smem_bytes() { return kSmemBytes; }
 
-cudaError_t launch_gemm_up(const GemmArgs &a, int grid, cudaStream_t s) { return launch<true>(a, grid, s); }
-cudaError_t launch_gemm_down(const GemmArgs &a, int grid, cudaStream_t s) { return launch<false>(a, grid, s); }
+cudaError_t launch_gemm_up(const GemmArgs &a, int max_clusters, cudaStream_t s) {
+    return launch<true>(a, max_clusters, s);
+}
+cudaError_t launch_gemm_down(const GemmArgs &a, int max_clusters, cudaStream_t s) {
+    return launch<false>(a, max_clusters, s);
+}
 
 }  // namespace moe

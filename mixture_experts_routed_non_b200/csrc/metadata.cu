@@ -195,7 +195,7 @@ __global__ void __launch_bounds__(kMetaThreads) meta_scatter_kernel(const MetaAr
         }
         off[e] = all;             // scanned below
         part_before[e] = before;  // this tile's prefix per expert (rows g > 0 no longer needed)
-        gt[e] = (all + kBM - 1) / kBM;
+        gt[e] = (all + kTileRows - 1) / kTileRows;
     }
     __syncthreads();
     const int P = block_exclusive_scan(off, off, E);
