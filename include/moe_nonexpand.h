@@ -129,6 +129,37 @@ MOE_API int moe_nonexpand_metadata(const int32_t *topk_idx, const float *topk_w,
                            moe_stream_t stream);
 
 /*
+ * moe_nonexpand_metadata without a workspace: the same metadata, bit for bit,
+ * for callers that cannot allocate device memory when they call in -- for
+ * example a serving process whose memory pool is sized and frozen at start-up,
+ * or a plugin whose host framework owns every device allocation -- and so
+ * cannot provide the `ws` buffer the other entry points need.  The pages have
+ * no counterpart to this call; it exists for those callers only.
+ *
+ * Scratch: a fixed 640 KiB array in device memory that belongs to the library
+ * (a file-scope __device__ array: every GPU that loads the library keeps it
+ * until the process exits).  It holds what the metadata kernels need besides
+ * their inputs and outputs -- a header, the per-tile histogram table of at
+ * most 148 tiles x E experts, and the GEMM tile table -- which fits for every
+ * supported size (E <= 1024); a size that would not fit returns MOE_ERR_WS.
+ * The call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ * routine.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array, which keeps the last call's
+ * contents (the kernels write every scratch byte they read, so nothing has to
+ * be cleared): calls that can overlap on the GPU -- on different streams, or
+ * on one device from several host threads without ordering -- race and must
+ * not be issued.  Device-side error bits (bad ids, pair-count mismatch) are
+ * kept in the library's scratch and are not reported by this call; the
+ * outputs follow the same rules as moe_nonexpand_metadata.
+ */
+MOE_API int moe_nonexpand_metadata_noalloc(const int32_t *topk_idx, const float *topk_w,
+                                   int64_t N, int32_t K, int32_t E, int64_t total_pairs,
+                                   const moe_meta_t *meta, moe_stream_t stream);
+
+/*
  * The whole local expert forward: metadata, gathered grouped GEMM up with
  * bias and SwiGLU fused in its epilogue (rows of x are gathered straight
  * through x_gather_idx; no permuted copy of x is made), grouped GEMM down

@@ -42,6 +42,7 @@ EXPORTED = (
     "moe_nonexpand_workspace_layout",
     "moe_nonexpand_read_error",
     "moe_nonexpand_strerror",
+    "moe_nonexpand_metadata_noalloc",
 )
 
 
@@ -93,6 +94,8 @@ def load() -> ctypes.CDLL:
     lib.moe_nonexpand_workspace_layout.argtypes = [i64, i32, i32, i32, i32, i64, ctypes.POINTER(WsLayout)]
     lib.moe_nonexpand_read_error.restype = ctypes.c_int
     lib.moe_nonexpand_read_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.moe_nonexpand_metadata_noalloc.restype = ctypes.c_int
+    lib.moe_nonexpand_metadata_noalloc.argtypes = [P, P, i64, i32, i32, i64, ctypes.POINTER(MoeMeta), P]
     lib.moe_nonexpand_strerror.restype = ctypes.c_char_p
     lib.moe_nonexpand_strerror.argtypes = [ctypes.c_int]
     _lib = lib
@@ -229,6 +232,23 @@ def metadata(topk_idx: torch.Tensor, topk_w: torch.Tensor, E: int, total_pairs: 
     _check(load().moe_nonexpand_metadata(topk_idx.data_ptr(), topk_w.data_ptr(), N, K, E, total_pairs,
                                          ctypes.byref(m), ws.data_ptr(), ws.numel(), _stream_handle(stream)),
            "moe_nonexpand_metadata")
+    return meta
+
+
+def metadata_noalloc(topk_idx: torch.Tensor, topk_w: torch.Tensor, E: int, meta: dict,
+                     total_pairs: int = -1, stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """moe_nonexpand_metadata_noalloc: the metadata into the caller's `meta`
+    buffers (see alloc_meta) using the library's own fixed device scratch, for
+    callers that cannot allocate a workspace.  Calls that can overlap on the
+    GPU must not be issued (they share the scratch)."""
+    N, K = topk_idx.shape
+    dev = topk_idx.device
+    _need(topk_idx, "topk_idx", torch.int32, (N, K), dev)
+    _need(topk_w, "topk_w", torch.float32, (N, K), dev)
+    m = _meta_struct(meta)
+    _check(load().moe_nonexpand_metadata_noalloc(topk_idx.data_ptr(), topk_w.data_ptr(), N, K, E, total_pairs,
+                                                 ctypes.byref(m), _stream_handle(stream)),
+           "moe_nonexpand_metadata_noalloc")
     return meta
 
 
