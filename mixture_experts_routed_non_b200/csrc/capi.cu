@@ -165,15 +165,29 @@ bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer
 }
 
 // A row-major weight [rows][ncols] (ncols % 64 == 0) viewed as
-// (64 columns, rows, ncols/64 column chunks): one box of 64 x kBK x 2 lands in
-// shared memory as two 64-column chunks of kBK rows each, 8 KB apart -- the
+// (64 columns, rows, ncols/64 column chunks): one box of 64 x stage-K x 2 lands in
+// shared memory as two 64-column chunks of stage-K rows each -- the
 // N-major operand layout of one CTA's 128-column half of a 256-column stage.
 bool make_map_b_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t rows) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
     cuuint64_t dims[3] = {64, rows, ncols / 64};
     cuuint64_t strides[2] = {ncols * 2, 128};
-    cuuint32_t box[3] = {64, (cuuint32_t)kBK, (cuuint32_t)(kBN / 128)};
+    cuuint32_t box[3] = {64, (cuuint32_t)kGemmStageK, (cuuint32_t)(kBN / 128)};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// h [rows][I] viewed as (64 columns, rows, I/64 column chunks): one box of
+// 64 x 128 rows x (stage K / 64) is one CTA's A stage, 64-wide K atoms 16 KB apart.
+bool make_map_a_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {64, rows, ncols / 64};
+    cuuint64_t strides[2] = {ncols * 2, 128};
+    cuuint32_t box[3] = {64, (cuuint32_t)kBM, (cuuint32_t)(kGemmStageK / 64)};
     cuuint32_t estr[3] = {1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -181,14 +195,14 @@ bool make_map_b_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t
 }
 
 // w1 in the concatenated layout [rows][2][I] viewed as (64 columns, rows,
-// I/64 chunks, gate/up half): one box of 64 x kBK x 2 x 1 is two 64-column
+// I/64 chunks, gate/up half): one box of 64 x stage-K x 2 x 1 is two 64-column
 // chunks of the gate half (even CTA) or of the up half (odd CTA), 8 KB apart.
 bool make_map_w1_concat(CUtensorMap *m, const void *ptr, uint64_t I, uint64_t rows) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
     cuuint64_t dims[4] = {64, rows, I / 64, 2};
     cuuint64_t strides[3] = {I * 4, 128, I * 2};
-    cuuint32_t box[4] = {64, (cuuint32_t)kBK, 2, 1};
+    cuuint32_t box[4] = {64, (cuuint32_t)kGemmStageK, 2, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -307,7 +321,7 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
         // ---- down: h . w2 -> y
         GemmArgs dn;
         memset(&dn, 0, sizeof dn);
-        if (!make_map_2d(&dn.tmap_a, hbuf, (uint64_t)I, (uint64_t)l.p_cap, 64, kBM)) return MOE_ERR_CUDA;
+        if (!make_map_a_chunks(&dn.tmap_a, hbuf, (uint64_t)I, (uint64_t)l.p_cap)) return MOE_ERR_CUDA;
         if (!make_map_b_chunks(&dn.tmap_b, w2, (uint64_t)H, (uint64_t)E * I)) return MOE_ERR_CUDA;
         if (!make_map_2d(&dn.tmap_out, ybuf, (uint64_t)H, (uint64_t)l.p_cap, 64, 32)) return MOE_ERR_CUDA;
         dn.expert_off = meta.expert_frequency_offset;

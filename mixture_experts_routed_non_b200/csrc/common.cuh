@@ -28,7 +28,11 @@ static_assert(sizeof(WsHeader) == 256, "header size");
 constexpr int kBM = 128;        // rows (pairs) per CTA of a tile
 constexpr int kTileRows = 256;  // rows per GEMM tile (a CTA pair); the metadata's tile table counts these
 constexpr int kBN = 256;        // accumulator columns per tile = UMMA N
-constexpr int kBK = 64;         // K per pipeline stage (one 128-byte swizzle row of bf16)
+constexpr int kBK = 64;         // K of one 128-byte swizzle atom of bf16
+#ifndef MOE_STAGE_K
+#define MOE_STAGE_K 128
+#endif
+constexpr int kGemmStageK = MOE_STAGE_K;  // K per GEMM pipeline stage (64 or 128)
 constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
 constexpr int kStages = 4;      // shared-memory pipeline depth (4 x 48 KB)
 
@@ -65,7 +69,7 @@ struct MetaArgs {
 };
 
 struct GemmArgs {
-    CUtensorMap tmap_a;       // down: h [P_cap,I], box 64 x 128 (up: unused)
+    CUtensorMap tmap_a;       // down: h [P_cap,I] as (64, rows, I/64), box = one CTA's A stage (up: unused)
     CUtensorMap tmap_b;       // w1 / w2 viewed as (64 columns, K rows, column chunk[, half]):
                               // one box = this CTA's 64 x 128 half of a B stage
     CUtensorMap tmap_out;     // h [P_cap,I] / y [P_cap,H], box 64 columns x 32 rows (stores)

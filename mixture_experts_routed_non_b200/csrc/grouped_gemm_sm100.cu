@@ -32,7 +32,9 @@
 // TMEM allocator, and the MMA issuer (even CTA) or, in the up GEMM, the relay
 // that tells the even CTA when the odd CTA's gathered rows have landed (odd
 // CTA); warps 2-5 = epilogue (TMEM lane quarter warp%4); warps 6-9 (up only)
-// = A-row gather.  Six shared-memory stages; two TMEM accumulators so the
+// = A-row gather.  The even CTA's gather threads arrive with cp.async straight
+// on the stage barrier, so the MMA thread checks a single barrier per stage:
+// its per-stage work is on the tensor pipe's critical path.  Six shared-memory stages; two TMEM accumulators so the
 // epilogue of one tile overlaps the MMAs of the next.  Rows past the end of an
 // expert's segment are computed (clamped gather / neighbouring rows) but never
 // stored.
@@ -47,12 +49,18 @@ namespace moe {
 namespace {
 
 constexpr int kPairM = 256;                     // rows per tile (two CTAs x kBM)
-constexpr int kPairStages = 6;
+#ifndef MOE_STAGE_K
+#define MOE_STAGE_K 128
+#endif
+constexpr int kStageK = MOE_STAGE_K;            // K per pipeline stage: 64 or 128
+constexpr int kAtoms = kStageK / 64;            // 128-byte-swizzle atoms along K per stage
+constexpr int kPairStages = kStageK == 128 ? 3 : 6;
 constexpr int kGatherWarps = 4;
 constexpr int kGatherThreads = 32 * kGatherWarps;
-constexpr uint32_t kStageA = kBM * kBK * 2;     // 16 KB: this CTA's 128 rows x 64 K
-constexpr uint32_t kStageB = kBK * (kBN / 2) * 2;  // 16 KB: this CTA's 128 columns x 64 K
-constexpr uint32_t kChunkB = kBK * 64 * 2;      // 8 KB: 64 columns x 64 K
+constexpr uint32_t kAtomA = kBM * 64 * 2;       // 16 KB: 128 rows x 64 K (one swizzle atom column)
+constexpr uint32_t kStageA = kAtomA * kAtoms;   // this CTA's 128 rows x kStageK
+constexpr uint32_t kChunkB = kStageK * 64 * 2;  // 64 columns x kStageK rows of K
+constexpr uint32_t kStageB = 2 * kChunkB;       // this CTA's 128 columns x kStageK
 constexpr uint32_t kStageBytes = kStageA + kStageB;
 constexpr uint32_t kTmemCols = 2 * kBN;         // two accumulators
 constexpr uint32_t kNumBars = 3 * kPairStages + 5;
@@ -144,9 +152,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kPairStages; ++s) {
-            // even CTA: producer's arrive (+ both CTAs' TMA bytes), plus the odd
-            // CTA's relay in the up GEMM
-            mbar_init(full_bar(s), 1 + (kUp ? 1 : 0));
+            // even CTA: producer's arrive (+ both CTAs' TMA bytes); in the up GEMM
+            // also its own gather threads' cp.async arrivals and the odd CTA's relay
+            mbar_init(full_bar(s), 1 + (kUp ? 1 + kGatherThreads : 0));
             mbar_init(empty_bar(s), 1);
             mbar_init(gfull_bar(s), kGatherThreads);
         }
@@ -178,7 +186,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
     volatile uint32_t *abort = &misc[1];
     const int n_tiles = a.n_tiles;
     const int total_tiles = tile_off_s[E] * n_tiles;
-    const int nk = a.k_dim / kBK;
+    const int nk = (a.k_dim + kStageK - 1) / kStageK;   // K % kStageK is 0 or 64
+    const int last_mmas = (a.k_dim % kStageK) ? (a.k_dim % kStageK) / kUmmaK : kStageK / kUmmaK;
     const int cluster = blockIdx.x >> 1;
     const int n_clusters = gridDim.x >> 1;
     const int row0 = (int)rank * kBM;  // this CTA's first row inside a tile
@@ -201,9 +210,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                     }
                     if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), kTxBytes);
                     const uint32_t fb = mapa_shared(full_bar(stage), 0);
-                    const int k0 = kb * kBK;
+                    const int k0 = kb * kStageK;
                     const uint32_t b_dst = sB + stage * kStageB;
-                    if (!kUp) tma_load_2d_pair(sA + stage * kStageA, &a.tmap_a, fb, k0, t.m0 + row0);
+                    if (!kUp) tma_load_3d_pair(sA + stage * kStageA, &a.tmap_a, fb, 0, t.m0 + row0, k0 / 64);
                     if (kUp && a.layout == MOE_LAYOUT_CONCATENATED)
                         tma_load_4d_pair(b_dst, &a.tmap_b, fb, 0, brow0 + k0, t.nt * 2, (int)rank);
                     else
@@ -239,19 +248,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + acc * kBN;
                     for (int kb = 0; kb < nk; ++kb) {
-                        if (!mbar_wait_bounded(full_bar(stage), phase, abort) ||
-                            (kUp && !mbar_wait_bounded(gfull_bar(stage), phase, abort))) {
+                        // one barrier per stage: every wait here is on the MMA's critical path
+                        if (!mbar_wait_bounded(full_bar(stage), phase, abort)) {
                             ok = false;
                             break;
                         }
-                        if (kUp) fence_proxy_async_smem();
                         tc_fence_after();
                         const uint32_t a_addr = sA + stage * kStageA;
                         const uint32_t b_addr = sB + stage * kStageB;
 #pragma unroll
-                        for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-                            // A: K-major, 128-byte rows, 8-row atoms 1024 B apart; K step 32 B.
-                            const uint64_t adesc = smem_desc_sw128(a_addr + kk * (kUmmaK * 2), 16, 1024);
+                        for (int kk = 0; kk < kStageK / kUmmaK; ++kk) {
+                            if (kb == nk - 1 && kk >= last_mmas) break;  // K tail of 64
+                            // A: K-major, 128-byte rows, 8-row atoms 1024 B apart, 64-wide K
+                            // atoms 16 KB apart; K step 32 B inside an atom.
+                            const uint64_t adesc = smem_desc_sw128(
+                                a_addr + (kk >> 2) * kAtomA + (kk & 3) * (kUmmaK * 2), 16, 1024);
                             // B: N-major, 64-column chunks 8 KB apart (LBO), 8-row K atoms
                             // 1024 B apart (SBO); K step = 16 rows = 2 KB.
                             const uint64_t bdesc =
@@ -478,13 +489,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                     break;
                 }
                 const uint32_t a_dst = sA + stage * kStageA;
-                const size_t koff = (size_t)kb * kBK * 2;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int rr = r0 + 16 * i;
-                    cp_async_16(a_dst + rr * 128 + ((chunk ^ (rr & 7)) << 4), src[i] + koff);
+                for (int at = 0; at < kAtoms; ++at) {
+                    const int k0 = kb * kStageK + at * 64;
+                    if (k0 >= a.k_dim) break;  // K tail of 64: that atom is not multiplied
+                    const size_t koff = (size_t)k0 * 2;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int rr = r0 + 16 * i;
+                        cp_async_16(a_dst + at * kAtomA + rr * 128 + ((chunk ^ (rr & 7)) << 4), src[i] + koff);
+                    }
                 }
-                cp_async_arrive_noinc(gfull_bar(stage));
+                // even CTA: straight onto the stage barrier the MMA waits on; odd
+                // CTA: onto gfull, which its relay forwards to the even CTA
+                cp_async_arrive_noinc(rank == 0 ? full_bar(stage) : gfull_bar(stage));
                 if (++stage == kPairStages) {
                     stage = 0;
                     phase ^= 1u;
