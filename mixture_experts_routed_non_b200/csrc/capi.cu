@@ -180,14 +180,16 @@ bool make_map_b_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// h [rows][I] viewed as (64 columns, rows, I/64 column chunks): one box of
-// 64 x 128 rows x (stage K / 64) is one CTA's A stage, 64-wide K atoms 16 KB apart.
-bool make_map_a_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t rows) {
+// h [rows][I] viewed as (64 columns, rows, I/64 column chunks): a box of
+// 64 x 128 rows x (stage K / 64) is one CTA's A stage (64-wide K atoms 16 KB
+// apart); a box of 64 x 16 rows x 1 is one 16-row group of one atom.
+bool make_map_a_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t rows, uint32_t box_rows,
+                       uint32_t box_atoms) {
     EncodeTiledFn f = encode_fn();
     if (!f) return false;
     cuuint64_t dims[3] = {64, rows, ncols / 64};
     cuuint64_t strides[2] = {ncols * 2, 128};
-    cuuint32_t box[3] = {64, (cuuint32_t)kBM, (cuuint32_t)(kGemmStageK / 64)};
+    cuuint32_t box[3] = {64, box_rows, box_atoms};
     cuuint32_t estr[3] = {1, 1, 1};
     return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -321,7 +323,9 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
         // ---- down: h . w2 -> y
         GemmArgs dn;
         memset(&dn, 0, sizeof dn);
-        if (!make_map_a_chunks(&dn.tmap_a, hbuf, (uint64_t)I, (uint64_t)l.p_cap)) return MOE_ERR_CUDA;
+        if (!make_map_a_chunks(&dn.tmap_a, hbuf, (uint64_t)I, (uint64_t)l.p_cap, kBM, kGemmStageK / 64))
+            return MOE_ERR_CUDA;
+        if (!make_map_a_chunks(&dn.tmap_a16, hbuf, (uint64_t)I, (uint64_t)l.p_cap, 16, 1)) return MOE_ERR_CUDA;
         if (!make_map_b_chunks(&dn.tmap_b, w2, (uint64_t)H, (uint64_t)E * I)) return MOE_ERR_CUDA;
         if (!make_map_2d(&dn.tmap_out, ybuf, (uint64_t)H, (uint64_t)l.p_cap, 64, 32)) return MOE_ERR_CUDA;
         dn.expert_off = meta.expert_frequency_offset;

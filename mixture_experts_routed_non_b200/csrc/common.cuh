@@ -73,6 +73,7 @@ struct GemmArgs {
     CUtensorMap tmap_b;       // w1 / w2 viewed as (64 columns, K rows, column chunk[, half]):
                               // one box = this CTA's 64 x 128 half of a B stage
     CUtensorMap tmap_out;     // h [P_cap,I] / y [P_cap,H], box 64 columns x 32 rows (stores)
+    CUtensorMap tmap_a16;     // down: h as (64, rows, I/64), box 64 x 16 rows x 1 (short segments)
     const __nv_bfloat16 *x;   // up: x [N,H], rows gathered with cp.async
     const int32_t *x_gather_idx;
     const int32_t *expert_off;    // [E+1]

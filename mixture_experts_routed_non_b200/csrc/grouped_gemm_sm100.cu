@@ -194,7 +194,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
-        constexpr uint32_t kTxBytes = 2 * (kUp ? kStageB : kStageBytes);  // both CTAs' TMA bytes
+        // A rows of one CTA in the down GEMM: a full 128-row box, or, for a short
+        // segment, only its 16-row groups (rows past the segment end are never
+        // stored, so they need no data)
+        auto a_groups = [&](const Tile &tt, int r) {
+            const int v = min(max(tt.m_end - (tt.m0 + r * kBM), 0), kBM);
+            const int g = (v + 15) / 16;
+            return g >= 6 ? 8 : g;  // 8 = one full box
+        };
+        auto a_bytes = [&](int groups) { return (uint32_t)groups * 16 * 128 * kAtoms; };
         int stage = 0;
         uint32_t phase = 0;
         uint32_t issued = 0, issued_parity = 0;
@@ -202,17 +210,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
             for (int tile = cluster; tile < total_tiles; tile += n_clusters) {
                 const Tile t = decode_tile(tile, n_tiles, E, tile_off_s, off_s);
                 const int brow0 = t.e * a.k_dim;
+                const int ga0 = kUp ? 0 : a_groups(t, 0), ga1 = kUp ? 0 : a_groups(t, 1);
+                const int ga_mine = rank == 0 ? ga0 : ga1;
                 bool ok = true;
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort)) {
                         ok = false;
                         break;
                     }
-                    if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), kTxBytes);
+                    // both CTAs' TMA bytes land on the even CTA's barrier
+                    if (rank == 0)
+                        mbar_arrive_expect_tx(full_bar(stage),
+                                              2 * kStageB + (kUp ? 0u : a_bytes(ga0) + a_bytes(ga1)));
                     const uint32_t fb = mapa_shared(full_bar(stage), 0);
                     const int k0 = kb * kStageK;
                     const uint32_t b_dst = sB + stage * kStageB;
-                    if (!kUp) tma_load_3d_pair(sA + stage * kStageA, &a.tmap_a, fb, 0, t.m0 + row0, k0 / 64);
+                    if (!kUp) {
+                        const uint32_t a_dst = sA + stage * kStageA;
+                        if (ga_mine == 8) {
+                            tma_load_3d_pair(a_dst, &a.tmap_a, fb, 0, t.m0 + row0, k0 / 64);
+                        } else {
+                            for (int g = 0; g < ga_mine; ++g)
+#pragma unroll
+                                for (int at = 0; at < kAtoms; ++at)
+                                    tma_load_3d_pair(a_dst + at * kAtomA + g * 16 * 128, &a.tmap_a16, fb, 0,
+                                                     t.m0 + row0 + 16 * g, k0 / 64 + at);
+                        }
+                    }
                     if (kUp && a.layout == MOE_LAYOUT_CONCATENATED)
                         tma_load_4d_pair(b_dst, &a.tmap_b, fb, 0, brow0 + k0, t.nt * 2, (int)rank);
                     else
@@ -497,7 +521,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
                         const int rr = r0 + 16 * i;
-                        cp_async_16(a_dst + at * kAtomA + rr * 128 + ((chunk ^ (rr & 7)) << 4), src[i] + koff);
+                        // rows past the segment end are never stored: skip their copies
+                        // (the stage keeps stale data there, which only feeds those rows)
+                        if (t.m0 + row0 + rr < t.m_end)
+                            cp_async_16(a_dst + at * kAtomA + rr * 128 + ((chunk ^ (rr & 7)) << 4),
+                                        src[i] + koff);
                     }
                 }
                 // even CTA: straight onto the stage barrier the MMA waits on; odd
