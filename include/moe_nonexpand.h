@@ -234,6 +234,18 @@ MOE_API int moe_nonexpand_workspace_layout(int64_t N, int32_t H, int32_t I, int3
  */
 MOE_API int moe_nonexpand_read_error(const void *ws, moe_stream_t stream, uint32_t *err_word);
 
+/*
+ * Self-test of the device failure path (no counterpart on the pages): launches
+ * one bounded pipeline wait that nothing completes, with a limit of
+ * `timeout_us` microseconds (1 .. 2,000,000).  When the wait gives up, the
+ * kernel records MOE_DEVERR_TIMEOUT in the error word of `ws` (cleared first)
+ * and returns; read it with moe_nonexpand_read_error.  The GEMM kernels take
+ * the same path, with a 4 s limit, if a pipeline stage never completes.  Only
+ * the 256-byte header of `ws` is used.
+ */
+MOE_API int moe_nonexpand_selftest_wait_timeout(void *ws, size_t ws_bytes, uint32_t timeout_us,
+                                        moe_stream_t stream);
+
 /* Static string for a MOE_OK / MOE_ERR_* code. */
 MOE_API const char *moe_nonexpand_strerror(int status);
 

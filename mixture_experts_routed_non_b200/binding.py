@@ -43,6 +43,7 @@ EXPORTED = (
     "moe_nonexpand_read_error",
     "moe_nonexpand_strerror",
     "moe_nonexpand_metadata_noalloc",
+    "moe_nonexpand_selftest_wait_timeout",
 )
 
 
@@ -96,6 +97,8 @@ def load() -> ctypes.CDLL:
     lib.moe_nonexpand_read_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
     lib.moe_nonexpand_metadata_noalloc.restype = ctypes.c_int
     lib.moe_nonexpand_metadata_noalloc.argtypes = [P, P, i64, i32, i32, i64, ctypes.POINTER(MoeMeta), P]
+    lib.moe_nonexpand_selftest_wait_timeout.restype = ctypes.c_int
+    lib.moe_nonexpand_selftest_wait_timeout.argtypes = [P, sz, ctypes.c_uint32, P]
     lib.moe_nonexpand_strerror.restype = ctypes.c_char_p
     lib.moe_nonexpand_strerror.argtypes = [ctypes.c_int]
     _lib = lib
@@ -317,6 +320,15 @@ def combine(y: torch.Tensor, meta: dict, N: int, out: Optional[torch.Tensor] = N
     _check(load().moe_nonexpand_combine(y.data_ptr(), ctypes.byref(m), N, H, out.data_ptr(),
                                         _stream_handle(stream)), "moe_nonexpand_combine")
     return out
+
+
+def selftest_wait_timeout(ws: torch.Tensor, timeout_us: int,
+                          stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Run one bounded device wait that nothing completes (limit timeout_us);
+    afterwards read_error(ws) reports DEVERR_TIMEOUT."""
+    _check(load().moe_nonexpand_selftest_wait_timeout(ws.data_ptr(), ws.numel(), timeout_us,
+                                                      _stream_handle(stream)),
+           "moe_nonexpand_selftest_wait_timeout")
 
 
 def read_error(ws: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:
