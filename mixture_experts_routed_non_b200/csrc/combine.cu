@@ -9,9 +9,13 @@
 // fp32; the sum is rounded once to bf16.  The result is deterministic and
 // independent of the launch shape.
 //
-// One thread owns 8 consecutive columns (one 16-byte vector) of one token;
-// the K row reads of a token are issued four at a time before accumulating,
-// to keep several HBM requests in flight per thread.
+// A block owns up to kTokPerBlock consecutive tokens.  Their token offsets and
+// the row index and score of every one of their pairs (a contiguous q range)
+// are loaded into shared memory once, with coalesced loads; then each thread
+// owns 16-byte column chunks and walks the block's pairs in batches of eight
+// rows whose loads are all issued before any is accumulated -- across token
+// boundaries, so the loads in flight do not depend on how many pairs each
+// token has -- and no per-element index chain remains.
 #include "common.cuh"
 
 namespace moe {
@@ -19,6 +23,8 @@ namespace moe {
 namespace {
 
 constexpr int kCombineThreads = 256;
+constexpr int kTokPerBlock = 8;
+constexpr int kMaxK = 32;
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
     uint4 v;
@@ -39,47 +45,71 @@ __device__ __forceinline__ void fma8(float (&acc)[8], float w, const uint4 &v) {
     acc[7] = fmaf(w, bf16hi(v.w), acc[7]);
 }
 
+__device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    return o;
+}
+
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
     const __nv_bfloat16 *__restrict__ y, const int32_t *__restrict__ token_offset,
     const int32_t *__restrict__ s_rev, const float *__restrict__ scores, int64_t N, int32_t H,
-    __nv_bfloat16 *__restrict__ out, const WsHeader *hdr) {
+    __nv_bfloat16 *__restrict__ out, const WsHeader *hdr, int tok_per_block) {
+    __shared__ int s_off[kTokPerBlock + 1];
+    __shared__ int s_p[kTokPerBlock * kMaxK];
+    __shared__ float s_w[kTokPerBlock * kMaxK];
     if (hdr && *(volatile const uint32_t *)&hdr->abort) return;
     const int chunks = H >> 3;
-    const int64_t total = N * chunks;
-    for (int64_t i = (int64_t)blockIdx.x * kCombineThreads + threadIdx.x; i < total;
-         i += (int64_t)gridDim.x * kCombineThreads) {
-        const int64_t t = i / chunks;
-        const int c = (int)(i - t * chunks);
-        const int q0 = __ldg(token_offset + t);
-        const int q1 = __ldg(token_offset + t + 1);
-        const __nv_bfloat16 *ycol = y + (size_t)c * 8;
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        int q = q0;
-        for (; q + 4 <= q1; q += 4) {
-            int p[4];
-            float w[4];
-            uint4 v[4];
+    const int64_t n_groups = (N + tok_per_block - 1) / tok_per_block;
+    for (int64_t grp = blockIdx.x; grp < n_groups; grp += gridDim.x) {
+        const int64_t t0 = grp * tok_per_block;
+        const int nt = (int)min((int64_t)tok_per_block, N - t0);
+        if (threadIdx.x <= nt) s_off[threadIdx.x] = __ldg(token_offset + t0 + threadIdx.x);
+        __syncthreads();
+        const int qa = s_off[0];
+        const int np = s_off[nt] - qa;  // pairs of the block's tokens, a contiguous q range
+        for (int i = threadIdx.x; i < np; i += kCombineThreads) {
+            s_p[i] = __ldg(s_rev + qa + i);
+            s_w[i] = __ldg(scores + qa + i);
+        }
+        __syncthreads();
+        for (int c = threadIdx.x; c < chunks; c += kCombineThreads) {
+            const __nv_bfloat16 *ycol = y + (size_t)c * 8;
+            __nv_bfloat16 *ocol = out + (size_t)t0 * H + (size_t)c * 8;
+            // walk the block's pairs in batches of 8 rows in flight, across token
+            // boundaries; each token's pairs are still summed in q order
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            int j = 0;                       // current token (block-local)
+            int tok_end = s_off[1] - qa;     // its pairs end here
+            for (int base = 0; base < np; base += 8) {
+                uint4 v[8];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                p[j] = __ldg(s_rev + q + j);
-                w[j] = __ldg(scores + q + j);
+                for (int u = 0; u < 8; ++u)
+                    v[u] = (base + u < np) ? ld_stream_v4(ycol + (size_t)s_p[base + u] * H) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int q = base + u;
+                    if (q >= np) break;
+                    while (q >= tok_end) {  // finish token j (and any token without pairs)
+                        *reinterpret_cast<uint4 *>(ocol + (size_t)j * H) = pack8(acc);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+                        ++j;
+                        tok_end = s_off[j + 1] - qa;
+                    }
+                    fma8(acc, s_w[q], v[u]);
+                }
             }
+            for (; j < nt; ++j) {  // the last token with pairs, then trailing tokens without
+                *reinterpret_cast<uint4 *>(ocol + (size_t)j * H) = pack8(acc);
 #pragma unroll
-            for (int j = 0; j < 4; ++j) v[j] = ld_stream_v4(ycol + (size_t)p[j] * H);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) fma8(acc, w[j], v[j]);
+                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+            }
         }
-        for (; q < q1; ++q) {
-            const int p = __ldg(s_rev + q);
-            const float w = __ldg(scores + q);
-            fma8(acc, w, ld_stream_v4(ycol + (size_t)p * H));
-        }
-        uint4 o;
-        o.x = pack_bf16x2(acc[0], acc[1]);
-        o.y = pack_bf16x2(acc[2], acc[3]);
-        o.z = pack_bf16x2(acc[4], acc[5]);
-        o.w = pack_bf16x2(acc[6], acc[7]);
-        *reinterpret_cast<uint4 *>(out + (size_t)t * H + (size_t)c * 8) = o;
+        __syncthreads();  // shared indices are reused by the next group
     }
 }
 
@@ -88,13 +118,18 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
 cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *token_offset, const int32_t *s_rev,
                            const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
                            const WsHeader *hdr, int num_sms, cudaStream_t s) {
-    const int64_t total = N * (H / 8);
-    if (total == 0) return cudaSuccess;
-    int64_t blocks = (total + kCombineThreads - 1) / kCombineThreads;
-    const int64_t cap = (int64_t)num_sms * 8;
+    if (N == 0) return cudaSuccess;
+    // tokens per block: up to kTokPerBlock, fewer when that would leave SMs idle
+    const int64_t chunks = H / 8;
+    int64_t tpb = (N * chunks) / ((int64_t)num_sms * 4 * kCombineThreads);
+    if (tpb < 1) tpb = 1;
+    if (tpb > kTokPerBlock) tpb = kTokPerBlock;
+    const int64_t groups = (N + tpb - 1) / tpb;
+    int64_t blocks = groups;
+    const int64_t cap = (int64_t)num_sms * 16;
     if (blocks > cap) blocks = cap;
-    combine_kernel<<<(unsigned)blocks, kCombineThreads, 0, s>>>(y, token_offset, s_rev, scores, N, H, out,
-                                                                 hdr);
+    combine_kernel<<<(unsigned)blocks, kCombineThreads, 0, s>>>(y, token_offset, s_rev, scores, N, H, out, hdr,
+                                                                 (int)tpb);
     return cudaGetLastError();
 }
 
