@@ -16,7 +16,7 @@ namespace moe {
 // Workspace header (first 256 bytes of the workspace).
 // ---------------------------------------------------------------------------
 struct WsHeader {
-    uint32_t reserved;
+    uint32_t grid_arrive;  // metadata kernel's grid barrier: CTAs arrived (cleared per call)
     uint32_t err;      // MOE_DEVERR_* bits of the current call
     int32_t P;         // pairs counted on the device
     uint32_t abort;    // nonzero: later kernels of this call skip their work
@@ -37,7 +37,10 @@ constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
 constexpr int kStages = 4;      // shared-memory pipeline depth (4 x 48 KB)
 
 // Metadata kernels: tiles of kMetaTileUnit * c slots, at most kMetaMaxTiles tiles.
-constexpr int kMetaTileUnit = 4096;
+#ifndef MOE_META_TILE_UNIT
+#define MOE_META_TILE_UNIT 1024
+#endif
+constexpr int kMetaTileUnit = MOE_META_TILE_UNIT;
 constexpr int kMetaMaxTiles = 148;
 constexpr int kMetaThreads = 512;
 constexpr int kMetaWarps = kMetaThreads / 32;

@@ -5,24 +5,27 @@
 // s_reverse_scatter_idx, num_activated_expert_per_token_offset, compact
 // router_scores -- and question 3: pairs are numbered in ascending token
 // order).  The sort by expert is a stable counting sort (the segmented-sort
-// recipe of the qwen3_5.py commit notes, steps 1-2), in two kernels over T
-// tiles of consecutive slots (T <= number of SMs):
+// recipe of the qwen3_5.py commit notes, steps 1-2) done by one cooperative
+// kernel over T tiles of consecutive slots (T <= number of SMs, one CTA each):
 //
-//   meta_count_kernel    per tile: expert histogram in shared memory (match_any
-//                        aggregation) and valid-slot count -> hist[T][E].
-//   meta_scatter_kernel  per tile: reads the whole (small) hist table and
-//                        derives, with no inter-block waiting, the global
-//                        offsets, this tile's base per expert and its pair base;
-//                        then each warp ranks its own contiguous slice (per-warp
-//                        counts, then popc(peers & lanes below) inside each
-//                        32-slot step) and writes the outputs.  Block 0 also
-//                        writes the histogram, offsets, the GEMM tile table and
-//                        the call's error word.
+//   phase A  each warp of a tile owns a contiguous slice of its slots and
+//            counts the experts in it (match_any aggregation, per-warp rows
+//            in shared memory, no atomics); the tile's histogram, valid count
+//            and error bits go to the workspace.
+//   barrier  all T CTAs (co-resident by the cooperative launch) meet at a
+//            bounded grid barrier whose counter the host clears per call.
+//   phase B  every CTA reads the whole (small) [T,E] histogram table and
+//            derives the global offsets, its tile's base per expert and its
+//            pair base; its warps' bases follow from the per-warp counts of
+//            phase A; then each warp ranks its slice (popc(peers & lanes
+//            below) inside each 32-slot step) and writes the outputs.  CTA 0
+//            also writes the histogram, offsets, the GEMM tile table and the
+//            call's error word.
 //
 // Every result is a pure function of the input (no atomic decides an order),
 // so the output is bit-exact and deterministic.  Each lane keeps kV slots in
-// flight (all loads issued before use) so that a warp pays one memory latency
-// per 32*kV slots.
+// flight; the first kWarpChunk slots of every warp, and their weights, stay in
+// registers from phase A to phase B.
 #include "common.cuh"
 
 namespace moe {
@@ -32,6 +35,7 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kV = 8;                     // slots per lane per step
 constexpr int kWarpChunk = 32 * kV;       // slots per warp step
+constexpr unsigned long long kGridBarrierTimeoutNs = 1000000000ull;
 
 // Exclusive scan of n ints in shared memory (in place allowed) by the whole
 // block; returns the total.
@@ -94,66 +98,111 @@ __device__ __forceinline__ void load_chunk(const int32_t *idx, int base, int end
     }
 }
 
-__global__ void __launch_bounds__(kMetaThreads) meta_count_kernel(const MetaArgs a) {
-    extern __shared__ int hist[];  // [E]
-    __shared__ int s_valid;
-    __shared__ unsigned s_err;
-    const int E = a.E;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int e = threadIdx.x; e < E; e += kMetaThreads) hist[e] = 0;
-    if (threadIdx.x == 0) {
-        s_valid = 0;
-        s_err = 0;
-    }
-    __syncthreads();
+// Shared memory (ints): cnt[kMetaWarps][E] | part_all[kPartInts] | part_before[kPartInts]
+//                       | off[kMaxExperts+1] | gt[kMaxExperts+1]
+constexpr int kPartInts = kMaxExperts;   // G*E <= max(kMetaThreads, E) <= kMaxExperts
 
+__global__ void __launch_bounds__(kMetaThreads) meta_kernel(const MetaArgs a) {
+    extern __shared__ int sm[];
+    const int E = a.E, K = a.K, T = a.tiles;
+    int *cnt = sm;
+    int *part_all = cnt + kMetaWarps * E;
+    int *part_before = part_all + kPartInts;
+    int *off = part_before + kPartInts;
+    int *gt = off + (kMaxExperts + 1);
+    __shared__ int wq[kMetaWarps];
+    __shared__ unsigned s_err;
+    __shared__ int s_bar_ok;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = lanemask_lt();
     const int tile = blockIdx.x;
+
+    // this warp's contiguous slice of the tile
     const int s0 = tile * a.tile_slots;
     const int s1 = (int)min((int64_t)s0 + a.tile_slots, a.NK);
-    int my_valid = 0;
+    const int sub = a.tile_slots / kMetaWarps;
+    const int w0 = s0 + warp * sub;
+    const int w1 = min(w0 + sub, s1);
+    int ev0[kV];
+    load_chunk(a.topk_idx, w0, w1, lane, ev0);
+    for (int i = threadIdx.x; i < kMetaWarps * E; i += kMetaThreads) cnt[i] = 0;
+    if (threadIdx.x == 0) s_err = 0;
+    __syncthreads();
+
+    // ---- phase A: per-warp expert counts of the slice
+    int *mycnt = cnt + warp * E;
+    int nvalid = 0;
     unsigned my_err = 0;
-    for (int base = s0 + warp * kWarpChunk; base < s1; base += kMetaWarps * kWarpChunk) {
+    for (int base = w0; base < w1; base += kWarpChunk) {
         int ev[kV];
-        load_chunk(a.topk_idx, base, s1, lane, ev);
+        if (base == w0) {
+#pragma unroll
+            for (int v = 0; v < kV; ++v) ev[v] = ev0[v];
+        } else {
+            load_chunk(a.topk_idx, base, w1, lane, ev);
+        }
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
             const int e = ev[v];
             const bool valid = (e >= 0) && (e < E);
             if (!valid && e != -1) my_err = MOE_DEVERR_BAD_EXPERT_ID;
             const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
-            if (valid && lane == __ffs(peers) - 1) atomicAdd(&hist[e], __popc(peers));
-            my_valid += __popc(__ballot_sync(kFull, valid));
+            if (valid && lane == __ffs(peers) - 1) mycnt[e] += __popc(peers);
+            nvalid += __popc(__ballot_sync(kFull, valid));
+            __syncwarp();
         }
     }
-    if (lane == 0 && my_valid) atomicAdd(&s_valid, my_valid);
+    // weights of the first chunk's valid slots, kept for phase B (invalid
+    // slots' weights are never read)
+    float wv0[kV];
+#pragma unroll
+    for (int v = 0; v < kV; ++v) {
+        const bool valid = (ev0[v] >= 0) && (ev0[v] < E);
+        wv0[v] = valid ? __ldg(a.topk_w + w0 + 32 * v + lane) : 0.f;
+    }
+    if (lane == 0) wq[warp] = nvalid;
     if (my_err) atomicOr(&s_err, my_err);
     __syncthreads();
+    // tile histogram = sum of the warps' rows
     int *th = a.tile_hist + (size_t)tile * E;
-    for (int e = threadIdx.x; e < E; e += kMetaThreads) th[e] = hist[e];
+    for (int e = threadIdx.x; e < E; e += kMetaThreads) {
+        int sum = 0;
+        for (int w = 0; w < kMetaWarps; ++w) sum += cnt[w * E + e];
+        th[e] = sum;
+    }
     if (threadIdx.x == 0) {
-        a.tile_valid[tile] = s_valid;
+        int v = 0;
+        for (int w = 0; w < kMetaWarps; ++w) v += wq[w];
+        a.tile_valid[tile] = v;
         a.tile_err[tile] = (int)s_err;
     }
-}
 
-// Shared memory of the scatter kernel (ints), after cnt[kMetaWarps][E].
-constexpr int kPartInts = kMaxExperts;   // G*E <= max(kMetaThreads, E) <= kMaxExperts
+    // ---- grid barrier (bounded)
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        atomicAdd(&a.hdr->grid_arrive, 1u);
+        const uint64_t t0 = globaltimer_ns();
+        int ok = 1;
+        while (*(volatile uint32_t *)&a.hdr->grid_arrive < (uint32_t)T) {
+            if (globaltimer_ns() - t0 > kGridBarrierTimeoutNs) {
+                ok = 0;
+                break;
+            }
+        }
+        s_bar_ok = ok;
+        __threadfence();
+    }
+    __syncthreads();
+    if (!s_bar_ok) {
+        if (threadIdx.x == 0) {
+            atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);
+            a.hdr->abort = 1u;
+        }
+        return;
+    }
 
-__global__ void __launch_bounds__(kMetaThreads) meta_scatter_kernel(const MetaArgs a) {
-    extern __shared__ int sm[];
-    const int E = a.E, K = a.K, T = a.tiles;
-    int *cnt = sm;                              // [kMetaWarps][E]
-    int *part_all = cnt + kMetaWarps * E;       // [G][E]
-    int *part_before = part_all + kPartInts;    // [G][E]
-    int *off = part_before + kPartInts;         // [E+1]
-    int *gt = off + (kMaxExperts + 1);          // [E+1]
-    __shared__ int wq[kMetaWarps];
-    __shared__ unsigned s_err;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lt = lanemask_lt();
-    const int tile = blockIdx.x;
-
-    // ---- 1. global column sums and this tile's column prefix, from hist[T][E]
+    // ---- phase B.1: global column sums and this tile's column prefix
     int G = E <= kMetaThreads ? kMetaThreads / E : 1;
     if (G > T) G = T;
     for (int i = threadIdx.x; i < G * E; i += kMetaThreads) {
@@ -175,14 +224,11 @@ __global__ void __launch_bounds__(kMetaThreads) meta_scatter_kernel(const MetaAr
         part_all[i] = all;
         part_before[i] = before;
     }
-    for (int i = threadIdx.x; i < kMetaWarps * E; i += kMetaThreads) cnt[i] = 0;
-    int tv = 0, tv_before = 0;
+    int tv_before = 0;
     unsigned terr = 0;
     for (int t = threadIdx.x; t < T; t += kMetaThreads) {
-        const int v = __ldcg(a.tile_valid + t);
-        tv += v;
-        if (t < tile) tv_before += v;
-        terr |= (unsigned)__ldcg(a.tile_err + t);
+        if (t < tile) tv_before += __ldcg(a.tile_valid + t);
+        if (tile == 0) terr |= (unsigned)__ldcg(a.tile_err + t);
     }
     if (threadIdx.x == 0) s_err = 0;
     __syncthreads();
@@ -223,31 +269,7 @@ __global__ void __launch_bounds__(kMetaThreads) meta_scatter_kernel(const MetaAr
     }
     if (abort) return;  // the pair arrays are too small for the pairs seen
 
-    // ---- 2. per-warp counts of this tile's slots
-    const int s0 = tile * a.tile_slots;
-    const int s1 = (int)min((int64_t)s0 + a.tile_slots, a.NK);
-    const int sub = a.tile_slots / kMetaWarps;
-    const int w0 = s0 + warp * sub;
-    const int w1 = min(w0 + sub, s1);
-    int *mycnt = cnt + warp * E;
-    int nvalid = 0;
-    for (int base = w0; base < w1; base += kWarpChunk) {
-        int ev[kV];
-        load_chunk(a.topk_idx, base, w1, lane, ev);
-#pragma unroll
-        for (int v = 0; v < kV; ++v) {
-            const int e = ev[v];
-            const bool valid = (e >= 0) && (e < E);
-            const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
-            if (valid && lane == __ffs(peers) - 1) mycnt[e] += __popc(peers);
-            nvalid += __popc(__ballot_sync(kFull, valid));
-            __syncwarp();
-        }
-    }
-    if (lane == 0) wq[warp] = nvalid;
-    __syncthreads();
-
-    // ---- 3. bases: global offset + earlier tiles + earlier warps of this tile
+    // ---- phase B.2: bases: global offset + earlier tiles + earlier warps
     for (int e = threadIdx.x; e < E; e += kMetaThreads) {
         int run = off[e] + part_before[e];
         for (int w = 0; w < kMetaWarps; ++w) {
@@ -266,17 +288,25 @@ __global__ void __launch_bounds__(kMetaThreads) meta_scatter_kernel(const MetaAr
     }
     __syncthreads();
 
-    // ---- 4. positions, in slot order
+    // ---- phase B.3: positions, in slot order
     int q_run = wq[warp];
     for (int base = w0; base < w1; base += kWarpChunk) {
         int ev[kV];
         float wv[kV];
-        load_chunk(a.topk_idx, base, w1, lane, ev);
+        if (base == w0) {
 #pragma unroll
-        for (int v = 0; v < kV; ++v) {
-            const int s = base + 32 * v + lane;
-            const bool valid = (ev[v] >= 0) && (ev[v] < E);
-            wv[v] = valid ? __ldg(a.topk_w + s) : 0.f;  // invalid slots' weights are never read
+            for (int v = 0; v < kV; ++v) {
+                ev[v] = ev0[v];
+                wv[v] = wv0[v];
+            }
+        } else {
+            load_chunk(a.topk_idx, base, w1, lane, ev);
+#pragma unroll
+            for (int v = 0; v < kV; ++v) {
+                const int s = base + 32 * v + lane;
+                const bool valid = (ev[v] >= 0) && (ev[v] < E);
+                wv[v] = valid ? __ldg(a.topk_w + s) : 0.f;
+            }
         }
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
@@ -305,7 +335,7 @@ __global__ void __launch_bounds__(kMetaThreads) meta_scatter_kernel(const MetaAr
 
 }  // namespace
 
-size_t meta_scatter_smem_bytes(int E) {
+size_t meta_smem_bytes(int E) {
     return ((size_t)kMetaWarps * E + 2 * kPartInts + 2 * (kMaxExperts + 1)) * sizeof(int);
 }
 
@@ -315,16 +345,19 @@ cudaError_t launch_meta(const MetaArgs &a, cudaStream_t s) {
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev < 64 && !configured[dev]) {
-        err = cudaFuncSetAttribute(meta_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)meta_scatter_smem_bytes(kMaxExperts));
+        err = cudaFuncSetAttribute(meta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)meta_smem_bytes(kMaxExperts));
         if (err != cudaSuccess) return err;
         configured[dev] = true;
     }
-    meta_count_kernel<<<a.tiles, kMetaThreads, a.E * sizeof(int), s>>>(a);
-    err = cudaGetLastError();
+    // the grid barrier's arrival counter starts from zero in every call
+    err = cudaMemsetAsync(&a.hdr->grid_arrive, 0, sizeof(a.hdr->grid_arrive), s);
     if (err != cudaSuccess) return err;
-    meta_scatter_kernel<<<a.tiles, kMetaThreads, meta_scatter_smem_bytes(a.E), s>>>(a);
-    return cudaGetLastError();
+    MetaArgs args = a;
+    void *params[] = {&args};
+    // cooperative: all T CTAs are resident at once, so the grid barrier ends
+    return cudaLaunchCooperativeKernel((const void *)meta_kernel, dim3(a.tiles), dim3(kMetaThreads), params,
+                                       meta_smem_bytes(a.E), s);
 }
 
 }  // namespace moe

@@ -29,7 +29,7 @@ struct ScratchLayout {
     int32_t tiles, tile_slots;
 };
 
-// Tiles of 4096 * c slots, at most 148 of them (the same rule the workspace
+// Tiles of kMetaTileUnit * c slots, at most 148 of them (the same rule the workspace
 // path uses).
 ScratchLayout scratch_layout(int64_t NK, int32_t E) {
     ScratchLayout l;

@@ -72,7 +72,7 @@ def test_workspace_layout_is_consistent(lib):
         if args[1]:
             assert lay.h % 1024 == 0 and lay.y % 1024 == 0
             assert lay.y > lay.h if lay.p_cap > 0 else lay.y == lay.h
-        assert lay.meta_tile_slots % 4096 == 0 and lay.meta_tiles <= 148
+        assert lay.meta_tile_slots % 1024 == 0 and lay.meta_tiles <= 148
         assert lay.meta_tiles * lay.meta_tile_slots >= args[0] * args[4]
 
 
