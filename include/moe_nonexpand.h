@@ -79,6 +79,8 @@ extern "C" {
 #define MOE_DEVERR_PAIR_COUNT 0x2u    /* counted P != total_pairs (total_pairs >= 0) or P > P_cap */
 #define MOE_DEVERR_TIMEOUT 0x4u       /* an internal pipeline wait gave up; outputs are invalid */
 #define MOE_DEVERR_ABORTED 0x8u       /* P > P_cap: GEMMs and combine were skipped, out unwritten */
+#define MOE_DEVERR_BAD_TOKEN 0x10u    /* pair list: a token id outside [0,N) (that pair was skipped)
+                                         or token ids not in ascending order (offsets unspecified) */
 
 /* activation argument */
 #define MOE_ACT_SWIGLU 0
@@ -205,6 +207,60 @@ MOE_API int moe_nonexpand_forward_timed(const void *x, const int32_t *topk_idx, 
  */
 MOE_API int moe_nonexpand_combine(const void *y, const moe_meta_t *meta, int64_t N, int32_t H,
                           void *out, moe_stream_t stream);
+
+/*
+ * Routing input in either of two layouts, for the moe_nonexpand_routed_* calls.
+ *
+ *   MOE_ROUTING_TOPK   the non-expand table of sonic-moe issue #68:
+ *                      expert_idx = topk_idx [N,K] (-1 = invalid slot),
+ *                      weights = topk_w [N,K], token_idx = NULL, K slots per
+ *                      token, pairs = total_pairs (>= 0) or -1 when unknown.
+ *   MOE_ROUTING_PAIRS  the compact pair list of sonic-moe's general routing API
+ *                      (issue #68: token_indices / expert_indices /
+ *                      router_scores [P], one entry per (token, expert) pair):
+ *                      token_idx = token_indices [P], ascending, each in
+ *                      [0,N); expert_idx = expert_indices [P]; weights =
+ *                      router_scores [P]; pairs = P; K is ignored.  Pair q of
+ *                      the metadata is the q-th entry that is kept.
+ *
+ * index_dtype gives the dtype of expert_idx and token_idx (int32 or int64;
+ * int64 ids outside the int32 range are invalid).  An expert id outside
+ * [0,E) other than -1 sets MOE_DEVERR_BAD_EXPERT_ID and a token id outside
+ * [0,N) sets MOE_DEVERR_BAD_TOKEN; either way that entry is skipped.  A pair
+ * list whose tokens are not ascending sets MOE_DEVERR_BAD_TOKEN and leaves
+ * token_offset unspecified.  All arrays are device memory, caller-owned.
+ */
+#define MOE_ROUTING_TOPK 0
+#define MOE_ROUTING_PAIRS 1
+#define MOE_INDEX_INT32 0
+#define MOE_INDEX_INT64 1
+
+typedef struct moe_routing_t {
+    int32_t kind;              /* MOE_ROUTING_TOPK or MOE_ROUTING_PAIRS */
+    int32_t index_dtype;       /* MOE_INDEX_INT32 or MOE_INDEX_INT64 */
+    int64_t N;                 /* tokens: rows of x and out */
+    int32_t K;                 /* TOPK: slots per token (1..32); PAIRS: ignored */
+    int64_t pairs;             /* TOPK: total_pairs or -1; PAIRS: P >= 0 */
+    const void *expert_idx;    /* TOPK: [N,K]; PAIRS: [P] */
+    const float *weights;      /* TOPK: [N,K]; PAIRS: [P] */
+    const void *token_idx;     /* PAIRS: [P] ascending; TOPK: NULL */
+} moe_routing_t;
+
+/* Workspace bytes for a routed call (H = I = 0: metadata only); 0 = invalid. */
+MOE_API size_t moe_nonexpand_routed_workspace_bytes(const moe_routing_t *routing, int32_t H, int32_t I,
+                                                    int32_t E);
+
+/* moe_nonexpand_metadata for either routing layout (P_cap = pairs for a pair
+ * list, as for the table). */
+MOE_API int moe_nonexpand_routed_metadata(const moe_routing_t *routing, int32_t E, const moe_meta_t *meta,
+                                  void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_nonexpand_forward for either routing layout: out[t,:] sums, in pair
+ * order, the score-weighted expert rows of the pairs of token t. */
+MOE_API int moe_nonexpand_routed_forward(const void *x, const moe_routing_t *routing, int32_t H, int32_t I,
+                                 int32_t E, const void *w1, const void *b1, const void *w2, const void *b2,
+                                 int32_t activation, int32_t gate_up_layout, void *out,
+                                 const moe_meta_t *meta_out, void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* Byte offsets of the workspace's internal arrays (for inspection and tests).
  * Offsets of arrays that the given sizes do not need are 0. */

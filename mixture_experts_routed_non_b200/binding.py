@@ -28,6 +28,12 @@ DEVERR_BAD_EXPERT_ID = 0x1
 DEVERR_PAIR_COUNT = 0x2
 DEVERR_TIMEOUT = 0x4
 DEVERR_ABORTED = 0x8
+DEVERR_BAD_TOKEN = 0x10
+
+ROUTING_TOPK = 0
+ROUTING_PAIRS = 1
+INDEX_INT32 = 0
+INDEX_INT64 = 1
 
 ACT_SWIGLU = 0
 LAYOUT_INTERLEAVED = 0
@@ -44,6 +50,9 @@ EXPORTED = (
     "moe_nonexpand_strerror",
     "moe_nonexpand_metadata_noalloc",
     "moe_nonexpand_selftest_wait_timeout",
+    "moe_nonexpand_routed_workspace_bytes",
+    "moe_nonexpand_routed_metadata",
+    "moe_nonexpand_routed_forward",
 )
 
 
@@ -59,6 +68,12 @@ class WsLayout(ctypes.Structure):
         "meta_freq", "meta_off", "meta_x_gather", "meta_s_scatter", "meta_s_rev",
         "meta_token_offset", "meta_scores", "h", "y")] + [
         ("p_cap", ctypes.c_int64), ("meta_tiles", ctypes.c_int32), ("meta_tile_slots", ctypes.c_int32)]
+
+
+class MoeRouting(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("index_dtype", ctypes.c_int32), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int32), ("pairs", ctypes.c_int64), ("expert_idx", ctypes.c_void_p),
+                ("weights", ctypes.c_void_p), ("token_idx", ctypes.c_void_p)]
 
 
 class MoeError(RuntimeError):
@@ -99,6 +114,14 @@ def load() -> ctypes.CDLL:
     lib.moe_nonexpand_metadata_noalloc.argtypes = [P, P, i64, i32, i32, i64, ctypes.POINTER(MoeMeta), P]
     lib.moe_nonexpand_selftest_wait_timeout.restype = ctypes.c_int
     lib.moe_nonexpand_selftest_wait_timeout.argtypes = [P, sz, ctypes.c_uint32, P]
+    R = ctypes.POINTER(MoeRouting)
+    lib.moe_nonexpand_routed_workspace_bytes.restype = sz
+    lib.moe_nonexpand_routed_workspace_bytes.argtypes = [R, i32, i32, i32]
+    lib.moe_nonexpand_routed_metadata.restype = ctypes.c_int
+    lib.moe_nonexpand_routed_metadata.argtypes = [R, i32, ctypes.POINTER(MoeMeta), P, sz, P]
+    lib.moe_nonexpand_routed_forward.restype = ctypes.c_int
+    lib.moe_nonexpand_routed_forward.argtypes = [P, R, i32, i32, i32, P, P, P, P, i32, i32, P,
+                                                 ctypes.POINTER(MoeMeta), P, sz, P]
     lib.moe_nonexpand_strerror.restype = ctypes.c_char_p
     lib.moe_nonexpand_strerror.argtypes = [ctypes.c_int]
     _lib = lib
@@ -337,3 +360,112 @@ def read_error(ws: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> 
     _check(load().moe_nonexpand_read_error(ws.data_ptr(), _stream_handle(stream), ctypes.byref(v)),
            "moe_nonexpand_read_error")
     return int(v.value)
+
+
+# ---------------------------------------------------------------------------
+# Either routing layout, int32 or int64 ids (moe_nonexpand_routed_*)
+# ---------------------------------------------------------------------------
+
+_INDEX_DTYPES = {torch.int32: INDEX_INT32, torch.int64: INDEX_INT64}
+
+
+def routing(expert_idx: torch.Tensor, weights: torch.Tensor, *, token_idx: Optional[torch.Tensor] = None,
+            N: Optional[int] = None, total_pairs: int = -1) -> MoeRouting:
+    """The routing descriptor.  Without ``token_idx``: the non-expand table
+    (expert_idx [N,K], weights [N,K]).  With it: a compact pair list
+    (token_idx / expert_idx / weights [P], tokens ascending, N tokens)."""
+    dev = expert_idx.device
+    if expert_idx.dtype not in _INDEX_DTYPES:
+        raise TypeError(f"expert_idx: expected int32 or int64, got {expert_idx.dtype}")
+    r = MoeRouting()
+    r.index_dtype = _INDEX_DTYPES[expert_idx.dtype]
+    if token_idx is None:
+        if expert_idx.dim() != 2:
+            raise ValueError("expert_idx: expected [N,K]")
+        n, k = expert_idx.shape
+        _need(expert_idx, "expert_idx", expert_idx.dtype, (n, k), dev)
+        _need(weights, "weights", torch.float32, (n, k), dev)
+        if N is not None and N != n:
+            raise ValueError("N does not match expert_idx")
+        r.kind, r.N, r.K, r.pairs = ROUTING_TOPK, n, k, total_pairs
+        r.token_idx = None
+    else:
+        if N is None:
+            raise ValueError("a pair list needs N")
+        p = expert_idx.numel()
+        _need(expert_idx, "expert_idx", expert_idx.dtype, (p,), dev)
+        _need(token_idx, "token_idx", expert_idx.dtype, (p,), dev)
+        _need(weights, "weights", torch.float32, (p,), dev)
+        r.kind, r.N, r.K, r.pairs = ROUTING_PAIRS, N, 1, p
+        r.token_idx = token_idx.data_ptr()
+    r.expert_idx = expert_idx.data_ptr()
+    r.weights = weights.data_ptr()
+    return r
+
+
+def routing_p_cap(r: MoeRouting) -> int:
+    if r.kind == ROUTING_PAIRS:
+        return r.pairs
+    return p_cap(r.N, r.K, r.pairs)
+
+
+def routed_workspace_bytes(r: MoeRouting, H: int, I: int, E: int) -> int:
+    n = load().moe_nonexpand_routed_workspace_bytes(ctypes.byref(r), H, I, E)
+    if n == 0:
+        raise MoeError(MOE_ERR_ARG, "moe_nonexpand_routed_workspace_bytes")
+    return n
+
+
+def alloc_routed_meta(r: MoeRouting, E: int, device=None) -> dict:
+    return alloc_meta(r.N, 1, E, routing_p_cap(r), device)
+
+
+def routed_metadata(expert_idx: torch.Tensor, weights: torch.Tensor, E: int, *,
+                    token_idx: Optional[torch.Tensor] = None, N: Optional[int] = None, total_pairs: int = -1,
+                    meta: Optional[dict] = None, ws: Optional[torch.Tensor] = None,
+                    stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """moe_nonexpand_routed_metadata: the metadata of either routing layout."""
+    r = routing(expert_idx, weights, token_idx=token_idx, N=N, total_pairs=total_pairs)
+    dev = expert_idx.device
+    if meta is None:
+        meta = alloc_routed_meta(r, E, dev)
+    if ws is None:
+        ws = torch.empty(routed_workspace_bytes(r, 0, 0, E), dtype=torch.uint8, device=dev)
+    m = _meta_struct(meta)
+    _check(load().moe_nonexpand_routed_metadata(ctypes.byref(r), E, ctypes.byref(m), ws.data_ptr(), ws.numel(),
+                                                _stream_handle(stream)), "moe_nonexpand_routed_metadata")
+    return meta
+
+
+def routed_forward(x: torch.Tensor, expert_idx: torch.Tensor, weights: torch.Tensor,
+                   w1: torch.Tensor, w2: torch.Tensor, b1: Optional[torch.Tensor] = None,
+                   b2: Optional[torch.Tensor] = None, *, token_idx: Optional[torch.Tensor] = None,
+                   layout: int = LAYOUT_INTERLEAVED, total_pairs: int = -1,
+                   out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                   meta: Optional[dict] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """moe_nonexpand_routed_forward: the forward for either routing layout
+    (see ``routing``); other arguments as ``forward``."""
+    N, H = x.shape
+    E, _, I2 = w1.shape
+    I = I2 // 2
+    dev = x.device
+    _need(x, "x", torch.bfloat16, (N, H), dev)
+    _need(w1, "w1", torch.bfloat16, (E, H, 2 * I), dev)
+    _need(w2, "w2", torch.bfloat16, (E, I, H), dev)
+    if b1 is not None:
+        _need(b1, "b1", torch.bfloat16, (E, 2 * I), dev)
+    if b2 is not None:
+        _need(b2, "b2", torch.bfloat16, (E, H), dev)
+    r = routing(expert_idx, weights, token_idx=token_idx, N=N, total_pairs=total_pairs)
+    if out is None:
+        out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (N, H), dev)
+    if ws is None:
+        ws = torch.empty(routed_workspace_bytes(r, H, I, E), dtype=torch.uint8, device=dev)
+    m = _meta_struct(meta) if meta is not None else None
+    mp = ctypes.byref(m) if m is not None else None
+    _check(load().moe_nonexpand_routed_forward(x.data_ptr(), ctypes.byref(r), H, I, E, w1.data_ptr(), _ptr(b1),
+                                               w2.data_ptr(), _ptr(b2), ACT_SWIGLU, layout, out.data_ptr(), mp,
+                                               ws.data_ptr(), ws.numel(), _stream_handle(stream)),
+           "moe_nonexpand_routed_forward")
+    return out

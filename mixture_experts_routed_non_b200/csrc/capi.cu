@@ -19,6 +19,8 @@ constexpr size_t kAlign = 256;
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
 struct Layout {
     moe_ws_layout_t l;
 };
@@ -52,11 +54,10 @@ int check_dense(int64_t p_cap, int32_t H, int32_t I, int32_t E) {
     return MOE_OK;
 }
 
-moe_ws_layout_t compute_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K, int64_t total_pairs) {
+// Workspace layout for N tokens, NK routing slots and room for p_cap pairs.
+moe_ws_layout_t compute_layout_nk(int64_t N, int32_t H, int32_t I, int32_t E, int64_t NK, int64_t pc) {
     moe_ws_layout_t l;
     memset(&l, 0, sizeof l);
-    const int64_t NK = N * K;
-    const int64_t pc = total_pairs >= 0 ? total_pairs : NK;
     l.p_cap = pc;
     meta_tiling(NK, &l.meta_tile_slots, &l.meta_tiles);
     const size_t T = (size_t)l.meta_tiles;
@@ -94,6 +95,78 @@ moe_ws_layout_t compute_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32
     }
     l.total = o;
     return l;
+}
+
+moe_ws_layout_t compute_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K, int64_t total_pairs) {
+    return compute_layout_nk(N, H, I, E, N * K, total_pairs >= 0 ? total_pairs : N * K);
+}
+
+// ---------------------------------------------------------------------------
+// Routing input, either layout (checked).
+// ---------------------------------------------------------------------------
+struct Routing {
+    bool pairs;               // compact pair list (else the non-expand [N,K] table)
+    int idx64;
+    int64_t N;
+    int32_t K;                // [N,K] table: slots per token; pair list: 1
+    int64_t NK;               // slots
+    int64_t total_pairs;      // -1: unknown
+    int64_t p_cap;
+    const void *expert_idx;
+    const float *weights;
+    const void *token_idx;
+};
+
+Routing routing_topk32(const int32_t *topk_idx, const float *topk_w, int64_t N, int32_t K, int64_t total_pairs) {
+    Routing r;
+    r.pairs = false;
+    r.idx64 = 0;
+    r.N = N;
+    r.K = K;
+    r.NK = N * K;
+    r.total_pairs = total_pairs;
+    r.p_cap = total_pairs >= 0 ? total_pairs : N * K;
+    r.expert_idx = topk_idx;
+    r.weights = topk_w;
+    r.token_idx = nullptr;
+    return r;
+}
+
+int routing_from_desc(const moe_routing_t *d, int32_t E, Routing *r) {
+    if (!d || E < 1 || E > kMaxExperts) return MOE_ERR_ARG;
+    if (d->index_dtype != MOE_INDEX_INT32 && d->index_dtype != MOE_INDEX_INT64) return MOE_ERR_ARG;
+    const size_t isz = d->index_dtype == MOE_INDEX_INT64 ? 8 : 4;
+    if (d->N < 0) return MOE_ERR_ARG;
+    r->idx64 = d->index_dtype == MOE_INDEX_INT64;
+    r->N = d->N;
+    r->expert_idx = d->expert_idx;
+    r->weights = d->weights;
+    if (d->kind == MOE_ROUTING_TOPK) {
+        if (check_sizes(d->N, E, d->K, d->pairs)) return MOE_ERR_ARG;
+        r->pairs = false;
+        r->K = d->K;
+        r->NK = d->N * d->K;
+        r->total_pairs = d->pairs;
+        r->p_cap = d->pairs >= 0 ? d->pairs : r->NK;
+        r->token_idx = nullptr;
+        if (d->token_idx) return MOE_ERR_ARG;
+    } else if (d->kind == MOE_ROUTING_PAIRS) {
+        if (d->pairs < 0 || d->pairs >= (int64_t)(1u << 31) - (1 << 20)) return MOE_ERR_ARG;
+        if (d->N >= (int64_t)(1u << 31) - (1 << 20)) return MOE_ERR_ARG;
+        r->pairs = true;
+        r->K = 1;
+        r->NK = d->pairs;
+        r->total_pairs = -1;      // the list's own length bounds the pairs
+        r->p_cap = d->pairs;
+        r->token_idx = d->token_idx;
+        if (r->NK > 0 && !r->token_idx) return MOE_ERR_ARG;
+        if (r->token_idx && !aligned_to(r->token_idx, isz)) return MOE_ERR_ARG;
+    } else {
+        return MOE_ERR_ARG;
+    }
+    if (r->NK > 0 && (!r->expert_idx || !r->weights)) return MOE_ERR_ARG;
+    if (!aligned_to(r->expert_idx, isz) || !aligned_to(r->weights, 4)) return MOE_ERR_ARG;
+    return MOE_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -213,15 +286,17 @@ bool make_map_w1_concat(CUtensorMap *m, const void *ptr, uint64_t I, uint64_t ro
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-MetaArgs meta_args(const int32_t *topk_idx, const float *topk_w, int64_t N, int32_t K, int32_t E,
-                   int64_t total_pairs, const moe_ws_layout_t &l, uint8_t *ws, const moe_meta_t &meta) {
+MetaArgs meta_args(const Routing &r, int32_t E, const moe_ws_layout_t &l, uint8_t *ws, const moe_meta_t &meta) {
     MetaArgs a;
-    a.topk_idx = topk_idx;
-    a.topk_w = topk_w;
-    a.NK = N * K;
-    a.K = K;
+    a.topk_idx = r.expert_idx;
+    a.topk_w = r.weights;
+    a.token_idx = r.token_idx;
+    a.pair_list = r.pairs ? 1 : 0;
+    a.idx64 = r.idx64;
+    a.NK = r.NK;
+    a.K = r.K;
     a.E = E;
-    a.total_pairs = total_pairs;
+    a.total_pairs = r.total_pairs;
     a.p_cap = l.p_cap;
     a.tiles = l.meta_tiles;
     a.tile_slots = l.meta_tile_slots;
@@ -231,7 +306,7 @@ MetaArgs meta_args(const int32_t *topk_idx, const float *topk_w, int64_t N, int3
     a.tile_err = reinterpret_cast<int32_t *>(ws + l.tile_err);
     a.gemm_tile_off = reinterpret_cast<int32_t *>(ws + l.gemm_tile_offset);
     a.meta = meta;
-    a.N = N;
+    a.N = r.N;
     return a;
 }
 
@@ -257,21 +332,22 @@ int record(const moe_event_t *ev, int i, cudaStream_t s) {
     return cudaEventRecord(reinterpret_cast<cudaEvent_t>(ev[i]), s) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, int64_t N, int32_t H, int32_t I,
-                 int32_t E, int32_t K, int64_t total_pairs, const void *w1, const void *b1, const void *w2,
-                 const void *b2, int32_t activation, int32_t layout_kind, void *out, const moe_meta_t *meta_out,
-                 void *ws, size_t ws_bytes, cudaStream_t s, const moe_event_t *ev) {
-    int st = check_sizes(N, E, K, total_pairs);
-    if (st) return st;
+int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t E, const void *w1,
+                 const void *b1, const void *w2, const void *b2, int32_t activation, int32_t layout_kind,
+                 void *out, const moe_meta_t *meta_out, void *ws, size_t ws_bytes, cudaStream_t s,
+                 const moe_event_t *ev) {
+    const int64_t N = r.N;
+    int st = MOE_OK;
     // with N == 0 the token-sized buffers may be empty (null)
-    if ((N > 0 && (!x || !topk_idx || !topk_w || !out)) || !w1 || !w2) return MOE_ERR_ARG;
+    if ((N > 0 && (!x || !out)) || (r.NK > 0 && (!r.expert_idx || !r.weights)) || !w1 || !w2)
+        return MOE_ERR_ARG;
     if (activation != MOE_ACT_SWIGLU) return MOE_ERR_ARG;
     if (layout_kind != MOE_LAYOUT_INTERLEAVED && layout_kind != MOE_LAYOUT_CONCATENATED) return MOE_ERR_ARG;
     if (meta_out && !meta_complete(meta_out)) return MOE_ERR_ARG;
     if (!aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(out, 16) ||
-        (b1 && !aligned(b1, 16)) || (b2 && !aligned(b2, 16)) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+        (b1 && !aligned(b1, 16)) || (b2 && !aligned(b2, 16)))
         return MOE_ERR_ARG;
-    const moe_ws_layout_t l = compute_layout(N, H, I, E, K, total_pairs);
+    const moe_ws_layout_t l = compute_layout_nk(N, H, I, E, r.NK, r.p_cap);
     st = check_dense(l.p_cap, H, I, E);
     if (st) return st;
     if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MOE_ERR_WS;
@@ -281,7 +357,7 @@ int forward_impl(const void *x, const int32_t *topk_idx, const float *topk_w, in
 
     uint8_t *w = static_cast<uint8_t *>(ws);
     const moe_meta_t meta = meta_out ? *meta_out : ws_meta(l, w);
-    const MetaArgs ma = meta_args(topk_idx, topk_w, N, K, E, total_pairs, l, w, meta);
+    const MetaArgs ma = meta_args(r, E, l, w, meta);
     WsHeader *hdr = ma.hdr;
 
     if ((st = record(ev, 0, s))) return st;
@@ -396,8 +472,49 @@ extern "C" MOE_API int moe_nonexpand_metadata(const int32_t *topk_idx, const flo
     DeviceInfo dev;
     st = device_info(&dev);
     if (st) return st;
-    const MetaArgs ma = meta_args(topk_idx, topk_w, N, K, E, total_pairs, l, static_cast<uint8_t *>(ws), *meta);
+    const MetaArgs ma =
+        meta_args(routing_topk32(topk_idx, topk_w, N, K, total_pairs), E, l, static_cast<uint8_t *>(ws), *meta);
     return launch_meta(ma, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" MOE_API size_t moe_nonexpand_routed_workspace_bytes(const moe_routing_t *routing, int32_t H, int32_t I,
+                                                               int32_t E) {
+    Routing r;
+    if (routing_from_desc(routing, E, &r)) return 0;
+    if (H < 0 || I < 0) return 0;
+    const moe_ws_layout_t l = compute_layout_nk(r.N, H, I, E, r.NK, r.p_cap);
+    if ((H > 0 || I > 0) && check_dense(l.p_cap, H, I, E)) return 0;
+    return l.total;
+}
+
+extern "C" MOE_API int moe_nonexpand_routed_metadata(const moe_routing_t *routing, int32_t E,
+                                                     const moe_meta_t *meta, void *ws, size_t ws_bytes,
+                                                     moe_stream_t stream) {
+    Routing r;
+    int st = routing_from_desc(routing, E, &r);
+    if (st) return st;
+    if (!meta || !meta->token_offset || !meta->expert_frequency || !meta->expert_frequency_offset)
+        return MOE_ERR_ARG;
+    if (r.NK > 0 && !meta_complete(meta)) return MOE_ERR_ARG;
+    const moe_ws_layout_t l = compute_layout_nk(r.N, 0, 0, E, r.NK, r.p_cap);
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MOE_ERR_WS;
+    DeviceInfo dev;
+    st = device_info(&dev);
+    if (st) return st;
+    const MetaArgs ma = meta_args(r, E, l, static_cast<uint8_t *>(ws), *meta);
+    return launch_meta(ma, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" MOE_API int moe_nonexpand_routed_forward(const void *x, const moe_routing_t *routing, int32_t H,
+                                                    int32_t I, int32_t E, const void *w1, const void *b1,
+                                                    const void *w2, const void *b2, int32_t activation,
+                                                    int32_t gate_up_layout, void *out, const moe_meta_t *meta_out,
+                                                    void *ws, size_t ws_bytes, moe_stream_t stream) {
+    Routing r;
+    const int st = routing_from_desc(routing, E, &r);
+    if (st) return st;
+    return forward_impl(x, r, H, I, E, w1, b1, w2, b2, activation, gate_up_layout, out, meta_out, ws, ws_bytes,
+                        reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 extern "C" MOE_API int moe_nonexpand_forward(const void *x, const int32_t *topk_idx, const float *topk_w, int64_t N,
@@ -405,9 +522,12 @@ extern "C" MOE_API int moe_nonexpand_forward(const void *x, const int32_t *topk_
                                   const void *w1, const void *b1, const void *w2, const void *b2,
                                   int32_t activation, int32_t gate_up_layout, void *out,
                                   const moe_meta_t *meta_out, void *ws, size_t ws_bytes, moe_stream_t stream) {
-    return forward_impl(x, topk_idx, topk_w, N, H, I, E, K, total_pairs, w1, b1, w2, b2, activation,
-                        gate_up_layout, out, meta_out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
-                        nullptr);
+    int st = check_sizes(N, E, K, total_pairs);
+    if (st) return st;
+    if (!aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_ARG;
+    return forward_impl(x, routing_topk32(topk_idx, topk_w, N, K, total_pairs), H, I, E, w1, b1, w2, b2,
+                        activation, gate_up_layout, out, meta_out, ws, ws_bytes,
+                        reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 extern "C" MOE_API int moe_nonexpand_forward_timed(const void *x, const int32_t *topk_idx, const float *topk_w, int64_t N,
@@ -419,9 +539,12 @@ extern "C" MOE_API int moe_nonexpand_forward_timed(const void *x, const int32_t 
     if (!stage_events) return MOE_ERR_ARG;
     for (int i = 0; i < 5; ++i)
         if (!stage_events[i]) return MOE_ERR_ARG;
-    return forward_impl(x, topk_idx, topk_w, N, H, I, E, K, total_pairs, w1, b1, w2, b2, activation,
-                        gate_up_layout, out, meta_out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
-                        stage_events);
+    int st = check_sizes(N, E, K, total_pairs);
+    if (st) return st;
+    if (!aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_ARG;
+    return forward_impl(x, routing_topk32(topk_idx, topk_w, N, K, total_pairs), H, I, E, w1, b1, w2, b2,
+                        activation, gate_up_layout, out, meta_out, ws, ws_bytes,
+                        reinterpret_cast<cudaStream_t>(stream), stage_events);
 }
 
 extern "C" MOE_API int moe_nonexpand_combine(const void *y, const moe_meta_t *meta, int64_t N, int32_t H, void *out,

@@ -11,7 +11,10 @@
 //
 // A block owns up to kTokPerBlock consecutive tokens.  Their token offsets and
 // the row index and score of every one of their pairs (a contiguous q range)
-// are loaded into shared memory once, with coalesced loads; then each thread
+// are loaded into shared memory once, with coalesced loads (a block whose
+// tokens have more pairs than the staging arrays hold -- possible for a pair
+// list, which bounds no token's pair count -- reads them from global memory
+// instead); then each thread
 // owns 16-byte column chunks and walks the block's pairs in batches of eight
 // rows whose loads are all issued before any is accumulated -- across token
 // boundaries, so the loads in flight do not depend on how many pairs each
@@ -24,7 +27,7 @@ namespace {
 
 constexpr int kCombineThreads = 256;
 constexpr int kTokPerBlock = 8;
-constexpr int kMaxK = 32;
+constexpr int kStagedPairs = kTokPerBlock * 32;  // pair indices staged in shared memory per block
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
     uint4 v;
@@ -54,15 +57,60 @@ __device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
     return o;
 }
 
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(
+// One block's tokens [t0, t0+nt): their pairs are q in [qa, qa+np) with
+// token-local ends s_off[j+1]-qa.  pidx/pw are the pairs' row indices and
+// scores: in shared memory when staged, else read from global memory.
+template <bool kStaged>
+__device__ __forceinline__ void combine_tokens(const __nv_bfloat16 *__restrict__ y, const int *pidx,
+                                               const float *pw, const int *s_off, int qa, int np, int nt,
+                                               int32_t H, __nv_bfloat16 *__restrict__ out_t0) {
+    const int chunks = H >> 3;
+    for (int c = threadIdx.x; c < chunks; c += kCombineThreads) {
+        const __nv_bfloat16 *ycol = y + (size_t)c * 8;
+        __nv_bfloat16 *ocol = out_t0 + (size_t)c * 8;
+        // walk the block's pairs in batches of 8 rows in flight, across token
+        // boundaries; each token's pairs are still summed in q order
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        int j = 0;                       // current token (block-local)
+        int tok_end = s_off[1] - qa;     // its pairs end here
+        for (int base = 0; base < np; base += 8) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int q = base + u;
+                const int row = q < np ? (kStaged ? pidx[q] : __ldg(pidx + q)) : 0;
+                v[u] = q < np ? ld_stream_v4(ycol + (size_t)row * H) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int q = base + u;
+                if (q >= np) break;
+                while (q >= tok_end) {  // finish token j (and any token without pairs)
+                    *reinterpret_cast<uint4 *>(ocol + (size_t)j * H) = pack8(acc);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+                    ++j;
+                    tok_end = s_off[j + 1] - qa;
+                }
+                fma8(acc, kStaged ? pw[q] : __ldg(pw + q), v[u]);
+            }
+        }
+        for (; j < nt; ++j) {  // the last token with pairs, then trailing tokens without
+            *reinterpret_cast<uint4 *>(ocol + (size_t)j * H) = pack8(acc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kCombineThreads, 4) combine_kernel(
     const __nv_bfloat16 *__restrict__ y, const int32_t *__restrict__ token_offset,
     const int32_t *__restrict__ s_rev, const float *__restrict__ scores, int64_t N, int32_t H,
     __nv_bfloat16 *__restrict__ out, const WsHeader *hdr, int tok_per_block) {
     __shared__ int s_off[kTokPerBlock + 1];
-    __shared__ int s_p[kTokPerBlock * kMaxK];
-    __shared__ float s_w[kTokPerBlock * kMaxK];
+    __shared__ int s_p[kStagedPairs];
+    __shared__ float s_w[kStagedPairs];
     if (hdr && *(volatile const uint32_t *)&hdr->abort) return;
-    const int chunks = H >> 3;
     const int64_t n_groups = (N + tok_per_block - 1) / tok_per_block;
     for (int64_t grp = blockIdx.x; grp < n_groups; grp += gridDim.x) {
         const int64_t t0 = grp * tok_per_block;
@@ -71,43 +119,16 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(
         __syncthreads();
         const int qa = s_off[0];
         const int np = s_off[nt] - qa;  // pairs of the block's tokens, a contiguous q range
-        for (int i = threadIdx.x; i < np; i += kCombineThreads) {
-            s_p[i] = __ldg(s_rev + qa + i);
-            s_w[i] = __ldg(scores + qa + i);
-        }
-        __syncthreads();
-        for (int c = threadIdx.x; c < chunks; c += kCombineThreads) {
-            const __nv_bfloat16 *ycol = y + (size_t)c * 8;
-            __nv_bfloat16 *ocol = out + (size_t)t0 * H + (size_t)c * 8;
-            // walk the block's pairs in batches of 8 rows in flight, across token
-            // boundaries; each token's pairs are still summed in q order
-            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            int j = 0;                       // current token (block-local)
-            int tok_end = s_off[1] - qa;     // its pairs end here
-            for (int base = 0; base < np; base += 8) {
-                uint4 v[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    v[u] = (base + u < np) ? ld_stream_v4(ycol + (size_t)s_p[base + u] * H) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int q = base + u;
-                    if (q >= np) break;
-                    while (q >= tok_end) {  // finish token j (and any token without pairs)
-                        *reinterpret_cast<uint4 *>(ocol + (size_t)j * H) = pack8(acc);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-                        ++j;
-                        tok_end = s_off[j + 1] - qa;
-                    }
-                    fma8(acc, s_w[q], v[u]);
-                }
+        __nv_bfloat16 *out_t0 = out + (size_t)t0 * H;
+        if (np <= kStagedPairs) {
+            for (int i = threadIdx.x; i < np; i += kCombineThreads) {
+                s_p[i] = __ldg(s_rev + qa + i);
+                s_w[i] = __ldg(scores + qa + i);
             }
-            for (; j < nt; ++j) {  // the last token with pairs, then trailing tokens without
-                *reinterpret_cast<uint4 *>(ocol + (size_t)j * H) = pack8(acc);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-            }
+            __syncthreads();
+            combine_tokens<true>(y, s_p, s_w, s_off, qa, np, nt, H, out_t0);
+        } else {  // more pairs than the staging arrays hold (a pair list may give a token any number)
+            combine_tokens<false>(y, s_rev + qa, scores + qa, s_off, qa, np, nt, H, out_t0);
         }
         __syncthreads();  // shared indices are reused by the next group
     }

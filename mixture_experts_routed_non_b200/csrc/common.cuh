@@ -53,9 +53,12 @@ constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;
 // Host-side launch descriptions (filled by capi.cu).
 // ---------------------------------------------------------------------------
 struct MetaArgs {
-    const int32_t *topk_idx;
-    const float *topk_w;
-    int64_t NK;
+    const void *topk_idx;     // expert id per slot: [N,K] non-expand table, or [P] pair list
+    const float *topk_w;      // weight per slot
+    const void *token_idx;    // pair list: token of each slot ([P], ascending)
+    int32_t pair_list;        // 1: compact pair list (token from token_idx); 0: table (slot s is token s/K)
+    int32_t idx64;            // ids are int64 (else int32)
+    int64_t NK;               // slots
     int32_t K;
     int32_t E;
     int64_t total_pairs;  // -1: unknown

@@ -90,19 +90,57 @@ __device__ int block_sum(int v) {
     return t;
 }
 
-__device__ __forceinline__ void load_chunk(const int32_t *idx, int base, int end, int lane, int (&e)[kV]) {
+// An id read as int: int64 values are clamped to the int range, which keeps
+// their order and keeps every out-of-range id out of range (and off -1).
+template <bool kIdx64>
+__device__ __forceinline__ int load_id(const void *ids, int s) {
+    if (kIdx64) {
+        const long long v = __ldg(static_cast<const long long *>(ids) + s);
+        return (int)max(min(v, 0x7fffffffLL), -0x80000000LL);
+    }
+    return __ldg(static_cast<const int *>(ids) + s);
+}
+
+// An id at its own width (for the order check of a pair list's tokens).
+template <bool kIdx64>
+__device__ __forceinline__ long long load_id_wide(const void *ids, int s) {
+    return kIdx64 ? __ldg(static_cast<const long long *>(ids) + s) : (long long)__ldg(static_cast<const int *>(ids) + s);
+}
+
+template <bool kIdx64>
+__device__ __forceinline__ void load_chunk(const void *ids, int base, int end, int lane, int (&e)[kV]) {
 #pragma unroll
     for (int v = 0; v < kV; ++v) {
         const int s = base + 32 * v + lane;
-        e[v] = s < end ? __ldg(idx + s) : -1;
+        e[v] = s < end ? load_id<kIdx64>(ids, s) : -1;
     }
+}
+
+// Token of slot s: s / K for the [N,K] table, token_idx[s] for a pair list.
+template <bool kPairs, bool kIdx64>
+__device__ __forceinline__ int slot_token(const MetaArgs &a, int s) {
+    return kPairs ? load_id<kIdx64>(a.token_idx, s) : s / a.K;
+}
+
+// A slot becomes a pair when its expert id is in [0,E) and (pair list) its
+// token id is in [0,N).  Sets *bad for ids that are neither valid nor -1.
+template <bool kPairs>
+__device__ __forceinline__ bool slot_valid(const MetaArgs &a, int e, int t, unsigned *bad) {
+    const bool e_ok = (e >= 0) && (e < a.E);
+    if (!e_ok && e != -1) *bad |= MOE_DEVERR_BAD_EXPERT_ID;
+    if (kPairs && e_ok && (t < 0 || (int64_t)t >= a.N)) {
+        *bad |= MOE_DEVERR_BAD_TOKEN;
+        return false;
+    }
+    return e_ok;
 }
 
 // Shared memory (ints): cnt[kMetaWarps][E] | part_all[kPartInts] | part_before[kPartInts]
 //                       | off[kMaxExperts+1] | gt[kMaxExperts+1]
 constexpr int kPartInts = kMaxExperts;   // G*E <= max(kMetaThreads, E) <= kMaxExperts
 
-__global__ void __launch_bounds__(kMetaThreads) meta_kernel(const MetaArgs a) {
+template <bool kPairs, bool kIdx64>
+__global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a) {
     extern __shared__ int sm[];
     const int E = a.E, K = a.K, T = a.tiles;
     int *cnt = sm;
@@ -123,8 +161,13 @@ __global__ void __launch_bounds__(kMetaThreads) meta_kernel(const MetaArgs a) {
     const int sub = a.tile_slots / kMetaWarps;
     const int w0 = s0 + warp * sub;
     const int w1 = min(w0 + sub, s1);
-    int ev0[kV];
-    load_chunk(a.topk_idx, w0, w1, lane, ev0);
+    int ev0[kV], tv0[kV];
+    load_chunk<kIdx64>(a.topk_idx, w0, w1, lane, ev0);
+#pragma unroll
+    for (int v = 0; v < kV; ++v) {
+        const int s = w0 + 32 * v + lane;
+        tv0[v] = (kPairs && s < w1) ? slot_token<kPairs, kIdx64>(a, s) : 0;
+    }
     for (int i = threadIdx.x; i < kMetaWarps * E; i += kMetaThreads) cnt[i] = 0;
     if (threadIdx.x == 0) s_err = 0;
     __syncthreads();
@@ -134,18 +177,31 @@ __global__ void __launch_bounds__(kMetaThreads) meta_kernel(const MetaArgs a) {
     int nvalid = 0;
     unsigned my_err = 0;
     for (int base = w0; base < w1; base += kWarpChunk) {
-        int ev[kV];
+        int ev[kV], tv[kV];
         if (base == w0) {
 #pragma unroll
-            for (int v = 0; v < kV; ++v) ev[v] = ev0[v];
+            for (int v = 0; v < kV; ++v) {
+                ev[v] = ev0[v];
+                tv[v] = tv0[v];
+            }
         } else {
-            load_chunk(a.topk_idx, base, w1, lane, ev);
+            load_chunk<kIdx64>(a.topk_idx, base, w1, lane, ev);
+#pragma unroll
+            for (int v = 0; v < kV; ++v) {
+                const int s = base + 32 * v + lane;
+                tv[v] = (kPairs && s < w1) ? slot_token<kPairs, kIdx64>(a, s) : 0;
+            }
         }
 #pragma unroll
         for (int v = 0; v < kV; ++v) {
             const int e = ev[v];
-            const bool valid = (e >= 0) && (e < E);
-            if (!valid && e != -1) my_err = MOE_DEVERR_BAD_EXPERT_ID;
+            const bool valid = slot_valid<kPairs>(a, e, tv[v], &my_err);
+            if (kPairs) {  // a pair list must be in ascending token order
+                const int s = base + 32 * v + lane;
+                if (s > 0 && s < w1 &&
+                    load_id_wide<kIdx64>(a.token_idx, s - 1) > load_id_wide<kIdx64>(a.token_idx, s))
+                    my_err |= MOE_DEVERR_BAD_TOKEN;
+            }
             const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
             if (valid && lane == __ffs(peers) - 1) mycnt[e] += __popc(peers);
             nvalid += __popc(__ballot_sync(kFull, valid));
@@ -157,7 +213,8 @@ __global__ void __launch_bounds__(kMetaThreads) meta_kernel(const MetaArgs a) {
     float wv0[kV];
 #pragma unroll
     for (int v = 0; v < kV; ++v) {
-        const bool valid = (ev0[v] >= 0) && (ev0[v] < E);
+        unsigned ignore = 0;
+        const bool valid = slot_valid<kPairs>(a, ev0[v], tv0[v], &ignore);
         wv0[v] = valid ? __ldg(a.topk_w + w0 + 32 * v + lane) : 0.f;
     }
     if (lane == 0) wq[warp] = nvalid;
@@ -266,6 +323,13 @@ __global__ void __launch_bounds__(kMetaThreads) meta_kernel(const MetaArgs a) {
             a.hdr->err = err;
             a.hdr->abort = abort ? 1u : 0u;
         }
+        if (kPairs) {
+            // tokens after the last listed token (all tokens if the list is empty)
+            int last = a.NK > 0 ? slot_token<kPairs, kIdx64>(a, (int)a.NK - 1) : -1;
+            if (last < -1) last = -1;
+            for (int64_t tt = (int64_t)last + 1 + threadIdx.x; tt < a.N; tt += kMetaThreads)
+                a.meta.token_offset[tt] = P;
+        }
     }
     if (abort) return;  // the pair arrays are too small for the pairs seen
 
@@ -291,20 +355,23 @@ __global__ void __launch_bounds__(kMetaThreads) meta_kernel(const MetaArgs a) {
     // ---- phase B.3: positions, in slot order
     int q_run = wq[warp];
     for (int base = w0; base < w1; base += kWarpChunk) {
-        int ev[kV];
+        int ev[kV], tv[kV];
         float wv[kV];
         if (base == w0) {
 #pragma unroll
             for (int v = 0; v < kV; ++v) {
                 ev[v] = ev0[v];
+                tv[v] = tv0[v];
                 wv[v] = wv0[v];
             }
         } else {
-            load_chunk(a.topk_idx, base, w1, lane, ev);
+            load_chunk<kIdx64>(a.topk_idx, base, w1, lane, ev);
 #pragma unroll
             for (int v = 0; v < kV; ++v) {
                 const int s = base + 32 * v + lane;
-                const bool valid = (ev[v] >= 0) && (ev[v] < E);
+                tv[v] = (kPairs && s < w1) ? slot_token<kPairs, kIdx64>(a, s) : 0;
+                unsigned ignore = 0;
+                const bool valid = slot_valid<kPairs>(a, ev[v], tv[v], &ignore);
                 wv[v] = valid ? __ldg(a.topk_w + s) : 0.f;
             }
         }
@@ -312,7 +379,8 @@ __global__ void __launch_bounds__(kMetaThreads) meta_kernel(const MetaArgs a) {
         for (int v = 0; v < kV; ++v) {
             const int s = base + 32 * v + lane;
             const int e = ev[v];
-            const bool valid = (e >= 0) && (e < E);
+            unsigned ignore = 0;
+            const bool valid = slot_valid<kPairs>(a, e, tv[v], &ignore);
             const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
             const int pb = valid ? mycnt[e] : 0;
             __syncwarp();
@@ -321,12 +389,24 @@ __global__ void __launch_bounds__(kMetaThreads) meta_kernel(const MetaArgs a) {
             const int q = q_run + __popc(vb & lt);
             if (valid) {
                 const int p = pb + __popc(peers & lt);
-                a.meta.x_gather_idx[p] = s / K;
+                a.meta.x_gather_idx[p] = kPairs ? tv[v] : s / K;
                 a.meta.s_scatter_idx[p] = q;
                 a.meta.s_reverse_scatter_idx[q] = p;
                 a.meta.scores[q] = wv[v];
             }
-            if (s < w1 && (s % K) == 0) a.meta.token_offset[s / K] = q;
+            if (s < w1) {
+                if (!kPairs) {
+                    if ((s % K) == 0) a.meta.token_offset[s / K] = q;
+                } else {
+                    // tokens (previous slot's token, this slot's token] start at q
+                    // (an order violation was flagged in phase A; offsets then unspecified)
+                    const int t = tv[v];
+                    const int tprev = s > 0 ? slot_token<kPairs, kIdx64>(a, s - 1) : -1;
+                    const int64_t lo = max((int64_t)tprev + 1, (int64_t)0);
+                    const int64_t hi = min((int64_t)t, a.N - 1);
+                    for (int64_t tt = lo; tt <= hi; ++tt) a.meta.token_offset[tt] = q;
+                }
+            }
             q_run += __popc(vb);
             __syncwarp();
         }
@@ -339,25 +419,32 @@ size_t meta_smem_bytes(int E) {
     return ((size_t)kMetaWarps * E + 2 * kPartInts + 2 * (kMaxExperts + 1)) * sizeof(int);
 }
 
-cudaError_t launch_meta(const MetaArgs &a, cudaStream_t s) {
+template <bool kPairs, bool kIdx64>
+cudaError_t launch_meta_as(const MetaArgs &a, cudaStream_t s, int dev) {
     static bool configured[64] = {};
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess) return err;
     if (dev < 64 && !configured[dev]) {
-        err = cudaFuncSetAttribute(meta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)meta_smem_bytes(kMaxExperts));
+        const cudaError_t err = cudaFuncSetAttribute(meta_kernel<kPairs, kIdx64>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)meta_smem_bytes(kMaxExperts));
         if (err != cudaSuccess) return err;
         configured[dev] = true;
     }
-    // the grid barrier's arrival counter starts from zero in every call
-    err = cudaMemsetAsync(&a.hdr->grid_arrive, 0, sizeof(a.hdr->grid_arrive), s);
-    if (err != cudaSuccess) return err;
     MetaArgs args = a;
     void *params[] = {&args};
     // cooperative: all T CTAs are resident at once, so the grid barrier ends
-    return cudaLaunchCooperativeKernel((const void *)meta_kernel, dim3(a.tiles), dim3(kMetaThreads), params,
-                                       meta_smem_bytes(a.E), s);
+    return cudaLaunchCooperativeKernel((const void *)meta_kernel<kPairs, kIdx64>, dim3(a.tiles),
+                                       dim3(kMetaThreads), params, meta_smem_bytes(a.E), s);
+}
+
+cudaError_t launch_meta(const MetaArgs &a, cudaStream_t s) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    // the grid barrier's arrival counter starts from zero in every call
+    err = cudaMemsetAsync(&a.hdr->grid_arrive, 0, sizeof(a.hdr->grid_arrive), s);
+    if (err != cudaSuccess) return err;
+    if (a.pair_list) return a.idx64 ? launch_meta_as<true, true>(a, s, dev) : launch_meta_as<true, false>(a, s, dev);
+    return a.idx64 ? launch_meta_as<false, true>(a, s, dev) : launch_meta_as<false, false>(a, s, dev);
 }
 
 }  // namespace moe

@@ -106,6 +106,9 @@ extern "C" MOE_API int moe_nonexpand_metadata_noalloc(const int32_t *topk_idx, c
     MetaArgs a;
     a.topk_idx = topk_idx;
     a.topk_w = topk_w;
+    a.token_idx = nullptr;
+    a.pair_list = 0;
+    a.idx64 = 0;
     a.NK = N * K;
     a.K = K;
     a.E = E;

@@ -236,3 +236,34 @@ def custom(N: int, H: int, I: int, E: int, K: int, *, routing_kind="uniform",
     """A workload with arbitrary sizes (tests use it for ragged and edge cases)."""
     return Workload(name, N=N, H=H, I=I, E=E, K=K, routing=routing_kind, zipf_s=zipf_s,
                     p_invalid=p_invalid, scores=scores_kind, bias=bias, seed=seed)
+
+
+def pair_list_from_table(idx: np.ndarray, w: np.ndarray, *, keep_invalid: bool = False,
+                         empty_tokens: Optional[np.ndarray] = None):
+    """A compact pair list (token_idx, expert_idx, weights; tokens ascending)
+    holding the slots of an [N,K] routing table in row-major order.  Slots
+    marked -1 are dropped unless ``keep_invalid``; tokens listed in
+    ``empty_tokens`` lose all their entries (tokens without pairs)."""
+    N, K = idx.shape
+    tok = np.repeat(np.arange(N, dtype=np.int64), K)
+    exp = idx.reshape(-1).astype(np.int64)
+    wt = w.reshape(-1).astype(np.float32)
+    keep = np.ones(N * K, bool) if keep_invalid else exp >= 0
+    if empty_tokens is not None:
+        keep &= ~np.isin(tok, empty_tokens)
+    return tok[keep], exp[keep], wt[keep]
+
+
+def many_pair_tokens(N: int, E: int, heavy: np.ndarray, K: int, rng: np.random.Generator):
+    """A pair list where the tokens in ``heavy`` route to every expert and the
+    others to K distinct experts (tokens ascending, experts in random order
+    within a token); weights uniform in [0,1)."""
+    toks, exps = [], []
+    for t in range(N):
+        k = E if t in set(heavy.tolist()) else K
+        e = rng.permutation(E)[:k]
+        toks.append(np.full(k, t, np.int64))
+        exps.append(e.astype(np.int64))
+    tok = np.concatenate(toks)
+    exp = np.concatenate(exps)
+    return tok, exp, rng.random(tok.shape[0]).astype(np.float32)

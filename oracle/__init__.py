@@ -58,6 +58,8 @@ def _load(path: str | None = None):
         i64, i32 = ctypes.c_int64, ctypes.c_int32
         lib.oracle_metadata.restype = i64
         lib.oracle_metadata.argtypes = [i64, i32, i32, P, P, P, P, P, P, P, P, P, P]
+        lib.oracle_metadata_pairs.restype = i64
+        lib.oracle_metadata_pairs.argtypes = [i64, i64, i32, P, P, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_expert_row.restype = None
         lib.oracle_expert_row.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P]
         lib.oracle_forward_rows.restype = None
@@ -106,6 +108,34 @@ def metadata(topk_idx: np.ndarray, topk_w: np.ndarray, E: int, lib_path: str | N
     return dict(freq=freq, off=off, x_gather_idx=xg[:P].copy(), s_scatter_idx=ss[:P].copy(),
                 s_reverse_scatter_idx=sr[:P].copy(), token_offset=to, scores=sc[:P].copy(),
                 P=int(P), bad_ids=int(bad[0]))
+
+
+def metadata_pairs(token_idx: np.ndarray, expert_idx: np.ndarray, weights: np.ndarray, N: int, E: int,
+                   lib_path: str | None = None) -> dict:
+    """Routing metadata of a compact pair list (token_idx ascending).  Returns
+    the keys of ``metadata`` plus bad_tokens and unsorted."""
+    lib = _load(lib_path)
+    ti = np.ascontiguousarray(token_idx, dtype=np.int64).reshape(-1)
+    ei = np.ascontiguousarray(expert_idx, dtype=np.int64).reshape(-1)
+    w = np.ascontiguousarray(weights, dtype=np.float32).reshape(-1)
+    PL = ti.shape[0]
+    assert ei.shape[0] == PL and w.shape[0] == PL
+    cap = max(1, PL)
+    freq = np.zeros(E, np.int32)
+    off = np.zeros(E + 1, np.int32)
+    xg = np.zeros(cap, np.int32)
+    ss = np.zeros(cap, np.int32)
+    sr = np.zeros(cap, np.int32)
+    to = np.zeros(N + 1, np.int32)
+    sc = np.zeros(cap, np.float32)
+    bad = np.zeros(1, np.int64)
+    badt = np.zeros(1, np.int64)
+    uns = np.zeros(1, np.int32)
+    P = lib.oracle_metadata_pairs(N, PL, E, _ptr(ti), _ptr(ei), _ptr(w), _ptr(freq), _ptr(off), _ptr(xg),
+                                  _ptr(ss), _ptr(sr), _ptr(to), _ptr(sc), _ptr(bad), _ptr(badt), _ptr(uns))
+    return dict(freq=freq, off=off, x_gather_idx=xg[:P].copy(), s_scatter_idx=ss[:P].copy(),
+                s_reverse_scatter_idx=sr[:P].copy(), token_offset=to, scores=sc[:P].copy(),
+                P=int(P), bad_ids=int(bad[0]), bad_tokens=int(badt[0]), unsorted=bool(uns[0]))
 
 
 def expert_row(x_row, w1e, b1e, w2e, b2e, layout: int = LAYOUT_INTERLEAVED, lib_path: str | None = None):

@@ -118,6 +118,87 @@ int64_t oracle_metadata(int64_t N, int32_t K, int32_t E,
 }
 
 /* ------------------------------------------------------------------------
+ * Routing metadata of a compact pair list (sonic-moe issue #68, the general
+ * routing API the non-expand path is proposed beside: token_indices,
+ * expert_indices and router_scores, one entry per (token, expert) pair, in
+ * ascending token order).
+ *
+ * Entry i of the list is kept when expert_idx[i] is in [0,E) and
+ * token_idx[i] is in [0,N); pair q counts the kept entries in list order.
+ * Expert id -1 drops an entry silently; any other out-of-range expert id is
+ * counted in *bad_ids; a kept-looking entry (valid expert) whose token is out
+ * of range is counted in *bad_tokens.  *unsorted is set when some entry's
+ * token is smaller than the one before it (the metadata then assumes an
+ * order it does not have and token_offset means nothing).
+ *
+ * Outputs are those of oracle_metadata, with
+ *   token_offset[t] = number of kept entries whose token is below t
+ * (t = 0..N), which for an ascending list makes pairs of token t the q in
+ * [token_offset[t], token_offset[t+1]).  Pair arrays need room for P_list.
+ * Returns P.
+ * ---------------------------------------------------------------------- */
+int64_t oracle_metadata_pairs(int64_t N, int64_t P_list, int32_t E,
+                              const int64_t *token_idx, const int64_t *expert_idx,
+                              const float *weights,
+                              int32_t *freq, int32_t *off,
+                              int32_t *x_gather_idx, int32_t *s_scatter_idx,
+                              int32_t *s_rev, int32_t *token_offset, float *scores,
+                              int64_t *bad_ids, int64_t *bad_tokens, int32_t *unsorted)
+{
+    int64_t nbad = 0, nbadtok = 0, q = 0;
+    int32_t *pair_token = (int32_t *)malloc(sizeof(int32_t) * (size_t)(P_list + 1));
+    int32_t *pair_expert = (int32_t *)malloc(sizeof(int32_t) * (size_t)(P_list + 1));
+    int32_t *cursor = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E + 1));
+
+    /* 1. kept entries in list order */
+    *unsorted = 0;
+    for (int64_t i = 0; i < P_list; ++i) {
+        int64_t t = token_idx[i], e = expert_idx[i];
+        if (i > 0 && token_idx[i - 1] > t) *unsorted = 1;
+        if (e >= 0 && e < E) {
+            if (t >= 0 && t < N) {
+                pair_token[q] = (int32_t)t;
+                pair_expert[q] = (int32_t)e;
+                scores[q] = weights[i];
+                ++q;
+            } else {
+                ++nbadtok;
+            }
+        } else if (e != -1) {
+            ++nbad;
+        }
+    }
+
+    /* 2. token offsets: kept pairs whose token is below t */
+    for (int64_t t = 0; t <= N; ++t) {
+        int64_t below = 0;
+        for (int64_t j = 0; j < q; ++j)
+            if (pair_token[j] < t) ++below;
+        token_offset[t] = (int32_t)below;
+    }
+
+    /* 3. histogram, offsets and the stable counting sort by expert */
+    for (int32_t e = 0; e < E; ++e) freq[e] = 0;
+    for (int64_t j = 0; j < q; ++j) freq[pair_expert[j]] += 1;
+    off[0] = 0;
+    for (int32_t e = 0; e < E; ++e) off[e + 1] = off[e] + freq[e];
+    for (int32_t e = 0; e < E; ++e) cursor[e] = off[e];
+    for (int64_t j = 0; j < q; ++j) {
+        int32_t p = cursor[pair_expert[j]]++;
+        x_gather_idx[p] = pair_token[j];
+        s_scatter_idx[p] = (int32_t)j;
+        s_rev[j] = p;
+    }
+
+    free(pair_token);
+    free(pair_expert);
+    free(cursor);
+    *bad_ids = nbad;
+    *bad_tokens = nbadtok;
+    return q;
+}
+
+/* ------------------------------------------------------------------------
  * One expert applied to one token row, in double.
  *   z   = x_t . W1[e] + b1[e]                       (2I values)
  *   h_j = silu(gate_j) * up_j,  silu(g) = g / (1 + exp(-g))

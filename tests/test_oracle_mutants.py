@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 from mixture_experts_routed_non_b200 import synthetic
+from test_oracle_pairs import check_pair_fixture, check_table_equivalence
 from test_oracle_pins import (GOLDEN, _bf, _load, _num, _recipe_torch_cpu,
                               check_metadata_invariants)
 
@@ -38,6 +39,11 @@ MUTANTS = {
                           "        for (int32_t k = 0; k < K; ++k) {"),
     "offsets_inclusive": ("off[e + 1] = off[e] + freq[e];", "off[e + 1] = off[e] + freq[e] + (e == 0);"),
     "invalid_counted": ("if (e >= 0 && e < E) {", "if (e < E) { if (e < 0) e = 0;"),
+    "pairs_offset_inclusive": ("if (pair_token[j] < t) ++below;", "if (pair_token[j] <= t) ++below;"),
+    "pairs_bad_token_kept": ("if (t >= 0 && t < N) {", "if (t >= 0) {"),
+    "pairs_sort_unstable": ("for (int64_t j = 0; j < q; ++j) {\n        int32_t p = cursor[pair_expert[j]]++;",
+                            "for (int64_t j = q - 1; j >= 0; --j) {\n        int32_t p = cursor[pair_expert[j]]++;"),
+    "pairs_score_of_next": ("scores[q] = weights[i];", "scores[q] = weights[i + 1 < P_list ? i + 1 : i];"),
 }
 
 
@@ -79,6 +85,11 @@ def _pins_pass(lib):
             out_ex = [eval(s, env) for s in g["expected_closed_form"][key]["out"]]
             if not np.allclose(out[0], out_ex, rtol=1e-12, atol=1e-12):
                 return False
+        # pair-list metadata: hand-worked fixture, table oracle on a flattened table
+        check_pair_fixture(lib)
+        wl = synthetic.WORKLOADS["tiny"]
+        idx, w = synthetic.make_routing(wl, invalid_value=float("nan"))
+        check_table_equivalence(idx, w, wl.E, lib)
         # torch-CPU sort recipe on the tiny workload
         inp = synthetic.make_inputs("tiny", device="cpu")
         wts = oracle.Weights(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
