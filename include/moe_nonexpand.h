@@ -262,6 +262,39 @@ MOE_API int moe_nonexpand_routed_forward(const void *x, const moe_routing_t *rou
                                  int32_t activation, int32_t gate_up_layout, void *out,
                                  const moe_meta_t *meta_out, void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/*
+ * Router top-k: router logits [N,E] -> the routing table topk_idx [N,K] /
+ * topk_w [N,K] that moe_nonexpand_forward takes (sonic-moe write-up, "Three
+ * routing strategies, selected on the command line": TC top-K routing is the
+ * softmax over the top-k logits; Qwen3-style routing is the top-k of the
+ * softmax over all experts, with optional renormalisation of the chosen
+ * probabilities).
+ *
+ *   MOE_ROUTER_SOFTMAX_TOPK         w = softmax over the K chosen logits
+ *   MOE_ROUTER_TOPK_SOFTMAX         w = softmax over all E logits, at the chosen
+ *   MOE_ROUTER_TOPK_SOFTMAX_RENORM  the same, divided by its sum over the K chosen
+ *
+ * The chosen experts are the K largest logits (softmax is increasing, so all
+ * modes choose alike), compared as given: fp32, or bf16 widened exactly.
+ * Slot k holds the k-th largest; equal logits go to the lower expert id.  A
+ * NaN logit is read as -inf.  A token whose chosen logits are all -inf gets
+ * NaN weights.  Weights are computed in fp32 with expf.
+ *
+ * logits: device, [N,E] row-major, dtype MOE_DTYPE_F32 or MOE_DTYPE_BF16.
+ * topk_idx: device int32 [N,K]; topk_w: device fp32 [N,K]; both written.
+ * 1 <= K <= min(E, 32), 1 <= E <= 1024.  Enqueued on stream, no sync; one
+ * kernel launch.  Returns MOE_ERR_ARG for bad sizes, modes, dtypes, null or
+ * misaligned pointers.
+ */
+#define MOE_ROUTER_SOFTMAX_TOPK 0
+#define MOE_ROUTER_TOPK_SOFTMAX 1
+#define MOE_ROUTER_TOPK_SOFTMAX_RENORM 2
+#define MOE_DTYPE_F32 0
+#define MOE_DTYPE_BF16 1
+
+MOE_API int moe_router_topk(const void *logits, int32_t logits_dtype, int64_t N, int32_t E, int32_t K,
+                            int32_t mode, int32_t *topk_idx, float *topk_w, moe_stream_t stream);
+
 /* Byte offsets of the workspace's internal arrays (for inspection and tests).
  * Offsets of arrays that the given sizes do not need are 0. */
 typedef struct moe_ws_layout_t {

@@ -53,7 +53,14 @@ EXPORTED = (
     "moe_nonexpand_routed_workspace_bytes",
     "moe_nonexpand_routed_metadata",
     "moe_nonexpand_routed_forward",
+    "moe_router_topk",
 )
+
+ROUTER_SOFTMAX_TOPK = 0
+ROUTER_TOPK_SOFTMAX = 1
+ROUTER_TOPK_SOFTMAX_RENORM = 2
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
 
 
 class MoeMeta(ctypes.Structure):
@@ -122,6 +129,8 @@ def load() -> ctypes.CDLL:
     lib.moe_nonexpand_routed_forward.restype = ctypes.c_int
     lib.moe_nonexpand_routed_forward.argtypes = [P, R, i32, i32, i32, P, P, P, P, i32, i32, P,
                                                  ctypes.POINTER(MoeMeta), P, sz, P]
+    lib.moe_router_topk.restype = ctypes.c_int
+    lib.moe_router_topk.argtypes = [P, i32, i64, i32, i32, i32, P, P, P]
     lib.moe_nonexpand_strerror.restype = ctypes.c_char_p
     lib.moe_nonexpand_strerror.argtypes = [ctypes.c_int]
     _lib = lib
@@ -469,3 +478,28 @@ def routed_forward(x: torch.Tensor, expert_idx: torch.Tensor, weights: torch.Ten
                                                ws.data_ptr(), ws.numel(), _stream_handle(stream)),
            "moe_nonexpand_routed_forward")
     return out
+
+
+# ---------------------------------------------------------------------------
+# Router top-k (moe_router_topk)
+# ---------------------------------------------------------------------------
+
+def router_topk(logits: torch.Tensor, K: int, mode: int = ROUTER_SOFTMAX_TOPK,
+                topk_idx: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                stream: Optional[torch.cuda.Stream] = None):
+    """Router logits [N,E] (fp32 or bf16) -> (topk_idx [N,K] int32, topk_w [N,K] fp32)."""
+    N, E = logits.shape
+    dev = logits.device
+    dtypes = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}
+    if logits.dtype not in dtypes:
+        raise TypeError(f"logits: expected float32 or bfloat16, got {logits.dtype}")
+    _need(logits, "logits", logits.dtype, (N, E), dev)
+    if topk_idx is None:
+        topk_idx = torch.empty((N, K), dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty((N, K), dtype=torch.float32, device=dev)
+    _need(topk_idx, "topk_idx", torch.int32, (N, K), dev)
+    _need(topk_w, "topk_w", torch.float32, (N, K), dev)
+    _check(load().moe_router_topk(logits.data_ptr(), dtypes[logits.dtype], N, E, K, mode, topk_idx.data_ptr(),
+                                  topk_w.data_ptr(), _stream_handle(stream)), "moe_router_topk")
+    return topk_idx, topk_w

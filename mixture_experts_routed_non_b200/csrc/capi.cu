@@ -564,6 +564,25 @@ extern "C" MOE_API int moe_nonexpand_combine(const void *y, const moe_meta_t *me
                : MOE_ERR_CUDA;
 }
 
+extern "C" MOE_API int moe_router_topk(const void *logits, int32_t logits_dtype, int64_t N, int32_t E, int32_t K,
+                                       int32_t mode, int32_t *topk_idx, float *topk_w, moe_stream_t stream) {
+    if (N < 0 || E < 1 || E > kMaxExperts || K < 1 || K > 32 || K > E) return MOE_ERR_ARG;
+    if (N * (int64_t)E >= ((int64_t)1 << 40)) return MOE_ERR_ARG;
+    if (logits_dtype != MOE_DTYPE_F32 && logits_dtype != MOE_DTYPE_BF16) return MOE_ERR_ARG;
+    if (mode != MOE_ROUTER_SOFTMAX_TOPK && mode != MOE_ROUTER_TOPK_SOFTMAX && mode != MOE_ROUTER_TOPK_SOFTMAX_RENORM)
+        return MOE_ERR_ARG;
+    if (N > 0 && (!logits || !topk_idx || !topk_w)) return MOE_ERR_ARG;
+    if (!aligned(logits, logits_dtype == MOE_DTYPE_F32 ? 4 : 2) || !aligned(topk_idx, 4) || !aligned(topk_w, 4))
+        return MOE_ERR_ARG;
+    DeviceInfo dev;
+    const int st = device_info(&dev);
+    if (st) return st;
+    return launch_router(logits, logits_dtype == MOE_DTYPE_BF16, N, E, K, mode, topk_idx, topk_w, dev.sms,
+                         reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
 extern "C" MOE_API int moe_nonexpand_read_error(const void *ws, moe_stream_t stream, uint32_t *err_word) {
     if (!ws || !err_word) return MOE_ERR_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -103,6 +103,8 @@ cudaError_t launch_gemm_down(const GemmArgs &a, int max_clusters, cudaStream_t s
 cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *token_offset, const int32_t *s_rev,
                            const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
                            const WsHeader *hdr, int num_sms, cudaStream_t s);
+cudaError_t launch_router(const void *logits, bool bf16, int64_t N, int E, int K, int mode, int32_t *idx, float *w,
+                          int num_sms, cudaStream_t s);
 size_t gemm_smem_bytes();
 
 // ---------------------------------------------------------------------------

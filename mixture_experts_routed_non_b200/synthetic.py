@@ -267,3 +267,17 @@ def many_pair_tokens(N: int, E: int, heavy: np.ndarray, K: int, rng: np.random.G
     tok = np.concatenate(toks)
     exp = np.concatenate(exps)
     return tok, exp, rng.random(tok.shape[0]).astype(np.float32)
+
+
+def make_logits(N: int, E: int, seed: int = 0, dtype=torch.float32, kind: str = "normal",
+                device="cpu") -> torch.Tensor:
+    """Router logits [N,E]: ``normal`` draws N(0,1) (distinct values in
+    practice); ``ties`` draws integers in [-2,2] (many equal logits per row)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    if kind == "normal":
+        a = rng.standard_normal((N, E)).astype(np.float32)
+    elif kind == "ties":
+        a = rng.integers(-2, 3, size=(N, E)).astype(np.float32)
+    else:
+        raise ValueError(kind)
+    return torch.from_numpy(a).to(dtype).to(device)

@@ -60,6 +60,8 @@ def _load(path: str | None = None):
         lib.oracle_metadata.argtypes = [i64, i32, i32, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_metadata_pairs.restype = i64
         lib.oracle_metadata_pairs.argtypes = [i64, i64, i32, P, P, P, P, P, P, P, P, P, P, P, P, P]
+        lib.oracle_router_topk.restype = None
+        lib.oracle_router_topk.argtypes = [i64, i32, i32, i32, P, P, P]
         lib.oracle_expert_row.restype = None
         lib.oracle_expert_row.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P]
         lib.oracle_forward_rows.restype = None
@@ -136,6 +138,28 @@ def metadata_pairs(token_idx: np.ndarray, expert_idx: np.ndarray, weights: np.nd
     return dict(freq=freq, off=off, x_gather_idx=xg[:P].copy(), s_scatter_idx=ss[:P].copy(),
                 s_reverse_scatter_idx=sr[:P].copy(), token_offset=to, scores=sc[:P].copy(),
                 P=int(P), bad_ids=int(bad[0]), bad_tokens=int(badt[0]), unsorted=bool(uns[0]))
+
+
+ROUTER_SOFTMAX_TOPK = 0
+ROUTER_TOPK_SOFTMAX = 1
+ROUTER_TOPK_SOFTMAX_RENORM = 2
+
+
+def router_topk(logits, K: int, mode: int = ROUTER_SOFTMAX_TOPK, lib_path: str | None = None):
+    """Router top-k of logits [N,E] (a torch fp32/bf16 tensor or a numpy
+    array; widened exactly to double, NaN read as -inf).  Returns
+    (topk_idx [N,K] int32, topk_w [N,K] float64)."""
+    lib = _load(lib_path)
+    if not isinstance(logits, np.ndarray):
+        import torch
+        logits = logits.detach().cpu().to(torch.float64).numpy()
+    lg = np.ascontiguousarray(logits, dtype=np.float64).copy()
+    lg[np.isnan(lg)] = -np.inf
+    N, E = lg.shape
+    idx = np.zeros((N, K), np.int32)
+    w = np.zeros((N, K), np.float64)
+    lib.oracle_router_topk(N, E, K, mode, _ptr(lg), _ptr(idx), _ptr(w))
+    return idx, w
 
 
 def expert_row(x_row, w1e, b1e, w2e, b2e, layout: int = LAYOUT_INTERLEAVED, lib_path: str | None = None):

@@ -199,6 +199,55 @@ int64_t oracle_metadata_pairs(int64_t N, int64_t P_list, int32_t E,
 }
 
 /* ------------------------------------------------------------------------
+ * Router top-k (sonic-moe write-up, "Three routing strategies, selected on
+ * the command line").  Per token, from its E logits:
+ *
+ *   chosen experts  the K largest logits, largest first; equal logits are
+ *                   taken in ascending expert id
+ *   mode 0          TC top-K: softmax over the K chosen logits
+ *   mode 1          Qwen3-style: softmax over all E logits, read at the chosen
+ *   mode 2          mode 1 divided by its sum over the K chosen
+ *
+ * logits are doubles (the caller widens fp32 or bf16 exactly and reads NaN
+ * as -inf); topk_w is double.
+ * ---------------------------------------------------------------------- */
+void oracle_router_topk(int64_t N, int32_t E, int32_t K, int32_t mode,
+                        const double *logits, int32_t *topk_idx, double *topk_w)
+{
+    char *taken = (char *)malloc((size_t)E);
+    for (int64_t t = 0; t < N; ++t) {
+        const double *row = logits + t * E;
+        int32_t *ix = topk_idx + t * K;
+        double *w = topk_w + t * K;
+        memset(taken, 0, (size_t)E);
+        /* the K largest, one at a time */
+        for (int32_t k = 0; k < K; ++k) {
+            int32_t best = -1;
+            for (int32_t e = 0; e < E; ++e)
+                if (!taken[e] && (best < 0 || row[e] > row[best])) best = e;
+            taken[best] = 1;
+            ix[k] = best;
+        }
+        const double top = row[ix[0]];
+        if (mode == 0) {
+            double s = 0.0;
+            for (int32_t k = 0; k < K; ++k) s += exp(row[ix[k]] - top);
+            for (int32_t k = 0; k < K; ++k) w[k] = exp(row[ix[k]] - top) / s;
+        } else {
+            double z = 0.0;
+            for (int32_t e = 0; e < E; ++e) z += exp(row[e] - top);
+            for (int32_t k = 0; k < K; ++k) w[k] = exp(row[ix[k]] - top) / z;
+            if (mode == 2) {
+                double s = 0.0;
+                for (int32_t k = 0; k < K; ++k) s += w[k];
+                for (int32_t k = 0; k < K; ++k) w[k] /= s;
+            }
+        }
+    }
+    free(taken);
+}
+
+/* ------------------------------------------------------------------------
  * One expert applied to one token row, in double.
  *   z   = x_t . W1[e] + b1[e]                       (2I values)
  *   h_j = silu(gate_j) * up_j,  silu(g) = g / (1 + exp(-g))

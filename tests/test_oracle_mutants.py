@@ -15,6 +15,7 @@ import pytest
 import oracle
 from mixture_experts_routed_non_b200 import synthetic
 from test_oracle_pairs import check_pair_fixture, check_table_equivalence
+from test_oracle_router import check_router_against_torch, check_router_fixture
 from test_oracle_pins import (GOLDEN, _bf, _load, _num, _recipe_torch_cpu,
                               check_metadata_invariants)
 
@@ -43,6 +44,13 @@ MUTANTS = {
     "pairs_bad_token_kept": ("if (t >= 0 && t < N) {", "if (t >= 0) {"),
     "pairs_sort_unstable": ("for (int64_t j = 0; j < q; ++j) {\n        int32_t p = cursor[pair_expert[j]]++;",
                             "for (int64_t j = q - 1; j >= 0; --j) {\n        int32_t p = cursor[pair_expert[j]]++;"),
+    "router_ties_to_higher_id": ("if (!taken[e] && (best < 0 || row[e] > row[best])) best = e;",
+                                 "if (!taken[e] && (best < 0 || row[e] >= row[best])) best = e;"),
+    "router_picks_smallest": ("if (!taken[e] && (best < 0 || row[e] > row[best])) best = e;",
+                              "if (!taken[e] && (best < 0 || row[e] < row[best])) best = e;"),
+    "router_topk_softmax_over_all": ("for (int32_t k = 0; k < K; ++k) s += exp(row[ix[k]] - top);",
+                                     "for (int32_t e = 0; e < E; ++e) s += exp(row[e] - top);"),
+    "router_no_renorm": ("if (mode == 2) {", "if (mode == 3) {"),
     "pairs_score_of_next": ("scores[q] = weights[i];", "scores[q] = weights[i + 1 < P_list ? i + 1 : i];"),
 }
 
@@ -85,6 +93,9 @@ def _pins_pass(lib):
             out_ex = [eval(s, env) for s in g["expected_closed_form"][key]["out"]]
             if not np.allclose(out[0], out_ex, rtol=1e-12, atol=1e-12):
                 return False
+        # router top-k: hand-worked closed forms, torch.topk / torch.softmax
+        check_router_fixture(lib)
+        check_router_against_torch(lib)
         # pair-list metadata: hand-worked fixture, table oracle on a flattened table
         check_pair_fixture(lib)
         wl = synthetic.WORKLOADS["tiny"]
