@@ -62,6 +62,10 @@ def _load(path: str | None = None):
         lib.oracle_metadata_pairs.argtypes = [i64, i64, i32, P, P, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_router_topk.restype = None
         lib.oracle_router_topk.argtypes = [i64, i32, i32, i32, P, P, P]
+        lib.oracle_pair_backward.restype = None
+        lib.oracle_pair_backward.argtypes = [i32, i32, i32, P, P, P, P, P, P, ctypes.c_double, P, P, P, P, P, P]
+        lib.oracle_pairs_backward.restype = None
+        lib.oracle_pairs_backward.argtypes = [i32, i32, i32, P, P, P, P, P, P, i64, P, P, P, P, P, P, P, P, i32]
         lib.oracle_expert_row.restype = None
         lib.oracle_expert_row.argtypes = [i32, i32, i32, P, P, P, P, P, P, P, P]
         lib.oracle_forward_rows.restype = None
@@ -241,3 +245,80 @@ def combine(token_offset: np.ndarray, s_rev: np.ndarray, scores: np.ndarray,
     out = np.zeros((N, H), np.float64)
     lib.oracle_combine(N, H, _ptr(to), _ptr(sr), _ptr(sc), _ptr(ys), _ptr(out))
     return out
+
+
+# ---------------------------------------------------------------------------
+# Backward (chain rule of the forward above, in double)
+# ---------------------------------------------------------------------------
+
+def _f64(t):
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return np.ascontiguousarray(t, dtype=np.float64)
+    import torch
+    return np.ascontiguousarray(t.detach().cpu().to(torch.float64).numpy())
+
+
+class WeightsF64:
+    """float64 copies of the dense inputs (bf16 values widened exactly)."""
+
+    def __init__(self, x, w1, b1, w2, b2):
+        self.x, self.w1, self.b1, self.w2, self.b2 = (_f64(v) for v in (x, w1, b1, w2, b2))
+        self.N, self.H = self.x.shape
+        self.E, _, two_i = self.w1.shape
+        self.I = two_i // 2
+
+
+def pairs_backward(wd: WeightsF64, dout, tokens, experts, scores, layout: int = LAYOUT_INTERLEAVED,
+                   n_threads: int = 0, lib_path: str | None = None) -> dict:
+    """Per pair (tokens[i], experts[i], scores[i]): h [n,I], y [n,H],
+    dy [n,H], dz [n,2I] and ds [n], all float64."""
+    lib = _load(lib_path)
+    do = _f64(dout)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    experts = np.ascontiguousarray(experts, dtype=np.int32)
+    scores = np.ascontiguousarray(scores, dtype=np.float64)
+    n = tokens.shape[0]
+    H, I = wd.H, wd.I
+    out = dict(h=np.zeros((n, I)), y=np.zeros((n, H)), dy=np.zeros((n, H)), dz=np.zeros((n, 2 * I)),
+               ds=np.zeros(n))
+    if n_threads <= 0:
+        n_threads = len(os.sched_getaffinity(0))
+    lib.oracle_pairs_backward(H, I, layout, _ptr(wd.x), _ptr(wd.w1), _ptr(wd.b1), _ptr(wd.w2), _ptr(wd.b2),
+                              _ptr(do), n, _ptr(tokens), _ptr(experts), _ptr(scores), _ptr(out["h"]),
+                              _ptr(out["y"]), _ptr(out["dy"]), _ptr(out["dz"]), _ptr(out["ds"]), n_threads)
+    return out
+
+
+def backward(wd: WeightsF64, topk_idx: np.ndarray, topk_w: np.ndarray, dout, layout: int = LAYOUT_INTERLEAVED,
+             experts_only=None, lib_path: str | None = None) -> dict:
+    """Gradients of sum_t <dout_t, out_t> for the [N,K] non-expand routing:
+    dx [N,H], dw1 [E,H,2I], db1 [E,2I], dw2 [E,I,H], db2 [E,H], dtopk_w [N,K]
+    (0 at invalid slots).  The per-pair terms come from pairs_backward; the
+    sums over pairs use float64 matrix products.  With ``experts_only`` only
+    those experts' pairs are computed (their weight gradients are complete;
+    dx and dtopk_w then hold only those pairs' shares)."""
+    idx = np.asarray(topk_idx)
+    w = np.asarray(topk_w)
+    N, K = idx.shape
+    H, I, E = wd.H, wd.I, wd.E
+    valid = (idx >= 0) & (idx < E)
+    if experts_only is not None:
+        valid &= np.isin(idx, np.asarray(experts_only))
+    tok, slot = np.nonzero(valid)
+    exp = idx[tok, slot].astype(np.int32)
+    sc = w[tok, slot].astype(np.float64)
+    r = pairs_backward(wd, dout, tok, exp, sc, layout, lib_path=lib_path)
+    g = dict(dx=np.zeros((N, H)), dw1=np.zeros((E, H, 2 * I)), db1=np.zeros((E, 2 * I)),
+             dw2=np.zeros((E, I, H)), db2=np.zeros((E, H)), dtopk_w=np.zeros((N, K)))
+    g["dtopk_w"][tok, slot] = r["ds"]
+    for e in np.unique(exp):
+        sel = exp == e
+        te = tok[sel]
+        g["dw2"][e] = r["h"][sel].T @ r["dy"][sel]
+        g["db2"][e] = r["dy"][sel].sum(0)
+        g["dw1"][e] = wd.x[te].T @ r["dz"][sel]
+        g["db1"][e] = r["dz"][sel].sum(0)
+        np.add.at(g["dx"], te, r["dz"][sel] @ wd.w1[e].T)
+    return g

@@ -384,3 +384,91 @@ void oracle_pair_rows(int32_t H, int32_t I, int32_t layout,
         free(z);
     }
 }
+
+/* ------------------------------------------------------------------------
+ * Backward of the local expert compute, in double (the pages leave the
+ * backward open; this is the chain rule applied to the forward above).
+ *
+ * For one pair (token row x, expert e, score s) and the output gradient dout
+ * of its token:
+ *   forward  z = x.W1[e] + b1[e];  h_j = silu(g_j) u_j;  y = h.W2[e] + b2[e]
+ *   dy   = s dout                      (the pair's share of out = sum s y)
+ *   ds   = <dout, y>                   (gradient of the score)
+ *   dh   = dy . W2[e]^T                (I values)
+ *   dg_j = dh_j u_j silu'(g_j),  silu'(g) = sig(g) (1 + g (1 - sig(g)))
+ *   du_j = dh_j silu(g_j)
+ *   dz   = (dg, du) at the gate/up columns of the layout
+ * The caller sums dW2[e] += h^T dy, db2[e] += dy, dW1[e] += x^T dz,
+ * db1[e] += dz and dx[t] += dz . W1[e]^T over the pairs.
+ *
+ * w1e [H][2I], w2e [I][H] row-major doubles; b1e / b2e may be NULL.
+ * ---------------------------------------------------------------------- */
+void oracle_pair_backward(int32_t H, int32_t I, int32_t layout,
+                          const double *x, const double *w1e, const double *b1e,
+                          const double *w2e, const double *b2e,
+                          const double *dout, double s,
+                          double *z, double *h, double *y, double *dy, double *dz, double *ds)
+{
+    for (int32_t j = 0; j < 2 * I; ++j) z[j] = b1e ? b1e[j] : 0.0;
+    for (int32_t k = 0; k < H; ++k) {
+        const double xv = x[k];
+        const double *wr = w1e + (size_t)k * 2 * I;
+        for (int32_t j = 0; j < 2 * I; ++j) z[j] += xv * wr[j];
+    }
+    for (int32_t j = 0; j < I; ++j) {
+        const int32_t gi = layout == 0 ? 2 * j : j, ui = layout == 0 ? 2 * j + 1 : I + j;
+        const double g = z[gi], u = z[ui];
+        h[j] = g / (1.0 + exp(-g)) * u;
+    }
+    for (int32_t n = 0; n < H; ++n) y[n] = b2e ? b2e[n] : 0.0;
+    for (int32_t j = 0; j < I; ++j) {
+        const double *wr = w2e + (size_t)j * H;
+        for (int32_t n = 0; n < H; ++n) y[n] += h[j] * wr[n];
+    }
+    double acc = 0.0;
+    for (int32_t n = 0; n < H; ++n) {
+        dy[n] = s * dout[n];
+        acc += dout[n] * y[n];
+    }
+    *ds = acc;
+    for (int32_t j = 0; j < I; ++j) {
+        const double *wr = w2e + (size_t)j * H;
+        double dh = 0.0;
+        for (int32_t n = 0; n < H; ++n) dh += dy[n] * wr[n];
+        const int32_t gi = layout == 0 ? 2 * j : j, ui = layout == 0 ? 2 * j + 1 : I + j;
+        const double g = z[gi], u = z[ui];
+        const double sig = 1.0 / (1.0 + exp(-g));
+        dz[gi] = dh * u * sig * (1.0 + g * (1.0 - sig));
+        dz[ui] = dh * g * sig;
+    }
+}
+
+/* oracle_pair_backward over n pairs (OpenMP).  x [N][H], w1 [E][H][2I],
+ * w2 [E][I][H], b1 [E][2I] / b2 [E][H] or NULL, dout [N][H]; pair i is
+ * (tokens[i], experts[i], scores[i]).  Outputs per pair: h [n][I], y [n][H],
+ * dy [n][H], dz [n][2I], ds [n]. */
+void oracle_pairs_backward(int32_t H, int32_t I, int32_t layout,
+                           const double *x, const double *w1, const double *b1,
+                           const double *w2, const double *b2, const double *dout,
+                           int64_t n, const int64_t *tokens, const int32_t *experts,
+                           const double *scores, double *h, double *y, double *dy,
+                           double *dz, double *ds, int32_t n_threads)
+{
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#endif
+#pragma omp parallel
+    {
+        double *z = (double *)malloc(sizeof(double) * (size_t)(2 * I));
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t i = 0; i < n; ++i) {
+            const int64_t t = tokens[i];
+            const int32_t e = experts[i];
+            oracle_pair_backward(H, I, layout, x + t * H, w1 + (size_t)e * H * 2 * I,
+                                 b1 ? b1 + (size_t)e * 2 * I : NULL, w2 + (size_t)e * I * H,
+                                 b2 ? b2 + (size_t)e * H : NULL, dout + t * H, scores[i],
+                                 z, h + i * I, y + i * H, dy + i * H, dz + i * 2 * I, ds + i);
+        }
+        free(z);
+    }
+}

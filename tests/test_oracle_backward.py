@@ -1,0 +1,157 @@
+"""Pins of the backward oracle (oracle.pairs_backward / oracle.backward).
+
+The pages leave the backward open (sonic-moe issue #68 asks how the routing
+scores get their gradient back to [N,K]); the oracle applies the chain rule
+to the forward.  Pinned by: its forward part against the pinned forward
+oracle; central finite differences of sum_t <dout_t, out_t> for every input;
+torch autograd through an independent float64 implementation of the
+sort-by-expert recipe (qwen3_5.py commit notes, steps 1-5).
+"""
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from mixture_experts_routed_non_b200 import synthetic
+
+GRADS = ("dx", "dw1", "db1", "dw2", "db2", "dtopk_w")
+
+
+def _small_problem(seed=0, layout=0):
+    rng = np.random.default_rng(seed)
+    N, H, I, E, K = 4, 8, 4, 3, 2
+    wd = oracle.WeightsF64(rng.standard_normal((N, H)), rng.standard_normal((E, H, 2 * I)) * 0.4,
+                           rng.standard_normal((E, 2 * I)) * 0.2, rng.standard_normal((E, I, H)) * 0.4,
+                           rng.standard_normal((E, H)) * 0.2)
+    idx = np.array([[0, 2], [1, -1], [2, 0], [-1, -1]], np.int32)
+    tw = rng.random((N, K))
+    dout = rng.standard_normal((N, H))
+    return wd, idx, tw, dout
+
+
+def _loss(wd, idx, tw, dout, layout, lib=None):
+    """sum_t <dout_t, out_t> with out from the oracle's double forward."""
+    N, K = idx.shape
+    tok, slot = np.nonzero(idx >= 0)
+    r = oracle.pairs_backward(wd, dout, tok, idx[tok, slot], tw[tok, slot], layout, lib_path=lib)
+    out = np.zeros((N, wd.H))
+    np.add.at(out, tok, tw[tok, slot][:, None] * r["y"])
+    return float((out * dout).sum())
+
+
+def check_finite_differences(layout, lib=None, eps=1e-6):
+    wd, idx, tw, dout = _small_problem(1, layout)
+    g = oracle.backward(wd, idx, tw, dout, layout, lib_path=lib)
+    fields = {"dx": (wd, "x"), "dw1": (wd, "w1"), "db1": (wd, "b1"), "dw2": (wd, "w2"), "db2": (wd, "b2")}
+    for gname, (obj, attr) in fields.items():
+        arr = getattr(obj, attr)
+        num = np.zeros_like(arr)
+        for i in np.ndindex(arr.shape):
+            keep = arr[i]
+            arr[i] = keep + eps
+            lp = _loss(wd, idx, tw, dout, layout, lib)
+            arr[i] = keep - eps
+            lm = _loss(wd, idx, tw, dout, layout, lib)
+            arr[i] = keep
+            num[i] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(g[gname], num, rtol=1e-6, atol=1e-7, err_msg=gname)
+    num = np.zeros_like(tw)
+    for i in np.ndindex(tw.shape):
+        if idx[i] < 0:
+            continue
+        keep = tw[i]
+        tw[i] = keep + eps
+        lp = _loss(wd, idx, tw, dout, layout, lib)
+        tw[i] = keep - eps
+        lm = _loss(wd, idx, tw, dout, layout, lib)
+        tw[i] = keep
+        num[i] = (lp - lm) / (2 * eps)
+    np.testing.assert_allclose(g["dtopk_w"], num, rtol=1e-6, atol=1e-7, err_msg="dtopk_w")
+
+
+def _recipe_autograd(inp, dout, layout):
+    """float64 torch autograd through the sort-by-expert recipe: flatten the
+    valid assignments, stable sort by expert, F.linear per expert slice,
+    silu x up, index_add_ of the score-weighted rows."""
+    x = inp.x.double().requires_grad_()
+    w1 = inp.w1.double().requires_grad_()
+    w2 = inp.w2.double().requires_grad_()
+    b1 = inp.b1.double().requires_grad_()
+    b2 = inp.b2.double().requires_grad_()
+    tw = inp.topk_w.double().requires_grad_()
+    idx = inp.topk_idx.long()
+    N, K = idx.shape
+    E, H, I2 = w1.shape
+    I = I2 // 2
+    flat_e = idx.reshape(-1)
+    flat_t = torch.arange(N).repeat_interleave(K)
+    flat_s = torch.arange(N * K)
+    keep = flat_e >= 0
+    flat_e, flat_t, flat_s = flat_e[keep], flat_t[keep], flat_s[keep]
+    order = torch.sort(flat_e, stable=True).indices
+    e_s, t_s, s_s = flat_e[order], flat_t[order], flat_s[order]
+    xs = x[t_s]
+    zs, ys = [], []
+    for e in range(E):
+        sel = e_s == e
+        zs.append(F.linear(xs[sel], w1[e].t(), b1[e]))
+    z = torch.cat(zs)
+    g, u = (z[:, 0::2], z[:, 1::2]) if layout == 0 else (z[:, :I], z[:, I:])
+    hs = F.silu(g) * u
+    start = 0
+    for e in range(E):
+        n = int((e_s == e).sum())
+        ys.append(F.linear(hs[start:start + n], w2[e].t(), b2[e]))
+        start += n
+    y = torch.cat(ys)
+    out = torch.zeros(N, H, dtype=torch.float64).index_add(0, t_s, y * tw.reshape(-1)[s_s][:, None])
+    out.backward(torch.from_numpy(dout))
+    return dict(dx=x.grad.numpy(), dw1=w1.grad.numpy(), db1=b1.grad.numpy(), dw2=w2.grad.numpy(),
+                db2=b2.grad.numpy(), dtopk_w=tw.grad.numpy())
+
+
+def check_autograd(layout, lib=None):
+    inp = synthetic.make_inputs("tiny", device="cpu")
+    dout = np.random.default_rng(2).standard_normal((inp.wl.N, inp.wl.H))
+    wd = oracle.WeightsF64(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    g = oracle.backward(wd, inp.topk_idx.numpy(), inp.topk_w.numpy(), dout, layout, lib_path=lib)
+    ref = _recipe_autograd(inp, dout, layout)
+    for k in GRADS:
+        np.testing.assert_allclose(g[k], ref[k], rtol=1e-9, atol=1e-10, err_msg=k)
+
+
+def test_backward_forward_part_matches_forward_oracle():
+    inp = synthetic.make_inputs("tiny", device="cpu")
+    wl = inp.wl
+    wd = oracle.WeightsF64(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    wts = oracle.Weights(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    idx = inp.topk_idx.numpy()
+    tok, slot = np.nonzero(idx >= 0)
+    tok, slot = tok[:200], slot[:200]
+    for layout in (0, 1):
+        r = oracle.pairs_backward(wd, np.zeros((wl.N, wl.H)), tok, idx[tok, slot], np.ones(len(tok)), layout)
+        h, y = oracle.pair_rows(wts, tok, idx[tok, slot], layout=layout)
+        np.testing.assert_allclose(r["h"], h, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(r["y"], y, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_backward_finite_differences(layout):
+    check_finite_differences(layout)
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_backward_matches_torch_autograd(layout):
+    check_autograd(layout)
+
+
+def test_backward_experts_only_is_complete_for_those_experts():
+    inp = synthetic.make_inputs("tiny", device="cpu")
+    dout = np.random.default_rng(4).standard_normal((inp.wl.N, inp.wl.H))
+    wd = oracle.WeightsF64(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    idx, w = inp.topk_idx.numpy(), inp.topk_w.numpy()
+    full = oracle.backward(wd, idx, w, dout)
+    part = oracle.backward(wd, idx, w, dout, experts_only=[3, 5])
+    for k in ("dw1", "db1", "dw2", "db2"):
+        np.testing.assert_array_equal(part[k][[3, 5]], full[k][[3, 5]])

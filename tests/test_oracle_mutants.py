@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 from mixture_experts_routed_non_b200 import synthetic
+from test_oracle_backward import check_autograd, check_finite_differences
 from test_oracle_pairs import check_pair_fixture, check_table_equivalence
 from test_oracle_router import check_router_against_torch, check_router_fixture
 from test_oracle_pins import (GOLDEN, _bf, _load, _num, _recipe_torch_cpu,
@@ -51,6 +52,12 @@ MUTANTS = {
     "router_topk_softmax_over_all": ("for (int32_t k = 0; k < K; ++k) s += exp(row[ix[k]] - top);",
                                      "for (int32_t e = 0; e < E; ++e) s += exp(row[e] - top);"),
     "router_no_renorm": ("if (mode == 2) {", "if (mode == 3) {"),
+    "bwd_silu_derivative": ("dz[gi] = dh * u * sig * (1.0 + g * (1.0 - sig));", "dz[gi] = dh * u * sig;"),
+    "bwd_gate_up_swapped": ("dz[ui] = dh * g * sig;", "dz[ui] = dh * u * sig;"),
+    "bwd_score_dropped": ("dy[n] = s * dout[n];", "dy[n] = dout[n];"),
+    "bwd_score_grad_of_dy": ("acc += dout[n] * y[n];", "acc += dy[n] * y[n];"),
+    "bwd_w2_not_transposed": ("for (int32_t n = 0; n < H; ++n) dh += dy[n] * wr[n];",
+                              "for (int32_t n = 0; n < H; ++n) dh += dy[n] * w2e[(size_t)n * I + j];"),
     "pairs_score_of_next": ("scores[q] = weights[i];", "scores[q] = weights[i + 1 < P_list ? i + 1 : i];"),
 }
 
@@ -93,6 +100,9 @@ def _pins_pass(lib):
             out_ex = [eval(s, env) for s in g["expected_closed_form"][key]["out"]]
             if not np.allclose(out[0], out_ex, rtol=1e-12, atol=1e-12):
                 return False
+        # backward: finite differences, torch autograd through the recipe
+        check_finite_differences(0, lib)
+        check_autograd(1, lib)
         # router top-k: hand-worked closed forms, torch.topk / torch.softmax
         check_router_fixture(lib)
         check_router_against_torch(lib)
