@@ -263,6 +263,68 @@ MOE_API int moe_nonexpand_routed_forward(const void *x, const moe_routing_t *rou
                                  const moe_meta_t *meta_out, void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Training: forward that keeps what the backward needs, and the backward.
+ *
+ * The pages leave the backward open (sonic-moe issue #68 asks how the routing
+ * scores' gradient gets back to [N_recv,K]; the write-up names the layer a
+ * training layer).  These calls apply the chain rule to the forward above,
+ * for the non-expand [N,K] routing:
+ *   dy_q  = s_q dout_t               (the pair's share of out_t = sum_q s_q y_q)
+ *   ds_q  = <dout_t, y_q>            -> dtopk_w[t,k] of the slot of q (0 at invalid slots)
+ *   dh_q  = dy_q . W2[e]^T
+ *   dg    = dh u silu'(g), du = dh silu(g), silu'(g) = sig(g)(1 + g(1 - sig(g)))
+ *   dz_q  = (dg, du) at the gate/up columns of the layout
+ *   dW2[e] = sum h_q^T dy_q,  db2[e] = sum dy_q,
+ *   dW1[e] = sum x_t^T dz_q,  db1[e] = sum dz_q,  dx_t = sum over t's pairs of dz_q . W1[e]^T
+ * (sums over the pairs q of expert e, or of token t).
+ *
+ * moe_nonexpand_train_workspace_bytes: a larger workspace that also holds z
+ * (fp32 [P_cap,2I], bias included: the SwiGLU derivative is sensitive to the
+ * gate's precision near silu's minimum), dz (bf16 [P_cap,2I]) and dy (bf16
+ * [P_cap,H]).
+ *
+ * moe_nonexpand_forward_train: moe_nonexpand_forward that keeps the metadata,
+ * h, y and z in the training workspace for the backward.
+ *
+ * moe_nonexpand_backward: the gradients, given dout [N,H] bf16 and the
+ * training workspace of a forward_train call with the same x, routing,
+ * weights, layout and sizes (nothing in between may use that workspace).
+ * Outputs (device, caller-owned, all written): dx [N,H], dw1 [E,H,2I],
+ * dw2 [E,I,H] bf16; dtopk_w [N,K] fp32; db1 [E,2I] and db2 [E,H] bf16 when
+ * not NULL.  The workspace's dy, dz and y regions are overwritten.  Products
+ * accumulate in fp32; dh is computed from dout and the weights (bf16 inputs)
+ * with the score applied in fp32; dy, dz and the per-pair dx rows are stored
+ * in bf16.
+ * Deterministic: no atomics decide any sum.  Enqueued on stream, no sync.
+ * Same return codes as moe_nonexpand_forward; MOE_ERR_WS for a workspace
+ * smaller than the training size.
+ */
+MOE_API size_t moe_nonexpand_train_workspace_bytes(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
+                                                   int64_t total_pairs);
+
+MOE_API int moe_nonexpand_forward_train(const void *x, const int32_t *topk_idx, const float *topk_w, int64_t N,
+                                        int32_t H, int32_t I, int32_t E, int32_t K, int64_t total_pairs,
+                                        const void *w1, const void *b1, const void *w2, const void *b2,
+                                        int32_t activation, int32_t gate_up_layout, void *out, void *ws,
+                                        size_t ws_bytes, moe_stream_t stream);
+
+MOE_API int moe_nonexpand_backward(const void *dout, const void *x, const int32_t *topk_idx, const float *topk_w,
+                                   int64_t N, int32_t H, int32_t I, int32_t E, int32_t K, int64_t total_pairs,
+                                   const void *w1, const void *w2, int32_t activation, int32_t gate_up_layout,
+                                   void *dx, void *dw1, void *db1, void *dw2, void *db2, float *dtopk_w,
+                                   void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_nonexpand_backward plus eight events recorded on the stream around its
+ * seven steps: score gradients and dy, dh + SwiGLU backward, dW2, dx rows,
+ * dW1, the dx combine, the bias gradients. */
+MOE_API int moe_nonexpand_backward_timed(const void *dout, const void *x, const int32_t *topk_idx,
+                                         const float *topk_w, int64_t N, int32_t H, int32_t I, int32_t E,
+                                         int32_t K, int64_t total_pairs, const void *w1, const void *w2,
+                                         int32_t activation, int32_t gate_up_layout, void *dx, void *dw1,
+                                         void *db1, void *dw2, void *db2, float *dtopk_w, void *ws,
+                                         size_t ws_bytes, moe_stream_t stream, const moe_event_t *stage_events);
+
+/*
  * Router top-k: router logits [N,E] -> the routing table topk_idx [N,K] /
  * topk_w [N,K] that moe_nonexpand_forward takes (sonic-moe write-up, "Three
  * routing strategies, selected on the command line": TC top-K routing is the
@@ -311,6 +373,10 @@ typedef struct moe_ws_layout_t {
     int64_t p_cap;
     int32_t meta_tiles;        /* T */
     int32_t meta_tile_slots;   /* slots per metadata tile */
+    size_t z;                  /* training workspace: fp32 [P_cap,2I], z saved by the forward */
+    size_t dz;                 /* training workspace: bf16 [P_cap,2I], dz of the backward */
+    size_t dy;                 /* training workspace: bf16 [P_cap,H], dy of the backward */
+    size_t train_total;        /* == moe_nonexpand_train_workspace_bytes(...) */
 } moe_ws_layout_t;
 
 MOE_API int moe_nonexpand_workspace_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,

@@ -54,6 +54,10 @@ EXPORTED = (
     "moe_nonexpand_routed_metadata",
     "moe_nonexpand_routed_forward",
     "moe_router_topk",
+    "moe_nonexpand_train_workspace_bytes",
+    "moe_nonexpand_forward_train",
+    "moe_nonexpand_backward",
+    "moe_nonexpand_backward_timed",
 )
 
 ROUTER_SOFTMAX_TOPK = 0
@@ -74,7 +78,9 @@ class WsLayout(ctypes.Structure):
         "total", "header", "tile_hist", "tile_valid", "tile_err", "gemm_tile_offset",
         "meta_freq", "meta_off", "meta_x_gather", "meta_s_scatter", "meta_s_rev",
         "meta_token_offset", "meta_scores", "h", "y")] + [
-        ("p_cap", ctypes.c_int64), ("meta_tiles", ctypes.c_int32), ("meta_tile_slots", ctypes.c_int32)]
+        ("p_cap", ctypes.c_int64), ("meta_tiles", ctypes.c_int32), ("meta_tile_slots", ctypes.c_int32),
+        ("z", ctypes.c_size_t), ("dz", ctypes.c_size_t), ("dy", ctypes.c_size_t),
+        ("train_total", ctypes.c_size_t)]
 
 
 class MoeRouting(ctypes.Structure):
@@ -131,6 +137,16 @@ def load() -> ctypes.CDLL:
                                                  ctypes.POINTER(MoeMeta), P, sz, P]
     lib.moe_router_topk.restype = ctypes.c_int
     lib.moe_router_topk.argtypes = [P, i32, i64, i32, i32, i32, P, P, P]
+    lib.moe_nonexpand_train_workspace_bytes.restype = sz
+    lib.moe_nonexpand_train_workspace_bytes.argtypes = [i64, i32, i32, i32, i32, i64]
+    lib.moe_nonexpand_forward_train.restype = ctypes.c_int
+    lib.moe_nonexpand_forward_train.argtypes = [P, P, P, i64, i32, i32, i32, i32, i64, P, P, P, P, i32, i32, P, P,
+                                                sz, P]
+    bwd = [P, P, P, P, i64, i32, i32, i32, i32, i64, P, P, i32, i32, P, P, P, P, P, P, P, sz, P]
+    lib.moe_nonexpand_backward.restype = ctypes.c_int
+    lib.moe_nonexpand_backward.argtypes = bwd
+    lib.moe_nonexpand_backward_timed.restype = ctypes.c_int
+    lib.moe_nonexpand_backward_timed.argtypes = bwd + [P]
     lib.moe_nonexpand_strerror.restype = ctypes.c_char_p
     lib.moe_nonexpand_strerror.argtypes = [ctypes.c_int]
     _lib = lib
@@ -503,3 +519,90 @@ def router_topk(logits: torch.Tensor, K: int, mode: int = ROUTER_SOFTMAX_TOPK,
     _check(load().moe_router_topk(logits.data_ptr(), dtypes[logits.dtype], N, E, K, mode, topk_idx.data_ptr(),
                                   topk_w.data_ptr(), _stream_handle(stream)), "moe_router_topk")
     return topk_idx, topk_w
+
+
+# ---------------------------------------------------------------------------
+# Training: forward that keeps z, and the backward
+# ---------------------------------------------------------------------------
+
+def train_workspace_bytes(N: int, H: int, I: int, E: int, K: int, total_pairs: int = -1) -> int:
+    n = load().moe_nonexpand_train_workspace_bytes(N, H, I, E, K, total_pairs)
+    if n == 0:
+        raise MoeError(MOE_ERR_ARG, "moe_nonexpand_train_workspace_bytes")
+    return n
+
+
+def alloc_train_workspace(N: int, H: int, I: int, E: int, K: int, total_pairs: int = -1,
+                          device=None) -> torch.Tensor:
+    n = train_workspace_bytes(N, H, I, E, K, total_pairs)
+    return torch.empty(n, dtype=torch.uint8, device=device or torch.device("cuda"))
+
+
+def forward_train(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor, w1: torch.Tensor,
+                  w2: torch.Tensor, b1: Optional[torch.Tensor] = None, b2: Optional[torch.Tensor] = None, *,
+                  ws: torch.Tensor, layout: int = LAYOUT_INTERLEAVED, total_pairs: int = -1,
+                  out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """moe_nonexpand_forward_train: the forward, keeping metadata, h, y and z
+    in ``ws`` (see alloc_train_workspace) for ``backward``."""
+    N, H = x.shape
+    K = topk_idx.shape[1]
+    E, _, I2 = w1.shape
+    I = I2 // 2
+    dev = x.device
+    _need(x, "x", torch.bfloat16, (N, H), dev)
+    _need(topk_idx, "topk_idx", torch.int32, (N, K), dev)
+    _need(topk_w, "topk_w", torch.float32, (N, K), dev)
+    _need(w1, "w1", torch.bfloat16, (E, H, 2 * I), dev)
+    _need(w2, "w2", torch.bfloat16, (E, I, H), dev)
+    if b1 is not None:
+        _need(b1, "b1", torch.bfloat16, (E, 2 * I), dev)
+    if b2 is not None:
+        _need(b2, "b2", torch.bfloat16, (E, H), dev)
+    if out is None:
+        out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (N, H), dev)
+    _check(load().moe_nonexpand_forward_train(x.data_ptr(), topk_idx.data_ptr(), topk_w.data_ptr(), N, H, I, E, K,
+                                              total_pairs, w1.data_ptr(), _ptr(b1), w2.data_ptr(), _ptr(b2),
+                                              ACT_SWIGLU, layout, out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                              _stream_handle(stream)), "moe_nonexpand_forward_train")
+    return out
+
+
+def backward(dout: torch.Tensor, x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,
+             w1: torch.Tensor, w2: torch.Tensor, *, ws: torch.Tensor, layout: int = LAYOUT_INTERLEAVED,
+             total_pairs: int = -1, bias_grads: bool = False, stream: Optional[torch.cuda.Stream] = None,
+             events: Optional[Sequence[torch.cuda.Event]] = None, grads: Optional[dict] = None) -> dict:
+    """moe_nonexpand_backward after forward_train on the same ``ws``.  Returns
+    dict(dx, dw1, dw2, dtopk_w[, db1, db2]).  ``events`` (eight timing
+    events) bracket its seven steps."""
+    N, H = x.shape
+    K = topk_idx.shape[1]
+    E, _, I2 = w1.shape
+    I = I2 // 2
+    dev = x.device
+    _need(dout, "dout", torch.bfloat16, (N, H), dev)
+    if grads is None:
+        grads = dict(dx=torch.empty((N, H), dtype=torch.bfloat16, device=dev),
+                     dw1=torch.empty((E, H, 2 * I), dtype=torch.bfloat16, device=dev),
+                     dw2=torch.empty((E, I, H), dtype=torch.bfloat16, device=dev),
+                     dtopk_w=torch.empty((N, K), dtype=torch.float32, device=dev))
+        if bias_grads:
+            grads["db1"] = torch.empty((E, 2 * I), dtype=torch.bfloat16, device=dev)
+            grads["db2"] = torch.empty((E, H), dtype=torch.bfloat16, device=dev)
+    args = (dout.data_ptr(), x.data_ptr(), topk_idx.data_ptr(), topk_w.data_ptr(), N, H, I, E, K, total_pairs,
+            w1.data_ptr(), w2.data_ptr(), ACT_SWIGLU, layout, grads["dx"].data_ptr(), grads["dw1"].data_ptr(),
+            _ptr(grads.get("db1")), grads["dw2"].data_ptr(), _ptr(grads.get("db2")), grads["dtopk_w"].data_ptr(),
+            ws.data_ptr(), ws.numel(), _stream_handle(stream))
+    lib = load()
+    if events is None:
+        _check(lib.moe_nonexpand_backward(*args), "moe_nonexpand_backward")
+    else:
+        if len(events) != 8:
+            raise ValueError("events: expected 8 CUDA events")
+        s = stream if stream is not None else torch.cuda.current_stream()
+        for ev in events:
+            if not ev.cuda_event:
+                ev.record(s)
+        arr = (ctypes.c_void_p * 8)(*[ev.cuda_event for ev in events])
+        _check(lib.moe_nonexpand_backward_timed(*args, arr), "moe_nonexpand_backward_timed")
+    return grads

@@ -1,0 +1,156 @@
+// Memory-bound steps of the backward (the GEMMs are in
+// grouped_gemm_bwd_sm100.cu; the pages leave the backward open, so these are
+// the chain rule of the forward):
+//
+//   prep      per token t and each of its pairs q (sorted position p):
+//             ds_q = <dout_t, y_p> (the score's gradient, fp32, summed in a
+//             fixed order) and dy_p = s_q dout_t (bf16 [P_cap,H]); ds is then
+//             scattered to the [N,K] slot it came from (0 at invalid slots) --
+//             sonic-moe issue #68 asks for the scores' gradient back in the
+//             non-expand layout.
+//   bias      db[e,c] = sum of the segment's rows of dy (db2) or dz (db1), in
+//             row order, fp32, rounded once to bf16.
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kPrepThreads = 256;
+constexpr int kPrepWarps = kPrepThreads / 32;
+constexpr int kMaxSlots = 32;
+
+__device__ __forceinline__ float dot8(const uint4 &a, const uint4 &b) {
+    return bf16lo(a.x) * bf16lo(b.x) + bf16hi(a.x) * bf16hi(b.x) + bf16lo(a.y) * bf16lo(b.y) +
+           bf16hi(a.y) * bf16hi(b.y) + bf16lo(a.z) * bf16lo(b.z) + bf16hi(a.z) * bf16hi(b.z) +
+           bf16lo(a.w) * bf16lo(b.w) + bf16hi(a.w) * bf16hi(b.w);
+}
+
+__device__ __forceinline__ uint4 scale8(const uint4 &v, float s) {
+    return make_uint4(pack_bf16x2(s * bf16lo(v.x), s * bf16hi(v.x)), pack_bf16x2(s * bf16lo(v.y), s * bf16hi(v.y)),
+                      pack_bf16x2(s * bf16lo(v.z), s * bf16hi(v.z)), pack_bf16x2(s * bf16lo(v.w), s * bf16hi(v.w)));
+}
+
+// One block per token (grid-stride).  Each thread owns 16-byte column chunks
+// of the row; per pair it accumulates its share of the dot product, then the
+// block reduces all pairs' partials at once (warp butterfly, then warps in
+// order).
+__global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
+    const __nv_bfloat16 *__restrict__ dout, const __nv_bfloat16 *__restrict__ y, const int32_t *__restrict__ topk_idx,
+    const int32_t *__restrict__ token_offset, const int32_t *__restrict__ s_rev, const float *__restrict__ scores,
+    int64_t N, int32_t H, int32_t K, int32_t E, __nv_bfloat16 *__restrict__ dy, float *__restrict__ dtopk_w,
+    const WsHeader *hdr) {
+    __shared__ float part[kPrepWarps][kMaxSlots];
+    __shared__ float ds_s[kMaxSlots];
+    if (hdr && *(volatile const uint32_t *)&hdr->abort) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int chunks = H >> 3;
+    for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
+        const int q0 = __ldg(token_offset + t), q1 = __ldg(token_offset + t + 1);
+        const int np = q1 - q0;  // <= K
+        const __nv_bfloat16 *drow = dout + (size_t)t * H;
+        float acc[kMaxSlots];
+#pragma unroll
+        for (int j = 0; j < kMaxSlots; ++j) acc[j] = 0.f;
+        for (int c = threadIdx.x; c < chunks; c += kPrepThreads) {
+            const uint4 d = __ldg(reinterpret_cast<const uint4 *>(drow) + c);
+#pragma unroll
+            for (int j = 0; j < kMaxSlots; ++j) {
+                if (j >= np) break;
+                const int p = __ldg(s_rev + q0 + j);
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + (size_t)p * H) + c);
+                acc[j] += dot8(d, v);
+                reinterpret_cast<uint4 *>(dy + (size_t)p * H)[c] = scale8(d, __ldg(scores + q0 + j));
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxSlots; ++j) {
+            if (j >= np) break;
+            float v = acc[j];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) part[warp][j] = v;
+        }
+        __syncthreads();
+        if (threadIdx.x < np) {
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < kPrepWarps; ++w) v += part[w][threadIdx.x];
+            ds_s[threadIdx.x] = v;
+        }
+        __syncthreads();
+        if (threadIdx.x < K) {
+            // the j-th valid slot of the row holds pair q0 + j
+            const int32_t *row = topk_idx + (size_t)t * K;
+            const int k = threadIdx.x;
+            const int e = __ldg(row + k);
+            float g = 0.f;
+            if (e >= 0 && e < E) {
+                int j = 0;
+                for (int kk = 0; kk < k; ++kk) {
+                    const int ek = __ldg(row + kk);
+                    j += (ek >= 0 && ek < E) ? 1 : 0;
+                }
+                g = j < np ? ds_s[j] : 0.f;
+            }
+            dtopk_w[(size_t)t * K + k] = g;
+        }
+        __syncthreads();  // part / ds_s are reused by the next token
+    }
+}
+
+// db[e, c] = sum over rows p in [off[e], off[e+1]) of src[p, c]; one thread per
+// column pair, rows in order.
+__global__ void __launch_bounds__(256) bias_grad_kernel(const __nv_bfloat16 *__restrict__ src, int32_t cols,
+                                                        const int32_t *__restrict__ expert_off,
+                                                        __nv_bfloat16 *__restrict__ db, const WsHeader *hdr) {
+    if (hdr && *(volatile const uint32_t *)&hdr->abort) return;
+    const int e = blockIdx.y;
+    const int c2 = blockIdx.x * blockDim.x + threadIdx.x;  // column pair
+    if (2 * c2 >= cols) return;
+    const int p0 = __ldg(expert_off + e), p1 = __ldg(expert_off + e + 1);
+    float s0 = 0.f, s1 = 0.f;
+    const uint32_t *base = reinterpret_cast<const uint32_t *>(src) + c2;
+    const int ld = cols >> 1;
+    int p = p0;
+    for (; p + 4 <= p1; p += 4) {
+        uint32_t v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = __ldg(base + (size_t)(p + u) * ld);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            s0 += bf16lo(v[u]);
+            s1 += bf16hi(v[u]);
+        }
+    }
+    for (; p < p1; ++p) {
+        const uint32_t v = __ldg(base + (size_t)p * ld);
+        s0 += bf16lo(v);
+        s1 += bf16hi(v);
+    }
+    reinterpret_cast<uint32_t *>(db + (size_t)e * cols)[c2] = pack_bf16x2(s0, s1);
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const __nv_bfloat16 *y, const int32_t *topk_idx,
+                            const moe_meta_t &meta, int64_t N, int32_t H, int32_t K, int32_t E, __nv_bfloat16 *dy,
+                            float *dtopk_w, const WsHeader *hdr, int num_sms, cudaStream_t s) {
+    if (N == 0) return cudaSuccess;
+    int64_t blocks = N;
+    const int64_t cap = (int64_t)num_sms * 8;
+    if (blocks > cap) blocks = cap;
+    bwd_prep_kernel<<<(unsigned)blocks, kPrepThreads, 0, s>>>(dout, y, topk_idx, meta.token_offset,
+                                                              meta.s_reverse_scatter_idx, meta.scores, N, H, K, E,
+                                                              dy, dtopk_w, hdr);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bias_grad(const __nv_bfloat16 *src, int32_t cols, const int32_t *expert_off, int32_t E,
+                             __nv_bfloat16 *db, const WsHeader *hdr, cudaStream_t s) {
+    const dim3 grid((unsigned)((cols / 2 + 255) / 256), (unsigned)E);
+    bias_grad_kernel<<<grid, 256, 0, s>>>(src, cols, expert_off, db, hdr);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -94,6 +94,15 @@ moe_ws_layout_t compute_layout_nk(int64_t N, int32_t H, int32_t I, int32_t E, in
         o = align_up(o + (size_t)pc * H * 2, 1024);
     }
     l.total = o;
+    if (H > 0 && I > 0) {  // training: z (fp32), dz and dy after the inference workspace
+        l.z = o;
+        o = align_up(o + (size_t)pc * 2 * I * 4, 1024);
+        l.dz = o;
+        o = align_up(o + (size_t)pc * 2 * I * 2, 1024);
+        l.dy = o;
+        o = align_up(o + (size_t)pc * H * 2, 1024);
+    }
+    l.train_total = o;
     return l;
 }
 
@@ -335,7 +344,7 @@ int record(const moe_event_t *ev, int i, cudaStream_t s) {
 int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t E, const void *w1,
                  const void *b1, const void *w2, const void *b2, int32_t activation, int32_t layout_kind,
                  void *out, const moe_meta_t *meta_out, void *ws, size_t ws_bytes, cudaStream_t s,
-                 const moe_event_t *ev) {
+                 const moe_event_t *ev, bool train = false) {
     const int64_t N = r.N;
     int st = MOE_OK;
     // with N == 0 the token-sized buffers may be empty (null)
@@ -350,7 +359,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
     const moe_ws_layout_t l = compute_layout_nk(N, H, I, E, r.NK, r.p_cap);
     st = check_dense(l.p_cap, H, I, E);
     if (st) return st;
-    if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MOE_ERR_WS;
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < (train ? l.train_total : l.total)) return MOE_ERR_WS;
     DeviceInfo dev;
     st = device_info(&dev);
     if (st) return st;
@@ -383,6 +392,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         up.tile_off = ma.gemm_tile_off;
         up.bias = static_cast<const __nv_bfloat16 *>(b1);
         up.out = hbuf;
+        up.z_out = train ? reinterpret_cast<float *>(w + l.z) : nullptr;
         up.hdr = hdr;
         up.E = E;
         up.k_dim = H;
@@ -431,10 +441,179 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
     return MOE_OK;
 }
 
+int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, const float *topk_w, int64_t N,
+                  int32_t H, int32_t I, int32_t E, int32_t K, int64_t total_pairs, const void *w1, const void *w2,
+                  int32_t activation, int32_t layout_kind, void *dx, void *dw1, void *db1, void *dw2, void *db2,
+                  float *dtopk_w, void *ws, size_t ws_bytes, cudaStream_t s, const moe_event_t *ev) {
+    int st = check_sizes(N, E, K, total_pairs);
+    if (st) return st;
+    if ((N > 0 && (!dout || !x || !topk_idx || !topk_w || !dx || !dtopk_w)) || !w1 || !w2 || !dw1 || !dw2)
+        return MOE_ERR_ARG;
+    if (activation != MOE_ACT_SWIGLU) return MOE_ERR_ARG;
+    if (layout_kind != MOE_LAYOUT_INTERLEAVED && layout_kind != MOE_LAYOUT_CONCATENATED) return MOE_ERR_ARG;
+    if (!aligned(dout, 16) || !aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(dx, 16) ||
+        !aligned(dw1, 16) || !aligned(dw2, 16) || (db1 && !aligned(db1, 16)) || (db2 && !aligned(db2, 16)) ||
+        !aligned(topk_idx, 4) || !aligned(topk_w, 4) || !aligned(dtopk_w, 4))
+        return MOE_ERR_ARG;
+    const moe_ws_layout_t l = compute_layout(N, H, I, E, K, total_pairs);
+    st = check_dense(l.p_cap, H, I, E);
+    if (st) return st;
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < l.train_total) return MOE_ERR_WS;
+    DeviceInfo dev;
+    st = device_info(&dev);
+    if (st) return st;
+
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    const moe_meta_t meta = ws_meta(l, w);
+    WsHeader *hdr = reinterpret_cast<WsHeader *>(w + l.header);
+    auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16 *>(w + off); };
+    __nv_bfloat16 *hbuf = bf(l.h), *ybuf = bf(l.y), *dzbuf = bf(l.dz), *dybuf = bf(l.dy);
+    const float *zbuf = reinterpret_cast<const float *>(w + l.z);
+    const __nv_bfloat16 *w1b = static_cast<const __nv_bfloat16 *>(w1);
+    const __nv_bfloat16 *w2b = static_cast<const __nv_bfloat16 *>(w2);
+
+    if ((st = record(ev, 0, s))) return st;
+    // score gradients (to the [N,K] slots) and dy = s dout per pair
+    if (launch_bwd_prep(static_cast<const __nv_bfloat16 *>(dout), ybuf, topk_idx, meta, N, H, K, E, dybuf, dtopk_w,
+                        hdr, dev.sms, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if ((st = record(ev, 1, s))) return st;
+
+    BwdGemmArgs g;
+    memset(&g, 0, sizeof g);
+    g.expert_off = meta.expert_frequency_offset;
+    g.hdr = hdr;
+    g.E = E;
+    g.I = I;
+    g.layout = layout_kind;
+    // dh = s (dout[x_gather_idx] . W2[e]^T), SwiGLU backward: z -> dz
+    {
+        BwdGemmArgs a = g;
+        a.a = static_cast<const __nv_bfloat16 *>(dout);
+        a.a_rows = meta.x_gather_idx;
+        a.a_ld = H;
+        a.b = w2b;
+        a.b_ld = H;
+        a.b_estride = (int64_t)I * H;
+        a.z = zbuf;
+        a.dz = dzbuf;
+        a.row_scale = meta.scores;
+        a.row_pair = meta.s_scatter_idx;
+        a.N_dim = I;
+        a.K_dim = H;
+        if (launch_gemm_bwd(kBwdDH, a, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if ((st = record(ev, 2, s))) return st;
+    // dW2[e] = h^T dy
+    {
+        BwdGemmArgs a = g;
+        a.a = hbuf;
+        a.a_ld = I;
+        a.b = dybuf;
+        a.b_ld = H;
+        a.out = static_cast<__nv_bfloat16 *>(dw2);
+        a.out_ld = H;
+        a.M_dim = I;
+        a.N_dim = H;
+        if (launch_gemm_bwd(kBwdDW, a, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if ((st = record(ev, 3, s))) return st;
+    // dx rows = dz . W1[e]^T, into the (no longer needed) y region
+    {
+        BwdGemmArgs a = g;
+        a.a = dzbuf;
+        a.a_ld = 2 * I;
+        a.b = w1b;
+        a.b_ld = 2 * I;
+        a.b_estride = (int64_t)H * 2 * I;
+        a.out = ybuf;
+        a.out_ld = H;
+        a.N_dim = H;
+        a.K_dim = 2 * I;
+        if (launch_gemm_bwd(kBwdDX, a, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if ((st = record(ev, 4, s))) return st;
+    // dW1[e] = x[x_gather_idx]^T dz
+    {
+        BwdGemmArgs a = g;
+        a.a = static_cast<const __nv_bfloat16 *>(x);
+        a.a_rows = meta.x_gather_idx;
+        a.a_ld = H;
+        a.b = dzbuf;
+        a.b_ld = 2 * I;
+        a.out = static_cast<__nv_bfloat16 *>(dw1);
+        a.out_ld = 2 * I;
+        a.M_dim = H;
+        a.N_dim = 2 * I;
+        if (launch_gemm_bwd(kBwdDW, a, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if ((st = record(ev, 5, s))) return st;
+    // dx[t] = sum of its pairs' dx rows (weight 1)
+    if (launch_combine(ybuf, meta.token_offset, meta.s_reverse_scatter_idx, nullptr, N, H,
+                       static_cast<__nv_bfloat16 *>(dx), hdr, dev.sms, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if ((st = record(ev, 6, s))) return st;
+    if (db2 && launch_bias_grad(dybuf, H, meta.expert_frequency_offset, E, static_cast<__nv_bfloat16 *>(db2), hdr,
+                                s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (db1 && launch_bias_grad(dzbuf, 2 * I, meta.expert_frequency_offset, E, static_cast<__nv_bfloat16 *>(db1),
+                                hdr, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if ((st = record(ev, 7, s))) return st;
+    return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
 using namespace moe;
+
+extern "C" MOE_API size_t moe_nonexpand_train_workspace_bytes(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
+                                                              int64_t total_pairs) {
+    if (check_sizes(N, E, K, total_pairs)) return 0;
+    if (H <= 0 || I <= 0) return 0;
+    const moe_ws_layout_t l = compute_layout(N, H, I, E, K, total_pairs);
+    if (check_dense(l.p_cap, H, I, E)) return 0;
+    return l.train_total;
+}
+
+extern "C" MOE_API int moe_nonexpand_forward_train(const void *x, const int32_t *topk_idx, const float *topk_w,
+                                                   int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
+                                                   int64_t total_pairs, const void *w1, const void *b1,
+                                                   const void *w2, const void *b2, int32_t activation,
+                                                   int32_t gate_up_layout, void *out, void *ws, size_t ws_bytes,
+                                                   moe_stream_t stream) {
+    int st = check_sizes(N, E, K, total_pairs);
+    if (st) return st;
+    if (!aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_ARG;
+    return forward_impl(x, routing_topk32(topk_idx, topk_w, N, K, total_pairs), H, I, E, w1, b1, w2, b2,
+                        activation, gate_up_layout, out, nullptr, ws, ws_bytes,
+                        reinterpret_cast<cudaStream_t>(stream), nullptr, true);
+}
+
+extern "C" MOE_API int moe_nonexpand_backward(const void *dout, const void *x, const int32_t *topk_idx,
+                                              const float *topk_w, int64_t N, int32_t H, int32_t I, int32_t E,
+                                              int32_t K, int64_t total_pairs, const void *w1, const void *w2,
+                                              int32_t activation, int32_t gate_up_layout, void *dx, void *dw1,
+                                              void *db1, void *dw2, void *db2, float *dtopk_w, void *ws,
+                                              size_t ws_bytes, moe_stream_t stream) {
+    return backward_impl(dout, x, topk_idx, topk_w, N, H, I, E, K, total_pairs, w1, w2, activation, gate_up_layout,
+                         dx, dw1, db1, dw2, db2, dtopk_w, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                         nullptr);
+}
+
+extern "C" MOE_API int moe_nonexpand_backward_timed(const void *dout, const void *x, const int32_t *topk_idx,
+                                                    const float *topk_w, int64_t N, int32_t H, int32_t I,
+                                                    int32_t E, int32_t K, int64_t total_pairs, const void *w1,
+                                                    const void *w2, int32_t activation, int32_t gate_up_layout,
+                                                    void *dx, void *dw1, void *db1, void *dw2, void *db2,
+                                                    float *dtopk_w, void *ws, size_t ws_bytes, moe_stream_t stream,
+                                                    const moe_event_t *stage_events) {
+    if (!stage_events) return MOE_ERR_ARG;
+    return backward_impl(dout, x, topk_idx, topk_w, N, H, I, E, K, total_pairs, w1, w2, activation, gate_up_layout,
+                         dx, dw1, db1, dw2, db2, dtopk_w, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
+                         stage_events);
+}
 
 extern "C" MOE_API size_t moe_nonexpand_workspace_bytes(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
                                              int64_t total_pairs) {

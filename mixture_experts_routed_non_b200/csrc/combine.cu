@@ -1,4 +1,5 @@
-// Score-weighted combine back to token order (sonic-moe issue #68 dataflow:
+// Score-weighted combine back to token order (with null scores every weight
+// is 1: the backward sums a token's dx rows the same way) (sonic-moe issue #68 dataflow:
 // the local expert compute ends in local_out [N,H]; the qwen3_5.py commit
 // notes, recipe step 5, scatter the expert rows back to their tokens).
 //
@@ -92,7 +93,7 @@ __device__ __forceinline__ void combine_tokens(const __nv_bfloat16 *__restrict__
                     ++j;
                     tok_end = s_off[j + 1] - qa;
                 }
-                fma8(acc, kStaged ? pw[q] : __ldg(pw + q), v[u]);
+                fma8(acc, kStaged ? pw[q] : (pw ? __ldg(pw + q) : 1.f), v[u]);
             }
         }
         for (; j < nt; ++j) {  // the last token with pairs, then trailing tokens without
@@ -123,12 +124,12 @@ __global__ void __launch_bounds__(kCombineThreads, 4) combine_kernel(
         if (np <= kStagedPairs) {
             for (int i = threadIdx.x; i < np; i += kCombineThreads) {
                 s_p[i] = __ldg(s_rev + qa + i);
-                s_w[i] = __ldg(scores + qa + i);
+                s_w[i] = scores ? __ldg(scores + qa + i) : 1.f;
             }
             __syncthreads();
             combine_tokens<true>(y, s_p, s_w, s_off, qa, np, nt, H, out_t0);
         } else {  // more pairs than the staging arrays hold (a pair list may give a token any number)
-            combine_tokens<false>(y, s_rev + qa, scores + qa, s_off, qa, np, nt, H, out_t0);
+            combine_tokens<false>(y, s_rev + qa, scores ? scores + qa : nullptr, s_off, qa, np, nt, H, out_t0);
         }
         __syncthreads();  // shared indices are reused by the next group
     }

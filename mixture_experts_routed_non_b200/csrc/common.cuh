@@ -86,6 +86,7 @@ struct GemmArgs {
     const int32_t *tile_off;      // [E+1]
     const __nv_bfloat16 *bias;    // b1 [E,2I] / b2 [E,H] or null
     __nv_bfloat16 *out;           // h [P_cap,I] / y [P_cap,H]
+    float *z_out;                 // up, training: z [P_cap,2I] fp32 (bias added, W1 column order) or null
     WsHeader *hdr;
     int32_t E;
     int32_t k_dim;        // H (up) / I (down)
@@ -94,6 +95,36 @@ struct GemmArgs {
     int32_t out_cols;     // I (up) / H (down)
     int32_t I;            // intermediate size (up, concatenated layout)
     int32_t layout;       // MOE_LAYOUT_*
+};
+
+// Backward grouped GEMMs (one CTA per tile, M=128 x N=256, cp.async operands).
+enum BwdMode : int32_t {
+    kBwdDH = 0,  // dz = SwiGLU'(z) applied to s * (dout[x_gather_idx[p]] . W2[e]^T)
+    kBwdDX = 1,  // dxs[P,H] = dz[P,2I] . W1[e]^T
+    kBwdDW = 2,  // out[e] [M,N] = sum over the segment's rows p of A[p,:]^T B[p,:]
+};
+
+struct BwdGemmArgs {
+    const __nv_bfloat16 *a;    // DH: dout [N,H]; DX: dz [P_cap,2I]; DW: rows of length M_dim
+    const int32_t *a_rows;     // DH/DW: row of `a` for segment row p (null: p itself)
+    int64_t a_ld;              // elements per row of `a`
+    const __nv_bfloat16 *b;    // DH/DX: weights [E][N][K] (K contiguous); DW: [P_cap, N_dim] rows p
+    int64_t b_ld;              // elements per row of `b`
+    int64_t b_estride;         // DH/DX: elements between experts of `b`
+    const int32_t *expert_off; // [E+1] segment offsets
+    __nv_bfloat16 *out;        // DX: [P_cap, N]; DW: [E][M][N]; DH: unused (writes z)
+    int64_t out_ld;
+    const float *z;            // DH: z [P_cap, 2I] fp32 (saved by the training forward)
+    __nv_bfloat16 *dz;         // DH: dz [P_cap, 2I] out
+    const float *row_scale;    // DH: scores in pair order, read at s_scatter_idx[p]
+    const int32_t *row_pair;   // DH: s_scatter_idx (sorted position -> pair)
+    WsHeader *hdr;
+    int32_t E;
+    int32_t M_dim;             // DW: rows of each expert's output
+    int32_t N_dim;             // columns of the output (DH: I)
+    int32_t K_dim;             // DH/DX: reduction length (multiple of 64)
+    int32_t I;                 // DH: intermediate size
+    int32_t layout;            // DH: MOE_LAYOUT_*
 };
 
 // Launchers (each defined next to its kernel).
@@ -106,6 +137,12 @@ cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *token_offset, 
 cudaError_t launch_router(const void *logits, bool bf16, int64_t N, int E, int K, int mode, int32_t *idx, float *w,
                           int num_sms, cudaStream_t s);
 size_t gemm_smem_bytes();
+cudaError_t launch_gemm_bwd(int mode, const BwdGemmArgs &a, int max_ctas, cudaStream_t s);
+cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const __nv_bfloat16 *y, const int32_t *topk_idx,
+                            const moe_meta_t &meta, int64_t N, int32_t H, int32_t K, int32_t E, __nv_bfloat16 *dy,
+                            float *dtopk_w, const WsHeader *hdr, int num_sms, cudaStream_t s);
+cudaError_t launch_bias_grad(const __nv_bfloat16 *src, int32_t cols, const int32_t *expert_off, int32_t E,
+                             __nv_bfloat16 *db, const WsHeader *hdr, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Device primitives.
@@ -227,6 +264,11 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const void *tmap, uint
 // --- cp.async (16-byte, L2 only) feeding shared memory ----------------------
 __device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// 16-byte copy that reads src_bytes (0 or 16) and zero-fills the rest.
+__device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
 }
 // Arrive on `bar` once every cp.async this thread issued so far has landed
 // (the arrival is one of the barrier's expected arrivals).

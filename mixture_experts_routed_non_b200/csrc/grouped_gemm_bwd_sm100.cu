@@ -1,0 +1,493 @@
+// Grouped GEMMs of the backward on sm_100a: tcgen05 MMAs (cta_group::1,
+// M=128 x N=256 x K=16) with TMEM accumulators, operands staged in shared
+// memory by cp.async producer warps.  The pages leave the backward open
+// (sonic-moe issue #68 asks how the scores' gradient returns to [N,K]; the
+// write-up names the layer a training layer); these are the chain rule of the
+// forward, over the same expert-sorted segments:
+//
+//   DH  dh = s_p (dout[x_gather_idx[p],:] . W2[e]^T)  (K = H, N = I; the
+//       A rows are gathered from dout and the score applied in fp32, so dh
+//       sees no rounded operand), then the SwiGLU backward in the epilogue:
+//       with (g, u) read from the fp32 z the training forward saved,
+//       dg = dh u silu'(g), du = dh silu(g), written as bf16 dz at the
+//       gate/up columns of the layout (so dz keeps W1's column order).
+//   DX  dxs[p,:] = dz[p,:] . W1[e]^T  (K = 2I, N = H).
+//   DW  out[e] = sum over the rows p of segment e of A[p,:]^T B[p,:]:
+//       dW2[e] = h^T dy (A = h, B = dy) and dW1[e] = x[x_gather_idx]^T dz
+//       (A = x rows gathered by token, B = dz).  K is the segment length; the
+//       rows past its end are zero-filled in both operands.
+//
+// DH and DX tile the segments in 128-row tiles (the tile table is rebuilt in
+// each CTA from the expert offsets); DW tiles each expert's [M,N] output.
+// Operands: K-major (rows of 64 contiguous K values, 128-byte swizzle) for
+// the row operands of DH/DX and for the weights read as [N][K]; MN-major
+// (rows = K, 64-element MN atoms, 128-byte swizzle) for both DW operands.
+// Warp roles: warp 0 = TMEM allocator and MMA issuer, warps 1-4 = epilogue
+// (TMEM lane quarter warp % 4), warps 5-8 = cp.async producers.  Four
+// shared-memory stages, two TMEM accumulators.  Every wait is bounded; on a
+// timeout the CTA raises its abort flag, records MOE_DEVERR_TIMEOUT, drains
+// its MMAs and copies and frees its TMEM.
+#include "common.cuh"
+
+namespace moe {
+
+namespace {
+
+constexpr int kM = 128;                      // tile rows (TMEM lanes)
+constexpr int kN = 256;                      // tile columns (UMMA N)
+constexpr int kSK = 64;                      // K per stage: one 128-byte swizzle atom of bf16
+constexpr int kBwdStages = 4;
+constexpr int kProducerThreads = 128;
+constexpr int kThreads = 32 + 128 + kProducerThreads;
+constexpr uint32_t kStageA = kM * kSK * 2;   // 16 KB
+constexpr uint32_t kStageB = kN * kSK * 2;   // 32 KB
+constexpr uint32_t kStageBytes = kStageA + kStageB;
+constexpr uint32_t kMnAtom = kSK * 128;      // MN-major: one 64-element column of a stage (8 KB)
+constexpr uint32_t kTmemCols = 2 * kN;
+constexpr uint32_t kNumBars = 2 * kBwdStages + 5;
+constexpr size_t kSmemBarOff = (size_t)kBwdStages * kStageBytes;
+constexpr size_t kSmemMiscOff = kSmemBarOff + 8 * kNumBars;
+constexpr size_t kSmemTableOff = kSmemMiscOff + 16;
+constexpr size_t kSmemBytes = 1024 + kSmemTableOff + 2 * (kMaxExperts + 1) * 4;
+constexpr unsigned long long kAbortSettleNs = 2000000ull;
+
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, M x N,
+// each operand K-major or MN-major.
+__host__ __device__ constexpr uint32_t idesc(bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(kN >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
+}
+
+struct BTile {
+    int e, m0, m_end, n0, nk;   // DW: m0 = output row, m_end = M_dim; segment rows via kp0/kp1
+    int kp0, kp1;               // DW: segment rows [kp0, kp1)
+};
+
+// DH/DX: tile -> (expert, 128-row tile of its segment, 256-column tile)
+__device__ __forceinline__ BTile decode_rows(int tile, int n_tiles, int E, const int *tile_off, const int *off,
+                                             int K_dim) {
+    BTile t;
+    const int mt = tile / n_tiles;
+    const int nt = tile - mt * n_tiles;
+    int lo = 0, hi = E - 1;  // largest e with tile_off[e] <= mt
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tile_off[mid] <= mt) lo = mid;
+        else hi = mid - 1;
+    }
+    t.e = lo;
+    t.m0 = off[lo] + (mt - tile_off[lo]) * kM;
+    t.m_end = off[lo + 1];
+    t.n0 = nt * kN;
+    t.nk = K_dim / kSK;
+    t.kp0 = t.kp1 = 0;
+    return t;
+}
+
+// DW: tile -> (expert, 128-row tile of its [M,N] output, 256-column tile)
+__device__ __forceinline__ BTile decode_weights(int tile, int m_tiles, int n_tiles, const int *off) {
+    BTile t;
+    const int per = m_tiles * n_tiles;
+    t.e = tile / per;
+    const int r = tile - t.e * per;
+    const int mt = r / n_tiles;
+    t.m0 = mt * kM;
+    t.n0 = (r - mt * n_tiles) * kN;
+    t.kp0 = off[t.e];
+    t.kp1 = off[t.e + 1];
+    t.nk = (t.kp1 - t.kp0 + kSK - 1) / kSK;
+    t.m_end = 0;
+    return t;
+}
+
+__device__ __forceinline__ void settle_after_abort() {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < kAbortSettleNs) {
+    }
+}
+
+__device__ __forceinline__ float silu_f(float g, float &sig) {
+    sig = 1.0f / (1.0f + __expf(-g));
+    return g * sig;
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_constant__ BwdGemmArgs a) {
+    constexpr bool kMN = kMode == kBwdDW;  // both operands MN-major, K = segment rows
+    constexpr uint32_t kIdesc = idesc(kMN, kMN);
+    extern __shared__ uint8_t smem_raw[];
+    if (*(volatile uint32_t *)&a.hdr->abort) return;  // an earlier step of this call gave up
+
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *base_ptr = smem_raw + (base - raw);
+    auto a_stage = [&](int s) { return base + (uint32_t)s * kStageBytes; };
+    auto b_stage = [&](int s) { return base + (uint32_t)s * kStageBytes + kStageA; };
+    const uint32_t bars = base + (uint32_t)kSmemBarOff;
+    auto full_bar = [&](int s) { return bars + 8u * s; };
+    auto empty_bar = [&](int s) { return bars + 8u * (kBwdStages + s); };
+    auto tfull_bar = [&](int b) { return bars + 8u * (2 * kBwdStages + b); };
+    auto tempty_bar = [&](int b) { return bars + 8u * (2 * kBwdStages + 2 + b); };
+    const uint32_t drain_bar = bars + 8u * (2 * kBwdStages + 4);
+    uint32_t *misc = reinterpret_cast<uint32_t *>(base_ptr + kSmemMiscOff);
+    int *tile_off_s = reinterpret_cast<int *>(base_ptr + kSmemTableOff);
+    int *off_s = tile_off_s + (kMaxExperts + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = a.E;
+    for (int i = threadIdx.x; i <= E; i += kThreads) off_s[i] = __ldg(a.expert_off + i);
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kBwdStages; ++s) {
+            mbar_init(full_bar(s), kProducerThreads);
+            mbar_init(empty_bar(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull_bar(b), 1);
+            mbar_init(tempty_bar(b), 4);
+        }
+        mbar_init(drain_bar, 1);
+        misc[1] = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (!kMN && warp == 1) {
+        // 128-row tiles per expert, exclusive prefix (one warp)
+        const int per = (E + 31) / 32;
+        const int e0 = lane * per;
+        int sum = 0;
+        for (int i = 0; i < per; ++i) {
+            const int e = e0 + i;
+            if (e < E) sum += (off_s[e + 1] - off_s[e] + kM - 1) / kM;
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        int run = incl - sum;
+        for (int i = 0; i < per; ++i) {
+            const int e = e0 + i;
+            if (e < E) {
+                tile_off_s[e] = run;
+                run += (off_s[e + 1] - off_s[e] + kM - 1) / kM;
+            }
+        }
+        if (lane == 31) tile_off_s[E] = incl;
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&misc[0]), kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = misc[0];
+    volatile uint32_t *abort = &misc[1];
+    const int n_tiles = (a.N_dim + kN - 1) / kN;
+    const int m_tiles = kMN ? (a.M_dim + kM - 1) / kM : 0;
+    const int total = kMN ? E * m_tiles * n_tiles : tile_off_s[E] * n_tiles;
+    auto decode = [&](int tile) {
+        return kMN ? decode_weights(tile, m_tiles, n_tiles, off_s)
+                   : decode_rows(tile, n_tiles, E, tile_off_s, off_s, a.K_dim);
+    };
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int tcount = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++tcount) {
+                const BTile t = decode(tile);
+                const int acc = tcount & 1;
+                const uint32_t acc_phase = (tcount >> 1) & 1;
+                if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * kN;
+                for (int kb = 0; kb < t.nk; ++kb) {
+                    if (!mbar_wait_bounded(full_bar(stage), phase, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    fence_proxy_async_smem();  // cp.async (generic proxy) data -> tensor-core reads
+                    const uint32_t sa = a_stage(stage), sb = b_stage(stage);
+#pragma unroll
+                    for (int kk = 0; kk < kSK / kUmmaK; ++kk) {
+                        uint64_t ad, bd;
+                        if (kMN) {
+                            // rows = K (128 B each, 8-row groups 1024 B apart), 64-element
+                            // MN columns kMnAtom apart; K step = 16 rows
+                            ad = smem_desc_sw128(sa + kk * (kUmmaK * 128), kMnAtom, 1024);
+                            bd = smem_desc_sw128(sb + kk * (kUmmaK * 128), kMnAtom, 1024);
+                        } else {
+                            // rows = M or N (128 B of K each, 8-row groups 1024 B apart);
+                            // K step = 32 B inside the swizzle atom
+                            ad = smem_desc_sw128(sa + kk * (kUmmaK * 2), 16, 1024);
+                            bd = smem_desc_sw128(sb + kk * (kUmmaK * 2), 16, 1024);
+                        }
+                        umma_f16(d_tmem, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(empty_bar(stage));
+                    if (++stage == kBwdStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(tfull_bar(acc));  // with no MMA (empty segment) it arrives at once
+            }
+            umma_commit(drain_bar);  // every MMA issued here completes before TMEM is freed
+            mbar_wait_timed(drain_bar, 0);
+        }
+        __syncwarp();
+    } else if (warp < 5) {
+        // ------------------------------------------------------------ epilogue
+        const int quarter = warp & 3;
+        const int rl = quarter * 32 + lane;  // this thread's tile row (TMEM lane)
+        int tcount = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+            const BTile t = decode(tile);
+            const int acc = tcount & 1;
+            const uint32_t acc_phase = (tcount >> 1) & 1;
+            bool w = true;
+            if (lane == 0) w = mbar_wait_bounded(tfull_bar(acc), acc_phase, abort);
+            w = __shfl_sync(0xffffffffu, w, 0);
+            if (!w) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + acc * kN + ((uint32_t)(quarter * 32) << 16);
+            if (kMode == kBwdDH) {
+                const int p = t.m0 + rl;
+                const bool valid = p < t.m_end;
+                const size_t zoff = (size_t)(valid ? p : 0) * (2 * a.I);
+                const float *zrow = a.z + zoff;
+                __nv_bfloat16 *dzrow = a.dz + zoff;
+                // the pair's score: dh = s (dout . W2^T)
+                const float sc = valid ? __ldg(a.row_scale + __ldg(a.row_pair + p)) : 0.f;
+#pragma unroll 1
+                for (int c = 0; c < kN / 32; ++c) {
+                    const int i0 = t.n0 + 32 * c;
+                    if (i0 >= a.I) break;
+                    uint32_t dh[32];
+                    tmem_ld_32x32b_x32(tbase + c * 32, dh);
+                    tmem_ld_wait();
+                    if (!valid) continue;
+                    if (a.layout == MOE_LAYOUT_INTERLEAVED) {
+                        // (g_i, u_i) adjacent: 32 pairs = 64 fp32 in, 64 bf16 out
+                        const float4 *zp = reinterpret_cast<const float4 *>(zrow + 2 * i0);
+                        uint4 *dp = reinterpret_cast<uint4 *>(dzrow + 2 * i0);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            const float4 z0 = zp[2 * q], z1 = zp[2 * q + 1];
+                            const float g[4] = {z0.x, z0.z, z1.x, z1.z};
+                            const float u[4] = {z0.y, z0.w, z1.y, z1.w};
+                            uint32_t o[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float d = sc * __uint_as_float(dh[4 * q + j]);
+                                float sig;
+                                const float sl = silu_f(g[j], sig);
+                                o[j] = pack_bf16x2(d * u[j] * sig * (1.0f + g[j] * (1.0f - sig)), d * sl);
+                            }
+                            dp[q] = make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                    } else {
+                        // gates at [i0, i0+32), ups at [I+i0, I+i0+32)
+                        const float4 *gp = reinterpret_cast<const float4 *>(zrow + i0);
+                        const float4 *up = reinterpret_cast<const float4 *>(zrow + a.I + i0);
+                        uint4 *dg_out = reinterpret_cast<uint4 *>(dzrow + i0);
+                        uint4 *du_out = reinterpret_cast<uint4 *>(dzrow + a.I + i0);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float4 g0 = gp[2 * q], g1 = gp[2 * q + 1];
+                            const float4 u0 = up[2 * q], u1 = up[2 * q + 1];
+                            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                            const float u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+                            float dg[8], du[8];
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) {
+                                const float d = sc * __uint_as_float(dh[8 * q + j]);
+                                float sig;
+                                const float sl = silu_f(g[j], sig);
+                                dg[j] = d * u[j] * sig * (1.0f + g[j] * (1.0f - sig));
+                                du[j] = d * sl;
+                            }
+                            dg_out[q] = make_uint4(pack_bf16x2(dg[0], dg[1]), pack_bf16x2(dg[2], dg[3]),
+                                                   pack_bf16x2(dg[4], dg[5]), pack_bf16x2(dg[6], dg[7]));
+                            du_out[q] = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]),
+                                                   pack_bf16x2(du[4], du[5]), pack_bf16x2(du[6], du[7]));
+                        }
+                    }
+                }
+            } else {
+                // DX: row p of dxs; DW: row m of expert e's [M,N] output
+                const int r = kMode == kBwdDX ? t.m0 + rl : t.m0 + rl;
+                const bool valid = kMode == kBwdDX ? r < t.m_end : r < a.M_dim;
+                const size_t row_off = kMode == kBwdDX
+                                           ? (size_t)(valid ? r : 0) * a.out_ld
+                                           : ((size_t)t.e * a.M_dim + (valid ? r : 0)) * a.out_ld;
+                __nv_bfloat16 *orow = a.out + row_off;
+                const bool zero = kMode == kBwdDW && t.nk == 0;  // empty segment: the gradient is 0
+#pragma unroll 1
+                for (int g = 0; g < kN / 64; ++g) {
+                    const int col0 = t.n0 + 64 * g;
+                    if (col0 >= a.N_dim) break;
+                    uint32_t r0[32], r1[32];
+                    if (!zero) {
+                        tmem_ld_32x32b_x32(tbase + g * 64, r0);
+                        tmem_ld_32x32b_x32(tbase + g * 64 + 32, r1);
+                        tmem_ld_wait();
+                    }
+                    if (!valid) continue;
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + col0);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t o[4], o2[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            o[j] = zero ? 0u
+                                        : pack_bf16x2(__uint_as_float(r0[8 * q + 2 * j]),
+                                                      __uint_as_float(r0[8 * q + 2 * j + 1]));
+                            o2[j] = zero ? 0u
+                                         : pack_bf16x2(__uint_as_float(r1[8 * q + 2 * j]),
+                                                       __uint_as_float(r1[8 * q + 2 * j + 1]));
+                        }
+                        dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
+                        dst[4 + q] = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(tempty_bar(acc));
+        }
+    } else {
+        // ------------------------------------------------------------ producers
+        const int pt = threadIdx.x - 160;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        const int gl = pt & 31;
+        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            const BTile t = decode(tile);
+            for (int kb = 0; kb < t.nk; ++kb) {
+                bool w = true;
+                if (gl == 0) w = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort);
+                w = __shfl_sync(0xffffffffu, w, 0);
+                if (!w) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = a_stage(stage), sb = b_stage(stage);
+                if (!kMN) {
+                    // K-major rows: 8 chunks of 16 B per 128-byte row, swizzled by row & 7
+                    const int c = pt & 7, r0 = pt >> 3;
+                    const int k0 = kb * kSK + 8 * c;
+#pragma unroll
+                    for (int i = 0; i < kM / 16; ++i) {
+                        const int r = r0 + 16 * i;
+                        const int p = t.m0 + r;  // rows past the segment end feed unstored rows only
+                        if (p < t.m_end) {
+                            const int row = a.a_rows ? __ldg(a.a_rows + p) : p;
+                            cp_async_16(sa + r * 128 + ((c ^ (r & 7)) << 4), a.a + (size_t)row * a.a_ld + k0);
+                        }
+                    }
+                    const __nv_bfloat16 *bw = a.b + (size_t)t.e * a.b_estride;
+#pragma unroll
+                    for (int i = 0; i < kN / 16; ++i) {
+                        const int r = r0 + 16 * i;
+                        const int n = t.n0 + r;  // columns past N_dim are never stored
+                        if (n < a.N_dim)
+                            cp_async_16(sb + r * 128 + ((c ^ (r & 7)) << 4), bw + (size_t)n * a.b_ld + k0);
+                    }
+                } else {
+                    // MN-major: row kr of the stage = segment row p; rows past the
+                    // segment end are zero in both operands
+                    const int kbase = t.kp0 + kb * kSK;
+                    {
+                        const int c = pt & 15, kr0 = pt >> 4;  // 16 chunks per 128-element A row
+                        const int m = t.m0 + 8 * c;
+#pragma unroll
+                        for (int i = 0; i < kSK / 8; ++i) {
+                            const int kr = kr0 + 8 * i;
+                            const int p = kbase + kr;
+                            const bool in = p < t.kp1;
+                            const uint32_t dst = sa + (c >> 3) * kMnAtom + kr * 128 + (((c & 7) ^ (kr & 7)) << 4);
+                            if (m < a.M_dim) {
+                                const int row = in ? (a.a_rows ? __ldg(a.a_rows + p) : p) : 0;
+                                cp_async_16_zfill(dst, a.a + (size_t)row * a.a_ld + m, in ? 16u : 0u);
+                            }
+                        }
+                    }
+                    {
+                        const int c = pt & 31, kr0 = pt >> 5;  // 32 chunks per 256-element B row
+                        const int n = t.n0 + 8 * c;
+#pragma unroll
+                        for (int i = 0; i < kSK / 4; ++i) {
+                            const int kr = kr0 + 4 * i;
+                            const int p = kbase + kr;
+                            const bool in = p < t.kp1;
+                            const uint32_t dst = sb + (c >> 3) * kMnAtom + kr * 128 + (((c & 7) ^ (kr & 7)) << 4);
+                            if (n < a.N_dim)
+                                cp_async_16_zfill(dst, a.b + (size_t)(in ? p : 0) * a.b_ld + n, in ? 16u : 0u);
+                        }
+                    }
+                }
+                cp_async_arrive_noinc(full_bar(stage));
+                if (++stage == kBwdStages) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        cp_async_wait_all();
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (*abort) {
+        if (threadIdx.x == 0) atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);
+        settle_after_abort();
+    }
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+template <int kMode>
+cudaError_t launch_mode(const BwdGemmArgs &a, int max_ctas, cudaStream_t s) {
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev >= 64) return cudaErrorInvalidDevice;
+    if (!configured[dev]) {
+        err = cudaFuncSetAttribute(bwd_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kSmemBytes);
+        if (err != cudaSuccess) return err;
+        configured[dev] = true;
+    }
+    int ctas = max_ctas;
+    if (kMode == kBwdDW) {
+        const int total = a.E * ((a.M_dim + kM - 1) / kM) * ((a.N_dim + kN - 1) / kN);
+        if (total < ctas) ctas = total;
+    }
+    if (ctas < 1) ctas = 1;
+    bwd_gemm_kernel<kMode><<<ctas, kThreads, kSmemBytes, s>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_bwd(int mode, const BwdGemmArgs &a, int max_ctas, cudaStream_t s) {
+    if (mode == kBwdDH) return launch_mode<kBwdDH>(a, max_ctas, s);
+    if (mode == kBwdDX) return launch_mode<kBwdDX>(a, max_ctas, s);
+    return launch_mode<kBwdDW>(a, max_ctas, s);
+}
+
+}  // namespace moe

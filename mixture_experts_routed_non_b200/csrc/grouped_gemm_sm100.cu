@@ -116,6 +116,13 @@ __device__ __forceinline__ void add_bias32(uint32_t (&r)[32], const __nv_bfloat1
     }
 }
 
+// 32 fp32 values (as bits) to dst (128 bytes, 16-byte aligned)
+__device__ __forceinline__ void store_f32x32(float *dst, const uint32_t (&r)[32]) {
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) d[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+}
+
 __device__ __forceinline__ void settle_after_abort() {
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < kAbortSettleNs) {
@@ -395,6 +402,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                             add_bias32(g, brow + col0 + hf * 32);
                             add_bias32(u, brow + a.I + col0 + hf * 32);
                         }
+                        if (a.z_out && valid) {  // training: keep z for the backward
+                            float *zr = a.z_out + (size_t)p * (2 * a.I);
+                            store_f32x32(zr + col0 + hf * 32, g);
+                            store_f32x32(zr + a.I + col0 + hf * 32, u);
+                        }
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const float h0 = silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]));
@@ -423,6 +435,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                         if (brow) {
                             add_bias32(r0, brow + acol);
                             add_bias32(r1, brow + acol + 32);
+                        }
+                        if (a.z_out && valid) {  // training: keep z for the backward
+                            float *zr = a.z_out + (size_t)p * (2 * a.I);
+                            store_f32x32(zr + acol, r0);
+                            store_f32x32(zr + acol + 32, r1);
                         }
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {

@@ -261,13 +261,22 @@ def _f64(t):
 
 
 class WeightsF64:
-    """float64 copies of the dense inputs (bf16 values widened exactly)."""
+    """The dense inputs for the backward oracle: x and the biases widened to
+    float64 at once, each expert's weights widened exactly on demand (full
+    float64 copies of large expert banks would not fit in host memory)."""
 
     def __init__(self, x, w1, b1, w2, b2):
-        self.x, self.w1, self.b1, self.w2, self.b2 = (_f64(v) for v in (x, w1, b1, w2, b2))
+        self.x, self.b1, self.b2 = _f64(x), _f64(b1), _f64(b2)
+        self._w1, self._w2 = w1, w2
         self.N, self.H = self.x.shape
-        self.E, _, two_i = self.w1.shape
+        self.E, _, two_i = w1.shape
         self.I = two_i // 2
+
+    def w1e(self, e):
+        return _f64(self._w1[e])
+
+    def w2e(self, e):
+        return _f64(self._w2[e])
 
 
 def pairs_backward(wd: WeightsF64, dout, tokens, experts, scores, layout: int = LAYOUT_INTERLEAVED,
@@ -285,9 +294,22 @@ def pairs_backward(wd: WeightsF64, dout, tokens, experts, scores, layout: int = 
                ds=np.zeros(n))
     if n_threads <= 0:
         n_threads = len(os.sched_getaffinity(0))
-    lib.oracle_pairs_backward(H, I, layout, _ptr(wd.x), _ptr(wd.w1), _ptr(wd.b1), _ptr(wd.w2), _ptr(wd.b2),
-                              _ptr(do), n, _ptr(tokens), _ptr(experts), _ptr(scores), _ptr(out["h"]),
-                              _ptr(out["y"]), _ptr(out["dy"]), _ptr(out["dz"]), _ptr(out["ds"]), n_threads)
+    for e in np.unique(experts):  # one expert's weights at a time
+        sel = np.nonzero(experts == e)[0]
+        m = sel.shape[0]
+        w1e, w2e = wd.w1e(e), wd.w2e(e)
+        b1e = None if wd.b1 is None else np.ascontiguousarray(wd.b1[e])
+        b2e = None if wd.b2 is None else np.ascontiguousarray(wd.b2[e])
+        part = dict(h=np.zeros((m, I)), y=np.zeros((m, H)), dy=np.zeros((m, H)), dz=np.zeros((m, 2 * I)),
+                    ds=np.zeros(m))
+        tk = np.ascontiguousarray(tokens[sel])
+        ex = np.zeros(m, np.int32)
+        sc = np.ascontiguousarray(scores[sel])
+        lib.oracle_pairs_backward(H, I, layout, _ptr(wd.x), _ptr(w1e), _ptr(b1e), _ptr(w2e), _ptr(b2e), _ptr(do),
+                                  m, _ptr(tk), _ptr(ex), _ptr(sc), _ptr(part["h"]), _ptr(part["y"]),
+                                  _ptr(part["dy"]), _ptr(part["dz"]), _ptr(part["ds"]), n_threads)
+        for k in out:
+            out[k][sel] = part[k]
     return out
 
 
@@ -313,6 +335,7 @@ def backward(wd: WeightsF64, topk_idx: np.ndarray, topk_w: np.ndarray, dout, lay
     g = dict(dx=np.zeros((N, H)), dw1=np.zeros((E, H, 2 * I)), db1=np.zeros((E, 2 * I)),
              dw2=np.zeros((E, I, H)), db2=np.zeros((E, H)), dtopk_w=np.zeros((N, K)))
     g["dtopk_w"][tok, slot] = r["ds"]
+    g["pairs"] = dict(tok=tok, slot=slot, exp=exp, **r)  # the per-pair terms, for the tests' error scales
     for e in np.unique(exp):
         sel = exp == e
         te = tok[sel]
@@ -320,5 +343,5 @@ def backward(wd: WeightsF64, topk_idx: np.ndarray, topk_w: np.ndarray, dout, lay
         g["db2"][e] = r["dy"][sel].sum(0)
         g["dw1"][e] = wd.x[te].T @ r["dz"][sel]
         g["db1"][e] = r["dz"][sel].sum(0)
-        np.add.at(g["dx"], te, r["dz"][sel] @ wd.w1[e].T)
+        np.add.at(g["dx"], te, r["dz"][sel] @ wd.w1e(e).T)
     return g

@@ -46,3 +46,46 @@ def check_meta_equal(gpu_meta: dict, ref: dict):
     np.testing.assert_array_equal(to_np(gpu_meta["token_offset"]), ref["token_offset"])
     np.testing.assert_array_equal(to_np(gpu_meta["scores"])[:P].view(np.int32),
                                   ref["scores"].view(np.int32))
+
+
+# Backward tolerance.  A gradient entry is a sum of products whose factors
+# carry at most a few bf16 roundings on the GPU path (dz or dy, the stored dx
+# rows, the output itself; z is kept in fp32 and dh is formed from bf16
+# inputs in fp32), each a relative error within the bf16 unit roundoff
+# u = 2^-8 of the factor it rounds and independent across terms, so the
+# entry's error is of order u * rss, rss = the root sum of squares of its
+# terms; over ~10^6 entries the largest reaches ~5 standard deviations.  The
+# bound adds 8 u rss to the forward's bound.
+BWD_ULP = 2.0 ** -8
+BWD_RSS_FACTOR = 8.0
+
+
+def backward_rss(g, wd, dout):
+    """Root sum of squares of the terms of every gradient entry, from the
+    oracle's per-pair values (oracle.backward(...)["pairs"])."""
+    pr = g["pairs"]
+    tok, slot, exp = pr["tok"], pr["slot"], pr["exp"]
+    rss = {k: np.zeros_like(g[k]) for k in ("dx", "dw1", "db1", "dw2", "db2", "dtopk_w")}
+    x2 = wd.x ** 2
+    for e in np.unique(exp):
+        sel = exp == e
+        h2, dy2, dz2 = pr["h"][sel] ** 2, pr["dy"][sel] ** 2, pr["dz"][sel] ** 2
+        rss["dw2"][e] = h2.T @ dy2
+        rss["dw1"][e] = x2[tok[sel]].T @ dz2
+        rss["db2"][e] = dy2.sum(0)
+        rss["db1"][e] = dz2.sum(0)
+        np.add.at(rss["dx"], tok[sel], dz2 @ (wd.w1e(e) ** 2).T)
+    d = dout.detach().double().cpu().numpy() if hasattr(dout, "detach") else np.asarray(dout, np.float64)
+    rss["dtopk_w"][tok, slot] = (pr["y"] ** 2 * d[tok] ** 2).sum(1)
+    return {k: np.sqrt(v) for k, v in rss.items()}
+
+
+def assert_close_bwd(gpu, ref, rss, what=""):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    bound = RTOL * np.abs(ref) + ATOL_RMS * rms + BWD_RSS_FACTOR * BWD_ULP * rss
+    err = np.abs(gpu - ref)
+    bad = ~(err <= bound)
+    assert not bad.any(), (f"{what}: max_err {err.max():.4g}, rms {rms:.4g}, n_bad {int(bad.sum())}/{err.size}, "
+                           f"worst {np.unravel_index(int(np.argmax(err - bound)), err.shape)}")

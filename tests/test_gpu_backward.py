@@ -1,0 +1,118 @@
+"""GPU backward (moe_nonexpand_forward_train + moe_nonexpand_backward)
+against the backward oracle.
+
+Every gradient is compared with the forward's tolerance widened by the
+rounding noise of the backward's bf16 intermediates,
+|gpu - ref| <= 2e-2 |ref| + 2e-2 rms(ref) + 8 * 2^-8 * rss (tests/helpers.py):
+the GPU keeps z, dy, dz and the per-pair dx rows in bf16 and accumulates in
+fp32, the oracle is exact double on the same bf16 inputs, and rss, the root
+sum of squares of an entry's terms, is the scale of that noise.  Small cases are compared
+everywhere; the prefill workload, at full size, on two experts' complete
+weight gradients and on a sample of tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import assert_close_bwd, backward_rss, to_np
+from mixture_experts_routed_non_b200 import binding, synthetic
+
+pytestmark = pytest.mark.gpu
+
+GRADS = ("dx", "dw1", "dw2", "dtopk_w")
+
+
+def _concat_from_interleaved(w1, b1):
+    w1c = torch.cat([w1[:, :, 0::2], w1[:, :, 1::2]], dim=2).contiguous()
+    b1c = None if b1 is None else torch.cat([b1[:, 0::2], b1[:, 1::2]], dim=1).contiguous()
+    return w1c, b1c
+
+
+def _dout(wl, seed):
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    return torch.randn((wl.N, wl.H), generator=g, device="cuda").to(torch.bfloat16)
+
+
+def _run(inp, layout, dout, bias_grads=True):
+    wl = inp.wl
+    w1, b1 = inp.w1, inp.b1
+    if layout == 1:
+        w1, b1 = _concat_from_interleaved(w1, b1)
+    ws = binding.alloc_train_workspace(wl.N, wl.H, wl.I, wl.E, wl.K)
+    out = binding.forward_train(inp.x, inp.topk_idx, inp.topk_w, w1, inp.w2, b1, inp.b2, ws=ws, layout=layout)
+    grads = binding.backward(dout, inp.x, inp.topk_idx, inp.topk_w, w1, inp.w2, ws=ws, layout=layout,
+                             bias_grads=bias_grads and inp.b1 is not None)
+    torch.cuda.synchronize()
+    assert binding.read_error(ws) == 0
+    return out, grads, w1, b1
+
+
+def _check_full(inp, layout, seed=0):
+    wl = inp.wl
+    dout = _dout(wl, seed + 100)
+    out, grads, w1, b1 = _run(inp, layout, dout)
+    # the training forward computes the same output as the forward
+    ref_out = binding.forward(inp.x, inp.topk_idx, inp.topk_w, w1, inp.w2, b1, inp.b2, layout=layout)
+    assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
+    wd = oracle.WeightsF64(inp.x, w1, b1, inp.w2, inp.b2)
+    ref = oracle.backward(wd, inp.topk_idx.cpu().numpy(), inp.topk_w.cpu().numpy(), dout, layout)
+    rss = backward_rss(ref, wd, dout)
+    for k in GRADS + (("db1", "db2") if "db1" in grads else ()):
+        assert_close_bwd(to_np(grads[k]), ref[k], rss[k], f"{k} ({wl.name}, layout {layout})")
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_tiny_backward_full(layout):
+    inp = synthetic.make_inputs("tiny", device="cuda", invalid_value=float("nan"))
+    _check_full(inp, layout)
+
+
+@pytest.mark.parametrize("N,H,I,E,K,p_invalid,bias,seed", [
+    (300, 256, 192, 5, 3, 0.2, True, 2),      # I % 128 == 64: partial column tiles
+    (129, 192, 128, 3, 2, 0.0, False, 3),     # H % 256 == 192
+    (700, 128, 64, 9, 4, 0.3, True, 4),       # I = 64
+    (64, 320, 320, 2, 1, 0.5, True, 6),
+    (50, 128, 128, 64, 2, 0.0, True, 7),      # most experts empty: zero weight gradients
+])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_ragged_backward_full(N, H, I, E, K, p_invalid, bias, seed, layout):
+    wl = synthetic.custom(N, H, I, E, K, p_invalid=p_invalid, bias=bias, seed=seed)
+    inp = synthetic.make_inputs(wl, device="cuda", invalid_value=float("nan"))
+    _check_full(inp, layout, seed)
+
+
+def test_backward_deterministic():
+    inp = synthetic.make_inputs("tiny", device="cuda")
+    dout = _dout(inp.wl, 5)
+    _, g1, _, _ = _run(inp, 0, dout)
+    _, g2, _, _ = _run(inp, 0, dout)
+    for k in g1:
+        assert torch.equal(g1[k].view(torch.uint8), g2[k].view(torch.uint8)), k
+
+
+def test_prefill_backward_sampled():
+    """Full-size prefill, the launch configuration the benchmark times: two
+    experts' dW1/dW2 complete, and the dx / score-gradient rows of 24 tokens."""
+    inp = synthetic.make_inputs("prefill", device="cuda")
+    wl = inp.wl
+    dout = _dout(wl, 11)
+    _, grads, _, _ = _run(inp, 0, dout, bias_grads=False)
+    idx, w = inp.topk_idx.cpu().numpy(), inp.topk_w.cpu().numpy()
+    wd = oracle.WeightsF64(inp.x, inp.w1, None, inp.w2, None)
+    experts = [7, 100]
+    ref = oracle.backward(wd, idx, w, dout, 0, experts_only=experts)
+    rss = backward_rss(ref, wd, dout)
+    for k in ("dw1", "dw2"):
+        assert_close_bwd(to_np(grads[k][experts]), ref[k][experts], rss[k][experts],
+                         f"{k} (prefill, experts {experts})")
+    tokens = np.sort(np.random.default_rng(3).choice(wl.N, size=24, replace=False))
+    sub = np.full_like(idx, -1)
+    sub[tokens] = idx[tokens]
+    ref_t = oracle.backward(wd, sub, w, dout, 0)
+    rss_t = backward_rss(ref_t, wd, dout)
+    assert_close_bwd(to_np(grads["dx"])[tokens], ref_t["dx"][tokens], rss_t["dx"][tokens],
+                     "dx (prefill, sampled tokens)")
+    assert_close_bwd(to_np(grads["dtopk_w"])[tokens], ref_t["dtopk_w"][tokens], rss_t["dtopk_w"][tokens],
+                     "dtopk_w (prefill, sampled tokens)")

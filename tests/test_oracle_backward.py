@@ -43,7 +43,7 @@ def _loss(wd, idx, tw, dout, layout, lib=None):
 def check_finite_differences(layout, lib=None, eps=1e-6):
     wd, idx, tw, dout = _small_problem(1, layout)
     g = oracle.backward(wd, idx, tw, dout, layout, lib_path=lib)
-    fields = {"dx": (wd, "x"), "dw1": (wd, "w1"), "db1": (wd, "b1"), "dw2": (wd, "w2"), "db2": (wd, "b2")}
+    fields = {"dx": (wd, "x"), "dw1": (wd, "_w1"), "db1": (wd, "b1"), "dw2": (wd, "_w2"), "db2": (wd, "b2")}
     for gname, (obj, attr) in fields.items():
         arr = getattr(obj, attr)
         num = np.zeros_like(arr)
