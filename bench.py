@@ -285,6 +285,63 @@ def router_only(dev, peaks, reps: int = 10, ring: int = 20):
             "l2": f"ring of {ring} logits buffers ({ring * N * E * 4 / 1e6:.0f} MB) in one graph"}
 
 
+def backward_leg(inp, w1, b1, layout, dev, peaks, steps: int = 30, warmup: int = 3):
+    """One training step, forward_train + backward, on the bench workload:
+    mean device time per step with the backward's seven stages timed by
+    events on the launching stream.  Inputs are larger than L2 (1.2 GB of
+    expert weights and their gradients per step)."""
+    import numpy as np
+    import torch
+
+    from mixture_experts_routed_non_b200 import binding
+    wl = inp.wl
+    N, H, I, E, K = wl.N, wl.H, wl.I, wl.E, wl.K
+    ws = binding.alloc_train_workspace(N, H, I, E, K, -1, dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(77)
+    dout = torch.randn((N, H), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty(N, H, dtype=torch.bfloat16, device=dev)
+    grads = None
+    fev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(steps)]
+    bias = b1 is not None
+    for i in range(warmup + steps):
+        j = i - warmup
+        if j >= 0:
+            fev[j][0].record()
+        binding.forward_train(inp.x, inp.topk_idx, inp.topk_w, w1, inp.w2, b1, inp.b2, ws=ws, layout=layout,
+                              out=out)
+        if j >= 0:
+            fev[j][1].record()
+        grads = binding.backward(dout, inp.x, inp.topk_idx, inp.topk_w, w1, inp.w2, ws=ws, layout=layout,
+                                 bias_grads=bias, grads=grads, events=bev[j] if j >= 0 else None)
+    torch.cuda.synchronize(dev)
+    if binding.read_error(ws):
+        raise SystemExit("bench.py: device error in the backward")
+    P = int((inp.topk_idx >= 0).sum().item())
+    fwd = float(np.mean([a.elapsed_time(b) for a, b in fev]))
+    st = np.mean([[e[k].elapsed_time(e[k + 1]) for k in range(7)] for e in bev], axis=0)
+    names = ["prep", "dh", "dw2", "dx", "dw1", "combine", "bias"]
+    phi = P * H * I
+    flops = {"dh": 2 * phi, "dw2": 2 * phi, "dx": 4 * phi, "dw1": 4 * phi}
+    tf = {k: flops[k] / (st[names.index(k)] * 1e-3) / 1e12 for k in flops}
+    gemm_ms = float(sum(st[names.index(k)] for k in flops))
+    bwd_ms = float(st.sum())
+    dom = max(flops, key=lambda k: st[names.index(k)])
+    peak = peaks["bf16_tflops_sustained"]
+    prep_bytes = 2 * P * H * 2 + N * H * 2  # y read, dy written, dout read
+    del ws
+    return {"workload": wl.name, "steps": steps, "train_step_ms": fwd + bwd_ms,
+            "tokens_per_s": N / ((fwd + bwd_ms) * 1e-3), "forward_train_ms": fwd, "backward_ms": bwd_ms,
+            "stages_ms": dict(zip(names, [float(v) for v in st])),
+            "gemm_tflops": {k: float(v) for k, v in tf.items()},
+            "bwd_gemm_tflops": 12 * phi / (gemm_ms * 1e-3) / 1e12,
+            "bwd_gemm_frac_of_peak": 12 * phi / (gemm_ms * 1e-3) / 1e12 / peak,
+            "prep_gbs": prep_bytes / (st[0] * 1e-3) / 1e9,
+            "dominant": {"kernel": f"backward grouped GEMM {dom}", "tflops": float(tf[dom]), "peak": peak,
+                         "frac": float(tf[dom] / peak), "peak_source": "measured bf16 sustained"}}
+
+
 def run_reference(args, rank, world):
     """The reference arm: the CPU oracle as it stands, rank 0 only."""
     if rank != 0:
@@ -491,6 +548,7 @@ def run_ours(args, rank, world, local):
 
     meta_c2 = metadata_only(dev, peaks) if rank == 0 else None
     router = router_only(dev, peaks) if rank == 0 else None
+    train = backward_leg(inp, w1, b1, args.layout, dev, peaks) if rank == 0 else None
 
     if world > 1:
         dist.destroy_process_group()
@@ -540,6 +598,7 @@ def run_ours(args, rank, world, local):
                 "steps": e2e_steps, "pipelining": "copy-in / compute / copy-out streams, 2 buffer sets"},
         "metadata_only": meta_c2,
         "router_only": router,
+        "training": train,
         "gpu_launches": 4 * args.steps,  # meta, up, down, combine (plus one 4-byte memset)
         "clocks": clocks,
     }

@@ -479,6 +479,7 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         return MOE_ERR_CUDA;
     if ((st = record(ev, 1, s))) return st;
 
+    const uint64_t prow = (uint64_t)(l.p_cap > 0 ? l.p_cap : 1);
     BwdGemmArgs g;
     memset(&g, 0, sizeof g);
     g.expert_off = meta.expert_frequency_offset;
@@ -494,7 +495,9 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         a.a_ld = H;
         a.b = w2b;
         a.b_ld = H;
-        a.b_estride = (int64_t)I * H;
+        a.b_rows_per_expert = I;
+        if (!make_map_a_chunks(&a.tmap_b, w2b, (uint64_t)H, (uint64_t)E * I, 256, 1)) return MOE_ERR_CUDA;
+        a.b_tma = 1;
         a.z = zbuf;
         a.dz = dzbuf;
         a.row_scale = meta.scores;
@@ -511,6 +514,10 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         a.a_ld = I;
         a.b = dybuf;
         a.b_ld = H;
+        if (!make_map_a_chunks(&a.tmap_a, hbuf, (uint64_t)I, prow, 64, 2) ||
+            !make_map_a_chunks(&a.tmap_b, dybuf, (uint64_t)H, prow, 64, 4))
+            return MOE_ERR_CUDA;
+        a.a_tma = a.b_tma = 1;
         a.out = static_cast<__nv_bfloat16 *>(dw2);
         a.out_ld = H;
         a.M_dim = I;
@@ -525,7 +532,11 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         a.a_ld = 2 * I;
         a.b = w1b;
         a.b_ld = 2 * I;
-        a.b_estride = (int64_t)H * 2 * I;
+        a.b_rows_per_expert = H;
+        if (!make_map_a_chunks(&a.tmap_a, dzbuf, (uint64_t)2 * I, prow, 128, 1) ||
+            !make_map_a_chunks(&a.tmap_b, w1b, (uint64_t)2 * I, (uint64_t)E * H, 256, 1))
+            return MOE_ERR_CUDA;
+        a.a_tma = a.b_tma = 1;
         a.out = ybuf;
         a.out_ld = H;
         a.N_dim = H;
@@ -541,6 +552,8 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         a.a_ld = H;
         a.b = dzbuf;
         a.b_ld = 2 * I;
+        if (!make_map_a_chunks(&a.tmap_b, dzbuf, (uint64_t)2 * I, prow, 64, 4)) return MOE_ERR_CUDA;
+        a.b_tma = 1;
         a.out = static_cast<__nv_bfloat16 *>(dw1);
         a.out_ld = 2 * I;
         a.M_dim = H;

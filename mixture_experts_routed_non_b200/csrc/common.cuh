@@ -105,12 +105,15 @@ enum BwdMode : int32_t {
 };
 
 struct BwdGemmArgs {
+    CUtensorMap tmap_a;        // (64, rows, cols/64) view of `a` when a_tma
+    CUtensorMap tmap_b;        // (64, rows, cols/64) view of `b` when b_tma
+    int32_t a_tma, b_tma;      // load that operand's whole stages with TMA
+    int32_t b_rows_per_expert; // DH/DX: rows of `b` per expert (N of the weights)
     const __nv_bfloat16 *a;    // DH: dout [N,H]; DX: dz [P_cap,2I]; DW: rows of length M_dim
     const int32_t *a_rows;     // DH/DW: row of `a` for segment row p (null: p itself)
     int64_t a_ld;              // elements per row of `a`
     const __nv_bfloat16 *b;    // DH/DX: weights [E][N][K] (K contiguous); DW: [P_cap, N_dim] rows p
     int64_t b_ld;              // elements per row of `b`
-    int64_t b_estride;         // DH/DX: elements between experts of `b`
     const int32_t *expert_off; // [E+1] segment offsets
     __nv_bfloat16 *out;        // DX: [P_cap, N]; DW: [E][M][N]; DH: unused (writes z)
     int64_t out_ld;

@@ -23,7 +23,9 @@
 // the row operands of DH/DX and for the weights read as [N][K]; MN-major
 // (rows = K, 64-element MN atoms, 128-byte swizzle) for both DW operands.
 // Warp roles: warp 0 = TMEM allocator and MMA issuer, warps 1-4 = epilogue
-// (TMEM lane quarter warp % 4), warps 5-8 = cp.async producers.  Four
+// (TMEM lane quarter warp % 4), warp 5 = TMA producer (whole-stage boxes of
+// every operand that needs no gather), warps 6-9 = cp.async producers (the
+// gathered rows, and the zero-filled last stage of a DW segment).  Four
 // shared-memory stages, two TMEM accumulators.  Every wait is bounded; on a
 // timeout the CTA raises its abort flag, records MOE_DEVERR_TIMEOUT, drains
 // its MMAs and copies and frees its TMEM.
@@ -38,7 +40,7 @@ constexpr int kN = 256;                      // tile columns (UMMA N)
 constexpr int kSK = 64;                      // K per stage: one 128-byte swizzle atom of bf16
 constexpr int kBwdStages = 4;
 constexpr int kProducerThreads = 128;
-constexpr int kThreads = 32 + 128 + kProducerThreads;
+constexpr int kThreads = 32 + 128 + 32 + kProducerThreads;  // MMA, epilogue, TMA, cp.async
 constexpr uint32_t kStageA = kM * kSK * 2;   // 16 KB
 constexpr uint32_t kStageB = kN * kSK * 2;   // 32 KB
 constexpr uint32_t kStageBytes = kStageA + kStageB;
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
     for (int i = threadIdx.x; i <= E; i += kThreads) off_s[i] = __ldg(a.expert_off + i);
     if (threadIdx.x == 0) {
         for (int s = 0; s < kBwdStages; ++s) {
-            mbar_init(full_bar(s), kProducerThreads);
+            mbar_init(full_bar(s), kProducerThreads + 1);  // cp.async threads + TMA thread
             mbar_init(empty_bar(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -364,16 +366,91 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(acc));
         }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------- TMA producer
+        // whole-stage boxes of the operands that need no gather: 128-byte-swizzled
+        // [atom][row][128 B] boxes of a (64, rows, cols/64) view of each matrix
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_parity = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+                const BTile t = decode(tile);
+                for (int kb = 0; kb < t.nk; ++kb) {
+                    if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    const int kbase = t.kp0 + kb * kSK;
+                    const bool tail = kMN && kbase + kSK > t.kp1;  // the copy warps zero-fill it
+                    const bool ta = a.a_tma && !tail, tb = a.b_tma && !tail;
+                    const uint32_t bytes = (ta ? kStageA : 0u) + (tb ? kStageB : 0u);
+                    if (bytes) {
+                        mbar_arrive_expect_tx(full_bar(stage), bytes);
+                        if (kMN) {
+                            if (ta) tma_load_3d(a_stage(stage), &a.tmap_a, full_bar(stage), 0, kbase, t.m0 / 64);
+                            if (tb) tma_load_3d(b_stage(stage), &a.tmap_b, full_bar(stage), 0, kbase, t.n0 / 64);
+                        } else {
+                            if (ta) tma_load_3d(a_stage(stage), &a.tmap_a, full_bar(stage), 0, t.m0, kb);
+                            if (tb)
+                                tma_load_3d(b_stage(stage), &a.tmap_b, full_bar(stage), 0,
+                                            t.e * a.b_rows_per_expert + t.n0, kb);
+                        }
+                        issued |= 1u << stage;
+                        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    } else {
+                        mbar_arrive(full_bar(stage));
+                    }
+                    if (++stage == kBwdStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // the CTA may not exit while a TMA it issued can still write its memory
+            for (int st = 0; st < kBwdStages; ++st)
+                if (issued & (1u << st)) mbar_wait_timed(full_bar(st), (issued_parity >> st) & 1u);
+        }
+        __syncwarp();
     } else {
-        // ------------------------------------------------------------ producers
-        const int pt = threadIdx.x - 160;
+        // ------------------------------------------------------ cp.async producers
+        // the gathered operand (dout rows in DH, x rows in dW1) and, in DW, the
+        // segment's last stage of both operands with the rows past its end zeroed
+        const int pt = threadIdx.x - 192;
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         const int gl = pt & 31;
         for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
             const BTile t = decode(tile);
+            // K-major gathered rows (DH): this thread's 8 row pointers, once per tile
+            // (null past the segment end: those rows feed unstored outputs only)
+            const __nv_bfloat16 *arow[kM / 16];
+            if (!kMN && !a.a_tma) {
+#pragma unroll
+                for (int i = 0; i < kM / 16; ++i) {
+                    const int p = t.m0 + (pt >> 3) + 16 * i;
+                    arow[i] = p < t.m_end ? a.a + (size_t)(a.a_rows ? __ldg(a.a_rows + p) : p) * a.a_ld : nullptr;
+                }
+            }
+            // MN-major gathered rows (dW1): the next stage's row indices are loaded
+            // while this stage's copies are in flight
+            int nrow[kSK / 8];
+            auto load_rows = [&](int kb) {
+                const int kbase = t.kp0 + kb * kSK;
+#pragma unroll
+                for (int i = 0; i < kSK / 8; ++i) {
+                    const int p = kbase + (pt >> 4) + 8 * i;
+                    nrow[i] = p < t.kp1 ? (a.a_rows ? __ldg(a.a_rows + p) : p) : -1;
+                }
+            };
+            if (kMN && t.nk > 0) load_rows(0);
             for (int kb = 0; kb < t.nk; ++kb) {
+                int crow[kSK / 8];
+#pragma unroll
+                for (int i = 0; i < kSK / 8; ++i) crow[i] = nrow[i];
+                if (kMN && kb + 1 < t.nk) load_rows(kb + 1);
                 bool w = true;
                 if (gl == 0) w = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort);
                 w = __shfl_sync(0xffffffffu, w, 0);
@@ -386,43 +463,40 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
                     // K-major rows: 8 chunks of 16 B per 128-byte row, swizzled by row & 7
                     const int c = pt & 7, r0 = pt >> 3;
                     const int k0 = kb * kSK + 8 * c;
+                    if (!a.a_tma) {
 #pragma unroll
-                    for (int i = 0; i < kM / 16; ++i) {
-                        const int r = r0 + 16 * i;
-                        const int p = t.m0 + r;  // rows past the segment end feed unstored rows only
-                        if (p < t.m_end) {
-                            const int row = a.a_rows ? __ldg(a.a_rows + p) : p;
-                            cp_async_16(sa + r * 128 + ((c ^ (r & 7)) << 4), a.a + (size_t)row * a.a_ld + k0);
+                        for (int i = 0; i < kM / 16; ++i) {
+                            const int r = r0 + 16 * i;
+                            if (arow[i]) cp_async_16(sa + r * 128 + ((c ^ (r & 7)) << 4), arow[i] + k0);
                         }
                     }
-                    const __nv_bfloat16 *bw = a.b + (size_t)t.e * a.b_estride;
+                    if (!a.b_tma) {
+                        const __nv_bfloat16 *bw = a.b + (size_t)t.e * a.b_rows_per_expert * a.b_ld;
 #pragma unroll
-                    for (int i = 0; i < kN / 16; ++i) {
-                        const int r = r0 + 16 * i;
-                        const int n = t.n0 + r;  // columns past N_dim are never stored
-                        if (n < a.N_dim)
-                            cp_async_16(sb + r * 128 + ((c ^ (r & 7)) << 4), bw + (size_t)n * a.b_ld + k0);
+                        for (int i = 0; i < kN / 16; ++i) {
+                            const int r = r0 + 16 * i;
+                            const int n = t.n0 + r;  // columns past N_dim are never stored
+                            if (n < a.N_dim)
+                                cp_async_16(sb + r * 128 + ((c ^ (r & 7)) << 4), bw + (size_t)n * a.b_ld + k0);
+                        }
                     }
                 } else {
-                    // MN-major: row kr of the stage = segment row p; rows past the
-                    // segment end are zero in both operands
+                    // MN-major: row kr of the stage = segment row p
                     const int kbase = t.kp0 + kb * kSK;
-                    {
+                    const bool tail = kbase + kSK > t.kp1;
+                    if (!a.a_tma || tail) {
                         const int c = pt & 15, kr0 = pt >> 4;  // 16 chunks per 128-element A row
                         const int m = t.m0 + 8 * c;
 #pragma unroll
                         for (int i = 0; i < kSK / 8; ++i) {
                             const int kr = kr0 + 8 * i;
-                            const int p = kbase + kr;
-                            const bool in = p < t.kp1;
+                            const bool in = crow[i] >= 0;  // rows past the segment end are zero
                             const uint32_t dst = sa + (c >> 3) * kMnAtom + kr * 128 + (((c & 7) ^ (kr & 7)) << 4);
-                            if (m < a.M_dim) {
-                                const int row = in ? (a.a_rows ? __ldg(a.a_rows + p) : p) : 0;
-                                cp_async_16_zfill(dst, a.a + (size_t)row * a.a_ld + m, in ? 16u : 0u);
-                            }
+                            if (m < a.M_dim)
+                                cp_async_16_zfill(dst, a.a + (size_t)(in ? crow[i] : 0) * a.a_ld + m, in ? 16u : 0u);
                         }
                     }
-                    {
+                    if (!a.b_tma || tail) {
                         const int c = pt & 31, kr0 = pt >> 5;  // 32 chunks per 256-element B row
                         const int n = t.n0 + 8 * c;
 #pragma unroll
