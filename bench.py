@@ -321,7 +321,7 @@ def backward_leg(inp, w1, b1, layout, dev, peaks, steps: int = 30, warmup: int =
     P = int((inp.topk_idx >= 0).sum().item())
     fwd = float(np.mean([a.elapsed_time(b) for a, b in fev]))
     st = np.mean([[e[k].elapsed_time(e[k + 1]) for k in range(7)] for e in bev], axis=0)
-    names = ["prep", "dh", "dw2", "dx", "dw1", "combine", "bias"]
+    names = ["prep", "dh", "dw2", "dw1", "dx", "combine", "bias"]  # dw1 includes gathering x rows
     phi = P * H * I
     flops = {"dh": 2 * phi, "dw2": 2 * phi, "dx": 4 * phi, "dw1": 4 * phi}
     tf = {k: flops[k] / (st[names.index(k)] * 1e-3) / 1e12 for k in flops}

@@ -315,8 +315,9 @@ MOE_API int moe_nonexpand_backward(const void *dout, const void *x, const int32_
                                    void *ws, size_t ws_bytes, moe_stream_t stream);
 
 /* moe_nonexpand_backward plus eight events recorded on the stream around its
- * seven steps: score gradients and dy, dh + SwiGLU backward, dW2, dx rows,
- * dW1, the dx combine, the bias gradients. */
+ * seven steps: score gradients and dy, dh + SwiGLU backward, dW2, dW1 (with
+ * the gather of x rows it reads), dx rows, the dx combine, the bias
+ * gradients. */
 MOE_API int moe_nonexpand_backward_timed(const void *dout, const void *x, const int32_t *topk_idx,
                                          const float *topk_w, int64_t N, int32_t H, int32_t I, int32_t E,
                                          int32_t K, int64_t total_pairs, const void *w1, const void *w2,

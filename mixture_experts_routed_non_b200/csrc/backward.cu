@@ -10,6 +10,8 @@
 //             non-expand layout.
 //   bias      db[e,c] = sum of the segment's rows of dy (db2) or dz (db1), in
 //             row order, fp32, rounded once to bf16.
+//   gather    xs[p,:] = x[x_gather_idx[p],:], so the dW1 GEMM reads its A
+//             operand with whole-stage TMA boxes instead of per-row copies.
 #include "common.cuh"
 
 namespace moe {
@@ -131,7 +133,31 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(const __nv_bfloat16 *__r
     reinterpret_cast<uint32_t *>(db + (size_t)e * cols)[c2] = pack_bf16x2(s0, s1);
 }
 
+// dst[p, :] = src[idx[p], :] for p < P = expert_off[E] (16-byte chunks).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16 *__restrict__ src,
+                                                          const int32_t *__restrict__ idx,
+                                                          const int32_t *__restrict__ p_total, int32_t cols,
+                                                          __nv_bfloat16 *__restrict__ dst, const WsHeader *hdr) {
+    if (hdr && *(volatile const uint32_t *)&hdr->abort) return;
+    const int P = __ldg(p_total);
+    const int chunks = cols >> 3;
+    const int64_t total = (int64_t)P * chunks;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t p = i / chunks;
+        const int c = (int)(i - p * chunks);
+        const int row = __ldg(idx + p);
+        reinterpret_cast<uint4 *>(dst + (size_t)p * cols)[c] =
+            __ldg(reinterpret_cast<const uint4 *>(src + (size_t)row * cols) + c);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_gather_rows(const __nv_bfloat16 *src, const int32_t *idx, const int32_t *p_total, int32_t cols,
+                               __nv_bfloat16 *dst, const WsHeader *hdr, int num_sms, cudaStream_t s) {
+    gather_rows_kernel<<<(unsigned)(num_sms * 8), 256, 0, s>>>(src, idx, p_total, cols, dst, hdr);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const __nv_bfloat16 *y, const int32_t *topk_idx,
                             const moe_meta_t &meta, int64_t N, int32_t H, int32_t K, int32_t E, __nv_bfloat16 *dy,

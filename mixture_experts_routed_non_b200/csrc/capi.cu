@@ -525,7 +525,29 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         if (launch_gemm_bwd(kBwdDW, a, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if ((st = record(ev, 3, s))) return st;
-    // dx rows = dz . W1[e]^T, into the (no longer needed) y region
+    // dW1[e] = xs^T dz with xs = x[x_gather_idx] gathered into the (no longer
+    // needed) y region, so both operands load by TMA
+    if (launch_gather_rows(static_cast<const __nv_bfloat16 *>(x), meta.x_gather_idx, meta.expert_frequency_offset + E,
+                           H, ybuf, hdr, dev.sms, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    {
+        BwdGemmArgs a = g;
+        a.a = ybuf;
+        a.a_ld = H;
+        a.b = dzbuf;
+        a.b_ld = 2 * I;
+        if (!make_map_a_chunks(&a.tmap_a, ybuf, (uint64_t)H, prow, 64, 2) ||
+            !make_map_a_chunks(&a.tmap_b, dzbuf, (uint64_t)2 * I, prow, 64, 4))
+            return MOE_ERR_CUDA;
+        a.a_tma = a.b_tma = 1;
+        a.out = static_cast<__nv_bfloat16 *>(dw1);
+        a.out_ld = 2 * I;
+        a.M_dim = H;
+        a.N_dim = 2 * I;
+        if (launch_gemm_bwd(kBwdDW, a, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    if ((st = record(ev, 4, s))) return st;
+    // dx rows = dz . W1[e]^T, into the y region (xs is no longer needed)
     {
         BwdGemmArgs a = g;
         a.a = dzbuf;
@@ -542,23 +564,6 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         a.N_dim = H;
         a.K_dim = 2 * I;
         if (launch_gemm_bwd(kBwdDX, a, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
-    }
-    if ((st = record(ev, 4, s))) return st;
-    // dW1[e] = x[x_gather_idx]^T dz
-    {
-        BwdGemmArgs a = g;
-        a.a = static_cast<const __nv_bfloat16 *>(x);
-        a.a_rows = meta.x_gather_idx;
-        a.a_ld = H;
-        a.b = dzbuf;
-        a.b_ld = 2 * I;
-        if (!make_map_a_chunks(&a.tmap_b, dzbuf, (uint64_t)2 * I, prow, 64, 4)) return MOE_ERR_CUDA;
-        a.b_tma = 1;
-        a.out = static_cast<__nv_bfloat16 *>(dw1);
-        a.out_ld = 2 * I;
-        a.M_dim = H;
-        a.N_dim = 2 * I;
-        if (launch_gemm_bwd(kBwdDW, a, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
     }
     if ((st = record(ev, 5, s))) return st;
     // dx[t] = sum of its pairs' dx rows (weight 1)

@@ -144,6 +144,8 @@ cudaError_t launch_gemm_bwd(int mode, const BwdGemmArgs &a, int max_ctas, cudaSt
 cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const __nv_bfloat16 *y, const int32_t *topk_idx,
                             const moe_meta_t &meta, int64_t N, int32_t H, int32_t K, int32_t E, __nv_bfloat16 *dy,
                             float *dtopk_w, const WsHeader *hdr, int num_sms, cudaStream_t s);
+cudaError_t launch_gather_rows(const __nv_bfloat16 *src, const int32_t *idx, const int32_t *p_total, int32_t cols,
+                               __nv_bfloat16 *dst, const WsHeader *hdr, int num_sms, cudaStream_t s);
 cudaError_t launch_bias_grad(const __nv_bfloat16 *src, int32_t cols, const int32_t *expert_off, int32_t E,
                              __nv_bfloat16 *db, const WsHeader *hdr, cudaStream_t s);
 

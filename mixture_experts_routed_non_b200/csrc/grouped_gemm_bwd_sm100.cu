@@ -22,10 +22,11 @@
 // Operands: K-major (rows of 64 contiguous K values, 128-byte swizzle) for
 // the row operands of DH/DX and for the weights read as [N][K]; MN-major
 // (rows = K, 64-element MN atoms, 128-byte swizzle) for both DW operands.
-// Warp roles: warp 0 = TMEM allocator and MMA issuer, warps 1-4 = epilogue
-// (TMEM lane quarter warp % 4), warp 5 = TMA producer (whole-stage boxes of
-// every operand that needs no gather), warps 6-9 = cp.async producers (the
-// gathered rows, and the zero-filled last stage of a DW segment).  Four
+// Warp roles: warp 0 = TMEM allocator and MMA issuer, then the epilogue warps
+// (TMEM lane quarter warp % 4; DH has two per quarter, splitting the columns),
+// one TMA producer warp (whole-stage boxes of every operand that needs no
+// gather) and four cp.async producer warps (the gathered rows, and the
+// zero-filled last stage of a DW segment).  Four
 // shared-memory stages, two TMEM accumulators.  Every wait is bounded; on a
 // timeout the CTA raises its abort flag, records MOE_DEVERR_TIMEOUT, drains
 // its MMAs and copies and frees its TMEM.
@@ -40,7 +41,16 @@ constexpr int kN = 256;                      // tile columns (UMMA N)
 constexpr int kSK = 64;                      // K per stage: one 128-byte swizzle atom of bf16
 constexpr int kBwdStages = 4;
 constexpr int kProducerThreads = 128;
-constexpr int kThreads = 32 + 128 + 32 + kProducerThreads;  // MMA, epilogue, TMA, cp.async
+// Epilogue warps: 4 (one per TMEM lane quarter), or 8 for DH, whose SwiGLU
+// backward is heavy: two warps per quarter, each on half the columns.
+template <int kMode>
+struct Roles {
+    static constexpr int kEpiWarps = kMode == kBwdDH ? 8 : 4;
+    static constexpr int kParts = kEpiWarps / 4;
+    static constexpr int kTmaWarp = 1 + kEpiWarps;
+    static constexpr int kCopyThread0 = 32 * (kTmaWarp + 1);
+    static constexpr int kThreads = kCopyThread0 + kProducerThreads;  // MMA, epilogue, TMA, cp.async
+};
 constexpr uint32_t kStageA = kM * kSK * 2;   // 16 KB
 constexpr uint32_t kStageB = kN * kSK * 2;   // 32 KB
 constexpr uint32_t kStageBytes = kStageA + kStageB;
@@ -108,13 +118,19 @@ __device__ __forceinline__ void settle_after_abort() {
     }
 }
 
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ float silu_f(float g, float &sig) {
-    sig = 1.0f / (1.0f + __expf(-g));
+    sig = __fdividef(1.0f, 1.0f + __expf(-g));  // 0 once exp(-g) overflows, as the limit
     return g * sig;
 }
 
 template <int kMode>
-__global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_constant__ BwdGemmArgs a) {
+__global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(const __grid_constant__ BwdGemmArgs a) {
+    using R = Roles<kMode>;
+    constexpr int kThreads = R::kThreads;
     constexpr bool kMN = kMode == kBwdDW;  // both operands MN-major, K = segment rows
     constexpr uint32_t kIdesc = idesc(kMN, kMN);
     extern __shared__ uint8_t smem_raw[];
@@ -145,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), 4);
+            mbar_init(tempty_bar(b), R::kEpiWarps);
         }
         mbar_init(drain_bar, 1);
         misc[1] = 0;
@@ -246,15 +262,33 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
             mbar_wait_timed(drain_bar, 0);
         }
         __syncwarp();
-    } else if (warp < 5) {
+    } else if (warp < R::kTmaWarp) {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;
         const int rl = quarter * 32 + lane;  // this thread's tile row (TMEM lane)
+        const int part = (warp - 1) >> 2;    // this warp's part of the tile's columns
         int tcount = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
             const BTile t = decode(tile);
             const int acc = tcount & 1;
             const uint32_t acc_phase = (tcount >> 1) & 1;
+            if (kMode == kBwdDH) {
+                // bring this row's z columns of the tile into L2 while the MMAs run
+                const int p = t.m0 + rl;
+                if (p < t.m_end) {
+                    const int c0 = t.n0 + part * (kN / R::kParts);  // this warp's first I column
+                    const int ncols = min(kN / R::kParts, a.I - c0);
+                    const float *zr = a.z + (size_t)p * (2 * a.I);
+                    if (a.layout == MOE_LAYOUT_INTERLEAVED) {
+                        for (int b = 0; b < 2 * ncols * 4; b += 128) prefetch_l2((const char *)(zr + 2 * c0) + b);
+                    } else {
+                        for (int b = 0; b < ncols * 4; b += 128) {
+                            prefetch_l2((const char *)(zr + c0) + b);
+                            prefetch_l2((const char *)(zr + a.I + c0) + b);
+                        }
+                    }
+                }
+            }
             bool w = true;
             if (lane == 0) w = mbar_wait_bounded(tfull_bar(acc), acc_phase, abort);
             w = __shfl_sync(0xffffffffu, w, 0);
@@ -270,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
                 // the pair's score: dh = s (dout . W2^T)
                 const float sc = valid ? __ldg(a.row_scale + __ldg(a.row_pair + p)) : 0.f;
 #pragma unroll 1
-                for (int c = 0; c < kN / 32; ++c) {
+                for (int c = part * (kN / 32 / R::kParts); c < (part + 1) * (kN / 32 / R::kParts); ++c) {
                     const int i0 = t.n0 + 32 * c;
                     if (i0 >= a.I) break;
                     uint32_t dh[32];
@@ -334,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
                 __nv_bfloat16 *orow = a.out + row_off;
                 const bool zero = kMode == kBwdDW && t.nk == 0;  // empty segment: the gradient is 0
 #pragma unroll 1
-                for (int g = 0; g < kN / 64; ++g) {
+                for (int g = part * (kN / 64 / R::kParts); g < (part + 1) * (kN / 64 / R::kParts); ++g) {
                     const int col0 = t.n0 + 64 * g;
                     if (col0 >= a.N_dim) break;
                     uint32_t r0[32], r1[32];
@@ -366,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
             __syncwarp();
             if (lane == 0) mbar_arrive(tempty_bar(acc));
         }
-    } else if (warp == 5) {
+    } else if (warp == R::kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
         // whole-stage boxes of the operands that need no gather: 128-byte-swizzled
         // [atom][row][128 B] boxes of a (64, rows, cols/64) view of each matrix
@@ -417,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_gemm_kernel(const __grid_cons
         // ------------------------------------------------------ cp.async producers
         // the gathered operand (dout rows in DH, x rows in dW1) and, in DW, the
         // segment's last stage of both operands with the rows past its end zeroed
-        const int pt = threadIdx.x - 192;
+        const int pt = threadIdx.x - R::kCopyThread0;
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
@@ -552,7 +586,7 @@ cudaError_t launch_mode(const BwdGemmArgs &a, int max_ctas, cudaStream_t s) {
         if (total < ctas) ctas = total;
     }
     if (ctas < 1) ctas = 1;
-    bwd_gemm_kernel<kMode><<<ctas, kThreads, kSmemBytes, s>>>(a);
+    bwd_gemm_kernel<kMode><<<ctas, Roles<kMode>::kThreads, kSmemBytes, s>>>(a);
     return cudaGetLastError();
 }
 
