@@ -56,7 +56,7 @@ constexpr uint32_t kStageB = kN * kSK * 2;   // 32 KB
 constexpr uint32_t kStageBytes = kStageA + kStageB;
 constexpr uint32_t kMnAtom = kSK * 128;      // MN-major: one 64-element column of a stage (8 KB)
 constexpr uint32_t kTmemCols = 2 * kN;
-constexpr uint32_t kNumBars = 2 * kBwdStages + 5;
+constexpr uint32_t kNumBars = 3 * kBwdStages + 5;
 constexpr size_t kSmemBarOff = (size_t)kBwdStages * kStageBytes;
 constexpr size_t kSmemMiscOff = kSmemBarOff + 8 * kNumBars;
 constexpr size_t kSmemTableOff = kSmemMiscOff + 16;
@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
     auto tfull_bar = [&](int b) { return bars + 8u * (2 * kBwdStages + b); };
     auto tempty_bar = [&](int b) { return bars + 8u * (2 * kBwdStages + 2 + b); };
     const uint32_t drain_bar = bars + 8u * (2 * kBwdStages + 4);
+    auto tail_bar = [&](int s) { return bars + 8u * (2 * kBwdStages + 5 + s); };  // DW: a tail stage's TMA
     uint32_t *misc = reinterpret_cast<uint32_t *>(base_ptr + kSmemMiscOff);
     int *tile_off_s = reinterpret_cast<int *>(base_ptr + kSmemTableOff);
     int *off_s = tile_off_s + (kMaxExperts + 1);
@@ -164,6 +165,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
             mbar_init(tempty_bar(b), R::kEpiWarps);
         }
         mbar_init(drain_bar, 1);
+        for (int s = 0; s < kBwdStages; ++s) mbar_init(tail_bar(s), 1);
         misc[1] = 0;
         fence_barrier_init();
     }
@@ -408,6 +410,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, issued_parity = 0;
+            uint32_t tissued = 0, tissued_parity = 0, tphase = 0;  // tail-stage TMAs (DW)
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
                 const BTile t = decode(tile);
@@ -417,10 +420,22 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                         break;
                     }
                     const int kbase = t.kp0 + kb * kSK;
-                    const bool tail = kMN && kbase + kSK > t.kp1;  // the copy warps zero-fill it
-                    const bool ta = a.a_tma && !tail, tb = a.b_tma && !tail;
+                    // a DW segment's last stage: the TMA lands on tail_bar, the copy
+                    // warps zero the rows past the segment end, then arrive on full
+                    const bool tail = kMN && kbase + kSK > t.kp1;
+                    const bool ta = a.a_tma != 0, tb = a.b_tma != 0;
                     const uint32_t bytes = (ta ? kStageA : 0u) + (tb ? kStageB : 0u);
-                    if (bytes) {
+                    if (tail && bytes) {
+                        const uint32_t tb_bar = tail_bar(stage);
+                        mbar_arrive_expect_tx(tb_bar, bytes);
+                        if (ta) tma_load_3d(a_stage(stage), &a.tmap_a, tb_bar, 0, kbase, t.m0 / 64);
+                        if (tb) tma_load_3d(b_stage(stage), &a.tmap_b, tb_bar, 0, kbase, t.n0 / 64);
+                        const uint32_t par = (tphase >> stage) & 1u;
+                        tissued |= 1u << stage;
+                        tissued_parity = (tissued_parity & ~(1u << stage)) | (par << stage);
+                        tphase ^= 1u << stage;
+                        mbar_arrive(full_bar(stage));
+                    } else if (bytes) {
                         mbar_arrive_expect_tx(full_bar(stage), bytes);
                         if (kMN) {
                             if (ta) tma_load_3d(a_stage(stage), &a.tmap_a, full_bar(stage), 0, kbase, t.m0 / 64);
@@ -443,8 +458,10 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                 }
             }
             // the CTA may not exit while a TMA it issued can still write its memory
-            for (int st = 0; st < kBwdStages; ++st)
+            for (int st = 0; st < kBwdStages; ++st) {
                 if (issued & (1u << st)) mbar_wait_timed(full_bar(st), (issued_parity >> st) & 1u);
+                if (tissued & (1u << st)) mbar_wait_timed(tail_bar(st), (tissued_parity >> st) & 1u);
+            }
         }
         __syncwarp();
     } else {
@@ -454,6 +471,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
         const int pt = threadIdx.x - R::kCopyThread0;
         int stage = 0;
         uint32_t phase = 0;
+        uint32_t tpar = 0;  // parity of each stage's next tail_bar phase
         bool ok = true;
         const int gl = pt & 31;
         for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
@@ -518,7 +536,30 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                     // MN-major: row kr of the stage = segment row p
                     const int kbase = t.kp0 + kb * kSK;
                     const bool tail = kbase + kSK > t.kp1;
-                    if (!a.a_tma || tail) {
+                    if (tail && (a.a_tma || a.b_tma)) {
+                        // the TMA brought whole boxes: zero the rows past the segment
+                        // end (they hold the next expert's rows, or unwritten memory)
+                        bool tw = true;
+                        if (gl == 0) tw = mbar_wait_bounded(tail_bar(stage), (tpar >> stage) & 1u, abort);
+                        tw = __shfl_sync(0xffffffffu, tw, 0);
+                        tpar ^= 1u << stage;
+                        if (!tw) {
+                            ok = false;
+                            break;
+                        }
+                        const int rv = t.kp1 - kbase;  // rows of the segment in this stage
+                        const int nz = kSK - rv;
+                        const int atoms = (a.a_tma ? 2 : 0) + (a.b_tma ? 4 : 0);
+                        for (int i = pt; i < nz * atoms * 8; i += kProducerThreads) {
+                            const int chunk = i & 7, rest = i >> 3;
+                            const int row = rv + rest % nz, at = rest / nz;
+                            const uint32_t base_at = (a.a_tma && at < 2) ? sa + at * kMnAtom
+                                                                         : sb + (at - (a.a_tma ? 2 : 0)) * kMnAtom;
+                            st_shared_v4(base_at + row * 128 + chunk * 16, 0u, 0u, 0u, 0u);
+                        }
+                        fence_proxy_async_smem();  // the zeros are read by the tensor cores
+                    }
+                    if (!a.a_tma) {
                         const int c = pt & 15, kr0 = pt >> 4;  // 16 chunks per 128-element A row
                         const int m = t.m0 + 8 * c;
 #pragma unroll
@@ -530,7 +571,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                                 cp_async_16_zfill(dst, a.a + (size_t)(in ? crow[i] : 0) * a.a_ld + m, in ? 16u : 0u);
                         }
                     }
-                    if (!a.b_tma || tail) {
+                    if (!a.b_tma) {
                         const int c = pt & 31, kr0 = pt >> 5;  // 32 chunks per 256-element B row
                         const int n = t.n0 + 8 * c;
 #pragma unroll
