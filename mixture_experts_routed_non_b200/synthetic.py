@@ -81,6 +81,11 @@ WORKLOADS = {
         "decode256", N=128, H=2048, I=512, E=256, K=8, routing="zipf", zipf_s=1.2,
         scores="softmax", seed=5,
         description="256-expert Zipf(1.2) imbalance, decode-sized"),
+    "profile_small": Workload(
+        "profile_small", N=4096, H=2048, I=768, E=32, K=8, routing="uniform",
+        scores="softmax", seed=7,
+        description="profiling case: the prefill shape with 32 experts and 4096 tokens "
+                    "(1024 rows per expert as in prefill, about 1 GB on the device)"),
     "prefill256": Workload(
         "prefill256", N=16384, H=2048, I=512, E=256, K=8, routing="zipf", zipf_s=1.2,
         scores="softmax", seed=6,
