@@ -483,6 +483,7 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
     BwdGemmArgs g;
     memset(&g, 0, sizeof g);
     g.expert_off = meta.expert_frequency_offset;
+    g.tile_off = reinterpret_cast<const int32_t *>(w + l.gemm_tile_offset);
     g.hdr = hdr;
     g.E = E;
     g.I = I;
@@ -496,7 +497,7 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         a.b = w2b;
         a.b_ld = H;
         a.b_rows_per_expert = I;
-        if (!make_map_a_chunks(&a.tmap_b, w2b, (uint64_t)H, (uint64_t)E * I, 256, 1)) return MOE_ERR_CUDA;
+        if (!make_map_a_chunks(&a.tmap_b, w2b, (uint64_t)H, (uint64_t)E * I, 128, 1)) return MOE_ERR_CUDA;
         a.b_tma = 1;
         a.z = zbuf;
         a.dz = dzbuf;
@@ -515,7 +516,7 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         a.b = dybuf;
         a.b_ld = H;
         if (!make_map_a_chunks(&a.tmap_a, hbuf, (uint64_t)I, prow, 64, 2) ||
-            !make_map_a_chunks(&a.tmap_b, dybuf, (uint64_t)H, prow, 64, 4))
+            !make_map_a_chunks(&a.tmap_b, dybuf, (uint64_t)H, prow, 64, 2))
             return MOE_ERR_CUDA;
         a.a_tma = a.b_tma = 1;
         a.out = static_cast<__nv_bfloat16 *>(dw2);
@@ -537,7 +538,7 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         a.b = dzbuf;
         a.b_ld = 2 * I;
         if (!make_map_a_chunks(&a.tmap_a, ybuf, (uint64_t)H, prow, 64, 2) ||
-            !make_map_a_chunks(&a.tmap_b, dzbuf, (uint64_t)2 * I, prow, 64, 4))
+            !make_map_a_chunks(&a.tmap_b, dzbuf, (uint64_t)2 * I, prow, 64, 2))
             return MOE_ERR_CUDA;
         a.a_tma = a.b_tma = 1;
         a.out = static_cast<__nv_bfloat16 *>(dw1);
@@ -556,7 +557,7 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
         a.b_ld = 2 * I;
         a.b_rows_per_expert = H;
         if (!make_map_a_chunks(&a.tmap_a, dzbuf, (uint64_t)2 * I, prow, 128, 1) ||
-            !make_map_a_chunks(&a.tmap_b, w1b, (uint64_t)2 * I, (uint64_t)E * H, 256, 1))
+            !make_map_a_chunks(&a.tmap_b, w1b, (uint64_t)2 * I, (uint64_t)E * H, 128, 1))
             return MOE_ERR_CUDA;
         a.a_tma = a.b_tma = 1;
         a.out = ybuf;

@@ -115,6 +115,7 @@ struct BwdGemmArgs {
     const __nv_bfloat16 *b;    // DH/DX: weights [E][N][K] (K contiguous); DW: [P_cap, N_dim] rows p
     int64_t b_ld;              // elements per row of `b`
     const int32_t *expert_off; // [E+1] segment offsets
+    const int32_t *tile_off;   // DH/DX: [E+1] prefix of ceil(freq / 256) (the metadata's GEMM tile table)
     __nv_bfloat16 *out;        // DX: [P_cap, N]; DW: [E][M][N]; DH: unused (writes z)
     int64_t out_ld;
     const float *z;            // DH: z [P_cap, 2I] fp32 (saved by the training forward)

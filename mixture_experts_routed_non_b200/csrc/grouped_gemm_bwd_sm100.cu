@@ -1,6 +1,6 @@
-// Grouped GEMMs of the backward on sm_100a: tcgen05 MMAs (cta_group::1,
-// M=128 x N=256 x K=16) with TMEM accumulators, operands staged in shared
-// memory by cp.async producer warps.  The pages leave the backward open
+// Grouped GEMMs of the backward on sm_100a: tcgen05 MMAs issued for a CTA pair
+// (cta_group::2, M=256 x N=256 x K=16) with TMEM accumulators, operands staged
+// in shared memory by TMA and cp.async.  The pages leave the backward open
 // (sonic-moe issue #68 asks how the scores' gradient returns to [N,K]; the
 // write-up names the layer a training layer); these are the chain rule of the
 // forward, over the same expert-sorted segments:
@@ -17,17 +17,21 @@
 //       (A = x rows gathered by token, B = dz).  K is the segment length; the
 //       rows past its end are zero-filled in both operands.
 //
-// DH and DX tile the segments in 128-row tiles (the tile table is rebuilt in
-// each CTA from the expert offsets); DW tiles each expert's [M,N] output.
+// A cluster of two CTAs owns a 256 x 256 tile: CTA r holds rows [128r, 128r+128)
+// of A and columns [128r, 128r+128) of B per stage, and its TMEM the fp32
+// accumulator of its 128 rows; the even CTA issues the pair MMAs and the
+// commits reach both CTAs.  DH and DX tile the segments in 256-row tiles (the
+// metadata's GEMM tile table); DW tiles each expert's [M,N] output.
 // Operands: K-major (rows of 64 contiguous K values, 128-byte swizzle) for
 // the row operands of DH/DX and for the weights read as [N][K]; MN-major
 // (rows = K, 64-element MN atoms, 128-byte swizzle) for both DW operands.
-// Warp roles: warp 0 = TMEM allocator and MMA issuer, then the epilogue warps
+// Warp roles: warp 0 = TMEM allocator and MMA issuer (even CTA) or the relay
+// that forwards the odd CTA's copy completions to the even CTA, then the epilogue warps
 // (TMEM lane quarter warp % 4; DH has two per quarter, splitting the columns),
 // one TMA producer warp (whole-stage boxes of every operand that needs no
 // gather) and four cp.async producer warps (the gathered rows, and the
-// zero-filled last stage of a DW segment).  Four
-// shared-memory stages, two TMEM accumulators.  Every wait is bounded; on a
+// zero-filled last stage of a DW segment).  Six
+// shared-memory stages of 32 KB per CTA, two TMEM accumulators.  Every wait is bounded; on a
 // timeout the CTA raises its abort flag, records MOE_DEVERR_TIMEOUT, drains
 // its MMAs and copies and frees its TMEM.
 #include "common.cuh"
@@ -36,10 +40,12 @@ namespace moe {
 
 namespace {
 
-constexpr int kM = 128;                      // tile rows (TMEM lanes)
+constexpr int kM = 128;                      // rows per CTA (TMEM lanes)
+constexpr int kPairM = 2 * kM;               // rows per tile (UMMA M of the pair)
 constexpr int kN = 256;                      // tile columns (UMMA N)
+constexpr int kNh = kN / 2;                  // B columns per CTA
 constexpr int kSK = 64;                      // K per stage: one 128-byte swizzle atom of bf16
-constexpr int kBwdStages = 4;
+constexpr int kBwdStages = 6;
 constexpr int kProducerThreads = 128;
 // Epilogue warps: 4 (one per TMEM lane quarter), or 8 for DH, whose SwiGLU
 // backward is heavy: two warps per quarter, each on half the columns.
@@ -52,11 +58,11 @@ struct Roles {
     static constexpr int kThreads = kCopyThread0 + kProducerThreads;  // MMA, epilogue, TMA, cp.async
 };
 constexpr uint32_t kStageA = kM * kSK * 2;   // 16 KB
-constexpr uint32_t kStageB = kN * kSK * 2;   // 32 KB
+constexpr uint32_t kStageB = kNh * kSK * 2;  // 16 KB
 constexpr uint32_t kStageBytes = kStageA + kStageB;
 constexpr uint32_t kMnAtom = kSK * 128;      // MN-major: one 64-element column of a stage (8 KB)
 constexpr uint32_t kTmemCols = 2 * kN;
-constexpr uint32_t kNumBars = 3 * kBwdStages + 5;
+constexpr uint32_t kNumBars = 4 * kBwdStages + 5;
 constexpr size_t kSmemBarOff = (size_t)kBwdStages * kStageBytes;
 constexpr size_t kSmemMiscOff = kSmemBarOff + 8 * kNumBars;
 constexpr size_t kSmemTableOff = kSmemMiscOff + 16;
@@ -67,7 +73,7 @@ constexpr unsigned long long kAbortSettleNs = 2000000ull;
 // each operand K-major or MN-major.
 __host__ __device__ constexpr uint32_t idesc(bool a_mn, bool b_mn) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
-           ((uint32_t)(kN >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
+           ((uint32_t)(kN >> 3) << 17) | ((uint32_t)(kPairM >> 4) << 24);
 }
 
 struct BTile {
@@ -75,7 +81,7 @@ struct BTile {
     int kp0, kp1;               // DW: segment rows [kp0, kp1)
 };
 
-// DH/DX: tile -> (expert, 128-row tile of its segment, 256-column tile)
+// DH/DX: tile -> (expert, 256-row tile of its segment, 256-column tile)
 __device__ __forceinline__ BTile decode_rows(int tile, int n_tiles, int E, const int *tile_off, const int *off,
                                              int K_dim) {
     BTile t;
@@ -88,7 +94,7 @@ __device__ __forceinline__ BTile decode_rows(int tile, int n_tiles, int E, const
         else hi = mid - 1;
     }
     t.e = lo;
-    t.m0 = off[lo] + (mt - tile_off[lo]) * kM;
+    t.m0 = off[lo] + (mt - tile_off[lo]) * kPairM;
     t.m_end = off[lo + 1];
     t.n0 = nt * kN;
     t.nk = K_dim / kSK;
@@ -96,15 +102,24 @@ __device__ __forceinline__ BTile decode_rows(int tile, int n_tiles, int E, const
     return t;
 }
 
-// DW: tile -> (expert, 128-row tile of its [M,N] output, 256-column tile)
-__device__ __forceinline__ BTile decode_weights(int tile, int m_tiles, int n_tiles, const int *off) {
+// DW: tile -> (expert, 256-row tile of its [M,N] output, 256-column tile).
+// Experts are taken kDwGroup at a time, the expert index varying fastest, so
+// the clusters running at once stream the rows of several experts from DRAM
+// while each expert's rows stay in L2 for its other tiles.
+constexpr int kDwGroup = 16;
+
+__device__ __forceinline__ BTile decode_weights(int tile, int m_tiles, int n_tiles, int E, const int *off) {
     BTile t;
     const int per = m_tiles * n_tiles;
-    t.e = tile / per;
-    const int r = tile - t.e * per;
-    const int mt = r / n_tiles;
-    t.m0 = mt * kM;
-    t.n0 = (r - mt * n_tiles) * kN;
+    const int g = tile / (kDwGroup * per);
+    const int e0 = g * kDwGroup;
+    const int ng = min(kDwGroup, E - e0);
+    const int r = tile - g * (kDwGroup * per);
+    t.e = e0 + r % ng;
+    const int tn = r / ng;
+    const int mt = tn / n_tiles;
+    t.m0 = mt * kPairM;
+    t.n0 = (tn - mt * n_tiles) * kN;
     t.kp0 = off[t.e];
     t.kp1 = off[t.e + 1];
     t.nk = (t.kp1 - t.kp0 + kSK - 1) / kSK;
@@ -128,7 +143,8 @@ __device__ __forceinline__ float silu_f(float g, float &sig) {
 }
 
 template <int kMode>
-__global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(const __grid_constant__ BwdGemmArgs a) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThreads, 1)
+    bwd_gemm_kernel(const __grid_constant__ BwdGemmArgs a) {
     using R = Roles<kMode>;
     constexpr int kThreads = R::kThreads;
     constexpr bool kMN = kMode == kBwdDW;  // both operands MN-major, K = segment rows
@@ -142,126 +158,136 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
     auto a_stage = [&](int s) { return base + (uint32_t)s * kStageBytes; };
     auto b_stage = [&](int s) { return base + (uint32_t)s * kStageBytes + kStageA; };
     const uint32_t bars = base + (uint32_t)kSmemBarOff;
-    auto full_bar = [&](int s) { return bars + 8u * s; };
+    auto full_bar = [&](int s) { return bars + 8u * s; };                       // even CTA: stage ready
     auto empty_bar = [&](int s) { return bars + 8u * (kBwdStages + s); };
-    auto tfull_bar = [&](int b) { return bars + 8u * (2 * kBwdStages + b); };
-    auto tempty_bar = [&](int b) { return bars + 8u * (2 * kBwdStages + 2 + b); };
-    const uint32_t drain_bar = bars + 8u * (2 * kBwdStages + 4);
-    auto tail_bar = [&](int s) { return bars + 8u * (2 * kBwdStages + 5 + s); };  // DW: a tail stage's TMA
+    auto gfull_bar = [&](int s) { return bars + 8u * (2 * kBwdStages + s); };   // odd CTA: its copies
+    auto tail_bar = [&](int s) { return bars + 8u * (3 * kBwdStages + s); };    // DW: a tail stage's TMA
+    auto tfull_bar = [&](int b) { return bars + 8u * (4 * kBwdStages + b); };
+    auto tempty_bar = [&](int b) { return bars + 8u * (4 * kBwdStages + 2 + b); };
+    const uint32_t drain_bar = bars + 8u * (4 * kBwdStages + 4);
     uint32_t *misc = reinterpret_cast<uint32_t *>(base_ptr + kSmemMiscOff);
     int *tile_off_s = reinterpret_cast<int *>(base_ptr + kSmemTableOff);
     int *off_s = tile_off_s + (kMaxExperts + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int row0 = (int)rank * kM;   // this CTA's first row inside a tile
+    const int col0b = (int)rank * kNh; // this CTA's first B column inside a tile
     const int E = a.E;
-    for (int i = threadIdx.x; i <= E; i += kThreads) off_s[i] = __ldg(a.expert_off + i);
+    for (int i = threadIdx.x; i <= E; i += kThreads) {
+        off_s[i] = __ldg(a.expert_off + i);
+        if (!kMN) tile_off_s[i] = __ldg(a.tile_off + i);
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kBwdStages; ++s) {
-            mbar_init(full_bar(s), kProducerThreads + 1);  // cp.async threads + TMA thread
+            // even CTA: its TMA thread + its copy threads + the odd CTA's relay
+            mbar_init(full_bar(s), 1 + kProducerThreads + 1);
             mbar_init(empty_bar(s), 1);
+            mbar_init(gfull_bar(s), kProducerThreads);
+            mbar_init(tail_bar(s), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(tfull_bar(b), 1);
-            mbar_init(tempty_bar(b), R::kEpiWarps);
+            mbar_init(tempty_bar(b), 2 * R::kEpiWarps);  // both CTAs' epilogue warps
         }
         mbar_init(drain_bar, 1);
-        for (int s = 0; s < kBwdStages; ++s) mbar_init(tail_bar(s), 1);
         misc[1] = 0;
         fence_barrier_init();
     }
     __syncthreads();
-    if (!kMN && warp == 1) {
-        // 128-row tiles per expert, exclusive prefix (one warp)
-        const int per = (E + 31) / 32;
-        const int e0 = lane * per;
-        int sum = 0;
-        for (int i = 0; i < per; ++i) {
-            const int e = e0 + i;
-            if (e < E) sum += (off_s[e + 1] - off_s[e] + kM - 1) / kM;
-        }
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-        }
-        int run = incl - sum;
-        for (int i = 0; i < per; ++i) {
-            const int e = e0 + i;
-            if (e < E) {
-                tile_off_s[e] = run;
-                run += (off_s[e + 1] - off_s[e] + kM - 1) / kM;
-            }
-        }
-        if (lane == 31) tile_off_s[E] = incl;
-    }
     if (warp == 0) {
-        tmem_alloc(smem_u32(&misc[0]), kTmemCols);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_u32(&misc[0]), kTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers initialised before any remote arrive
     tc_fence_after();
 
     const uint32_t tmem_base = misc[0];
     volatile uint32_t *abort = &misc[1];
     const int n_tiles = (a.N_dim + kN - 1) / kN;
-    const int m_tiles = kMN ? (a.M_dim + kM - 1) / kM : 0;
+    const int m_tiles = kMN ? (a.M_dim + kPairM - 1) / kPairM : 0;
+    const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
     const int total = kMN ? E * m_tiles * n_tiles : tile_off_s[E] * n_tiles;
     auto decode = [&](int tile) {
-        return kMN ? decode_weights(tile, m_tiles, n_tiles, off_s)
+        return kMN ? decode_weights(tile, m_tiles, n_tiles, E, off_s)
                    : decode_rows(tile, n_tiles, E, tile_off_s, off_s, a.K_dim);
     };
 
     if (warp == 0) {
-        // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        if (rank == 0) {
+            // ---------------------------------------------------- MMA issuer (even CTA)
+            if (lane == 0) {
+                int stage = 0;
+                uint32_t phase = 0;
+                int tcount = 0;
+                bool ok = true;
+                for (int tile = cluster; ok && tile < total; tile += n_clusters, ++tcount) {
+                    const BTile t = decode(tile);
+                    const int acc = tcount & 1;
+                    const uint32_t acc_phase = (tcount >> 1) & 1;
+                    if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort)) break;
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + acc * kN;
+                    for (int kb = 0; kb < t.nk; ++kb) {
+                        // one barrier per stage: both CTAs' TMA bytes, this CTA's copies
+                        // and the relayed copies of the odd CTA
+                        if (!mbar_wait_bounded(full_bar(stage), phase, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        fence_proxy_async_smem();  // copies and zeroed rows (generic proxy) -> tensor cores
+                        const uint32_t sa = a_stage(stage), sb = b_stage(stage);
+#pragma unroll
+                        for (int kk = 0; kk < kSK / kUmmaK; ++kk) {
+                            uint64_t ad, bd;
+                            if (kMN) {
+                                // rows = K (128 B each, 8-row groups 1024 B apart), 64-element
+                                // MN columns kMnAtom apart; K step = 16 rows
+                                ad = smem_desc_sw128(sa + kk * (kUmmaK * 128), kMnAtom, 1024);
+                                bd = smem_desc_sw128(sb + kk * (kUmmaK * 128), kMnAtom, 1024);
+                            } else {
+                                // rows = M or N (128 B of K each, 8-row groups 1024 B apart);
+                                // K step = 32 B inside the swizzle atom
+                                ad = smem_desc_sw128(sa + kk * (kUmmaK * 2), 16, 1024);
+                                bd = smem_desc_sw128(sb + kk * (kUmmaK * 2), 16, 1024);
+                            }
+                            umma_f16_pair(d_tmem, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                        }
+                        umma_commit_pair_mc(empty_bar(stage), 0x3);
+                        if (++stage == kBwdStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit_pair_mc(tfull_bar(acc), 0x3);  // with no MMA (empty segment) at once
+                }
+                umma_commit_pair(drain_bar);  // every MMA issued here completes before TMEM is freed
+                mbar_wait_timed(drain_bar, 0);
+            }
+        } else if (lane == 0) {
+            // ------------------------------------------------------- relay (odd CTA)
+            // forwards the completion of this CTA's copy threads to the even CTA
             int stage = 0;
             uint32_t phase = 0;
-            int tcount = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x, ++tcount) {
+            for (int tile = cluster; ok && tile < total; tile += n_clusters) {
                 const BTile t = decode(tile);
-                const int acc = tcount & 1;
-                const uint32_t acc_phase = (tcount >> 1) & 1;
-                if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * kN;
                 for (int kb = 0; kb < t.nk; ++kb) {
-                    if (!mbar_wait_bounded(full_bar(stage), phase, abort)) {
+                    if (!mbar_wait_bounded(gfull_bar(stage), phase, abort)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    fence_proxy_async_smem();  // cp.async (generic proxy) data -> tensor-core reads
-                    const uint32_t sa = a_stage(stage), sb = b_stage(stage);
-#pragma unroll
-                    for (int kk = 0; kk < kSK / kUmmaK; ++kk) {
-                        uint64_t ad, bd;
-                        if (kMN) {
-                            // rows = K (128 B each, 8-row groups 1024 B apart), 64-element
-                            // MN columns kMnAtom apart; K step = 16 rows
-                            ad = smem_desc_sw128(sa + kk * (kUmmaK * 128), kMnAtom, 1024);
-                            bd = smem_desc_sw128(sb + kk * (kUmmaK * 128), kMnAtom, 1024);
-                        } else {
-                            // rows = M or N (128 B of K each, 8-row groups 1024 B apart);
-                            // K step = 32 B inside the swizzle atom
-                            ad = smem_desc_sw128(sa + kk * (kUmmaK * 2), 16, 1024);
-                            bd = smem_desc_sw128(sb + kk * (kUmmaK * 2), 16, 1024);
-                        }
-                        umma_f16(d_tmem, ad, bd, kIdesc, (kb | kk) != 0 ? 1u : 0u);
-                    }
-                    umma_commit(empty_bar(stage));
+                    fence_proxy_async_smem();
+                    mbar_arrive_cluster(mapa_shared(full_bar(stage), 0));
                     if (++stage == kBwdStages) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
-                if (!ok) break;
-                umma_commit(tfull_bar(acc));  // with no MMA (empty segment) it arrives at once
             }
-            umma_commit(drain_bar);  // every MMA issued here completes before TMEM is freed
-            mbar_wait_timed(drain_bar, 0);
         }
         __syncwarp();
     } else if (warp < R::kTmaWarp) {
@@ -270,13 +296,13 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
         const int rl = quarter * 32 + lane;  // this thread's tile row (TMEM lane)
         const int part = (warp - 1) >> 2;    // this warp's part of the tile's columns
         int tcount = 0;
-        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++tcount) {
+        for (int tile = cluster; tile < total; tile += n_clusters, ++tcount) {
             const BTile t = decode(tile);
             const int acc = tcount & 1;
             const uint32_t acc_phase = (tcount >> 1) & 1;
             if (kMode == kBwdDH) {
                 // bring this row's z columns of the tile into L2 while the MMAs run
-                const int p = t.m0 + rl;
+                const int p = t.m0 + row0 + rl;
                 if (p < t.m_end) {
                     const int c0 = t.n0 + part * (kN / R::kParts);  // this warp's first I column
                     const int ncols = min(kN / R::kParts, a.I - c0);
@@ -298,7 +324,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
             tc_fence_after();
             const uint32_t tbase = tmem_base + acc * kN + ((uint32_t)(quarter * 32) << 16);
             if (kMode == kBwdDH) {
-                const int p = t.m0 + rl;
+                const int p = t.m0 + row0 + rl;
                 const bool valid = p < t.m_end;
                 const size_t zoff = (size_t)(valid ? p : 0) * (2 * a.I);
                 const float *zrow = a.z + zoff;
@@ -362,7 +388,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                 }
             } else {
                 // DX: row p of dxs; DW: row m of expert e's [M,N] output
-                const int r = kMode == kBwdDX ? t.m0 + rl : t.m0 + rl;
+                const int r = t.m0 + row0 + rl;
                 const bool valid = kMode == kBwdDX ? r < t.m_end : r < a.M_dim;
                 const size_t row_off = kMode == kBwdDX
                                            ? (size_t)(valid ? r : 0) * a.out_ld
@@ -400,19 +426,24 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(tempty_bar(acc));
+            if (lane == 0) {
+                if (rank == 0) mbar_arrive(tempty_bar(acc));
+                else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
+            }
         }
     } else if (warp == R::kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
         // whole-stage boxes of the operands that need no gather: 128-byte-swizzled
-        // [atom][row][128 B] boxes of a (64, rows, cols/64) view of each matrix
+        // [atom][row][128 B] boxes of a (64, rows, cols/64) view of each matrix.
+        // Both CTAs' boxes complete on the even CTA's stage barrier; a DW
+        // segment's last stage instead lands on each CTA's own tail barrier.
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, issued_parity = 0;
             uint32_t tissued = 0, tissued_parity = 0, tphase = 0;  // tail-stage TMAs (DW)
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+            for (int tile = cluster; ok && tile < total; tile += n_clusters) {
                 const BTile t = decode(tile);
                 for (int kb = 0; kb < t.nk; ++kb) {
                     if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort)) {
@@ -420,35 +451,38 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                         break;
                     }
                     const int kbase = t.kp0 + kb * kSK;
-                    // a DW segment's last stage: the TMA lands on tail_bar, the copy
-                    // warps zero the rows past the segment end, then arrive on full
                     const bool tail = kMN && kbase + kSK > t.kp1;
                     const bool ta = a.a_tma != 0, tb = a.b_tma != 0;
                     const uint32_t bytes = (ta ? kStageA : 0u) + (tb ? kStageB : 0u);
                     if (tail && bytes) {
+                        // this CTA's boxes, on its own barrier; the copy warps zero the
+                        // rows past the segment end, then release the stage
                         const uint32_t tb_bar = tail_bar(stage);
                         mbar_arrive_expect_tx(tb_bar, bytes);
-                        if (ta) tma_load_3d(a_stage(stage), &a.tmap_a, tb_bar, 0, kbase, t.m0 / 64);
-                        if (tb) tma_load_3d(b_stage(stage), &a.tmap_b, tb_bar, 0, kbase, t.n0 / 64);
+                        if (ta) tma_load_3d(a_stage(stage), &a.tmap_a, tb_bar, 0, kbase, (t.m0 + row0) / 64);
+                        if (tb) tma_load_3d(b_stage(stage), &a.tmap_b, tb_bar, 0, kbase, (t.n0 + col0b) / 64);
                         const uint32_t par = (tphase >> stage) & 1u;
                         tissued |= 1u << stage;
                         tissued_parity = (tissued_parity & ~(1u << stage)) | (par << stage);
                         tphase ^= 1u << stage;
-                        mbar_arrive(full_bar(stage));
+                        if (rank == 0) mbar_arrive(full_bar(stage));
                     } else if (bytes) {
-                        mbar_arrive_expect_tx(full_bar(stage), bytes);
+                        // both CTAs' bytes are expected by the even CTA's barrier
+                        if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * bytes);
+                        const uint32_t fb = mapa_shared(full_bar(stage), 0);
                         if (kMN) {
-                            if (ta) tma_load_3d(a_stage(stage), &a.tmap_a, full_bar(stage), 0, kbase, t.m0 / 64);
-                            if (tb) tma_load_3d(b_stage(stage), &a.tmap_b, full_bar(stage), 0, kbase, t.n0 / 64);
-                        } else {
-                            if (ta) tma_load_3d(a_stage(stage), &a.tmap_a, full_bar(stage), 0, t.m0, kb);
+                            if (ta) tma_load_3d_pair(a_stage(stage), &a.tmap_a, fb, 0, kbase, (t.m0 + row0) / 64);
                             if (tb)
-                                tma_load_3d(b_stage(stage), &a.tmap_b, full_bar(stage), 0,
-                                            t.e * a.b_rows_per_expert + t.n0, kb);
+                                tma_load_3d_pair(b_stage(stage), &a.tmap_b, fb, 0, kbase, (t.n0 + col0b) / 64);
+                        } else {
+                            if (ta) tma_load_3d_pair(a_stage(stage), &a.tmap_a, fb, 0, t.m0 + row0, kb);
+                            if (tb)
+                                tma_load_3d_pair(b_stage(stage), &a.tmap_b, fb, 0,
+                                                 t.e * a.b_rows_per_expert + t.n0 + col0b, kb);
                         }
                         issued |= 1u << stage;
                         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
-                    } else {
+                    } else if (rank == 0) {
                         mbar_arrive(full_bar(stage));
                     }
                     if (++stage == kBwdStages) {
@@ -457,9 +491,11 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                     }
                 }
             }
-            // the CTA may not exit while a TMA it issued can still write its memory
+            // the CTA may not exit while a TMA it issued can still write its memory:
+            // the even CTA's stage barriers count both CTAs' boxes (the odd CTA is
+            // held by the final cluster barrier until this drain ends)
             for (int st = 0; st < kBwdStages; ++st) {
-                if (issued & (1u << st)) mbar_wait_timed(full_bar(st), (issued_parity >> st) & 1u);
+                if (rank == 0 && (issued & (1u << st))) mbar_wait_timed(full_bar(st), (issued_parity >> st) & 1u);
                 if (tissued & (1u << st)) mbar_wait_timed(tail_bar(st), (tissued_parity >> st) & 1u);
             }
         }
@@ -474,7 +510,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
         uint32_t tpar = 0;  // parity of each stage's next tail_bar phase
         bool ok = true;
         const int gl = pt & 31;
-        for (int tile = blockIdx.x; ok && tile < total; tile += gridDim.x) {
+        for (int tile = cluster; ok && tile < total; tile += n_clusters) {
             const BTile t = decode(tile);
             // K-major gathered rows (DH): this thread's 8 row pointers, once per tile
             // (null past the segment end: those rows feed unstored outputs only)
@@ -482,7 +518,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
             if (!kMN && !a.a_tma) {
 #pragma unroll
                 for (int i = 0; i < kM / 16; ++i) {
-                    const int p = t.m0 + (pt >> 3) + 16 * i;
+                    const int p = t.m0 + row0 + (pt >> 3) + 16 * i;
                     arow[i] = p < t.m_end ? a.a + (size_t)(a.a_rows ? __ldg(a.a_rows + p) : p) * a.a_ld : nullptr;
                 }
             }
@@ -525,9 +561,9 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                     if (!a.b_tma) {
                         const __nv_bfloat16 *bw = a.b + (size_t)t.e * a.b_rows_per_expert * a.b_ld;
 #pragma unroll
-                        for (int i = 0; i < kN / 16; ++i) {
+                        for (int i = 0; i < kNh / 16; ++i) {
                             const int r = r0 + 16 * i;
-                            const int n = t.n0 + r;  // columns past N_dim are never stored
+                            const int n = t.n0 + col0b + r;  // columns past N_dim are never stored
                             if (n < a.N_dim)
                                 cp_async_16(sb + r * 128 + ((c ^ (r & 7)) << 4), bw + (size_t)n * a.b_ld + k0);
                         }
@@ -549,7 +585,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                         }
                         const int rv = t.kp1 - kbase;  // rows of the segment in this stage
                         const int nz = kSK - rv;
-                        const int atoms = (a.a_tma ? 2 : 0) + (a.b_tma ? 4 : 0);
+                        const int atoms = (a.a_tma ? 2 : 0) + (a.b_tma ? 2 : 0);
                         for (int i = pt; i < nz * atoms * 8; i += kProducerThreads) {
                             const int chunk = i & 7, rest = i >> 3;
                             const int row = rv + rest % nz, at = rest / nz;
@@ -561,7 +597,7 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                     }
                     if (!a.a_tma) {
                         const int c = pt & 15, kr0 = pt >> 4;  // 16 chunks per 128-element A row
-                        const int m = t.m0 + 8 * c;
+                        const int m = t.m0 + row0 + 8 * c;
 #pragma unroll
                         for (int i = 0; i < kSK / 8; ++i) {
                             const int kr = kr0 + 8 * i;
@@ -572,11 +608,11 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                         }
                     }
                     if (!a.b_tma) {
-                        const int c = pt & 31, kr0 = pt >> 5;  // 32 chunks per 256-element B row
-                        const int n = t.n0 + 8 * c;
+                        const int c = pt & 15, kr0 = pt >> 4;  // 16 chunks per 128-element B row
+                        const int n = t.n0 + col0b + 8 * c;
 #pragma unroll
-                        for (int i = 0; i < kSK / 4; ++i) {
-                            const int kr = kr0 + 4 * i;
+                        for (int i = 0; i < kSK / 8; ++i) {
+                            const int kr = kr0 + 8 * i;
                             const int p = kbase + kr;
                             const bool in = p < t.kp1;
                             const uint32_t dst = sb + (c >> 3) * kMnAtom + kr * 128 + (((c & 7) ^ (kr & 7)) << 4);
@@ -585,7 +621,9 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
                         }
                     }
                 }
-                cp_async_arrive_noinc(full_bar(stage));
+                // even CTA: straight onto the stage barrier; odd CTA: onto gfull,
+                // which its relay forwards to the even CTA
+                cp_async_arrive_noinc(rank == 0 ? full_bar(stage) : gfull_bar(stage));
                 if (++stage == kBwdStages) {
                     stage = 0;
                     phase ^= 1u;
@@ -600,34 +638,47 @@ __global__ void __launch_bounds__(Roles<kMode>::kThreads, 1) bwd_gemm_kernel(con
     __syncthreads();
     if (*abort) {
         if (threadIdx.x == 0) atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);
-        settle_after_abort();
+        settle_after_abort();  // let copies issued by the peer CTA land
     }
+    cluster_sync_all();  // no CTA leaves while its peer may still touch it
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 }
 
 template <int kMode>
 cudaError_t launch_mode(const BwdGemmArgs &a, int max_ctas, cudaStream_t s) {
-    static bool configured[64] = {};
+    static int fit_cache[64] = {};
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
     if (err != cudaSuccess) return err;
     if (dev >= 64) return cudaErrorInvalidDevice;
-    if (!configured[dev]) {
+    int &fit = fit_cache[dev];
+    if (fit == 0) {
         err = cudaFuncSetAttribute(bwd_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)kSmemBytes);
         if (err != cudaSuccess) return err;
-        configured[dev] = true;
+        // clusters that can be resident at once (one CTA per SM: the shared
+        // memory allows no second)
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(max_ctas & ~1));
+        cfg.blockDim = dim3(Roles<kMode>::kThreads);
+        cfg.dynamicSmemBytes = kSmemBytes;
+        int n = 0;
+        err = cudaOccupancyMaxActiveClusters(&n, bwd_gemm_kernel<kMode>, &cfg);
+        if (err != cudaSuccess) return err;
+        fit = n > 0 ? n : 1;
     }
-    int ctas = max_ctas;
+    int clusters = max_ctas / 2;
+    if (clusters > fit) clusters = fit;
     if (kMode == kBwdDW) {
-        const int total = a.E * ((a.M_dim + kM - 1) / kM) * ((a.N_dim + kN - 1) / kN);
-        if (total < ctas) ctas = total;
+        const int total = a.E * ((a.M_dim + kPairM - 1) / kPairM) * ((a.N_dim + kN - 1) / kN);
+        if (total < clusters) clusters = total;
     }
-    if (ctas < 1) ctas = 1;
-    bwd_gemm_kernel<kMode><<<ctas, Roles<kMode>::kThreads, kSmemBytes, s>>>(a);
+    if (clusters < 1) clusters = 1;
+    // the kernel's cluster shape (2,1,1) is compiled in (__cluster_dims__)
+    bwd_gemm_kernel<kMode><<<2 * clusters, Roles<kMode>::kThreads, kSmemBytes, s>>>(a);
     return cudaGetLastError();
 }
 
