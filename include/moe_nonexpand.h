@@ -326,6 +326,27 @@ MOE_API int moe_nonexpand_backward_timed(const void *dout, const void *x, const 
                                          size_t ws_bytes, moe_stream_t stream, const moe_event_t *stage_events);
 
 /*
+ * Training for either routing layout (moe_routing_t; see the routed calls):
+ * the same computation as moe_nonexpand_forward_train / moe_nonexpand_backward.
+ * dweights has the shape of routing->weights ([N,K] for the table, [P] for a
+ * pair list) and receives each slot's score gradient, 0 at slots that are no
+ * pair (expert -1, bad ids, bad tokens).
+ */
+MOE_API size_t moe_nonexpand_routed_train_workspace_bytes(const moe_routing_t *routing, int32_t H, int32_t I,
+                                                          int32_t E);
+
+MOE_API int moe_nonexpand_routed_forward_train(const void *x, const moe_routing_t *routing, int32_t H, int32_t I,
+                                               int32_t E, const void *w1, const void *b1, const void *w2,
+                                               const void *b2, int32_t activation, int32_t gate_up_layout,
+                                               void *out, void *ws, size_t ws_bytes, moe_stream_t stream);
+
+MOE_API int moe_nonexpand_routed_backward(const void *dout, const void *x, const moe_routing_t *routing, int32_t H,
+                                          int32_t I, int32_t E, const void *w1, const void *w2, int32_t activation,
+                                          int32_t gate_up_layout, void *dx, void *dw1, void *db1, void *dw2,
+                                          void *db2, float *dweights, void *ws, size_t ws_bytes,
+                                          moe_stream_t stream);
+
+/*
  * Router top-k: router logits [N,E] -> the routing table topk_idx [N,K] /
  * topk_w [N,K] that moe_nonexpand_forward takes (sonic-moe write-up, "Three
  * routing strategies, selected on the command line": TC top-K routing is the
@@ -377,6 +398,8 @@ typedef struct moe_ws_layout_t {
     size_t z;                  /* training workspace: fp32 [P_cap,2I], z saved by the forward */
     size_t dz;                 /* training workspace: bf16 [P_cap,2I], dz of the backward */
     size_t dy;                 /* training workspace: bf16 [P_cap,H], dy of the backward */
+    size_t slot_pair;          /* training workspace: int32 [slots], the pair of each routing slot or -1 */
+    size_t ds;                 /* training workspace: fp32 [P_cap], score gradients in pair order */
     size_t train_total;        /* == moe_nonexpand_train_workspace_bytes(...) */
 } moe_ws_layout_t;
 

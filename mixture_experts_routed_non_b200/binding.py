@@ -58,6 +58,9 @@ EXPORTED = (
     "moe_nonexpand_forward_train",
     "moe_nonexpand_backward",
     "moe_nonexpand_backward_timed",
+    "moe_nonexpand_routed_train_workspace_bytes",
+    "moe_nonexpand_routed_forward_train",
+    "moe_nonexpand_routed_backward",
 )
 
 ROUTER_SOFTMAX_TOPK = 0
@@ -80,7 +83,7 @@ class WsLayout(ctypes.Structure):
         "meta_token_offset", "meta_scores", "h", "y")] + [
         ("p_cap", ctypes.c_int64), ("meta_tiles", ctypes.c_int32), ("meta_tile_slots", ctypes.c_int32),
         ("z", ctypes.c_size_t), ("dz", ctypes.c_size_t), ("dy", ctypes.c_size_t),
-        ("train_total", ctypes.c_size_t)]
+        ("slot_pair", ctypes.c_size_t), ("ds", ctypes.c_size_t), ("train_total", ctypes.c_size_t)]
 
 
 class MoeRouting(ctypes.Structure):
@@ -147,6 +150,12 @@ def load() -> ctypes.CDLL:
     lib.moe_nonexpand_backward.argtypes = bwd
     lib.moe_nonexpand_backward_timed.restype = ctypes.c_int
     lib.moe_nonexpand_backward_timed.argtypes = bwd + [P]
+    lib.moe_nonexpand_routed_train_workspace_bytes.restype = sz
+    lib.moe_nonexpand_routed_train_workspace_bytes.argtypes = [R, i32, i32, i32]
+    lib.moe_nonexpand_routed_forward_train.restype = ctypes.c_int
+    lib.moe_nonexpand_routed_forward_train.argtypes = [P, R, i32, i32, i32, P, P, P, P, i32, i32, P, P, sz, P]
+    lib.moe_nonexpand_routed_backward.restype = ctypes.c_int
+    lib.moe_nonexpand_routed_backward.argtypes = [P, P, R, i32, i32, i32, P, P, i32, i32, P, P, P, P, P, P, P, sz, P]
     lib.moe_nonexpand_strerror.restype = ctypes.c_char_p
     lib.moe_nonexpand_strerror.argtypes = [ctypes.c_int]
     _lib = lib
@@ -606,3 +615,56 @@ def backward(dout: torch.Tensor, x: torch.Tensor, topk_idx: torch.Tensor, topk_w
         arr = (ctypes.c_void_p * 8)(*[ev.cuda_event for ev in events])
         _check(lib.moe_nonexpand_backward_timed(*args, arr), "moe_nonexpand_backward_timed")
     return grads
+
+
+def routed_train_workspace_bytes(r: MoeRouting, H: int, I: int, E: int) -> int:
+    n = load().moe_nonexpand_routed_train_workspace_bytes(ctypes.byref(r), H, I, E)
+    if n == 0:
+        raise MoeError(MOE_ERR_ARG, "moe_nonexpand_routed_train_workspace_bytes")
+    return n
+
+
+def routed_forward_train(x: torch.Tensor, expert_idx: torch.Tensor, weights: torch.Tensor, w1: torch.Tensor,
+                         w2: torch.Tensor, b1: Optional[torch.Tensor] = None, b2: Optional[torch.Tensor] = None, *,
+                         ws: torch.Tensor, token_idx: Optional[torch.Tensor] = None,
+                         layout: int = LAYOUT_INTERLEAVED, total_pairs: int = -1,
+                         out: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """moe_nonexpand_routed_forward_train for either routing layout."""
+    N, H = x.shape
+    E, _, I2 = w1.shape
+    I = I2 // 2
+    dev = x.device
+    r = routing(expert_idx, weights, token_idx=token_idx, N=N, total_pairs=total_pairs)
+    if out is None:
+        out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+    _check(load().moe_nonexpand_routed_forward_train(x.data_ptr(), ctypes.byref(r), H, I, E, w1.data_ptr(),
+                                                     _ptr(b1), w2.data_ptr(), _ptr(b2), ACT_SWIGLU, layout,
+                                                     out.data_ptr(), ws.data_ptr(), ws.numel(),
+                                                     _stream_handle(stream)), "moe_nonexpand_routed_forward_train")
+    return out
+
+
+def routed_backward(dout: torch.Tensor, x: torch.Tensor, expert_idx: torch.Tensor, weights: torch.Tensor,
+                    w1: torch.Tensor, w2: torch.Tensor, *, ws: torch.Tensor, token_idx: Optional[torch.Tensor] = None,
+                    layout: int = LAYOUT_INTERLEAVED, total_pairs: int = -1, bias_grads: bool = False,
+                    stream: Optional[torch.cuda.Stream] = None) -> dict:
+    """moe_nonexpand_routed_backward: dict(dx, dw1, dw2, dweights[, db1, db2]);
+    dweights has the shape of ``weights``."""
+    N, H = x.shape
+    E, _, I2 = w1.shape
+    I = I2 // 2
+    dev = x.device
+    r = routing(expert_idx, weights, token_idx=token_idx, N=N, total_pairs=total_pairs)
+    g = dict(dx=torch.empty((N, H), dtype=torch.bfloat16, device=dev),
+             dw1=torch.empty((E, H, 2 * I), dtype=torch.bfloat16, device=dev),
+             dw2=torch.empty((E, I, H), dtype=torch.bfloat16, device=dev),
+             dweights=torch.empty(weights.shape, dtype=torch.float32, device=dev))
+    if bias_grads:
+        g["db1"] = torch.empty((E, 2 * I), dtype=torch.bfloat16, device=dev)
+        g["db2"] = torch.empty((E, H), dtype=torch.bfloat16, device=dev)
+    _check(load().moe_nonexpand_routed_backward(dout.data_ptr(), x.data_ptr(), ctypes.byref(r), H, I, E,
+                                                w1.data_ptr(), w2.data_ptr(), ACT_SWIGLU, layout, g["dx"].data_ptr(),
+                                                g["dw1"].data_ptr(), _ptr(g.get("db1")), g["dw2"].data_ptr(),
+                                                _ptr(g.get("db2")), g["dweights"].data_ptr(), ws.data_ptr(),
+                                                ws.numel(), _stream_handle(stream)), "moe_nonexpand_routed_backward")
+    return g

@@ -5,9 +5,10 @@
 //   prep      per token t and each of its pairs q (sorted position p):
 //             ds_q = <dout_t, y_p> (the score's gradient, fp32, summed in a
 //             fixed order) and dy_p = s_q dout_t (bf16 [P_cap,H]); ds is then
-//             scattered to the [N,K] slot it came from (0 at invalid slots) --
-//             sonic-moe issue #68 asks for the scores' gradient back in the
-//             non-expand layout.
+//             scattered to the routing slot each pair came from through the
+//             slot -> pair index the training forward's metadata recorded (0 at
+//             slots that are no pair) -- sonic-moe issue #68 asks for the
+//             scores' gradient back in the routing layout.
 //   bias      db[e,c] = sum of the segment's rows of dy (db2) or dz (db1), in
 //             row order, fp32, rounded once to bf16.
 //   gather    xs[p,:] = x[x_gather_idx[p],:], so the dW1 GEMM reads its A
@@ -34,70 +35,65 @@ __device__ __forceinline__ uint4 scale8(const uint4 &v, float s) {
 }
 
 // One block per token (grid-stride).  Each thread owns 16-byte column chunks
-// of the row; per pair it accumulates its share of the dot product, then the
-// block reduces all pairs' partials at once (warp butterfly, then warps in
-// order).
+// of the row; for up to 32 pairs at a time it accumulates its share of each
+// dot product, then the block reduces those partials at once (warp
+// butterfly, then warps in order).  A pair list may give a token any number
+// of pairs, hence the batches of 32.
 __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
-    const __nv_bfloat16 *__restrict__ dout, const __nv_bfloat16 *__restrict__ y, const int32_t *__restrict__ topk_idx,
+    const __nv_bfloat16 *__restrict__ dout, const __nv_bfloat16 *__restrict__ y,
     const int32_t *__restrict__ token_offset, const int32_t *__restrict__ s_rev, const float *__restrict__ scores,
-    int64_t N, int32_t H, int32_t K, int32_t E, __nv_bfloat16 *__restrict__ dy, float *__restrict__ dtopk_w,
-    const WsHeader *hdr) {
+    int64_t N, int32_t H, __nv_bfloat16 *__restrict__ dy, float *__restrict__ ds, const WsHeader *hdr) {
     __shared__ float part[kPrepWarps][kMaxSlots];
-    __shared__ float ds_s[kMaxSlots];
     if (hdr && *(volatile const uint32_t *)&hdr->abort) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int chunks = H >> 3;
     for (int64_t t = blockIdx.x; t < N; t += gridDim.x) {
         const int q0 = __ldg(token_offset + t), q1 = __ldg(token_offset + t + 1);
-        const int np = q1 - q0;  // <= K
         const __nv_bfloat16 *drow = dout + (size_t)t * H;
-        float acc[kMaxSlots];
+        for (int qb = q0; qb < q1; qb += kMaxSlots) {
+            const int np = min(kMaxSlots, q1 - qb);
+            float acc[kMaxSlots];
 #pragma unroll
-        for (int j = 0; j < kMaxSlots; ++j) acc[j] = 0.f;
-        for (int c = threadIdx.x; c < chunks; c += kPrepThreads) {
-            const uint4 d = __ldg(reinterpret_cast<const uint4 *>(drow) + c);
+            for (int j = 0; j < kMaxSlots; ++j) acc[j] = 0.f;
+            for (int c = threadIdx.x; c < chunks; c += kPrepThreads) {
+                const uint4 d = __ldg(reinterpret_cast<const uint4 *>(drow) + c);
+#pragma unroll
+                for (int j = 0; j < kMaxSlots; ++j) {
+                    if (j >= np) break;
+                    const int p = __ldg(s_rev + qb + j);
+                    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + (size_t)p * H) + c);
+                    acc[j] += dot8(d, v);
+                    reinterpret_cast<uint4 *>(dy + (size_t)p * H)[c] = scale8(d, __ldg(scores + qb + j));
+                }
+            }
 #pragma unroll
             for (int j = 0; j < kMaxSlots; ++j) {
                 if (j >= np) break;
-                const int p = __ldg(s_rev + q0 + j);
-                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + (size_t)p * H) + c);
-                acc[j] += dot8(d, v);
-                reinterpret_cast<uint4 *>(dy + (size_t)p * H)[c] = scale8(d, __ldg(scores + q0 + j));
+                float v = acc[j];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0) part[warp][j] = v;
             }
-        }
+            __syncthreads();
+            if (threadIdx.x < np) {
+                float v = 0.f;
 #pragma unroll
-        for (int j = 0; j < kMaxSlots; ++j) {
-            if (j >= np) break;
-            float v = acc[j];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) part[warp][j] = v;
-        }
-        __syncthreads();
-        if (threadIdx.x < np) {
-            float v = 0.f;
-#pragma unroll
-            for (int w = 0; w < kPrepWarps; ++w) v += part[w][threadIdx.x];
-            ds_s[threadIdx.x] = v;
-        }
-        __syncthreads();
-        if (threadIdx.x < K) {
-            // the j-th valid slot of the row holds pair q0 + j
-            const int32_t *row = topk_idx + (size_t)t * K;
-            const int k = threadIdx.x;
-            const int e = __ldg(row + k);
-            float g = 0.f;
-            if (e >= 0 && e < E) {
-                int j = 0;
-                for (int kk = 0; kk < k; ++kk) {
-                    const int ek = __ldg(row + kk);
-                    j += (ek >= 0 && ek < E) ? 1 : 0;
-                }
-                g = j < np ? ds_s[j] : 0.f;
+                for (int w = 0; w < kPrepWarps; ++w) v += part[w][threadIdx.x];
+                ds[qb + threadIdx.x] = v;  // pair order; scattered to the slots afterwards
             }
-            dtopk_w[(size_t)t * K + k] = g;
+            __syncthreads();  // part is reused by the next batch
         }
-        __syncthreads();  // part / ds_s are reused by the next token
+    }
+}
+
+// dweights[s] = ds[slot_pair[s]] where slot s is a pair, else 0.
+__global__ void __launch_bounds__(256) scatter_slots_kernel(const int32_t *__restrict__ slot_pair,
+                                                            const float *__restrict__ ds, int64_t NK,
+                                                            float *__restrict__ dweights, const WsHeader *hdr) {
+    if (hdr && *(volatile const uint32_t *)&hdr->abort) return;
+    for (int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; s < NK; s += (int64_t)gridDim.x * blockDim.x) {
+        const int q = __ldg(slot_pair + s);
+        dweights[s] = q >= 0 ? __ldg(ds + q) : 0.f;
     }
 }
 
@@ -159,16 +155,25 @@ cudaError_t launch_gather_rows(const __nv_bfloat16 *src, const int32_t *idx, con
     return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const __nv_bfloat16 *y, const int32_t *topk_idx,
-                            const moe_meta_t &meta, int64_t N, int32_t H, int32_t K, int32_t E, __nv_bfloat16 *dy,
-                            float *dtopk_w, const WsHeader *hdr, int num_sms, cudaStream_t s) {
-    if (N == 0) return cudaSuccess;
-    int64_t blocks = N;
-    const int64_t cap = (int64_t)num_sms * 8;
-    if (blocks > cap) blocks = cap;
-    bwd_prep_kernel<<<(unsigned)blocks, kPrepThreads, 0, s>>>(dout, y, topk_idx, meta.token_offset,
-                                                              meta.s_reverse_scatter_idx, meta.scores, N, H, K, E,
-                                                              dy, dtopk_w, hdr);
+cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const __nv_bfloat16 *y, const moe_meta_t &meta, int64_t N,
+                            int32_t H, __nv_bfloat16 *dy, float *ds, const int32_t *slot_pair, int64_t NK,
+                            float *dweights, const WsHeader *hdr, int num_sms, cudaStream_t s) {
+    if (N > 0) {
+        int64_t blocks = N;
+        const int64_t cap = (int64_t)num_sms * 8;
+        if (blocks > cap) blocks = cap;
+        bwd_prep_kernel<<<(unsigned)blocks, kPrepThreads, 0, s>>>(dout, y, meta.token_offset,
+                                                                  meta.s_reverse_scatter_idx, meta.scores, N, H,
+                                                                  dy, ds, hdr);
+        const cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
+    if (NK > 0) {
+        int64_t blocks = (NK + 255) / 256;
+        const int64_t cap = (int64_t)num_sms * 8;
+        if (blocks > cap) blocks = cap;
+        scatter_slots_kernel<<<(unsigned)blocks, 256, 0, s>>>(slot_pair, ds, NK, dweights, hdr);
+    }
     return cudaGetLastError();
 }
 

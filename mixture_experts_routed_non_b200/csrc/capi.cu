@@ -101,6 +101,10 @@ moe_ws_layout_t compute_layout_nk(int64_t N, int32_t H, int32_t I, int32_t E, in
         o = align_up(o + (size_t)pc * 2 * I * 2, 1024);
         l.dy = o;
         o = align_up(o + (size_t)pc * H * 2, 1024);
+        l.slot_pair = o;
+        o = align_up(o + (size_t)NK * 4, kAlign);
+        l.ds = o;
+        o = align_up(o + (size_t)pc * 4, kAlign);
     }
     l.train_total = o;
     return l;
@@ -316,6 +320,7 @@ MetaArgs meta_args(const Routing &r, int32_t E, const moe_ws_layout_t &l, uint8_
     a.gemm_tile_off = reinterpret_cast<int32_t *>(ws + l.gemm_tile_offset);
     a.meta = meta;
     a.N = r.N;
+    a.slot_pair = nullptr;
     return a;
 }
 
@@ -366,7 +371,8 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
 
     uint8_t *w = static_cast<uint8_t *>(ws);
     const moe_meta_t meta = meta_out ? *meta_out : ws_meta(l, w);
-    const MetaArgs ma = meta_args(r, E, l, w, meta);
+    MetaArgs ma = meta_args(r, E, l, w, meta);
+    if (train) ma.slot_pair = reinterpret_cast<int32_t *>(w + l.slot_pair);  // for the backward's score gradients
     WsHeader *hdr = ma.hdr;
 
     if ((st = record(ev, 0, s))) return st;
@@ -441,21 +447,21 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
     return MOE_OK;
 }
 
-int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, const float *topk_w, int64_t N,
-                  int32_t H, int32_t I, int32_t E, int32_t K, int64_t total_pairs, const void *w1, const void *w2,
-                  int32_t activation, int32_t layout_kind, void *dx, void *dw1, void *db1, void *dw2, void *db2,
-                  float *dtopk_w, void *ws, size_t ws_bytes, cudaStream_t s, const moe_event_t *ev) {
-    int st = check_sizes(N, E, K, total_pairs);
-    if (st) return st;
-    if ((N > 0 && (!dout || !x || !topk_idx || !topk_w || !dx || !dtopk_w)) || !w1 || !w2 || !dw1 || !dw2)
+int backward_impl(const void *dout, const void *x, const Routing &r, int32_t H, int32_t I, int32_t E,
+                  const void *w1, const void *w2, int32_t activation, int32_t layout_kind, void *dx, void *dw1,
+                  void *db1, void *dw2, void *db2, float *dweights, void *ws, size_t ws_bytes, cudaStream_t s,
+                  const moe_event_t *ev) {
+    const int64_t N = r.N;
+    int st = MOE_OK;
+    if ((N > 0 && (!dout || !x || !dx)) || (r.NK > 0 && !dweights) || !w1 || !w2 || !dw1 || !dw2)
         return MOE_ERR_ARG;
     if (activation != MOE_ACT_SWIGLU) return MOE_ERR_ARG;
     if (layout_kind != MOE_LAYOUT_INTERLEAVED && layout_kind != MOE_LAYOUT_CONCATENATED) return MOE_ERR_ARG;
     if (!aligned(dout, 16) || !aligned(x, 16) || !aligned(w1, 16) || !aligned(w2, 16) || !aligned(dx, 16) ||
         !aligned(dw1, 16) || !aligned(dw2, 16) || (db1 && !aligned(db1, 16)) || (db2 && !aligned(db2, 16)) ||
-        !aligned(topk_idx, 4) || !aligned(topk_w, 4) || !aligned(dtopk_w, 4))
+        !aligned(dweights, 4))
         return MOE_ERR_ARG;
-    const moe_ws_layout_t l = compute_layout(N, H, I, E, K, total_pairs);
+    const moe_ws_layout_t l = compute_layout_nk(N, H, I, E, r.NK, r.p_cap);
     st = check_dense(l.p_cap, H, I, E);
     if (st) return st;
     if (!ws || !aligned(ws, kAlign) || ws_bytes < l.train_total) return MOE_ERR_WS;
@@ -474,8 +480,9 @@ int backward_impl(const void *dout, const void *x, const int32_t *topk_idx, cons
 
     if ((st = record(ev, 0, s))) return st;
     // score gradients (to the [N,K] slots) and dy = s dout per pair
-    if (launch_bwd_prep(static_cast<const __nv_bfloat16 *>(dout), ybuf, topk_idx, meta, N, H, K, E, dybuf, dtopk_w,
-                        hdr, dev.sms, s) != cudaSuccess)
+    if (launch_bwd_prep(static_cast<const __nv_bfloat16 *>(dout), ybuf, meta, N, H, dybuf,
+                        reinterpret_cast<float *>(w + l.ds), reinterpret_cast<const int32_t *>(w + l.slot_pair),
+                        r.NK, dweights, hdr, dev.sms, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     if ((st = record(ev, 1, s))) return st;
 
@@ -616,9 +623,12 @@ extern "C" MOE_API int moe_nonexpand_backward(const void *dout, const void *x, c
                                               int32_t activation, int32_t gate_up_layout, void *dx, void *dw1,
                                               void *db1, void *dw2, void *db2, float *dtopk_w, void *ws,
                                               size_t ws_bytes, moe_stream_t stream) {
-    return backward_impl(dout, x, topk_idx, topk_w, N, H, I, E, K, total_pairs, w1, w2, activation, gate_up_layout,
-                         dx, dw1, db1, dw2, db2, dtopk_w, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
-                         nullptr);
+    int st = check_sizes(N, E, K, total_pairs);
+    if (st) return st;
+    if ((N > 0 && (!topk_idx || !topk_w)) || !aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_ARG;
+    return backward_impl(dout, x, routing_topk32(topk_idx, topk_w, N, K, total_pairs), H, I, E, w1, w2, activation,
+                         gate_up_layout, dx, dw1, db1, dw2, db2, dtopk_w, ws, ws_bytes,
+                         reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 extern "C" MOE_API int moe_nonexpand_backward_timed(const void *dout, const void *x, const int32_t *topk_idx,
@@ -629,9 +639,47 @@ extern "C" MOE_API int moe_nonexpand_backward_timed(const void *dout, const void
                                                     float *dtopk_w, void *ws, size_t ws_bytes, moe_stream_t stream,
                                                     const moe_event_t *stage_events) {
     if (!stage_events) return MOE_ERR_ARG;
-    return backward_impl(dout, x, topk_idx, topk_w, N, H, I, E, K, total_pairs, w1, w2, activation, gate_up_layout,
-                         dx, dw1, db1, dw2, db2, dtopk_w, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream),
-                         stage_events);
+    int st = check_sizes(N, E, K, total_pairs);
+    if (st) return st;
+    if ((N > 0 && (!topk_idx || !topk_w)) || !aligned(topk_idx, 4) || !aligned(topk_w, 4)) return MOE_ERR_ARG;
+    return backward_impl(dout, x, routing_topk32(topk_idx, topk_w, N, K, total_pairs), H, I, E, w1, w2, activation,
+                         gate_up_layout, dx, dw1, db1, dw2, db2, dtopk_w, ws, ws_bytes,
+                         reinterpret_cast<cudaStream_t>(stream), stage_events);
+}
+
+extern "C" MOE_API size_t moe_nonexpand_routed_train_workspace_bytes(const moe_routing_t *routing, int32_t H,
+                                                                     int32_t I, int32_t E) {
+    Routing r;
+    if (routing_from_desc(routing, E, &r)) return 0;
+    if (H <= 0 || I <= 0) return 0;
+    const moe_ws_layout_t l = compute_layout_nk(r.N, H, I, E, r.NK, r.p_cap);
+    if (check_dense(l.p_cap, H, I, E)) return 0;
+    return l.train_total;
+}
+
+extern "C" MOE_API int moe_nonexpand_routed_forward_train(const void *x, const moe_routing_t *routing, int32_t H,
+                                                          int32_t I, int32_t E, const void *w1, const void *b1,
+                                                          const void *w2, const void *b2, int32_t activation,
+                                                          int32_t gate_up_layout, void *out, void *ws,
+                                                          size_t ws_bytes, moe_stream_t stream) {
+    Routing r;
+    const int st = routing_from_desc(routing, E, &r);
+    if (st) return st;
+    return forward_impl(x, r, H, I, E, w1, b1, w2, b2, activation, gate_up_layout, out, nullptr, ws, ws_bytes,
+                        reinterpret_cast<cudaStream_t>(stream), nullptr, true);
+}
+
+extern "C" MOE_API int moe_nonexpand_routed_backward(const void *dout, const void *x, const moe_routing_t *routing,
+                                                     int32_t H, int32_t I, int32_t E, const void *w1,
+                                                     const void *w2, int32_t activation, int32_t gate_up_layout,
+                                                     void *dx, void *dw1, void *db1, void *dw2, void *db2,
+                                                     float *dweights, void *ws, size_t ws_bytes,
+                                                     moe_stream_t stream) {
+    Routing r;
+    const int st = routing_from_desc(routing, E, &r);
+    if (st) return st;
+    return backward_impl(dout, x, r, H, I, E, w1, w2, activation, gate_up_layout, dx, dw1, db1, dw2, db2, dweights,
+                         ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream), nullptr);
 }
 
 extern "C" MOE_API size_t moe_nonexpand_workspace_bytes(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,

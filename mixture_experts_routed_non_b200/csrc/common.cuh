@@ -72,6 +72,7 @@ struct MetaArgs {
     int32_t *gemm_tile_off;  // [E+1] prefix of ceil(freq / kTileRows)
     moe_meta_t meta;
     int64_t N;
+    int32_t *slot_pair;   // training: [NK] pair index q of each slot, -1 where the slot is no pair (or null)
 };
 
 struct GemmArgs {
@@ -142,9 +143,9 @@ cudaError_t launch_router(const void *logits, bool bf16, int64_t N, int E, int K
                           int num_sms, cudaStream_t s);
 size_t gemm_smem_bytes();
 cudaError_t launch_gemm_bwd(int mode, const BwdGemmArgs &a, int max_ctas, cudaStream_t s);
-cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const __nv_bfloat16 *y, const int32_t *topk_idx,
-                            const moe_meta_t &meta, int64_t N, int32_t H, int32_t K, int32_t E, __nv_bfloat16 *dy,
-                            float *dtopk_w, const WsHeader *hdr, int num_sms, cudaStream_t s);
+cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const __nv_bfloat16 *y, const moe_meta_t &meta, int64_t N,
+                            int32_t H, __nv_bfloat16 *dy, float *ds, const int32_t *slot_pair, int64_t NK,
+                            float *dweights, const WsHeader *hdr, int num_sms, cudaStream_t s);
 cudaError_t launch_gather_rows(const __nv_bfloat16 *src, const int32_t *idx, const int32_t *p_total, int32_t cols,
                                __nv_bfloat16 *dst, const WsHeader *hdr, int num_sms, cudaStream_t s);
 cudaError_t launch_bias_grad(const __nv_bfloat16 *src, int32_t cols, const int32_t *expert_off, int32_t E,

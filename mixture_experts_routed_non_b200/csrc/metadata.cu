@@ -395,6 +395,7 @@ __global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a)
                 a.meta.scores[q] = wv[v];
             }
             if (s < w1) {
+                if (a.slot_pair) a.slot_pair[s] = valid ? q : -1;  // training: slot -> pair
                 if (!kPairs) {
                     if ((s % K) == 0) a.meta.token_offset[s / K] = q;
                 } else {

@@ -123,5 +123,6 @@ extern "C" MOE_API int moe_nonexpand_metadata_noalloc(const int32_t *topk_idx, c
     a.gemm_tile_off = reinterpret_cast<int32_t *>(s + l.gemm_tiles);
     a.meta = *meta;
     a.N = N;
+    a.slot_pair = nullptr;
     return launch_meta(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

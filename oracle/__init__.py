@@ -324,18 +324,45 @@ def backward(wd: WeightsF64, topk_idx: np.ndarray, topk_w: np.ndarray, dout, lay
     idx = np.asarray(topk_idx)
     w = np.asarray(topk_w)
     N, K = idx.shape
-    H, I, E = wd.H, wd.I, wd.E
+    E = wd.E
     valid = (idx >= 0) & (idx < E)
     if experts_only is not None:
         valid &= np.isin(idx, np.asarray(experts_only))
     tok, slot = np.nonzero(valid)
     exp = idx[tok, slot].astype(np.int32)
     sc = w[tok, slot].astype(np.float64)
+    g = _sum_pair_terms(wd, dout, tok, exp, sc, N, layout, lib_path)
+    g["dtopk_w"] = np.zeros((N, K))
+    g["dtopk_w"][tok, slot] = g["pairs"]["ds"]
+    g["pairs"]["slot"] = slot
+    return g
+
+
+def backward_pairs(wd: WeightsF64, token_idx, expert_idx, weights, dout, layout: int = LAYOUT_INTERLEAVED,
+                   lib_path: str | None = None) -> dict:
+    """Gradients for a compact pair list (entries kept as in metadata_pairs:
+    expert in [0,E) and token in [0,N)); dweights [P_list] holds each entry's
+    score gradient, 0 for dropped entries."""
+    ti = np.asarray(token_idx, dtype=np.int64).reshape(-1)
+    ei = np.asarray(expert_idx, dtype=np.int64).reshape(-1)
+    w = np.asarray(weights, dtype=np.float64).reshape(-1)
+    N, E = wd.N, wd.E
+    keep = (ei >= 0) & (ei < E) & (ti >= 0) & (ti < N)
+    entry = np.nonzero(keep)[0]
+    g = _sum_pair_terms(wd, dout, ti[entry], ei[entry].astype(np.int32), w[entry], N, layout, lib_path)
+    g["dweights"] = np.zeros(ti.shape[0])
+    g["dweights"][entry] = g["pairs"]["ds"]
+    g["pairs"]["entry"] = entry
+    return g
+
+
+def _sum_pair_terms(wd, dout, tok, exp, sc, N, layout, lib_path):
+    """Per-pair terms (pairs_backward) summed into dx, dW1, db1, dW2, db2."""
+    H, I, E = wd.H, wd.I, wd.E
     r = pairs_backward(wd, dout, tok, exp, sc, layout, lib_path=lib_path)
     g = dict(dx=np.zeros((N, H)), dw1=np.zeros((E, H, 2 * I)), db1=np.zeros((E, 2 * I)),
-             dw2=np.zeros((E, I, H)), db2=np.zeros((E, H)), dtopk_w=np.zeros((N, K)))
-    g["dtopk_w"][tok, slot] = r["ds"]
-    g["pairs"] = dict(tok=tok, slot=slot, exp=exp, **r)  # the per-pair terms, for the tests' error scales
+             dw2=np.zeros((E, I, H)), db2=np.zeros((E, H)))
+    g["pairs"] = dict(tok=tok, exp=exp, **r)  # the per-pair terms, for the tests' error scales
     for e in np.unique(exp):
         sel = exp == e
         te = tok[sel]

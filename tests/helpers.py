@@ -64,8 +64,9 @@ def backward_rss(g, wd, dout):
     """Root sum of squares of the terms of every gradient entry, from the
     oracle's per-pair values (oracle.backward(...)["pairs"])."""
     pr = g["pairs"]
-    tok, slot, exp = pr["tok"], pr["slot"], pr["exp"]
-    rss = {k: np.zeros_like(g[k]) for k in ("dx", "dw1", "db1", "dw2", "db2", "dtopk_w")}
+    tok, exp = pr["tok"], pr["exp"]
+    score = "dtopk_w" if "dtopk_w" in g else "dweights"
+    rss = {k: np.zeros_like(g[k]) for k in ("dx", "dw1", "db1", "dw2", "db2", score)}
     x2 = wd.x ** 2
     for e in np.unique(exp):
         sel = exp == e
@@ -76,7 +77,8 @@ def backward_rss(g, wd, dout):
         rss["db1"][e] = dz2.sum(0)
         np.add.at(rss["dx"], tok[sel], dz2 @ (wd.w1e(e) ** 2).T)
     d = dout.detach().double().cpu().numpy() if hasattr(dout, "detach") else np.asarray(dout, np.float64)
-    rss["dtopk_w"][tok, slot] = (pr["y"] ** 2 * d[tok] ** 2).sum(1)
+    where = (tok, pr["slot"]) if score == "dtopk_w" else pr["entry"]
+    rss[score][where] = (pr["y"] ** 2 * d[tok] ** 2).sum(1)
     return {k: np.sqrt(v) for k, v in rss.items()}
 
 

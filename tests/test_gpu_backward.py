@@ -116,3 +116,59 @@ def test_prefill_backward_sampled():
                      "dx (prefill, sampled tokens)")
     assert_close_bwd(to_np(grads["dtopk_w"])[tokens], ref_t["dtopk_w"][tokens], rss_t["dtopk_w"][tokens],
                      "dtopk_w (prefill, sampled tokens)")
+
+
+@pytest.mark.parametrize("bits", [32, 64])
+def test_pair_list_backward_equals_table_backward_bitwise(bits):
+    """The pair list of a table (invalid slots dropped) is the same routing in
+    the same pair order: every gradient is bit-identical, and each entry's
+    score gradient is its slot's."""
+    dt = {32: torch.int32, 64: torch.int64}[bits]
+    inp = synthetic.make_inputs("tiny", device="cuda", invalid_value=float("nan"))
+    wl = inp.wl
+    dout = _dout(wl, 21)
+    _, ga, _, _ = _run(inp, 0, dout)
+    tok, exp, wt = synthetic.pair_list_from_table(inp.topk_idx.cpu().numpy(), inp.topk_w.cpu().numpy())
+    ti, ei, wi = (torch.from_numpy(v).cuda() for v in (tok, exp, wt))
+    ti, ei = ti.to(dt), ei.to(dt)
+    r = binding.routing(ei, wi, token_idx=ti, N=wl.N)
+    ws = torch.empty(binding.routed_train_workspace_bytes(r, wl.H, wl.I, wl.E), dtype=torch.uint8, device="cuda")
+    binding.routed_forward_train(inp.x, ei, wi, inp.w1, inp.w2, inp.b1, inp.b2, ws=ws, token_idx=ti)
+    gb = binding.routed_backward(dout, inp.x, ei, wi, inp.w1, inp.w2, ws=ws, token_idx=ti, bias_grads=True)
+    torch.cuda.synchronize()
+    assert binding.read_error(ws) == 0
+    for k in ("dx", "dw1", "dw2", "db1", "db2"):
+        assert torch.equal(ga[k].view(torch.int16), gb[k].view(torch.int16)), k
+    valid = inp.topk_idx >= 0
+    assert torch.equal(gb["dweights"].view(torch.int32), ga["dtopk_w"][valid].view(torch.int32))
+
+
+@pytest.mark.parametrize("bits", [32, 64])
+def test_pair_list_backward_heavy_tokens_and_dropped_entries(bits):
+    """Tokens routed to all 300 experts (more pairs than one batch of the
+    score-gradient kernel), tokens without pairs, dropped entries."""
+    dt = {32: torch.int32, 64: torch.int64}[bits]
+    wl = synthetic.custom(N=300, H=256, I=192, E=300, K=4, bias=True, seed=12, name="heavy")
+    inp = synthetic.make_inputs(wl, device="cuda")
+    rng = np.random.default_rng(4)
+    heavy = np.array([0, 7, 150, 299])
+    tok, exp, wt = synthetic.many_pair_tokens(wl.N, wl.E, heavy, wl.K, rng)
+    keep = ~np.isin(tok, [30, 31, 200])
+    tok, exp, wt = tok[keep], exp[keep].copy(), wt[keep]
+    exp[3] = -1
+    exp[100] = wl.E + 5
+    ti, ei, wi = (torch.from_numpy(np.ascontiguousarray(v)).cuda() for v in (tok, exp, wt))
+    ti, ei = ti.to(dt), ei.to(dt)
+    r = binding.routing(ei, wi, token_idx=ti, N=wl.N)
+    ws = torch.empty(binding.routed_train_workspace_bytes(r, wl.H, wl.I, wl.E), dtype=torch.uint8, device="cuda")
+    binding.routed_forward_train(inp.x, ei, wi, inp.w1, inp.w2, inp.b1, inp.b2, ws=ws, token_idx=ti)
+    dout = _dout(wl, 22)
+    g = binding.routed_backward(dout, inp.x, ei, wi, inp.w1, inp.w2, ws=ws, token_idx=ti, bias_grads=True)
+    torch.cuda.synchronize()
+    assert binding.read_error(ws) == binding.DEVERR_BAD_EXPERT_ID
+    wd = oracle.WeightsF64(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    ref = oracle.backward_pairs(wd, tok, exp, wt, dout)
+    rss = backward_rss(ref, wd, dout)
+    for k in ("dx", "dw1", "dw2", "db1", "db2", "dweights"):
+        assert_close_bwd(to_np(g[k]), ref[k], rss[k], f"{k} (pair list, heavy tokens)")
+    assert g["dweights"][3].item() == 0.0 and g["dweights"][100].item() == 0.0

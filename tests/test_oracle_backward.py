@@ -155,3 +155,39 @@ def test_backward_experts_only_is_complete_for_those_experts():
     part = oracle.backward(wd, idx, w, dout, experts_only=[3, 5])
     for k in ("dw1", "db1", "dw2", "db2"):
         np.testing.assert_array_equal(part[k][[3, 5]], full[k][[3, 5]])
+
+
+def test_backward_pairs_equals_table_backward_on_its_flattening():
+    """A pair list holding a table's valid slots in row-major order is the same
+    routing: every gradient matches, and each entry's score gradient is its
+    slot's."""
+    inp = synthetic.make_inputs("tiny", device="cpu", invalid_value=float("nan"))
+    dout = np.random.default_rng(8).standard_normal((inp.wl.N, inp.wl.H))
+    wd = oracle.WeightsF64(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    idx, w = inp.topk_idx.numpy(), inp.topk_w.numpy()
+    tok, exp, wt = synthetic.pair_list_from_table(idx, w)
+    for layout in (0, 1):
+        a = oracle.backward(wd, idx, w, dout, layout)
+        b = oracle.backward_pairs(wd, tok, exp, wt, dout, layout)
+        for k in ("dx", "dw1", "db1", "dw2", "db2"):
+            np.testing.assert_allclose(b[k], a[k], rtol=1e-13, atol=1e-13, err_msg=k)
+        np.testing.assert_allclose(b["dweights"], a["dtopk_w"][idx >= 0], rtol=1e-13, atol=1e-13)
+
+
+def test_backward_pairs_dropped_entries_have_zero_gradient():
+    inp = synthetic.make_inputs("tiny", device="cpu")
+    dout = np.random.default_rng(9).standard_normal((inp.wl.N, inp.wl.H))
+    wd = oracle.WeightsF64(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    tok, exp, wt = synthetic.pair_list_from_table(inp.topk_idx.numpy(), inp.topk_w.numpy())
+    tok, exp = tok.copy(), exp.copy()
+    exp[5] = -1
+    exp[9] = inp.wl.E + 2
+    tok[-2:] = inp.wl.N
+    g = oracle.backward_pairs(wd, tok, exp, wt, dout)
+    assert g["dweights"][[5, 9, len(tok) - 2, len(tok) - 1]].tolist() == [0.0] * 4
+    keep = np.ones(len(tok), bool)
+    keep[[5, 9, len(tok) - 2, len(tok) - 1]] = False
+    h = oracle.backward_pairs(wd, tok[keep], exp[keep], wt[keep], dout)
+    for k in ("dx", "dw1", "dw2"):
+        np.testing.assert_array_equal(g[k], h[k])
+    np.testing.assert_array_equal(g["dweights"][keep], h["dweights"])
