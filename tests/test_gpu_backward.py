@@ -172,3 +172,32 @@ def test_pair_list_backward_heavy_tokens_and_dropped_entries(bits):
     for k in ("dx", "dw1", "dw2", "db1", "db2", "dweights"):
         assert_close_bwd(to_np(g[k]), ref[k], rss[k], f"{k} (pair list, heavy tokens)")
     assert g["dweights"][3].item() == 0.0 and g["dweights"][100].item() == 0.0
+
+
+def test_backward_with_no_pairs_gives_zero_gradients():
+    """Every slot invalid (P = 0): the weight gradients are written as zeros,
+    dx and the score gradients are zero."""
+    wl = synthetic.custom(50, 128, 128, 6, 2, bias=True, seed=13)
+    inp = synthetic.make_inputs(wl, device="cuda")
+    inp.topk_idx.fill_(-1)
+    dout = _dout(wl, 31)
+    _, g, _, _ = _run(inp, 0, dout)
+    for k, v in g.items():
+        assert torch.count_nonzero(v) == 0, k
+
+
+def test_backward_int64_table_equals_int32_table_bitwise():
+    inp = synthetic.make_inputs("tiny", device="cuda", invalid_value=float("nan"))
+    wl = inp.wl
+    dout = _dout(wl, 41)
+    _, ga, _, _ = _run(inp, 1, dout)
+    idx64 = inp.topk_idx.to(torch.int64)
+    w1c, b1c = _concat_from_interleaved(inp.w1, inp.b1)
+    r = binding.routing(idx64, inp.topk_w)
+    ws = torch.empty(binding.routed_train_workspace_bytes(r, wl.H, wl.I, wl.E), dtype=torch.uint8, device="cuda")
+    binding.routed_forward_train(inp.x, idx64, inp.topk_w, w1c, inp.w2, b1c, inp.b2, ws=ws, layout=1)
+    gb = binding.routed_backward(dout, inp.x, idx64, inp.topk_w, w1c, inp.w2, ws=ws, layout=1, bias_grads=True)
+    torch.cuda.synchronize()
+    for k in ("dx", "dw1", "dw2", "db1", "db2"):
+        assert torch.equal(ga[k].view(torch.int16), gb[k].view(torch.int16)), k
+    assert torch.equal(ga["dtopk_w"].view(torch.int32), gb["dweights"].view(torch.int32))
