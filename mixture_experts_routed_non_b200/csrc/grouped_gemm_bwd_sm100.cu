@@ -480,11 +480,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                                 tma_load_3d_pair(b_stage(stage), &a.tmap_b, fb, 0,
                                                  t.e * a.b_rows_per_expert + t.n0 + col0b, kb);
                         }
-                        issued |= 1u << stage;
-                        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                     } else if (rank == 0) {
                         mbar_arrive(full_bar(stage));
                     }
+                    // the last use of each stage, whatever filled it: its full phase
+                    // completes only after every earlier phase (and its bytes)
+                    issued |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                     if (++stage == kBwdStages) {
                         stage = 0;
                         phase ^= 1u;

@@ -65,6 +65,11 @@ constexpr uint32_t kStageBytes = kStageA + kStageB;
 constexpr uint32_t kTmemCols = 2 * kBN;         // two accumulators
 constexpr uint32_t kNumBars = 3 * kPairStages + 5;
 constexpr uint32_t kIdesc = idesc_bf16_f32(kPairM, kBN, /*b_mn_major=*/true);
+// A segment's last tile with at most 128 rows runs the pair MMA at M=128: each
+// CTA holds 64 rows of A, and its TMEM accumulator holds those 64 rows with
+// columns [0,128) in lanes 0-63 and columns [128,256) in lanes 64-127.
+constexpr uint32_t kIdescTail = idesc_bf16_f32(kBM, kBN, /*b_mn_major=*/true);
+constexpr int kTailRows = kBM / 2;  // rows per CTA of a tail tile
 constexpr unsigned long long kAbortSettleNs = 2000000ull;
 
 constexpr uint32_t kStoreBuf = 32 * 128;        // 4 KB per epilogue warp: 32 rows x 64 bf16
@@ -197,7 +202,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
     const int last_mmas = (a.k_dim % kStageK) ? (a.k_dim % kStageK) / kUmmaK : kStageK / kUmmaK;
     const int cluster = blockIdx.x >> 1;
     const int n_clusters = gridDim.x >> 1;
-    const int row0 = (int)rank * kBM;  // this CTA's first row inside a tile
+    const int row0 = (int)rank * kBM;  // this CTA's first row inside a full tile
+    // a tail tile (at most 128 rows; the concatenated up GEMM keeps full tiles, its
+    // gate and up halves sit in different CTAs) and this CTA's first row and rows in it
+    auto is_tail = [&](const Tile &tt) {
+        return tt.m_end - tt.m0 <= kBM && (!kUp || a.layout != MOE_LAYOUT_CONCATENATED);
+    };
+    auto rbase = [&](const Tile &tt) { return is_tail(tt) ? (int)rank * kTailRows : row0; };
+    auto rspan = [&](const Tile &tt) { return is_tail(tt) ? kTailRows : kBM; };
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -205,9 +217,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
         // segment, only its 16-row groups (rows past the segment end are never
         // stored, so they need no data)
         auto a_groups = [&](const Tile &tt, int r) {
-            const int v = min(max(tt.m_end - (tt.m0 + r * kBM), 0), kBM);
+            const bool tl = is_tail(tt);
+            const int span = tl ? kTailRows : kBM;
+            const int v = min(max(tt.m_end - (tt.m0 + r * span), 0), span);
             const int g = (v + 15) / 16;
-            return g >= 6 ? 8 : g;  // 8 = one full box
+            return (!tl && g >= 6) ? 8 : g;  // 8 = one full box
         };
         auto a_bytes = [&](int groups) { return (uint32_t)groups * 16 * 128 * kAtoms; };
         int stage = 0;
@@ -241,7 +255,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
 #pragma unroll
                                 for (int at = 0; at < kAtoms; ++at)
                                     tma_load_3d_pair(a_dst + at * kAtomA + g * 16 * 128, &a.tmap_a16, fb, 0,
-                                                     t.m0 + row0 + 16 * g, k0 / 64 + at);
+                                                     t.m0 + rbase(t) + 16 * g, k0 / 64 + at);
                         }
                     }
                     if (kUp && a.layout == MOE_LAYOUT_CONCATENATED)
@@ -272,7 +286,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                 uint32_t phase = 0;
                 int tcount = 0;
                 bool ok = true;
+                int e_cur = 0;  // tiles come in increasing order: the expert only moves forward
                 for (int tile = cluster; ok && tile < total_tiles; tile += n_clusters, ++tcount) {
+                    const int mt = tile / n_tiles;
+                    while (tile_off_s[e_cur + 1] <= mt) ++e_cur;
+                    Tile tt;
+                    tt.m0 = off_s[e_cur] + (mt - tile_off_s[e_cur]) * kPairM;
+                    tt.m_end = off_s[e_cur + 1];
+                    const bool tail = is_tail(tt);
                     const int acc = tcount & 1;
                     const uint32_t acc_phase = (tcount >> 1) & 1;
                     if (!mbar_wait_bounded(tempty_bar(acc), acc_phase ^ 1u, abort)) break;
@@ -298,7 +319,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                             // 1024 B apart (SBO); K step = 16 rows = 2 KB.
                             const uint64_t bdesc =
                                 smem_desc_sw128(b_addr + kk * (kUmmaK * 128), kChunkB, 1024);
-                            umma_f16_pair(d_tmem, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+                            umma_f16_pair(d_tmem, adesc, bdesc, tail ? kIdescTail : kIdesc, (kb | kk) != 0 ? 1u : 0u);
                         }
                         umma_commit_pair_mc(empty_bar(stage), 0x3);
                         if (++stage == kPairStages) {
@@ -337,7 +358,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
     } else if (warp < 6) {
         // ------------------------------------------------------------ epilogue
         const int quarter = warp & 3;
-        const int row = row0 + quarter * 32 + lane;
         const uint32_t store_buf = base + (uint32_t)kSmemStoreOff + (uint32_t)(warp - 2) * kStoreBuf;
         int tcount = 0;
         for (int tile = cluster; tile < total_tiles; tile += n_clusters, ++tcount) {
@@ -349,12 +369,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
             w = __shfl_sync(0xffffffffu, w, 0);
             if (!w) break;
             tc_fence_after();
-            const int p = t.m0 + row;
+            // full tile: this warp's 32 rows (TMEM lanes) hold all 256 accumulator
+            // columns.  Tail tile: the CTA holds 64 rows; lanes 0-63 hold columns
+            // [0,128) of them and lanes 64-127 columns [128,256), at TMEM columns [0,128)
+            const bool tail = is_tail(t);
+            const int chalf = tail ? (quarter >> 1) : 0;  // which 128 logical columns (tail)
+            const int wrow0 = t.m0 + (tail ? rbase(t) + (quarter & 1) * 32 : row0 + quarter * 32);
+            const int p = wrow0 + lane;
             const bool valid = p < t.m_end;
             // whole warp inside the segment: stage in shared memory, one TMA store
             // per 32 x 64 block; otherwise masked per-row stores
-            const bool warp_full = t.m0 + row0 + quarter * 32 + 31 < t.m_end;
-            const int wrow0 = t.m0 + row0 + quarter * 32;
+            const bool warp_full = wrow0 + 31 < t.m_end;
             const uint32_t tbase = tmem_base + acc * kBN + ((uint32_t)(quarter * 32) << 16);
             __nv_bfloat16 *orow = a.out + (size_t)(valid ? p : 0) * a.out_cols;
             const __nv_bfloat16 *brow = a.bias ? a.bias + (size_t)t.e * a.n_dim : nullptr;
@@ -420,8 +445,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
             } else if (kUp) {
                 // interleaved: accumulator columns (2j, 2j+1) = (gate_j, up_j)
 #pragma unroll 1
-                for (int gi = 0; gi < 2; ++gi) {
-                    const int col0 = t.nt * (kBN / 2) + gi * 64;  // output column
+                for (int gi = 0; gi < (tail ? 1 : 2); ++gi) {
+                    const int col0 = t.nt * (kBN / 2) + (tail ? chalf : gi) * 64;  // output column
                     if (col0 >= a.out_cols) break;
                     uint32_t packed[32];
 #pragma unroll
@@ -431,7 +456,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                         tmem_ld_32x32b_x32(tbase + c * 32, r0);
                         tmem_ld_32x32b_x32(tbase + (c + 1) * 32, r1);
                         tmem_ld_wait();
-                        const int acol = t.nt * kBN + c * 32;
+                        const int acol = t.nt * kBN + chalf * (kBN / 2) + c * 32;  // logical column
                         if (brow) {
                             add_bias32(r0, brow + acol);
                             add_bias32(r1, brow + acol + 32);
@@ -455,8 +480,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                 }
             } else {
 #pragma unroll 1
-                for (int gi = 0; gi < 4; ++gi) {
-                    const int col0 = t.nt * kBN + gi * 64;
+                for (int gi = 0; gi < (tail ? 2 : 4); ++gi) {
+                    const int col0 = t.nt * kBN + chalf * (kBN / 2) + gi * 64;
                     if (col0 >= a.n_dim) break;
                     uint32_t r0[32], r1[32];
                     tmem_ld_32x32b_x32(tbase + gi * 64, r0);
@@ -502,7 +527,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
         auto load_rows = [&](const Tile &tt, const char *(&pp)[8]) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const int pr = min(tt.m0 + row0 + r0 + 16 * i, tt.m_end - 1);
+                const int pr = min(tt.m0 + rbase(tt) + r0 + 16 * i, tt.m_end - 1);
                 pp[i] = xb + (size_t)__ldg(a.x_gather_idx + pr) * ld + chunk * 16;
             }
         };
@@ -530,6 +555,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                     break;
                 }
                 const uint32_t a_dst = sA + stage * kStageA;
+                const int rb = rbase(t), rs = rspan(t);  // a tail tile: 64 rows per CTA
 #pragma unroll
                 for (int at = 0; at < kAtoms; ++at) {
                     const int k0 = kb * kStageK + at * 64;
@@ -540,7 +566,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                         const int rr = r0 + 16 * i;
                         // rows past the segment end are never stored: skip their copies
                         // (the stage keeps stale data there, which only feeds those rows)
-                        if (t.m0 + row0 + rr < t.m_end)
+                        if (rr < rs && t.m0 + rb + rr < t.m_end)
                             cp_async_16(a_dst + at * kAtomA + rr * 128 + ((chunk ^ (rr & 7)) << 4),
                                         src[i] + koff);
                     }
