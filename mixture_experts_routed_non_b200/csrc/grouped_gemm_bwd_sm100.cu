@@ -265,7 +265,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                     umma_commit_pair_mc(tfull_bar(acc), 0x3);  // with no MMA (empty segment) at once
                 }
                 umma_commit_pair(drain_bar);  // every MMA issued here completes before TMEM is freed
-                mbar_wait_timed(drain_bar, 0);
+                if (!mbar_wait_timed(drain_bar, 0)) atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);
             }
         } else if (lane == 0) {
             // ------------------------------------------------------- relay (odd CTA)
@@ -497,8 +497,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
             // the even CTA's stage barriers count both CTAs' boxes (the odd CTA is
             // held by the final cluster barrier until this drain ends)
             for (int st = 0; st < kBwdStages; ++st) {
-                if (rank == 0 && (issued & (1u << st))) mbar_wait_timed(full_bar(st), (issued_parity >> st) & 1u);
-                if (tissued & (1u << st)) mbar_wait_timed(tail_bar(st), (tissued_parity >> st) & 1u);
+                bool drained = true;
+                if (rank == 0 && (issued & (1u << st)))
+                    drained &= mbar_wait_timed(full_bar(st), (issued_parity >> st) & 1u);
+                if (tissued & (1u << st)) drained &= mbar_wait_timed(tail_bar(st), (tissued_parity >> st) & 1u);
+                if (!drained) atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);  // a drain that ran out is an error too
             }
         }
         __syncwarp();

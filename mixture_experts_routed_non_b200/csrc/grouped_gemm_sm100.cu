@@ -275,7 +275,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
             // phase this CTA issued before the CTA may exit
             if (rank == 0)
                 for (int s = 0; s < kPairStages; ++s)
-                    if (issued & (1u << s)) mbar_wait_timed(full_bar(s), (issued_parity >> s) & 1u);
+                    if ((issued & (1u << s)) && !mbar_wait_timed(full_bar(s), (issued_parity >> s) & 1u))
+                        atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);  // a drain that ran out is an error too
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -332,7 +333,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                 }
                 // all pair MMAs issued here complete before TMEM is freed
                 umma_commit_pair(drain_bar);
-                mbar_wait_timed(drain_bar, 0);
+                if (!mbar_wait_timed(drain_bar, 0)) atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);
             }
         } else if (kUp && lane == 0) {
             // ------------------------------------------- relay (odd CTA, up)

@@ -201,3 +201,28 @@ def test_backward_int64_table_equals_int32_table_bitwise():
     for k in ("dx", "dw1", "dw2", "db1", "db2"):
         assert torch.equal(ga[k].view(torch.int16), gb[k].view(torch.int16)), k
     assert torch.equal(ga["dtopk_w"].view(torch.int32), gb["dweights"].view(torch.int32))
+
+
+def test_prefill256_backward_skewed_routing():
+    """Zipf routing over 256 experts at full size: no wait may run out (the
+    error word stays 0), a mid-sized and a small expert's weight gradients
+    match the oracle, and experts without pairs get zero gradients."""
+    inp = synthetic.make_inputs("prefill256", device="cuda")
+    wl = inp.wl
+    dout = _dout(wl, 51)
+    _, grads, _, _ = _run(inp, 0, dout, bias_grads=False)  # asserts the error word is 0
+    idx, w = inp.topk_idx.cpu().numpy(), inp.topk_w.cpu().numpy()
+    freq = np.bincount(idx[idx >= 0], minlength=wl.E)
+    mid = int(np.argmin(np.abs(freq - 600)))
+    small = int(np.argmin(np.where(freq > 0, np.abs(freq - 40), 1 << 30)))
+    experts = [mid, small]
+    wd = oracle.WeightsF64(inp.x, inp.w1, None, inp.w2, None)
+    ref = oracle.backward(wd, idx, w, dout, 0, experts_only=experts)
+    rss = backward_rss(ref, wd, dout)
+    for k in ("dw1", "dw2"):
+        assert_close_bwd(to_np(grads[k][experts]), ref[k][experts], rss[k][experts],
+                         f"{k} (prefill256, experts {experts} with {freq[experts].tolist()} rows)")
+    empty = np.nonzero(freq == 0)[0]
+    if empty.size:
+        e = torch.from_numpy(empty).cuda()
+        assert torch.count_nonzero(grads["dw1"][e]) == 0 and torch.count_nonzero(grads["dw2"][e]) == 0
