@@ -51,6 +51,19 @@ def dist_env():
     return rank, world, local
 
 
+def max_over_ranks(value: float, device, world: int) -> float:
+    """The largest of every rank's `value` (a device-timed duration); every
+    rank calls it at the same point, so the collective order stays the same on
+    all ranks.  With one rank it returns `value` unchanged."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------------------
 # clocks sampled during the timed region
 # ---------------------------------------------------------------------------
@@ -199,6 +212,8 @@ def parse():
     ap.add_argument("--layout", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=6.0,
+                    help="oracle work per step of --impl reference (sets its token sample)")
     return ap.parse_args()
 
 
@@ -357,12 +372,12 @@ def run_reference(args, rank, world):
     idx = inp.topk_idx.numpy()
     w = inp.topk_w.numpy()
     threads = len(os.sched_getaffinity(0))
-    # sample size per step: about 6 s of oracle work
+    # sample size per step: about --ref-seconds of oracle work
     probe = np.arange(min(wl.N, 4))
     t0 = time.perf_counter()
     oracle.forward_rows(wts, idx, w, tokens=probe, layout=args.layout, n_threads=threads)
     per_tok = (time.perf_counter() - t0) / len(probe)
-    n = int(max(1, min(wl.N, 6.0 / max(per_tok, 1e-6))))
+    n = int(max(1, min(wl.N, args.ref_seconds / max(per_tok, 1e-6))))
     rng = np.random.default_rng(7)
     times = []
     for step in range(args.warmup + args.steps):
@@ -455,11 +470,7 @@ def run_ours(args, rank, world, local):
         for j in range(4):
             stage_ms[j] += e[j].elapsed_time(e[j + 1])
     stage_ms /= args.steps
-    max_ms = elapsed_ms
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        max_ms = float(t.item())
+    max_ms = max_over_ranks(elapsed_ms, dev, world)
     ms_per_step = max_ms / args.steps
     value = N * world * args.steps / (max_ms / 1000.0)
 
@@ -521,11 +532,7 @@ def run_ours(args, rank, world, local):
     s_out.wait_stream(s_cmp)
     e2.record(s_out)
     torch.cuda.synchronize(dev)
-    e2e_ms = s2.elapsed_time(e2)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(s2.elapsed_time(e2), dev, world)
     e2e_value = N * world * e2e_steps / (e2e_ms / 1000.0)
     h2d = nx + ni + nw
     d2h = outs_h[0].numel() * 2
