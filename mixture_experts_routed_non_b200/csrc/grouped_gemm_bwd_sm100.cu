@@ -127,6 +127,11 @@ __device__ __forceinline__ BTile decode_weights(int tile, int m_tiles, int n_til
     return t;
 }
 
+// `count` arrivals on a barrier of this CTA at once
+__device__ __forceinline__ void mbar_arrive_n(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void settle_after_abort() {
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < kAbortSettleNs) {
@@ -213,6 +218,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
         return kMN ? decode_weights(tile, m_tiles, n_tiles, E, off_s)
                    : decode_rows(tile, n_tiles, E, tile_off_s, off_s, a.K_dim);
     };
+    // whether the copy warps (and, for the odd CTA, the relay) take part in
+    // this stage: an operand comes by cp.async, or a DW segment's last stage
+    // has rows past the segment end to zero.  In the other stages the even
+    // CTA's TMA thread makes their arrivals on the stage barrier itself, which
+    // keeps the copy warps and the relay off the stage's critical path.
+    auto stage_copies = [&](const BTile &tt, int kb) {
+        if (!a.a_tma || !a.b_tma) return true;
+        return kMN && tt.kp0 + (kb + 1) * kSK > tt.kp1;
+    };
 
     if (warp == 0) {
         if (rank == 0) {
@@ -271,21 +285,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
             // ------------------------------------------------------- relay (odd CTA)
             // forwards the completion of this CTA's copy threads to the even CTA
             int stage = 0;
-            uint32_t phase = 0;
+            uint32_t gpar = 0;  // parity of each stage's next gfull phase (stages with copies only)
             bool ok = true;
             for (int tile = cluster; ok && tile < total; tile += n_clusters) {
                 const BTile t = decode(tile);
                 for (int kb = 0; kb < t.nk; ++kb) {
-                    if (!mbar_wait_bounded(gfull_bar(stage), phase, abort)) {
-                        ok = false;
-                        break;
+                    if (stage_copies(t, kb)) {
+                        if (!mbar_wait_bounded(gfull_bar(stage), (gpar >> stage) & 1u, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        gpar ^= 1u << stage;
+                        fence_proxy_async_smem();
+                        mbar_arrive_cluster(mapa_shared(full_bar(stage), 0));
                     }
-                    fence_proxy_async_smem();
-                    mbar_arrive_cluster(mapa_shared(full_bar(stage), 0));
-                    if (++stage == kBwdStages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
+                    if (++stage == kBwdStages) stage = 0;
                 }
             }
         }
@@ -467,8 +481,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                         tphase ^= 1u << stage;
                         if (rank == 0) mbar_arrive(full_bar(stage));
                     } else if (bytes) {
-                        // both CTAs' bytes are expected by the even CTA's barrier
-                        if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * bytes);
+                        // both CTAs' bytes are expected by the even CTA's barrier; with
+                        // no copies in this stage its TMA thread also arrives for the
+                        // copy threads and the odd CTA's relay
+                        if (rank == 0) {
+                            mbar_arrive_expect_tx(full_bar(stage), 2 * bytes);
+                            if (!stage_copies(t, kb)) mbar_arrive_n(full_bar(stage), kProducerThreads + 1);
+                        }
                         const uint32_t fb = mapa_shared(full_bar(stage), 0);
                         if (kMN) {
                             if (ta) tma_load_3d_pair(a_stage(stage), &a.tmap_a, fb, 0, kbase, (t.m0 + row0) / 64);
@@ -540,12 +559,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
             };
             if (kMN && t.nk > 0) load_rows(0);
             for (int kb = 0; kb < t.nk; ++kb) {
+                if (!stage_copies(t, kb)) {  // the TMA thread arrived for this stage
+                    if (++stage == kBwdStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    continue;
+                }
                 int crow[kSK / 8];
 #pragma unroll
                 for (int i = 0; i < kSK / 8; ++i) crow[i] = nrow[i];
                 if (kMN && kb + 1 < t.nk) load_rows(kb + 1);
+                // The stage is free once the MMAs of its previous use completed.  That
+                // wait is only meaningful when these warps take part in every use of
+                // every stage: a parity wait cannot tell a phase from the one two
+                // phases earlier.  When they only zero the TMA-loaded last stage of a
+                // DW segment, the tail barrier below orders them instead (its TMA is
+                // issued after the producer's own wait for the free stage).
                 bool w = true;
-                if (gl == 0) w = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort);
+                if (gl == 0 && (!a.a_tma || !a.b_tma)) w = mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort);
                 w = __shfl_sync(0xffffffffu, w, 0);
                 if (!w) {
                     ok = false;
