@@ -526,6 +526,7 @@ int backward_impl(const void *dout, const void *x, const Routing &r, int32_t H, 
             !make_map_a_chunks(&a.tmap_b, dybuf, (uint64_t)H, prow, 64, 2))
             return MOE_ERR_CUDA;
         a.a_tma = a.b_tma = 1;
+        if (!make_map_2d(&a.tmap_out, dw2, (uint64_t)H, (uint64_t)E * I, 64, 32)) return MOE_ERR_CUDA;
         a.out = static_cast<__nv_bfloat16 *>(dw2);
         a.out_ld = H;
         a.M_dim = I;
@@ -548,6 +549,7 @@ int backward_impl(const void *dout, const void *x, const Routing &r, int32_t H, 
             !make_map_a_chunks(&a.tmap_b, dzbuf, (uint64_t)2 * I, prow, 64, 2))
             return MOE_ERR_CUDA;
         a.a_tma = a.b_tma = 1;
+        if (!make_map_2d(&a.tmap_out, dw1, (uint64_t)2 * I, (uint64_t)E * H, 64, 32)) return MOE_ERR_CUDA;
         a.out = static_cast<__nv_bfloat16 *>(dw1);
         a.out_ld = 2 * I;
         a.M_dim = H;
@@ -567,6 +569,7 @@ int backward_impl(const void *dout, const void *x, const Routing &r, int32_t H, 
             !make_map_a_chunks(&a.tmap_b, w1b, (uint64_t)2 * I, (uint64_t)E * H, 128, 1))
             return MOE_ERR_CUDA;
         a.a_tma = a.b_tma = 1;
+        if (!make_map_2d(&a.tmap_out, ybuf, (uint64_t)H, prow, 64, 32)) return MOE_ERR_CUDA;
         a.out = ybuf;
         a.out_ld = H;
         a.N_dim = H;

@@ -63,7 +63,9 @@ constexpr uint32_t kStageBytes = kStageA + kStageB;
 constexpr uint32_t kMnAtom = kSK * 128;      // MN-major: one 64-element column of a stage (8 KB)
 constexpr uint32_t kTmemCols = 2 * kN;
 constexpr uint32_t kNumBars = 4 * kBwdStages + 5;
-constexpr size_t kSmemBarOff = (size_t)kBwdStages * kStageBytes;
+constexpr uint32_t kStoreBuf = 32 * 128;     // DX/DW: 4 KB per epilogue warp, 32 rows x 64 bf16
+constexpr size_t kSmemStoreOff = (size_t)kBwdStages * kStageBytes;
+constexpr size_t kSmemBarOff = kSmemStoreOff + 4 * kStoreBuf;
 constexpr size_t kSmemMiscOff = kSmemBarOff + 8 * kNumBars;
 constexpr size_t kSmemTableOff = kSmemMiscOff + 16;
 constexpr size_t kSmemBytes = 1024 + kSmemTableOff + 2 * (kMaxExperts + 1) * 4;
@@ -401,13 +403,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                     }
                 }
             } else {
-                // DX: row p of dxs; DW: row m of expert e's [M,N] output
-                const int r = t.m0 + row0 + rl;
+                // DX: row p of dxs; DW: row m of expert e's [M,N] output.  A warp whose
+                // 32 rows are all stored stages each 32 x 64 block in shared memory
+                // (128-byte swizzle) and writes it with one TMA store; a DX warp that
+                // straddles a segment end stores its valid rows one by one.
+                const int wrow0 = t.m0 + row0 + quarter * 32;  // this warp's first tile row
+                const int r = wrow0 + lane;
                 const bool valid = kMode == kBwdDX ? r < t.m_end : r < a.M_dim;
+                const bool warp_full = kMode == kBwdDX ? wrow0 + 31 < t.m_end : wrow0 + 31 < a.M_dim;
+                const int out_row0 = kMode == kBwdDX ? wrow0 : t.e * a.M_dim + wrow0;  // row in tmap_out
                 const size_t row_off = kMode == kBwdDX
                                            ? (size_t)(valid ? r : 0) * a.out_ld
                                            : ((size_t)t.e * a.M_dim + (valid ? r : 0)) * a.out_ld;
                 __nv_bfloat16 *orow = a.out + row_off;
+                const uint32_t store_buf = base + (uint32_t)kSmemStoreOff + (uint32_t)(warp - 1) * kStoreBuf;
                 const bool zero = kMode == kBwdDW && t.nk == 0;  // empty segment: the gradient is 0
 #pragma unroll 1
                 for (int g = part * (kN / 64 / R::kParts); g < (part + 1) * (kN / 64 / R::kParts); ++g) {
@@ -419,22 +428,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                         tmem_ld_32x32b_x32(tbase + g * 64 + 32, r1);
                         tmem_ld_wait();
                     }
-                    if (!valid) continue;
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + col0);
+                    uint32_t o[32];  // 64 bf16 of this thread's row
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint32_t o[4], o2[4];
+                    for (int j = 0; j < 16; ++j) {
+                        o[j] = zero ? 0u : pack_bf16x2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1]));
+                        o[16 + j] =
+                            zero ? 0u : pack_bf16x2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1]));
+                    }
+                    if (warp_full) {
+                        if (lane == 0) bulk_wait_read0();  // the buffer's previous store has been read
+                        __syncwarp();
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            o[j] = zero ? 0u
-                                        : pack_bf16x2(__uint_as_float(r0[8 * q + 2 * j]),
-                                                      __uint_as_float(r0[8 * q + 2 * j + 1]));
-                            o2[j] = zero ? 0u
-                                         : pack_bf16x2(__uint_as_float(r1[8 * q + 2 * j]),
-                                                       __uint_as_float(r1[8 * q + 2 * j + 1]));
+                        for (int c = 0; c < 8; ++c)
+                            st_shared_v4(store_buf + lane * 128 + ((c ^ (lane & 7)) << 4), o[4 * c], o[4 * c + 1],
+                                         o[4 * c + 2], o[4 * c + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&a.tmap_out, store_buf, col0, out_row0);
+                            bulk_commit();
                         }
-                        dst[q] = make_uint4(o[0], o[1], o[2], o[3]);
-                        dst[4 + q] = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+                    } else if (valid) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(orow + col0);
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) dst[c] = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
                     }
                 }
             }
@@ -445,6 +462,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                 else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
             }
         }
+        if (kMode != kBwdDH && lane == 0) bulk_wait0();  // this warp's TMA stores have landed
     } else if (warp == R::kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
         // whole-stage boxes of the operands that need no gather: 128-byte-swizzled
