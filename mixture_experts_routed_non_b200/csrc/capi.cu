@@ -250,6 +250,20 @@ bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same for fp32 [outer][inner] (a box of 32 fp32 is one 128-byte row).
+bool make_map_2d_f32(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
+                     uint32_t box_outer) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 4};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // A row-major weight [rows][ncols] (ncols % 64 == 0) viewed as
 // (64 columns, rows, ncols/64 column chunks): one box of 64 x stage-K x 2 lands in
 // shared memory as two 64-column chunks of stage-K rows each -- the
@@ -506,6 +520,9 @@ int backward_impl(const void *dout, const void *x, const Routing &r, int32_t H, 
         a.b_rows_per_expert = I;
         if (!make_map_a_chunks(&a.tmap_b, w2b, (uint64_t)H, (uint64_t)E * I, 128, 1)) return MOE_ERR_CUDA;
         a.b_tma = 1;
+        if (!make_map_2d_f32(&a.tmap_z, zbuf, (uint64_t)2 * I, prow, 32, 32) ||
+            !make_map_2d(&a.tmap_out, dzbuf, (uint64_t)2 * I, prow, 64, 32))
+            return MOE_ERR_CUDA;
         a.z = zbuf;
         a.dz = dzbuf;
         a.row_scale = meta.scores;

@@ -108,7 +108,8 @@ enum BwdMode : int32_t {
 struct BwdGemmArgs {
     CUtensorMap tmap_a;        // (64, rows, cols/64) view of `a` when a_tma
     CUtensorMap tmap_b;        // (64, rows, cols/64) view of `b` when b_tma
-    CUtensorMap tmap_out;      // DX/DW: `out` as [rows][N], box 64 columns x 32 rows (stores)
+    CUtensorMap tmap_out;      // DX/DW: `out` as [rows][N]; DH: dz [P_cap, 2I]; box 64 columns x 32 rows (stores)
+    CUtensorMap tmap_z;        // DH: z [P_cap, 2I] fp32, box 32 columns x 32 rows
     int32_t a_tma, b_tma;      // load that operand's whole stages with TMA
     int32_t b_rows_per_expert; // DH/DX: rows of `b` per expert (N of the weights)
     const __nv_bfloat16 *a;    // DH: dout [N,H]; DX: dz [P_cap,2I]; DW: rows of length M_dim

@@ -45,30 +45,34 @@ constexpr int kPairM = 2 * kM;               // rows per tile (UMMA M of the pai
 constexpr int kN = 256;                      // tile columns (UMMA N)
 constexpr int kNh = kN / 2;                  // B columns per CTA
 constexpr int kSK = 64;                      // K per stage: one 128-byte swizzle atom of bf16
-constexpr int kBwdStages = 6;
 constexpr int kProducerThreads = 128;
-// Epilogue warps: 4 (one per TMEM lane quarter), or 8 for DH, whose SwiGLU
-// backward is heavy: two warps per quarter, each on half the columns.
-template <int kMode>
-struct Roles {
-    static constexpr int kEpiWarps = kMode == kBwdDH ? 8 : 4;
-    static constexpr int kParts = kEpiWarps / 4;
-    static constexpr int kTmaWarp = 1 + kEpiWarps;
-    static constexpr int kCopyThread0 = 32 * (kTmaWarp + 1);
-    static constexpr int kThreads = kCopyThread0 + kProducerThreads;  // MMA, epilogue, TMA, cp.async
-};
 constexpr uint32_t kStageA = kM * kSK * 2;   // 16 KB
 constexpr uint32_t kStageB = kNh * kSK * 2;  // 16 KB
 constexpr uint32_t kStageBytes = kStageA + kStageB;
 constexpr uint32_t kMnAtom = kSK * 128;      // MN-major: one 64-element column of a stage (8 KB)
 constexpr uint32_t kTmemCols = 2 * kN;
-constexpr uint32_t kNumBars = 4 * kBwdStages + 5;
-constexpr uint32_t kStoreBuf = 32 * 128;     // DX/DW: 4 KB per epilogue warp, 32 rows x 64 bf16
-constexpr size_t kSmemStoreOff = (size_t)kBwdStages * kStageBytes;
-constexpr size_t kSmemBarOff = kSmemStoreOff + 4 * kStoreBuf;
-constexpr size_t kSmemMiscOff = kSmemBarOff + 8 * kNumBars;
-constexpr size_t kSmemTableOff = kSmemMiscOff + 16;
-constexpr size_t kSmemBytes = 1024 + kSmemTableOff + 2 * (kMaxExperts + 1) * 4;
+constexpr uint32_t kStoreBuf = 32 * 128;     // 4 KB per epilogue warp: 32 rows x 64 bf16 (TMA stores)
+constexpr uint32_t kZBox = 32 * 128;         // DH: 32 rows x 32 fp32 of z (one TMA box)
+constexpr uint32_t kZBuf = 2 * kZBox;        // DH: z of 32 dh columns, (g, u) interleaved
+// Four epilogue warps, one per TMEM lane quarter.  DH also stages z per
+// epilogue warp, which costs it one pipeline stage.
+template <int kMode>
+struct Roles {
+    static constexpr int kEpiWarps = 4;
+    static constexpr int kParts = 1;
+    static constexpr int kTmaWarp = 1 + kEpiWarps;
+    static constexpr int kCopyThread0 = 32 * (kTmaWarp + 1);
+    static constexpr int kThreads = kCopyThread0 + kProducerThreads;  // MMA, epilogue, TMA, cp.async
+    static constexpr int kStages = kMode == kBwdDH ? 5 : 6;
+    static constexpr uint32_t kNumBars = 4 * kStages + 5 + kEpiWarps;  // + one z barrier per epilogue warp
+    static constexpr size_t kStoreOff = (size_t)kStages * kStageBytes;
+    static constexpr size_t kZOff = kStoreOff + (size_t)kEpiWarps * kStoreBuf;
+    static constexpr size_t kBarOff = kZOff + (kMode == kBwdDH ? (size_t)kEpiWarps * kZBuf : 0);
+    static constexpr size_t kMiscOff = kBarOff + 8 * kNumBars;
+    static constexpr size_t kTableOff = kMiscOff + 16;
+    static constexpr size_t kSmemBytes = 1024 + kTableOff + 2 * (kMaxExperts + 1) * 4;
+    static_assert(kSmemBytes <= 232448, "shared memory per CTA");
+};
 constexpr unsigned long long kAbortSettleNs = 2000000ull;
 
 // Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, M x N,
@@ -134,6 +138,12 @@ __device__ __forceinline__ void mbar_arrive_n(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ void settle_after_abort() {
     const uint64_t t0 = globaltimer_ns();
     while (globaltimer_ns() - t0 < kAbortSettleNs) {
@@ -154,6 +164,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
     bwd_gemm_kernel(const __grid_constant__ BwdGemmArgs a) {
     using R = Roles<kMode>;
     constexpr int kThreads = R::kThreads;
+    constexpr int kBwdStages = R::kStages;
     constexpr bool kMN = kMode == kBwdDW;  // both operands MN-major, K = segment rows
     constexpr uint32_t kIdesc = idesc(kMN, kMN);
     extern __shared__ uint8_t smem_raw[];
@@ -164,7 +175,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
     uint8_t *base_ptr = smem_raw + (base - raw);
     auto a_stage = [&](int s) { return base + (uint32_t)s * kStageBytes; };
     auto b_stage = [&](int s) { return base + (uint32_t)s * kStageBytes + kStageA; };
-    const uint32_t bars = base + (uint32_t)kSmemBarOff;
+    const uint32_t bars = base + (uint32_t)R::kBarOff;
     auto full_bar = [&](int s) { return bars + 8u * s; };                       // even CTA: stage ready
     auto empty_bar = [&](int s) { return bars + 8u * (kBwdStages + s); };
     auto gfull_bar = [&](int s) { return bars + 8u * (2 * kBwdStages + s); };   // odd CTA: its copies
@@ -172,8 +183,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
     auto tfull_bar = [&](int b) { return bars + 8u * (4 * kBwdStages + b); };
     auto tempty_bar = [&](int b) { return bars + 8u * (4 * kBwdStages + 2 + b); };
     const uint32_t drain_bar = bars + 8u * (4 * kBwdStages + 4);
-    uint32_t *misc = reinterpret_cast<uint32_t *>(base_ptr + kSmemMiscOff);
-    int *tile_off_s = reinterpret_cast<int *>(base_ptr + kSmemTableOff);
+    auto z_bar = [&](int w) { return bars + 8u * (4 * kBwdStages + 5 + w); };  // DH: epilogue warp w's z
+    uint32_t *misc = reinterpret_cast<uint32_t *>(base_ptr + R::kMiscOff);
+    int *tile_off_s = reinterpret_cast<int *>(base_ptr + R::kTableOff);
     int *off_s = tile_off_s + (kMaxExperts + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -198,6 +210,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
             mbar_init(tempty_bar(b), 2 * R::kEpiWarps);  // both CTAs' epilogue warps
         }
         mbar_init(drain_bar, 1);
+        for (int w = 0; w < R::kEpiWarps; ++w) mbar_init(z_bar(w), 1);
         misc[1] = 0;
         fence_barrier_init();
     }
@@ -311,11 +324,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
         const int quarter = warp & 3;
         const int rl = quarter * 32 + lane;  // this thread's tile row (TMEM lane)
         const int part = (warp - 1) >> 2;    // this warp's part of the tile's columns
+        const uint32_t store_buf = base + (uint32_t)R::kStoreOff + (uint32_t)(warp - 1) * kStoreBuf;
+        const uint32_t zbuf = base + (uint32_t)R::kZOff + (uint32_t)(warp - 1) * kZBuf;  // DH
+        const uint32_t zbar = z_bar(warp - 1);
+        uint32_t zphase = 0;
+        bool zpending = false;  // a z load of this warp is in flight
+        // DH: z of 32 dh columns [i0, i0+32) of this warp's 32 rows, two boxes of
+        // 32 fp32 per row, by TMA
+        auto load_z = [&](int i0, int wrow0) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(zbar, kZBuf);
+                tma_load_2d(zbuf, &a.tmap_z, zbar, 2 * i0, wrow0);
+                tma_load_2d(zbuf + kZBox, &a.tmap_z, zbar, 2 * i0 + 32, wrow0);
+            }
+            zpending = true;
+        };
+        bool ok = true;
         int tcount = 0;
-        for (int tile = cluster; tile < total; tile += n_clusters, ++tcount) {
+        for (int tile = cluster; ok && tile < total; tile += n_clusters, ++tcount) {
             const BTile t = decode(tile);
             const int acc = tcount & 1;
             const uint32_t acc_phase = (tcount >> 1) & 1;
+            const int wrow0 = t.m0 + row0 + quarter * 32;  // this warp's first tile row
+            // DH, interleaved gate/up, all 32 rows of the warp in the segment: z comes
+            // in and dz goes out by TMA through shared memory, in coalesced boxes;
+            // otherwise each thread reads and writes its own row
+            const bool dh_tma = kMode == kBwdDH && a.layout == MOE_LAYOUT_INTERLEAVED && wrow0 + 31 < t.m_end;
+            if (dh_tma) load_z(t.n0, wrow0);
             if (kMode == kBwdDH) {
                 // bring this row's z columns of the tile into L2 while the MMAs run
                 const int p = t.m0 + row0 + rl;
@@ -353,6 +388,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                     if (i0 >= a.I) break;
                     uint32_t dh[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, dh);
+                    if (dh_tma) {
+                        bool zw = true;
+                        if (lane == 0) zw = mbar_wait_bounded(zbar, zphase, abort);
+                        zw = __shfl_sync(0xffffffffu, zw, 0);
+                        if (!zw) {  // the load stays pending: the exit path waits for it
+                            tmem_ld_wait();
+                            ok = false;
+                            break;
+                        }
+                        zphase ^= 1u;
+                        zpending = false;
+                        // this row's 64 z values: (g_j, u_j) of columns i0 + j at 2j, 2j + 1
+                        float zr[64];
+#pragma unroll
+                        for (int b = 0; b < 2; ++b)
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const float4 v = ld_shared_f4(zbuf + b * kZBox + lane * 128 + ((q ^ (lane & 7)) << 4));
+                                zr[32 * b + 4 * q] = v.x;
+                                zr[32 * b + 4 * q + 1] = v.y;
+                                zr[32 * b + 4 * q + 2] = v.z;
+                                zr[32 * b + 4 * q + 3] = v.w;
+                            }
+                        __syncwarp();  // every lane has read the buffer: the next chunk may land
+                        if (c + 1 < (part + 1) * (kN / 32 / R::kParts) && i0 + 32 < a.I) {
+                            fence_proxy_async_smem();
+                            load_z(i0 + 32, wrow0);
+                        }
+                        tmem_ld_wait();
+                        uint32_t o[32];  // (dg_j, du_j) packed: dz columns 2 i0 .. 2 i0 + 63
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float d = sc * __uint_as_float(dh[j]);
+                            const float g = zr[2 * j], u = zr[2 * j + 1];
+                            float sig;
+                            const float sl = silu_f(g, sig);
+                            o[j] = pack_bf16x2(d * u * sig * (1.0f + g * (1.0f - sig)), d * sl);
+                        }
+                        if (lane == 0) bulk_wait_read0();  // the buffer's previous store has been read
+                        __syncwarp();
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            st_shared_v4(store_buf + lane * 128 + ((q ^ (lane & 7)) << 4), o[4 * q], o[4 * q + 1],
+                                         o[4 * q + 2], o[4 * q + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&a.tmap_out, store_buf, 2 * i0, wrow0);
+                            bulk_commit();
+                        }
+                        continue;
+                    }
                     tmem_ld_wait();
                     if (!valid) continue;
                     if (a.layout == MOE_LAYOUT_INTERLEAVED) {
@@ -407,7 +494,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                 // 32 rows are all stored stages each 32 x 64 block in shared memory
                 // (128-byte swizzle) and writes it with one TMA store; a DX warp that
                 // straddles a segment end stores its valid rows one by one.
-                const int wrow0 = t.m0 + row0 + quarter * 32;  // this warp's first tile row
                 const int r = wrow0 + lane;
                 const bool valid = kMode == kBwdDX ? r < t.m_end : r < a.M_dim;
                 const bool warp_full = kMode == kBwdDX ? wrow0 + 31 < t.m_end : wrow0 + 31 < a.M_dim;
@@ -416,7 +502,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                                            ? (size_t)(valid ? r : 0) * a.out_ld
                                            : ((size_t)t.e * a.M_dim + (valid ? r : 0)) * a.out_ld;
                 __nv_bfloat16 *orow = a.out + row_off;
-                const uint32_t store_buf = base + (uint32_t)kSmemStoreOff + (uint32_t)(warp - 1) * kStoreBuf;
                 const bool zero = kMode == kBwdDW && t.nk == 0;  // empty segment: the gradient is 0
 #pragma unroll 1
                 for (int g = part * (kN / 64 / R::kParts); g < (part + 1) * (kN / 64 / R::kParts); ++g) {
@@ -462,7 +547,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                 else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
             }
         }
-        if (kMode != kBwdDH && lane == 0) bulk_wait0();  // this warp's TMA stores have landed
+        if (zpending && lane == 0 && !mbar_wait_timed(zbar, zphase))
+            atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);  // a z load still in flight: wait for it
+        if (lane == 0) bulk_wait0();                    // this warp's TMA stores have landed
     } else if (warp == R::kTmaWarp) {
         // ---------------------------------------------------------- TMA producer
         // whole-stage boxes of the operands that need no gather: 128-byte-swizzled
@@ -712,14 +799,14 @@ cudaError_t launch_mode(const BwdGemmArgs &a, int max_ctas, cudaStream_t s) {
     int &fit = fit_cache[dev];
     if (fit == 0) {
         err = cudaFuncSetAttribute(bwd_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)kSmemBytes);
+                                   (int)Roles<kMode>::kSmemBytes);
         if (err != cudaSuccess) return err;
         // clusters that can be resident at once (one CTA per SM: the shared
         // memory allows no second)
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(max_ctas & ~1));
         cfg.blockDim = dim3(Roles<kMode>::kThreads);
-        cfg.dynamicSmemBytes = kSmemBytes;
+        cfg.dynamicSmemBytes = Roles<kMode>::kSmemBytes;
         int n = 0;
         err = cudaOccupancyMaxActiveClusters(&n, bwd_gemm_kernel<kMode>, &cfg);
         if (err != cudaSuccess) return err;
@@ -733,7 +820,7 @@ cudaError_t launch_mode(const BwdGemmArgs &a, int max_ctas, cudaStream_t s) {
     }
     if (clusters < 1) clusters = 1;
     // the kernel's cluster shape (2,1,1) is compiled in (__cluster_dims__)
-    bwd_gemm_kernel<kMode><<<2 * clusters, Roles<kMode>::kThreads, kSmemBytes, s>>>(a);
+    bwd_gemm_kernel<kMode><<<2 * clusters, Roles<kMode>::kThreads, Roles<kMode>::kSmemBytes, s>>>(a);
     return cudaGetLastError();
 }
 
