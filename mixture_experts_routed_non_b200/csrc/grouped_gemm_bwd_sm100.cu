@@ -26,14 +26,17 @@
 // the row operands of DH/DX and for the weights read as [N][K]; MN-major
 // (rows = K, 64-element MN atoms, 128-byte swizzle) for both DW operands.
 // Warp roles: warp 0 = TMEM allocator and MMA issuer (even CTA) or the relay
-// that forwards the odd CTA's copy completions to the even CTA, then the epilogue warps
-// (TMEM lane quarter warp % 4; DH has two per quarter, splitting the columns),
-// one TMA producer warp (whole-stage boxes of every operand that needs no
-// gather) and four cp.async producer warps (the gathered rows, and the
-// zero-filled last stage of a DW segment).  Six
-// shared-memory stages of 32 KB per CTA, two TMEM accumulators.  Every wait is bounded; on a
-// timeout the CTA raises its abort flag, records MOE_DEVERR_TIMEOUT, drains
-// its MMAs and copies and frees its TMEM.
+// that forwards the odd CTA's copy completions to the even CTA; four epilogue
+// warps (TMEM lane quarter warp % 4), which write full 32 x 64 output blocks
+// through shared memory with TMA stores (DH also reads z through shared memory
+// by TMA); one TMA producer warp (whole-stage boxes of every operand that needs
+// no gather); four cp.async producer warps (the gathered dout rows of DH, and
+// the zero-filled last stage of a DW segment).  In a stage with no copies the
+// even CTA's TMA thread arrives for the copy warps and the relay, which keeps
+// them off that stage's critical path.  Shared-memory stages of 32 KB per CTA
+// (six; five for DH, whose z staging takes the room of one), two TMEM
+// accumulators.  Every wait is bounded; on a timeout the CTA raises its abort
+// flag, records MOE_DEVERR_TIMEOUT, drains its MMAs and copies and frees its TMEM.
 #include "common.cuh"
 
 namespace moe {
