@@ -113,9 +113,12 @@ __device__ __forceinline__ BTile decode_rows(int tile, int n_tiles, int E, const
 
 // DW: tile -> (expert, 256-row tile of its [M,N] output, 256-column tile).
 // Experts are taken kDwGroup at a time, the expert index varying fastest, so
-// the clusters running at once stream the rows of several experts from DRAM
-// while each expert's rows stay in L2 for its other tiles.
-constexpr int kDwGroup = 16;
+// the clusters running at once read the rows of a few experts, each expert's
+// A columns and B columns shared by several tiles, and the rows stay in L2
+// while its other tiles run.  Four experts (a working set of ~28 MB on
+// prefill) measured best: sixteen thrashed L2 (DRAM reads twice the operand
+// bytes), one or two left too few tiles per group for short segments.
+constexpr int kDwGroup = 4;
 
 __device__ __forceinline__ BTile decode_weights(int tile, int m_tiles, int n_tiles, int E, const int *off) {
     BTile t;
