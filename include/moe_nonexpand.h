@@ -379,6 +379,88 @@ MOE_API int moe_nonexpand_routed_backward(const void *dout, const void *x, const
 MOE_API int moe_router_topk(const void *logits, int32_t logits_dtype, int64_t N, int32_t E, int32_t K,
                             int32_t mode, int32_t *topk_idx, float *topk_w, moe_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Expert-parallel dispatch and combine around the local path (non-expand).
+ *
+ * The dataflow of "End-to-end DeepEP v2 non-expand + SonicMoE integration
+ * #68": a non-expand dispatch hands every rank recv_x [N_recv,H],
+ * recv_topk_idx [N_recv,K] (local expert ids, -1 for a slot whose expert
+ * lives on another rank) and recv_topk_weights; the local expert compute
+ * (moe_nonexpand_forward) turns them into local_out [N_recv,H]; the combine
+ * returns routed_out [T,H] in the source's token order.  Non-expand: a token
+ * row travels once to each rank that owns at least one of its experts.
+ *
+ * Conventions (readings where the pages leave the layout open):
+ *  - R ranks of E_local experts each; global expert e lives on rank
+ *    e / E_local as local expert e % E_local;
+ *  - a destination's receive rows are blocks by source rank in rank order,
+ *    the source's tokens ascending inside its block; the block of source s
+ *    on rank d starts at row_off = sum over s' < s of counts[s'][d], where
+ *    counts[s][d] is send_count[d] of source s (exchanged between ranks by
+ *    the caller, e.g. an all-gather of the R send counts);
+ *  - the combine adds the destinations' rows in ascending rank order, in
+ *    fp32, with one bf16 rounding: deterministic, no atomics.
+ *
+ * Peer buffers: entry d of the pointer tables below is rank d's buffer as
+ * seen from the calling GPU (a peer pointer, through CUDA IPC or symmetric
+ * memory, when d is another GPU; plain loads and stores over NVLink, no TMA
+ * and no multicast).  The caller orders the phases across ranks: every
+ * rank's dispatch completes before any rank reads its receive buffers, and
+ * every rank's local forward completes before any rank's combine reads it.
+ * All calls are enqueued on `stream` without a host sync.
+ * ------------------------------------------------------------------------- */
+#define MOE_EP_MAX_RANKS 32
+
+/*
+ * Layout on one source rank.  topk_idx: device int32 [T,K] global expert ids
+ * (-1: empty slot; any other id outside [0, R*E_local) is not sent and sets
+ * MOE_DEVERR_BAD_EXPERT_ID in *err_word).  Writes send_idx: device int32
+ * [T,R], the token's row inside its block for destination d, or -1 when d
+ * owns none of its experts; send_count: device int32 [R], rows per
+ * destination.  err_word: device uint32 or NULL (bits are OR-ed in, never
+ * cleared).  1 <= R <= MOE_EP_MAX_RANKS, 1 <= K <= 32, E_local >= 1,
+ * R*E_local < 2^31, T*R < 2^31.  One kernel launch (one CTA).
+ */
+MOE_API int moe_ep_layout(const int32_t *topk_idx, int64_t T, int32_t K, int32_t R, int32_t E_local,
+                          int32_t *send_idx, int32_t *send_count, uint32_t *err_word, moe_stream_t stream);
+
+/* Receive buffers of every rank, as seen from the calling (source) rank. */
+typedef struct moe_ep_peers_t {
+    void *recv_x[MOE_EP_MAX_RANKS];      /* rank d: bf16 [N_recv_d, H], 16-byte aligned   */
+    int32_t *recv_idx[MOE_EP_MAX_RANKS]; /* rank d: int32 [N_recv_d, K] local ids or -1  */
+    float *recv_w[MOE_EP_MAX_RANKS];     /* rank d: fp32 [N_recv_d, K], 0 where -1       */
+    int64_t row_off[MOE_EP_MAX_RANKS];   /* first row of this source's block on rank d   */
+} moe_ep_peers_t;
+
+/*
+ * Dispatch on one source rank: for every token t and destination d with
+ * send_idx[t,d] >= 0, row row_off[d] + send_idx[t,d] of rank d's buffers gets
+ * x[t,:] (copied exactly), the local ids of t's experts on d (-1 elsewhere)
+ * and their weights (0 elsewhere).  x: device bf16 [T,H] (16-byte aligned,
+ * H % 8 == 0); topk_idx / topk_w: device [T,K]; send_idx: device [T,R] from
+ * moe_ep_layout; peers: host struct (copied; entries d < R must be non-null).
+ * One kernel launch.
+ */
+MOE_API int moe_ep_dispatch(const void *x, const int32_t *topk_idx, const float *topk_w, const int32_t *send_idx,
+                            int64_t T, int32_t H, int32_t K, int32_t R, int32_t E_local,
+                            const moe_ep_peers_t *peers, moe_stream_t stream);
+
+/* local_out buffers of every rank, as seen from the calling (source) rank. */
+typedef struct moe_ep_sources_t {
+    const void *local_out[MOE_EP_MAX_RANKS]; /* rank d: bf16 [N_recv_d, H], 16-byte aligned */
+    int64_t row_off[MOE_EP_MAX_RANKS];       /* first row of this source's block on rank d  */
+} moe_ep_sources_t;
+
+/*
+ * Combine on one source rank: out[t,:] = sum over d ascending with
+ * send_idx[t,d] >= 0 of local_out_d[row_off[d] + send_idx[t,d], :], summed in
+ * fp32 and rounded once to bf16; a token sent nowhere gets 0.  out: device
+ * bf16 [T,H] (16-byte aligned, H % 8 == 0); src: host struct (copied).  One
+ * kernel launch.
+ */
+MOE_API int moe_ep_combine(const moe_ep_sources_t *src, const int32_t *send_idx, int64_t T, int32_t H, int32_t R,
+                           void *out, moe_stream_t stream);
+
 /* Byte offsets of the workspace's internal arrays (for inspection and tests).
  * Offsets of arrays that the given sizes do not need are 0. */
 typedef struct moe_ws_layout_t {

@@ -61,7 +61,12 @@ EXPORTED = (
     "moe_nonexpand_routed_train_workspace_bytes",
     "moe_nonexpand_routed_forward_train",
     "moe_nonexpand_routed_backward",
+    "moe_ep_layout",
+    "moe_ep_dispatch",
+    "moe_ep_combine",
 )
+
+EP_MAX_RANKS = 32
 
 ROUTER_SOFTMAX_TOPK = 0
 ROUTER_TOPK_SOFTMAX = 1
@@ -99,6 +104,20 @@ class MoeError(RuntimeError):
 
 
 _lib = None
+
+
+class MoeEpPeers(ctypes.Structure):
+    """moe_ep_peers_t: every rank's receive buffers as seen from the caller."""
+    _fields_ = [("recv_x", ctypes.c_void_p * EP_MAX_RANKS),
+                ("recv_idx", ctypes.c_void_p * EP_MAX_RANKS),
+                ("recv_w", ctypes.c_void_p * EP_MAX_RANKS),
+                ("row_off", ctypes.c_int64 * EP_MAX_RANKS)]
+
+
+class MoeEpSources(ctypes.Structure):
+    """moe_ep_sources_t: every rank's local_out as seen from the caller."""
+    _fields_ = [("local_out", ctypes.c_void_p * EP_MAX_RANKS),
+                ("row_off", ctypes.c_int64 * EP_MAX_RANKS)]
 
 
 def load() -> ctypes.CDLL:
@@ -156,6 +175,12 @@ def load() -> ctypes.CDLL:
     lib.moe_nonexpand_routed_forward_train.argtypes = [P, R, i32, i32, i32, P, P, P, P, i32, i32, P, P, sz, P]
     lib.moe_nonexpand_routed_backward.restype = ctypes.c_int
     lib.moe_nonexpand_routed_backward.argtypes = [P, P, R, i32, i32, i32, P, P, i32, i32, P, P, P, P, P, P, P, sz, P]
+    lib.moe_ep_layout.restype = ctypes.c_int
+    lib.moe_ep_layout.argtypes = [P, i64, i32, i32, i32, P, P, P, P]
+    lib.moe_ep_dispatch.restype = ctypes.c_int
+    lib.moe_ep_dispatch.argtypes = [P, P, P, P, i64, i32, i32, i32, i32, ctypes.POINTER(MoeEpPeers), P]
+    lib.moe_ep_combine.restype = ctypes.c_int
+    lib.moe_ep_combine.argtypes = [ctypes.POINTER(MoeEpSources), P, i64, i32, i32, P, P]
     lib.moe_nonexpand_strerror.restype = ctypes.c_char_p
     lib.moe_nonexpand_strerror.argtypes = [ctypes.c_int]
     _lib = lib
@@ -528,6 +553,84 @@ def router_topk(logits: torch.Tensor, K: int, mode: int = ROUTER_SOFTMAX_TOPK,
     _check(load().moe_router_topk(logits.data_ptr(), dtypes[logits.dtype], N, E, K, mode, topk_idx.data_ptr(),
                                   topk_w.data_ptr(), _stream_handle(stream)), "moe_router_topk")
     return topk_idx, topk_w
+
+
+# ---------------------------------------------------------------------------
+# Expert-parallel dispatch / combine (non-expand); see include/moe_nonexpand.h
+# ---------------------------------------------------------------------------
+
+def ep_layout(topk_idx: torch.Tensor, R: int, E_local: int, send_idx: Optional[torch.Tensor] = None,
+              send_count: Optional[torch.Tensor] = None, err: Optional[torch.Tensor] = None,
+              stream: Optional[torch.cuda.Stream] = None):
+    """Source-rank layout: (send_idx [T,R] int32, send_count [R] int32)."""
+    T, K = topk_idx.shape
+    dev = topk_idx.device
+    _need(topk_idx, "topk_idx", torch.int32, (T, K), dev)
+    if send_idx is None:
+        send_idx = torch.empty((T, R), dtype=torch.int32, device=dev)
+    if send_count is None:
+        send_count = torch.empty((R,), dtype=torch.int32, device=dev)
+    _need(send_idx, "send_idx", torch.int32, (T, R), dev)
+    _need(send_count, "send_count", torch.int32, (R,), dev)
+    if err is not None:
+        _need(err, "err", torch.int32, (1,), dev)
+    _check(load().moe_ep_layout(topk_idx.data_ptr(), T, K, R, E_local, send_idx.data_ptr(), send_count.data_ptr(),
+                                _ptr(err), _stream_handle(stream)), "moe_ep_layout")
+    return send_idx, send_count
+
+
+def ep_peers(recv_x, recv_idx, recv_w, row_off) -> MoeEpPeers:
+    """A moe_ep_peers_t from per-rank buffer addresses (ints or tensors) and the
+    caller's block offsets on every rank."""
+    R = len(recv_x)
+    if not (1 <= R <= EP_MAX_RANKS) or not (len(recv_idx) == len(recv_w) == len(row_off) == R):
+        raise ValueError("ep_peers: one entry per rank, 1..32 ranks")
+    p = MoeEpPeers()
+    addr = lambda v: v.data_ptr() if isinstance(v, torch.Tensor) else int(v)
+    for d in range(R):
+        p.recv_x[d], p.recv_idx[d], p.recv_w[d] = addr(recv_x[d]), addr(recv_idx[d]), addr(recv_w[d])
+        p.row_off[d] = int(row_off[d])
+    return p
+
+
+def ep_sources(local_out, row_off) -> MoeEpSources:
+    R = len(local_out)
+    if not (1 <= R <= EP_MAX_RANKS) or len(row_off) != R:
+        raise ValueError("ep_sources: one entry per rank, 1..32 ranks")
+    src = MoeEpSources()
+    for d in range(R):
+        v = local_out[d]
+        src.local_out[d] = v.data_ptr() if isinstance(v, torch.Tensor) else int(v)
+        src.row_off[d] = int(row_off[d])
+    return src
+
+
+def ep_dispatch(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor, send_idx: torch.Tensor,
+                E_local: int, peers: MoeEpPeers, R: int, stream: Optional[torch.cuda.Stream] = None):
+    """Write this source rank's rows into every destination's receive buffers."""
+    T, H = x.shape
+    K = topk_idx.shape[1]
+    dev = x.device
+    _need(x, "x", torch.bfloat16, (T, H), dev)
+    _need(topk_idx, "topk_idx", torch.int32, (T, K), dev)
+    _need(topk_w, "topk_w", torch.float32, (T, K), dev)
+    _need(send_idx, "send_idx", torch.int32, (T, R), dev)
+    _check(load().moe_ep_dispatch(x.data_ptr(), topk_idx.data_ptr(), topk_w.data_ptr(), send_idx.data_ptr(), T, H,
+                                  K, R, E_local, ctypes.byref(peers), _stream_handle(stream)), "moe_ep_dispatch")
+
+
+def ep_combine(src: MoeEpSources, send_idx: torch.Tensor, H: int, out: Optional[torch.Tensor] = None,
+               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """routed_out [T,H] bf16 of this source rank from every destination's local_out."""
+    T, R = send_idx.shape
+    dev = send_idx.device
+    _need(send_idx, "send_idx", torch.int32, (T, R), dev)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (T, H), dev)
+    _check(load().moe_ep_combine(ctypes.byref(src), send_idx.data_ptr(), T, H, R, out.data_ptr(),
+                                 _stream_handle(stream)), "moe_ep_combine")
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -10,6 +10,7 @@
 #include <string.h>
 
 #include "common.cuh"
+#include "ep.cuh"
 
 
 namespace moe {
@@ -845,6 +846,66 @@ extern "C" MOE_API int moe_router_topk(const void *logits, int32_t logits_dtype,
     if (st) return st;
     return launch_router(logits, logits_dtype == MOE_DTYPE_BF16, N, E, K, mode, topk_idx, topk_w, dev.sms,
                          reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+// ---- expert-parallel dispatch / combine (non-expand) ----------------------
+extern "C" MOE_API int moe_ep_layout(const int32_t *topk_idx, int64_t T, int32_t K, int32_t R, int32_t E_local,
+                                     int32_t *send_idx, int32_t *send_count, uint32_t *err_word,
+                                     moe_stream_t stream) {
+    if (T < 0 || K < 1 || K > 32 || R < 1 || R > MOE_EP_MAX_RANKS || E_local < 1) return MOE_ERR_ARG;
+    if ((int64_t)R * E_local >= ((int64_t)1 << 31) || T * (int64_t)R >= ((int64_t)1 << 31) ||
+        T * (int64_t)K >= ((int64_t)1 << 40))
+        return MOE_ERR_ARG;
+    if (!send_count || (T > 0 && (!topk_idx || !send_idx))) return MOE_ERR_ARG;
+    if (!aligned(topk_idx, 4) || !aligned(send_idx, 4) || !aligned(send_count, 4) || !aligned(err_word, 4))
+        return MOE_ERR_ARG;
+    DeviceInfo dev;
+    const int st = device_info(&dev);
+    if (st) return st;
+    return launch_ep_layout(topk_idx, T, K, R, E_local, send_idx, send_count, err_word,
+                            reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+extern "C" MOE_API int moe_ep_dispatch(const void *x, const int32_t *topk_idx, const float *topk_w,
+                                       const int32_t *send_idx, int64_t T, int32_t H, int32_t K, int32_t R,
+                                       int32_t E_local, const moe_ep_peers_t *peers, moe_stream_t stream) {
+    if (T < 0 || H < 8 || H % 8 != 0 || K < 1 || K > 32 || R < 1 || R > MOE_EP_MAX_RANKS || E_local < 1 || !peers)
+        return MOE_ERR_ARG;
+    if ((int64_t)R * E_local >= ((int64_t)1 << 31) || T * (int64_t)R >= ((int64_t)1 << 31)) return MOE_ERR_ARG;
+    if (T > 0 && (!x || !topk_idx || !topk_w || !send_idx)) return MOE_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) || !aligned(send_idx, 4)) return MOE_ERR_ARG;
+    for (int d = 0; d < R; ++d) {
+        if (!peers->recv_x[d] || !peers->recv_idx[d] || !peers->recv_w[d] || peers->row_off[d] < 0)
+            return MOE_ERR_ARG;
+        if (!aligned(peers->recv_x[d], 16) || !aligned(peers->recv_idx[d], 4) || !aligned(peers->recv_w[d], 4))
+            return MOE_ERR_ARG;
+    }
+    DeviceInfo dev;
+    const int st = device_info(&dev);
+    if (st) return st;
+    return launch_ep_dispatch(x, topk_idx, topk_w, send_idx, T, H, K, R, E_local, *peers, dev.sms,
+                              reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
+
+extern "C" MOE_API int moe_ep_combine(const moe_ep_sources_t *src, const int32_t *send_idx, int64_t T, int32_t H,
+                                      int32_t R, void *out, moe_stream_t stream) {
+    if (T < 0 || H < 8 || H % 8 != 0 || R < 1 || R > MOE_EP_MAX_RANKS || !src) return MOE_ERR_ARG;
+    if (T * (int64_t)R >= ((int64_t)1 << 31)) return MOE_ERR_ARG;
+    if (T > 0 && (!send_idx || !out)) return MOE_ERR_ARG;
+    if (!aligned(send_idx, 4) || !aligned(out, 16)) return MOE_ERR_ARG;
+    for (int d = 0; d < R; ++d)
+        if (!src->local_out[d] || !aligned(src->local_out[d], 16) || src->row_off[d] < 0) return MOE_ERR_ARG;
+    DeviceInfo dev;
+    const int st = device_info(&dev);
+    if (st) return st;
+    return launch_ep_combine(*src, send_idx, T, H, R, out, dev.sms, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }

@@ -24,6 +24,23 @@ def within_tolerance(gpu: np.ndarray, ref: np.ndarray, rtol=RTOL, atol_rms=ATOL_
                                  if err.size else None)
 
 
+def assert_close_ep(gpu, ref, mag, what=""):
+    """Expert-parallel routed_out: every rank's partial (its local forward
+    output) carries the forward tolerance of that partial and is rounded to
+    bf16 before the combine adds the partials.  So |ref| and rms(ref) of the
+    forward bound become S = sum over the partials of |partial| (``mag``) and
+    rms(S); with a single partial this is the forward tolerance itself."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    mag = np.asarray(mag, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(mag * mag))) if mag.size else 0.0
+    bound = RTOL * mag + ATOL_RMS * rms
+    err = np.abs(gpu - ref)
+    bad = ~(err <= bound)
+    assert not bad.any(), (f"{what}: max_err {err.max():.4g}, rms(S) {rms:.4g}, n_bad {int(bad.sum())}/{err.size}, "
+                           f"worst {np.unravel_index(int(np.argmax(err - bound)), err.shape)}")
+
+
 def assert_close(gpu, ref, what=""):
     ok, info = within_tolerance(gpu, ref)
     assert ok, f"{what}: {info}"

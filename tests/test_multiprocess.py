@@ -15,6 +15,7 @@ import socket
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 import torch.multiprocessing as mp
 
@@ -98,3 +99,51 @@ def test_reference_arm_torchrun_two_ranks():
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == "tiny"
+
+
+def _counts_worker(rank: int, world: int, port: int, counts, out_dir: str) -> None:
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    sys.path.insert(0, ROOT)
+    from mixture_experts_routed_non_b200 import ep
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        got = ep.exchange_counts(torch.tensor(counts[rank], dtype=torch.int32))
+        off, n_recv = ep.block_offsets(got)
+    finally:
+        dist.destroy_process_group()
+    with open(os.path.join(out_dir, f"counts{rank}.json"), "w") as f:
+        json.dump({"counts": got.tolist(), "off": off.tolist(), "n_recv": n_recv.tolist()}, f)
+
+
+def test_ep_count_exchange_gloo(tmp_path):
+    """The expert-parallel count exchange (an all-gather of every rank's send
+    counts) and the receive-block offsets derived from it agree on every rank
+    with the oracle's offsets."""
+    sys.path.insert(0, ROOT)
+    from oracle import ep as oep
+    world = 2
+    counts = [[3, 5], [0, 7]]  # counts[s][d]
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_counts_worker, args=(r, world, port, counts, str(tmp_path))) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+    for p in procs:
+        if p.is_alive():
+            p.kill()
+            p.join()
+    assert [p.exitcode for p in procs] == [0, 0]
+    ref_off, ref_n = oep.recv_offsets(np.array(counts))
+    for r in range(world):
+        with open(tmp_path / f"counts{r}.json") as f:
+            got = json.load(f)
+        assert got["counts"] == counts
+        assert got["off"] == ref_off.tolist() and got["n_recv"] == ref_n.tolist()
