@@ -300,6 +300,76 @@ def router_only(dev, peaks, reps: int = 10, ring: int = 20):
             "l2": f"ring of {ring} logits buffers ({ring * N * E * 4 / 1e6:.0f} MB) in one graph"}
 
 
+def ep_emulated(dev, peaks, reps: int = 20):
+    """Expert-parallel dispatch and combine with 8 ranks emulated on this GPU,
+    sized like the rank-local shape after 8-way dispatch (H=7168, 32 local
+    experts per rank, K=8 global slots, ~8192 receive rows per rank): 1560
+    tokens per source rank.  Device time of the eight dispatch launches and
+    of the eight combine launches (median over ``reps``).  Emulated ranks
+    move rows HBM to HBM; across GPUs the same stores and loads cross NVLink.
+    Algorithmic bytes: dispatch reads x once per source row and writes each
+    receive row (x, ids, weights); combine reads each receive row and writes
+    the routed rows."""
+    import numpy as np
+    import torch
+
+    from mixture_experts_routed_non_b200 import binding
+    from mixture_experts_routed_non_b200.ep import EmulatedRanks
+    R, E_local, T, K, H = 8, 32, 1560, 8, 7168
+    g = torch.Generator(device=dev).manual_seed(3)
+    xs = [torch.randn((T, H), generator=g, device=dev).to(torch.bfloat16) for _ in range(R)]
+    idxs = [torch.argsort(torch.rand((T, R * E_local), generator=g, device=dev), dim=1)[:, :K].to(torch.int32)
+            .contiguous() for _ in range(R)]
+    ws = [torch.rand((T, K), generator=g, device=dev) for _ in range(R)]
+    er = EmulatedRanks(R, E_local, dev)
+    st = er.dispatch(xs, idxs, ws)
+    recv_x, recv_idx, recv_w = st["_bufs"]
+    peers = [binding.ep_peers(recv_x, recv_idx, recv_w, st["off"][:, s]) for s in range(R)]
+    local = [t.clone() for t in st["recv_x"]]
+    srcs = [binding.ep_sources(local, st["off"][:, s]) for s in range(R)]
+    outs = [torch.empty((T, H), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        times = []
+        for i in range(reps + 3):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            if i >= 3:
+                times.append(a.elapsed_time(b))
+        return float(np.median(times))
+
+    def dispatch():
+        for s in range(R):
+            binding.ep_dispatch(xs[s], idxs[s], ws[s], st["send_idx"][s], E_local, peers[s], R)
+
+    def combine():
+        for s in range(R):
+            binding.ep_combine(srcs[s], st["send_idx"][s], H, out=outs[s])
+
+    def layout():
+        for s in range(R):
+            binding.ep_layout(idxs[s], R, E_local, send_idx=st["send_idx"][s])
+
+    ms_d, ms_c, ms_l = timed(dispatch), timed(combine), timed(layout)
+    rows = int(st["n_recv"].sum())
+    b_d = R * T * H * 2 + rows * (H * 2 + K * 8)
+    b_c = rows * H * 2 + R * T * H * 2
+    return {"ranks": R, "E_local": E_local, "tokens_per_rank": T, "K": K, "H": H,
+            "recv_rows_per_rank": float(rows / R), "layout_ms": ms_l,
+            "dispatch_ms": ms_d, "dispatch_gbs": b_d / (ms_d * 1e-3) / 1e9,
+            "combine_ms": ms_c, "combine_gbs": b_c / (ms_c * 1e-3) / 1e9,
+            "frac_hbm": {"dispatch": b_d / (ms_d * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "combine": b_c / (ms_c * 1e-3) / 1e9 / peaks["hbm_gbs"]},
+            "launches": {"layout": R, "dispatch": R, "combine": R},
+            "note": "8 ranks emulated on one GPU (HBM to HBM); L2 flushed before each timed phase"}
+
+
 def backward_leg(inp, w1, b1, layout, dev, peaks, steps: int = 30, warmup: int = 3):
     """One training step, forward_train + backward, on the bench workload:
     mean device time per step with the backward's seven stages timed by
@@ -559,6 +629,7 @@ def run_ours(args, rank, world, local):
     meta_c2 = metadata_only(dev, peaks) if rank == 0 else None
     router = router_only(dev, peaks) if rank == 0 else None
     train = backward_leg(inp, w1, b1, args.layout, dev, peaks) if rank == 0 else None
+    ep = ep_emulated(dev, peaks) if rank == 0 else None
 
     if world > 1:
         dist.destroy_process_group()
@@ -609,6 +680,7 @@ def run_ours(args, rank, world, local):
         "metadata_only": meta_c2,
         "router_only": router,
         "training": train,
+        "ep_emulated": ep,
         "gpu_launches": 4 * args.steps,  # meta, up, down, combine (plus one 4-byte memset)
         "clocks": clocks,
     }

@@ -124,24 +124,37 @@ __global__ void __launch_bounds__(kEpThreads) ep_dispatch_kernel(const uint4 *__
 __global__ void __launch_bounds__(kEpThreads) ep_combine_kernel(const moe_ep_sources_t src,
                                                                const int32_t *__restrict__ send_idx, int64_t T,
                                                                int H, int R, uint4 *__restrict__ out) {
-    __shared__ int64_t row[MOE_EP_MAX_RANKS];
+    // the token's destinations in ascending rank order, compacted: their row pointers
+    __shared__ const uint4 *vrow[MOE_EP_MAX_RANKS];
+    __shared__ int nv;
     const int chunks = H >> 3;
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
-        if (threadIdx.x < R) {
-            const int j = __ldg(send_idx + t * R + threadIdx.x);
-            row[threadIdx.x] = j >= 0 ? src.row_off[threadIdx.x] + j : -1;
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            const int j = lane < R ? __ldg(send_idx + t * R + lane) : -1;
+            const unsigned b = __ballot_sync(0xffffffffu, j >= 0);
+            if (j >= 0)
+                vrow[__popc(b & ((1u << lane) - 1u))] =
+                    reinterpret_cast<const uint4 *>(src.local_out[lane]) + (src.row_off[lane] + j) * chunks;
+            if (lane == 0) nv = __popc(b);
         }
         __syncthreads();
+        const int n = nv;
         for (int c = threadIdx.x; c < chunks; c += kEpThreads) {
             float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-            for (int d = 0; d < R; ++d) {  // ascending rank order: a fixed summation order
-                if (row[d] < 0) continue;
-                const uint4 v = reinterpret_cast<const uint4 *>(src.local_out[d])[row[d] * chunks + c];
-                const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+            for (int i0 = 0; i0 < n; i0 += 4) {  // four rows in flight, added in ascending rank order
+                uint4 v[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    acc[2 * i] += bf16lo(q[i]);
-                    acc[2 * i + 1] += bf16hi(q[i]);
+                for (int u = 0; u < 4; ++u) v[u] = i0 + u < n ? vrow[i0 + u][c] : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    if (i0 + u >= n) break;
+                    const uint32_t q[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        acc[2 * i] += bf16lo(q[i]);
+                        acc[2 * i + 1] += bf16hi(q[i]);
+                    }
                 }
             }
             out[t * chunks + c] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
