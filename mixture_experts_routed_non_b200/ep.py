@@ -117,8 +117,10 @@ class ProcessGroupRanks:
 
     Phases per call: layout -> all-gather of counts -> dispatch (peer stores)
     -> barrier -> local forward -> barrier -> combine (peer loads) -> barrier.
-    Not run on more than one GPU by the tests of this repository (its calls
-    get one GPU); the count exchange and the offsets are tested with gloo.
+    Tested on one GPU with a one-rank NCCL group (count all-gather, barriers,
+    buffers; no IPC), and the count exchange with two gloo ranks on CPU; not
+    run on more than one GPU by the tests of this repository (its calls get
+    one GPU).
     """
 
     def __init__(self, E_local: int, capacity: int, H: int, K: int, group=None, device=None, opener=None):
@@ -140,6 +142,8 @@ class ProcessGroupRanks:
         the peer's opened from the IPC handle it published."""
         import torch.distributed as dist
         from torch.multiprocessing.reductions import reduce_tensor
+        if self.R == 1:
+            return [mine]
         handles = [None] * self.R
         dist.all_gather_object(handles, [reduce_tensor(t) for t in mine], group=self.group)
         out = []

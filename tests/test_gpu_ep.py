@@ -232,3 +232,33 @@ def test_argument_errors():
     with pytest.raises(binding.MoeError):
         binding.ep_dispatch(xs[0], idxs[0], ws[0], send_idx, E_local, bad, R)
     assert block_offsets(np.array([[1, 2], [3, 4]]))[0].tolist() == [[0, 1], [0, 2]]
+
+
+def test_process_group_ranks_single_rank():
+    """The one-process-per-GPU path with a one-rank NCCL group: the count
+    all-gather, barriers and buffers of ProcessGroupRanks around dispatch ->
+    local forward -> combine.  With one rank the routed output must equal the
+    plain forward bit for bit (same rows, same arithmetic, one partial)."""
+    import socket
+    from datetime import timedelta
+
+    import torch.distributed as dist
+
+    from mixture_experts_routed_non_b200.ep import ProcessGroupRanks
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True, timeout=timedelta(seconds=60))
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        E, T, K, H, I = 8, 300, 4, 128, 128
+        xs, idxs, ws = _problem(1, E, T, K, H, seed=21)
+        w1, w2, _, _ = _weights(E, H, I, seed=3, bias=False)
+        pg = ProcessGroupRanks(E_local=E, capacity=T, H=H, K=K)
+        out = pg.forward(xs[0], idxs[0], ws[0], w1, w2)
+        ref = binding.forward(xs[0], idxs[0], ws[0], w1, w2)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+    finally:
+        dist.destroy_process_group()
