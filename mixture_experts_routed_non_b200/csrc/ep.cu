@@ -7,9 +7,9 @@
 //
 //   layout    one CTA walks the source's tokens in chunks of 1024: each thread
 //             forms its token's destination mask, warp ballots per destination
-//             give the token's rank inside its warp, a scan over the warps and
-//             a running base give its row inside each destination's block
-//             (stable: tokens ascending).
+//             give the token's rank inside its warp, a shuffle scan over the
+//             warps (one warp per destination) and a running base give its
+//             row inside each destination's block (stable: tokens ascending).
 //   dispatch  one CTA per token (grid-stride): each thread loads 16-byte chunks
 //             of x[t] once and stores them to every destination's receive
 //             rows; stores to another GPU's buffers go over NVLink as plain
@@ -49,10 +49,15 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) ep_layout_kernel(const int3
         const int64_t t = t0 + tid;
         uint32_t mask = 0;
         if (t < T) {
-            for (int k = 0; k < K; ++k) {
-                const int e = __ldg(topk_idx + t * K + k);
-                if (e >= 0 && e < n_exp) mask |= 1u << (e / E_local);
-                else if (e != -1) bad = true;
+            for (int k0 = 0; k0 < K; k0 += 8) {  // eight ids in flight at once
+                int e[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) e[u] = k0 + u < K ? __ldg(topk_idx + t * K + k0 + u) : -1;
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (e[u] >= 0 && e[u] < n_exp) mask |= 1u << (e[u] / E_local);
+                    else if (e[u] != -1) bad = true;
+                }
             }
         }
         int pre[MOE_EP_MAX_RANKS];  // this token's rank among its warp's tokens bound for d
@@ -65,14 +70,19 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) ep_layout_kernel(const int3
             }
         }
         __syncthreads();
-        if (tid < R) {  // exclusive scan over the warps, on top of the running base
-            int acc = run[tid];
-            for (int w = 0; w < kLayoutWarps; ++w) {
-                const int c = warp_base[w][tid];
-                warp_base[w][tid] = acc;
-                acc += c;
+        if (warp < R) {  // warp d: exclusive scan over the 32 warps' counts for destination d
+            const int d = warp;
+            const int c = warp_base[lane][d];
+            int v = c;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += u;
             }
-            run[tid] = acc;
+            const int base = run[d];
+            warp_base[lane][d] = base + v - c;
+            __syncwarp();
+            if (lane == 31) run[d] = base + v;
         }
         __syncthreads();
         if (t < T) {
