@@ -262,3 +262,44 @@ def test_process_group_ranks_single_rank():
         assert torch.equal(out, ref)
     finally:
         dist.destroy_process_group()
+
+
+def test_duplicate_experts_and_all_slots_on_one_rank():
+    """A row naming the same expert twice keeps both slots (one receive row);
+    a row whose slots all live on one rank is sent to that rank only."""
+    R, E_local, K, H, I = 4, 3, 4, 64, 64
+    T = 40
+    rng = np.random.default_rng(8)
+    idx = np.stack([rng.choice(R * E_local, size=K, replace=False) for _ in range(T)]).astype(np.int32)
+    idx[0] = [5, 5, 1, -1]               # expert 5 twice
+    idx[1] = [6, 7, 8, 6]                # all on rank 2, expert 6 twice
+    idx[2] = [-1, -1, -1, -1]            # sent nowhere
+    xs = [torch.randn((T, H), device="cuda").to(torch.bfloat16) for _ in range(R)]
+    idxs = [torch.from_numpy(idx).cuda() for _ in range(R)]
+    ws = [torch.rand((T, K), device="cuda") for _ in range(R)]
+    ref = _oracle_dispatch(xs, idxs, ws, R, E_local)
+    st = EmulatedRanks(R, E_local).dispatch(xs, idxs, ws)
+    for d in range(R):
+        assert np.array_equal(st["recv_idx"][d].cpu().numpy(), ref["recv_idx"][d])
+        assert np.array_equal(st["recv_w"][d].cpu().numpy(), ref["recv_w"][d])
+    si = st["send_idx"][0].cpu().numpy()
+    assert (si[1] >= 0).tolist() == [False, False, True, False]
+    assert (si[2] < 0).all()
+    w1, w2, b1, b2 = _weights(R * E_local, H, I, seed=9)
+    outs = EmulatedRanks(R, E_local).forward(xs, idxs, ws, w1, w2, b1, b2)
+    torch.cuda.synchronize()
+    for s in range(R):
+        wts = oracle.Weights(xs[s].cpu(), w1.cpu(), b1.cpu(), w2.cpu(), b2.cpu())
+        fwd = oracle.forward_rows(wts, idx, ws[s].cpu().numpy())
+        # each token here has at most two partials; the bound uses their magnitudes
+        d = _oracle_dispatch(xs[s:s + 1] * R, idxs[s:s + 1] * R, ws[s:s + 1] * R, R, E_local)
+        part = []
+        for r in range(R):
+            rx = torch.from_numpy(d["recv_x"][r]).view(torch.bfloat16)
+            sl = slice(r * E_local, (r + 1) * E_local)
+            wr = oracle.Weights(rx, w1[sl].cpu(), b1[sl].cpu(), w2[sl].cpu(), b2[sl].cpu())
+            part.append(oracle.forward_rows(wr, d["recv_idx"][r], d["recv_w"][r]) if rx.shape[0] else
+                        np.zeros((0, H)))
+        mag = oep.ep_combine([np.abs(p) for p in part], d["send_idx"], d["off"])[0]
+        assert_close_ep(to_np(outs[s]), fwd, mag, f"rank {s}")
+        assert (to_np(outs[s])[2] == 0).all()
