@@ -83,3 +83,37 @@ def test_router_feeds_the_forward():
     wts = oracle.Weights(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
     ref = oracle.forward_rows(wts, ri, rw.astype(np.float32))
     assert_close(to_np(out), ref, "out (router -> forward)")
+
+
+@pytest.mark.parametrize("mode", MODES)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("E", [32, 64, 128, 256])
+@pytest.mark.parametrize("K", [1, 3, 8])
+def test_router_common_shapes(E, K, dtype, mode):
+    """Expert counts of the common MoE shapes with K <= 8, N not a multiple of
+    the tokens a block handles."""
+    _check(synthetic.make_logits(1003, E, seed=E * 10 + K, dtype=dtype, device="cuda"), K, mode)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_router_ties_nan_inf_at_128_and_256(mode):
+    _check(synthetic.make_logits(2051, 128, seed=5, kind="ties", device="cuda"), 8, mode)
+    _check(synthetic.make_logits(515, 256, seed=6, kind="ties", dtype=torch.bfloat16, device="cuda"), 6, mode)
+    lg = synthetic.make_logits(40, 128, seed=7, device="cuda")
+    lg[0, :] = float("-inf")
+    lg[1, 5] = float("nan")
+    lg[2, :120] = float("-inf")   # fewer finite logits than K
+    lg[3, 77] = float("inf")
+    lg[4, ::3] = float("nan")
+    lg[5, :] = 1.0                # every logit equal: ids 0..K-1
+    lg[6, 96:] = 3.0              # the largest all in the last lane
+    _check(lg, 8, mode)
+
+
+def test_router_logits_not_16_byte_aligned():
+    """Logits 4 bytes past a 16-byte boundary (a slice) give the same results."""
+    big = synthetic.make_logits(301 * 128 + 1, 1, seed=8, device="cuda").reshape(-1)
+    lg = big[1:].view(301, 128)
+    assert lg.data_ptr() % 16 == 4
+    for mode in MODES:
+        _check(lg, 8, mode)
