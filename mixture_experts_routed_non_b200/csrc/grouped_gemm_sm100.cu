@@ -121,6 +121,12 @@ __device__ __forceinline__ void add_bias32(uint32_t (&r)[32], const __nv_bfloat1
     }
 }
 
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
 // 32 fp32 values (as bits) to dst (128 bytes, 16-byte aligned)
 __device__ __forceinline__ void store_f32x32(float *dst, const uint32_t (&r)[32]) {
     uint4 *d = reinterpret_cast<uint4 *>(dst);
@@ -385,6 +391,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
             __nv_bfloat16 *orow = a.out + (size_t)(valid ? p : 0) * a.out_cols;
             const __nv_bfloat16 *brow = a.bias ? a.bias + (size_t)t.e * a.n_dim : nullptr;
 
+            // training: 32 fp32 of z (this thread's row, columns zc .. zc+31).  A full
+            // warp passes its 32 x 32 block through the store buffer (swizzled) and
+            // writes it row by row, eight lanes per 128-byte row, so each store
+            // instruction covers four whole rows instead of 32 pieces of 32 rows.
+            auto store_z32 = [&](int zc, const uint32_t (&v)[32]) {
+                if (warp_full) {
+                    if (lane == 0) bulk_wait_read0();  // the buffer's previous TMA store has been read
+                    __syncwarp();
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        st_shared_v4(store_buf + lane * 128 + ((c ^ (lane & 7)) << 4), v[4 * c], v[4 * c + 1],
+                                     v[4 * c + 2], v[4 * c + 3]);
+                    __syncwarp();
+                    const int ch = lane & 7;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int rr = 4 * j + (lane >> 3);
+                        const uint4 q = ld_shared_v4(store_buf + rr * 128 + ((ch ^ (rr & 7)) << 4));
+                        *reinterpret_cast<uint4 *>(a.z_out + (size_t)(wrow0 + rr) * (2 * a.I) + zc + 4 * ch) = q;
+                    }
+                    __syncwarp();  // the buffer is free again
+                } else if (valid) {
+                    store_f32x32(a.z_out + (size_t)p * (2 * a.I) + zc, v);
+                }
+            };
+
             // 64 output columns (32 packed bf16 pairs) of this thread's row
             auto store64 = [&](int col0, const uint32_t (&v)[32]) {
                 if (warp_full) {
@@ -428,10 +460,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                             add_bias32(g, brow + col0 + hf * 32);
                             add_bias32(u, brow + a.I + col0 + hf * 32);
                         }
-                        if (a.z_out && valid) {  // training: keep z for the backward
-                            float *zr = a.z_out + (size_t)p * (2 * a.I);
-                            store_f32x32(zr + col0 + hf * 32, g);
-                            store_f32x32(zr + a.I + col0 + hf * 32, u);
+                        if (a.z_out) {  // training: keep z for the backward
+                            store_z32(col0 + hf * 32, g);
+                            store_z32(a.I + col0 + hf * 32, u);
                         }
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
@@ -462,10 +493,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                             add_bias32(r0, brow + acol);
                             add_bias32(r1, brow + acol + 32);
                         }
-                        if (a.z_out && valid) {  // training: keep z for the backward
-                            float *zr = a.z_out + (size_t)p * (2 * a.I);
-                            store_f32x32(zr + acol, r0);
-                            store_f32x32(zr + acol + 32, r1);
+                        if (a.z_out) {  // training: keep z for the backward
+                            store_z32(acol, r0);
+                            store_z32(acol + 32, r1);
                         }
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
