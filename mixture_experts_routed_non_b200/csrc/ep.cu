@@ -5,7 +5,8 @@
 // combine -> routed_out).  A token row travels once to each rank owning one
 // of its experts.
 //
-//   layout    one CTA walks the source's tokens in chunks of 1024: each thread
+//   layout    one CTA walks the source's tokens in chunks (ids read and rows
+//             written through shared memory, coalesced): each thread
 //             forms its token's destination mask, warp ballots per destination
 //             give the token's rank inside its warp, a shuffle scan over the
 //             warps (one warp per destination) and a running base give its
@@ -32,32 +33,34 @@ constexpr int kLayoutThreads = 1024;
 constexpr int kLayoutWarps = kLayoutThreads / 32;
 constexpr int kEpThreads = 256;
 
+constexpr int kLayoutStage = 8192;  // ints staged per chunk (32 KB): ids in, then rows out
+
 __global__ void __launch_bounds__(kLayoutThreads, 1) ep_layout_kernel(const int32_t *__restrict__ topk_idx,
                                                                      int64_t T, int K, int R, int E_local,
                                                                      int32_t *__restrict__ send_idx,
                                                                      int32_t *__restrict__ send_count,
                                                                      uint32_t *err) {
+    __shared__ int stage[kLayoutStage];                            // a chunk's ids, then its send_idx rows
     __shared__ int warp_base[kLayoutWarps][MOE_EP_MAX_RANKS + 1];  // per warp and destination
     __shared__ int run[MOE_EP_MAX_RANKS];                          // rows given out so far
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const unsigned lt = (1u << lane) - 1u;
     const int64_t n_exp = (int64_t)R * E_local;
+    // tokens per chunk: both the chunk's [C,K] ids and its [C,R] rows fit the stage
+    const int C = min(kLayoutThreads, kLayoutStage / max(K, R));
     if (tid < MOE_EP_MAX_RANKS) run[tid] = 0;
     bool bad = false;
-    __syncthreads();
-    for (int64_t t0 = 0; t0 < T; t0 += kLayoutThreads) {
-        const int64_t t = t0 + tid;
+    for (int64_t t0 = 0; t0 < T; t0 += C) {
+        const int nt = (int)min((int64_t)C, T - t0);
+        __syncthreads();  // the stage's previous rows have been written out
+        for (int i = tid; i < nt * K; i += kLayoutThreads) stage[i] = __ldg(topk_idx + t0 * K + i);  // coalesced
+        __syncthreads();
         uint32_t mask = 0;
-        if (t < T) {
-            for (int k0 = 0; k0 < K; k0 += 8) {  // eight ids in flight at once
-                int e[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) e[u] = k0 + u < K ? __ldg(topk_idx + t * K + k0 + u) : -1;
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    if (e[u] >= 0 && e[u] < n_exp) mask |= 1u << (e[u] / E_local);
-                    else if (e[u] != -1) bad = true;
-                }
+        if (tid < nt) {
+            for (int k = 0; k < K; ++k) {
+                const int e = stage[tid * K + k];
+                if (e >= 0 && e < n_exp) mask |= 1u << (e / E_local);
+                else if (e != -1) bad = true;
             }
         }
         int pre[MOE_EP_MAX_RANKS];  // this token's rank among its warp's tokens bound for d
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) ep_layout_kernel(const int3
                 if (lane == 0) warp_base[warp][d] = __popc(b);
             }
         }
-        __syncthreads();
+        __syncthreads();  // counts in; every thread has read its ids from the stage
         if (warp < R) {  // warp d: exclusive scan over the 32 warps' counts for destination d
             const int d = warp;
             const int c = warp_base[lane][d];
@@ -85,13 +88,15 @@ __global__ void __launch_bounds__(kLayoutThreads, 1) ep_layout_kernel(const int3
             if (lane == 31) run[d] = base + v;
         }
         __syncthreads();
-        if (t < T) {
+        if (tid < nt) {
 #pragma unroll
             for (int d = 0; d < MOE_EP_MAX_RANKS; ++d)
-                if (d < R) send_idx[t * R + d] = ((mask >> d) & 1u) ? warp_base[warp][d] + pre[d] : -1;
+                if (d < R) stage[tid * R + d] = ((mask >> d) & 1u) ? warp_base[warp][d] + pre[d] : -1;
         }
-        __syncthreads();  // warp_base is rewritten by the next chunk
+        __syncthreads();
+        for (int i = tid; i < nt * R; i += kLayoutThreads) send_idx[t0 * R + i] = stage[i];  // coalesced
     }
+    __syncthreads();
     if (tid < R) send_count[tid] = run[tid];
     if (bad && err) atomicOr(err, MOE_DEVERR_BAD_EXPERT_ID);
 }
