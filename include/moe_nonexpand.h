@@ -424,12 +424,16 @@ MOE_API int moe_router_topk(const void *logits, int32_t logits_dtype, int64_t N,
 MOE_API int moe_ep_layout(const int32_t *topk_idx, int64_t T, int32_t K, int32_t R, int32_t E_local,
                           int32_t *send_idx, int32_t *send_count, uint32_t *err_word, moe_stream_t stream);
 
-/* Receive buffers of every rank, as seen from the calling (source) rank. */
+/* Receive buffers of every rank, as seen from the calling (source) rank.  A row
+ * at or past recv_rows[d] is never written: it sets MOE_DEVERR_ABORTED in
+ * *err_word (device uint32, may be NULL) instead. */
 typedef struct moe_ep_peers_t {
-    void *recv_x[MOE_EP_MAX_RANKS];      /* rank d: bf16 [N_recv_d, H], 16-byte aligned   */
-    int32_t *recv_idx[MOE_EP_MAX_RANKS]; /* rank d: int32 [N_recv_d, K] local ids or -1  */
-    float *recv_w[MOE_EP_MAX_RANKS];     /* rank d: fp32 [N_recv_d, K], 0 where -1       */
-    int64_t row_off[MOE_EP_MAX_RANKS];   /* first row of this source's block on rank d   */
+    void *recv_x[MOE_EP_MAX_RANKS];      /* rank d: bf16 [recv_rows_d, H], 16-byte aligned */
+    int32_t *recv_idx[MOE_EP_MAX_RANKS]; /* rank d: int32 [recv_rows_d, K] local ids or -1 */
+    float *recv_w[MOE_EP_MAX_RANKS];     /* rank d: fp32 [recv_rows_d, K], 0 where -1      */
+    int64_t row_off[MOE_EP_MAX_RANKS];   /* first row of this source's block on rank d    */
+    int64_t recv_rows[MOE_EP_MAX_RANKS]; /* rows rank d's buffers hold                     */
+    uint32_t *err_word;                  /* this rank's device error word, or NULL         */
 } moe_ep_peers_t;
 
 /*
@@ -445,10 +449,14 @@ MOE_API int moe_ep_dispatch(const void *x, const int32_t *topk_idx, const float 
                             int64_t T, int32_t H, int32_t K, int32_t R, int32_t E_local,
                             const moe_ep_peers_t *peers, moe_stream_t stream);
 
-/* local_out buffers of every rank, as seen from the calling (source) rank. */
+/* local_out buffers of every rank, as seen from the calling (source) rank.  A row
+ * at or past rows[d] is never read: it counts as 0 and sets MOE_DEVERR_ABORTED in
+ * *err_word (device uint32, may be NULL). */
 typedef struct moe_ep_sources_t {
-    const void *local_out[MOE_EP_MAX_RANKS]; /* rank d: bf16 [N_recv_d, H], 16-byte aligned */
-    int64_t row_off[MOE_EP_MAX_RANKS];       /* first row of this source's block on rank d  */
+    const void *local_out[MOE_EP_MAX_RANKS]; /* rank d: bf16 [rows_d, H], 16-byte aligned */
+    int64_t row_off[MOE_EP_MAX_RANKS];       /* first row of this source's block on rank d */
+    int64_t rows[MOE_EP_MAX_RANKS];          /* rows rank d's local_out holds              */
+    uint32_t *err_word;                      /* this rank's device error word, or NULL     */
 } moe_ep_sources_t;
 
 /*

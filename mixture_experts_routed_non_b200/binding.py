@@ -111,13 +111,17 @@ class MoeEpPeers(ctypes.Structure):
     _fields_ = [("recv_x", ctypes.c_void_p * EP_MAX_RANKS),
                 ("recv_idx", ctypes.c_void_p * EP_MAX_RANKS),
                 ("recv_w", ctypes.c_void_p * EP_MAX_RANKS),
-                ("row_off", ctypes.c_int64 * EP_MAX_RANKS)]
+                ("row_off", ctypes.c_int64 * EP_MAX_RANKS),
+                ("recv_rows", ctypes.c_int64 * EP_MAX_RANKS),
+                ("err_word", ctypes.c_void_p)]
 
 
 class MoeEpSources(ctypes.Structure):
     """moe_ep_sources_t: every rank's local_out as seen from the caller."""
     _fields_ = [("local_out", ctypes.c_void_p * EP_MAX_RANKS),
-                ("row_off", ctypes.c_int64 * EP_MAX_RANKS)]
+                ("row_off", ctypes.c_int64 * EP_MAX_RANKS),
+                ("rows", ctypes.c_int64 * EP_MAX_RANKS),
+                ("err_word", ctypes.c_void_p)]
 
 
 def load() -> ctypes.CDLL:
@@ -579,29 +583,48 @@ def ep_layout(topk_idx: torch.Tensor, R: int, E_local: int, send_idx: Optional[t
     return send_idx, send_count
 
 
-def ep_peers(recv_x, recv_idx, recv_w, row_off) -> MoeEpPeers:
-    """A moe_ep_peers_t from per-rank buffer addresses (ints or tensors) and the
-    caller's block offsets on every rank."""
+def _rows_of(bufs, rows, what):
+    if rows is not None:
+        return [int(r) for r in rows]
+    if all(isinstance(b, torch.Tensor) for b in bufs):
+        return [int(b.shape[0]) for b in bufs]
+    raise ValueError(f"{what}: give the row counts when the buffers are raw addresses")
+
+
+def ep_peers(recv_x, recv_idx, recv_w, row_off, recv_rows=None, err: Optional[torch.Tensor] = None) -> MoeEpPeers:
+    """A moe_ep_peers_t from per-rank buffers (tensors, or raw addresses with
+    ``recv_rows``) and the caller's block offsets on every rank.  The dispatch
+    writes no row at or past a rank's row count (it flags the error in
+    ``err`` instead)."""
     R = len(recv_x)
     if not (1 <= R <= EP_MAX_RANKS) or not (len(recv_idx) == len(recv_w) == len(row_off) == R):
         raise ValueError("ep_peers: one entry per rank, 1..32 ranks")
+    rows = _rows_of(recv_x, recv_rows, "ep_peers")
     p = MoeEpPeers()
     addr = lambda v: v.data_ptr() if isinstance(v, torch.Tensor) else int(v)
     for d in range(R):
         p.recv_x[d], p.recv_idx[d], p.recv_w[d] = addr(recv_x[d]), addr(recv_idx[d]), addr(recv_w[d])
         p.row_off[d] = int(row_off[d])
+        p.recv_rows[d] = rows[d]
+    p.err_word = _ptr(err)
     return p
 
 
-def ep_sources(local_out, row_off) -> MoeEpSources:
+def ep_sources(local_out, row_off, rows=None, err: Optional[torch.Tensor] = None) -> MoeEpSources:
+    """A moe_ep_sources_t from per-rank local outputs (tensors, or raw
+    addresses with ``rows``); the combine reads no row at or past a rank's
+    row count (it counts 0 and flags the error in ``err``)."""
     R = len(local_out)
     if not (1 <= R <= EP_MAX_RANKS) or len(row_off) != R:
         raise ValueError("ep_sources: one entry per rank, 1..32 ranks")
+    nrows = _rows_of(local_out, rows, "ep_sources")
     src = MoeEpSources()
     for d in range(R):
         v = local_out[d]
         src.local_out[d] = v.data_ptr() if isinstance(v, torch.Tensor) else int(v)
         src.row_off[d] = int(row_off[d])
+        src.rows[d] = nrows[d]
+    src.err_word = _ptr(err)
     return src
 
 

@@ -878,8 +878,10 @@ extern "C" MOE_API int moe_ep_dispatch(const void *x, const int32_t *topk_idx, c
     if ((int64_t)R * E_local >= ((int64_t)1 << 31) || T * (int64_t)R >= ((int64_t)1 << 31)) return MOE_ERR_ARG;
     if (T > 0 && (!x || !topk_idx || !topk_w || !send_idx)) return MOE_ERR_ARG;
     if (!aligned(x, 16) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) || !aligned(send_idx, 4)) return MOE_ERR_ARG;
+    if (!aligned(peers->err_word, 4)) return MOE_ERR_ARG;
     for (int d = 0; d < R; ++d) {
-        if (!peers->recv_x[d] || !peers->recv_idx[d] || !peers->recv_w[d] || peers->row_off[d] < 0)
+        if (!peers->recv_x[d] || !peers->recv_idx[d] || !peers->recv_w[d] || peers->row_off[d] < 0 ||
+            peers->recv_rows[d] < 0)
             return MOE_ERR_ARG;
         if (!aligned(peers->recv_x[d], 16) || !aligned(peers->recv_idx[d], 4) || !aligned(peers->recv_w[d], 4))
             return MOE_ERR_ARG;
@@ -900,7 +902,9 @@ extern "C" MOE_API int moe_ep_combine(const moe_ep_sources_t *src, const int32_t
     if (T > 0 && (!send_idx || !out)) return MOE_ERR_ARG;
     if (!aligned(send_idx, 4) || !aligned(out, 16)) return MOE_ERR_ARG;
     for (int d = 0; d < R; ++d)
-        if (!src->local_out[d] || !aligned(src->local_out[d], 16) || src->row_off[d] < 0) return MOE_ERR_ARG;
+        if (!src->local_out[d] || !aligned(src->local_out[d], 16) || src->row_off[d] < 0 || src->rows[d] < 0)
+            return MOE_ERR_ARG;
+    if (!aligned(src->err_word, 4)) return MOE_ERR_ARG;
     DeviceInfo dev;
     const int st = device_info(&dev);
     if (st) return st;

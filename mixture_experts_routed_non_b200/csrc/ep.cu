@@ -112,7 +112,12 @@ __global__ void __launch_bounds__(kEpThreads) ep_dispatch_kernel(const uint4 *__
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         if (threadIdx.x < R) {
             const int j = __ldg(send_idx + t * R + threadIdx.x);
-            row[threadIdx.x] = j >= 0 ? peers.row_off[threadIdx.x] + j : -1;
+            int64_t r = j >= 0 ? peers.row_off[threadIdx.x] + j : -1;
+            if (r >= peers.recv_rows[threadIdx.x]) {  // past the destination's buffer: not written
+                if (peers.err_word) atomicOr(peers.err_word, MOE_DEVERR_ABORTED);
+                r = -1;
+            }
+            row[threadIdx.x] = r;
         }
         __syncthreads();
         const uint4 *src = x + t * chunks;
@@ -146,7 +151,11 @@ __global__ void __launch_bounds__(kEpThreads) ep_combine_kernel(const moe_ep_sou
     for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
         if (threadIdx.x < 32) {
             const int lane = threadIdx.x;
-            const int j = lane < R ? __ldg(send_idx + t * R + lane) : -1;
+            int j = lane < R ? __ldg(send_idx + t * R + lane) : -1;
+            if (j >= 0 && src.row_off[lane] + j >= src.rows[lane]) {  // past the buffer: not read
+                if (src.err_word) atomicOr(src.err_word, MOE_DEVERR_ABORTED);
+                j = -1;
+            }
             const unsigned b = __ballot_sync(0xffffffffu, j >= 0);
             if (j >= 0)
                 vrow[__popc(b & ((1u << lane) - 1u))] =

@@ -228,7 +228,7 @@ def test_argument_errors():
     with pytest.raises(binding.MoeError):
         binding.ep_layout(idxs[0], 33, E_local)  # more ranks than the tables hold
     send_idx, _ = binding.ep_layout(idxs[0], R, E_local)
-    bad = binding.ep_peers([0, 0], [0, 0], [0, 0], [0, 0])
+    bad = binding.ep_peers([0, 0], [0, 0], [0, 0], [0, 0], recv_rows=[1, 1])
     with pytest.raises(binding.MoeError):
         binding.ep_dispatch(xs[0], idxs[0], ws[0], send_idx, E_local, bad, R)
     assert block_offsets(np.array([[1, 2], [3, 4]]))[0].tolist() == [[0, 1], [0, 2]]
@@ -303,3 +303,45 @@ def test_duplicate_experts_and_all_slots_on_one_rank():
         mag = oep.ep_combine([np.abs(p) for p in part], d["send_idx"], d["off"])[0]
         assert_close_ep(to_np(outs[s]), fwd, mag, f"rank {s}")
         assert (to_np(outs[s])[2] == 0).all()
+
+
+def test_rows_past_a_buffer_are_neither_written_nor_read():
+    """A destination buffer smaller than its rows: the dispatch skips the rows
+    past it and flags MOE_DEVERR_ABORTED; the combine reads no row past a
+    local_out's row count, counts it 0 and flags the same bit."""
+    R, E_local, T, K, H = 2, 2, 64, 2, 64
+    xs, idxs, ws = _problem(R, E_local, T, K, H, seed=12, p_invalid=0.0)
+    ref = _oracle_dispatch(xs, idxs, ws, R, E_local)
+    n0 = int(ref["n_recv"][0])
+    cap = n0 - 5
+    pad = 16  # guard rows after the declared capacity, checked untouched
+    rx = [torch.full((cap + pad, H), 7.0, device="cuda").to(torch.bfloat16),
+          torch.empty((int(ref["n_recv"][1]), H), dtype=torch.bfloat16, device="cuda")]
+    ri = [torch.full((cap + pad, K), 99, dtype=torch.int32, device="cuda"),
+          torch.empty((int(ref["n_recv"][1]), K), dtype=torch.int32, device="cuda")]
+    rw = [torch.full((cap + pad, K), 9.0, device="cuda"),
+          torch.empty((int(ref["n_recv"][1]), K), device="cuda")]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for s in range(R):
+        send_idx, _ = binding.ep_layout(idxs[s], R, E_local)
+        peers = binding.ep_peers(rx, ri, rw, ref["off"][:, s], recv_rows=[cap, int(ref["n_recv"][1])], err=err)
+        binding.ep_dispatch(xs[s], idxs[s], ws[s], send_idx, E_local, peers, R)
+    torch.cuda.synchronize()
+    assert int(err.item()) & 0x8
+    assert np.array_equal(rx[0][:cap].view(torch.int16).cpu().numpy(), ref["recv_x"][0][:cap])
+    assert np.array_equal(ri[0][:cap].cpu().numpy(), ref["recv_idx"][0][:cap])
+    assert (rx[0][cap:].float() == 7.0).all() and (ri[0][cap:] == 99).all() and (rw[0][cap:] == 9.0).all()
+    # combine of the last source (its block ends rank 0's rows) reading a local_out that
+    # holds fewer rows than that block needs
+    local = [torch.randn((int(n), H), device="cuda").to(torch.bfloat16) for n in ref["n_recv"]]
+    err.zero_()
+    last = R - 1
+    send_idx_l, _ = binding.ep_layout(idxs[last], R, E_local)
+    out = binding.ep_combine(binding.ep_sources(local, ref["off"][:, last], rows=[cap, int(ref["n_recv"][1])],
+                                                err=err), send_idx_l, H)
+    torch.cuda.synchronize()
+    assert int(err.item()) & 0x8
+    short = [np.where(np.arange(int(n))[:, None] < (cap if d == 0 else int(n)), to_np(l), 0.0)
+             for d, (n, l) in enumerate(zip(ref["n_recv"], local))]
+    exp = oep.ep_combine(short, ref["send_idx"], ref["off"])[last]
+    assert_close(to_np(out), exp, "combine with a short local_out")
