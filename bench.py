@@ -252,6 +252,46 @@ def metadata_only(dev, peaks, reps: int = 50):
             "launches": 1, "l2": "flushed before every rep"}
 
 
+def metadata_pairs_only(dev, peaks, reps: int = 50):
+    """moe_nonexpand_routed_metadata on the metadata workload given as the
+    compact pair list (token / expert / score per pair, tokens ascending),
+    with int32 and with int64 ids; L2 flushed before every rep, median device
+    time.  The pair-list read replaces the table's N*K slots by P pairs."""
+    import numpy as np
+    import torch
+
+    from mixture_experts_routed_non_b200 import binding, synthetic
+    wl = synthetic.WORKLOADS["metadata"]
+    idx, w = synthetic.make_routing(wl)
+    tok, exp, wt = synthetic.pair_list_from_table(idx, w)
+    P = int(tok.shape[0])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    res = {"workload": "metadata (pair list)", "N": wl.N, "E": wl.E, "P": P, "l2": "flushed before every rep"}
+    for bits, dt in ((32, torch.int32), (64, torch.int64)):
+        t_ = torch.from_numpy(tok).to(dt).to(dev)
+        e_ = torch.from_numpy(exp).to(dt).to(dev)
+        w_ = torch.from_numpy(wt).to(dev)
+        r = binding.routing(e_, w_, token_idx=t_, N=wl.N)
+        meta = binding.alloc_routed_meta(r, wl.E, dev)
+        ws = torch.empty(binding.routed_workspace_bytes(r, 0, 0, wl.E), dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            binding.routed_metadata(e_, w_, wl.E, token_idx=t_, N=wl.N, meta=meta, ws=ws)
+        times = []
+        for _ in range(reps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            binding.routed_metadata(e_, w_, wl.E, token_idx=t_, N=wl.N, meta=meta, ws=ws)
+            b.record()
+            b.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = float(np.median(times))
+        nbytes = P * (2 * (bits // 8) + 4) + 4 * P * 4 + 4 * (wl.N + 1) + 8 * wl.E
+        res[f"int{bits}"] = {"ms": ms, "algorithmic_bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9}
+    return res
+
+
 def router_only(dev, peaks, reps: int = 10, ring: int = 20):
     """moe_router_topk alone on the prefill sizes (N=16384, E=128, K=8, fp32
     logits, top-k of the softmax renormalised).  A ring of ``ring`` logits
@@ -640,6 +680,7 @@ def run_ours(args, rank, world, local):
     clocks = sampler.summary(t_wall0, t_wall1)
 
     meta_c2 = metadata_only(dev, peaks) if rank == 0 else None
+    meta_pairs = metadata_pairs_only(dev, peaks) if rank == 0 else None
     router = router_only(dev, peaks) if rank == 0 else None
     train = backward_leg(inp, w1, b1, args.layout, dev, peaks) if rank == 0 else None
     ep = ep_emulated(dev, peaks) if rank == 0 else None
@@ -691,6 +732,7 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "pipelining": "copy-in / compute / copy-out streams, 3 buffer sets, inputs packed in one copy"},
         "metadata_only": meta_c2,
+        "metadata_pairs_only": meta_pairs,
         "router_only": router,
         "training": train,
         "ep_emulated": ep,
