@@ -213,7 +213,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=6.0,
-                    help="oracle work per step of --impl reference (sets its token sample)")
+                    help="at most this much oracle work per step of --impl reference (sets its token sample)")
+    ap.add_argument("--ref-budget", type=float, default=150.0,
+                    help="oracle work of the whole --impl reference run, spread over its warm-up and timed steps")
     return ap.parse_args()
 
 
@@ -495,12 +497,14 @@ def run_reference(args, rank, world):
     idx = inp.topk_idx.numpy()
     w = inp.topk_w.numpy()
     threads = len(os.sched_getaffinity(0))
-    # sample size per step: about --ref-seconds of oracle work
+    # sample size per step: about --ref-seconds of oracle work, less when the whole run
+    # (warm-up and timed steps) would exceed --ref-budget
+    per_step_s = min(args.ref_seconds, args.ref_budget / max(1, args.warmup + args.steps))
     probe = np.arange(min(wl.N, 4))
     t0 = time.perf_counter()
     oracle.forward_rows(wts, idx, w, tokens=probe, layout=args.layout, n_threads=threads)
     per_tok = (time.perf_counter() - t0) / len(probe)
-    n = int(max(1, min(wl.N, args.ref_seconds / max(per_tok, 1e-6))))
+    n = int(max(1, min(wl.N, per_step_s / max(per_tok, 1e-6))))
     rng = np.random.default_rng(7)
     times = []
     for step in range(args.warmup + args.steps):
