@@ -34,10 +34,13 @@
 // CTA); warps 2-5 = epilogue (TMEM lane quarter warp%4); warps 6-9 (up only)
 // = A-row gather.  The even CTA's gather threads arrive with cp.async straight
 // on the stage barrier, so the MMA thread checks a single barrier per stage:
-// its per-stage work is on the tensor pipe's critical path.  Six shared-memory stages; two TMEM accumulators so the
-// epilogue of one tile overlaps the MMAs of the next.  Rows past the end of an
-// expert's segment are computed (clamped gather / neighbouring rows) but never
-// stored.
+// its per-stage work is on the tensor pipe's critical path.  Three
+// shared-memory stages of 128 K (64 KB per CTA); two TMEM accumulators so the
+// epilogue of one tile overlaps the MMAs of the next.  A segment's last tile
+// with at most 128 rows runs the pair MMA at M=128 (64 rows per CTA).  Rows
+// past the end of an expert's segment are computed (stale stage rows) but
+// never stored.  In training the up GEMM also writes z (fp32), staged through
+// the epilogue warp's store buffer and written in whole 128-byte rows.
 //
 // Every wait is bounded (common.cuh); on a timeout a CTA raises its abort
 // flag, records MOE_DEVERR_TIMEOUT, drains what it has in flight and returns
