@@ -732,14 +732,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                             break;
                         }
                         const int rv = t.kp1 - kbase;  // rows of the segment in this stage
-                        const int nz = kSK - rv;
                         const int atoms = (a.a_tma ? 2 : 0) + (a.b_tma ? 2 : 0);
-                        for (int i = pt; i < nz * atoms * 8; i += kProducerThreads) {
-                            const int chunk = i & 7, rest = i >> 3;
-                            const int row = rv + rest % nz, at = rest / nz;
+                        // 16 rows of 8 chunks per pass of the 128 threads; whole 128-byte rows
+                        // are zeroed, so the swizzle does not matter
+                        const int zc = pt & 7, zr = pt >> 3;
+                        for (int at = 0; at < atoms; ++at) {
                             const uint32_t base_at = (a.a_tma && at < 2) ? sa + at * kMnAtom
                                                                          : sb + (at - (a.a_tma ? 2 : 0)) * kMnAtom;
-                            st_shared_v4(base_at + row * 128 + chunk * 16, 0u, 0u, 0u, 0u);
+                            for (int row = rv + zr; row < kSK; row += kProducerThreads / 8)
+                                st_shared_v4(base_at + row * 128 + zc * 16, 0u, 0u, 0u, 0u);
                         }
                         fence_proxy_async_smem();  // the zeros are read by the tensor cores
                     }
