@@ -129,7 +129,10 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(const __nv_bfloat16 *__r
     reinterpret_cast<uint32_t *>(db + (size_t)e * cols)[c2] = pack_bf16x2(s0, s1);
 }
 
-// dst[p, :] = src[idx[p], :] for p < P = expert_off[E] (16-byte chunks).
+// dst[p, :] = src[idx[p], :] for p < P = expert_off[E] (16-byte chunks): four
+// rows per block iteration (grid-stride over rows, their loads in flight
+// together), the block's threads over the chunks, so no per-chunk division
+// is needed.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16 *__restrict__ src,
                                                           const int32_t *__restrict__ idx,
                                                           const int32_t *__restrict__ p_total, int32_t cols,
@@ -137,13 +140,20 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16 *_
     if (hdr && *(volatile const uint32_t *)&hdr->abort) return;
     const int P = __ldg(p_total);
     const int chunks = cols >> 3;
-    const int64_t total = (int64_t)P * chunks;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t p = i / chunks;
-        const int c = (int)(i - p * chunks);
-        const int row = __ldg(idx + p);
-        reinterpret_cast<uint4 *>(dst + (size_t)p * cols)[c] =
-            __ldg(reinterpret_cast<const uint4 *>(src + (size_t)row * cols) + c);
+    constexpr int kRows = 4;  // rows in flight per block iteration
+    for (int p0 = blockIdx.x * kRows; p0 < P; p0 += gridDim.x * kRows) {
+        const uint4 *s[kRows];
+#pragma unroll
+        for (int u = 0; u < kRows; ++u)
+            s[u] = reinterpret_cast<const uint4 *>(src + (size_t)__ldg(idx + min(p0 + u, P - 1)) * cols);
+        for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+            uint4 v[kRows];
+#pragma unroll
+            for (int u = 0; u < kRows; ++u) v[u] = __ldg(s[u] + c);
+#pragma unroll
+            for (int u = 0; u < kRows; ++u)
+                if (p0 + u < P) reinterpret_cast<uint4 *>(dst + (size_t)(p0 + u) * cols)[c] = v[u];
+        }
     }
 }
 
