@@ -1,0 +1,56 @@
+"""Host-side pieces of bench.py and the expert-parallel host module, on CPU:
+the DRAM-traffic record is used only while the kernel sources hash to it,
+the roofline arithmetic, and the receive-block offsets against the oracle's."""
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from mixture_experts_routed_non_b200.ep import block_offsets  # noqa: E402
+from oracle import ep as oep  # noqa: E402
+
+
+def test_traffic_record_matches_current_sources():
+    up = bench.traffic_record("gemm_up", "prefill")
+    down = bench.traffic_record("gemm_down", "prefill")
+    assert up is not None and down is not None  # recorded for the sources as they are
+    assert up > 1e9 and down > 1e9
+    assert bench.traffic_record("gemm_up", "no-such-workload") is None
+
+
+def test_traffic_record_rejects_changed_sources(tmp_path, monkeypatch):
+    # a copy of the tree whose kernel source differs by one byte has no record
+    import shutil
+    root = tmp_path / "repo"
+    (root / "profiles").mkdir(parents=True)
+    shutil.copy(os.path.join(ROOT, "profiles", "ncu_traffic.txt"), root / "profiles")
+    csrc = root / "mixture_experts_routed_non_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for f in ("grouped_gemm_sm100.cu", "common.cuh"):
+        shutil.copy(os.path.join(ROOT, "mixture_experts_routed_non_b200", "csrc", f), csrc / f)
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.traffic_record("gemm_up", "prefill") is not None
+    with open(csrc / "common.cuh", "a") as fh:
+        fh.write("\n")
+    assert bench.traffic_record("gemm_up", "prefill") is None
+
+
+def test_gemm_flops_and_peaks():
+    up, down = bench.gemm_flops(131072, 2048, 768)
+    assert up == 4 * 131072 * 2048 * 768 and down == 2 * 131072 * 2048 * 768
+    peaks, src = bench.load_peaks()
+    assert src in ("measured", "fallback")
+    assert peaks["hbm_gbs"] > 1000 and peaks["bf16_tflops_sustained"] > 100
+
+
+def test_block_offsets_match_the_oracle():
+    rng = np.random.default_rng(0)
+    for R in (1, 2, 5, 8, 32):
+        counts = rng.integers(0, 50, size=(R, R))
+        off, n = block_offsets(counts)
+        ref_off, ref_n = oep.recv_offsets(counts)
+        assert np.array_equal(off, ref_off) and np.array_equal(n, ref_n)
