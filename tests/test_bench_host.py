@@ -1,6 +1,7 @@
 """Host-side pieces of bench.py and the expert-parallel host module, on CPU:
-the DRAM-traffic record is used only while the kernel sources hash to it,
-the roofline arithmetic, and the receive-block offsets against the oracle's."""
+the DRAM-traffic record file, its use only while the kernel sources hash to
+it (checked on a copy of the sources), the roofline arithmetic, and the
+receive-block offsets against the oracle's."""
 import os
 import sys
 
@@ -14,11 +15,19 @@ from mixture_experts_routed_non_b200.ep import block_offsets  # noqa: E402
 from oracle import ep as oep  # noqa: E402
 
 
-def test_traffic_record_matches_current_sources():
-    up = bench.traffic_record("gemm_up", "prefill")
-    down = bench.traffic_record("gemm_down", "prefill")
-    assert up is not None and down is not None  # recorded for the sources as they are
-    assert up > 1e9 and down > 1e9
+def test_traffic_record_file_parses():
+    """Every record names a kernel, a workload, a 16-hex-digit source hash and
+    read + write = per-launch bytes."""
+    n = 0
+    for line in open(os.path.join(ROOT, "profiles", "ncu_traffic.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        kv = dict(p.split("=", 1) for p in line.split())
+        assert kv["kernel"] in ("gemm_up", "gemm_down") and kv["workload"]
+        assert len(kv["sources"]) == 16 and int(kv["sources"], 16) >= 0
+        assert int(kv["read"]) + int(kv["write"]) == int(kv["dram_bytes_per_launch"])
+        n += 1
+    assert n >= 2
     assert bench.traffic_record("gemm_up", "no-such-workload") is None
 
 
