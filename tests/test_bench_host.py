@@ -32,17 +32,23 @@ def test_traffic_record_file_parses():
 
 
 def test_traffic_record_rejects_changed_sources(tmp_path, monkeypatch):
-    # a copy of the tree whose kernel source differs by one byte has no record
+    """A record is used only while the kernel sources hash to it: a copy of the
+    sources with a record written for them finds it; one byte more, and not."""
+    import hashlib
     import shutil
     root = tmp_path / "repo"
     (root / "profiles").mkdir(parents=True)
-    shutil.copy(os.path.join(ROOT, "profiles", "ncu_traffic.txt"), root / "profiles")
     csrc = root / "mixture_experts_routed_non_b200" / "csrc"
     csrc.mkdir(parents=True)
+    h = hashlib.sha256()
     for f in ("grouped_gemm_sm100.cu", "common.cuh"):
         shutil.copy(os.path.join(ROOT, "mixture_experts_routed_non_b200", "csrc", f), csrc / f)
+        h.update(open(csrc / f, "rb").read())
+    with open(root / "profiles" / "ncu_traffic.txt", "w") as fh:
+        fh.write(f"kernel=gemm_up workload=prefill sources={h.hexdigest()[:16]} "
+                 f"dram_bytes_per_launch=300 read=200 write=100\n")
     monkeypatch.setattr(bench, "ROOT", str(root))
-    assert bench.traffic_record("gemm_up", "prefill") is not None
+    assert bench.traffic_record("gemm_up", "prefill") == 300.0
     with open(csrc / "common.cuh", "a") as fh:
         fh.write("\n")
     assert bench.traffic_record("gemm_up", "prefill") is None
