@@ -17,12 +17,14 @@
 //   phase B  every CTA reads the whole (small) [T,E] histogram table and
 //            derives the global offsets, its tile's base per expert and its
 //            pair base; its warps' bases follow from the per-warp counts of
-//            phase A; then each warp ranks its slice (popc(peers & lanes
-//            below) inside each 32-slot step) and writes the outputs.  CTA 0
+//            phase A; then each warp ranks its slice (match_any finds the
+//            lanes with the same expert, popc(peers & lanes below) orders
+//            them inside each 32-slot step) and writes the outputs.  CTA 0
 //            also writes the histogram, offsets, the GEMM tile table and the
 //            call's error word.
 //
-// Every result is a pure function of the input (no atomic decides an order),
+// Every result is a pure function of the input (no atomic decides an order;
+// the grid barrier is a GPU-scope release add polled with acquire loads),
 // so the output is bit-exact and deterministic.  Each lane keeps kV slots in
 // flight; the first kWarpChunk slots of every warp, and their weights, stay in
 // registers from phase A to phase B.
@@ -36,6 +38,20 @@ constexpr unsigned kFull = 0xffffffffu;
 constexpr int kV = 8;                     // slots per lane per step
 constexpr int kWarpChunk = 32 * kV;       // slots per warp step
 constexpr unsigned long long kGridBarrierTimeoutNs = 1000000000ull;
+static_assert(kMetaMaxTiles < kMetaThreads, "phase B reads one tile's counts per thread");
+
+// The grid barrier's arrival: a GPU-scope release add (the block's earlier
+// writes, ordered before it by __syncthreads, become visible with it) and an
+// acquire load for the polling.
+__device__ __forceinline__ void red_add_release_gpu(uint32_t *p, uint32_t v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 
 // Exclusive scan of n ints in shared memory (in place allowed) by the whole
 // block; returns the total.
@@ -162,10 +178,12 @@ __global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a)
     const int w0 = s0 + warp * sub;
     const int w1 = min(w0 + sub, s1);
     int ev0[kV], tv0[kV];
+    float wv0[kV];  // kept for phase B; an invalid slot's weight is never written
     load_chunk<kIdx64>(a.topk_idx, w0, w1, lane, ev0);
 #pragma unroll
     for (int v = 0; v < kV; ++v) {
         const int s = w0 + 32 * v + lane;
+        wv0[v] = s < w1 ? __ldg(a.topk_w + s) : 0.f;
         tv0[v] = (kPairs && s < w1) ? slot_token<kPairs, kIdx64>(a, s) : 0;
     }
     for (int i = threadIdx.x; i < kMetaWarps * E; i += kMetaThreads) cnt[i] = 0;
@@ -208,15 +226,6 @@ __global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a)
             __syncwarp();
         }
     }
-    // weights of the first chunk's valid slots, kept for phase B (invalid
-    // slots' weights are never read)
-    float wv0[kV];
-#pragma unroll
-    for (int v = 0; v < kV; ++v) {
-        unsigned ignore = 0;
-        const bool valid = slot_valid<kPairs>(a, ev0[v], tv0[v], &ignore);
-        wv0[v] = valid ? __ldg(a.topk_w + w0 + 32 * v + lane) : 0.f;
-    }
     if (lane == 0) wq[warp] = nvalid;
     if (my_err) atomicOr(&s_err, my_err);
     __syncthreads();
@@ -235,20 +244,18 @@ __global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a)
     }
 
     // ---- grid barrier (bounded)
-    __threadfence();
     __syncthreads();
     if (threadIdx.x == 0) {
-        atomicAdd(&a.hdr->grid_arrive, 1u);
+        red_add_release_gpu(&a.hdr->grid_arrive, 1u);
         const uint64_t t0 = globaltimer_ns();
         int ok = 1;
-        while (*(volatile uint32_t *)&a.hdr->grid_arrive < (uint32_t)T) {
+        while (ld_acquire_gpu(&a.hdr->grid_arrive) < (uint32_t)T) {
             if (globaltimer_ns() - t0 > kGridBarrierTimeoutNs) {
                 ok = 0;
                 break;
             }
         }
         s_bar_ok = ok;
-        __threadfence();
     }
     __syncthreads();
     if (!s_bar_ok) {
@@ -259,7 +266,12 @@ __global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a)
         return;
     }
 
-    // ---- phase B.1: global column sums and this tile's column prefix
+    // ---- phase B.1: global column sums and this tile's column prefix.  T is at
+    // most kMetaMaxTiles < kMetaThreads, so one thread reads each tile's valid
+    // count and error bits; they are issued before the histogram table loads.
+    const int tq = threadIdx.x;
+    const int tv_before = (tq < T && tq < tile) ? __ldcg(a.tile_valid + tq) : 0;
+    const unsigned terr = (tile == 0 && tq < T) ? (unsigned)__ldcg(a.tile_err + tq) : 0u;
     int G = E <= kMetaThreads ? kMetaThreads / E : 1;
     if (G > T) G = T;
     for (int i = threadIdx.x; i < G * E; i += kMetaThreads) {
@@ -280,12 +292,6 @@ __global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a)
         }
         part_all[i] = all;
         part_before[i] = before;
-    }
-    int tv_before = 0;
-    unsigned terr = 0;
-    for (int t = threadIdx.x; t < T; t += kMetaThreads) {
-        if (t < tile) tv_before += __ldcg(a.tile_valid + t);
-        if (tile == 0) terr |= (unsigned)__ldcg(a.tile_err + t);
     }
     if (threadIdx.x == 0) s_err = 0;
     __syncthreads();
@@ -369,10 +375,8 @@ __global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a)
 #pragma unroll
             for (int v = 0; v < kV; ++v) {
                 const int s = base + 32 * v + lane;
+                wv[v] = s < w1 ? __ldg(a.topk_w + s) : 0.f;
                 tv[v] = (kPairs && s < w1) ? slot_token<kPairs, kIdx64>(a, s) : 0;
-                unsigned ignore = 0;
-                const bool valid = slot_valid<kPairs>(a, ev[v], tv[v], &ignore);
-                wv[v] = valid ? __ldg(a.topk_w + s) : 0.f;
             }
         }
 #pragma unroll
