@@ -9,9 +9,9 @@
 // kernel over T tiles of consecutive slots (T <= number of SMs, one CTA each):
 //
 //   phase A  each warp of a tile owns a contiguous slice of its slots and
-//            counts the experts in it (match_any aggregation, per-warp rows
-//            in shared memory, no atomics); the tile's histogram, valid count
-//            and error bits go to the workspace.
+//            counts the experts in it (shared-memory increments into a row of
+//            its own: integer counts, so their order does not matter); the
+//            tile's histogram, valid count and error bits go to the workspace.
 //   barrier  all T CTAs (co-resident by the cooperative launch) meet at a
 //            bounded grid barrier whose counter the host clears per call.
 //   phase B  every CTA reads the whole (small) [T,E] histogram table and
@@ -220,12 +220,13 @@ __global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a)
                     load_id_wide<kIdx64>(a.token_idx, s - 1) > load_id_wide<kIdx64>(a.token_idx, s))
                     my_err |= MOE_DEVERR_BAD_TOKEN;
             }
-            const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
-            if (valid && lane == __ffs(peers) - 1) mycnt[e] += __popc(peers);
-            nvalid += __popc(__ballot_sync(kFull, valid));
-            __syncwarp();
+            if (valid) {  // integer counts: the order of the atomics does not matter
+                atomicAdd(&mycnt[e], 1);
+                ++nvalid;
+            }
         }
     }
+    nvalid = (int)__reduce_add_sync(kFull, (unsigned)nvalid);
     if (lane == 0) wq[warp] = nvalid;
     if (my_err) atomicOr(&s_err, my_err);
     __syncthreads();
