@@ -123,7 +123,8 @@ MOE_API size_t moe_nonexpand_workspace_bytes(int64_t N, int32_t H, int32_t I, in
  * histogram, exclusive offsets, stable counting sort of the pairs by expert,
  * per-token pair offsets and compact scores.  Results are bit-exact and
  * deterministic.  `meta` (host struct of device pointers) must be non-null
- * with every field set.  Invalid slots' weights are never read.
+ * with every field set.  Invalid slots' weights are loaded with their ids
+ * but never used: any value, NaN included, leaves every result unchanged.
  */
 MOE_API int moe_nonexpand_metadata(const int32_t *topk_idx, const float *topk_w,
                            int64_t N, int32_t K, int32_t E, int64_t total_pairs,

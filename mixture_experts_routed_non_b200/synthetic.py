@@ -152,7 +152,7 @@ def routing(wl: Workload, rng: np.random.Generator) -> np.ndarray:
 def scores(wl: Workload, idx: np.ndarray, rng: np.random.Generator,
            invalid_value: float = 0.0) -> np.ndarray:
     """Router scores [N,K] fp32.  Invalid slots get ``invalid_value`` (tests
-    pass NaN to prove they are never read)."""
+    pass NaN to prove their values are never used)."""
     valid = idx >= 0
     if wl.scores == "softmax":
         logits = rng.standard_normal(idx.shape)
