@@ -276,3 +276,83 @@ def test_ep_combine_argument_checks(lib):
     assert _ep_combine(lib, rows=(3, -1)) == binding.MOE_ERR_ARG
     if _no_device():
         assert _ep_combine(lib) in NO_DEVICE
+
+
+# ---------------------------------------------------------------------------
+# training pair
+# ---------------------------------------------------------------------------
+def test_train_workspace_bytes(lib):
+    n = lib.moe_nonexpand_train_workspace_bytes(64, 128, 128, 8, 4, -1)
+    assert n > lib.moe_nonexpand_workspace_bytes(64, 128, 128, 8, 4, -1) > 0
+    assert lib.moe_nonexpand_train_workspace_bytes(64, 0, 128, 8, 4, -1) == 0     # H needed
+    assert lib.moe_nonexpand_train_workspace_bytes(64, 128, 96, 8, 4, -1) == 0    # I % 64
+    assert lib.moe_nonexpand_train_workspace_bytes(64, 128, 128, 8, 0, -1) == 0
+    r = _routing()
+    assert lib.moe_nonexpand_routed_train_workspace_bytes(ctypes.byref(r), 128, 128, 8) == n
+    bad = _routing(kind=7)
+    assert lib.moe_nonexpand_routed_train_workspace_bytes(ctypes.byref(bad), 128, 128, 8) == 0
+
+
+def _fwd_train(lib, x=A, idx=A, w=A, N=64, H=128, I=128, E=8, K=4, tp=-1, w1=A, b1=None, w2=A, b2=None,
+               act=binding.ACT_SWIGLU, lay=binding.LAYOUT_INTERLEAVED, out=A, ws=A, wsb=1 << 30):
+    return lib.moe_nonexpand_forward_train(x, idx, w, N, H, I, E, K, tp, w1, b1, w2, b2, act, lay, out, ws, wsb,
+                                           None)
+
+
+def test_forward_train_argument_checks(lib):
+    total = lib.moe_nonexpand_workspace_bytes(64, 128, 128, 8, 4, -1)
+    assert _fwd_train(lib, K=0) == binding.MOE_ERR_ARG
+    assert _fwd_train(lib, idx=A2) == binding.MOE_ERR_ARG
+    assert _fwd_train(lib, x=None) == binding.MOE_ERR_ARG
+    assert _fwd_train(lib, w2=None) == binding.MOE_ERR_ARG
+    assert _fwd_train(lib, act=3) == binding.MOE_ERR_ARG
+    assert _fwd_train(lib, lay=5) == binding.MOE_ERR_ARG
+    assert _fwd_train(lib, b1=A8) == binding.MOE_ERR_ARG
+    assert _fwd_train(lib, H=100) == binding.MOE_ERR_SHAPE
+    assert _fwd_train(lib, wsb=total) == binding.MOE_ERR_WS     # the inference size is too small
+    if _no_device():
+        assert _fwd_train(lib) in NO_DEVICE
+
+
+def _bwd(lib, fn="moe_nonexpand_backward", dout=A, x=A, idx=A, w=A, N=64, H=128, I=128, E=8, K=4, tp=-1,
+         w1=A, w2=A, act=binding.ACT_SWIGLU, lay=binding.LAYOUT_INTERLEAVED, dx=A, dw1=A, db1=None, dw2=A,
+         db2=None, dw=A, ws=A, wsb=1 << 30, events="none"):
+    args = [dout, x, idx, w, N, H, I, E, K, tp, w1, w2, act, lay, dx, dw1, db1, dw2, db2, dw, ws, wsb, None]
+    if fn == "moe_nonexpand_backward_timed":
+        args.append(None if events == "none" else events)
+    return getattr(lib, fn)(*args)
+
+
+def test_backward_argument_checks(lib):
+    train_total = lib.moe_nonexpand_train_workspace_bytes(64, 128, 128, 8, 4, -1)
+    assert _bwd(lib, N=-1) == binding.MOE_ERR_ARG
+    assert _bwd(lib, idx=None) == binding.MOE_ERR_ARG
+    assert _bwd(lib, dout=None) == binding.MOE_ERR_ARG
+    assert _bwd(lib, dx=None) == binding.MOE_ERR_ARG
+    assert _bwd(lib, dw=None) == binding.MOE_ERR_ARG           # the score gradient is always produced
+    assert _bwd(lib, dw1=None) == binding.MOE_ERR_ARG
+    assert _bwd(lib, act=1) == binding.MOE_ERR_ARG
+    assert _bwd(lib, lay=2) == binding.MOE_ERR_ARG
+    assert _bwd(lib, dx=A8) == binding.MOE_ERR_ARG
+    assert _bwd(lib, db2=A8) == binding.MOE_ERR_ARG
+    assert _bwd(lib, dw=A2) == binding.MOE_ERR_ARG
+    assert _bwd(lib, I=32) == binding.MOE_ERR_SHAPE
+    assert _bwd(lib, wsb=train_total - 1) == binding.MOE_ERR_WS
+    assert _bwd(lib, ws=A + 64) == binding.MOE_ERR_WS
+    assert _bwd(lib, fn="moe_nonexpand_backward_timed") == binding.MOE_ERR_ARG   # events required
+    if _no_device():
+        assert _bwd(lib) in NO_DEVICE
+
+
+def test_routed_training_rejects_bad_descriptors(lib):
+    bad = _routing(kind=binding.ROUTING_PAIRS, pairs=10, t=None)
+    assert lib.moe_nonexpand_routed_forward_train(A, ctypes.byref(bad), 128, 128, 8, A, None, A, None,
+                                                  binding.ACT_SWIGLU, binding.LAYOUT_INTERLEAVED, A, A, 1 << 30,
+                                                  None) == binding.MOE_ERR_ARG
+    assert lib.moe_nonexpand_routed_backward(A, A, ctypes.byref(bad), 128, 128, 8, A, A, binding.ACT_SWIGLU,
+                                             binding.LAYOUT_INTERLEAVED, A, A, None, A, None, A, A, 1 << 30,
+                                             None) == binding.MOE_ERR_ARG
+    good = _routing()
+    assert lib.moe_nonexpand_routed_backward(A, A, ctypes.byref(good), 128, 128, 8, A, A, binding.ACT_SWIGLU,
+                                             binding.LAYOUT_INTERLEAVED, A, A, None, A, None, None, A, 1 << 30,
+                                             None) == binding.MOE_ERR_ARG   # no score-gradient buffer
