@@ -18,7 +18,7 @@ from test_oracle_backward import check_autograd, check_finite_differences
 from test_oracle_pairs import check_pair_fixture, check_table_equivalence
 from test_oracle_router import check_router_against_torch, check_router_fixture
 from test_oracle_pins import (GOLDEN, _bf, _load, _num, _recipe_torch_cpu,
-                              check_metadata_invariants)
+                              check_combine_direct_sum, check_metadata_invariants)
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "moe_oracle.c")
 
@@ -59,6 +59,12 @@ MUTANTS = {
     "bwd_w2_not_transposed": ("for (int32_t n = 0; n < H; ++n) dh += dy[n] * wr[n];",
                               "for (int32_t n = 0; n < H; ++n) dh += dy[n] * w2e[(size_t)n * I + j];"),
     "pairs_score_of_next": ("scores[q] = weights[i];", "scores[q] = weights[i + 1 < P_list ? i + 1 : i];"),
+    "gather_holds_pair_index": ("x_gather_idx[p] = pair_token[i];", "x_gather_idx[p] = (int32_t)i;"),
+    "reverse_scatter_identity": ("s_rev[i] = p;", "s_rev[i] = (int32_t)i;"),
+    "score_of_next_slot": ("scores[q] = topk_w[t * K + k];", "scores[q] = topk_w[t * K + (k + 1) % K];"),
+    "combine_reverse_index_ignored": ("const double *yr = ysorted + (size_t)s_rev[q] * H;",
+                                      "const double *yr = ysorted + (size_t)q * H;"),
+    "combine_score_ignored": ("const double w = (double)scores[q];", "const double w = 1.0;"),
 }
 
 
@@ -88,6 +94,8 @@ def _pins_pass(lib):
                 or md["x_gather_idx"].tolist() != ex["x_gather_idx"]):
             return False
         check_metadata_invariants(idx, w, g["E"], md)
+        # the combine against a per-slot sum
+        check_combine_direct_sum(lib)
         # closed-form SwiGLU fixture, both layouts
         g = _load("swiglu_closed_form.json")
         x, w1, b1, w2, b2 = (_bf(g[k]) for k in ("x", "w1", "b1", "w2", "b2"))

@@ -309,13 +309,15 @@ def test_oracle_matches_sort_recipe_on_tiny_workload(layout):
     np.testing.assert_allclose(out, ref, rtol=1e-10, atol=1e-11)
 
 
-def test_combine_oracle_against_direct_sum():
+def check_combine_direct_sum(lib=None):
+    """The combine oracle against a per-slot sum that finds each pair's sorted
+    position by search (raises AssertionError on a mismatch)."""
     rng = np.random.default_rng(5)
     idx = rng.integers(-1, 4, size=(9, 3)).astype(np.int32)
     w = rng.random((9, 3)).astype(np.float32)
-    md = oracle.metadata(idx, w, 4)
+    md = oracle.metadata(idx, w, 4, lib_path=lib)
     ys = rng.standard_normal((md["P"], 7))
-    out = oracle.combine(md["token_offset"], md["s_reverse_scatter_idx"], md["scores"], ys)
+    out = oracle.combine(md["token_offset"], md["s_reverse_scatter_idx"], md["scores"], ys, lib_path=lib)
     ref = np.zeros((9, 7))
     for t in range(9):
         for k in range(3):
@@ -327,3 +329,7 @@ def test_combine_oracle_against_direct_sum():
             p = int(np.nonzero(md["s_scatter_idx"] == q)[0][0])
             ref[t] += float(w[t, k]) * ys[p]
     np.testing.assert_allclose(out, ref, rtol=1e-13, atol=1e-13)
+
+
+def test_combine_oracle_against_direct_sum():
+    check_combine_direct_sum()
