@@ -118,9 +118,8 @@ class ProcessGroupRanks:
     Phases per call: layout -> all-gather of counts -> dispatch (peer stores)
     -> barrier -> local forward -> barrier -> combine (peer loads) -> barrier.
     Tested on one GPU with a one-rank NCCL group (count all-gather, barriers,
-    buffers; no IPC), and the count exchange with two gloo ranks on CPU; not
-    run on more than one GPU by the tests of this repository (its calls get
-    one GPU).
+    buffers; no IPC), and the count exchange with two gloo ranks on CPU; the
+    tests do not run it on more than one GPU.
     """
 
     def __init__(self, E_local: int, capacity: int, H: int, K: int, group=None, device=None, opener=None):
