@@ -118,8 +118,10 @@ class ProcessGroupRanks:
     Phases per call: layout -> all-gather of counts -> dispatch (peer stores)
     -> barrier -> local forward -> barrier -> combine (peer loads) -> barrier.
     Tested on one GPU with a one-rank NCCL group (count all-gather, barriers,
-    buffers; no IPC), and the count exchange with two gloo ranks on CPU; the
-    tests do not run it on more than one GPU.
+    buffers; no IPC), and on two gloo ranks on CPU with stand-ins for the
+    library calls and file-shared buffers in place of IPC (count exchange,
+    block offsets, capacity check, buffer slicing, combine sources); the tests
+    do not run it on more than one GPU.
     """
 
     def __init__(self, E_local: int, capacity: int, H: int, K: int, group=None, device=None, opener=None):
