@@ -1,7 +1,8 @@
 """Host-side pieces of bench.py and the expert-parallel host module, on CPU:
 the DRAM-traffic record file, its use only while the kernel sources hash to
-it (checked on a copy of the sources), the roofline arithmetic, and the
-receive-block offsets against the oracle's."""
+it (checked on a copy of the sources), the roofline arithmetic, the clocks
+record of the timed region, and the receive-block offsets against the
+oracle's."""
 import os
 import sys
 
@@ -69,3 +70,25 @@ def test_block_offsets_match_the_oracle():
         off, n = block_offsets(counts)
         ref_off, ref_n = oep.recv_offsets(counts)
         assert np.array_equal(off, ref_off) and np.array_equal(n, ref_n)
+
+
+def test_clock_summary_window_median_and_reasons():
+    """The clocks record of the timed region: samples outside the window and
+    malformed lines are dropped; the SM clock is the median of the rest, and
+    every throttle reason seen active in the window is listed."""
+    s = bench.ClockSampler(0)
+    na = "Not Active"
+    s.lines = [
+        (0.5, f"1965, 1965, 300.0, 0x0, {na}, {na}, {na}, {na}"),            # before the window
+        (1.0, f"1500, 1965, 990.0, 0x4, {na}, {na}, {na}, Active"),
+        (1.1, f"1400, 1965, 1000.0, 0x4, {na}, {na}, {na}, Active"),
+        (1.2, "garbage"),
+        (1.3, f"[N/A], 1965, 1000.0, 0x4, {na}, {na}, {na}, Active"),          # unreadable clock
+        (1.4, f"1300, 1965, 1000.0, 0x44, {na}, Active, {na}, Active"),
+        (3.0, f"900, 1965, 1000.0, 0x8, Active, {na}, {na}, {na}"),          # after the window
+    ]
+    out = s.summary(0.9, 2.0)
+    assert out["sm_mhz"] == 1400.0 and out["sm_max_mhz"] == 1965.0 and out["samples"] == 3
+    assert out["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert bench.ClockSampler(0).summary(0.0, 1.0) == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                                                        "samples": 0}
