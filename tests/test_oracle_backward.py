@@ -191,3 +191,41 @@ def test_backward_pairs_dropped_entries_have_zero_gradient():
     for k in ("dx", "dw1", "dw2"):
         np.testing.assert_array_equal(g[k], h[k])
     np.testing.assert_array_equal(g["dweights"][keep], h["dweights"])
+
+
+def _sum_pair_terms_mutant(kind):
+    """A copy of the oracle's summation of the per-pair backward terms with one
+    plausible mistake planted (test code; the oracle itself is untouched)."""
+    def summed(wd, dout, tok, exp, sc, N, layout, lib_path):
+        H, I, E = wd.H, wd.I, wd.E
+        r = oracle.pairs_backward(wd, dout, tok, exp, sc, layout, lib_path=lib_path)
+        g = dict(dx=np.zeros((N, H)), dw1=np.zeros((E, H, 2 * I)), db1=np.zeros((E, 2 * I)),
+                 dw2=np.zeros((E, I, H)), db2=np.zeros((E, H)))
+        g["pairs"] = dict(tok=tok, exp=exp, **r)
+        for e in np.unique(exp):
+            sel = exp == e
+            te = tok[sel]
+            g["dw2"][e] = r["h"][sel].T @ r["dy"][sel]
+            g["db2"][e] = r["dy"][sel].sum(0)
+            rows = tok[:int(sel.sum())] if kind == "dw1_rows_of_first_tokens" else te
+            g["dw1"][e] = wd.x[rows].T @ r["dz"][sel]
+            if kind != "db1_dropped":
+                g["db1"][e] = r["dz"][sel].sum(0)
+            if kind == "dx_overwritten_per_expert":
+                g["dx"][te] = r["dz"][sel] @ wd.w1e(e).T
+            else:
+                np.add.at(g["dx"], te, r["dz"][sel] @ wd.w1e(e).T)
+        return g
+    return summed
+
+
+@pytest.mark.parametrize("kind", ["db1_dropped", "dw1_rows_of_first_tokens", "dx_overwritten_per_expert"])
+def test_finite_differences_reject_summation_mistakes(monkeypatch, kind):
+    """The summation of the per-pair terms is numpy code outside the C source
+    the mutation suite edits; the finite-difference pin must still catch a
+    mistake planted there."""
+    monkeypatch.setattr(oracle, "_sum_pair_terms", _sum_pair_terms_mutant(None))
+    check_finite_differences(0)                      # the unmutated copy passes
+    monkeypatch.setattr(oracle, "_sum_pair_terms", _sum_pair_terms_mutant(kind))
+    with pytest.raises(AssertionError):
+        check_finite_differences(0)
