@@ -72,8 +72,9 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, interval_ms: int = 20):
         self.device_index = device_index
+        self.interval_ms = interval_ms
         self.proc = None
         self.lines = []
         self.thread = None
@@ -82,7 +83,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
@@ -136,6 +137,31 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 def gemm_flops(P: int, H: int, I: int):
     return 4.0 * P * H * I, 2.0 * P * H * I
+
+
+def choose_tensor_peak(peaks, clocks, timed_s: float):
+    """The bf16 peak a GEMM timed inside a region of ``timed_s`` seconds is
+    held to: the burst figure (a short region runs at full clock) unless the
+    region lasts seconds and its clock record shows the power cap, in which
+    case the sustained figure.  Returns (TFLOP/s, label)."""
+    capped = "sw_power_cap" in (clocks or {}).get("reasons", [])
+    if timed_s >= 1.0 and capped:
+        return peaks["bf16_tflops_sustained"], "sustained"
+    return peaks["bf16_tflops"], "burst"
+
+
+def clocks_for(sampler, t0: float, t1: float, leg0: float, leg1: float):
+    """The clock record of the timed region [t0, t1]; when the region is
+    shorter than the sampling interval and holds no sample, that of the whole
+    forward leg [leg0, leg1] (warm-up, timed steps and end-to-end steps, the
+    same kernels back to back), with the window named."""
+    c = sampler.summary(t0, t1)
+    c["window"] = "timed region"
+    if c["samples"] == 0:
+        c = sampler.summary(leg0, leg1)
+        c["window"] = "forward leg (timed region shorter than the sampling interval)"
+    c["interval_ms"] = sampler.interval_ms
+    return c
 
 
 def algorithmic_bytes(inp, P: int, freq):
@@ -211,6 +237,9 @@ def parse():
     ap.add_argument("--workload", default="prefill")
     ap.add_argument("--layout", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true", help="skip the other configured workloads")
+    ap.add_argument("--check-launch", action="store_true",
+                    help="every rank prints its rank and world size and exits (checks the --gpus launch)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=6.0,
                     help="at most this much oracle work per step of --impl reference (sets its token sample)")
@@ -425,7 +454,7 @@ def ep_emulated(dev, peaks, reps: int = 20):
                     "L2 flushed before each replay"}
 
 
-def backward_leg(inp, w1, b1, layout, dev, peaks, steps: int = 30, warmup: int = 3):
+def backward_leg(inp, w1, b1, layout, dev, peaks, peak_tf, peak_label, steps: int = 30, warmup: int = 3):
     """One training step, forward_train + backward, on the bench workload:
     mean device time per step with the backward's seven stages timed by
     events on the launching stream.  Inputs are larger than L2 (1.2 GB of
@@ -468,7 +497,7 @@ def backward_leg(inp, w1, b1, layout, dev, peaks, steps: int = 30, warmup: int =
     gemm_ms = float(sum(st[names.index(k)] for k in flops))
     bwd_ms = float(st.sum())
     dom = max(flops, key=lambda k: st[names.index(k)])
-    peak = peaks["bf16_tflops_sustained"]
+    peak = peak_tf
     prep_bytes = 2 * P * H * 2 + N * H * 2  # y read, dy written, dout read
     del ws
     return {"workload": wl.name, "steps": steps, "train_step_ms": fwd + bwd_ms,
@@ -479,7 +508,16 @@ def backward_leg(inp, w1, b1, layout, dev, peaks, steps: int = 30, warmup: int =
             "bwd_gemm_frac_of_peak": 12 * phi / (gemm_ms * 1e-3) / 1e12 / peak,
             "prep_gbs": prep_bytes / (st[0] * 1e-3) / 1e9,
             "dominant": {"kernel": f"backward grouped GEMM {dom}", "tflops": float(tf[dom]), "peak": peak,
-                         "frac": float(tf[dom] / peak), "peak_source": "measured bf16 sustained"}}
+                         "frac": float(tf[dom] / peak), "peak_source": f"bf16 {peak_label}"},
+            "gemm_frac_of_peak": {k: float(v / peak) for k, v in tf.items()}}
+
+
+def bench_config(wl, layout: int, world: int, P: int, w_bytes: int):
+    """The ``config`` object of the JSON line, the same for both arms."""
+    return {"workload": wl.name, "N": wl.N, "H": wl.H, "I": wl.I, "E": wl.E, "K": wl.K, "P": P,
+            "layout": "interleaved" if layout == 0 else "concatenated",
+            "routing": wl.description, "parallelism": f"replicas x{world} (token shards)",
+            "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (w_bytes / 1e9)}
 
 
 def run_reference(args, rank, world):
@@ -516,18 +554,135 @@ def run_reference(args, rank, world):
             times.append(dt)
     total = sum(times)
     value = n * len(times) / total
+    P = int((idx >= 0).sum())
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * total / len(times), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "N": wl.N, "H": wl.H, "I": wl.I, "E": wl.E, "K": wl.K,
-                   "layout": args.layout, "sample_tokens_per_step": n},
+        "config": bench_config(wl, args.layout, world, P, (inp.w1.numel() + inp.w2.numel()) * 2),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                          "sample": f"{n} seeded tokens of the {wl.name} workload per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def timed_forwards(step, steps: int, stream, dev):
+    """``steps`` back-to-back forwards, each with its five stage events on the
+    launching stream; returns (elapsed ms, mean ms of the four stages)."""
+    import numpy as np
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    start.record(stream)
+    for i in range(steps):
+        step(ev[i])
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    stage_ms = np.zeros(4)
+    for e in ev:
+        for j in range(4):
+            stage_ms[j] += e[j].elapsed_time(e[j + 1])
+    return start.elapsed_time(end), stage_ms / steps
+
+
+def graph_forward_ms(step, steps: int, dev):
+    """One forward captured in a CUDA graph and replayed ``steps`` times back
+    to back: device ms per replay (the launch sequence without host calls)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    cs = torch.cuda.Stream(dev)
+    cs.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(cs):
+        step(None, cs)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.graph(g, stream=cs):
+            step(None, cs)
+    torch.cuda.current_stream(dev).wait_stream(cs)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        g.replay()
+    b.record()
+    b.synchronize()
+    ms = a.elapsed_time(b) / steps
+    del g
+    return ms
+
+
+def forward_summary(wl, P, freq, inp, stage_ms, ms_per_step, peaks, peak_tf, peak_label):
+    """Per-stage rates and roofline fractions of one workload's forward."""
+    H, I, N, K, E = wl.H, wl.I, wl.N, wl.K, wl.E
+    up_flops, down_flops = gemm_flops(P, H, I)
+    up_tf = up_flops / (stage_ms[1] * 1e-3) / 1e12 if stage_ms[1] > 0 else 0.0
+    down_tf = down_flops / (stage_ms[2] * 1e-3) / 1e12 if stage_ms[2] > 0 else 0.0
+    # the combine reads each pair's bf16 row and its e5m2 residual (3 bytes per element)
+    comb_bytes = P * H * 3 + N * H * 2 + (N + 1) * 4 + P * 8
+    meta_bytes = N * K * 8 + 4 * P * 4 + 4 * (N + 1) + 8 * E
+    alg_bytes = algorithmic_bytes(inp, P, freq)
+    t_tensor = (up_flops + down_flops) / (peak_tf * 1e12)
+    t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    return {
+        "stages_ms": {"metadata": float(stage_ms[0]), "gemm_up": float(stage_ms[1]),
+                      "gemm_down": float(stage_ms[2]), "combine": float(stage_ms[3])},
+        "gemm_up_tflops": up_tf, "gemm_down_tflops": down_tf,
+        "gemm_up_frac": up_tf / peak_tf, "gemm_down_frac": down_tf / peak_tf,
+        "gemm_up_frac_of_burst": up_tf / peaks["bf16_tflops"],
+        "gemm_down_frac_of_burst": down_tf / peaks["bf16_tflops"],
+        "gemm_peak": {"tflops": peak_tf, "kind": peak_label},
+        "combine_gbs": comb_bytes / (stage_ms[3] * 1e-3) / 1e9,
+        "combine_frac_hbm": comb_bytes / (stage_ms[3] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "metadata_gbs": meta_bytes / (stage_ms[0] * 1e-3) / 1e9,
+        "algorithmic_bytes": alg_bytes, "flops": up_flops + down_flops,
+        "step_roofline_ms": max(t_tensor, t_hbm) * 1e3,
+        "step_bound": "tensor" if t_tensor >= t_hbm else "hbm",
+        "step_frac_of_roofline": max(t_tensor, t_hbm) * 1e3 / ms_per_step,
+    }
+
+
+def workload_leg(name: str, dev, peaks, peak_tf, peak_label, steps: int, warmup: int):
+    """One configured workload timed like the headline one (interleaved
+    layout): ``steps`` back-to-back forwards after ``warmup`` untimed ones,
+    stage events on the launching stream, plus the CUDA-graph time."""
+    import torch
+
+    from mixture_experts_routed_non_b200 import binding, synthetic
+    wl = synthetic.WORKLOADS[name]
+    inp = synthetic.make_inputs(wl, device=dev)
+    ws = binding.alloc_workspace(wl.N, wl.H, wl.I, wl.E, wl.K, -1, dev)
+    out = torch.empty(wl.N, wl.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(events=None, s=None):
+        binding.forward(inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, inp.b1, inp.b2, out=out, ws=ws,
+                        events=events, stream=s)
+
+    for _ in range(max(3, warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    if binding.read_error(ws):
+        raise SystemExit(f"bench.py: device error in workload {name}")
+    freq = binding.meta_from_workspace(ws, wl.N, wl.H, wl.I, wl.E, wl.K)["expert_frequency"].cpu().numpy()
+    P = int(freq.sum())
+    elapsed, stage_ms = timed_forwards(step, steps, stream, dev)
+    ms = elapsed / steps
+    g_ms = graph_forward_ms(step, steps, dev)
+    res = {"N": wl.N, "H": wl.H, "I": wl.I, "E": wl.E, "K": wl.K, "P": P, "routing": wl.description,
+           "steps": steps, "warmup": max(3, warmup), "ms_per_step": ms, "tokens_per_s": wl.N / (ms * 1e-3),
+           "graph_ms_per_step": g_ms, "graph_tokens_per_s": wl.N / (g_ms * 1e-3),
+           "active_experts": int((freq > 0).sum())}
+    res.update(forward_summary(wl, P, freq, inp, stage_ms, ms, peaks, peak_tf, peak_label))
+    if res["step_bound"] == "hbm":
+        res["note"] = "weight-read bound: step_frac_of_roofline is the algorithmic bytes at the copy bandwidth"
+    del inp, ws, out
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_ours(args, rank, world, local):
@@ -545,6 +700,12 @@ def run_ours(args, rank, world, local):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
+    peaks, peaks_src = load_peaks()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.2)
+    t_leg0 = time.time()
+
     wl = synthetic.WORKLOADS[args.workload]
     inp = synthetic.make_inputs(wl, device=dev, seed=wl.seed + 1000 * rank)
     N, H, I, E, K = wl.N, wl.H, wl.I, wl.E, wl.K
@@ -556,9 +717,9 @@ def run_ours(args, rank, world, local):
     out = torch.empty(N, H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step(events=None):
+    def step(events=None, s=None):
         binding.forward(inp.x, inp.topk_idx, inp.topk_w, w1, inp.w2, b1, inp.b2, layout=args.layout,
-                        out=out, ws=ws, events=events)
+                        out=out, ws=ws, events=events, stream=s)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -571,32 +732,14 @@ def run_ours(args, rank, world, local):
     P = int(freq.sum())
 
     # ---- timed region: K steps, stage events on the launching stream
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.3)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(args.steps):
-        step(ev[i])
-    end.record(stream)
-    torch.cuda.synchronize(dev)
+    elapsed_ms, stage_ms = timed_forwards(step, args.steps, stream, dev)
     t_wall1 = time.time()
     if world > 1:
         dist.barrier()
-    time.sleep(0.15)
-    sampler.stop()
-    elapsed_ms = start.elapsed_time(end)
-    stage_ms = np.zeros(4)
-    for e in ev:
-        for j in range(4):
-            stage_ms[j] += e[j].elapsed_time(e[j + 1])
-    stage_ms /= args.steps
     max_ms = max_over_ranks(elapsed_ms, dev, world)
     ms_per_step = max_ms / args.steps
     value = N * world * args.steps / (max_ms / 1000.0)
@@ -659,6 +802,7 @@ def run_ours(args, rank, world, local):
     s_out.wait_stream(s_cmp)
     e2.record(s_out)
     torch.cuda.synchronize(dev)
+    t_leg1 = time.time()
     e2e_ms = max_over_ranks(s2.elapsed_time(e2), dev, world)
     e2e_value = N * world * e2e_steps / (e2e_ms / 1000.0)
     h2d = nx + ni + nw
@@ -667,27 +811,30 @@ def run_ours(args, rank, world, local):
     last = (e2e_steps - 1) % nbuf
     if not torch.equal(outs_h[last], out.cpu()):
         raise SystemExit("bench.py: end-to-end result differs from the device-resident forward")
+    del packed_d, outs_d, xs_d, idxs_d, ws_d
 
-    peaks, peaks_src = load_peaks()
-    up_flops, down_flops = gemm_flops(P, H, I)
-    up_tflops = up_flops / (stage_ms[1] * 1e-3) / 1e12
-    down_tflops = down_flops / (stage_ms[2] * 1e-3) / 1e12
-    gemm_tflops = (up_flops + down_flops) / ((stage_ms[1] + stage_ms[2]) * 1e-3) / 1e12
-    # the GEMMs are timed inside a loop of back-to-back steps that runs long
-    # enough to reach the power cap: the sustained measured peak applies
-    peak_tf = peaks["bf16_tflops_sustained"]
-    comb_bytes = P * H * 2 + N * H * 2 + (N + 1) * 4 + P * 8
-    meta_bytes = N * K * 8 + 4 * P * 4 + 4 * (N + 1) + 8 * E
-    alg_bytes = algorithmic_bytes(inp, P, freq)
-    total_flops = up_flops + down_flops
-    t_roof = max(total_flops / (peak_tf * 1e12), alg_bytes / (peaks["hbm_gbs"] * 1e9))
-    clocks = sampler.summary(t_wall0, t_wall1)
+    # ---- the same forward replayed from a CUDA graph (no host calls between launches)
+    graph_ms = graph_forward_ms(step, args.steps, dev)
+
+    # ---- roofline of the headline workload, against the peak its clock record supports
+    time.sleep(0.1)
+    clocks = clocks_for(sampler, t_wall0, t_wall1, t_leg0, t_leg1)
+    peak_tf, peak_label = choose_tensor_peak(peaks, clocks, (t_wall1 - t_wall0))
+    summ = forward_summary(wl, P, freq, inp, stage_ms, ms_per_step, peaks, peak_tf, peak_label)
+
+    # ---- every other configured workload that has a forward, same timing rules
+    workloads = {}
+    if rank == 0 and not args.no_workloads:
+        for name in ("ranklocal", "prefill256", "decode256", "tiny"):
+            if name != wl.name:
+                workloads[name] = workload_leg(name, dev, peaks, peak_tf, peak_label, args.steps, args.warmup)
 
     meta_c2 = metadata_only(dev, peaks) if rank == 0 else None
     meta_pairs = metadata_pairs_only(dev, peaks) if rank == 0 else None
     router = router_only(dev, peaks) if rank == 0 else None
-    train = backward_leg(inp, w1, b1, args.layout, dev, peaks) if rank == 0 else None
+    train = backward_leg(inp, w1, b1, args.layout, dev, peaks, peak_tf, peak_label) if rank == 0 else None
     ep = ep_emulated(dev, peaks) if rank == 0 else None
+    sampler.stop()
 
     if world > 1:
         dist.destroy_process_group()
@@ -706,41 +853,38 @@ def run_ours(args, rank, world, local):
         "unit": "tokens/s",
         "n_gpus": world,
         "steps": args.steps,
-        "warmup": args.warmup,
+        "warmup": max(3, args.warmup),
         "ms_per_step": ms_per_step,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": wl.name, "N": N, "H": H, "I": I, "E": E, "K": K, "P": P,
-                   "layout": "interleaved" if args.layout == 0 else "concatenated",
-                   "routing": wl.description, "parallelism": f"replicas x{world} (token shards)",
-                   "l2": "inputs larger than L2 (expert weights %.2f GB per step)" % (
-                       (inp.w1.numel() + inp.w2.numel()) * 2 / 1e9)},
+        "config": bench_config(wl, args.layout, world, P, (inp.w1.numel() + inp.w2.numel()) * 2),
         "roofline": {"bound": "tensor", "kernel": "grouped GEMM up (gather + SwiGLU)",
-                     "achieved": up_tflops, "peak": peak_tf, "unit": "TFLOP/s",
-                     "frac": up_tflops / peak_tf, "peak_source": f"{peaks_src} bf16 sustained",
+                     "achieved": summ["gemm_up_tflops"], "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": summ["gemm_up_tflops"] / peak_tf,
+                     "peak_source": f"{peaks_src} bf16 {peak_label} (chosen from the clock record)",
+                     "frac_of_burst": summ["gemm_up_tflops"] / peaks["bf16_tflops"],
+                     "frac_of_sustained": summ["gemm_up_tflops"] / peaks["bf16_tflops_sustained"],
                      "traffic": traffic_record("gemm_up", wl.name)},
-        "gemm_tflops": gemm_tflops,
-        "gemm_frac_of_peak": gemm_tflops / peak_tf,
-        "step_frac_of_roofline": (t_roof * 1e3) / ms_per_step,
-        "stages_ms": {"metadata": stage_ms[0], "gemm_up": stage_ms[1], "gemm_down": stage_ms[2],
-                      "combine": stage_ms[3]},
-        "stages": {
-            "gemm_up_tflops": up_tflops, "gemm_down_tflops": down_tflops,
-            "combine_gbs": comb_bytes / (stage_ms[3] * 1e-3) / 1e9,
-            "combine_frac_hbm": comb_bytes / (stage_ms[3] * 1e-3) / 1e9 / peaks["hbm_gbs"],
-            "metadata_gbs": meta_bytes / (stage_ms[0] * 1e-3) / 1e9,
-        },
+        "gemm_tflops": (summ["flops"]) / ((stage_ms[1] + stage_ms[2]) * 1e-3) / 1e12,
+        "gemm_frac_of_peak": (summ["flops"]) / ((stage_ms[1] + stage_ms[2]) * 1e-3) / 1e12 / peak_tf,
+        "step_frac_of_roofline": summ["step_frac_of_roofline"],
+        "stages_ms": summ["stages_ms"],
+        "stages": {k: summ[k] for k in ("gemm_up_tflops", "gemm_down_tflops", "gemm_up_frac", "gemm_down_frac",
+                                        "combine_gbs", "combine_frac_hbm", "metadata_gbs")},
+        "graph": {"ms_per_step": graph_ms, "tokens_per_s": N * world / (graph_ms * 1e-3),
+                  "note": "one forward captured in a CUDA graph, replayed --steps times back to back"},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps, "pipelining": "copy-in / compute / copy-out streams, 3 buffer sets, inputs packed in one copy"},
+        "workloads": workloads,
         "metadata_only": meta_c2,
         "metadata_pairs_only": meta_pairs,
         "router_only": router,
         "training": train,
         "ep_emulated": ep,
-        "gpu_launches": 4 * args.steps,  # meta, up, down, combine (plus one 4-byte memset)
+        "gpu_launches": 5 * args.steps,  # metadata count + scatter, up, down, combine
         "clocks": clocks,
     }
     if cpu is not None:
@@ -748,9 +892,30 @@ def run_ours(args, rank, world, local):
     print(json.dumps(line), flush=True)
 
 
+def relaunch(n: int) -> int:
+    """Run this same command as n ranks, one process per GPU, under
+    torch.distributed.run (rendezvous on 127.0.0.1, a free port); returns its
+    exit code.  ``timeout -k`` bounds the whole launch."""
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = ["timeout", "-k", "60", "3600", sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        raise SystemExit(relaunch(args.gpus))
     rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but {world} ranks were launched (WORLD_SIZE)")
+    if args.check_launch:
+        print(json.dumps({"rank": rank, "world": world, "impl": args.impl}), flush=True)
+        return
     if args.impl == "reference":
         run_reference(args, rank, world)
     else:

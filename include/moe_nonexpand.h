@@ -139,14 +139,17 @@ MOE_API int moe_nonexpand_metadata(const int32_t *topk_idx, const float *topk_w,
  * cannot provide the `ws` buffer the other entry points need.  The pages have
  * no counterpart to this call; it exists for those callers only.
  *
- * Scratch: a fixed 640 KiB array in device memory that belongs to the library
+ * Scratch: a fixed 160 KiB array in device memory that belongs to the library
  * (a file-scope __device__ array: every GPU that loads the library keeps it
  * until the process exits).  It holds what the metadata kernels need besides
- * their inputs and outputs -- a header, the per-tile histogram table of at
- * most 148 tiles x E experts, and the GEMM tile table -- which fits for every
- * supported size (E <= 1024); a size that would not fit returns MOE_ERR_WS.
- * The call allocates nothing: no cudaMalloc, cudaFree or allocating library
- * routine.
+ * their inputs and outputs -- a header with the device error word, the
+ * per-tile histogram table (at most 32768 entries: the tiling keeps
+ * tiles x E within that), per-tile counts and the GEMM tile table -- which
+ * fits for every supported size (E <= 1024); a size that would not fit
+ * returns MOE_ERR_WS.  The call allocates nothing: no cudaMalloc, cudaFree or
+ * allocating library routine.  Argument checks are those of
+ * moe_nonexpand_metadata (sizes, null and misaligned pointers give
+ * MOE_ERR_ARG before any CUDA call).
  *
  * The first call on a device looks up the array's device address (with that
  * device current) and caches it; make that first call before any stream
@@ -154,13 +157,24 @@ MOE_API int moe_nonexpand_metadata(const int32_t *topk_idx, const float *topk_w,
  * contents (the kernels write every scratch byte they read, so nothing has to
  * be cleared): calls that can overlap on the GPU -- on different streams, or
  * on one device from several host threads without ordering -- race and must
- * not be issued.  Device-side error bits (bad ids, pair-count mismatch) are
- * kept in the library's scratch and are not reported by this call; the
- * outputs follow the same rules as moe_nonexpand_metadata.
+ * not be issued.  Device-side error bits (bad ids, pair-count mismatch) land
+ * in the scratch's error word, which every call rewrites whole; read them with
+ * moe_nonexpand_metadata_noalloc_read_error.  The outputs follow the same
+ * rules as moe_nonexpand_metadata.
  */
 MOE_API int moe_nonexpand_metadata_noalloc(const int32_t *topk_idx, const float *topk_w,
                                    int64_t N, int32_t K, int32_t E, int64_t total_pairs,
                                    const moe_meta_t *meta, moe_stream_t stream);
+
+/*
+ * The device error word (MOE_DEVERR_* bits) of the last
+ * moe_nonexpand_metadata_noalloc call on the current device, copied to the
+ * host pointer *err_word after `stream` has been synchronised -- the
+ * counterpart of moe_nonexpand_read_error for the library's own scratch.
+ * Call it on the stream of that metadata call (or after it has finished).
+ * Like the call it reports on, it has no counterpart on the pages.
+ */
+MOE_API int moe_nonexpand_metadata_noalloc_read_error(moe_stream_t stream, uint32_t *err_word);
 
 /*
  * The whole local expert forward: metadata, gathered grouped GEMM up with
@@ -492,6 +506,7 @@ typedef struct moe_ws_layout_t {
     size_t slot_pair;          /* training workspace: int32 [slots], the pair of each routing slot or -1 */
     size_t ds;                 /* training workspace: fp32 [P_cap], score gradients in pair order */
     size_t train_total;        /* == moe_nonexpand_train_workspace_bytes(...) */
+    size_t y_lo;               /* uint8 [P_cap,H]: e5m2 residual y - bf16(y) of every y element */
 } moe_ws_layout_t;
 
 MOE_API int moe_nonexpand_workspace_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,

@@ -49,6 +49,7 @@ EXPORTED = (
     "moe_nonexpand_read_error",
     "moe_nonexpand_strerror",
     "moe_nonexpand_metadata_noalloc",
+    "moe_nonexpand_metadata_noalloc_read_error",
     "moe_nonexpand_selftest_wait_timeout",
     "moe_nonexpand_routed_workspace_bytes",
     "moe_nonexpand_routed_metadata",
@@ -88,7 +89,8 @@ class WsLayout(ctypes.Structure):
         "meta_token_offset", "meta_scores", "h", "y")] + [
         ("p_cap", ctypes.c_int64), ("meta_tiles", ctypes.c_int32), ("meta_tile_slots", ctypes.c_int32),
         ("z", ctypes.c_size_t), ("dz", ctypes.c_size_t), ("dy", ctypes.c_size_t),
-        ("slot_pair", ctypes.c_size_t), ("ds", ctypes.c_size_t), ("train_total", ctypes.c_size_t)]
+        ("slot_pair", ctypes.c_size_t), ("ds", ctypes.c_size_t), ("train_total", ctypes.c_size_t),
+        ("y_lo", ctypes.c_size_t)]
 
 
 class MoeRouting(ctypes.Structure):
@@ -151,6 +153,8 @@ def load() -> ctypes.CDLL:
     lib.moe_nonexpand_read_error.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
     lib.moe_nonexpand_metadata_noalloc.restype = ctypes.c_int
     lib.moe_nonexpand_metadata_noalloc.argtypes = [P, P, i64, i32, i32, i64, ctypes.POINTER(MoeMeta), P]
+    lib.moe_nonexpand_metadata_noalloc_read_error.restype = ctypes.c_int
+    lib.moe_nonexpand_metadata_noalloc_read_error.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
     lib.moe_nonexpand_selftest_wait_timeout.restype = ctypes.c_int
     lib.moe_nonexpand_selftest_wait_timeout.argtypes = [P, sz, ctypes.c_uint32, P]
     R = ctypes.POINTER(MoeRouting)
@@ -290,13 +294,17 @@ def meta_from_workspace(ws: torch.Tensor, N: int, H: int, I: int, E: int, K: int
 
 
 def intermediates_from_workspace(ws: torch.Tensor, N: int, H: int, I: int, E: int, K: int,
-                                 total_pairs: int = -1):
+                                 total_pairs: int = -1, with_residual: bool = False):
     """Views (h [P_cap,I], y [P_cap,H], both bf16, expert-sorted rows) of the
-    intermediates that moe_nonexpand_forward keeps in the workspace."""
+    intermediates that moe_nonexpand_forward keeps in the workspace; with
+    ``with_residual`` also y_lo [P_cap,H] (uint8 bits of the e5m2 residual
+    y - bf16(y) that the combine adds back)."""
     lay = workspace_layout(N, H, I, E, K, total_pairs)
     pc = lay.p_cap
     h = ws[lay.h:lay.h + pc * I * 2].view(torch.bfloat16).view(pc, I)
     y = ws[lay.y:lay.y + pc * H * 2].view(torch.bfloat16).view(pc, H)
+    if with_residual:
+        return h, y, ws[lay.y_lo:lay.y_lo + pc * H].view(pc, H)
     return h, y
 
 
@@ -339,6 +347,15 @@ def metadata_noalloc(topk_idx: torch.Tensor, topk_w: torch.Tensor, E: int, meta:
                                                  ctypes.byref(m), _stream_handle(stream)),
            "moe_nonexpand_metadata_noalloc")
     return meta
+
+
+def metadata_noalloc_read_error(stream: Optional[torch.cuda.Stream] = None) -> int:
+    """The device error word of the last metadata_noalloc call on the current
+    device (syncs the stream)."""
+    v = ctypes.c_uint32(0)
+    _check(load().moe_nonexpand_metadata_noalloc_read_error(_stream_handle(stream), ctypes.byref(v)),
+           "moe_nonexpand_metadata_noalloc_read_error")
+    return int(v.value)
 
 
 def forward(x: torch.Tensor, topk_idx: torch.Tensor, topk_w: torch.Tensor,

@@ -14,6 +14,44 @@
 
 
 namespace moe {
+
+int check_routing_sizes(int64_t N, int32_t E, int32_t K, int64_t total_pairs) {
+    if (N < 0 || K < 1 || K > 32 || E < 1 || E > kMaxExperts) return MOE_ERR_ARG;
+    if (N * (int64_t)K >= (int64_t)(1u << 31) - (1 << 20)) return MOE_ERR_ARG;
+    if (total_pairs < -1 || total_pairs > N * K) return MOE_ERR_ARG;
+    return MOE_OK;
+}
+
+bool ptr_aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+cudaError_t launch_setup_once(const void *kernel, int *value,
+                              const std::function<cudaError_t(int dev, int *value)> &setup) {
+    struct Entry {
+        const void *kernel;
+        int dev;
+        int value;
+    };
+    static std::mutex mu;
+    static Entry done[1024];  // (kernel, device) pairs already set up
+    static int n_done = 0;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> g(mu);
+    for (int i = 0; i < n_done; ++i) {
+        if (done[i].kernel == kernel && done[i].dev == dev) {
+            *value = done[i].value;
+            return cudaSuccess;
+        }
+    }
+    int v = 0;
+    err = setup(dev, &v);
+    if (err != cudaSuccess) return err;
+    if (n_done < 1024) done[n_done++] = Entry{kernel, dev, v};
+    *value = v;
+    return cudaSuccess;
+}
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -26,26 +64,7 @@ struct Layout {
     moe_ws_layout_t l;
 };
 
-// Slots per metadata tile: a multiple of kMetaTileUnit, sized so that there
-// are at most kMetaMaxTiles tiles (one CTA per SM of a B200); the scatter
-// kernel reads the whole [T,E] histogram table, which stays small.
-void meta_tiling(int64_t NK, int32_t *tile_slots, int32_t *tiles) {
-    const int64_t per = (int64_t)kMetaTileUnit * kMetaMaxTiles;
-    int64_t c = (NK + per - 1) / per;
-    if (c < 1) c = 1;
-    const int64_t S = (int64_t)kMetaTileUnit * c;
-    int64_t T = (NK + S - 1) / S;
-    if (T < 1) T = 1;
-    *tile_slots = (int32_t)S;
-    *tiles = (int32_t)T;
-}
-
-int check_sizes(int64_t N, int32_t E, int32_t K, int64_t total_pairs) {
-    if (N < 0 || K < 1 || K > 32 || E < 1 || E > kMaxExperts) return MOE_ERR_ARG;
-    if (N * (int64_t)K >= (int64_t)(1u << 31) - (1 << 20)) return MOE_ERR_ARG;
-    if (total_pairs < -1 || total_pairs > N * K) return MOE_ERR_ARG;
-    return MOE_OK;
-}
+int check_sizes(int64_t N, int32_t E, int32_t K, int64_t total_pairs) { return check_routing_sizes(N, E, K, total_pairs); }
 
 int check_dense(int64_t p_cap, int32_t H, int32_t I, int32_t E) {
     if (H <= 0 || I <= 0 || (H % 64) != 0 || (I % 64) != 0) return MOE_ERR_SHAPE;
@@ -60,13 +79,13 @@ moe_ws_layout_t compute_layout_nk(int64_t N, int32_t H, int32_t I, int32_t E, in
     moe_ws_layout_t l;
     memset(&l, 0, sizeof l);
     l.p_cap = pc;
-    meta_tiling(NK, &l.meta_tile_slots, &l.meta_tiles);
+    meta_tiling(NK, E, &l.meta_tile_slots, &l.meta_tiles);
     const size_t T = (size_t)l.meta_tiles;
     size_t o = 0;
     l.header = o;
     o = align_up(o + sizeof(WsHeader), kAlign);
     l.tile_hist = o;
-    o = align_up(o + T * E * 4, kAlign);
+    o = align_up(o + T * meta_hist_ld(E) * 4, kAlign);
     l.tile_valid = o;
     o = align_up(o + T * 4, kAlign);
     l.tile_err = o;
@@ -93,6 +112,8 @@ moe_ws_layout_t compute_layout_nk(int64_t N, int32_t H, int32_t I, int32_t E, in
         o = align_up(o + (size_t)pc * I * 2, 1024);
         l.y = o;
         o = align_up(o + (size_t)pc * H * 2, 1024);
+        l.y_lo = o;
+        o = align_up(o + (size_t)pc * H, 1024);
     }
     l.total = o;
     if (H > 0 && I > 0) {  // training: z (fp32), dz and dy after the inference workspace
@@ -251,6 +272,20 @@ bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// uint8 [outer][inner] (inner % 16 == 0) with a box of 64 x box_outer bytes in
+// the 64-byte swizzle (16-byte chunk c of box row r at c ^ ((r >> 1) & 3)).
+bool make_map_2d_u8_sw64(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, uint32_t box_outer) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner};
+    cuuint32_t box[2] = {64, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The same for fp32 [outer][inner] (a box of 32 fp32 is one 128-byte row).
 bool make_map_2d_f32(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
                      uint32_t box_outer) {
@@ -328,6 +363,7 @@ MetaArgs meta_args(const Routing &r, int32_t E, const moe_ws_layout_t &l, uint8_
     a.p_cap = l.p_cap;
     a.tiles = l.meta_tiles;
     a.tile_slots = l.meta_tile_slots;
+    a.hist_ld = meta_hist_ld(E);
     a.hdr = reinterpret_cast<WsHeader *>(ws + l.header);
     a.tile_hist = reinterpret_cast<int32_t *>(ws + l.tile_hist);
     a.tile_valid = reinterpret_cast<int32_t *>(ws + l.tile_valid);
@@ -396,6 +432,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
 
     __nv_bfloat16 *hbuf = reinterpret_cast<__nv_bfloat16 *>(w + l.h);
     __nv_bfloat16 *ybuf = reinterpret_cast<__nv_bfloat16 *>(w + l.y);
+    uint8_t *ylo = w + l.y_lo;
     if (l.p_cap > 0) {
         const int64_t cap_mtiles = (l.p_cap + kTileRows - 1) / kTileRows + E;
         // ---- up: x gathered rows . w1 -> h
@@ -435,6 +472,8 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         if (!make_map_a_chunks(&dn.tmap_a16, hbuf, (uint64_t)I, (uint64_t)l.p_cap, 16, 1)) return MOE_ERR_CUDA;
         if (!make_map_b_chunks(&dn.tmap_b, w2, (uint64_t)H, (uint64_t)E * I)) return MOE_ERR_CUDA;
         if (!make_map_2d(&dn.tmap_out, ybuf, (uint64_t)H, (uint64_t)l.p_cap, 64, 32)) return MOE_ERR_CUDA;
+        if (!make_map_2d_u8_sw64(&dn.tmap_lo, ylo, (uint64_t)H, (uint64_t)l.p_cap, 32)) return MOE_ERR_CUDA;
+        dn.out_lo = ylo;
         dn.expert_off = meta.expert_frequency_offset;
         dn.tile_off = ma.gemm_tile_off;
         dn.bias = static_cast<const __nv_bfloat16 *>(b2);
@@ -455,7 +494,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         if ((st = record(ev, 2, s))) return st;
         if ((st = record(ev, 3, s))) return st;
     }
-    if (launch_combine(ybuf, meta.token_offset, meta.s_reverse_scatter_idx, meta.scores, N, H,
+    if (launch_combine(ybuf, ylo, meta.token_offset, meta.s_reverse_scatter_idx, meta.scores, N, H,
                        static_cast<__nv_bfloat16 *>(out), hdr, dev.sms, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     if ((st = record(ev, 4, s))) return st;
@@ -596,7 +635,7 @@ int backward_impl(const void *dout, const void *x, const Routing &r, int32_t H, 
     }
     if ((st = record(ev, 5, s))) return st;
     // dx[t] = sum of its pairs' dx rows (weight 1)
-    if (launch_combine(ybuf, meta.token_offset, meta.s_reverse_scatter_idx, nullptr, N, H,
+    if (launch_combine(ybuf, nullptr, meta.token_offset, meta.s_reverse_scatter_idx, nullptr, N, H,
                        static_cast<__nv_bfloat16 *>(dx), hdr, dev.sms, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     if ((st = record(ev, 6, s))) return st;
@@ -824,7 +863,7 @@ extern "C" MOE_API int moe_nonexpand_combine(const void *y, const moe_meta_t *me
     DeviceInfo dev;
     int st = device_info(&dev);
     if (st) return st;
-    return launch_combine(static_cast<const __nv_bfloat16 *>(y), meta->token_offset, meta->s_reverse_scatter_idx,
+    return launch_combine(static_cast<const __nv_bfloat16 *>(y), nullptr, meta->token_offset, meta->s_reverse_scatter_idx,
                           meta->scores, N, H, static_cast<__nv_bfloat16 *>(out), nullptr, dev.sms,
                           reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
                ? MOE_OK

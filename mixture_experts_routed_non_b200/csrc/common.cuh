@@ -5,8 +5,11 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <functional>
 
 #include "moe_nonexpand.h"
 
@@ -16,8 +19,8 @@ namespace moe {
 // Workspace header (first 256 bytes of the workspace).
 // ---------------------------------------------------------------------------
 struct WsHeader {
-    uint32_t grid_arrive;  // metadata kernel's grid barrier: CTAs arrived (cleared per call)
-    uint32_t err;      // MOE_DEVERR_* bits of the current call
+    uint32_t reserved0;
+    uint32_t err;      // MOE_DEVERR_* bits of the current call (stored whole by the metadata)
     int32_t P;         // pairs counted on the device
     uint32_t abort;    // nonzero: later kernels of this call skip their work
     uint32_t pad[60];
@@ -36,15 +39,37 @@ constexpr int kGemmStageK = MOE_STAGE_K;  // K per GEMM pipeline stage (64 or 12
 constexpr int kUmmaK = 16;      // K of one tcgen05.mma kind::f16
 constexpr int kStages = 4;      // shared-memory pipeline depth (4 x 48 KB)
 
-// Metadata kernels: tiles of kMetaTileUnit * c slots, at most kMetaMaxTiles tiles.
+// Metadata kernels: tiles of kMetaTileUnit * c slots, at most kMetaMaxTiles tiles,
+// and a histogram table [T, hist_ld] of at most kMetaTableInts entries (every
+// CTA of the scatter kernel reads all of it).
 #ifndef MOE_META_TILE_UNIT
 #define MOE_META_TILE_UNIT 1024
 #endif
 constexpr int kMetaTileUnit = MOE_META_TILE_UNIT;
 constexpr int kMetaMaxTiles = 148;
+constexpr int kMetaTableInts = 32768;
 constexpr int kMetaThreads = 512;
 constexpr int kMetaWarps = kMetaThreads / 32;
 constexpr int kMaxExperts = 1024;
+
+// Row stride of the per-tile histogram table: E rounded up to 4 (16-byte rows).
+inline int meta_hist_ld(int E) { return (E + 3) & ~3; }
+
+// Metadata tiling of NK routing slots over E experts: tiles of kMetaTileUnit * c
+// slots, as few c as keep T <= min(kMetaMaxTiles, kMetaTableInts / hist_ld).
+inline void meta_tiling(int64_t NK, int E, int32_t *tile_slots, int32_t *tiles) {
+    int64_t tmax = kMetaTableInts / meta_hist_ld(E);
+    if (tmax > kMetaMaxTiles) tmax = kMetaMaxTiles;
+    if (tmax < 1) tmax = 1;
+    const int64_t per = (int64_t)kMetaTileUnit * tmax;
+    int64_t c = (NK + per - 1) / per;
+    if (c < 1) c = 1;
+    const int64_t S = (int64_t)kMetaTileUnit * c;
+    int64_t T = (NK + S - 1) / S;
+    if (T < 1) T = 1;
+    *tile_slots = (int32_t)S;
+    *tiles = (int32_t)T;
+}
 
 // Timeout of every pipeline wait (ns of %globaltimer).
 constexpr unsigned long long kWaitTimeoutNs = 4000000000ull;
@@ -65,8 +90,9 @@ struct MetaArgs {
     int64_t p_cap;
     int32_t tiles;        // T
     int32_t tile_slots;   // slots per tile
+    int32_t hist_ld;      // row stride of tile_hist (meta_hist_ld(E))
     WsHeader *hdr;
-    int32_t *tile_hist;   // [T,E]
+    int32_t *tile_hist;   // [T,hist_ld]
     int32_t *tile_valid;  // [T]
     int32_t *tile_err;    // [T]
     int32_t *gemm_tile_off;  // [E+1] prefix of ceil(freq / kTileRows)
@@ -81,12 +107,14 @@ struct GemmArgs {
                               // one box = this CTA's 64 x 128 half of a B stage
     CUtensorMap tmap_out;     // h [P_cap,I] / y [P_cap,H], box 64 columns x 32 rows (stores)
     CUtensorMap tmap_a16;     // down: h as (64, rows, I/64), box 64 x 16 rows x 1 (short segments)
+    CUtensorMap tmap_lo;      // down: y_lo [P_cap,H] uint8, box 64 columns x 32 rows, 64-byte swizzle (stores)
     const __nv_bfloat16 *x;   // up: x [N,H], rows gathered with cp.async
     const int32_t *x_gather_idx;
     const int32_t *expert_off;    // [E+1]
     const int32_t *tile_off;      // [E+1]
     const __nv_bfloat16 *bias;    // b1 [E,2I] / b2 [E,H] or null
     __nv_bfloat16 *out;           // h [P_cap,I] / y [P_cap,H]
+    uint8_t *out_lo;              // down: y_lo [P_cap,H], e5m2 residual of each stored y element
     float *z_out;                 // up, training: z [P_cap,2I] fp32 (bias added, W1 column order) or null
     WsHeader *hdr;
     int32_t E;
@@ -134,11 +162,21 @@ struct BwdGemmArgs {
     int32_t layout;            // DH: MOE_LAYOUT_*
 };
 
+// One-time launch set-up per (kernel, device), safe to call from several host
+// threads: the first call for the current device runs `setup` (which may set
+// function attributes and returns an integer, e.g. an occupancy figure) under
+// a lock and caches the integer; later calls return the cached value.
+cudaError_t launch_setup_once(const void *kernel, int *value, const std::function<cudaError_t(int dev, int *value)> &setup);
+
+// Host-side argument checks shared by the entry points (capi.cu).
+int check_routing_sizes(int64_t N, int32_t E, int32_t K, int64_t total_pairs);
+bool ptr_aligned(const void *p, size_t a);
+
 // Launchers (each defined next to its kernel).
 cudaError_t launch_meta(const MetaArgs &a, cudaStream_t s);
 cudaError_t launch_gemm_up(const GemmArgs &a, int max_clusters, cudaStream_t s);
 cudaError_t launch_gemm_down(const GemmArgs &a, int max_clusters, cudaStream_t s);
-cudaError_t launch_combine(const __nv_bfloat16 *y, const int32_t *token_offset, const int32_t *s_rev,
+cudaError_t launch_combine(const __nv_bfloat16 *y, const uint8_t *y_lo, const int32_t *token_offset, const int32_t *s_rev,
                            const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
                            const WsHeader *hdr, int num_sms, cudaStream_t s);
 cudaError_t launch_router(const void *logits, bool bf16, int64_t N, int E, int K, int mode, int32_t *idx, float *w,
@@ -483,6 +521,23 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
            | ((b_mn_major ? 1u : 0u) << 16)       // B major
            | ((static_cast<uint32_t>(N) >> 3) << 17)
            | ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+
+// Residual storage of a bf16-rounded value: r = v - bf16(v) (exact in fp32)
+// rounded to e5m2, whose bits are the top byte of the fp16 with the same value.
+// Two residuals per call: `lo` goes to the low byte of the 16-bit result.
+__device__ __forceinline__ uint32_t e5m2x2_rn(float lo, float hi) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+// Bytes 0,1 (sel = 0x1404) or 2,3 (sel = 0x3424) of `v`, each an e5m2 value,
+// as two floats: byte b becomes the fp16 whose bits are b << 8.
+__device__ __forceinline__ float2 e5m2x2_to_f32(uint32_t v, uint32_t sel) {
+    const uint32_t h = __byte_perm(v, 0u, sel);
+    __half2 h2;
+    memcpy(&h2, &h, sizeof h);
+    return __half22float2(h2);
 }
 
 __device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }

@@ -798,27 +798,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
 
 template <int kMode>
 cudaError_t launch_mode(const BwdGemmArgs &a, int max_ctas, cudaStream_t s) {
-    static int fit_cache[64] = {};
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
+    // once per device: the shared-memory limit, and how many clusters can be
+    // resident at once (one CTA per SM: the shared memory allows no second)
+    int fit = 1;
+    cudaError_t err = launch_setup_once(
+        (const void *)bwd_gemm_kernel<kMode>, &fit, [max_ctas](int, int *v) -> cudaError_t {
+            cudaError_t e = cudaFuncSetAttribute(bwd_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)Roles<kMode>::kSmemBytes);
+            if (e != cudaSuccess) return e;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)(max_ctas & ~1));
+            cfg.blockDim = dim3(Roles<kMode>::kThreads);
+            cfg.dynamicSmemBytes = Roles<kMode>::kSmemBytes;
+            int n = 0;
+            e = cudaOccupancyMaxActiveClusters(&n, bwd_gemm_kernel<kMode>, &cfg);
+            if (e != cudaSuccess) return e;
+            *v = n > 0 ? n : 1;
+            return cudaSuccess;
+        });
     if (err != cudaSuccess) return err;
-    if (dev >= 64) return cudaErrorInvalidDevice;
-    int &fit = fit_cache[dev];
-    if (fit == 0) {
-        err = cudaFuncSetAttribute(bwd_gemm_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   (int)Roles<kMode>::kSmemBytes);
-        if (err != cudaSuccess) return err;
-        // clusters that can be resident at once (one CTA per SM: the shared
-        // memory allows no second)
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)(max_ctas & ~1));
-        cfg.blockDim = dim3(Roles<kMode>::kThreads);
-        cfg.dynamicSmemBytes = Roles<kMode>::kSmemBytes;
-        int n = 0;
-        err = cudaOccupancyMaxActiveClusters(&n, bwd_gemm_kernel<kMode>, &cfg);
-        if (err != cudaSuccess) return err;
-        fit = n > 0 ? n : 1;
-    }
     int clusters = max_ctas / 2;
     if (clusters > fit) clusters = fit;
     if (kMode == kBwdDW) {

@@ -5,29 +5,37 @@
 // s_reverse_scatter_idx, num_activated_expert_per_token_offset, compact
 // router_scores -- and question 3: pairs are numbered in ascending token
 // order).  The sort by expert is a stable counting sort (the segmented-sort
-// recipe of the qwen3_5.py commit notes, steps 1-2) done by one cooperative
-// kernel over T tiles of consecutive slots (T <= number of SMs, one CTA each):
+// recipe of the qwen3_5.py commit notes, steps 1-2) over T tiles of
+// consecutive slots, in two kernels on the caller's stream:
 //
-//   phase A  each warp of a tile owns a contiguous slice of its slots and
-//            counts the experts in it (shared-memory increments into a row of
-//            its own: integer counts, so their order does not matter); the
-//            tile's histogram, valid count and error bits go to the workspace.
-//   barrier  all T CTAs (co-resident by the cooperative launch) meet at a
-//            bounded grid barrier whose counter the host clears per call.
-//   phase B  every CTA reads the whole (small) [T,E] histogram table and
-//            derives the global offsets, its tile's base per expert and its
-//            pair base; its warps' bases follow from the per-warp counts of
-//            phase A; then each warp ranks its slice (match_any finds the
-//            lanes with the same expert, popc(peers & lanes below) orders
-//            them inside each 32-slot step) and writes the outputs.  CTA 0
-//            also writes the histogram, offsets, the GEMM tile table and the
+//   count    one CTA per tile counts the experts of its slots (shared-memory
+//            increments: integer counts, so their order does not matter) and
+//            stores the tile's histogram row, valid count and error bits.
+//            Its first instruction lets the scatter kernel start.
+//   scatter  launched as a programmatic dependent of the count kernel, so
+//            its CTAs start while the counts are still running.  Before it
+//            waits for them, each CTA loads its tile's ids and weights and
+//            ranks every valid slot stably inside the tile: each warp owns a
+//            contiguous slice, match_any groups the lanes of one expert in a
+//            32-slot step, popc(peers & lanes below) orders them, and a
+//            per-warp row of counts in shared memory carries the rank across
+//            steps; a scan over the warps then gives every pair its position
+//            in the tile's expert-sorted order, where its token and pair
+//            index are staged in shared memory.  After the wait (the count
+//            kernel has finished and its stores are visible) the CTA reads
+//            the whole [T,E] histogram table once, derives the global
+//            offsets and its tile's base per expert, and writes: the sorted
+//            arrays as contiguous runs per expert from the staged copy, and
+//            the pair-order arrays and token offsets in slot order.  CTA 0
+//            also writes the histogram, offsets, GEMM tile table and the
 //            call's error word.
 //
-// Every result is a pure function of the input (no atomic decides an order;
-// the grid barrier is a GPU-scope release add polled with acquire loads),
-// so the output is bit-exact and deterministic.  Each lane keeps kV slots in
-// flight; the first kWarpChunk slots of every warp, and their weights, stay in
-// registers from phase A to phase B.
+// Every result is a pure function of the input (no atomic decides an order),
+// so the output is bit-exact and deterministic.  Nothing waits on a flag: the
+// only dependency between CTAs is the kernel boundary, so no counter has to be
+// cleared between calls and no wait can hang.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -35,26 +43,31 @@ namespace moe {
 namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
-constexpr int kV = 8;                     // slots per lane per step
-constexpr int kWarpChunk = 32 * kV;       // slots per warp step
-constexpr unsigned long long kGridBarrierTimeoutNs = 1000000000ull;
-static_assert(kMetaMaxTiles < kMetaThreads, "phase B reads one tile's counts per thread");
+constexpr int kCountThreads = 256;
+constexpr int kCountUnroll = 8;                         // ids in flight per thread of the count kernel
+constexpr int kChunk = 4096;                            // slots staged per pass of the scatter kernel
+constexpr int kStepMax = kChunk / (32 * kMetaWarps);    // 32-slot steps per warp and pass (8)
+constexpr int kPartInts = 2 * 4 * kMetaThreads;         // table partial sums: 2 x G x hist_ld, G*hist_ld <= 4*512
+static_assert(kPartInts % 4 == 0, "the arrays after the partial sums start 16-byte aligned");
 
-// The grid barrier's arrival: a GPU-scope release add (the block's earlier
-// writes, ordered before it by __syncthreads, become visible with it) and an
-// acquire load for the polling.
-__device__ __forceinline__ void red_add_release_gpu(uint32_t *p, uint32_t v) {
-    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+// Programmatic dependent launch (sm_90+): the primary lets its dependent
+// start; the dependent waits until the primary grid has completed and its
+// memory operations are visible.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ int4 ld_cg_int4(const int *p) {
+    int4 v;
+    asm volatile("ld.global.cg.v4.s32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
     return v;
 }
 
 // Exclusive scan of n ints in shared memory (in place allowed) by the whole
-// block; returns the total.
+// 512-thread block; returns the total.
 __device__ int block_exclusive_scan(const int *in, int *out, int n) {
     __shared__ int warp_tot[kMetaWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -91,12 +104,11 @@ __device__ int block_exclusive_scan(const int *in, int *out, int n) {
     return carry;
 }
 
-// Sum over the block of one int per thread.
+// Sum over the 512-thread block of one int per thread.
 __device__ int block_sum(int v) {
     __shared__ int part[kMetaWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    v = (int)__reduce_add_sync(kFull, (unsigned)v);
     if (lane == 0) part[warp] = v;
     __syncthreads();
     int t = 0;
@@ -123,15 +135,6 @@ __device__ __forceinline__ long long load_id_wide(const void *ids, int s) {
     return kIdx64 ? __ldg(static_cast<const long long *>(ids) + s) : (long long)__ldg(static_cast<const int *>(ids) + s);
 }
 
-template <bool kIdx64>
-__device__ __forceinline__ void load_chunk(const void *ids, int base, int end, int lane, int (&e)[kV]) {
-#pragma unroll
-    for (int v = 0; v < kV; ++v) {
-        const int s = base + 32 * v + lane;
-        e[v] = s < end ? load_id<kIdx64>(ids, s) : -1;
-    }
-}
-
 // Token of slot s: s / K for the [N,K] table, token_idx[s] for a pair list.
 template <bool kPairs, bool kIdx64>
 __device__ __forceinline__ int slot_token(const MetaArgs &a, int s) {
@@ -151,175 +154,319 @@ __device__ __forceinline__ bool slot_valid(const MetaArgs &a, int e, int t, unsi
     return e_ok;
 }
 
-// Shared memory (ints): cnt[kMetaWarps][E] | part_all[kPartInts] | part_before[kPartInts]
-//                       | off[kMaxExperts+1] | gt[kMaxExperts+1]
-constexpr int kPartInts = kMaxExperts;   // G*E <= max(kMetaThreads, E) <= kMaxExperts
-
+// ---------------------------------------------------------------------------
+// count: tile histogram, valid count and error bits
+// ---------------------------------------------------------------------------
 template <bool kPairs, bool kIdx64>
-__global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a) {
-    extern __shared__ int sm[];
-    const int E = a.E, K = a.K, T = a.tiles;
-    int *cnt = sm;
-    int *part_all = cnt + kMetaWarps * E;
-    int *part_before = part_all + kPartInts;
-    int *off = part_before + kPartInts;
-    int *gt = off + (kMaxExperts + 1);
-    __shared__ int wq[kMetaWarps];
+__global__ void __launch_bounds__(kCountThreads) meta_count_kernel(const MetaArgs a) {
+    pdl_launch_dependents();
+    extern __shared__ int hist[];  // [hist_ld]
     __shared__ unsigned s_err;
-    __shared__ int s_bar_ok;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t lt = lanemask_lt();
-    const int tile = blockIdx.x;
-
-    // this warp's contiguous slice of the tile
-    const int s0 = tile * a.tile_slots;
-    const int s1 = (int)min((int64_t)s0 + a.tile_slots, a.NK);
-    const int sub = a.tile_slots / kMetaWarps;
-    const int w0 = s0 + warp * sub;
-    const int w1 = min(w0 + sub, s1);
-    int ev0[kV], tv0[kV];
-    float wv0[kV];  // kept for phase B; an invalid slot's weight is never written
-    load_chunk<kIdx64>(a.topk_idx, w0, w1, lane, ev0);
-#pragma unroll
-    for (int v = 0; v < kV; ++v) {
-        const int s = w0 + 32 * v + lane;
-        wv0[v] = s < w1 ? __ldg(a.topk_w + s) : 0.f;
-        tv0[v] = (kPairs && s < w1) ? slot_token<kPairs, kIdx64>(a, s) : 0;
+    __shared__ int s_valid;
+    for (int e = threadIdx.x; e < a.hist_ld; e += kCountThreads) hist[e] = 0;
+    if (threadIdx.x == 0) {
+        s_err = 0;
+        s_valid = 0;
     }
-    for (int i = threadIdx.x; i < kMetaWarps * E; i += kMetaThreads) cnt[i] = 0;
-    if (threadIdx.x == 0) s_err = 0;
     __syncthreads();
-
-    // ---- phase A: per-warp expert counts of the slice
-    int *mycnt = cnt + warp * E;
+    const int s0 = blockIdx.x * a.tile_slots;
+    const int s1 = (int)min((int64_t)s0 + a.tile_slots, a.NK);
+    unsigned err = 0;
     int nvalid = 0;
-    unsigned my_err = 0;
-    for (int base = w0; base < w1; base += kWarpChunk) {
-        int ev[kV], tv[kV];
-        if (base == w0) {
+    for (int base = s0; base < s1; base += kCountUnroll * kCountThreads) {
+        int e[kCountUnroll], t[kCountUnroll];
 #pragma unroll
-            for (int v = 0; v < kV; ++v) {
-                ev[v] = ev0[v];
-                tv[v] = tv0[v];
-            }
-        } else {
-            load_chunk<kIdx64>(a.topk_idx, base, w1, lane, ev);
-#pragma unroll
-            for (int v = 0; v < kV; ++v) {
-                const int s = base + 32 * v + lane;
-                tv[v] = (kPairs && s < w1) ? slot_token<kPairs, kIdx64>(a, s) : 0;
-            }
+        for (int u = 0; u < kCountUnroll; ++u) {
+            const int s = base + u * kCountThreads + threadIdx.x;
+            e[u] = s < s1 ? load_id<kIdx64>(a.topk_idx, s) : -1;
+            t[u] = (kPairs && s < s1) ? load_id<kIdx64>(a.token_idx, s) : 0;
         }
 #pragma unroll
-        for (int v = 0; v < kV; ++v) {
-            const int e = ev[v];
-            const bool valid = slot_valid<kPairs>(a, e, tv[v], &my_err);
-            if (kPairs) {  // a pair list must be in ascending token order
-                const int s = base + 32 * v + lane;
-                if (s > 0 && s < w1 &&
-                    load_id_wide<kIdx64>(a.token_idx, s - 1) > load_id_wide<kIdx64>(a.token_idx, s))
-                    my_err |= MOE_DEVERR_BAD_TOKEN;
-            }
-            if (valid) {  // integer counts: the order of the atomics does not matter
-                atomicAdd(&mycnt[e], 1);
+        for (int u = 0; u < kCountUnroll; ++u) {
+            const int s = base + u * kCountThreads + threadIdx.x;
+            if (kPairs && s > 0 && s < s1 &&
+                load_id_wide<kIdx64>(a.token_idx, s - 1) > load_id_wide<kIdx64>(a.token_idx, s))
+                err |= MOE_DEVERR_BAD_TOKEN;  // a pair list must be in ascending token order
+            if (slot_valid<kPairs>(a, e[u], t[u], &err)) {
+                atomicAdd(&hist[e[u]], 1);
                 ++nvalid;
             }
         }
     }
     nvalid = (int)__reduce_add_sync(kFull, (unsigned)nvalid);
-    if (lane == 0) wq[warp] = nvalid;
-    if (my_err) atomicOr(&s_err, my_err);
+    err = __reduce_or_sync(kFull, err);
+    if ((threadIdx.x & 31) == 0) {
+        if (nvalid) atomicAdd(&s_valid, nvalid);
+        if (err) atomicOr(&s_err, err);
+    }
     __syncthreads();
-    // tile histogram = sum of the warps' rows
-    int *th = a.tile_hist + (size_t)tile * E;
+    int *row = a.tile_hist + (size_t)blockIdx.x * a.hist_ld;
+    for (int e = threadIdx.x; e < a.hist_ld; e += kCountThreads) row[e] = hist[e];
+    if (threadIdx.x == 0) {
+        a.tile_valid[blockIdx.x] = s_valid;
+        a.tile_err[blockIdx.x] = (int)s_err;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// scatter: stable positions and every output array
+// ---------------------------------------------------------------------------
+
+// One pass's slots in registers: lane `lane` of warp `warp` holds slot
+// c0 + warp * slice + 32 v + lane for step v.
+struct PassRegs {
+    int e[kStepMax];    // expert, -1 for a slot that is no pair (or past the end)
+    int tok[kStepMax];  // token of the slot
+    float w[kStepMax];  // weight of the slot
+    int pos[kStepMax];  // rank among the warp's earlier pairs of its expert, then position in the pass's sorted order
+    int qv[kStepMax];   // valid slots before this one in the pass (its pair index within the pass if valid)
+};
+
+// Shared memory of the scatter kernel (ints), from a 16-byte aligned base:
+//   part [kPartInts]       column sums of the histogram table (all tiles / earlier tiles),
+//                          stored as int4: first, so that every row stays 16-byte aligned
+//   wrow [kMetaWarps][E]   per-warp expert counts, then the warps' bases inside the pass
+//   coff [E+1]             the pass's expert offsets (exclusive scan of its counts); [E] = its pairs
+//   gbase[E]               global position of each expert's next pair of this tile
+//   dlt  [E]               gbase - coff for the pass being written
+//   stok, sq, se [kChunk]  token, pair index in the pass and expert by position in the pass
+struct ScatterSmem {
+    int *wrow, *coff, *gbase, *dlt, *stok, *sq, *se, *part;
+};
+
+__host__ __device__ inline size_t scatter_smem_ints(int E) {
+    return (size_t)kMetaWarps * E + (E + 1) + 2 * E + 3 * kChunk + kPartInts;
+}
+
+__device__ __forceinline__ ScatterSmem scatter_smem(int *sm, int E) {
+    ScatterSmem m;
+    m.part = sm;
+    m.wrow = m.part + kPartInts;
+    m.coff = m.wrow + kMetaWarps * E;
+    m.gbase = m.coff + (E + 1);
+    m.dlt = m.gbase + E;
+    m.stok = m.dlt + E;
+    m.sq = m.stok + kChunk;
+    m.se = m.sq + kChunk;
+    return m;
+}
+
+// Slice of each warp in a pass of L slots: a multiple of 32, at most 32 * kStepMax.
+__device__ __forceinline__ int pass_slice(int L) {
+    return ((L + 32 * kMetaWarps - 1) / (32 * kMetaWarps)) * 32;
+}
+
+// Loads the slots [c0, c1) and gives every pair its position inside the
+// pass's expert-sorted order; stages (token, pair index in the pass, expert)
+// at that position.  Inputs only: runs before the wait on the count kernel.
+// Returns the pass's pair count (all threads).
+template <bool kPairs, bool kIdx64>
+__device__ int rank_pass(const MetaArgs &a, const ScatterSmem &m, int c0, int c1, PassRegs &r) {
+    __shared__ int s_wv[kMetaWarps];
+    const int E = a.E;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t lt = lanemask_lt();
+    const int slice = pass_slice(c1 - c0);
+    const int w0 = c0 + warp * slice;
+    const int w1 = min(w0 + slice, c1);
+    int *myrow = m.wrow + warp * E;
+#pragma unroll
+    for (int v = 0; v < kStepMax; ++v) {
+        const int s = w0 + 32 * v + lane;
+        const bool in = s < w1;
+        r.e[v] = in ? load_id<kIdx64>(a.topk_idx, s) : -1;
+        r.w[v] = in ? __ldg(a.topk_w + s) : 0.f;
+        r.tok[v] = in ? slot_token<kPairs, kIdx64>(a, s) : 0;
+    }
+    for (int e = lane; e < E; e += 32) myrow[e] = 0;
+    __syncwarp();
+    int q_run = 0;
+#pragma unroll
+    for (int v = 0; v < kStepMax; ++v) {
+        if (32 * v >= slice) break;  // uniform over the block
+        unsigned ignore = 0;
+        const bool valid = slot_valid<kPairs>(a, r.e[v], r.tok[v], &ignore);
+        if (!valid) r.e[v] = -1;
+        const unsigned peers = __match_any_sync(kFull, r.e[v]);
+        const int before = valid ? myrow[r.e[v]] : 0;
+        __syncwarp();
+        if (valid && lane == __ffs(peers) - 1) myrow[r.e[v]] = before + __popc(peers);
+        __syncwarp();
+        r.pos[v] = before + __popc(peers & lt);
+        const unsigned vb = __ballot_sync(kFull, valid);
+        r.qv[v] = q_run + __popc(vb & lt);
+        q_run += __popc(vb);
+    }
+    if (lane == 0) s_wv[warp] = q_run;
+    __syncthreads();
+    // per expert: the warps' bases inside the pass, and the pass's count
     for (int e = threadIdx.x; e < E; e += kMetaThreads) {
-        int sum = 0;
-        for (int w = 0; w < kMetaWarps; ++w) sum += cnt[w * E + e];
-        th[e] = sum;
-    }
-    if (threadIdx.x == 0) {
-        int v = 0;
-        for (int w = 0; w < kMetaWarps; ++w) v += wq[w];
-        a.tile_valid[tile] = v;
-        a.tile_err[tile] = (int)s_err;
-    }
-
-    // ---- grid barrier (bounded)
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        red_add_release_gpu(&a.hdr->grid_arrive, 1u);
-        const uint64_t t0 = globaltimer_ns();
-        int ok = 1;
-        while (ld_acquire_gpu(&a.hdr->grid_arrive) < (uint32_t)T) {
-            if (globaltimer_ns() - t0 > kGridBarrierTimeoutNs) {
-                ok = 0;
-                break;
-            }
-        }
-        s_bar_ok = ok;
-    }
-    __syncthreads();
-    if (!s_bar_ok) {
-        if (threadIdx.x == 0) {
-            atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);
-            a.hdr->abort = 1u;
-        }
-        return;
-    }
-
-    // ---- phase B.1: global column sums and this tile's column prefix.  T is at
-    // most kMetaMaxTiles < kMetaThreads, so one thread reads each tile's valid
-    // count and error bits; they are issued before the histogram table loads.
-    const int tq = threadIdx.x;
-    const int tv_before = (tq < T && tq < tile) ? __ldcg(a.tile_valid + tq) : 0;
-    const unsigned terr = (tile == 0 && tq < T) ? (unsigned)__ldcg(a.tile_err + tq) : 0u;
-    int G = E <= kMetaThreads ? kMetaThreads / E : 1;
-    if (G > T) G = T;
-    for (int i = threadIdx.x; i < G * E; i += kMetaThreads) {
-        const int g = i / E, e = i - g * E;
-        int all = 0, before = 0;
-        for (int t0 = g; t0 < T; t0 += 8 * G) {
-            int v[8];
+        int run = 0;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int t = t0 + u * G;
-                v[u] = t < T ? __ldcg(a.tile_hist + (size_t)t * E + e) : 0;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                all += v[u];
-                if (t0 + u * G < tile) before += v[u];
-            }
+        for (int w = 0; w < kMetaWarps; ++w) {
+            const int c = m.wrow[w * E + e];
+            m.wrow[w * E + e] = run;
+            run += c;
         }
-        part_all[i] = all;
-        part_before[i] = before;
+        m.coff[e] = run;
     }
+    if (warp == 0) {  // the warps' pair bases inside the pass
+        int x = lane < kMetaWarps ? s_wv[lane] : 0;
+        const int own = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane < kMetaWarps) s_wv[lane] = x - own;
+    }
+    __syncthreads();  // the counts in coff are complete before the scan reads them
+    const int npairs = block_exclusive_scan(m.coff, m.coff, E);
+    if (threadIdx.x == 0) m.coff[E] = npairs;
+    const int qw = s_wv[warp];
+#pragma unroll
+    for (int v = 0; v < kStepMax; ++v) {
+        if (32 * v >= slice) break;
+        r.qv[v] += qw;
+        const int e = r.e[v];
+        if (e >= 0) {
+            const int p = m.coff[e] + m.wrow[warp * E + e] + r.pos[v];
+            r.pos[v] = p;
+            m.stok[p] = r.tok[v];
+            m.sq[p] = r.qv[v];
+            m.se[p] = e;
+        }
+    }
+    __syncthreads();
+    return npairs;
+}
+
+// Writes one pass's outputs: qbase = pairs before the pass, m.gbase = the
+// global position of each expert's first pair in the pass (advanced here to
+// the next pass).
+template <bool kPairs, bool kIdx64>
+__device__ void write_pass(const MetaArgs &a, const ScatterSmem &m, int c0, int c1, int qbase, int npairs,
+                           const PassRegs &r) {
+    const int E = a.E, K = a.K;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int e = threadIdx.x; e < E; e += kMetaThreads) {
+        const int gb = m.gbase[e], cf = m.coff[e];
+        m.dlt[e] = gb - cf;
+        m.gbase[e] = gb + (m.coff[e + 1] - cf);
+    }
+    __syncthreads();
+    // sorted order: runs of consecutive positions per expert
+    for (int j = threadIdx.x; j < npairs; j += kMetaThreads) {
+        const int p = j + m.dlt[m.se[j]];
+        a.meta.x_gather_idx[p] = m.stok[j];
+        a.meta.s_scatter_idx[p] = qbase + m.sq[j];
+    }
+    // pair order and token offsets, in slot order
+    const int slice = pass_slice(c1 - c0);
+    const int w0 = c0 + warp * slice;
+    const int w1 = min(w0 + slice, c1);
+#pragma unroll
+    for (int v = 0; v < kStepMax; ++v) {
+        if (32 * v >= slice) break;
+        const int s = w0 + 32 * v + lane;
+        if (s >= w1) continue;
+        const int q = qbase + r.qv[v];
+        const int e = r.e[v];
+        if (e >= 0) {
+            a.meta.s_reverse_scatter_idx[q] = r.pos[v] + m.dlt[e];
+            a.meta.scores[q] = r.w[v];
+        }
+        if (a.slot_pair) a.slot_pair[s] = e >= 0 ? q : -1;  // training: slot -> pair
+        if (!kPairs) {
+            if (s - r.tok[v] * K == 0) a.meta.token_offset[r.tok[v]] = q;
+        } else {
+            // tokens (previous slot's token, this slot's token] start at q
+            // (an order violation is flagged by the count kernel; offsets then unspecified)
+            const int t = r.tok[v];
+            const int tprev = s > 0 ? slot_token<kPairs, kIdx64>(a, s - 1) : -1;
+            const int64_t lo = max((int64_t)tprev + 1, (int64_t)0);
+            const int64_t hi = min((int64_t)t, a.N - 1);
+            for (int64_t tt = lo; tt <= hi; ++tt) a.meta.token_offset[tt] = q;
+        }
+    }
+}
+
+template <bool kPairs, bool kIdx64>
+__global__ void __launch_bounds__(kMetaThreads, 1) meta_scatter_kernel(const MetaArgs a) {
+    extern __shared__ __align__(16) int sm[];
+    __shared__ unsigned s_err;
+    const int E = a.E, T = a.tiles, tile = blockIdx.x, ld = a.hist_ld;
+    const ScatterSmem m = scatter_smem(sm, E);
+    const int t0 = tile * a.tile_slots;
+    const int t1 = (int)min((int64_t)t0 + a.tile_slots, a.NK);
     if (threadIdx.x == 0) s_err = 0;
-    __syncthreads();
+
+    // ---- first pass: inputs only, overlapping the count kernel
+    PassRegs r;
+    int c0 = t0;
+    int c1 = min(c0 + kChunk, t1);
+    int npairs = rank_pass<kPairs, kIdx64>(a, m, c0, c1, r);
+
+    // ---- the count kernel has finished: read its table once
+    pdl_wait();
+    const int ld4 = ld >> 2;
+    const int G = min(kMetaThreads / ld4 > 0 ? kMetaThreads / ld4 : 1, T);
+    int *part_all = m.part;
+    int *part_before = m.part + G * ld;
+    const int tid = threadIdx.x;
+    const unsigned terr = (tile == 0 && tid < T) ? (unsigned)__ldcg(a.tile_err + tid) : 0u;
+    if (tid < G * ld4) {
+        const int g = tid / ld4, c4 = tid - (tid / ld4) * ld4;
+        int4 all = make_int4(0, 0, 0, 0), bef = make_int4(0, 0, 0, 0);
+        for (int tb = g; tb < T; tb += 8 * G) {
+            int4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int t = tb + u * G;
+                v[u] = t < T ? ld_cg_int4(a.tile_hist + (size_t)t * ld + 4 * c4) : make_int4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                all.x += v[u].x; all.y += v[u].y; all.z += v[u].z; all.w += v[u].w;
+                if (tb + u * G < tile) {
+                    bef.x += v[u].x; bef.y += v[u].y; bef.z += v[u].z; bef.w += v[u].w;
+                }
+            }
+        }
+        *reinterpret_cast<int4 *>(part_all + g * ld + 4 * c4) = all;
+        *reinterpret_cast<int4 *>(part_before + g * ld + 4 * c4) = bef;
+    }
     if (terr) atomicOr(&s_err, terr);
-    for (int e = threadIdx.x; e < E; e += kMetaThreads) {
+    __syncthreads();
+    int before_sum = 0;
+    for (int e = tid; e < E; e += kMetaThreads) {
         int all = 0, before = 0;
         for (int g = 0; g < G; ++g) {
-            all += part_all[g * E + e];
-            before += part_before[g * E + e];
+            all += part_all[g * ld + e];
+            before += part_before[g * ld + e];
         }
-        off[e] = all;             // scanned below
-        part_before[e] = before;  // this tile's prefix per expert (rows g > 0 no longer needed)
-        gt[e] = (all + kTileRows - 1) / kTileRows;
+        m.gbase[e] = all;          // scanned below
+        m.dlt[e] = before;         // this tile's pairs before it, per expert
+        before_sum += before;
     }
     __syncthreads();
-    const int P = block_exclusive_scan(off, off, E);
-    const int pbase = block_sum(tv_before);
+    const int P = block_exclusive_scan(m.gbase, m.gbase, E);
+    int qbase = block_sum(before_sum);  // pairs of the earlier tiles
     const bool abort = (int64_t)P > a.p_cap;
 
     if (tile == 0) {
-        const int GT = block_exclusive_scan(gt, gt, E);
-        for (int e = threadIdx.x; e < E; e += kMetaThreads) {
-            a.meta.expert_frequency[e] = (e + 1 < E ? off[e + 1] : P) - off[e];
-            a.meta.expert_frequency_offset[e] = off[e];
-            a.gemm_tile_off[e] = gt[e];
+        // histogram, offsets and the GEMM tile table: freq is the step of the offsets
+        int *gt = part_all;  // the partial sums are no longer needed
+        for (int e = tid; e < E; e += kMetaThreads) {
+            const int f = (e + 1 < E ? m.gbase[e + 1] : P) - m.gbase[e];
+            a.meta.expert_frequency[e] = f;
+            a.meta.expert_frequency_offset[e] = m.gbase[e];
+            gt[e] = (f + kTileRows - 1) / kTileRows;
         }
-        if (threadIdx.x == 0) {
+        __syncthreads();
+        const int GT = block_exclusive_scan(gt, gt, E);
+        for (int e = tid; e < E; e += kMetaThreads) a.gemm_tile_off[e] = gt[e];
+        if (tid == 0) {
             unsigned err = s_err;
             if (a.total_pairs >= 0 && (int64_t)P != a.total_pairs) err |= MOE_DEVERR_PAIR_COUNT;
             if (abort) err |= MOE_DEVERR_PAIR_COUNT | MOE_DEVERR_ABORTED;
@@ -334,123 +481,59 @@ __global__ void __launch_bounds__(kMetaThreads, 1) meta_kernel(const MetaArgs a)
             // tokens after the last listed token (all tokens if the list is empty)
             int last = a.NK > 0 ? slot_token<kPairs, kIdx64>(a, (int)a.NK - 1) : -1;
             if (last < -1) last = -1;
-            for (int64_t tt = (int64_t)last + 1 + threadIdx.x; tt < a.N; tt += kMetaThreads)
-                a.meta.token_offset[tt] = P;
+            for (int64_t tt = (int64_t)last + 1 + tid; tt < a.N; tt += kMetaThreads) a.meta.token_offset[tt] = P;
         }
     }
     if (abort) return;  // the pair arrays are too small for the pairs seen
-
-    // ---- phase B.2: bases: global offset + earlier tiles + earlier warps
-    for (int e = threadIdx.x; e < E; e += kMetaThreads) {
-        int run = off[e] + part_before[e];
-        for (int w = 0; w < kMetaWarps; ++w) {
-            const int c = cnt[w * E + e];
-            cnt[w * E + e] = run;
-            run += c;
-        }
-    }
-    if (threadIdx.x == 0) {
-        int run = pbase;
-        for (int w = 0; w < kMetaWarps; ++w) {
-            const int c = wq[w];
-            wq[w] = run;
-            run += c;
-        }
-    }
+    for (int e = tid; e < E; e += kMetaThreads) m.gbase[e] += m.dlt[e];
     __syncthreads();
 
-    // ---- phase B.3: positions, in slot order
-    int q_run = wq[warp];
-    for (int base = w0; base < w1; base += kWarpChunk) {
-        int ev[kV], tv[kV];
-        float wv[kV];
-        if (base == w0) {
-#pragma unroll
-            for (int v = 0; v < kV; ++v) {
-                ev[v] = ev0[v];
-                tv[v] = tv0[v];
-                wv[v] = wv0[v];
-            }
-        } else {
-            load_chunk<kIdx64>(a.topk_idx, base, w1, lane, ev);
-#pragma unroll
-            for (int v = 0; v < kV; ++v) {
-                const int s = base + 32 * v + lane;
-                wv[v] = s < w1 ? __ldg(a.topk_w + s) : 0.f;
-                tv[v] = (kPairs && s < w1) ? slot_token<kPairs, kIdx64>(a, s) : 0;
-            }
-        }
-#pragma unroll
-        for (int v = 0; v < kV; ++v) {
-            const int s = base + 32 * v + lane;
-            const int e = ev[v];
-            unsigned ignore = 0;
-            const bool valid = slot_valid<kPairs>(a, e, tv[v], &ignore);
-            const unsigned peers = __match_any_sync(kFull, valid ? e : -1);
-            const int pb = valid ? mycnt[e] : 0;
-            __syncwarp();
-            if (valid && lane == __ffs(peers) - 1) mycnt[e] = pb + __popc(peers);
-            const unsigned vb = __ballot_sync(kFull, valid);
-            const int q = q_run + __popc(vb & lt);
-            if (valid) {
-                const int p = pb + __popc(peers & lt);
-                a.meta.x_gather_idx[p] = kPairs ? tv[v] : s / K;
-                a.meta.s_scatter_idx[p] = q;
-                a.meta.s_reverse_scatter_idx[q] = p;
-                a.meta.scores[q] = wv[v];
-            }
-            if (s < w1) {
-                if (a.slot_pair) a.slot_pair[s] = valid ? q : -1;  // training: slot -> pair
-                if (!kPairs) {
-                    if ((s % K) == 0) a.meta.token_offset[s / K] = q;
-                } else {
-                    // tokens (previous slot's token, this slot's token] start at q
-                    // (an order violation was flagged in phase A; offsets then unspecified)
-                    const int t = tv[v];
-                    const int tprev = s > 0 ? slot_token<kPairs, kIdx64>(a, s - 1) : -1;
-                    const int64_t lo = max((int64_t)tprev + 1, (int64_t)0);
-                    const int64_t hi = min((int64_t)t, a.N - 1);
-                    for (int64_t tt = lo; tt <= hi; ++tt) a.meta.token_offset[tt] = q;
-                }
-            }
-            q_run += __popc(vb);
-            __syncwarp();
-        }
+    // ---- write the passes
+    for (;;) {
+        write_pass<kPairs, kIdx64>(a, m, c0, c1, qbase, npairs, r);
+        qbase += npairs;
+        c0 = c1;
+        if (c0 >= t1) break;
+        c1 = min(c0 + kChunk, t1);
+        __syncthreads();  // the staged copy is read before the next pass overwrites it
+        npairs = rank_pass<kPairs, kIdx64>(a, m, c0, c1, r);
     }
 }
 
 }  // namespace
 
-size_t meta_smem_bytes(int E) {
-    return ((size_t)kMetaWarps * E + 2 * kPartInts + 2 * (kMaxExperts + 1)) * sizeof(int);
-}
+size_t meta_smem_bytes(int E) { return scatter_smem_ints(E) * sizeof(int); }
 
 template <bool kPairs, bool kIdx64>
-cudaError_t launch_meta_as(const MetaArgs &a, cudaStream_t s, int dev) {
-    static bool configured[64] = {};
-    if (dev < 64 && !configured[dev]) {
-        const cudaError_t err = cudaFuncSetAttribute(meta_kernel<kPairs, kIdx64>,
-                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     (int)meta_smem_bytes(kMaxExperts));
-        if (err != cudaSuccess) return err;
-        configured[dev] = true;
-    }
-    MetaArgs args = a;
-    void *params[] = {&args};
-    // cooperative: all T CTAs are resident at once, so the grid barrier ends
-    return cudaLaunchCooperativeKernel((const void *)meta_kernel<kPairs, kIdx64>, dim3(a.tiles),
-                                       dim3(kMetaThreads), params, meta_smem_bytes(a.E), s);
+cudaError_t launch_meta_as(const MetaArgs &a, cudaStream_t s) {
+    int unused = 0;
+    cudaError_t err = launch_setup_once(
+        (const void *)meta_scatter_kernel<kPairs, kIdx64>, &unused, [](int, int *v) -> cudaError_t {
+            *v = 1;
+            return cudaFuncSetAttribute(meta_scatter_kernel<kPairs, kIdx64>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)meta_smem_bytes(kMaxExperts));
+        });
+    if (err != cudaSuccess) return err;
+    meta_count_kernel<kPairs, kIdx64><<<a.tiles, kCountThreads, (size_t)a.hist_ld * sizeof(int), s>>>(a);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)a.tiles);
+    cfg.blockDim = dim3(kMetaThreads);
+    cfg.dynamicSmemBytes = meta_smem_bytes(a.E);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, meta_scatter_kernel<kPairs, kIdx64>, a);
 }
 
 cudaError_t launch_meta(const MetaArgs &a, cudaStream_t s) {
-    int dev = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err != cudaSuccess) return err;
-    // the grid barrier's arrival counter starts from zero in every call
-    err = cudaMemsetAsync(&a.hdr->grid_arrive, 0, sizeof(a.hdr->grid_arrive), s);
-    if (err != cudaSuccess) return err;
-    if (a.pair_list) return a.idx64 ? launch_meta_as<true, true>(a, s, dev) : launch_meta_as<true, false>(a, s, dev);
-    return a.idx64 ? launch_meta_as<false, true>(a, s, dev) : launch_meta_as<false, false>(a, s, dev);
+    if (a.pair_list) return a.idx64 ? launch_meta_as<true, true>(a, s) : launch_meta_as<true, false>(a, s);
+    return a.idx64 ? launch_meta_as<false, true>(a, s) : launch_meta_as<false, false>(a, s);
 }
 
 }  // namespace moe

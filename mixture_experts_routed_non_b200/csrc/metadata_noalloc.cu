@@ -6,6 +6,8 @@
 // tile table [E+1]).  moe_nonexpand_metadata takes it from a caller workspace;
 // this entry point instead uses one fixed array in device memory that belongs
 // to the library, so it calls no allocator at all.
+#include <stddef.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -13,9 +15,10 @@
 namespace moe {
 namespace {
 
-// Largest scratch any supported size needs: 148 tiles x 1024 experts of
-// histogram (606,208 bytes) + per-tile tables + tile table + header, rounded up.
-constexpr size_t kNoAllocScratchBytes = 640 * 1024;
+// Largest scratch any supported size needs: the histogram table holds at most
+// kMetaTableInts entries (131,072 bytes), plus the per-tile tables of at most
+// 148 tiles, the tile table of E <= 1024 experts and the header, rounded up.
+constexpr size_t kNoAllocScratchBytes = 160 * 1024;
 
 // The scratch.  Every GPU that loads the library holds it until the process
 // exits.  All calls share it and it keeps the last call's contents; the
@@ -29,27 +32,20 @@ struct ScratchLayout {
     int32_t tiles, tile_slots;
 };
 
-// Tiles of kMetaTileUnit * c slots, at most 148 of them (the same rule the workspace
-// path uses).
+// The same tiling as the workspace path (meta_tiling).
 ScratchLayout scratch_layout(int64_t NK, int32_t E) {
     ScratchLayout l;
-    const int64_t per = (int64_t)kMetaTileUnit * kMetaMaxTiles;
-    int64_t c = (NK + per - 1) / per;
-    if (c < 1) c = 1;
-    const int64_t S = (int64_t)kMetaTileUnit * c;
-    int64_t T = (NK + S - 1) / S;
-    if (T < 1) T = 1;
-    l.tiles = (int32_t)T;
-    l.tile_slots = (int32_t)S;
+    meta_tiling(NK, E, &l.tile_slots, &l.tiles);
+    const size_t T = (size_t)l.tiles;
     size_t o = 0;
     l.header = o;
     o = up256(o + sizeof(WsHeader));
     l.hist = o;
-    o = up256(o + (size_t)T * E * 4);
+    o = up256(o + T * meta_hist_ld(E) * 4);
     l.valid = o;
-    o = up256(o + (size_t)T * 4);
+    o = up256(o + T * 4);
     l.err = o;
-    o = up256(o + (size_t)T * 4);
+    o = up256(o + T * 4);
     l.gemm_tiles = o;
     o = up256(o + (size_t)(E + 1) * 4);
     l.total = o;
@@ -92,16 +88,17 @@ using namespace moe;
 extern "C" MOE_API int moe_nonexpand_metadata_noalloc(const int32_t *topk_idx, const float *topk_w, int64_t N,
                                                       int32_t K, int32_t E, int64_t total_pairs,
                                                       const moe_meta_t *meta, moe_stream_t stream) {
-    if (N < 0 || K < 1 || K > 32 || E < 1 || E > kMaxExperts) return MOE_ERR_ARG;
-    if (N * (int64_t)K >= (int64_t)(1u << 31) - (1 << 20)) return MOE_ERR_ARG;
-    if (total_pairs < -1 || total_pairs > N * K) return MOE_ERR_ARG;
+    // the same argument checks as moe_nonexpand_metadata, before any CUDA call
+    int st = check_routing_sizes(N, E, K, total_pairs);
+    if (st != MOE_OK) return st;
     if (N > 0 && (!topk_idx || !topk_w || !meta_fields_set(meta))) return MOE_ERR_ARG;
     if (!meta || !meta->token_offset || !meta->expert_frequency || !meta->expert_frequency_offset)
         return MOE_ERR_ARG;
+    if (!ptr_aligned(topk_idx, 4) || !ptr_aligned(topk_w, 4)) return MOE_ERR_ARG;
     const ScratchLayout l = scratch_layout(N * K, E);
     if (l.total > kNoAllocScratchBytes) return MOE_ERR_WS;  // beyond the fixed scratch
     unsigned char *s = nullptr;
-    const int st = scratch_address(&s);
+    st = scratch_address(&s);
     if (st != MOE_OK) return st;
     MetaArgs a;
     a.topk_idx = topk_idx;
@@ -116,6 +113,7 @@ extern "C" MOE_API int moe_nonexpand_metadata_noalloc(const int32_t *topk_idx, c
     a.p_cap = total_pairs >= 0 ? total_pairs : N * K;
     a.tiles = l.tiles;
     a.tile_slots = l.tile_slots;
+    a.hist_ld = meta_hist_ld(E);
     a.hdr = reinterpret_cast<WsHeader *>(s + l.header);
     a.tile_hist = reinterpret_cast<int32_t *>(s + l.hist);
     a.tile_valid = reinterpret_cast<int32_t *>(s + l.valid);
@@ -125,4 +123,19 @@ extern "C" MOE_API int moe_nonexpand_metadata_noalloc(const int32_t *topk_idx, c
     a.N = N;
     a.slot_pair = nullptr;
     return launch_meta(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" MOE_API int moe_nonexpand_metadata_noalloc_read_error(moe_stream_t stream, uint32_t *err_word) {
+    if (!err_word) return MOE_ERR_ARG;
+    unsigned char *s = nullptr;
+    const int st = scratch_address(&s);  // also checks the device, like the first metadata call
+    if (st != MOE_OK) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_meta_scratch, sizeof v, offsetof(WsHeader, err), cudaMemcpyDeviceToHost,
+                                  cs) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(cs) != cudaSuccess) return MOE_ERR_CUDA;
+    *err_word = v;
+    return MOE_OK;
 }

@@ -108,3 +108,21 @@ def assert_close_bwd(gpu, ref, rss, what=""):
     bad = ~(err <= bound)
     assert not bad.any(), (f"{what}: max_err {err.max():.4g}, rms {rms:.4g}, n_bad {int(bad.sum())}/{err.size}, "
                            f"worst {np.unravel_index(int(np.argmax(err - bound)), err.shape)}")
+
+
+def tile_rows(off, tile=256):
+    """Expert-sorted rows to compare for every (expert, tile-row m-tile) of a
+    run, from the expert offsets [E+1]: each tile's first and last stored row
+    and the rows on both sides of the CTA-pair splits (64 and 128 rows into
+    the tile), so every m-tile -- tail tiles of at most 128 rows included -- and
+    every segment end is checked."""
+    off = np.asarray(off, dtype=np.int64)
+    rows = []
+    for e in range(off.shape[0] - 1):
+        a, b = int(off[e]), int(off[e + 1])
+        for t0 in range(a, b, tile):
+            t1 = min(t0 + tile, b)
+            for r in (t0, t0 + 63, t0 + 64, t0 + 127, t0 + 128, t1 - 1):
+                if t0 <= r < t1:
+                    rows.append(r)
+    return np.unique(np.asarray(rows, dtype=np.int64))

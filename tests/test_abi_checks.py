@@ -139,6 +139,40 @@ def test_metadata_argument_checks(lib):
         assert _meta_call(lib) in NO_DEVICE
 
 
+def _noalloc_call(lib, idx=A, w=A, N=64, K=4, E=8, tp=-1, meta="full"):
+    m = {"full": binding.MoeMeta(*([A] * 7)), "none": None,
+         "no_scores": binding.MoeMeta(*([A] * 6 + [None]))}[meta]
+    return lib.moe_nonexpand_metadata_noalloc(idx, w, N, K, E, tp, ctypes.byref(m) if m is not None else None,
+                                              None)
+
+
+def test_metadata_noalloc_argument_checks(lib):
+    """The no-allocation metadata rejects what the workspace entry point
+    rejects -- sizes, null and misaligned pointers -- before any CUDA call, so
+    a misaligned id or weight pointer never reaches a kernel."""
+    assert _noalloc_call(lib, N=-1) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, K=0) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, K=33) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, E=0) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, E=1025) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, N=1 << 28, K=8) == binding.MOE_ERR_ARG   # N*K beyond 2^31
+    assert _noalloc_call(lib, tp=64 * 4 + 1) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, tp=-2) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, idx=None) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, w=None) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, meta="none") == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, meta="no_scores") == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, idx=A + 1) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, idx=A2) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, w=A + 3) == binding.MOE_ERR_ARG
+    assert _noalloc_call(lib, w=A2) == binding.MOE_ERR_ARG
+    err = ctypes.c_uint32(0)
+    assert lib.moe_nonexpand_metadata_noalloc_read_error(None, None) == binding.MOE_ERR_ARG
+    if _no_device():
+        assert _noalloc_call(lib) in NO_DEVICE
+        assert lib.moe_nonexpand_metadata_noalloc_read_error(None, ctypes.byref(err)) in NO_DEVICE
+
+
 def test_combine_argument_checks(lib):
     meta = binding.MoeMeta(*([A] * 7))
     no_rev = binding.MoeMeta(A, A, A, A, None, A, A)

@@ -92,3 +92,70 @@ def test_clock_summary_window_median_and_reasons():
     assert out["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
     assert bench.ClockSampler(0).summary(0.0, 1.0) == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
                                                         "samples": 0}
+
+
+def test_tensor_peak_follows_the_clock_record():
+    """Burst for a short timed region or one without the power cap; the
+    sustained figure only for a region of seconds whose samples show the cap."""
+    peaks = {"hbm_gbs": 6500.0, "bf16_tflops": 1677.6, "bf16_tflops_sustained": 1391.2}
+    capped = {"reasons": ["sw_power_cap"], "sm_mhz": 1350.0, "sm_max_mhz": 1965.0, "samples": 40}
+    free = {"reasons": [], "sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "samples": 40}
+    assert bench.choose_tensor_peak(peaks, free, 0.023) == (1677.6, "burst")
+    assert bench.choose_tensor_peak(peaks, capped, 0.023) == (1677.6, "burst")
+    assert bench.choose_tensor_peak(peaks, free, 5.0) == (1677.6, "burst")
+    assert bench.choose_tensor_peak(peaks, capped, 5.0) == (1391.2, "sustained")
+    assert bench.choose_tensor_peak(peaks, {"reasons": [], "samples": 0}, 0.02) == (1677.6, "burst")
+
+
+def test_clock_record_widens_to_the_leg_when_the_region_is_short():
+    s = bench.ClockSampler(0)
+    na = "Not Active"
+    s.lines = [(1.00, f"1965, 1965, 500.0, 0x0, {na}, {na}, {na}, {na}"),
+               (1.02, f"1950, 1965, 600.0, 0x0, {na}, {na}, {na}, {na}"),
+               (1.30, f"1965, 1965, 700.0, 0x0, {na}, {na}, {na}, {na}")]
+    c = bench.clocks_for(s, 1.05, 1.07, 0.9, 1.4)          # no sample inside the 20 ms region
+    assert c["window"].startswith("forward leg") and c["samples"] == 3 and c["sm_mhz"] == 1965.0
+    c = bench.clocks_for(s, 1.01, 1.03, 0.9, 1.4)
+    assert c["window"] == "timed region" and c["samples"] == 1 and c["sm_mhz"] == 1950.0
+
+
+def _bench_lines(args, timeout=300):
+    import json
+    import subprocess
+    env = dict(os.environ)
+    env.pop("WORLD_SIZE", None)
+    env.pop("RANK", None)
+    env.pop("LOCAL_RANK", None)
+    env.setdefault("OMP_NUM_THREADS", "1")
+    r = subprocess.run([sys.executable, "bench.py", *args], cwd=ROOT, env=env, capture_output=True, text=True,
+                       timeout=timeout)
+    assert r.returncode == 0, r.stderr[-3000:]
+    return [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` run without a launcher starts two ranks itself
+    (torch.distributed.run, 127.0.0.1); each rank sees WORLD_SIZE 2."""
+    for impl in ("ours", "reference"):
+        lines = _bench_lines(["--gpus", "2", "--check-launch", "--impl", impl])
+        assert sorted(d["rank"] for d in lines) == [0, 1]
+        assert all(d["world"] == 2 and d["impl"] == impl for d in lines)
+
+
+def test_reference_arm_reports_the_ranks_it_ran():
+    lines = _bench_lines(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
+                          "--workload", "tiny", "--ref-seconds", "0.05"])
+    assert len(lines) == 1 and lines[0]["n_gpus"] == 2 and lines[0]["impl"] == "reference"
+
+
+def test_both_arms_share_one_config_object():
+    """The reference arm's config is built by the same function as ours, from
+    the same workload, so the two lines name the same configuration."""
+    import torch  # noqa: F401
+    from mixture_experts_routed_non_b200 import synthetic
+    wl = synthetic.WORKLOADS["tiny"]
+    inp = synthetic.make_inputs(wl, device="cpu")
+    P = int((inp.topk_idx >= 0).sum())
+    lines = _bench_lines(["--impl", "reference", "--steps", "1", "--warmup", "0", "--workload", "tiny",
+                          "--ref-seconds", "0.05"])
+    assert lines[0]["config"] == bench.bench_config(wl, 0, 1, P, (inp.w1.numel() + inp.w2.numel()) * 2)

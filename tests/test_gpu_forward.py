@@ -11,7 +11,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import assert_close, check_meta_equal, to_np, within_tolerance
+from helpers import assert_close, check_meta_equal, tile_rows, to_np, within_tolerance
 from mixture_experts_routed_non_b200 import binding, synthetic
 
 pytestmark = pytest.mark.gpu
@@ -23,7 +23,11 @@ def _concat_from_interleaved(w1, b1):
     return w1c, b1c
 
 
-def run_case(inp, layout=0, total_pairs=-1, sample=None, check_stages=True, seed=0):
+def run_case(inp, layout=0, total_pairs=-1, sample=None, check_stages=True, seed=0, every_tile=False):
+    """Forward of ``inp``; metadata compared bit-exactly, the output on all
+    tokens (or a seeded sample of ``sample`` tokens), and the bf16
+    intermediates h and y on every pair of the compared tokens -- plus, with
+    ``every_tile``, on the boundary rows of every (expert, m-tile) of the run."""
     wl = inp.wl
     N, H, I, E, K = wl.N, wl.H, wl.I, wl.E, wl.K
     w1, b1 = inp.w1, inp.b1
@@ -46,20 +50,31 @@ def run_case(inp, layout=0, total_pairs=-1, sample=None, check_stages=True, seed
     else:
         tokens = np.sort(np.random.default_rng(seed).choice(N, size=min(sample, N), replace=False))
     if check_stages and ref_meta["P"] > 0:
-        # intermediates of the pairs of the sampled tokens
+        # intermediates: every pair of the compared tokens, and the tile boundary rows
         P = ref_meta["P"]
-        h_gpu, y_gpu = binding.intermediates_from_workspace(ws, N, H, I, E, K, total_pairs)
+        h_gpu, y_hi, y_lo = binding.intermediates_from_workspace(ws, N, H, I, E, K, total_pairs,
+                                                                 with_residual=True)
+        assert P <= h_gpu.shape[0]
         to = ref_meta["token_offset"]
-        qs = np.concatenate([np.arange(to[t], to[t + 1]) for t in tokens[:64]] + [np.zeros(0, np.int64)])
-        if qs.size:
-            ps = ref_meta["s_reverse_scatter_idx"][qs]
+        qs = np.concatenate([np.arange(to[t], to[t + 1]) for t in tokens] + [np.zeros(0, np.int64)])
+        ps = ref_meta["s_reverse_scatter_idx"][qs].astype(np.int64)
+        if every_tile:
+            ps = np.union1d(ps, tile_rows(ref_meta["off"]))
+        if ps.size:
             tok = ref_meta["x_gather_idx"][ps]
             ex = np.searchsorted(ref_meta["off"], ps, side="right") - 1
             h_ref, y_ref = oracle.pair_rows(wts, tok, ex, layout=layout)
-            ps_t = torch.from_numpy(ps.astype(np.int64)).to(h_gpu.device)
-            assert_close(to_np(h_gpu[ps_t]), h_ref, "h (up GEMM + SwiGLU)")
-            assert_close(to_np(y_gpu[ps_t]), y_ref, "y (down GEMM)")
-            assert P <= h_gpu.shape[0]
+            ps_t = torch.from_numpy(ps).to(h_gpu.device)
+            assert_close(to_np(h_gpu[ps_t]), h_ref, f"h (up GEMM + SwiGLU, {ps.size} rows)")
+            yh = to_np(y_hi[ps_t]).astype(np.float64)
+            assert_close(yh, y_ref, f"y (down GEMM, bf16 part, {ps.size} rows)")
+            # the rows the combine sums: bf16 part plus its e5m2 rounding residual,
+            # which is at most half a bf16 step (times e5m2's own 1 + 2^-3)
+            lo = to_np(y_lo[ps_t].view(torch.float8_e5m2).float()).astype(np.float64)
+            yr = yh + lo
+            assert_close(yr, y_ref, f"y + residual ({ps.size} rows)")
+            half_step = np.exp2(np.floor(np.log2(np.maximum(np.abs(yh), 1e-30))) - 8)
+            assert np.all(np.abs(lo) <= half_step * 1.125 + 1e-30), "residual above half a bf16 step"
     ref = oracle.forward_rows(wts, idx, w, tokens=tokens, layout=layout)
     got = to_np(out)[tokens]
     assert_close(got, ref, f"out ({wl.name}, layout {layout})")
@@ -149,18 +164,24 @@ def test_bad_ids_flagged_forward_still_right():
 
 
 # ---- full-size workloads (the benchmark's launch configuration) ------------
+# Every (expert, 256-row m-tile) of each run is compared on its boundary rows
+# (tests/helpers.py tile_rows), and the output on a seeded 2048-token subset
+# (all 128 tokens of the decode shape) with h and y on all of their pairs.
 
-@pytest.mark.parametrize("name,sample", [("prefill", 192), ("ranklocal", 48), ("decode256", None),
-                                         ("prefill256", 192)])
-def test_full_size_workloads_sampled(name, sample):
+@pytest.mark.parametrize("name,sample", [("prefill", 2048), ("ranklocal", 2048), ("decode256", None),
+                                         ("prefill256", 2048)])
+def test_full_size_workloads_every_tile(name, sample):
     inp = synthetic.make_inputs(name, device="cuda")
-    run_case(inp, sample=sample, seed=17)
+    run_case(inp, sample=sample, seed=17, every_tile=True)
+    del inp
     torch.cuda.empty_cache()
 
 
-def test_prefill_with_total_pairs_and_concat_layout():
+def test_prefill_with_total_pairs_and_concat_layout_every_tile():
     inp = synthetic.make_inputs("prefill", device="cuda")
-    run_case(inp, layout=1, total_pairs=inp.total_pairs, sample=96, seed=18)
+    run_case(inp, layout=1, total_pairs=inp.total_pairs, sample=2048, seed=18, every_tile=True)
+    del inp
+    torch.cuda.empty_cache()
 
 
 def test_full_size_properties_hold_everywhere():

@@ -37,7 +37,9 @@ def test_metadata_workloads_bit_exact(name):
 @pytest.mark.parametrize("N,K,E,p_invalid,seed", [
     (1, 1, 1, 0.0, 1), (3, 2, 3, 0.3, 2), (37, 3, 5, 0.2, 3), (511, 1, 7, 0.0, 4),
     (513, 8, 64, 0.1, 5), (4097, 5, 1024, 0.05, 6), (1000, 32, 40, 0.5, 7), (2500, 7, 1, 0.3, 8),
-    (9999, 6, 300, 0.0, 9), (200003, 4, 17, 0.01, 10)])
+    (9999, 6, 300, 0.0, 9), (200003, 4, 17, 0.01, 10),
+    # tiles of more than 4096 slots, ranked and written in several passes
+    (70000, 8, 1024, 0.1, 11), (300001, 3, 513, 0.02, 12)])
 def test_metadata_ragged_sizes_bit_exact(N, K, E, p_invalid, seed):
     rng = np.random.default_rng(seed)
     idx = rng.integers(0, E, size=(N, K)).astype(np.int32)   # duplicates within a row allowed
@@ -98,6 +100,23 @@ def test_metadata_pair_count_mismatch_flagged():
     # declared smaller: flagged and the later steps are skipped (no overflow)
     meta, err, _ = run_meta(idx, w, 6, total_pairs=P - 1)
     assert err == binding.DEVERR_PAIR_COUNT | binding.DEVERR_ABORTED
+
+
+def test_error_word_is_rewritten_by_every_call():
+    """A call's error bits do not outlive it: after a call with a bad id, the
+    next good call on the same workspace reports 0."""
+    rng = np.random.default_rng(5)
+    idx = rng.integers(0, 6, size=(500, 4)).astype(np.int32)
+    w = rng.random((500, 4)).astype(np.float32)
+    dev = torch.device("cuda")
+    ws = binding.alloc_workspace(500, 0, 0, 6, 4, -1, dev)
+    bad = idx.copy()
+    bad[7, 1] = 42
+    binding.metadata(torch.from_numpy(bad).to(dev), torch.from_numpy(w).to(dev), 6, ws=ws)
+    assert binding.read_error(ws) == binding.DEVERR_BAD_EXPERT_ID
+    meta = binding.metadata(torch.from_numpy(idx).to(dev), torch.from_numpy(w).to(dev), 6, ws=ws)
+    assert binding.read_error(ws) == 0
+    check_meta_equal(meta, oracle.metadata(idx, w, 6))
 
 
 def test_metadata_deterministic_and_workspace_reusable():

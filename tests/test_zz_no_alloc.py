@@ -64,3 +64,49 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
 def test_noalloc_repeat_same_input_bitwise():
     _compare("prefill256")
     _compare("prefill256")
+
+
+def test_noalloc_reports_device_errors_and_clears_them():
+    """The scratch's error word: a bad expert id and a total_pairs below the
+    real pair count are reported through
+    moe_nonexpand_metadata_noalloc_read_error; the next good call rewrites the
+    word whole, so no bit of an earlier call is reported again."""
+    import oracle
+    from helpers import check_meta_equal
+
+    wl = synthetic.WORKLOADS["tiny"]
+    idx, w = synthetic.make_routing(wl, seed=wl.seed, invalid_value=float("nan"))
+    dev = torch.device("cuda")
+    P = int((idx >= 0).sum())
+
+    bad = idx.copy()
+    bad[3, 0] = 99                     # neither a valid id nor -1: flagged and skipped like -1
+    meta = binding.alloc_meta(wl.N, wl.K, wl.E, -1, dev)
+    binding.metadata_noalloc(torch.from_numpy(bad).to(dev), torch.from_numpy(w).to(dev), wl.E, meta)
+    assert binding.metadata_noalloc_read_error() == binding.DEVERR_BAD_EXPERT_ID
+    check_meta_equal(meta, oracle.metadata(bad, w, wl.E))
+
+    short = binding.alloc_meta(wl.N, wl.K, wl.E, P - 1, dev)
+    binding.metadata_noalloc(torch.from_numpy(idx).to(dev), torch.from_numpy(w).to(dev), wl.E, short,
+                             total_pairs=P - 1)
+    err = binding.metadata_noalloc_read_error()
+    assert err == binding.DEVERR_PAIR_COUNT | binding.DEVERR_ABORTED, hex(err)
+
+    good = binding.alloc_meta(wl.N, wl.K, wl.E, P, dev)
+    binding.metadata_noalloc(torch.from_numpy(idx).to(dev), torch.from_numpy(w).to(dev), wl.E, good,
+                             total_pairs=P)
+    assert binding.metadata_noalloc_read_error() == 0
+    check_meta_equal(good, oracle.metadata(idx, w, wl.E))
+
+
+def test_noalloc_bit_exact_against_the_oracle_at_full_size():
+    import oracle
+    from helpers import check_meta_equal
+
+    wl = synthetic.WORKLOADS["metadata"]   # 65536 x 8, Zipf, 5 % invalid
+    idx, w = synthetic.make_routing(wl, seed=wl.seed + 3)
+    dev = torch.device("cuda")
+    meta = binding.alloc_meta(wl.N, wl.K, wl.E, -1, dev)
+    binding.metadata_noalloc(torch.from_numpy(idx).to(dev), torch.from_numpy(w).to(dev), wl.E, meta)
+    assert binding.metadata_noalloc_read_error() == 0
+    check_meta_equal(meta, oracle.metadata(idx, w, wl.E))
