@@ -55,6 +55,7 @@ cudaError_t launch_setup_once(const void *kernel, int *value,
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr int64_t kDecodeRowsPerExpert = 32;  // decode GEMMs when P_cap <= 32 E
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -316,6 +317,36 @@ bool make_map_b_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A row-major weight [rows][ncols] viewed as (64 columns, rows, ncols/64
+// chunks) with a box of 64 x box_rows x 2: 128 columns of box_rows K rows
+// (the decode GEMMs' MN-major weight operand).
+bool make_map_w_chunks(CUtensorMap *m, const void *ptr, uint64_t ncols, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[3] = {64, rows, ncols / 64};
+    cuuint64_t strides[2] = {ncols * 2, 128};
+    cuuint32_t box[3] = {64, box_rows, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// w1 in the concatenated layout [rows][2][I] viewed as (64 columns, rows, I/64
+// chunks, gate/up half) with a box of 64 x box_rows x 1 x 1: one 64-column
+// chunk of the gate or of the up half (the decode up GEMM loads one of each).
+bool make_map_w1_concat_rows(CUtensorMap *m, const void *ptr, uint64_t I, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn f = encode_fn();
+    if (!f) return false;
+    cuuint64_t dims[4] = {64, rows, I / 64, 2};
+    cuuint64_t strides[3] = {I * 4, 128, I * 2};
+    cuuint32_t box[4] = {64, box_rows, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // h [rows][I] viewed as (64 columns, rows, I/64 column chunks): a box of
 // 64 x 128 rows x (stage K / 64) is one CTA's A stage (64-wide K atoms 16 KB
 // apart); a box of 64 x 16 rows x 1 is one 16-row group of one atom.
@@ -433,7 +464,51 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
     __nv_bfloat16 *hbuf = reinterpret_cast<__nv_bfloat16 *>(w + l.h);
     __nv_bfloat16 *ybuf = reinterpret_cast<__nv_bfloat16 *>(w + l.y);
     uint8_t *ylo = w + l.y_lo;
-    if (l.p_cap > 0) {
+    // Segments of a few rows on average (decode): swap-AB kernels that stream
+    // each active expert's weights once.  Chosen per call from the sizes alone
+    // (no host sync); they handle segments of any length.
+    const bool decode = !train && l.p_cap > 0 && l.p_cap <= (int64_t)kDecodeRowsPerExpert * E;
+    if (decode) {
+        DecodeArgs up;
+        memset(&up, 0, sizeof up);
+        if (layout_kind == MOE_LAYOUT_CONCATENATED) {
+            if (!make_map_w1_concat_rows(&up.tmap_w, w1, (uint64_t)I, (uint64_t)E * H, 64)) return MOE_ERR_CUDA;
+        } else {
+            if (!make_map_w_chunks(&up.tmap_w, w1, (uint64_t)2 * I, (uint64_t)E * H, 64)) return MOE_ERR_CUDA;
+        }
+        up.x = static_cast<const __nv_bfloat16 *>(x);
+        up.x_gather_idx = meta.x_gather_idx;
+        up.expert_off = meta.expert_frequency_offset;
+        up.bias = static_cast<const __nv_bfloat16 *>(b1);
+        up.out = hbuf;
+        up.hdr = hdr;
+        up.E = E;
+        up.k_dim = H;
+        up.n_out = 2 * I;
+        up.out_cols = I;
+        up.I = I;
+        up.layout = layout_kind;
+        if (launch_decode_up(up, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if ((st = record(ev, 2, s))) return st;
+        DecodeArgs dn;
+        memset(&dn, 0, sizeof dn);
+        if (!make_map_w_chunks(&dn.tmap_w, w2, (uint64_t)H, (uint64_t)E * I, 64) ||
+            !make_map_a_chunks(&dn.tmap_h, hbuf, (uint64_t)I, (uint64_t)l.p_cap, 32, 1))
+            return MOE_ERR_CUDA;
+        dn.expert_off = meta.expert_frequency_offset;
+        dn.bias = static_cast<const __nv_bfloat16 *>(b2);
+        dn.out = ybuf;
+        dn.out_lo = ylo;
+        dn.hdr = hdr;
+        dn.E = E;
+        dn.k_dim = I;
+        dn.n_out = H;
+        dn.out_cols = H;
+        dn.I = I;
+        dn.layout = MOE_LAYOUT_INTERLEAVED;
+        if (launch_decode_down(dn, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if ((st = record(ev, 3, s))) return st;
+    } else if (l.p_cap > 0) {
         const int64_t cap_mtiles = (l.p_cap + kTileRows - 1) / kTileRows + E;
         // ---- up: x gathered rows . w1 -> h
         GemmArgs up;

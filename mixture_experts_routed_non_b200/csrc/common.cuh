@@ -126,6 +126,27 @@ struct GemmArgs {
     int32_t layout;       // MOE_LAYOUT_*
 };
 
+// Decode-shaped grouped GEMMs (swap-AB): 128 weight columns on the MMA's M,
+// a segment's tokens (at most 128 per chunk) on its N.
+struct DecodeArgs {
+    CUtensorMap tmap_w;       // weights: up w1 as (64 cols, E*H rows, 2I/64 chunks) [interleaved] or
+                              // (64, E*H, I/64, 2) [concatenated]; down w2 as (64, E*I, H/64); box 64 x 64 K rows
+    CUtensorMap tmap_h;       // down: h [P_cap, I] as (64, rows, I/64), box 64 x 32 rows x 1
+    const __nv_bfloat16 *x;   // up: x [N,H], rows gathered through x_gather_idx
+    const int32_t *x_gather_idx;
+    const int32_t *expert_off;    // [E+1]
+    const __nv_bfloat16 *bias;    // b1 [E,2I] / b2 [E,H] or null
+    __nv_bfloat16 *out;           // h [P_cap, I] / y [P_cap, H]
+    uint8_t *out_lo;              // down: y_lo [P_cap, H]
+    WsHeader *hdr;
+    int32_t E;
+    int32_t k_dim;        // H (up) / I (down)
+    int32_t n_out;        // output columns of one expert: 2I (up, in w1 order) / H (down)
+    int32_t out_cols;     // I (up) / H (down): row length of out
+    int32_t I;
+    int32_t layout;       // up: MOE_LAYOUT_*
+};
+
 // Backward grouped GEMMs (one CTA per tile, M=128 x N=256, cp.async operands).
 enum BwdMode : int32_t {
     kBwdDH = 0,  // dz = SwiGLU'(z) applied to s * (dout[x_gather_idx[p]] . W2[e]^T)
@@ -176,6 +197,8 @@ bool ptr_aligned(const void *p, size_t a);
 cudaError_t launch_meta(const MetaArgs &a, cudaStream_t s);
 cudaError_t launch_gemm_up(const GemmArgs &a, int max_clusters, cudaStream_t s);
 cudaError_t launch_gemm_down(const GemmArgs &a, int max_clusters, cudaStream_t s);
+cudaError_t launch_decode_up(const DecodeArgs &a, int max_ctas, cudaStream_t s);
+cudaError_t launch_decode_down(const DecodeArgs &a, int max_ctas, cudaStream_t s);
 cudaError_t launch_combine(const __nv_bfloat16 *y, const uint8_t *y_lo, const int32_t *token_offset, const int32_t *s_rev,
                            const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
                            const WsHeader *hdr, int num_sms, cudaStream_t s);
@@ -512,12 +535,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_
     return d;
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B,
-// A K-major, B MN-major (N contiguous), shape M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, A
+// K-major (or MN-major: M contiguous), B MN-major (N contiguous) or K-major,
+// shape M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major, bool a_mn_major = false) {
     return (1u << 4)                              // D format: f32
            | (1u << 7)                            // A format: bf16
            | (1u << 10)                           // B format: bf16
+           | ((a_mn_major ? 1u : 0u) << 15)       // A major
            | ((b_mn_major ? 1u : 0u) << 16)       // B major
            | ((static_cast<uint32_t>(N) >> 3) << 17)
            | ((static_cast<uint32_t>(M) >> 4) << 24);

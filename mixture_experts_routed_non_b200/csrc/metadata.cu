@@ -16,8 +16,9 @@
 //            its CTAs start while the counts are still running.  Before it
 //            waits for them, each CTA loads its tile's ids and weights and
 //            ranks every valid slot stably inside the tile: each warp owns a
-//            contiguous slice, match_any groups the lanes of one expert in a
-//            32-slot step, popc(peers & lanes below) orders them, and a
+//            contiguous slice, ballots over the bits of the expert id group
+//            the lanes of one expert in a 32-slot step, popc(peers & lanes
+//            below) orders them, and a
 //            per-warp row of counts in shared memory carries the rank across
 //            steps; a scan over the warps then gives every pair its position
 //            in the tile's expert-sorted order, where its token and pair
@@ -256,6 +257,19 @@ __device__ __forceinline__ int pass_slice(int L) {
     return ((L + 32 * kMetaWarps - 1) / (32 * kMetaWarps)) * 32;
 }
 
+// Lanes of the warp whose key equals this lane's key (keys < 2^nbits): one
+// ballot per key bit, each lane keeping the lanes that agree with it on that
+// bit -- the mask match_any gives, in nbits ballots (measured faster here
+// than match_any on the 32-slot steps).
+__device__ __forceinline__ unsigned peers_of(unsigned key, int nbits) {
+    unsigned peers = kFull;
+    for (int b = 0; b < nbits; ++b) {
+        const unsigned bb = __ballot_sync(kFull, (key >> b) & 1u);
+        peers &= ((key >> b) & 1u) ? bb : ~bb;
+    }
+    return peers;
+}
+
 // Loads the slots [c0, c1) and gives every pair its position inside the
 // pass's expert-sorted order; stages (token, pair index in the pass, expert)
 // at that position.  Inputs only: runs before the wait on the count kernel.
@@ -270,6 +284,7 @@ __device__ int rank_pass(const MetaArgs &a, const ScatterSmem &m, int c0, int c1
     const int w0 = c0 + warp * slice;
     const int w1 = min(w0 + slice, c1);
     int *myrow = m.wrow + warp * E;
+    const int nbits = 32 - __clz(E);  // keys 0..E; E marks a slot that is no pair
 #pragma unroll
     for (int v = 0; v < kStepMax; ++v) {
         const int s = w0 + 32 * v + lane;
@@ -287,7 +302,7 @@ __device__ int rank_pass(const MetaArgs &a, const ScatterSmem &m, int c0, int c1
         unsigned ignore = 0;
         const bool valid = slot_valid<kPairs>(a, r.e[v], r.tok[v], &ignore);
         if (!valid) r.e[v] = -1;
-        const unsigned peers = __match_any_sync(kFull, r.e[v]);
+        const unsigned peers = peers_of(valid ? (unsigned)r.e[v] : (unsigned)E, nbits);
         const int before = valid ? myrow[r.e[v]] : 0;
         __syncwarp();
         if (valid && lane == __ffs(peers) - 1) myrow[r.e[v]] = before + __popc(peers);

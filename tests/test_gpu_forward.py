@@ -198,3 +198,37 @@ def test_full_size_properties_hold_everywhere():
     assert torch.count_nonzero(out[~empty].float().abs().sum(1) == 0) == 0
     out2 = binding.forward(inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, ws=ws)
     assert torch.equal(out, out2)
+
+
+# ---- decode-sized segments: the swap-AB kernels (chosen when P_cap <= 32 E) ----
+
+@pytest.mark.parametrize("N,H,I,E,K,p_invalid,bias,seed", [
+    (64, 256, 192, 64, 8, 0.1, True, 21),     # I % 128 == 64: a 64-column last unit in the up GEMM
+    (40, 320, 128, 32, 4, 0.0, False, 22),    # H % 128 == 64: half of the last down unit is out of range
+    (128, 512, 256, 256, 8, 0.0, True, 23),   # the decode shape, smaller
+    (1, 64, 64, 1, 1, 0.0, True, 24),         # one pair
+    (16, 128, 64, 16, 2, 0.5, True, 25),      # many empty experts
+])
+@pytest.mark.parametrize("layout", [0, 1])
+def test_decode_path_shapes_full(N, H, I, E, K, p_invalid, bias, seed, layout):
+    assert N * K <= 32 * E  # the sizes select the decode kernels
+    wl = synthetic.custom(N, H, I, E, K, p_invalid=p_invalid, bias=bias, seed=seed)
+    inp = synthetic.make_inputs(wl, device="cuda", invalid_value=float("nan"))
+    run_case(inp, layout=layout)
+    run_case(inp, layout=layout, total_pairs=int((inp.topk_idx >= 0).sum()))
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_decode_path_long_segment_and_duplicates(layout):
+    """One expert with 300 rows (three chunks of at most 128 tokens), the same
+    expert twice in some rows, the rest spread thinly."""
+    N, H, I, E, K = 320, 192, 128, 32, 2
+    wl = synthetic.custom(N, H, I, E, K, bias=True, seed=26)
+    inp = synthetic.make_inputs(wl, device="cuda")
+    rng = np.random.default_rng(26)
+    idx = rng.integers(0, E, size=(N, K)).astype(np.int32)
+    idx[:300, 0] = 5
+    idx[:40, 1] = 5
+    inp.topk_idx.copy_(torch.from_numpy(idx))
+    assert N * K <= 32 * E
+    run_case(inp, layout=layout)
