@@ -238,6 +238,9 @@ def parse():
     ap.add_argument("--layout", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true", help="skip the other configured workloads")
+    ap.add_argument("--forward-only", action="store_true",
+                    help="time the forward of --workload only (no end-to-end, graph, workloads or side legs); "
+                         "for profiler runs")
     ap.add_argument("--check-launch", action="store_true",
                     help="every rank prints its rank and world size and exits (checks the --gpus launch)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -743,6 +746,17 @@ def run_ours(args, rank, world, local):
     max_ms = max_over_ranks(elapsed_ms, dev, world)
     ms_per_step = max_ms / args.steps
     value = N * world * args.steps / (max_ms / 1000.0)
+    if args.forward_only:
+        sampler.stop()
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                              "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+                              "forward_only": True, "stages_ms": [float(v) for v in stage_ms],
+                              "config": bench_config(wl, args.layout, world, P,
+                                                     (inp.w1.numel() + inp.w2.numel()) * 2)}), flush=True)
+        return
 
     # ---- end to end: every step copies its inputs in from pinned host memory,
     # runs the forward and copies its result back out.  Steps are pipelined

@@ -340,6 +340,17 @@ __device__ __forceinline__ void cp_async_16_zfill(uint32_t dst, const void *src,
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
                  : "memory");
 }
+// An L2 cache policy that marks the lines an access brings in as evicted last.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// cp_async_16 with an L2 cache policy.
+__device__ __forceinline__ void cp_async_16_hint(uint32_t dst, const void *src, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "l"(pol)
+                 : "memory");
+}
 // Arrive on `bar` once every cp.async this thread issued so far has landed
 // (the arrival is one of the barrier's expected arrivals).
 __device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {

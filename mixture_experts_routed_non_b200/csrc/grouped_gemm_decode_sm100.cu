@@ -10,7 +10,9 @@
 //   down (kUp = false): Y^T[c, n] = sum_k w2[e][k][c] * h[off_e + n][k]
 //                       y[off_e + n][c] (bf16) and its e5m2 rounding residual y_lo
 //
-// A work unit is (expert e, 128 output columns mt); its segment's rows are
+// A work unit is (expert e with pairs, 128 output columns mt), dealt
+// round-robin over the CTAs from a list of the active experts that each CTA
+// builds first; its segment's rows are
 // taken in chunks of at most 32 tokens (one chunk for a decode-sized
 // segment, so each expert's weights are read once; longer segments re-read
 // the unit's weight slice from L2 per chunk).  The MMA is
@@ -50,7 +52,8 @@ constexpr size_t kDXchgOff = (size_t)kDStages * kDStage;          // concatenate
 constexpr size_t kDBarOff = kDXchgOff + 64 * 32 * 4;
 constexpr size_t kDMiscOff = kDBarOff + 8 * kDNumBars;
 constexpr size_t kDOffTableOff = kDMiscOff + 16;
-constexpr size_t kDSmemBytes = 1024 + kDOffTableOff + (kMaxExperts + 1) * 4;
+constexpr size_t kDActOff = kDOffTableOff + (kMaxExperts + 1) * 4;   // experts with at least one pair
+constexpr size_t kDSmemBytes = 1024 + kDActOff + kMaxExperts * 4;
 static_assert(kDSmemBytes <= 232448, "shared memory of one CTA (227 KB)");
 
 __host__ __device__ constexpr int decode_threads(bool up) { return up ? 192 + kDGatherThreads : 192; }
@@ -83,6 +86,7 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
     const uint32_t drain_bar = bars + 8u * (2 * kDStages + 4);
     uint32_t *misc = reinterpret_cast<uint32_t *>(base_ptr + kDMiscOff);
     int *off_s = reinterpret_cast<int *>(base_ptr + kDOffTableOff);
+    int *act_s = reinterpret_cast<int *>(base_ptr + kDActOff);
     float *xchg = reinterpret_cast<float *>(base_ptr + kDXchgOff);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -109,6 +113,20 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
         tmem_alloc(smem_u32(&misc[0]), kDTmemCols);
         tmem_relinquish();
     }
+    __syncthreads();
+    if (warp == 0) {
+        // the experts that have pairs, in order: work is dealt over these only, so
+        // empty experts (many, at random, in a skewed decode batch) unbalance no CTA
+        int n = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const bool has = e < E && off_s[e + 1] > off_s[e];
+            const unsigned m = __ballot_sync(0xffffffffu, has);
+            if (has) act_s[n + __popc(m & lanemask_lt())] = e;
+            n += __popc(m);
+        }
+        if (lane == 0) misc[3] = (uint32_t)n;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -118,7 +136,7 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
     const bool concat = kUp && a.layout == MOE_LAYOUT_CONCATENATED;
     // units: (expert, 128 output columns); concatenated up: 64 gate + 64 up columns
     const int n_mt = concat ? a.I / 64 : (a.n_out + kDM - 1) / kDM;
-    const int units = E * n_mt;
+    const int units = (int)misc[3] * n_mt;  // (active expert, 128 output columns)
     const int nk = a.k_dim / kDK;
     const uint32_t sA0 = base;  // stage s: weights at sA0 + s * kDStage, token rows kDStageA after them
 
@@ -129,7 +147,7 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
             uint32_t phase = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
-                const int e = u / n_mt, mt = u - (u / n_mt) * n_mt;
+                const int e = act_s[u / n_mt], mt = u - (u / n_mt) * n_mt;
                 const int m0 = off_s[e], Me = off_s[e + 1] - m0;
                 for (int c0 = 0; ok && c0 < Me; c0 += kDN) {
                     for (int kb = 0; kb < nk; ++kb) {
@@ -165,7 +183,7 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
             int tcount = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
-                const int e = u / n_mt;
+                const int e = act_s[u / n_mt];
                 const int Me = off_s[e + 1] - off_s[e];
                 for (int c0 = 0; ok && c0 < Me; c0 += kDN, ++tcount) {
                     const int nv = min(kDN, Me - c0);
@@ -216,7 +234,7 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
         int tcount = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
-            const int e = u / n_mt, mt = u - (u / n_mt) * n_mt;
+            const int e = act_s[u / n_mt], mt = u - (u / n_mt) * n_mt;
             const int m0 = off_s[e], Me = off_s[e + 1] - m0;
             for (int c0 = 0; c0 < Me; c0 += kDN, ++tcount) {
                 const int nv = min(kDN, Me - c0);
@@ -328,7 +346,7 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
         uint32_t phase = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
-            const int e = u / n_mt;
+            const int e = act_s[u / n_mt];
             const int m0 = off_s[e], Me = off_s[e + 1] - m0;
             for (int c0 = 0; ok && c0 < Me; c0 += kDN) {
                 const int nv = min(kDN, Me - c0);

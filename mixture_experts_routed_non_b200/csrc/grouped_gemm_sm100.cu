@@ -607,6 +607,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
         uint32_t phase = 0;
         const char *xb = reinterpret_cast<const char *>(a.x);
         const size_t ld = (size_t)a.k_dim * 2;
+        // x rows are read by every pair of their token, at different times (one
+        // expert after another) while the weights stream through L2: keep them
+        const uint64_t x_policy = l2_policy_evict_last();
         int tile = cluster;
         Tile t{};
         const char *src[8];
@@ -653,8 +656,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                         // rows past the segment end are never stored: skip their copies
                         // (the stage keeps stale data there, which only feeds those rows)
                         if (rr < rs && t.m0 + rb + rr < t.m_end)
-                            cp_async_16(a_dst + at * kAtomA + rr * 128 + ((chunk ^ (rr & 7)) << 4),
-                                        src[i] + koff);
+                            cp_async_16_hint(a_dst + at * kAtomA + rr * 128 + ((chunk ^ (rr & 7)) << 4),
+                                             src[i] + koff, x_policy);
                     }
                 }
                 // even CTA: straight onto the stage barrier the MMA waits on; odd
