@@ -238,9 +238,9 @@ def parse():
     ap.add_argument("--layout", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true", help="skip the other configured workloads")
-    ap.add_argument("--forward-only", action="store_true",
-                    help="time the forward of --workload only (no end-to-end, graph, workloads or side legs); "
-                         "for profiler runs")
+    ap.add_argument("--only", choices=["forward", "train", "metadata"], default=None,
+                    help="profiler runs: time only the forward of --workload, only its training step "
+                         "(forward_train + backward), or only the metadata on the metadata workload")
     ap.add_argument("--check-launch", action="store_true",
                     help="every rank prints its rank and world size and exits (checks the --gpus launch)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -704,6 +704,20 @@ def run_ours(args, rank, world, local):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     peaks, peaks_src = load_peaks()
+    if args.only in ("train", "metadata"):
+        if rank == 0:
+            if args.only == "metadata":
+                print(json.dumps({"only": "metadata", "metadata_only": metadata_only(dev, peaks, reps=args.steps)}),
+                      flush=True)
+            else:
+                wl = synthetic.WORKLOADS[args.workload]
+                inp = synthetic.make_inputs(wl, device=dev)
+                print(json.dumps({"only": "train", "training": backward_leg(
+                    inp, inp.w1, inp.b1, 0, dev, peaks, peaks["bf16_tflops"], "burst", steps=args.steps,
+                    warmup=max(1, args.warmup))}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.2)
@@ -746,14 +760,14 @@ def run_ours(args, rank, world, local):
     max_ms = max_over_ranks(elapsed_ms, dev, world)
     ms_per_step = max_ms / args.steps
     value = N * world * args.steps / (max_ms / 1000.0)
-    if args.forward_only:
+    if args.only == "forward":
         sampler.stop()
         if world > 1:
             dist.destroy_process_group()
         if rank == 0:
             print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
                               "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
-                              "forward_only": True, "stages_ms": [float(v) for v in stage_ms],
+                              "only": "forward", "stages_ms": [float(v) for v in stage_ms],
                               "config": bench_config(wl, args.layout, world, P,
                                                      (inp.w1.numel() + inp.w2.numel()) * 2)}), flush=True)
         return

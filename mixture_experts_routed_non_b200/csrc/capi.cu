@@ -56,6 +56,10 @@ namespace {
 
 constexpr size_t kAlign = 256;
 constexpr int64_t kDecodeRowsPerExpert = 32;  // decode GEMMs when P_cap <= 32 E
+#ifndef MOE_DECODE_N
+#define MOE_DECODE_N 128
+#endif
+constexpr uint32_t kDecodeChunkRows = MOE_DECODE_N;  // rows of one decode chunk (its h box)
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -493,7 +497,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         DecodeArgs dn;
         memset(&dn, 0, sizeof dn);
         if (!make_map_w_chunks(&dn.tmap_w, w2, (uint64_t)H, (uint64_t)E * I, 64) ||
-            !make_map_a_chunks(&dn.tmap_h, hbuf, (uint64_t)I, (uint64_t)l.p_cap, 32, 1))
+            !make_map_a_chunks(&dn.tmap_h, hbuf, (uint64_t)I, (uint64_t)l.p_cap, kDecodeChunkRows, 1))
             return MOE_ERR_CUDA;
         dn.expert_off = meta.expert_frequency_offset;
         dn.bias = static_cast<const __nv_bfloat16 *>(b2);

@@ -131,7 +131,7 @@ struct GemmArgs {
 struct DecodeArgs {
     CUtensorMap tmap_w;       // weights: up w1 as (64 cols, E*H rows, 2I/64 chunks) [interleaved] or
                               // (64, E*H, I/64, 2) [concatenated]; down w2 as (64, E*I, H/64); box 64 x 64 K rows
-    CUtensorMap tmap_h;       // down: h [P_cap, I] as (64, rows, I/64), box 64 x 32 rows x 1
+    CUtensorMap tmap_h;       // down: h [P_cap, I] as (64, rows, I/64), box 64 x (chunk rows) x 1
     const __nv_bfloat16 *x;   // up: x [N,H], rows gathered through x_gather_idx
     const int32_t *x_gather_idx;
     const int32_t *expert_off;    // [E+1]

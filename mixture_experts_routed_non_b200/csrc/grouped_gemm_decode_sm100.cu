@@ -13,14 +13,14 @@
 // A work unit is (expert e with pairs, 128 output columns mt), dealt
 // round-robin over the CTAs from a list of the active experts that each CTA
 // builds first; its segment's rows are
-// taken in chunks of at most 32 tokens (one chunk for a decode-sized
+// taken in chunks of at most 128 tokens (one chunk for a decode-sized
 // segment, so each expert's weights are read once; longer segments re-read
 // the unit's weight slice from L2 per chunk).  The MMA is
 // tcgen05.mma.cta_group::1.kind::f16 with M = 128 (A = the weights, MN-major:
 // a 64 x 64 TMA box per 64-column chunk lands in the 128-byte swizzle) and
 // N = the chunk's rows rounded up to 16 (B = the token rows, K-major).  Each
-// stage holds 64 K of both operands (16 KB + 4 KB) and ten stages are in
-// flight, so about 160 KB of weights stream into every SM at once.  The fp32
+// stage holds 64 K of both operands (16 KB + 16 KB) and six stages are in
+// flight, so about 96 KB of weights stream into every SM at once.  The fp32
 // accumulator (128 lanes = output columns x N columns = tokens) is
 // double-buffered in TMEM.
 //
@@ -37,12 +37,18 @@ namespace moe {
 namespace {
 
 constexpr int kDM = 128;                      // output columns per unit (MMA M)
-constexpr int kDN = 32;                       // rows (tokens) per chunk at most (MMA N)
+#ifndef MOE_DECODE_N
+#define MOE_DECODE_N 128
+#endif
+#ifndef MOE_DECODE_STAGES
+#define MOE_DECODE_STAGES 6
+#endif
+constexpr int kDN = MOE_DECODE_N;             // rows (tokens) per chunk at most (MMA N)
 constexpr int kDK = 64;                       // K per stage: one 128-byte swizzle atom of bf16
-constexpr int kDStages = 10;
+constexpr int kDStages = MOE_DECODE_STAGES;
 constexpr uint32_t kDChunkA = kDK * 64 * 2;   // 8 KB: 64 output columns x 64 K (MN-major)
 constexpr uint32_t kDStageA = 2 * kDChunkA;   // 128 output columns
-constexpr uint32_t kDStageB = kDN * kDK * 2;  // 4 KB: 32 rows x 64 K (K-major)
+constexpr uint32_t kDStageB = kDN * kDK * 2;  // 16 KB: 128 rows x 64 K (K-major)
 constexpr uint32_t kDStage = kDStageA + kDStageB;
 constexpr uint32_t kDTmemCols = 2 * kDN;      // two accumulators
 constexpr int kDGatherWarps = 2;
@@ -55,6 +61,7 @@ constexpr size_t kDOffTableOff = kDMiscOff + 16;
 constexpr size_t kDActOff = kDOffTableOff + (kMaxExperts + 1) * 4;   // experts with at least one pair
 constexpr size_t kDSmemBytes = 1024 + kDActOff + kMaxExperts * 4;
 static_assert(kDSmemBytes <= 232448, "shared memory of one CTA (227 KB)");
+static_assert(kDN % 32 == 0 && kDN <= 128, "chunks of whole 32-column TMEM loads, at most the 128 of one MMA tile here");
 
 __host__ __device__ constexpr int decode_threads(bool up) { return up ? 192 + kDGatherThreads : 192; }
 
