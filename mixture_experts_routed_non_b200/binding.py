@@ -308,6 +308,19 @@ def intermediates_from_workspace(ws: torch.Tensor, N: int, H: int, I: int, E: in
     return h, y
 
 
+def backward_intermediates_from_workspace(ws: torch.Tensor, N: int, H: int, I: int, E: int, K: int,
+                                          total_pairs: int = -1):
+    """Views, after moe_nonexpand_backward on a training workspace, of dz
+    [P_cap, 2I] (bf16, the SwiGLU backward in w1's column order) and of the
+    per-pair dx rows [P_cap, H] (bf16, dz . w1[e]^T, before they are summed
+    per token), both in expert-sorted row order."""
+    lay = workspace_layout(N, H, I, E, K, total_pairs)
+    pc = lay.p_cap
+    dz = ws[lay.dz:lay.dz + pc * 2 * I * 2].view(torch.bfloat16).view(pc, 2 * I)
+    dx_rows = ws[lay.y:lay.y + pc * H * 2].view(torch.bfloat16).view(pc, H)
+    return dz, dx_rows
+
+
 # ---------------------------------------------------------------------------
 # Entry points
 # ---------------------------------------------------------------------------

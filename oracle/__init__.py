@@ -313,6 +313,18 @@ def pairs_backward(wd: WeightsF64, dout, tokens, experts, scores, layout: int = 
     return out
 
 
+def pair_dx_rows(wd: WeightsF64, dz, experts) -> np.ndarray:
+    """Each pair's share of dx before the per-token sum: dz[i] . w1[experts[i]]^T
+    ([n, H], float64), from the per-pair dz of pairs_backward."""
+    dz = np.asarray(dz, dtype=np.float64)
+    experts = np.asarray(experts)
+    out = np.zeros((dz.shape[0], wd.H))
+    for e in np.unique(experts):
+        sel = experts == e
+        out[sel] = dz[sel] @ wd.w1e(e).T
+    return out
+
+
 def backward(wd: WeightsF64, topk_idx: np.ndarray, topk_w: np.ndarray, dout, layout: int = LAYOUT_INTERLEAVED,
              experts_only=None, lib_path: str | None = None) -> dict:
     """Gradients of sum_t <dout_t, out_t> for the [N,K] non-expand routing:

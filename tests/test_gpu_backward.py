@@ -15,7 +15,7 @@ import pytest
 import torch
 
 import oracle
-from helpers import assert_close_bwd, backward_rss, to_np
+from helpers import assert_close, assert_close_bwd, backward_rss, tile_rows, to_np
 from mixture_experts_routed_non_b200 import binding, synthetic
 
 pytestmark = pytest.mark.gpu
@@ -226,3 +226,49 @@ def test_prefill256_backward_skewed_routing():
     if empty.size:
         e = torch.from_numpy(empty).cuda()
         assert torch.count_nonzero(grads["dw1"][e]) == 0 and torch.count_nonzero(grads["dw2"][e]) == 0
+
+
+def test_prefill256_backward_every_tile():
+    """Full-size, Zipf-skewed (256 experts, segments of ~50 to ~15k rows), the
+    launch configuration the bench times: DH's dz and DX's per-pair dx rows on
+    the boundary rows of every (expert, 256-row m-tile), and the complete dW1
+    and dW2 -- every one of their tiles -- of the most and the least popular
+    expert with pairs."""
+    inp = synthetic.make_inputs("prefill256", device="cuda")
+    wl = inp.wl
+    dout = _dout(wl, 31)
+    _, grads, _, _ = _run(inp, 0, dout, bias_grads=False)
+    ws_args = (wl.N, wl.H, wl.I, wl.E, wl.K)
+    idx, w = inp.topk_idx.cpu().numpy(), inp.topk_w.cpu().numpy()
+    meta = oracle.metadata(idx, w, wl.E)
+    wd = oracle.WeightsF64(inp.x, inp.w1, None, inp.w2, None)
+    # the workspace of the run above holds dz and the dx rows: recompute them in a
+    # fresh training workspace so the views below belong to this call
+    ws = binding.alloc_train_workspace(*ws_args)
+    binding.forward_train(inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, ws=ws)
+    binding.backward(dout, inp.x, inp.topk_idx, inp.topk_w, inp.w1, inp.w2, ws=ws)
+    torch.cuda.synchronize()
+    assert binding.read_error(ws) == 0
+    dz_gpu, dxr_gpu = binding.backward_intermediates_from_workspace(ws, *ws_args)
+    ps = tile_rows(meta["off"])
+    tok = meta["x_gather_idx"][ps]
+    ex = (np.searchsorted(meta["off"], ps, side="right") - 1).astype(np.int32)
+    sc = meta["scores"][meta["s_scatter_idx"][ps]]
+    ref = oracle.pairs_backward(wd, dout, tok, ex, sc, 0)
+    ps_t = torch.from_numpy(ps).cuda()
+    assert_close(to_np(dz_gpu[ps_t]), ref["dz"], f"dz (DH) on {ps.size} tile boundary rows")
+    dxr_ref = oracle.pair_dx_rows(wd, ref["dz"], ex)
+    # root sum of squares of the terms of each dx-row entry: sum_c (dz_c w1[e][j, c])^2
+    rss = np.zeros_like(dxr_ref)
+    for e in np.unique(ex):
+        sel = ex == e
+        rss[sel] = (ref["dz"][sel] ** 2) @ (wd.w1e(e) ** 2).T
+    assert_close_bwd(to_np(dxr_gpu[ps_t]), dxr_ref, np.sqrt(rss), f"per-pair dx rows (DX) on {ps.size} rows")
+    freq = meta["freq"]
+    nz = np.nonzero(freq)[0]
+    experts = [int(nz[np.argmax(freq[nz])]), int(nz[np.argmin(freq[nz])])]
+    refw = oracle.backward(wd, idx, w, dout, 0, experts_only=experts)
+    rssw = backward_rss(refw, wd, dout)
+    for k in ("dw1", "dw2"):
+        assert_close_bwd(to_np(grads[k][experts]), refw[k][experts], rssw[k][experts],
+                         f"{k} (prefill256, experts {experts}, M_e {[int(freq[e]) for e in experts]})")

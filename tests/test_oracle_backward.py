@@ -229,3 +229,22 @@ def test_finite_differences_reject_summation_mistakes(monkeypatch, kind):
     monkeypatch.setattr(oracle, "_sum_pair_terms", _sum_pair_terms_mutant(kind))
     with pytest.raises(AssertionError):
         check_finite_differences(0)
+
+
+def test_pair_dx_rows_sum_to_the_pinned_dx():
+    """oracle.pair_dx_rows gives each pair's share of dx (dz . w1[e]^T); summed
+    per token they are the backward oracle's dx, which the finite differences
+    above pin."""
+    import torch
+
+    from mixture_experts_routed_non_b200 import synthetic
+    inp = synthetic.make_inputs("tiny", device="cpu")
+    wd = oracle.WeightsF64(inp.x, inp.w1, inp.b1, inp.w2, inp.b2)
+    g_ = torch.Generator().manual_seed(3)
+    dout = torch.randn((inp.wl.N, inp.wl.H), generator=g_).to(torch.bfloat16)
+    g = oracle.backward(wd, inp.topk_idx.numpy(), inp.topk_w.numpy(), dout, 0)
+    pr = g["pairs"]
+    rows = oracle.pair_dx_rows(wd, pr["dz"], pr["exp"])
+    dx = np.zeros_like(g["dx"])
+    np.add.at(dx, pr["tok"], rows)
+    np.testing.assert_allclose(dx, g["dx"], rtol=0, atol=1e-12)
