@@ -500,7 +500,8 @@ typedef struct moe_ws_layout_t {
     int64_t p_cap;
     int32_t meta_tiles;        /* T */
     int32_t meta_tile_slots;   /* slots per metadata tile */
-    size_t z;                  /* training workspace: fp32 [P_cap,2I], z saved by the forward */
+    size_t z;                  /* training workspace: bf16 [P_cap,2I], w1 column order: u silu'(g) at the
+                                  gate columns, silu(g) at the up columns, saved by the forward */
     size_t dz;                 /* training workspace: bf16 [P_cap,2I], dz of the backward */
     size_t dy;                 /* training workspace: bf16 [P_cap,H], dy of the backward */
     size_t slot_pair;          /* training workspace: int32 [slots], the pair of each routing slot or -1 */

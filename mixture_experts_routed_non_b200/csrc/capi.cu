@@ -122,8 +122,8 @@ moe_ws_layout_t compute_layout_nk(int64_t N, int32_t H, int32_t I, int32_t E, in
     }
     l.total = o;
     if (H > 0 && I > 0) {  // training: z (fp32), dz and dy after the inference workspace
-        l.z = o;
-        o = align_up(o + (size_t)pc * 2 * I * 4, 1024);
+        l.z = o;  // bf16: u silu'(g) at gate columns, silu(g) at up columns
+        o = align_up(o + (size_t)pc * 2 * I * 2, 1024);
         l.dz = o;
         o = align_up(o + (size_t)pc * 2 * I * 2, 1024);
         l.dy = o;
@@ -291,19 +291,6 @@ bool make_map_2d_u8_sw64(CUtensorMap *m, const void *ptr, uint64_t inner, uint64
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// The same for fp32 [outer][inner] (a box of 32 fp32 is one 128-byte row).
-bool make_map_2d_f32(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, uint32_t box_inner,
-                     uint32_t box_outer) {
-    EncodeTiledFn f = encode_fn();
-    if (!f) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {inner * 4};
-    cuuint32_t box[2] = {box_inner, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 // A row-major weight [rows][ncols] (ncols % 64 == 0) viewed as
 // (64 columns, rows, ncols/64 column chunks): one box of 64 x stage-K x 2 lands in
@@ -529,7 +516,9 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         up.tile_off = ma.gemm_tile_off;
         up.bias = static_cast<const __nv_bfloat16 *>(b1);
         up.out = hbuf;
-        up.z_out = train ? reinterpret_cast<float *>(w + l.z) : nullptr;
+        up.z_out = train ? reinterpret_cast<__nv_bfloat16 *>(w + l.z) : nullptr;
+        if (train && !make_map_2d(&up.tmap_z, up.z_out, (uint64_t)2 * I, (uint64_t)l.p_cap, 64, 32))
+            return MOE_ERR_CUDA;
         up.hdr = hdr;
         up.E = E;
         up.k_dim = H;
@@ -607,7 +596,7 @@ int backward_impl(const void *dout, const void *x, const Routing &r, int32_t H, 
     WsHeader *hdr = reinterpret_cast<WsHeader *>(w + l.header);
     auto bf = [&](size_t off) { return reinterpret_cast<__nv_bfloat16 *>(w + off); };
     __nv_bfloat16 *hbuf = bf(l.h), *ybuf = bf(l.y), *dzbuf = bf(l.dz), *dybuf = bf(l.dy);
-    const float *zbuf = reinterpret_cast<const float *>(w + l.z);
+    const __nv_bfloat16 *zbuf = reinterpret_cast<const __nv_bfloat16 *>(w + l.z);
     const __nv_bfloat16 *w1b = static_cast<const __nv_bfloat16 *>(w1);
     const __nv_bfloat16 *w2b = static_cast<const __nv_bfloat16 *>(w2);
 
@@ -639,7 +628,7 @@ int backward_impl(const void *dout, const void *x, const Routing &r, int32_t H, 
         a.b_rows_per_expert = I;
         if (!make_map_a_chunks(&a.tmap_b, w2b, (uint64_t)H, (uint64_t)E * I, 128, 1)) return MOE_ERR_CUDA;
         a.b_tma = 1;
-        if (!make_map_2d_f32(&a.tmap_z, zbuf, (uint64_t)2 * I, prow, 32, 32) ||
+        if (!make_map_2d(&a.tmap_z, zbuf, (uint64_t)2 * I, prow, 64, 32) ||
             !make_map_2d(&a.tmap_out, dzbuf, (uint64_t)2 * I, prow, 64, 32))
             return MOE_ERR_CUDA;
         a.z = zbuf;

@@ -115,7 +115,9 @@ struct GemmArgs {
     const __nv_bfloat16 *bias;    // b1 [E,2I] / b2 [E,H] or null
     __nv_bfloat16 *out;           // h [P_cap,I] / y [P_cap,H]
     uint8_t *out_lo;              // down: y_lo [P_cap,H], e5m2 residual of each stored y element
-    float *z_out;                 // up, training: z [P_cap,2I] fp32 (bias added, W1 column order) or null
+    __nv_bfloat16 *z_out;         // up, training: [P_cap,2I] bf16, w1 column order: u silu'(g) at the gate
+                                  // columns, silu(g) at the up columns (of z with bias), or null
+    CUtensorMap tmap_z;           // up, training: z_out as [P_cap][2I], box 64 columns x 32 rows (stores)
     WsHeader *hdr;
     int32_t E;
     int32_t k_dim;        // H (up) / I (down)
@@ -158,7 +160,7 @@ struct BwdGemmArgs {
     CUtensorMap tmap_a;        // (64, rows, cols/64) view of `a` when a_tma
     CUtensorMap tmap_b;        // (64, rows, cols/64) view of `b` when b_tma
     CUtensorMap tmap_out;      // DX/DW: `out` as [rows][N]; DH: dz [P_cap, 2I]; box 64 columns x 32 rows (stores)
-    CUtensorMap tmap_z;        // DH: z [P_cap, 2I] fp32, box 32 columns x 32 rows
+    CUtensorMap tmap_z;        // DH: the saved SwiGLU factors [P_cap, 2I] bf16, box 64 columns x 32 rows
     int32_t a_tma, b_tma;      // load that operand's whole stages with TMA
     int32_t b_rows_per_expert; // DH/DX: rows of `b` per expert (N of the weights)
     const __nv_bfloat16 *a;    // DH: dout [N,H]; DX: dz [P_cap,2I]; DW: rows of length M_dim
@@ -170,7 +172,7 @@ struct BwdGemmArgs {
     const int32_t *tile_off;   // DH/DX: [E+1] prefix of ceil(freq / 256) (the metadata's GEMM tile table)
     __nv_bfloat16 *out;        // DX: [P_cap, N]; DW: [E][M][N]; DH: unused (writes z)
     int64_t out_ld;
-    const float *z;            // DH: z [P_cap, 2I] fp32 (saved by the training forward)
+    const __nv_bfloat16 *z;    // DH: [P_cap, 2I] bf16 (u silu'(g), silu(g)) saved by the training forward
     __nv_bfloat16 *dz;         // DH: dz [P_cap, 2I] out
     const float *row_scale;    // DH: scores in pair order, read at s_scatter_idx[p]
     const int32_t *row_pair;   // DH: s_scatter_idx (sorted position -> pair)

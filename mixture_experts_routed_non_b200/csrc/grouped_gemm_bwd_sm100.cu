@@ -8,9 +8,10 @@
 //   DH  dh = s_p (dout[x_gather_idx[p],:] . W2[e]^T)  (K = H, N = I; the
 //       A rows are gathered from dout and the score applied in fp32, so dh
 //       sees no rounded operand), then the SwiGLU backward in the epilogue:
-//       with (g, u) read from the fp32 z the training forward saved,
+//       with the factors the training forward saved,
 //       dg = dh u silu'(g), du = dh silu(g), written as bf16 dz at the
-//       gate/up columns of the layout (so dz keeps W1's column order).
+//       gate/up columns of the layout (so dz keeps W1's column order); the
+//       training forward saved u silu'(g) and silu(g) (bf16) for this.
 //   DX  dxs[p,:] = dz[p,:] . W1[e]^T  (K = 2I, N = H).
 //   DW  out[e] = sum over the rows p of segment e of A[p,:]^T B[p,:]:
 //       dW2[e] = h^T dy (A = h, B = dy) and dW1[e] = x[x_gather_idx]^T dz
@@ -55,8 +56,8 @@ constexpr uint32_t kStageBytes = kStageA + kStageB;
 constexpr uint32_t kMnAtom = kSK * 128;      // MN-major: one 64-element column of a stage (8 KB)
 constexpr uint32_t kTmemCols = 2 * kN;
 constexpr uint32_t kStoreBuf = 32 * 128;     // 4 KB per epilogue warp: 32 rows x 64 bf16 (TMA stores)
-constexpr uint32_t kZBox = 32 * 128;         // DH: 32 rows x 32 fp32 of z (one TMA box)
-constexpr uint32_t kZBuf = 2 * kZBox;        // DH: z of 32 dh columns, (g, u) interleaved
+constexpr uint32_t kZBox = 32 * 128;         // DH: 32 rows x 64 bf16 of the saved factors (one TMA box)
+constexpr uint32_t kZBuf = 2 * kZBox;        // DH: two boxes in flight per epilogue warp (32 dh columns each)
 // Four epilogue warps, one per TMEM lane quarter.  DH also stages z per
 // epilogue warp, which costs it one pipeline stage.
 template <int kMode>
@@ -67,7 +68,7 @@ struct Roles {
     static constexpr int kCopyThread0 = 32 * (kTmaWarp + 1);
     static constexpr int kThreads = kCopyThread0 + kProducerThreads;  // MMA, epilogue, TMA, cp.async
     static constexpr int kStages = kMode == kBwdDH ? 5 : 6;
-    static constexpr uint32_t kNumBars = 4 * kStages + 5 + kEpiWarps;  // + one z barrier per epilogue warp
+    static constexpr uint32_t kNumBars = 4 * kStages + 5 + 2 * kEpiWarps;  // + two z barriers per epilogue warp
     static constexpr size_t kStoreOff = (size_t)kStages * kStageBytes;
     static constexpr size_t kZOff = kStoreOff + (size_t)kEpiWarps * kStoreBuf;
     static constexpr size_t kBarOff = kZOff + (kMode == kBwdDH ? (size_t)kEpiWarps * kZBuf : 0);
@@ -144,9 +145,9 @@ __device__ __forceinline__ void mbar_arrive_n(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
     return v;
 }
 
@@ -160,10 +161,6 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-__device__ __forceinline__ float silu_f(float g, float &sig) {
-    sig = __fdividef(1.0f, 1.0f + __expf(-g));  // 0 once exp(-g) overflows, as the limit
-    return g * sig;
-}
 
 template <int kMode>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThreads, 1)
@@ -189,7 +186,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
     auto tfull_bar = [&](int b) { return bars + 8u * (4 * kBwdStages + b); };
     auto tempty_bar = [&](int b) { return bars + 8u * (4 * kBwdStages + 2 + b); };
     const uint32_t drain_bar = bars + 8u * (4 * kBwdStages + 4);
-    auto z_bar = [&](int w) { return bars + 8u * (4 * kBwdStages + 5 + w); };  // DH: epilogue warp w's z
+    auto z_bar = [&](int w) { return bars + 8u * (4 * kBwdStages + 5 + w); };  // DH: z buffer w (two per warp)
     uint32_t *misc = reinterpret_cast<uint32_t *>(base_ptr + R::kMiscOff);
     int *tile_off_s = reinterpret_cast<int *>(base_ptr + R::kTableOff);
     int *off_s = tile_off_s + (kMaxExperts + 1);
@@ -216,7 +213,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
             mbar_init(tempty_bar(b), 2 * R::kEpiWarps);  // both CTAs' epilogue warps
         }
         mbar_init(drain_bar, 1);
-        for (int w = 0; w < R::kEpiWarps; ++w) mbar_init(z_bar(w), 1);
+        for (int w = 0; w < 2 * R::kEpiWarps; ++w) mbar_init(z_bar(w), 1);
         misc[1] = 0;
         fence_barrier_init();
     }
@@ -332,18 +329,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
         const int part = (warp - 1) >> 2;    // this warp's part of the tile's columns
         const uint32_t store_buf = base + (uint32_t)R::kStoreOff + (uint32_t)(warp - 1) * kStoreBuf;
         const uint32_t zbuf = base + (uint32_t)R::kZOff + (uint32_t)(warp - 1) * kZBuf;  // DH
-        const uint32_t zbar = z_bar(warp - 1);
-        uint32_t zphase = 0;
-        bool zpending = false;  // a z load of this warp is in flight
-        // DH: z of 32 dh columns [i0, i0+32) of this warp's 32 rows, two boxes of
-        // 32 fp32 per row, by TMA
-        auto load_z = [&](int i0, int wrow0) {
+        // DH: the saved factors (u silu'(g), silu(g)) of 32 dh columns [i0, i0+32) of this
+        // warp's 32 rows, one TMA box of 64 bf16 per row, in buffer b of two: two boxes
+        // in flight, so a chunk's DRAM latency hides behind the chunk before it
+        uint32_t zphase = 0;    // bit b: the phase buffer b's barrier completes next
+        uint32_t zpending = 0;  // bit b: a load into buffer b is in flight
+        auto load_z = [&](int i0, int wrow0, int b) {
             if (lane == 0) {
-                mbar_arrive_expect_tx(zbar, kZBuf);
-                tma_load_2d(zbuf, &a.tmap_z, zbar, 2 * i0, wrow0);
-                tma_load_2d(zbuf + kZBox, &a.tmap_z, zbar, 2 * i0 + 32, wrow0);
+                mbar_arrive_expect_tx(z_bar(2 * (warp - 1) + b), kZBox);
+                tma_load_2d(zbuf + b * kZBox, &a.tmap_z, z_bar(2 * (warp - 1) + b), 2 * i0, wrow0);
             }
-            zpending = true;
+            zpending |= 1u << b;
         };
         bool ok = true;
         int tcount = 0;
@@ -352,22 +348,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
             const int acc = tcount & 1;
             const uint32_t acc_phase = (tcount >> 1) & 1;
             const int wrow0 = t.m0 + row0 + quarter * 32;  // this warp's first tile row
-            // DH, interleaved gate/up, all 32 rows of the warp in the segment: z comes
-            // in and dz goes out by TMA through shared memory, in coalesced boxes;
+            // DH, interleaved gate/up, all 32 rows of the warp in the segment: the factors
+            // come in and dz goes out by TMA through shared memory, in coalesced boxes;
             // otherwise each thread reads and writes its own row
             const bool dh_tma = kMode == kBwdDH && a.layout == MOE_LAYOUT_INTERLEAVED && wrow0 + 31 < t.m_end;
-            if (dh_tma) load_z(t.n0, wrow0);
+            const int cfirst = part * (kN / 32 / R::kParts), clast = (part + 1) * (kN / 32 / R::kParts);
+            if (dh_tma) {
+                fence_proxy_async_smem();  // the buffers' last reads come before these writes
+                for (int b = 0; b < 2; ++b)
+                    if (cfirst + b < clast && t.n0 + 32 * (cfirst + b) < a.I) load_z(t.n0 + 32 * (cfirst + b), wrow0, b);
+            }
             if (kMode == kBwdDH) {
-                // bring this row's z columns of the tile into L2 while the MMAs run
+                // bring this row's factors of the tile into L2 while the MMAs run
                 const int p = t.m0 + row0 + rl;
                 if (p < t.m_end) {
                     const int c0 = t.n0 + part * (kN / R::kParts);  // this warp's first I column
                     const int ncols = min(kN / R::kParts, a.I - c0);
-                    const float *zr = a.z + (size_t)p * (2 * a.I);
+                    const __nv_bfloat16 *zr = a.z + (size_t)p * (2 * a.I);
                     if (a.layout == MOE_LAYOUT_INTERLEAVED) {
-                        for (int b = 0; b < 2 * ncols * 4; b += 128) prefetch_l2((const char *)(zr + 2 * c0) + b);
+                        for (int b = 0; b < 2 * ncols * 2; b += 128) prefetch_l2((const char *)(zr + 2 * c0) + b);
                     } else {
-                        for (int b = 0; b < ncols * 4; b += 128) {
+                        for (int b = 0; b < ncols * 2; b += 128) {
                             prefetch_l2((const char *)(zr + c0) + b);
                             prefetch_l2((const char *)(zr + a.I + c0) + b);
                         }
@@ -384,53 +385,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                 const int p = t.m0 + row0 + rl;
                 const bool valid = p < t.m_end;
                 const size_t zoff = (size_t)(valid ? p : 0) * (2 * a.I);
-                const float *zrow = a.z + zoff;
+                const __nv_bfloat16 *zrow = a.z + zoff;
                 __nv_bfloat16 *dzrow = a.dz + zoff;
                 // the pair's score: dh = s (dout . W2^T)
                 const float sc = valid ? __ldg(a.row_scale + __ldg(a.row_pair + p)) : 0.f;
 #pragma unroll 1
-                for (int c = part * (kN / 32 / R::kParts); c < (part + 1) * (kN / 32 / R::kParts); ++c) {
+                for (int c = cfirst; c < clast; ++c) {
                     const int i0 = t.n0 + 32 * c;
                     if (i0 >= a.I) break;
                     uint32_t dh[32];
                     tmem_ld_32x32b_x32(tbase + c * 32, dh);
                     if (dh_tma) {
+                        const int b = (c - cfirst) & 1;
                         bool zw = true;
-                        if (lane == 0) zw = mbar_wait_bounded(zbar, zphase, abort);
+                        if (lane == 0) zw = mbar_wait_bounded(z_bar(2 * (warp - 1) + b), (zphase >> b) & 1u, abort);
                         zw = __shfl_sync(0xffffffffu, zw, 0);
                         if (!zw) {  // the load stays pending: the exit path waits for it
                             tmem_ld_wait();
                             ok = false;
                             break;
                         }
-                        zphase ^= 1u;
-                        zpending = false;
-                        // this row's 64 z values: (g_j, u_j) of columns i0 + j at 2j, 2j + 1
-                        float zr[64];
+                        zphase ^= 1u << b;
+                        zpending &= ~(1u << b);
+                        // this row's 32 (a_j, b_j) factor pairs of columns i0 + j
+                        uint32_t zr[32];
 #pragma unroll
-                        for (int b = 0; b < 2; ++b)
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) {
-                                const float4 v = ld_shared_f4(zbuf + b * kZBox + lane * 128 + ((q ^ (lane & 7)) << 4));
-                                zr[32 * b + 4 * q] = v.x;
-                                zr[32 * b + 4 * q + 1] = v.y;
-                                zr[32 * b + 4 * q + 2] = v.z;
-                                zr[32 * b + 4 * q + 3] = v.w;
-                            }
-                        __syncwarp();  // every lane has read the buffer: the next chunk may land
-                        if (c + 1 < (part + 1) * (kN / 32 / R::kParts) && i0 + 32 < a.I) {
+                        for (int q = 0; q < 8; ++q) {
+                            const uint4 v = ld_shared_v4(zbuf + b * kZBox + lane * 128 + ((q ^ (lane & 7)) << 4));
+                            zr[4 * q] = v.x;
+                            zr[4 * q + 1] = v.y;
+                            zr[4 * q + 2] = v.z;
+                            zr[4 * q + 3] = v.w;
+                        }
+                        __syncwarp();  // every lane has read the buffer: the chunk two ahead may land
+                        if (c + 2 < clast && i0 + 64 < a.I) {
                             fence_proxy_async_smem();
-                            load_z(i0 + 32, wrow0);
+                            load_z(i0 + 64, wrow0, b);
                         }
                         tmem_ld_wait();
                         uint32_t o[32];  // (dg_j, du_j) packed: dz columns 2 i0 .. 2 i0 + 63
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             const float d = sc * __uint_as_float(dh[j]);
-                            const float g = zr[2 * j], u = zr[2 * j + 1];
-                            float sig;
-                            const float sl = silu_f(g, sig);
-                            o[j] = pack_bf16x2(d * u * sig * (1.0f + g * (1.0f - sig)), d * sl);
+                            o[j] = pack_bf16x2(d * bf16lo(zr[j]), d * bf16hi(zr[j]));
                         }
                         if (lane == 0) bulk_wait_read0();  // the buffer's previous store has been read
                         __syncwarp();
@@ -449,49 +446,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                     tmem_ld_wait();
                     if (!valid) continue;
                     if (a.layout == MOE_LAYOUT_INTERLEAVED) {
-                        // (g_i, u_i) adjacent: 32 pairs = 64 fp32 in, 64 bf16 out
-                        const float4 *zp = reinterpret_cast<const float4 *>(zrow + 2 * i0);
+                        // (a_i, b_i) adjacent: 32 pairs = 64 bf16 in, 64 bf16 out
+                        const uint4 *zp = reinterpret_cast<const uint4 *>(zrow + 2 * i0);
                         uint4 *dp = reinterpret_cast<uint4 *>(dzrow + 2 * i0);
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            const float4 z0 = zp[2 * q], z1 = zp[2 * q + 1];
-                            const float g[4] = {z0.x, z0.z, z1.x, z1.z};
-                            const float u[4] = {z0.y, z0.w, z1.y, z1.w};
+                            const uint4 zv = zp[q];
+                            const uint32_t zw4[4] = {zv.x, zv.y, zv.z, zv.w};
                             uint32_t o[4];
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 const float d = sc * __uint_as_float(dh[4 * q + j]);
-                                float sig;
-                                const float sl = silu_f(g[j], sig);
-                                o[j] = pack_bf16x2(d * u[j] * sig * (1.0f + g[j] * (1.0f - sig)), d * sl);
+                                o[j] = pack_bf16x2(d * bf16lo(zw4[j]), d * bf16hi(zw4[j]));
                             }
                             dp[q] = make_uint4(o[0], o[1], o[2], o[3]);
                         }
                     } else {
-                        // gates at [i0, i0+32), ups at [I+i0, I+i0+32)
-                        const float4 *gp = reinterpret_cast<const float4 *>(zrow + i0);
-                        const float4 *up = reinterpret_cast<const float4 *>(zrow + a.I + i0);
+                        // u silu'(g) at [i0, i0+32), silu(g) at [I+i0, I+i0+32)
+                        const uint4 *ap = reinterpret_cast<const uint4 *>(zrow + i0);
+                        const uint4 *bp = reinterpret_cast<const uint4 *>(zrow + a.I + i0);
                         uint4 *dg_out = reinterpret_cast<uint4 *>(dzrow + i0);
                         uint4 *du_out = reinterpret_cast<uint4 *>(dzrow + a.I + i0);
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            const float4 g0 = gp[2 * q], g1 = gp[2 * q + 1];
-                            const float4 u0 = up[2 * q], u1 = up[2 * q + 1];
-                            const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-                            const float u[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-                            float dg[8], du[8];
+                            const uint4 av = ap[q], bv = bp[q];
+                            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+                            const uint32_t bw[4] = {bv.x, bv.y, bv.z, bv.w};
+                            uint32_t og[4], ou[4];
 #pragma unroll
-                            for (int j = 0; j < 8; ++j) {
-                                const float d = sc * __uint_as_float(dh[8 * q + j]);
-                                float sig;
-                                const float sl = silu_f(g[j], sig);
-                                dg[j] = d * u[j] * sig * (1.0f + g[j] * (1.0f - sig));
-                                du[j] = d * sl;
+                            for (int j = 0; j < 4; ++j) {
+                                const float d0 = sc * __uint_as_float(dh[8 * q + 2 * j]);
+                                const float d1 = sc * __uint_as_float(dh[8 * q + 2 * j + 1]);
+                                og[j] = pack_bf16x2(d0 * bf16lo(aw[j]), d1 * bf16hi(aw[j]));
+                                ou[j] = pack_bf16x2(d0 * bf16lo(bw[j]), d1 * bf16hi(bw[j]));
                             }
-                            dg_out[q] = make_uint4(pack_bf16x2(dg[0], dg[1]), pack_bf16x2(dg[2], dg[3]),
-                                                   pack_bf16x2(dg[4], dg[5]), pack_bf16x2(dg[6], dg[7]));
-                            du_out[q] = make_uint4(pack_bf16x2(du[0], du[1]), pack_bf16x2(du[2], du[3]),
-                                                   pack_bf16x2(du[4], du[5]), pack_bf16x2(du[6], du[7]));
+                            dg_out[q] = make_uint4(og[0], og[1], og[2], og[3]);
+                            du_out[q] = make_uint4(ou[0], ou[1], ou[2], ou[3]);
                         }
                     }
                 }
@@ -553,8 +543,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(Roles<kMode>::kThrea
                 else mbar_arrive_cluster(mapa_shared(tempty_bar(acc), 0));
             }
         }
-        if (zpending && lane == 0 && !mbar_wait_timed(zbar, zphase))
-            atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);  // a z load still in flight: wait for it
+        for (int b = 0; b < 2; ++b)  // a z load still in flight: wait for it
+            if (kMode == kBwdDH && ((zpending >> b) & 1u) && lane == 0 &&
+                !mbar_wait_timed(z_bar(2 * (warp - 1) + b), (zphase >> b) & 1u))
+                atomicOr(&a.hdr->err, MOE_DEVERR_TIMEOUT);
         if (lane == 0) bulk_wait0();                    // this warp's TMA stores have landed
     } else if (warp == R::kTmaWarp) {
         // ---------------------------------------------------------- TMA producer

@@ -43,8 +43,8 @@
 // epilogue of one tile overlaps the MMAs of the next.  A segment's last tile
 // with at most 128 rows runs the pair MMA at M=128 (64 rows per CTA).  Rows
 // past the end of an expert's segment are computed (stale stage rows) but
-// never stored.  In training the up GEMM also writes z (fp32), staged through
-// the epilogue warp's store buffer and written in whole 128-byte rows.
+// never stored.  In training the up GEMM also writes the SwiGLU backward's
+// factors (u silu'(g), silu(g)) in bf16, by TMA through the store buffer.
 //
 // Every wait is bounded (common.cuh); on a timeout a CTA raises its abort
 // flag, records MOE_DEVERR_TIMEOUT, drains what it has in flight and returns
@@ -116,6 +116,21 @@ __device__ __forceinline__ Tile decode_tile(int tile, int n_tiles, int E, const 
 // silu(g) * u; for very negative g the quotient underflows to 0 as silu does.
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
+// Training: h = silu(g) u (bit for bit what silu_mul gives) and the two
+// factors of the SwiGLU backward the forward keeps for the backward, so that
+// dg = dh * fa and du = dh * fb there, all from one exponential:
+//   fa = u silu'(g) = u s (1 + g (1 - s)),  fb = silu(g) = g s,  s = sigmoid(g).
+// Each factor is rounded once to bf16 when stored; g itself is never rounded
+// (near silu's minimum, g ~ -1.28, silu'(g) of a rounded g would lose its
+// accuracy).
+__device__ __forceinline__ float swiglu_train(float g, float u, float &fa, float &fb) {
+    const float d = 1.0f + __expf(-g);
+    const float sg = __fdividef(1.0f, d);  // 0 once exp(-g) overflows, as the limit
+    fb = g * sg;
+    fa = u * sg * (1.0f + g * (1.0f - sg));
+    return __fdividef(g, d) * u;  // silu_mul(g, u), the same expression
+}
+
 // r[i] (fp32 bits) += bias[i] for 32 consecutive columns; nothing when bias is null.
 __device__ __forceinline__ void add_bias32(uint32_t (&r)[32], const __nv_bfloat16 *b) {
     if (!b) return;
@@ -132,17 +147,33 @@ __device__ __forceinline__ void add_bias32(uint32_t (&r)[32], const __nv_bfloat1
     }
 }
 
-__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
-    return v;
-}
 
-// 32 fp32 values (as bits) to dst (128 bytes, 16-byte aligned)
-__device__ __forceinline__ void store_f32x32(float *dst, const uint32_t (&r)[32]) {
-    uint4 *d = reinterpret_cast<uint4 *>(dst);
+
+// 64 bf16 columns (32 packed pairs) of one row per lane: a warp whose 32 rows
+// are all stored stages the 32 x 64 block in its store buffer (128-byte
+// swizzle) and writes it with one TMA store; otherwise each valid lane stores
+// its row's 128 bytes.
+__device__ __forceinline__ void store_block64(const CUtensorMap *map, uint32_t store_buf, int lane, bool warp_full,
+                                              bool valid, int wrow0, __nv_bfloat16 *row, int col0,
+                                              const uint32_t (&v)[32]) {
+    if (warp_full) {
+        if (lane == 0) bulk_wait_read0();  // the buffer's previous store has been read
+        __syncwarp();
 #pragma unroll
-    for (int q = 0; q < 8; ++q) d[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+        for (int c = 0; c < 8; ++c)
+            st_shared_v4(store_buf + lane * 128 + ((c ^ (lane & 7)) << 4), v[4 * c], v[4 * c + 1], v[4 * c + 2],
+                         v[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_2d(map, store_buf, col0, wrow0);
+            bulk_commit();
+        }
+    } else if (valid) {
+        uint4 *dst = reinterpret_cast<uint4 *>(row + col0);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) dst[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+    }
 }
 
 __device__ __forceinline__ void settle_after_abort() {
@@ -151,7 +182,9 @@ __device__ __forceinline__ void settle_after_abort() {
     }
 }
 
-template <bool kUp>
+// kTrain (up only): also store the SwiGLU backward's factors (a.z_out); a
+// separate instantiation keeps the inference kernel free of that code.
+template <bool kUp, bool kTrain = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
     grouped_gemm_kernel(const __grid_constant__ GemmArgs a) {
     constexpr int kThreads = threads_of(kUp);
@@ -402,56 +435,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
             __nv_bfloat16 *orow = a.out + (size_t)(valid ? p : 0) * a.out_cols;
             const __nv_bfloat16 *brow = a.bias ? a.bias + (size_t)t.e * a.n_dim : nullptr;
 
-            // training: 32 fp32 of z (this thread's row, columns zc .. zc+31).  A full
-            // warp passes its 32 x 32 block through the store buffer (swizzled) and
-            // writes it row by row, eight lanes per 128-byte row, so each store
-            // instruction covers four whole rows instead of 32 pieces of 32 rows.
-            auto store_z32 = [&](int zc, const uint32_t (&v)[32]) {
-                if (warp_full) {
-                    if (lane == 0) bulk_wait_read0();  // the buffer's previous TMA store has been read
-                    __syncwarp();
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        st_shared_v4(store_buf + lane * 128 + ((c ^ (lane & 7)) << 4), v[4 * c], v[4 * c + 1],
-                                     v[4 * c + 2], v[4 * c + 3]);
-                    __syncwarp();
-                    const int ch = lane & 7;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int rr = 4 * j + (lane >> 3);
-                        const uint4 q = ld_shared_v4(store_buf + rr * 128 + ((ch ^ (rr & 7)) << 4));
-                        *reinterpret_cast<uint4 *>(a.z_out + (size_t)(wrow0 + rr) * (2 * a.I) + zc + 4 * ch) = q;
-                    }
-                    __syncwarp();  // the buffer is free again
-                } else if (valid) {
-                    store_f32x32(a.z_out + (size_t)p * (2 * a.I) + zc, v);
-                }
-            };
-
-            // 64 output columns (32 packed bf16 pairs) of this thread's row
             auto store64 = [&](int col0, const uint32_t (&v)[32]) {
-                if (warp_full) {
-                    if (lane == 0) bulk_wait_read0();  // the buffer's previous store has been read
-                    __syncwarp();
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const int rr = lane;  // row inside the warp's 32-row block
-                        st_shared_v4(store_buf + rr * 128 + ((c ^ (rr & 7)) << 4), v[4 * c], v[4 * c + 1],
-                                     v[4 * c + 2], v[4 * c + 3]);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(&a.tmap_out, store_buf, col0, wrow0);
-                        bulk_commit();
-                    }
-                } else if (valid) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + col0);
-#pragma unroll
-                    for (int c = 0; c < 8; ++c)
-                        dst[c] = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-                }
+                store_block64(&a.tmap_out, store_buf, lane, warp_full, valid, wrow0, orow, col0, v);
             };
+            // training: the SwiGLU backward's factors, in w1's column order
+            __nv_bfloat16 *zrow = kTrain ? a.z_out + (size_t)(valid ? p : 0) * (2 * a.I) : nullptr;
 
             if (kUp && a.layout == MOE_LAYOUT_CONCATENATED) {
                 // gate = accumulator columns [0,128), up = [128,256)
@@ -471,16 +459,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                             add_bias32(g, brow + col0 + hf * 32);
                             add_bias32(u, brow + a.I + col0 + hf * 32);
                         }
-                        if (a.z_out) {  // training: keep z for the backward
-                            store_z32(col0 + hf * 32, g);
-                            store_z32(a.I + col0 + hf * 32, u);
-                        }
+                        // h, and in training u silu'(g) at the gate columns and silu(g) at the up
+                        // columns (each thread its own row, 16 bytes to each half per 8 columns),
+                        // one pair of columns at a time so that g and u die as they are used
+                        uint4 *za = kTrain ? reinterpret_cast<uint4 *>(zrow + col0 + hf * 32) : nullptr;
+                        uint4 *zb = kTrain ? reinterpret_cast<uint4 *>(zrow + a.I + col0 + hf * 32) : nullptr;
+                        uint32_t wa[4], wb[4];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            const float h0 = silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i]));
-                            const float h1 =
-                                silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1]));
-                            packed[16 * hf + i] = pack_bf16x2(h0, h1);
+                            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                            if (kTrain) {
+                                float a0, b0, a1, b1;
+                                const float h0 = swiglu_train(g0, u0, a0, b0);
+                                const float h1 = swiglu_train(g1, u1, a1, b1);
+                                packed[16 * hf + i] = pack_bf16x2(h0, h1);
+                                wa[i & 3] = pack_bf16x2(a0, a1);
+                                wb[i & 3] = pack_bf16x2(b0, b1);
+                                if ((i & 3) == 3 && valid) {
+                                    za[i >> 2] = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+                                    zb[i >> 2] = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+                                }
+                            } else {
+                                packed[16 * hf + i] = pack_bf16x2(silu_mul(g0, u0), silu_mul(g1, u1));
+                            }
                         }
                     }
                     store64(col0, packed);
@@ -504,18 +506,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                             add_bias32(r0, brow + acol);
                             add_bias32(r1, brow + acol + 32);
                         }
-                        if (a.z_out) {  // training: keep z for the backward
-                            store_z32(acol, r0);
-                            store_z32(acol + 32, r1);
-                        }
+                        if (kTrain) {
+                            // training: (u silu'(g), silu(g)) in place of (g, u), 64 columns of
+                            // w1's order, written 16 bytes at a time as they are computed (the
+                            // register budget of ten warps leaves no room for the whole row)
+                            if (warp_full) {
+                                if (lane == 0) bulk_wait_read0();  // the buffer's previous store has been read
+                                __syncwarp();
+                            }
+                            // four (gate, up) pairs per 16 bytes of factors; their h in the same pass
+                            auto train_group = [&](const uint32_t(&rr)[32], int qq, uint32_t &h01, uint32_t &h23,
+                                                   uint32_t (&w4)[4]) {
+                                float hv[4];
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            packed[16 * hf + i] =
-                                pack_bf16x2(silu_mul(__uint_as_float(r0[4 * i]), __uint_as_float(r0[4 * i + 1])),
-                                            silu_mul(__uint_as_float(r0[4 * i + 2]), __uint_as_float(r0[4 * i + 3])));
-                            packed[16 * hf + 8 + i] =
-                                pack_bf16x2(silu_mul(__uint_as_float(r1[4 * i]), __uint_as_float(r1[4 * i + 1])),
-                                            silu_mul(__uint_as_float(r1[4 * i + 2]), __uint_as_float(r1[4 * i + 3])));
+                                for (int k = 0; k < 4; ++k) {
+                                    float fa, fb;
+                                    const int j = 8 * qq + 2 * k;
+                                    hv[k] = swiglu_train(__uint_as_float(rr[j]), __uint_as_float(rr[j + 1]), fa, fb);
+                                    w4[k] = pack_bf16x2(fa, fb);
+                                }
+                                h01 = pack_bf16x2(hv[0], hv[1]);
+                                h23 = pack_bf16x2(hv[2], hv[3]);
+                            };
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                uint32_t w4[4];
+                                if (q < 4) train_group(r0, q, packed[16 * hf + 2 * q], packed[16 * hf + 2 * q + 1], w4);
+                                else train_group(r1, q - 4, packed[16 * hf + 8 + 2 * (q - 4)],
+                                                 packed[16 * hf + 8 + 2 * (q - 4) + 1], w4);
+                                if (warp_full)
+                                    st_shared_v4(store_buf + lane * 128 + ((q ^ (lane & 7)) << 4), w4[0], w4[1], w4[2],
+                                                 w4[3]);
+                                else if (valid)
+                                    reinterpret_cast<uint4 *>(zrow + acol)[q] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                            }
+                            if (warp_full) {
+                                fence_proxy_async_smem();
+                                __syncwarp();
+                                if (lane == 0) {
+                                    tma_store_2d(&a.tmap_z, store_buf, acol, wrow0);
+                                    bulk_commit();
+                                }
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                packed[16 * hf + i] =
+                                    pack_bf16x2(silu_mul(__uint_as_float(r0[4 * i]), __uint_as_float(r0[4 * i + 1])),
+                                                silu_mul(__uint_as_float(r0[4 * i + 2]), __uint_as_float(r0[4 * i + 3])));
+                                packed[16 * hf + 8 + i] =
+                                    pack_bf16x2(silu_mul(__uint_as_float(r1[4 * i]), __uint_as_float(r1[4 * i + 1])),
+                                                silu_mul(__uint_as_float(r1[4 * i + 2]), __uint_as_float(r1[4 * i + 3])));
+                            }
                         }
                     }
                     store64(col0, packed);
@@ -689,13 +731,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
     }
 }
 
-template <bool kUp>
+template <bool kUp, bool kTrain>
 cudaError_t launch(const GemmArgs &a, int max_clusters, cudaStream_t s) {
     // once per device: the shared-memory limit, and how many clusters fit at once
     int fit = 1;
     cudaError_t err = launch_setup_once(
-        (const void *)grouped_gemm_kernel<kUp>, &fit, [](int dev, int *v) -> cudaError_t {
-            cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kUp>,
+        (const void *)grouped_gemm_kernel<kUp, kTrain>, &fit, [](int dev, int *v) -> cudaError_t {
+            cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<kUp, kTrain>,
                                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
             if (e != cudaSuccess) return e;
             int sms = 0;
@@ -707,7 +749,7 @@ cudaError_t launch(const GemmArgs &a, int max_clusters, cudaStream_t s) {
             cfg.blockDim = dim3(threads_of(kUp));
             cfg.dynamicSmemBytes = kSmemBytes;
             int n = 0;
-            e = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<kUp>, &cfg);
+            e = cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<kUp, kTrain>, &cfg);
             if (e != cudaSuccess) return e;
             *v = n > 0 ? n : 1;
             return cudaSuccess;
@@ -715,7 +757,7 @@ cudaError_t launch(const GemmArgs &a, int max_clusters, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     int clusters = fit < max_clusters ? fit : max_clusters;
     if (clusters < 1) clusters = 1;
-    grouped_gemm_kernel<kUp><<<2 * clusters, threads_of(kUp), kSmemBytes, s>>>(a);
+    grouped_gemm_kernel<kUp, kTrain><<<2 * clusters, threads_of(kUp), kSmemBytes, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -724,10 +766,10 @@ cudaError_t launch(const GemmArgs &a, int max_clusters, cudaStream_t s) {
 size_t gemm_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_gemm_up(const GemmArgs &a, int max_clusters, cudaStream_t s) {
-    return launch<true>(a, max_clusters, s);
+    return a.z_out ? launch<true, true>(a, max_clusters, s) : launch<true, false>(a, max_clusters, s);
 }
 cudaError_t launch_gemm_down(const GemmArgs &a, int max_clusters, cudaStream_t s) {
-    return launch<false>(a, max_clusters, s);
+    return launch<false, false>(a, max_clusters, s);
 }
 
 }  // namespace moe
