@@ -50,6 +50,7 @@ constexpr int kChunk = 4096;                            // slots staged per pass
 constexpr int kStepMax = kChunk / (32 * kMetaWarps);    // 32-slot steps per warp and pass (8)
 constexpr int kPartInts = 2 * 4 * kMetaThreads;         // table partial sums: 2 x G x hist_ld, G*hist_ld <= 4*512
 static_assert(kPartInts % 4 == 0, "the arrays after the partial sums start 16-byte aligned");
+static_assert(kMetaMaxTiles <= kMetaThreads, "one thread of CTA 0 reads each tile's error bits");
 
 // Programmatic dependent launch (sm_90+): the primary lets its dependent
 // start; the dependent waits until the primary grid has completed and its
