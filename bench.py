@@ -238,9 +238,10 @@ def parse():
     ap.add_argument("--layout", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true", help="skip the other configured workloads")
-    ap.add_argument("--only", choices=["forward", "train", "metadata"], default=None,
+    ap.add_argument("--only", choices=["forward", "train", "metadata", "router"], default=None,
                     help="profiler runs: time only the forward of --workload, only its training step "
-                         "(forward_train + backward), or only the metadata on the metadata workload")
+                         "(forward_train + backward), only the metadata on the metadata workload, or "
+                         "only the router top-k on the prefill sizes")
     ap.add_argument("--check-launch", action="store_true",
                     help="every rank prints its rank and world size and exits (checks the --gpus launch)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -704,9 +705,12 @@ def run_ours(args, rank, world, local):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
 
     peaks, peaks_src = load_peaks()
-    if args.only in ("train", "metadata"):
+    if args.only in ("train", "metadata", "router"):
         if rank == 0:
-            if args.only == "metadata":
+            if args.only == "router":
+                print(json.dumps({"only": "router", "router_only": router_only(dev, peaks, reps=args.steps)}),
+                      flush=True)
+            elif args.only == "metadata":
                 print(json.dumps({"only": "metadata", "metadata_only": metadata_only(dev, peaks, reps=args.steps)}),
                       flush=True)
             else:

@@ -375,9 +375,11 @@ MOE_API int moe_nonexpand_routed_backward(const void *dout, const void *x, const
  *
  * The chosen experts are the K largest logits (softmax is increasing, so all
  * modes choose alike), compared as given: fp32, or bf16 widened exactly.
- * Slot k holds the k-th largest; equal logits go to the lower expert id.  A
- * NaN logit is read as -inf.  A token whose chosen logits are all -inf gets
- * NaN weights.  Weights are computed in fp32 with expf.
+ * Slot k holds the k-th largest; equal logits go to the lower expert id
+ * (-0.0 equals +0.0).  A NaN logit is read as -inf.  A token whose chosen
+ * logits are all -inf gets NaN weights.  Weights are computed in fp32: expf
+ * of the chosen logits' differences to the largest, and for the softmax over
+ * all E the fast exponential (relative error a few 1e-6) in its sum.
  *
  * logits: device, [N,E] row-major, dtype MOE_DTYPE_F32 or MOE_DTYPE_BF16.
  * topk_idx: device int32 [N,K]; topk_w: device fp32 [N,K]; both written.

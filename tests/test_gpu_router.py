@@ -1,10 +1,11 @@
 """Router top-k (moe_router_topk) on the GPU against the oracle.
 
 The chosen experts are an integer decision taken on the logits as given, on
-both sides, so topk_idx must match bit for bit.  The weights: the kernel uses
-fp32 expf (a few ulp) and warp sums of at most 1024 positive terms (at most
-37 roundings), so their relative error stays near 3e-6; the test allows
-RTOL = 1e-5 against the float64 oracle.
+both sides, so topk_idx must match bit for bit.  The weights: the kernels use
+fp32 expf for the chosen logits (a few ulp), the fast exponential for the
+full softmax's sum (relative error a few 1e-6 per term) and fixed-order sums
+of at most 1024 positive terms, so their relative error stays near 5e-6; the
+test allows RTOL = 1e-5 against the float64 oracle.
 """
 import numpy as np
 import pytest
@@ -108,6 +109,46 @@ def test_router_ties_nan_inf_at_128_and_256(mode):
     lg[5, :] = 1.0                # every logit equal: ids 0..K-1
     lg[6, 96:] = 3.0              # the largest all in the last lane
     _check(lg, 8, mode)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("E", [128, 1000])
+def test_router_negative_zero_ties_with_zero(E, dtype):
+    """-0.0 and +0.0 are equal logits: the lower id goes first."""
+    lg = torch.full((64, E), -1.0, device="cuda")
+    lg[:, 3] = -0.0
+    lg[:, 1] = 0.0
+    lg[:, 7] = -0.0
+    lg[1::2, 0] = -0.0
+    for mode in MODES:
+        _check(lg.to(dtype), 4, mode)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_router_near_ties_in_the_low_bits(mode):
+    """fp32 logits a few ulp apart, so that keys sharing their high bits
+    decide the result (the exact retry)."""
+    g = np.random.default_rng(11)
+    base = np.float32(1.25)
+    a = base + g.integers(-300, 300, size=(999, 128)).astype(np.float32) * np.spacing(base)
+    _check(torch.from_numpy(a.astype(np.float32)).cuda(), 8, mode)
+    _check(torch.from_numpy(a[:, :96].copy().astype(np.float32)).cuda(), 5, mode)
+
+
+@pytest.mark.parametrize("mode", MODES)
+def test_router_outputs_4_byte_aligned(mode):
+    """Output arrays 4 bytes past an 8-byte boundary (K = 8: the kernel's paired
+    stores fall back to single ones)."""
+    lg = synthetic.make_logits(333, 128, seed=12, device="cuda")
+    ib = torch.empty(333 * 8 + 1, dtype=torch.int32, device="cuda")
+    wb = torch.empty(333 * 8 + 1, dtype=torch.float32, device="cuda")
+    idx, w = ib[1:].view(333, 8), wb[1:].view(333, 8)
+    assert idx.data_ptr() % 8 == 4 and w.data_ptr() % 8 == 4
+    binding.router_topk(lg, 8, mode, idx, w)
+    torch.cuda.synchronize()
+    ri, rw = oracle.router_topk(lg, 8, mode)
+    np.testing.assert_array_equal(to_np(idx), ri)
+    np.testing.assert_allclose(to_np(w), rw, rtol=RTOL, atol=ATOL, equal_nan=True)
 
 
 def test_router_logits_not_16_byte_aligned():
