@@ -459,6 +459,10 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
     // each active expert's weights once.  Chosen per call from the sizes alone
     // (no host sync); they handle segments of any length.
     const bool decode = !train && l.p_cap > 0 && l.p_cap <= (int64_t)kDecodeRowsPerExpert * E;
+    // Kernels after the metadata start as programmatic dependents of the one
+    // before (their set-up and, in the decode down GEMM, the first weight
+    // loads overlap it), unless stage events sit between the launches.
+    const bool pdl = ev == nullptr;
     if (decode) {
         DecodeArgs up;
         memset(&up, 0, sizeof up);
@@ -479,7 +483,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         up.out_cols = I;
         up.I = I;
         up.layout = layout_kind;
-        if (launch_decode_up(up, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_decode_up(up, dev.sms, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
         if ((st = record(ev, 2, s))) return st;
         DecodeArgs dn;
         memset(&dn, 0, sizeof dn);
@@ -497,7 +501,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         dn.out_cols = H;
         dn.I = I;
         dn.layout = MOE_LAYOUT_INTERLEAVED;
-        if (launch_decode_down(dn, dev.sms, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (launch_decode_down(dn, dev.sms, s, pdl) != cudaSuccess) return MOE_ERR_CUDA;
         if ((st = record(ev, 3, s))) return st;
     } else if (l.p_cap > 0) {
         const int64_t cap_mtiles = (l.p_cap + kTileRows - 1) / kTileRows + E;
@@ -563,7 +567,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         if ((st = record(ev, 3, s))) return st;
     }
     if (launch_combine(ybuf, ylo, meta.token_offset, meta.s_reverse_scatter_idx, meta.scores, N, H,
-                       static_cast<__nv_bfloat16 *>(out), hdr, dev.sms, s) != cudaSuccess)
+                       static_cast<__nv_bfloat16 *>(out), hdr, dev.sms, s, pdl) != cudaSuccess)
         return MOE_ERR_CUDA;
     if ((st = record(ev, 4, s))) return st;
     return MOE_OK;
@@ -704,7 +708,7 @@ int backward_impl(const void *dout, const void *x, const Routing &r, int32_t H, 
     if ((st = record(ev, 5, s))) return st;
     // dx[t] = sum of its pairs' dx rows (weight 1)
     if (launch_combine(ybuf, nullptr, meta.token_offset, meta.s_reverse_scatter_idx, nullptr, N, H,
-                       static_cast<__nv_bfloat16 *>(dx), hdr, dev.sms, s) != cudaSuccess)
+                       static_cast<__nv_bfloat16 *>(dx), hdr, dev.sms, s, false) != cudaSuccess)
         return MOE_ERR_CUDA;
     if ((st = record(ev, 6, s))) return st;
     if (db2 && launch_bias_grad(dybuf, H, meta.expert_frequency_offset, E, static_cast<__nv_bfloat16 *>(db2), hdr,
@@ -933,7 +937,7 @@ extern "C" MOE_API int moe_nonexpand_combine(const void *y, const moe_meta_t *me
     if (st) return st;
     return launch_combine(static_cast<const __nv_bfloat16 *>(y), nullptr, meta->token_offset, meta->s_reverse_scatter_idx,
                           meta->scores, N, H, static_cast<__nv_bfloat16 *>(out), nullptr, dev.sms,
-                          reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                          reinterpret_cast<cudaStream_t>(stream), false) == cudaSuccess
                ? MOE_OK
                : MOE_ERR_CUDA;
 }

@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(kCombineThreads, kLo ? 3 : 4) combine_kernel(
     __shared__ int s_off[kTokPerBlock + 1];
     __shared__ int s_p[kStagedPairs];
     __shared__ float s_w[kStagedPairs];
+    pdl_wait();  // launched as a programmatic dependent: y is the kernel before's
     if (hdr && *(volatile const uint32_t *)&hdr->abort) return;
     const int64_t n_groups = (N + tok_per_block - 1) / tok_per_block;
     for (int64_t grp = blockIdx.x; grp < n_groups; grp += gridDim.x) {
@@ -169,7 +170,7 @@ __global__ void __launch_bounds__(kCombineThreads, kLo ? 3 : 4) combine_kernel(
 
 cudaError_t launch_combine(const __nv_bfloat16 *y, const uint8_t *y_lo, const int32_t *token_offset, const int32_t *s_rev,
                            const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
-                           const WsHeader *hdr, int num_sms, cudaStream_t s) {
+                           const WsHeader *hdr, int num_sms, cudaStream_t s, bool pdl) {
     if (N == 0) return cudaSuccess;
     // tokens per block: up to kTokPerBlock, fewer when that would leave SMs idle
     const int64_t chunks = H / 8;
@@ -181,13 +182,12 @@ cudaError_t launch_combine(const __nv_bfloat16 *y, const uint8_t *y_lo, const in
     int64_t blocks = groups;
     const int64_t cap = (int64_t)num_sms * 16;
     if (blocks > cap) blocks = cap;
+    const uint8_t *no_lo = nullptr;
     if (y_lo)
-        combine_kernel<true><<<(unsigned)blocks, kCombineThreads, 0, s>>>(y, y_lo, token_offset, s_rev, scores, N, H,
-                                                                          out, hdr, (int)tpb);
-    else
-        combine_kernel<false><<<(unsigned)blocks, kCombineThreads, 0, s>>>(y, nullptr, token_offset, s_rev, scores, N,
-                                                                           H, out, hdr, (int)tpb);
-    return cudaGetLastError();
+        return launch_maybe_pdl(combine_kernel<true>, dim3((unsigned)blocks), dim3(kCombineThreads), 0, s, pdl, y,
+                                y_lo, token_offset, s_rev, scores, N, H, out, hdr, (int)tpb);
+    return launch_maybe_pdl(combine_kernel<false>, dim3((unsigned)blocks), dim3(kCombineThreads), 0, s, pdl, y, no_lo,
+                            token_offset, s_rev, scores, N, H, out, hdr, (int)tpb);
 }
 
 }  // namespace moe

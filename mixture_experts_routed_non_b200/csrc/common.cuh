@@ -10,6 +10,7 @@
 #include <stdint.h>
 
 #include <functional>
+#include <utility>
 
 #include "moe_nonexpand.h"
 
@@ -191,6 +192,28 @@ struct BwdGemmArgs {
 // a lock and caches the integer; later calls return the cached value.
 cudaError_t launch_setup_once(const void *kernel, int *value, const std::function<cudaError_t(int dev, int *value)> &setup);
 
+#if defined(__CUDACC__)
+// Launches kernel<<<grid, block, smem, s>>>(args...), as a programmatic
+// dependent of the launch before it on s when pdl is set: the kernel may
+// start before that one has finished and must call pdl_wait() before it
+// reads what that one writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_maybe_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                             Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+#endif
+
 // Host-side argument checks shared by the entry points (capi.cu).
 int check_routing_sizes(int64_t N, int32_t E, int32_t K, int64_t total_pairs);
 bool ptr_aligned(const void *p, size_t a);
@@ -199,11 +222,13 @@ bool ptr_aligned(const void *p, size_t a);
 cudaError_t launch_meta(const MetaArgs &a, cudaStream_t s);
 cudaError_t launch_gemm_up(const GemmArgs &a, int max_clusters, cudaStream_t s);
 cudaError_t launch_gemm_down(const GemmArgs &a, int max_clusters, cudaStream_t s);
-cudaError_t launch_decode_up(const DecodeArgs &a, int max_ctas, cudaStream_t s);
-cudaError_t launch_decode_down(const DecodeArgs &a, int max_ctas, cudaStream_t s);
+// pdl: launched as a programmatic dependent of the previous launch on s (the
+// metadata's scatter kernel before the up GEMM, the up GEMM before the down).
+cudaError_t launch_decode_up(const DecodeArgs &a, int max_ctas, cudaStream_t s, bool pdl);
+cudaError_t launch_decode_down(const DecodeArgs &a, int max_ctas, cudaStream_t s, bool pdl);
 cudaError_t launch_combine(const __nv_bfloat16 *y, const uint8_t *y_lo, const int32_t *token_offset, const int32_t *s_rev,
                            const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
-                           const WsHeader *hdr, int num_sms, cudaStream_t s);
+                           const WsHeader *hdr, int num_sms, cudaStream_t s, bool pdl);
 cudaError_t launch_router(const void *logits, bool bf16, int64_t N, int E, int K, int mode, int32_t *idx, float *w,
                           int num_sms, cudaStream_t s);
 size_t gemm_smem_bytes();
@@ -230,6 +255,15 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
     return t;
 }
+
+// Programmatic dependent launch (sm_90+): the primary lets its dependent
+// start; the dependent waits until the primary grid has completed and its
+// memory operations are visible.  Both are no-ops in a kernel launched
+// without the programmatic-serialization attribute.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;

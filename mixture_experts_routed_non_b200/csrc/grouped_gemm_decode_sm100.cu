@@ -80,7 +80,6 @@ template <bool kUp>
 __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int kThreads = decode_threads(kUp);
     extern __shared__ uint8_t smem_raw[];
-    if (*(volatile uint32_t *)&a.hdr->abort) return;
 
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -115,11 +114,19 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
         tma_prefetch_desc(&a.tmap_w);
         if (!kUp) tma_prefetch_desc(&a.tmap_h);
     }
-    for (int i = threadIdx.x; i <= E; i += kThreads) off_s[i] = __ldg(a.expert_off + i);
     if (warp == 1) {
         tmem_alloc(smem_u32(&misc[0]), kDTmemCols);
         tmem_relinquish();
     }
+    // Launched as a programmatic dependent, the up GEMM starts while the
+    // metadata kernel runs: it waits for it here, and only then lets the
+    // down GEMM start, so a running down GEMM implies finished metadata.
+    // The down GEMM starts while the up GEMM runs: it reads the metadata (in
+    // L2, written before the up GEMM got past its wait) at once, and its
+    // producer waits for the up GEMM before the first load of h.
+    if (kUp) pdl_wait();
+    pdl_launch_dependents();
+    for (int i = threadIdx.x; i <= E; i += kThreads) off_s[i] = __ldcg(a.expert_off + i);
     __syncthreads();
     if (warp == 0) {
         // the experts that have pairs, in order: work is dealt over these only, so
@@ -132,7 +139,8 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
             if (has) act_s[n + __popc(m & lanemask_lt())] = e;
             n += __popc(m);
         }
-        if (lane == 0) misc[3] = (uint32_t)n;
+        // nothing to do when the metadata found more pairs than the arrays hold
+        if (lane == 0) misc[3] = __ldcg(&a.hdr->abort) ? 0u : (uint32_t)n;
     }
     tc_fence_before();
     __syncthreads();
@@ -150,27 +158,48 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            int stage = 0;
+            auto load_w = [&](uint32_t sa, uint32_t fb, int e, int mt, int kb) {
+                const int krow = e * a.k_dim + kb * kDK;
+                if (concat) {
+                    tma_load_4d(sa, &a.tmap_w, fb, 0, krow, mt, 0);             // gate columns
+                    tma_load_4d(sa + kDChunkA, &a.tmap_w, fb, 0, krow, mt, 1);  // up columns
+                } else {
+                    tma_load_3d(sa, &a.tmap_w, fb, 0, krow, 2 * mt);
+                }
+            };
+            // down: the weights of the first stages need nothing from the up
+            // GEMM; they are requested before waiting for it
+            int npre = 0;
+            if (!kUp) {
+                for (int u = blockIdx.x; npre < kDStages && u < units; u += gridDim.x) {
+                    const int e = act_s[u / n_mt], mt = u - (u / n_mt) * n_mt;
+                    const int Me = off_s[e + 1] - off_s[e];
+                    for (int c0 = 0; npre < kDStages && c0 < Me; c0 += kDN)
+                        for (int kb = 0; npre < kDStages && kb < nk; ++kb, ++npre) {
+                            const uint32_t fb = full_bar(npre);  // a fresh stage: nothing to wait for
+                            mbar_arrive_expect_tx(fb, kDStageA + kDStageB);
+                            load_w(sA0 + npre * kDStage, fb, e, mt, kb);
+                        }
+                }
+                pdl_wait();
+            }
+            int stage = 0, issued = 0;
             uint32_t phase = 0;
             bool ok = true;
             for (int u = blockIdx.x; ok && u < units; u += gridDim.x) {
                 const int e = act_s[u / n_mt], mt = u - (u / n_mt) * n_mt;
                 const int m0 = off_s[e], Me = off_s[e + 1] - m0;
                 for (int c0 = 0; ok && c0 < Me; c0 += kDN) {
-                    for (int kb = 0; kb < nk; ++kb) {
-                        if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort)) {
-                            ok = false;
-                            break;
-                        }
+                    for (int kb = 0; kb < nk; ++kb, ++issued) {
                         const uint32_t fb = full_bar(stage);
-                        mbar_arrive_expect_tx(fb, kDStageA + (kUp ? 0u : kDStageB));
                         const uint32_t sa = sA0 + stage * kDStage;
-                        const int krow = e * a.k_dim + kb * kDK;
-                        if (concat) {
-                            tma_load_4d(sa, &a.tmap_w, fb, 0, krow, mt, 0);              // gate columns
-                            tma_load_4d(sa + kDChunkA, &a.tmap_w, fb, 0, krow, mt, 1);   // up columns
-                        } else {
-                            tma_load_3d(sa, &a.tmap_w, fb, 0, krow, 2 * mt);
+                        if (issued >= npre) {
+                            if (!mbar_wait_bounded(empty_bar(stage), phase ^ 1u, abort)) {
+                                ok = false;
+                                break;
+                            }
+                            mbar_arrive_expect_tx(fb, kDStageA + (kUp ? 0u : kDStageB));
+                            load_w(sa, fb, e, mt, kb);
                         }
                         if (!kUp) tma_load_3d(sa + kDStageA, &a.tmap_h, fb, 0, m0 + c0, kb);
                         if (++stage == kDStages) {
@@ -404,7 +433,7 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
 }
 
 template <bool kUp>
-cudaError_t launch_decode(const DecodeArgs &a, int max_ctas, cudaStream_t s) {
+cudaError_t launch_decode(const DecodeArgs &a, int max_ctas, cudaStream_t s, bool pdl) {
     int unused = 0;
     cudaError_t err = launch_setup_once((const void *)decode_gemm_kernel<kUp>, &unused, [](int, int *v) -> cudaError_t {
         *v = 1;
@@ -416,15 +445,16 @@ cudaError_t launch_decode(const DecodeArgs &a, int max_ctas, cudaStream_t s) {
     int ctas = a.E * n_mt;
     if (ctas > max_ctas) ctas = max_ctas;
     if (ctas < 1) ctas = 1;
-    decode_gemm_kernel<kUp><<<ctas, decode_threads(kUp), kDSmemBytes, s>>>(a);
-    return cudaGetLastError();
+    return launch_maybe_pdl(decode_gemm_kernel<kUp>, dim3(ctas), dim3(decode_threads(kUp)), kDSmemBytes, s, pdl, a);
 }
 
 }  // namespace
 
-cudaError_t launch_decode_up(const DecodeArgs &a, int max_ctas, cudaStream_t s) { return launch_decode<true>(a, max_ctas, s); }
-cudaError_t launch_decode_down(const DecodeArgs &a, int max_ctas, cudaStream_t s) {
-    return launch_decode<false>(a, max_ctas, s);
+cudaError_t launch_decode_up(const DecodeArgs &a, int max_ctas, cudaStream_t s, bool pdl) {
+    return launch_decode<true>(a, max_ctas, s, pdl);
+}
+cudaError_t launch_decode_down(const DecodeArgs &a, int max_ctas, cudaStream_t s, bool pdl) {
+    return launch_decode<false>(a, max_ctas, s, pdl);
 }
 
 }  // namespace moe

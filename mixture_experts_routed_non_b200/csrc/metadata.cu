@@ -52,13 +52,6 @@ constexpr int kPartInts = 2 * 4 * kMetaThreads;         // table partial sums: 2
 static_assert(kPartInts % 4 == 0, "the arrays after the partial sums start 16-byte aligned");
 static_assert(kMetaMaxTiles <= kMetaThreads, "one thread of CTA 0 reads each tile's error bits");
 
-// Programmatic dependent launch (sm_90+): the primary lets its dependent
-// start; the dependent waits until the primary grid has completed and its
-// memory operations are visible.
-__device__ __forceinline__ void pdl_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ int4 ld_cg_int4(const int *p) {
     int4 v;
@@ -411,6 +404,9 @@ template <bool kPairs, bool kIdx64>
 __global__ void __launch_bounds__(kMetaThreads, 1) meta_scatter_kernel(const MetaArgs a) {
     extern __shared__ __align__(16) int sm[];
     __shared__ unsigned s_err;
+    // a programmatic dependent (the decode up GEMM) may start its set-up now;
+    // it waits for this grid to finish before it reads the metadata
+    pdl_launch_dependents();
     const int E = a.E, T = a.tiles, tile = blockIdx.x, ld = a.hist_ld;
     const ScatterSmem m = scatter_smem(sm, E);
     const int t0 = tile * a.tile_slots;
