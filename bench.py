@@ -875,7 +875,11 @@ def run_ours(args, rank, world, local):
     if rank == 0 and not args.no_workloads:
         for name in ("ranklocal", "prefill256", "decode256", "tiny"):
             if name != wl.name:
+                time.sleep(0.3)  # an idle gap: each leg starts from a cooled-down power state
+                t0 = time.time()
                 workloads[name] = workload_leg(name, dev, peaks, peak_tf, peak_label, args.steps, args.warmup)
+                # the clock record of the whole leg (warm-up, timed, staged and graph forwards)
+                workloads[name]["clocks"] = sampler.summary(t0, time.time())
 
     meta_c2 = metadata_only(dev, peaks) if rank == 0 else None
     meta_pairs = metadata_pairs_only(dev, peaks) if rank == 0 else None
