@@ -41,7 +41,7 @@ def test_selftest_rejects_bad_arguments():
         binding.selftest_wait_timeout(ws, 3_000_000)
 
 
-@pytest.mark.parametrize("name", ["tiny", "prefill"])
+@pytest.mark.parametrize("name", ["tiny", "prefill", "decode256"])
 def test_forward_captures_in_cuda_graph(name):
     inp = synthetic.make_inputs(name, device="cuda")
     wl = inp.wl

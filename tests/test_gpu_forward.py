@@ -232,3 +232,30 @@ def test_decode_path_long_segment_and_duplicates(layout):
     inp.topk_idx.copy_(torch.from_numpy(idx))
     assert N * K <= 32 * E
     run_case(inp, layout=layout)
+
+
+@pytest.mark.parametrize("name", ["decode256", "prefill256"])
+def test_back_to_back_forwards_match_serialised_ones(name):
+    """Forwards on changing routings enqueued back to back on one stream (every
+    kernel after the metadata starts as a programmatic dependent of the one
+    before it) give, bit for bit, the outputs of the same forwards run one at a
+    time with stage events between the launches (which serialise them) and the
+    host waiting after each."""
+    inp = synthetic.make_inputs(name, device="cuda")
+    wl = inp.wl
+    routes = [synthetic.make_routing(wl, seed=wl.seed + 7 * i) for i in range(4)]
+    idx = [torch.from_numpy(a).cuda() for a, _ in routes]
+    wts = [torch.from_numpy(b).cuda() for _, b in routes]
+    ws = binding.alloc_workspace(wl.N, wl.H, wl.I, wl.E, wl.K, -1)
+    outs = [torch.empty(wl.N, wl.H, dtype=torch.bfloat16, device="cuda") for _ in routes]
+    torch.cuda.synchronize()
+    for i in range(len(routes)):
+        binding.forward(inp.x, idx[i], wts[i], inp.w1, inp.w2, inp.b1, inp.b2, out=outs[i], ws=ws)
+    torch.cuda.synchronize()
+    assert binding.read_error(ws) == 0
+    for i in range(len(routes)):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ref = binding.forward(inp.x, idx[i], wts[i], inp.w1, inp.w2, inp.b1, inp.b2, ws=ws, events=ev)
+        torch.cuda.synchronize()
+        assert binding.read_error(ws) == 0
+        assert torch.equal(outs[i], ref), f"forward {i}"
