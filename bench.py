@@ -639,8 +639,9 @@ def forward_summary(wl, P, freq, inp, stage_ms, ms_per_step, peaks, peak_tf, pea
     up_flops, down_flops = gemm_flops(P, H, I)
     up_tf = up_flops / (stage_ms[1] * 1e-3) / 1e12 if stage_ms[1] > 0 else 0.0
     down_tf = down_flops / (stage_ms[2] * 1e-3) / 1e12 if stage_ms[2] > 0 else 0.0
-    # the combine reads each pair's bf16 row and its e5m2 residual (3 bytes per element)
-    comb_bytes = P * H * 3 + N * H * 2 + (N + 1) * 4 + P * 8
+    # the combine reads each pair's fp16 row (2 bytes per element) and its
+    # exponents (one byte per 32 elements), writes the bf16 output
+    comb_bytes = P * H * 2 + P * (H // 32) + N * H * 2 + (N + 1) * 4 + P * 8
     meta_bytes = N * K * 8 + 4 * P * 4 + 4 * (N + 1) + 8 * E
     alg_bytes = algorithmic_bytes(inp, P, freq)
     t_tensor = (up_flops + down_flops) / (peak_tf * 1e12)

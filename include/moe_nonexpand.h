@@ -498,7 +498,8 @@ typedef struct moe_ws_layout_t {
     size_t meta_freq, meta_off, meta_x_gather, meta_s_scatter, meta_s_rev,
            meta_token_offset, meta_scores;  /* metadata kept in the workspace */
     size_t h;                  /* bf16 [P_cap,I] */
-    size_t y;                  /* bf16 [P_cap,H] */
+    size_t y;                  /* fp16 bits [P_cap,H]: y (+ b2) per expert-sorted row, each 32-column
+                                  block scaled by a power of two: value = fp16 * 2^y_scale */
     int64_t p_cap;
     int32_t meta_tiles;        /* T */
     int32_t meta_tile_slots;   /* slots per metadata tile */
@@ -509,7 +510,10 @@ typedef struct moe_ws_layout_t {
     size_t slot_pair;          /* training workspace: int32 [slots], the pair of each routing slot or -1 */
     size_t ds;                 /* training workspace: fp32 [P_cap], score gradients in pair order */
     size_t train_total;        /* == moe_nonexpand_train_workspace_bytes(...) */
-    size_t y_lo;               /* uint8 [P_cap,H]: e5m2 residual y - bf16(y) of every y element */
+    size_t y_scale;            /* int8 [P_cap,H/32]: the exponent e of each row's 32-column block of y,
+                                  e in [-100,113], every |y| * 2^-e at most 2^15 (the grouped GEMM puts
+                                  the block's largest in [2^14, 2^15); decode-sized batches share e
+                                  over up to 32 rows of one expert) */
 } moe_ws_layout_t;
 
 MOE_API int moe_nonexpand_workspace_layout(int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,

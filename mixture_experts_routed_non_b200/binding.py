@@ -90,7 +90,7 @@ class WsLayout(ctypes.Structure):
         ("p_cap", ctypes.c_int64), ("meta_tiles", ctypes.c_int32), ("meta_tile_slots", ctypes.c_int32),
         ("z", ctypes.c_size_t), ("dz", ctypes.c_size_t), ("dy", ctypes.c_size_t),
         ("slot_pair", ctypes.c_size_t), ("ds", ctypes.c_size_t), ("train_total", ctypes.c_size_t),
-        ("y_lo", ctypes.c_size_t)]
+        ("y_scale", ctypes.c_size_t)]
 
 
 class MoeRouting(ctypes.Structure):
@@ -294,18 +294,16 @@ def meta_from_workspace(ws: torch.Tensor, N: int, H: int, I: int, E: int, K: int
 
 
 def intermediates_from_workspace(ws: torch.Tensor, N: int, H: int, I: int, E: int, K: int,
-                                 total_pairs: int = -1, with_residual: bool = False):
-    """Views (h [P_cap,I], y [P_cap,H], both bf16, expert-sorted rows) of the
-    intermediates that moe_nonexpand_forward keeps in the workspace; with
-    ``with_residual`` also y_lo [P_cap,H] (uint8 bits of the e5m2 residual
-    y - bf16(y) that the combine adds back)."""
+                                 total_pairs: int = -1):
+    """Views of the intermediates that moe_nonexpand_forward keeps in the
+    workspace, expert-sorted rows: h [P_cap,I] bf16; y [P_cap,H] fp16 and
+    y_scale [P_cap,H/32] int8, row p's element c being y[p,c] * 2^y_scale[p,c//32]."""
     lay = workspace_layout(N, H, I, E, K, total_pairs)
     pc = lay.p_cap
     h = ws[lay.h:lay.h + pc * I * 2].view(torch.bfloat16).view(pc, I)
-    y = ws[lay.y:lay.y + pc * H * 2].view(torch.bfloat16).view(pc, H)
-    if with_residual:
-        return h, y, ws[lay.y_lo:lay.y_lo + pc * H].view(pc, H)
-    return h, y
+    y = ws[lay.y:lay.y + pc * H * 2].view(torch.float16).view(pc, H)
+    y_scale = ws[lay.y_scale:lay.y_scale + pc * (H // 32)].view(torch.int8).view(pc, H // 32)
+    return h, y, y_scale
 
 
 def backward_intermediates_from_workspace(ws: torch.Tensor, N: int, H: int, I: int, E: int, K: int,

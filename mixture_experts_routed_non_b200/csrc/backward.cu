@@ -3,7 +3,8 @@
 // the chain rule of the forward):
 //
 //   prep      per token t and each of its pairs q (sorted position p):
-//             ds_q = <dout_t, y_p> (the score's gradient, fp32, summed in a
+//             ds_q = <dout_t, y_p> (y_p as the forward stored it: fp16 times
+//             2^e per 32 columns) (the score's gradient, fp32, summed in a
 //             fixed order) and dy_p = s_q dout_t (bf16 [P_cap,H]); ds is then
 //             scattered to the routing slot each pair came from through the
 //             slot -> pair index the training forward's metadata recorded (0 at
@@ -23,10 +24,11 @@ constexpr int kPrepThreads = 256;
 constexpr int kPrepWarps = kPrepThreads / 32;
 constexpr int kMaxSlots = 32;
 
-__device__ __forceinline__ float dot8(const uint4 &a, const uint4 &b) {
-    return bf16lo(a.x) * bf16lo(b.x) + bf16hi(a.x) * bf16hi(b.x) + bf16lo(a.y) * bf16lo(b.y) +
-           bf16hi(a.y) * bf16hi(b.y) + bf16lo(a.z) * bf16lo(b.z) + bf16hi(a.z) * bf16hi(b.z) +
-           bf16lo(a.w) * bf16lo(b.w) + bf16hi(a.w) * bf16hi(b.w);
+// eight bf16 dout values . eight fp16 y values (the row's 2^e applied by the caller)
+__device__ __forceinline__ float dot8_f16(const uint4 &d, const uint4 &v) {
+    const float2 a = f16x2_to_f32(v.x), b = f16x2_to_f32(v.y), c = f16x2_to_f32(v.z), e = f16x2_to_f32(v.w);
+    return bf16lo(d.x) * a.x + bf16hi(d.x) * a.y + bf16lo(d.y) * b.x + bf16hi(d.y) * b.y + bf16lo(d.z) * c.x +
+           bf16hi(d.z) * c.y + bf16lo(d.w) * e.x + bf16hi(d.w) * e.y;
 }
 
 __device__ __forceinline__ uint4 scale8(const uint4 &v, float s) {
@@ -39,8 +41,8 @@ __device__ __forceinline__ uint4 scale8(const uint4 &v, float s) {
 // dot product, then the block reduces those partials at once (warp
 // butterfly, then warps in order).  A pair list may give a token any number
 // of pairs, hence the batches of 32.
-__global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
-    const __nv_bfloat16 *__restrict__ dout, const __nv_bfloat16 *__restrict__ y,
+__global__ void __launch_bounds__(kPrepThreads, 4) bwd_prep_kernel(
+    const __nv_bfloat16 *__restrict__ dout, const uint16_t *__restrict__ y, const int8_t *__restrict__ y_scale,
     const int32_t *__restrict__ token_offset, const int32_t *__restrict__ s_rev, const float *__restrict__ scores,
     int64_t N, int32_t H, __nv_bfloat16 *__restrict__ dy, float *__restrict__ ds, const WsHeader *hdr) {
     __shared__ float part[kPrepWarps][kMaxSlots];
@@ -62,7 +64,7 @@ __global__ void __launch_bounds__(kPrepThreads) bwd_prep_kernel(
                     if (j >= np) break;
                     const int p = __ldg(s_rev + qb + j);
                     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(y + (size_t)p * H) + c);
-                    acc[j] += dot8(d, v);
+                    acc[j] += dot8_f16(d, v) * exp2i(__ldg(y_scale + (size_t)p * (H / kYBlock) + (c >> 2)));
                     reinterpret_cast<uint4 *>(dy + (size_t)p * H)[c] = scale8(d, __ldg(scores + qb + j));
                 }
             }
@@ -165,14 +167,15 @@ cudaError_t launch_gather_rows(const __nv_bfloat16 *src, const int32_t *idx, con
     return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const __nv_bfloat16 *y, const moe_meta_t &meta, int64_t N,
+cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const void *y, const int8_t *y_scale, const moe_meta_t &meta, int64_t N,
                             int32_t H, __nv_bfloat16 *dy, float *ds, const int32_t *slot_pair, int64_t NK,
                             float *dweights, const WsHeader *hdr, int num_sms, cudaStream_t s) {
     if (N > 0) {
         int64_t blocks = N;
         const int64_t cap = (int64_t)num_sms * 8;
         if (blocks > cap) blocks = cap;
-        bwd_prep_kernel<<<(unsigned)blocks, kPrepThreads, 0, s>>>(dout, y, meta.token_offset,
+        bwd_prep_kernel<<<(unsigned)blocks, kPrepThreads, 0, s>>>(dout, static_cast<const uint16_t *>(y), y_scale,
+                                                                  meta.token_offset,
                                                                   meta.s_reverse_scatter_idx, meta.scores, N, H,
                                                                   dy, ds, hdr);
         const cudaError_t err = cudaGetLastError();

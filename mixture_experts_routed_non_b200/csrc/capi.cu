@@ -117,11 +117,11 @@ moe_ws_layout_t compute_layout_nk(int64_t N, int32_t H, int32_t I, int32_t E, in
         o = align_up(o + (size_t)pc * I * 2, 1024);
         l.y = o;
         o = align_up(o + (size_t)pc * H * 2, 1024);
-        l.y_lo = o;
-        o = align_up(o + (size_t)pc * H, 1024);
+        l.y_scale = o;
+        o = align_up(o + (size_t)pc * (H / kYBlock), 1024);
     }
     l.total = o;
-    if (H > 0 && I > 0) {  // training: z (fp32), dz and dy after the inference workspace
+    if (H > 0 && I > 0) {  // training: z (bf16 factors), dz and dy after the inference workspace
         l.z = o;  // bf16: u silu'(g) at gate columns, silu(g) at up columns
         o = align_up(o + (size_t)pc * 2 * I * 2, 1024);
         l.dz = o;
@@ -276,21 +276,6 @@ bool make_map_2d(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-// uint8 [outer][inner] (inner % 16 == 0) with a box of 64 x box_outer bytes in
-// the 64-byte swizzle (16-byte chunk c of box row r at c ^ ((r >> 1) & 3)).
-bool make_map_2d_u8_sw64(CUtensorMap *m, const void *ptr, uint64_t inner, uint64_t outer, uint32_t box_outer) {
-    EncodeTiledFn f = encode_fn();
-    if (!f) return false;
-    cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {inner};
-    cuuint32_t box[2] = {64, box_outer};
-    cuuint32_t estr[2] = {1, 1};
-    return f(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(ptr), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 
 // A row-major weight [rows][ncols] (ncols % 64 == 0) viewed as
 // (64 columns, rows, ncols/64 column chunks): one box of 64 x stage-K x 2 lands in
@@ -454,7 +439,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
 
     __nv_bfloat16 *hbuf = reinterpret_cast<__nv_bfloat16 *>(w + l.h);
     __nv_bfloat16 *ybuf = reinterpret_cast<__nv_bfloat16 *>(w + l.y);
-    uint8_t *ylo = w + l.y_lo;
+    int8_t *yscale = reinterpret_cast<int8_t *>(w + l.y_scale);
     // Segments of a few rows on average (decode): swap-AB kernels that stream
     // each active expert's weights once.  Chosen per call from the sizes alone
     // (no host sync); they handle segments of any length.
@@ -493,7 +478,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         dn.expert_off = meta.expert_frequency_offset;
         dn.bias = static_cast<const __nv_bfloat16 *>(b2);
         dn.out = ybuf;
-        dn.out_lo = ylo;
+        dn.out_scale = yscale;
         dn.hdr = hdr;
         dn.E = E;
         dn.k_dim = I;
@@ -544,8 +529,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         if (!make_map_a_chunks(&dn.tmap_a16, hbuf, (uint64_t)I, (uint64_t)l.p_cap, 16, 1)) return MOE_ERR_CUDA;
         if (!make_map_b_chunks(&dn.tmap_b, w2, (uint64_t)H, (uint64_t)E * I)) return MOE_ERR_CUDA;
         if (!make_map_2d(&dn.tmap_out, ybuf, (uint64_t)H, (uint64_t)l.p_cap, 64, 32)) return MOE_ERR_CUDA;
-        if (!make_map_2d_u8_sw64(&dn.tmap_lo, ylo, (uint64_t)H, (uint64_t)l.p_cap, 32)) return MOE_ERR_CUDA;
-        dn.out_lo = ylo;
+        dn.out_scale = yscale;
         dn.expert_off = meta.expert_frequency_offset;
         dn.tile_off = ma.gemm_tile_off;
         dn.bias = static_cast<const __nv_bfloat16 *>(b2);
@@ -566,7 +550,7 @@ int forward_impl(const void *x, const Routing &r, int32_t H, int32_t I, int32_t 
         if ((st = record(ev, 2, s))) return st;
         if ((st = record(ev, 3, s))) return st;
     }
-    if (launch_combine(ybuf, ylo, meta.token_offset, meta.s_reverse_scatter_idx, meta.scores, N, H,
+    if (launch_combine(ybuf, yscale, meta.token_offset, meta.s_reverse_scatter_idx, meta.scores, N, H,
                        static_cast<__nv_bfloat16 *>(out), hdr, dev.sms, s, pdl) != cudaSuccess)
         return MOE_ERR_CUDA;
     if ((st = record(ev, 4, s))) return st;
@@ -606,7 +590,8 @@ int backward_impl(const void *dout, const void *x, const Routing &r, int32_t H, 
 
     if ((st = record(ev, 0, s))) return st;
     // score gradients (to the [N,K] slots) and dy = s dout per pair
-    if (launch_bwd_prep(static_cast<const __nv_bfloat16 *>(dout), ybuf, meta, N, H, dybuf,
+    if (launch_bwd_prep(static_cast<const __nv_bfloat16 *>(dout), ybuf, reinterpret_cast<const int8_t *>(w + l.y_scale),
+                        meta, N, H, dybuf,
                         reinterpret_cast<float *>(w + l.ds), reinterpret_cast<const int32_t *>(w + l.slot_pair),
                         r.NK, dweights, hdr, dev.sms, s) != cudaSuccess)
         return MOE_ERR_CUDA;

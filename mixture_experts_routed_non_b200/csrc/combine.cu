@@ -8,8 +8,11 @@
 // [token_offset[t], token_offset[t+1]) in q order (= slot order), fetches the
 // expert row y[s_reverse_scatter_idx[q]] and accumulates scores[q] * row in
 // fp32; the sum is rounded once to bf16.  The result is deterministic and
-// independent of the launch shape.  With a residual array y_lo (the down
-// GEMM's e5m2 rounding residuals) each row element is y + y_lo, exact in fp32.
+// independent of the launch shape.  The forward's rows are fp16 with a
+// power-of-two exponent per 32-column block (the down GEMM's y and y_scale):
+// each row element is fp16 * 2^e, exact in fp32, and the exponent folds into
+// the pair's weight.  The backward's dx rows and the public combine's rows are
+// plain bf16.
 //
 // A block owns up to kTokPerBlock consecutive tokens.  Their token offsets and
 // the row index and score of every one of their pairs (a contiguous q range)
@@ -39,24 +42,17 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
     return v;
 }
 
-__device__ __forceinline__ uint2 ld_stream_v2(const void *p) {
-    uint2 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
-    return v;
-}
-
-// acc += w * (bf16 row + e5m2 residual), eight columns
-__device__ __forceinline__ void fma8_lo(float (&acc)[8], float w, const uint4 &v, const uint2 &r) {
-    const float2 r0 = e5m2x2_to_f32(r.x, 0x1404u), r1 = e5m2x2_to_f32(r.x, 0x3424u);
-    const float2 r2 = e5m2x2_to_f32(r.y, 0x1404u), r3 = e5m2x2_to_f32(r.y, 0x3424u);
-    acc[0] = fmaf(w, bf16lo(v.x) + r0.x, acc[0]);
-    acc[1] = fmaf(w, bf16hi(v.x) + r0.y, acc[1]);
-    acc[2] = fmaf(w, bf16lo(v.y) + r1.x, acc[2]);
-    acc[3] = fmaf(w, bf16hi(v.y) + r1.y, acc[3]);
-    acc[4] = fmaf(w, bf16lo(v.z) + r2.x, acc[4]);
-    acc[5] = fmaf(w, bf16hi(v.z) + r2.y, acc[5]);
-    acc[6] = fmaf(w, bf16lo(v.w) + r3.x, acc[6]);
-    acc[7] = fmaf(w, bf16hi(v.w) + r3.y, acc[7]);
+// acc += w * fp16 row, eight columns (w carries the block's 2^e)
+__device__ __forceinline__ void fma8_f16(float (&acc)[8], float w, const uint4 &v) {
+    const float2 a = f16x2_to_f32(v.x), b = f16x2_to_f32(v.y), c = f16x2_to_f32(v.z), d = f16x2_to_f32(v.w);
+    acc[0] = fmaf(w, a.x, acc[0]);
+    acc[1] = fmaf(w, a.y, acc[1]);
+    acc[2] = fmaf(w, b.x, acc[2]);
+    acc[3] = fmaf(w, b.y, acc[3]);
+    acc[4] = fmaf(w, c.x, acc[4]);
+    acc[5] = fmaf(w, c.y, acc[5]);
+    acc[6] = fmaf(w, d.x, acc[6]);
+    acc[7] = fmaf(w, d.y, acc[7]);
 }
 
 __device__ __forceinline__ void fma8(float (&acc)[8], float w, const uint4 &v) {
@@ -82,14 +78,15 @@ __device__ __forceinline__ uint4 pack8(const float (&acc)[8]) {
 // One block's tokens [t0, t0+nt): their pairs are q in [qa, qa+np) with
 // token-local ends s_off[j+1]-qa.  pidx/pw are the pairs' row indices and
 // scores: in shared memory when staged, else read from global memory.
-template <bool kStaged, bool kLo>
-__device__ __forceinline__ void combine_tokens(const __nv_bfloat16 *__restrict__ y, const uint8_t *__restrict__ y_lo,
+template <bool kStaged, bool kScaled>
+__device__ __forceinline__ void combine_tokens(const uint16_t *__restrict__ y, const int8_t *__restrict__ y_scale,
                                                const int *pidx, const float *pw, const int *s_off, int qa, int np,
                                                int nt, int32_t H, __nv_bfloat16 *__restrict__ out_t0) {
     const int chunks = H >> 3;
+    const int sld = H / kYBlock;  // exponents per row
     for (int c = threadIdx.x; c < chunks; c += kCombineThreads) {
-        const __nv_bfloat16 *ycol = y + (size_t)c * 8;
-        const uint8_t *lcol = kLo ? y_lo + (size_t)c * 8 : nullptr;
+        const uint16_t *ycol = y + (size_t)c * 8;
+        const int8_t *scol = kScaled ? y_scale + (c >> 2) : nullptr;  // the chunk's 32-column block
         __nv_bfloat16 *ocol = out_t0 + (size_t)c * 8;
         // walk the block's pairs in batches of 8 rows in flight, across token
         // boundaries; each token's pairs are still summed in q order
@@ -98,13 +95,13 @@ __device__ __forceinline__ void combine_tokens(const __nv_bfloat16 *__restrict__
         int tok_end = s_off[1] - qa;     // its pairs end here
         for (int base = 0; base < np; base += 8) {
             uint4 v[8];
-            uint2 r[8];
+            int ex[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int q = base + u;
                 const int row = q < np ? (kStaged ? pidx[q] : __ldg(pidx + q)) : 0;
                 v[u] = q < np ? ld_stream_v4(ycol + (size_t)row * H) : make_uint4(0, 0, 0, 0);
-                if (kLo) r[u] = q < np ? ld_stream_v2(lcol + (size_t)row * H) : make_uint2(0, 0);
+                if (kScaled) ex[u] = q < np ? (int)__ldg(scol + (size_t)row * sld) : 0;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -118,7 +115,7 @@ __device__ __forceinline__ void combine_tokens(const __nv_bfloat16 *__restrict__
                     tok_end = s_off[j + 1] - qa;
                 }
                 const float wq = kStaged ? pw[q] : (pw ? __ldg(pw + q) : 1.f);
-                if (kLo) fma8_lo(acc, wq, v[u], r[u]);
+                if (kScaled) fma8_f16(acc, wq * exp2i(ex[u]), v[u]);
                 else fma8(acc, wq, v[u]);
             }
         }
@@ -130,11 +127,10 @@ __device__ __forceinline__ void combine_tokens(const __nv_bfloat16 *__restrict__
     }
 }
 
-// Blocks per SM: 4, or 3 with the residual rows (their registers; 8 rows of
-// 24 bytes in flight per thread still cover the memory latency).
-template <bool kLo>
-__global__ void __launch_bounds__(kCombineThreads, kLo ? 3 : 4) combine_kernel(
-    const __nv_bfloat16 *__restrict__ y, const uint8_t *__restrict__ y_lo, const int32_t *__restrict__ token_offset,
+// Four blocks per SM; eight 16-byte row chunks in flight per thread.
+template <bool kScaled>
+__global__ void __launch_bounds__(kCombineThreads, 4) combine_kernel(
+    const uint16_t *__restrict__ y, const int8_t *__restrict__ y_scale, const int32_t *__restrict__ token_offset,
     const int32_t *__restrict__ s_rev, const float *__restrict__ scores, int64_t N, int32_t H,
     __nv_bfloat16 *__restrict__ out, const WsHeader *hdr, int tok_per_block) {
     __shared__ int s_off[kTokPerBlock + 1];
@@ -157,10 +153,10 @@ __global__ void __launch_bounds__(kCombineThreads, kLo ? 3 : 4) combine_kernel(
                 s_w[i] = scores ? __ldg(scores + qa + i) : 1.f;
             }
             __syncthreads();
-            combine_tokens<true, kLo>(y, y_lo, s_p, s_w, s_off, qa, np, nt, H, out_t0);
+            combine_tokens<true, kScaled>(y, y_scale, s_p, s_w, s_off, qa, np, nt, H, out_t0);
         } else {  // more pairs than the staging arrays hold (a pair list may give a token any number)
-            combine_tokens<false, kLo>(y, y_lo, s_rev + qa, scores ? scores + qa : nullptr, s_off, qa, np, nt, H,
-                                       out_t0);
+            combine_tokens<false, kScaled>(y, y_scale, s_rev + qa, scores ? scores + qa : nullptr, s_off, qa, np, nt,
+                                           H, out_t0);
         }
         __syncthreads();  // shared indices are reused by the next group
     }
@@ -168,26 +164,26 @@ __global__ void __launch_bounds__(kCombineThreads, kLo ? 3 : 4) combine_kernel(
 
 }  // namespace
 
-cudaError_t launch_combine(const __nv_bfloat16 *y, const uint8_t *y_lo, const int32_t *token_offset, const int32_t *s_rev,
+cudaError_t launch_combine(const void *y, const int8_t *y_scale, const int32_t *token_offset, const int32_t *s_rev,
                            const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
                            const WsHeader *hdr, int num_sms, cudaStream_t s, bool pdl) {
     if (N == 0) return cudaSuccess;
     // tokens per block: up to kTokPerBlock, fewer when that would leave SMs idle
     const int64_t chunks = H / 8;
-    const int per_sm = y_lo ? 3 : 4;
-    int64_t tpb = (N * chunks) / ((int64_t)num_sms * per_sm * kCombineThreads);
+    int64_t tpb = (N * chunks) / ((int64_t)num_sms * 4 * kCombineThreads);
     if (tpb < 1) tpb = 1;
     if (tpb > kTokPerBlock) tpb = kTokPerBlock;
     const int64_t groups = (N + tpb - 1) / tpb;
     int64_t blocks = groups;
     const int64_t cap = (int64_t)num_sms * 16;
     if (blocks > cap) blocks = cap;
-    const uint8_t *no_lo = nullptr;
-    if (y_lo)
-        return launch_maybe_pdl(combine_kernel<true>, dim3((unsigned)blocks), dim3(kCombineThreads), 0, s, pdl, y,
-                                y_lo, token_offset, s_rev, scores, N, H, out, hdr, (int)tpb);
-    return launch_maybe_pdl(combine_kernel<false>, dim3((unsigned)blocks), dim3(kCombineThreads), 0, s, pdl, y, no_lo,
-                            token_offset, s_rev, scores, N, H, out, hdr, (int)tpb);
+    const uint16_t *rows = static_cast<const uint16_t *>(y);
+    if (y_scale)
+        return launch_maybe_pdl(combine_kernel<true>, dim3((unsigned)blocks), dim3(kCombineThreads), 0, s, pdl, rows,
+                                y_scale, token_offset, s_rev, scores, N, H, out, hdr, (int)tpb);
+    const int8_t *no_scale = nullptr;
+    return launch_maybe_pdl(combine_kernel<false>, dim3((unsigned)blocks), dim3(kCombineThreads), 0, s, pdl, rows,
+                            no_scale, token_offset, s_rev, scores, N, H, out, hdr, (int)tpb);
 }
 
 }  // namespace moe

@@ -108,14 +108,13 @@ struct GemmArgs {
                               // one box = this CTA's 64 x 128 half of a B stage
     CUtensorMap tmap_out;     // h [P_cap,I] / y [P_cap,H], box 64 columns x 32 rows (stores)
     CUtensorMap tmap_a16;     // down: h as (64, rows, I/64), box 64 x 16 rows x 1 (short segments)
-    CUtensorMap tmap_lo;      // down: y_lo [P_cap,H] uint8, box 64 columns x 32 rows, 64-byte swizzle (stores)
     const __nv_bfloat16 *x;   // up: x [N,H], rows gathered with cp.async
     const int32_t *x_gather_idx;
     const int32_t *expert_off;    // [E+1]
     const int32_t *tile_off;      // [E+1]
     const __nv_bfloat16 *bias;    // b1 [E,2I] / b2 [E,H] or null
-    __nv_bfloat16 *out;           // h [P_cap,I] / y [P_cap,H]
-    uint8_t *out_lo;              // down: y_lo [P_cap,H], e5m2 residual of each stored y element
+    __nv_bfloat16 *out;           // h [P_cap,I] bf16 / y [P_cap,H] (down: fp16 bits, scaled per 32 columns)
+    int8_t *out_scale;            // down: y_scale [P_cap, H/32], the exponent of each row's 32-column block
     __nv_bfloat16 *z_out;         // up, training: [P_cap,2I] bf16, w1 column order: u silu'(g) at the gate
                                   // columns, silu(g) at the up columns (of z with bias), or null
     CUtensorMap tmap_z;           // up, training: z_out as [P_cap][2I], box 64 columns x 32 rows (stores)
@@ -139,8 +138,8 @@ struct DecodeArgs {
     const int32_t *x_gather_idx;
     const int32_t *expert_off;    // [E+1]
     const __nv_bfloat16 *bias;    // b1 [E,2I] / b2 [E,H] or null
-    __nv_bfloat16 *out;           // h [P_cap, I] / y [P_cap, H]
-    uint8_t *out_lo;              // down: y_lo [P_cap, H]
+    __nv_bfloat16 *out;           // h [P_cap, I] bf16 / y [P_cap, H] (down: fp16 bits, scaled per 32 columns)
+    int8_t *out_scale;            // down: y_scale [P_cap, H/32]
     WsHeader *hdr;
     int32_t E;
     int32_t k_dim;        // H (up) / I (down)
@@ -226,14 +225,15 @@ cudaError_t launch_gemm_down(const GemmArgs &a, int max_clusters, cudaStream_t s
 // metadata's scatter kernel before the up GEMM, the up GEMM before the down).
 cudaError_t launch_decode_up(const DecodeArgs &a, int max_ctas, cudaStream_t s, bool pdl);
 cudaError_t launch_decode_down(const DecodeArgs &a, int max_ctas, cudaStream_t s, bool pdl);
-cudaError_t launch_combine(const __nv_bfloat16 *y, const uint8_t *y_lo, const int32_t *token_offset, const int32_t *s_rev,
+// y_scale null: y holds bf16 rows; else fp16 rows, y_scale [rows, H/32] their exponents.
+cudaError_t launch_combine(const void *y, const int8_t *y_scale, const int32_t *token_offset, const int32_t *s_rev,
                            const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
                            const WsHeader *hdr, int num_sms, cudaStream_t s, bool pdl);
 cudaError_t launch_router(const void *logits, bool bf16, int64_t N, int E, int K, int mode, int32_t *idx, float *w,
                           int num_sms, cudaStream_t s);
 size_t gemm_smem_bytes();
 cudaError_t launch_gemm_bwd(int mode, const BwdGemmArgs &a, int max_ctas, cudaStream_t s);
-cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const __nv_bfloat16 *y, const moe_meta_t &meta, int64_t N,
+cudaError_t launch_bwd_prep(const __nv_bfloat16 *dout, const void *y, const int8_t *y_scale, const moe_meta_t &meta, int64_t N,
                             int32_t H, __nv_bfloat16 *dy, float *ds, const int32_t *slot_pair, int64_t NK,
                             float *dweights, const WsHeader *hdr, int num_sms, cudaStream_t s);
 cudaError_t launch_gather_rows(const __nv_bfloat16 *src, const int32_t *idx, const int32_t *p_total, int32_t cols,
@@ -595,20 +595,27 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_ma
            | ((static_cast<uint32_t>(M) >> 4) << 24);
 }
 
-// Residual storage of a bf16-rounded value: r = v - bf16(v) (exact in fp32)
-// rounded to e5m2, whose bits are the top byte of the fp16 with the same value.
-// Two residuals per call: `lo` goes to the low byte of the 16-bit result.
-__device__ __forceinline__ uint32_t e5m2x2_rn(float lo, float hi) {
-    uint16_t d;
-    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
-    return d;
+// The expert rows y are stored as fp16 scaled by a power of two per row and
+// 32-column block: value = fp16 * 2^e, e an int8 in y_scale[p][c / 32].  fp16
+// keeps 11 significant bits (the combine sums rows that may cancel); the
+// exponent keeps bf16's range.  y_block_exp(m) puts m in [2^14, 2^15) (fp16
+// holds up to 65504), clamped to [-100, 113] so that 2^e and 2^-e are normal
+// floats.  The grouped GEMM takes m = the block's largest |value|; the decode
+// GEMM the largest over the block and up to 31 other tokens of its chunk.
+// Either way every element within 2^28 of m is a normal fp16, rounded once.
+constexpr int kYBlock = 32;
+__device__ __forceinline__ int y_block_exp(float amax) {  // amax >= 0 (inf and NaN: the top of the range)
+    const int biased = (int)((__float_as_uint(amax) >> 23) & 0xffu);
+    return min(max(biased - 127 - 14, -100), 113);
 }
-// Bytes 0,1 (sel = 0x1404) or 2,3 (sel = 0x3424) of `v`, each an e5m2 value,
-// as two floats: byte b becomes the fp16 whose bits are b << 8.
-__device__ __forceinline__ float2 e5m2x2_to_f32(uint32_t v, uint32_t sel) {
-    const uint32_t h = __byte_perm(v, 0u, sel);
+__device__ __forceinline__ float exp2i(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }  // e in [-126,127]
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+__device__ __forceinline__ float2 f16x2_to_f32(uint32_t v) {
     __half2 h2;
-    memcpy(&h2, &h, sizeof h);
+    memcpy(&h2, &v, sizeof v);
     return __half22float2(h2);
 }
 

@@ -8,7 +8,7 @@
 //   up   (kUp = true):  Z^T[c, n] = sum_k w1[e][k][c] * x[x_gather_idx[off_e + n]][k]
 //                       h[off_e + n][j] = silu(gate_j) * up_j      (bf16 [P_cap, I])
 //   down (kUp = false): Y^T[c, n] = sum_k w2[e][k][c] * h[off_e + n][k]
-//                       y[off_e + n][c] (bf16) and its e5m2 rounding residual y_lo
+//                       y[off_e + n][c] (fp16 with an exponent per 32 columns in y_scale)
 //
 // A work unit is (expert e with pairs, 128 output columns mt), dealt
 // round-robin over the CTAs from a list of the active experts that each CTA
@@ -299,19 +299,40 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
                     const int p0 = m0 + c0 + n0;  // segment row (sorted position) of column n0
                     const int nn = min(32, nv - n0);
                     if (!kUp) {
-                        // y[p][c] and its residual; lanes hold consecutive columns c
+                        // y[p][c] as fp16 scaled per 32-column block.  The warp's lanes hold
+                        // the 32 consecutive columns of one block (H and the warp's first
+                        // column are multiples of 32: a whole warp is inside or past H) for
+                        // this group of up to 32 tokens; one exponent for the group, from
+                        // its largest |y| (one warp reduction), serves every token's block
                         const int c = mt * kDM + r;
                         if (c < a.n_out) {
                             const float b = a.bias ? __bfloat162float(a.bias[(size_t)e * a.n_out + c]) : 0.f;
+                            float yv[32], am[16];
+#pragma unroll
+                            for (int n = 0; n < 32; ++n) yv[n] = __uint_as_float(v[n]) + b;
+                            // the group's largest |y| over its nn tokens (columns past them are
+                            // never stored): a pairwise tree, fmaxf dropping NaN
+#pragma unroll
+                            for (int n = 0; n < 16; ++n)
+                                am[n] = fmaxf(2 * n < nn ? fabsf(yv[2 * n]) : 0.f,
+                                              2 * n + 1 < nn ? fabsf(yv[2 * n + 1]) : 0.f);
+#pragma unroll
+                            for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+                                for (int n = 0; n < w; ++n) am[n] = fmaxf(am[n], am[n + w]);
+                            const float tmax = am[0];
+                            // |y| bits order like |y|
+                            const int ex = y_block_exp(
+                                __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(tmax))));
+                            const float sc = exp2i(-ex);
+                            uint16_t *yo = reinterpret_cast<uint16_t *>(a.out);
 #pragma unroll
                             for (int n = 0; n < 32; ++n) {
                                 if (n < nn) {
-                                    const float y = __uint_as_float(v[n]) + b;
-                                    const __nv_bfloat16 hi = __float2bfloat16_rn(y);
-                                    const float rr = y - __bfloat162float(hi);
-                                    a.out[(size_t)(p0 + n) * a.out_cols + c] = hi;
-                                    a.out_lo[(size_t)(p0 + n) * a.out_cols + c] =
-                                        (uint8_t)(e5m2x2_rn(rr, 0.f) & 0xffu);
+                                    yo[(size_t)(p0 + n) * a.out_cols + c] = __half_as_ushort(__float2half_rn(yv[n] * sc));
+                                    if (lane == n)
+                                        a.out_scale[(size_t)(p0 + n) * (a.out_cols / kYBlock) + c / kYBlock] =
+                                            (int8_t)ex;
                                 }
                             }
                         }

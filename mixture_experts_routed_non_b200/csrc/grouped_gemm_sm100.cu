@@ -18,11 +18,11 @@
 //        your model is HuggingFace") the even CTA loads 128 gate columns and
 //        the odd CTA the matching 128 up columns, so gate and up land in
 //        accumulator columns c and c+128.
-//   down (kUp = false): y[p, :] = h[p, :] . w2[e] (+ b2[e])  (bf16 [P_cap, H]),
-//        and y_lo[p, :] = e5m2(y - bf16(y)), the rounding residual of every
-//        stored element (uint8 [P_cap, H]): the combine adds it back, so the
-//        rows it sums carry about 11 bits instead of bf16's 8 at 1.5x the bytes
-//        of bf16 rows (fp32 rows would cost 2x).
+//   down (kUp = false): y[p, :] = h[p, :] . w2[e] (+ b2[e]), stored as fp16
+//        scaled by a power of two per 32-column block of each row ([P_cap, H]
+//        fp16 bits and the int8 exponents y_scale [P_cap, H/32]): the rows the
+//        combine sums carry 11 significant bits instead of bf16's 8, at bf16's
+//        range and 1/32 byte per element more than bf16 rows.
 //
 // Tiles: a cluster of two CTAs owns a tile of 256 rows of one expert's
 // segment x 256 accumulator columns.  CTA r holds A rows [128r, 128r+128) and
@@ -80,15 +80,12 @@ constexpr int kTailRows = kBM / 2;  // rows per CTA of a tail tile
 constexpr unsigned long long kAbortSettleNs = 2000000ull;
 
 constexpr uint32_t kStoreBuf = 32 * 128;        // 4 KB per epilogue warp: 32 rows x 64 bf16
-constexpr uint32_t kStoreBufLo = 32 * 64;       // 2 KB per epilogue warp: 32 rows x 64 residual bytes (down)
 constexpr size_t kSmemStoreOff = (size_t)kPairStages * kStageBytes;
-constexpr size_t kSmemLoOff = kSmemStoreOff + 4 * kStoreBuf;
-constexpr size_t kSmemBarOff = kSmemLoOff + 4 * kStoreBufLo;
+constexpr size_t kSmemBarOff = kSmemStoreOff + 4 * kStoreBuf;
 constexpr size_t kSmemMiscOff = kSmemBarOff + 8 * kNumBars;
 constexpr size_t kSmemTableOff = kSmemMiscOff + 16;
 constexpr size_t kSmemBytes = 1024 /*alignment slack*/ + kSmemTableOff + 2 * (kMaxExperts + 1) * 4;
 static_assert(kSmemBytes <= 232448, "shared memory of one CTA (227 KB)");
-static_assert(kSmemLoOff % 1024 == 0, "the 64-byte swizzle repeats every 512 bytes");
 
 __host__ __device__ constexpr int threads_of(bool up) { return up ? 192 + kGatherThreads : 192; }
 
@@ -563,8 +560,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                     store64(col0, packed);
                 }
             } else {
-                // y as bf16 plus the e5m2 residual of its rounding, 64 columns at a time
-                const uint32_t lo_buf = base + (uint32_t)kSmemLoOff + (uint32_t)(warp - 2) * kStoreBufLo;
+                // y as fp16 scaled per 32-column block (its exponents in y_scale), 64
+                // columns at a time: each thread holds its row's values, so a block's
+                // largest |value| needs no exchange
 #pragma unroll 1
                 for (int gi = 0; gi < (tail ? 2 : 4); ++gi) {
                     const int col0 = t.nt * kBN + chalf * (kBN / 2) + gi * 64;
@@ -573,59 +571,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(threads_of(kUp), 1)
                     tmem_ld_32x32b_x32(tbase + gi * 64, r0);
                     tmem_ld_32x32b_x32(tbase + gi * 64 + 32, r1);
                     tmem_ld_wait();
-                    uint32_t packed[32], lo[16];
                     if (brow) {
                         add_bias32(r0, brow + col0);
                         add_bias32(r1, brow + col0 + 32);
                     }
+                    float m0 = 0.f, m1 = 0.f;  // fmaxf drops NaN
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        m0 = fmaxf(m0, fabsf(__uint_as_float(r0[i])));
+                        m1 = fmaxf(m1, fabsf(__uint_as_float(r1[i])));
+                    }
+                    const int e0 = y_block_exp(m0), e1 = y_block_exp(m1);
+                    const float s0 = exp2i(-e0), s1 = exp2i(-e1);
+                    uint32_t packed[32];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        packed[i] = pack_bf16x2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
-                        packed[16 + i] = pack_bf16x2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
+                        packed[i] = pack_f16x2(__uint_as_float(r0[2 * i]) * s0, __uint_as_float(r0[2 * i + 1]) * s0);
+                        packed[16 + i] =
+                            pack_f16x2(__uint_as_float(r1[2 * i]) * s1, __uint_as_float(r1[2 * i + 1]) * s1);
                     }
-                    // residual v - bf16(v), exact in fp32 (the two differ by less than 2^-8 |v|)
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const uint32_t p0 = packed[2 * i], p1 = packed[2 * i + 1];
-                        const uint32_t q0 = packed[16 + 2 * i], q1 = packed[16 + 2 * i + 1];
-                        lo[i] = e5m2x2_rn(__uint_as_float(r0[4 * i]) - bf16lo(p0),
-                                          __uint_as_float(r0[4 * i + 1]) - bf16hi(p0)) |
-                                (e5m2x2_rn(__uint_as_float(r0[4 * i + 2]) - bf16lo(p1),
-                                           __uint_as_float(r0[4 * i + 3]) - bf16hi(p1)) << 16);
-                        lo[8 + i] = e5m2x2_rn(__uint_as_float(r1[4 * i]) - bf16lo(q0),
-                                              __uint_as_float(r1[4 * i + 1]) - bf16hi(q0)) |
-                                    (e5m2x2_rn(__uint_as_float(r1[4 * i + 2]) - bf16lo(q1),
-                                               __uint_as_float(r1[4 * i + 3]) - bf16hi(q1)) << 16);
-                    }
-                    if (warp_full) {
-                        if (lane == 0) bulk_wait_read0();  // both buffers' previous stores have been read
-                        __syncwarp();
-#pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            st_shared_v4(store_buf + lane * 128 + ((c ^ (lane & 7)) << 4), packed[4 * c],
-                                         packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-                        // 64-byte rows in the 64-byte swizzle: 16-byte chunk c of row r at c ^ ((r >> 1) & 3)
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            st_shared_v4(lo_buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4), lo[4 * c],
-                                         lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&a.tmap_out, store_buf, col0, wrow0);
-                            tma_store_2d(&a.tmap_lo, lo_buf, col0, wrow0);
-                            bulk_commit();
-                        }
-                    } else if (valid) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + col0);
-#pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            dst[c] = make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-                        uint4 *dlo = reinterpret_cast<uint4 *>(a.out_lo + (size_t)p * a.out_cols + col0);
-#pragma unroll
-                        for (int c = 0; c < 4; ++c)
-                            dlo[c] = make_uint4(lo[4 * c], lo[4 * c + 1], lo[4 * c + 2], lo[4 * c + 3]);
-                    }
+                    if (valid)  // the two blocks' exponents (col0 is a multiple of 64: 2-byte aligned)
+                        *reinterpret_cast<uint16_t *>(a.out_scale + (size_t)p * (a.n_dim / kYBlock) + col0 / kYBlock) =
+                            (uint16_t)((uint32_t)(uint8_t)e0 | ((uint32_t)(uint8_t)e1 << 8));
+                    store64(col0, packed);
                 }
             }
             tc_fence_before();
