@@ -296,6 +296,13 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(tb + n0, v);
                     tmem_ld_wait();
+                    if (n0 + 32 >= nv) {
+                        // the accumulator's last load has landed in registers: hand it back to
+                        // the MMA before this group's arithmetic and stores
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(tempty_bar(acc));
+                    }
                     const int p0 = m0 + c0 + n0;  // segment row (sorted position) of column n0
                     const int nn = min(32, nv - n0);
                     if (!kUp) {
@@ -385,9 +392,6 @@ __global__ void __launch_bounds__(decode_threads(kUp), 1) decode_gemm_kernel(con
                         epilogue_bar();
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(tempty_bar(acc));
             }
         }
     } else if (kUp) {
