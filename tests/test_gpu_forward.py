@@ -266,3 +266,28 @@ def test_back_to_back_forwards_match_serialised_ones(name):
         torch.cuda.synchronize()
         assert binding.read_error(ws) == 0
         assert torch.equal(outs[i], ref), f"forward {i}"
+
+
+@pytest.mark.parametrize("shift", [-100, -60, 60, 100])
+@pytest.mark.parametrize("shape", ["grouped", "decode"])
+def test_y_keeps_bf16_range(shift, shape):
+    """w2 and b2 scaled by 2^shift (exact in bf16) scale y and the output by
+    2^shift: the expert rows, stored as fp16 with a power-of-two exponent per
+    32-column block, keep bf16's range at both ends, on the grouped-GEMM path
+    and on the decode path, and the output stays within tolerance of the oracle
+    run on the same scaled weights."""
+    if shape == "grouped":
+        wl = synthetic.custom(300, 256, 128, 8, 2, p_invalid=0.1, bias=True, seed=31)
+    else:
+        wl = synthetic.custom(48, 256, 128, 32, 4, p_invalid=0.1, bias=True, seed=32)
+        assert wl.N * wl.K <= 32 * wl.E  # the sizes select the decode kernels
+    inp = synthetic.make_inputs(wl, device="cuda")
+    f = 2.0 ** shift
+    inp.w2 = (inp.w2.float() * f).to(torch.bfloat16)
+    inp.b2 = (inp.b2.float() * f).to(torch.bfloat16)
+    assert torch.isfinite(inp.w2.float()).all() and (inp.w2 != 0).any()
+    out, _ = run_case(inp)
+    o = out.float()
+    assert torch.isfinite(o).all()
+    mag = o.abs()[o != 0].log2().median().item()
+    assert abs(mag - shift) < 8, f"output magnitude 2^{mag:.1f} for weights scaled by 2^{shift}"
