@@ -817,7 +817,9 @@ def run_ours(args, rank, world, local):
     ev_in = [torch.cuda.Event() for _ in range(nbuf)]
     ev_cmp = [torch.cuda.Event() for _ in range(nbuf)]
     ev_out = [torch.cuda.Event() for _ in range(nbuf)]
-    e2e_steps = max(3, min(args.steps, 100))
+    # at least 100 steps: the three-stage pipeline's fill and drain (one copy each
+    # way) are amortised as in a serving loop, which runs continuously
+    e2e_steps = max(100, args.steps)
 
     def e2e_step(i):
         b = i % nbuf
