@@ -109,8 +109,9 @@ typedef struct CUevent_st *moe_event_t;
  * Bytes of workspace needed by moe_nonexpand_forward for these sizes (pass
  * H = I = 0 for what moe_nonexpand_metadata alone needs).  The workspace
  * holds the per-tile histograms, the GEMM tile table, the metadata when the
- * caller does not provide it, and the bf16 intermediates h [P_cap,I] and
- * y [P_cap,H].  Its contents need no initialisation: every call writes what
+ * caller does not provide it, and the intermediates h [P_cap,I] (bf16) and
+ * y [P_cap,H] (fp16 with a power-of-two exponent per 32-column block).  Its
+ * contents need no initialisation: every call writes what
  * it reads.  One workspace must not be used by two calls that can run at the
  * same time.
  * Returns 0 for arguments outside the supported sizes.
@@ -187,7 +188,9 @@ MOE_API int moe_nonexpand_metadata_noalloc_read_error(moe_stream_t stream, uint3
  *   out  [N,H]   bf16 (written; rounded to nearest even from an fp32 sum)
  *   meta_out: NULL keeps the metadata inside the workspace; otherwise the
  *             metadata is also left in the caller's buffers.
- * Intermediates h = silu(g)*u and y = h.w2 + b2 are stored as bf16.
+ * Intermediates: h = silu(g)*u is stored as bf16; y = h.w2 + b2 as fp16
+ * scaled by a power of two per row and 32-column block (11 significant bits
+ * at bf16's range; moe_ws_layout_t.y and .y_scale), which the combine reads.
  */
 MOE_API int moe_nonexpand_forward(const void *x, const int32_t *topk_idx, const float *topk_w,
                           int64_t N, int32_t H, int32_t I, int32_t E, int32_t K,
