@@ -3,9 +3,9 @@
 // the chain rule of the forward):
 //
 //   prep      per token t and each of its pairs q (sorted position p):
-//             ds_q = <dout_t, y_p> (y_p as the forward stored it: fp16 times
-//             2^e per 32 columns) (the score's gradient, fp32, summed in a
-//             fixed order) and dy_p = s_q dout_t (bf16 [P_cap,H]); ds is then
+//             ds_q = <dout_t, y_p>, the score's gradient (y_p as the forward
+//             stored it, fp16 times 2^e per 32 columns; fp32, summed in a
+//             fixed order), and dy_p = s_q dout_t (bf16 [P_cap,H]); ds is then
 //             scattered to the routing slot each pair came from through the
 //             slot -> pair index the training forward's metadata recorded (0 at
 //             slots that are no pair) -- sonic-moe issue #68 asks for the
