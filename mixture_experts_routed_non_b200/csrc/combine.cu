@@ -31,8 +31,8 @@ namespace moe {
 namespace {
 
 constexpr int kCombineThreads = 256;
-constexpr int kTokPerBlock = 8;
-constexpr int kStagedPairs = kTokPerBlock * 32;  // pair indices staged in shared memory per block
+constexpr int kTokPerBlock = 32;
+constexpr int kStagedPairs = 256;  // pair indices staged in shared memory per block (28 tokens of 8 pairs fit)
 
 __device__ __forceinline__ uint4 ld_stream_v4(const void *p) {
     uint4 v;
@@ -168,9 +168,10 @@ cudaError_t launch_combine(const void *y, const int8_t *y_scale, const int32_t *
                            const float *scores, int64_t N, int32_t H, __nv_bfloat16 *out,
                            const WsHeader *hdr, int num_sms, cudaStream_t s, bool pdl) {
     if (N == 0) return cudaSuccess;
-    // tokens per block: up to kTokPerBlock, fewer when that would leave SMs idle
-    const int64_t chunks = H / 8;
-    int64_t tpb = (N * chunks) / ((int64_t)num_sms * 4 * kCombineThreads);
+    // tokens per block: as many as fill every SM's four resident blocks once (one
+    // wave, no partial last wave), at most kTokPerBlock
+    const int64_t resident = (int64_t)num_sms * 4;
+    int64_t tpb = (N + resident - 1) / resident;
     if (tpb < 1) tpb = 1;
     if (tpb > kTokPerBlock) tpb = kTokPerBlock;
     const int64_t groups = (N + tpb - 1) / tpb;
